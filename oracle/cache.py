@@ -1,0 +1,131 @@
+"""Host-side bookkeeping of the oracle's hybrid KV cache (numpy only).
+
+TEST INFRASTRUCTURE ONLY.  This file decides which position lives in which
+segment of the cache; every number it stores comes from the oracle's own
+quantizer (``hyq_oracle.c`` via :func:`oracle.pack`) or is an input copied
+verbatim.
+
+Segments per unit (b, kv head), following the three token classes of the
+aifromscratch.in explainer ("How It Works"):
+  * quantized majority: packed INT4 codes + fp16 (scale, zero) for every
+    position that has left the local window, [0, T - W);
+  * vertical-line tokens: FP16 K/V rows of the selected positions, in
+    ascending position order;
+  * local window: FP16 K/V of the last W positions in a ring, slot = p % W.
+
+Readings where the pages are silent:
+  * every token is packed when it leaves the window, VL or not, so codes
+    exist for all of [0, T - W);
+  * re-selection from the cache keeps FP16 rows only for positions selected
+    again; newly selected positions have no FP16 source left and stay INT4
+    ("unpromoted"); dropped positions fall back to their codes.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import D, ROW_BYTES, pack
+
+
+class OracleCache:
+    def __init__(self, B, Hq, Hkv, cap, vl_cap, W=128):
+        assert Hq % Hkv == 0
+        vl_cap = max(int(vl_cap), 1)
+        self.B, self.Hq, self.Hkv, self.cap, self.vl_cap, self.W = B, Hq, Hkv, cap, vl_cap, W
+        U = B * Hkv
+        self.k_codes = np.zeros((U, cap, ROW_BYTES), np.uint8)
+        self.v_codes = np.zeros((U, cap, ROW_BYTES), np.uint8)
+        self.k_sz = np.zeros((U, cap, 8), np.uint16)
+        self.v_sz = np.zeros((U, cap, 8), np.uint16)
+        self.win_k = np.zeros((U, W, D), np.uint16)
+        self.win_v = np.zeros((U, W, D), np.uint16)
+        self.vl_k = np.zeros((U, vl_cap, D), np.uint16)
+        self.vl_v = np.zeros((U, vl_cap, D), np.uint16)
+        self.vl_pos = np.full((U, vl_cap), -1, np.int32)
+        self.vl_count = np.zeros(U, np.int32)
+        self.seq_len = np.zeros(B, np.int32)
+
+    # ------------------------------------------------------------ prompt
+    def load_prompt(self, K, V, seq_len):
+        """K, V: [B][Hkv][>=T][128] fp16 (as uint16 bits or float16).
+        Packs [0, T-W) and fills the window with [max(0, T-W), T)."""
+        K = np.asarray(K).view(np.uint16)
+        V = np.asarray(V).view(np.uint16)
+        seq_len = np.asarray(seq_len, np.int32)
+        for b in range(self.B):
+            T = int(seq_len[b])
+            assert 0 <= T <= self.cap
+            self.seq_len[b] = T
+            n_old = max(0, T - self.W)
+            for h in range(self.Hkv):
+                u = b * self.Hkv + h
+                if n_old:
+                    c, s, bad = pack(K[b, h, :n_old])
+                    assert bad == 0
+                    self.k_codes[u, :n_old], self.k_sz[u, :n_old] = c, s
+                    c, s, bad = pack(V[b, h, :n_old])
+                    assert bad == 0
+                    self.v_codes[u, :n_old], self.v_sz[u, :n_old] = c, s
+                for p in range(n_old, T):
+                    self.win_k[u, p % self.W] = K[b, h, p]
+                    self.win_v[u, p % self.W] = V[b, h, p]
+                self.vl_count[u] = 0
+                self.vl_pos[u] = -1
+
+    # ------------------------------------------------------------ VL set
+    def apply_vl(self, pos, K_full=None, V_full=None):
+        """pos: [B][Hkv][k] ascending.  With K_full/V_full (prefill mode) the
+        FP16 rows come from them; without (cache mode) only positions already
+        held in FP16 stay FP16.  Returns the number of unpromoted positions."""
+        pos = np.asarray(pos, np.int32)
+        k = pos.shape[-1]
+        assert k <= self.vl_cap
+        unpromoted = 0
+        if K_full is not None:
+            K_full = np.asarray(K_full).view(np.uint16)
+            V_full = np.asarray(V_full).view(np.uint16)
+        for b in range(self.B):
+            for h in range(self.Hkv):
+                u = b * self.Hkv + h
+                new = [int(p) for p in pos[b, h]]
+                if K_full is not None:
+                    rows_k = [K_full[b, h, p] for p in new]
+                    rows_v = [V_full[b, h, p] for p in new]
+                    kept = new
+                else:
+                    old = {int(self.vl_pos[u, i]): i for i in range(self.vl_count[u])}
+                    kept = [p for p in new if p in old]
+                    unpromoted += len(new) - len(kept)
+                    rows_k = [self.vl_k[u, old[p]].copy() for p in kept]
+                    rows_v = [self.vl_v[u, old[p]].copy() for p in kept]
+                self.vl_pos[u] = -1
+                for i, p in enumerate(kept):
+                    self.vl_pos[u, i] = p
+                    self.vl_k[u, i] = rows_k[i]
+                    self.vl_v[u, i] = rows_v[i]
+                self.vl_count[u] = len(kept)
+        return unpromoted
+
+    # ------------------------------------------------------------ decode
+    def append(self, k_new, v_new):
+        """k_new, v_new: [B][Hkv][128] fp16.  The row leaving the window
+        (position T - W) is packed first, then the new token takes its slot."""
+        k_new = np.asarray(k_new).view(np.uint16)
+        v_new = np.asarray(v_new).view(np.uint16)
+        for b in range(self.B):
+            T = int(self.seq_len[b])
+            assert T + 1 <= self.cap
+            slot = T % self.W
+            for h in range(self.Hkv):
+                u = b * self.Hkv + h
+                if T >= self.W:
+                    p_out = T - self.W
+                    c, s, bad = pack(self.win_k[u, slot])
+                    assert bad == 0
+                    self.k_codes[u, p_out], self.k_sz[u, p_out] = c[0], s[0]
+                    c, s, bad = pack(self.win_v[u, slot])
+                    assert bad == 0
+                    self.v_codes[u, p_out], self.v_sz[u, p_out] = c[0], s[0]
+                self.win_k[u, slot] = k_new[b, h]
+                self.win_v[u, slot] = v_new[b, h]
+            self.seq_len[b] = T + 1
