@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Benchmark: HyQuant hybrid INT4/FP16 KV-cache decode attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: Llama-3.1-8B-shaped decode attention at 32K context (batch 1 per
+GPU, 32 query / 8 KV heads, head_dim 128, window 128, 3% vertical-line
+tokens).  One step = one decode step of one attention layer through the
+library's C ABI: hyq_append (the token leaving the window is packed to INT4,
+the new K/V enters the window, the query enters the detector ring) and
+hyq_decode (fused dequant + attention, split-KV + combine); every 64 tokens
+of a layer the step also re-selects its vertical lines (hyq_select_vl over
+the cache + hyq_vl_apply).  Eight independent layer caches are cycled so the
+working set (~360 MB) exceeds the 126 MB L2 between successive steps.
+
+Metric: effective decode-attention HBM GB/s = algorithmic bytes of the
+decode steps (packed codes + scales + FP16 vertical-line/window K/V + Q/O) /
+time.  The timed region is one CUDA-graph replay of K steps, bracketed by
+a barrier and synchronize; per-launch decode durations come from CUDA
+events captured around every decode inside the graph.
+
+--impl reference times the CPU oracle (fp64, plain C) on a bounded sample of
+the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attention effective HBM GB/s (% of B200 peak); µs/step at 32K ctx"
+N_LAYERS = 8
+RESELECT = 64
+N_Q = 64
+
+
+def algorithmic_bytes(B, Hq, Hkv, T, k, W=128):
+    """Bytes one decode step must move: packed INT4 K/V + scale/zero (160 B
+    per token per unit), FP16 K/V of vertical-line and window tokens (512 B),
+    Q in and O out (fp16)."""
+    n_old = max(0, T - W)
+    per_unit = (n_old - k) * 160 + k * 512 + min(T, W) * 512
+    return B * Hkv * per_unit + B * Hq * 128 * 2 * 2
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=512)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=128)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9 and parts[1].isdigit():
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [int(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": int(statistics.median(sm)), "sm_max_mhz": int(rows[0][2]), "samples": len(rows),
+                "reasons": reasons}
+
+
+# --------------------------------------------------------------- setup
+def setup_layers(torch, hyq, synth, cfg, cap, n_layers):
+    """Build n_layers hybrid caches from the workload's prompt, entirely with
+    the library: prefill -> select_vl (prefill mode) -> vl_apply."""
+    K, V, _ = synth.kv_full(cfg, cap)
+    Kd = torch.from_numpy(K).cuda()
+    Vd = torch.from_numpy(V).cuda()
+    qs = torch.from_numpy(np.stack([synth.qsel(cfg, b) for b in range(cfg.B)])).cuda()
+    layers = []
+    for _ in range(n_layers):
+        c = hyq.HybridCache(cfg.B, cfg.Hq, cfg.Hkv, cap, cfg.k)
+        c.seq_len.fill_(cfg.T)
+        hyq.hyq_prefill(c, Kd, Vd)
+        pos = torch.zeros(cfg.B, cfg.Hkv, cfg.k, dtype=torch.int32, device="cuda")
+        ws = hyq.workspace(hyq.hyq_select_vl_workspace(c, N_Q))
+        hyq.hyq_select_vl(c, qs, cfg.k, pos, ws, k_full=Kd)
+        hyq.hyq_vl_apply(c, pos, Kd, Vd)
+        layers.append(c)
+    torch.cuda.synchronize()
+    return layers, Kd, Vd
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from fp16_kv_cache_b200 import build, hyq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    build.build()
+    cfg = synth.config(2)
+    K_steps, W_steps = args.steps, args.warmup
+    per_layer_tokens = (K_steps + W_steps + args.e2e_steps) // N_LAYERS + 2
+    cap = ((cfg.T + per_layer_tokens + 127) // 128) * 128
+    layers, Kd, Vd = setup_layers(torch, hyq, synth, cfg, cap, N_LAYERS)
+    B, Hq, Hkv = cfg.B, cfg.Hq, cfg.Hkv
+    dev = torch.device("cuda", local)
+
+    # per-step inputs (device) and detector rings / workspaces
+    n_total = W_steps + K_steps
+    q_in = torch.from_numpy(np.stack([synth.q(cfg, 10 + s) for s in range(64)])).to(dev)
+    kv = [synth.step_kv(cfg, s) for s in range(64)]
+    k_in = torch.from_numpy(np.stack([a for a, _ in kv])).to(dev)
+    v_in = torch.from_numpy(np.stack([b for _, b in kv])).to(dev)
+    rings = [torch.zeros(B, Hq, N_Q, 128, dtype=torch.float16, device=dev) for _ in layers]
+    out = torch.empty(B, Hq, 128, dtype=torch.float16, device=dev)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    n_ctas = hyq.hyq_decode_default_ctas()
+    dws = [hyq.workspace(hyq.hyq_decode_workspace(c, n_ctas)) for c in layers]
+    sws = hyq.workspace(hyq.hyq_select_vl_workspace(layers[0], N_Q))
+    sel_pos = torch.zeros(B, Hkv, cfg.k, dtype=torch.int32, device=dev)
+    nunp = torch.zeros(1, dtype=torch.int32, device=dev)
+    tokens = [cfg.T] * N_LAYERS        # host mirror of each layer's length
+    appended = [0] * N_LAYERS
+
+    resel_at = {}  # layer -> index of the step whose decode first sees the new VL set
+
+    def step(s, ev=None):
+        """Enqueue step s; returns (launches, layer, T seen by the decode)."""
+        li = s % N_LAYERS
+        c = layers[li]
+        i = s % 64
+        hyq.hyq_append(c, k_in[i], v_in[i], q_in[i], rings[li])
+        tokens[li] += 1
+        appended[li] += 1
+        launches = 2
+        if appended[li] % RESELECT == 0:
+            hyq.hyq_select_vl(c, rings[li], cfg.k, sel_pos, sws, q_is_ring=True)
+            hyq.hyq_vl_apply(c, sel_pos, n_unpromoted=nunp)
+            resel_at.setdefault(li, s)
+            launches += 5
+        if ev is not None:
+            ev[0].record()
+        hyq.hyq_decode(c, q_in[i], out, dws[li], lse=lse, n_ctas=n_ctas)
+        if ev is not None:
+            ev[1].record()
+        return launches, li, tokens[li]
+
+    # warm-up (eager, untimed) -- also sets kernel attributes before capture
+    for s in range(W_steps):
+        step(s)
+    torch.cuda.synchronize()
+
+    # capture K steps with events around every decode
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_steps)]
+    g = torch.cuda.CUDAGraph()
+    total_launches = 0
+    seen = []  # (step, layer, T)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for j in range(K_steps):
+                nl, li, T = step(W_steps + j, evs[j])
+                total_launches += nl
+                seen.append((W_steps + j, li, T))
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local) if not args.no_clocks else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    g.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    elapsed_ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    # algorithmic bytes of every timed decode, with the VL count it saw
+    # (a cache-mode re-selection keeps only rows still held in FP16)
+    k_after = [int(c.vl_count.min().item()) for c in layers]
+    k_after_max = [int(c.vl_count.max().item()) for c in layers]
+    total_bytes = 0
+    for s_, li, T in seen:
+        kk = cfg.k if (li not in resel_at or s_ < resel_at[li]) else k_after[li]
+        total_bytes += algorithmic_bytes(B, Hq, Hkv, T, kk)
+    dec_ms = [a.elapsed_time(b) for a, b in evs]
+    dec_avg_ms = float(np.mean(dec_ms))
+    status = max(c.status() for c in layers)
+
+    # roofline of the decode kernel (the dominant launch)
+    peak, peak_kind = measured_peaks()
+    bytes_per_decode = total_bytes / K_steps
+    achieved = bytes_per_decode / (dec_avg_ms * 1e-3) / 1e9
+    value = world * total_bytes / (elapsed_ms * 1e-3) / 1e9
+
+    # FP16 comparator (same kernel design over an all-FP16 cache), 3 copies > L2
+    fp16 = fp16_comparator(torch, hyq, cfg, Kd, Vd, q_in, dev)
+
+    # end to end through the public API with host buffers (eager loop)
+    e2e = run_e2e(torch, hyq, cfg, layers, rings, dws, sws, sel_pos, nunp, n_ctas, tokens, appended,
+                  args.e2e_steps, world, dev)
+
+    del g
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": K_steps, "warmup": W_steps, "ms_per_step": round(elapsed_ms / K_steps, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
+        "data": "synthetic (seeded N(0,1) fp16 Q/K/V, 4 K outlier channels x8, planted vertical lines)",
+        "config": {
+            "workload": "llama3.1-8b-32k-b1: decode attention, B=1/GPU, Hq=32, Hkv=8, d=128, T=32768, "
+                        "window 128, VL 3% (983), INT4 g32",
+            "step": "hyq_append + hyq_decode on one of 8 layer caches; hyq_select_vl(cache)+hyq_vl_apply "
+                    "every 64 tokens of a layer",
+            "l2": "inputs larger than L2: 8 rotating layer caches (~360 MB) per GPU",
+            "us_per_step": round(1000 * elapsed_ms / K_steps, 3),
+            "decode_us_avg": round(1000 * dec_avg_ms, 3),
+            "decode_bytes_per_step": int(bytes_per_decode),
+            "pct_of_peak_step": round(100 * value / world / peak, 1),
+            "n_ctas": n_ctas,
+            "fp16_comparator": fp16,
+            "dev_status": status,
+            "vl_rows_after_reselect": [min(k_after), max(k_after_max)],
+            "parallelism": f"replicas x{world} (independent sequences, no collective)",
+        },
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "hyq::decode_kernel<4,0>", "peak_source": f"{peak_kind} hbm_gbs",
+                     "bytes_per_launch": int(bytes_per_decode)},
+        "e2e": e2e,
+        "gpu_launches": total_launches,
+    }
+    if clk:
+        line["clocks"] = clk
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def fp16_comparator(torch, hyq, cfg, Kd, Vd, q_in, dev, copies=3, reps=60):
+    Ks = [Kd] + [Kd.clone() for _ in range(copies - 1)]
+    Vs = [Vd] + [Vd.clone() for _ in range(copies - 1)]
+    seq = torch.full((cfg.B,), cfg.T, dtype=torch.int32, device=dev)
+    o = torch.empty(cfg.B, cfg.Hq, 128, dtype=torch.float16, device=dev)
+    ws = hyq.workspace(hyq.hyq_decode_fp16_workspace(cfg.B, cfg.Hq, cfg.Hkv))
+    for i in range(6):
+        hyq.hyq_decode_fp16(q_in[i], Ks[i % copies], Vs[i % copies], seq, o, ws)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for i in range(reps):
+                evs[i][0].record()
+                hyq.hyq_decode_fp16(q_in[i % 64], Ks[i % copies], Vs[i % copies], seq, o, ws)
+                evs[i][1].record()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    nbytes = cfg.B * cfg.Hkv * cfg.T * 512 + cfg.B * cfg.Hq * 128 * 4
+    del g
+    return {"us": round(1000 * ms, 3), "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "bytes": nbytes}
+
+
+def run_e2e(torch, hyq, cfg, layers, rings, dws, sws, sel_pos, nunp, n_ctas, tokens, appended, n, world, dev):
+    """Same metric through the public API with host buffers: each step copies
+    its q / k_new / v_new from pinned host memory and reads o back."""
+    B, Hq, Hkv = cfg.B, cfg.Hq, cfg.Hkv
+    rng = np.random.default_rng(0)
+    hq = torch.from_numpy(rng.standard_normal((n, B, Hq, 128)).astype(np.float16)).pin_memory()
+    hk = torch.from_numpy(rng.standard_normal((n, B, Hkv, 128)).astype(np.float16)).pin_memory()
+    hv = torch.from_numpy(rng.standard_normal((n, B, Hkv, 128)).astype(np.float16)).pin_memory()
+    ho = torch.empty(n, B, Hq, 128, dtype=torch.float16).pin_memory()
+    dq = torch.empty(B, Hq, 128, dtype=torch.float16, device=dev)
+    dk = torch.empty(B, Hkv, 128, dtype=torch.float16, device=dev)
+    dv = torch.empty(B, Hkv, 128, dtype=torch.float16, device=dev)
+    do = torch.empty(B, Hq, 128, dtype=torch.float16, device=dev)
+    total = 0
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for s in range(n):
+        li = s % len(layers)
+        c = layers[li]
+        dq.copy_(hq[s], non_blocking=True)
+        dk.copy_(hk[s], non_blocking=True)
+        dv.copy_(hv[s], non_blocking=True)
+        hyq.hyq_append(c, dk, dv, dq, rings[li])
+        tokens[li] += 1
+        appended[li] += 1
+        if appended[li] % RESELECT == 0:
+            hyq.hyq_select_vl(c, rings[li], cfg.k, sel_pos, sws, q_is_ring=True)
+            hyq.hyq_vl_apply(c, sel_pos, n_unpromoted=nunp)
+        hyq.hyq_decode(c, dq, do, dws[li], n_ctas=n_ctas)
+        ho[s].copy_(do, non_blocking=True)
+        total += algorithmic_bytes(B, Hq, Hkv, tokens[li], cfg.k)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    return {"value": round(world * total / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": (B * Hq + 2 * B * Hkv) * 256, "d2h_bytes_per_step": B * Hq * 256,
+            "us_per_step": round(1000 * ms / n, 3), "steps": n,
+            "how": "eager loop of C-ABI calls via the ctypes binding; pinned H2D inputs + D2H output each step"}
+
+
+# --------------------------------------------------------------- CPU oracle
+def cpu_baseline(seconds, cid=2):
+    """The fp64 oracle as it stands, on the host cores, on a bounded sample:
+    whole decode steps of the same workload (all 8 units, 32K positions),
+    repeated until `seconds` of wall time; GB/s on the same algorithmic
+    bytes."""
+    import oracle
+    import synth
+    cfg = synth.config(cid)
+    K, V, planted = synth.kv_full(cfg)
+    c = oracle.OracleCache(cfg.B, cfg.Hq, cfg.Hkv, cfg.T, cfg.k)
+    c.load_prompt(K, V, [cfg.T] * cfg.B)
+    c.apply_vl(planted, K, V)
+    nbytes = algorithmic_bytes(cfg.B, cfg.Hq, cfg.Hkv, cfg.T, cfg.k)
+    steps = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.decode(c, synth.q(cfg, steps))
+        steps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": round(steps * nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{steps} full decode steps of llama3.1-8b-32k-b1 (8 units x 32768 positions), "
+                      f"{dt:.1f} s wall, OpenMP over units",
+            "us_per_step": round(1e6 * dt / steps, 1)}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    import synth
+    cfg = synth.config(2)
+    K, V, planted = synth.kv_full(cfg)
+    c = oracle.OracleCache(cfg.B, cfg.Hq, cfg.Hkv, cfg.T, cfg.k)
+    c.load_prompt(K, V, [cfg.T] * cfg.B)
+    c.apply_vl(planted, K, V)
+    # bounded sample per step: 2 of the 8 units (1/4 of a decode step)
+    units = [0, 5]
+    frac = len(units) / cfg.units
+    nbytes = algorithmic_bytes(cfg.B, cfg.Hq, cfg.Hkv, cfg.T, cfg.k) * frac
+    for s in range(args.warmup):
+        oracle.decode(c, synth.q(cfg, s), units=units)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        oracle.decode(c, synth.q(cfg, 100 + s), units=units)
+    dt = time.perf_counter() - t0
+    value = args.steps * nbytes / dt / 1e9
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * dt / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": "llama3.1-8b-32k-b1 (sample: 2 of 8 units per step)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": "each step decodes units 0 and 5 of the 32K workload (1/4 of a step)"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse_args()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)

@@ -1,0 +1,388 @@
+// hyq_pack.cu -- KV-cache compression kernels: hyq_pack (FP16 rows -> packed
+// INT4 codes + fp16 scale/zero), hyq_append (one decode step's new token:
+// the row leaving the local window is packed, the new row enters the ring)
+// and hyq_vl_apply (install a vertical-line set).
+//
+// Method: HyQuant ("HyQuant: Hybrid-Precision Quantization for LLM
+// Attention"), aifromscratch.in explainer, "How It Works" (quantized majority
+// K_Q at 4 bits for keys and values, local window K_Win of the last 128
+// tokens, vertical-line tokens K_VL in full precision) and "Two Operational
+// Modes / Decode Stage" (the KV cache is compressed to 4 bits).  The
+// quantization grid is the library's (see include/hyq.h): the pages do not
+// give one.
+//
+// One row of 128 channels is handled by 16 threads; thread t of the row owns
+// channels 8t..8t+7, i.e. group g = t/4, pieces 2(t%4) and 2(t%4)+1 of the
+// packed format.  The group min/max is a 4-lane shuffle reduction; all
+// arithmetic that decides a code is IEEE fp32 with explicit round-to-nearest
+// intrinsics (no contraction into FMA, no reciprocal).
+#include "hyq_common.cuh"
+
+namespace hyq {
+
+// Quantize this thread's 8 channels (x = 16 bytes of fp16) and write its
+// share of the packed row.  `hmask` = the 16 lanes that own this row.
+__device__ __forceinline__ void quantize_part(uint4 x, int t, unsigned hmask, uint8_t *codes_row,
+                                              uint32_t *sz_row, uint32_t *status) {
+  float v[8];
+  const __half2 *hx = reinterpret_cast<const __half2 *>(&x);
+  bool finite = true;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __half22float2(hx[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+  float mn = v[0], mx = v[0];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    finite = finite && isfinite(v[i]);
+    mn = fminf(mn, v[i]);
+    mx = fmaxf(mx, v[i]);
+  }
+  mn = fminf(mn, __shfl_xor_sync(hmask, mn, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 1));
+  mn = fminf(mn, __shfl_xor_sync(hmask, mn, 2));
+  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 2));
+  if (!finite) set_status(status, HYQ_DEV_NONFINITE);
+
+  const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+  const __half sh = __float2half_rn(s32);
+  __half zh = __float2half_rn(mn);  // exact: mn is an fp16 value
+  if (mn == 0.0f) zh = __ushort_as_half(0);
+  const float sf = __half2float(sh);
+  const float zf = __half2float(zh);
+
+  uint32_t c[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int q = 0;
+    if (sf != 0.0f) {
+      q = __float2int_rn(__fdiv_rn(__fsub_rn(v[i], zf), sf));  // ties to even
+      q = min(max(q, 0), 15);
+    }
+    c[i] = static_cast<uint32_t>(q);
+  }
+  // my bytes: piece p0 = 2(t%4): (j0, j1), piece p1 = p0 + 1: (j0, j1)
+  const uint32_t mine = (c[0] | (c[1] << 4)) | ((c[2] | (c[3] << 4)) << 8) |
+                        ((c[4] | (c[5] << 4)) << 16) | ((c[6] | (c[7] << 4)) << 24);
+  // the odd group of the pair (g = 2h+1) sits 4 lanes above the even one
+  const uint32_t other = __shfl_down_sync(hmask, mine, 4);
+  const int g = t >> 2, sub = t & 3;
+  if ((g & 1) == 0) {
+    const int h = g >> 1;
+    const int p0 = 2 * sub;
+    // word (p, h) = {g2h.j0, g2h+1.j0, g2h.j1, g2h+1.j1}
+    const uint32_t w0 = prmt(mine, other, 0x5140u);
+    const uint32_t w1 = prmt(mine, other, 0x7362u);
+    *reinterpret_cast<uint32_t *>(codes_row + 8 * p0 + 4 * h) = w0;
+    *reinterpret_cast<uint32_t *>(codes_row + 8 * (p0 + 1) + 4 * h) = w1;
+  }
+  if (sub == 0) {
+    __half2 szv = __halves2half2(sh, zh);
+    sz_row[g] = h2u(szv);
+  }
+}
+
+__global__ void __launch_bounds__(256) pack_kernel(const __half *__restrict__ x, int64_t n_rows,
+                                                   int64_t stride,
+                                                   const int64_t *__restrict__ dst_rows,
+                                                   uint8_t *__restrict__ codes,
+                                                   uint32_t *__restrict__ sz, uint32_t *status) {
+  const int lane = threadIdx.x & 31;
+  const int t = lane & 15;
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+  if (row >= n_rows) return;  // both halves of a warp exit or stay together per row
+  const unsigned hmask = 0xFFFFu << (lane & 16);
+  const uint4 xv = *reinterpret_cast<const uint4 *>(x + row * stride + 8 * t);
+  const int64_t dst = dst_rows ? dst_rows[row] : row;
+  quantize_part(xv, t, hmask, codes + dst * ROW_BYTES, sz + dst * (SZ_BYTES / 4), status);
+}
+
+// Prefill: one 16-thread group per (unit, position, K|V) row of the prompt.
+__global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half *__restrict__ k_full,
+                                                      const __half *__restrict__ v_full,
+                                                      int64_t n_rows) {
+  const int lane = threadIdx.x & 31;
+  const int t = lane & 15;
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+  if (row >= n_rows) return;
+  const bool is_v = row & 1;
+  const int64_t up = row >> 1;  // unit * capacity + position
+  const int p = static_cast<int>(up % c.capacity);
+  const int64_t u = up / c.capacity;
+  const int b = static_cast<int>(u / c.n_kv_heads);
+  const int T = c.seq_len[b];
+  if (T < 0 || T > c.capacity) {
+    if (p == 0 && t == 0 && !is_v && (u % c.n_kv_heads) == 0) set_status(c.dev_status, HYQ_DEV_BADLEN);
+    return;
+  }
+  // clear this unit's vertical-line set (bitmask words and count)
+  if (!is_v && t == 0 && p < c.capacity / 32) c.vl_mask[u * (c.capacity / 32) + p] = 0u;
+  if (!is_v && t == 0 && p == 0) c.vl_count[u] = 0;
+  if (p >= T) return;
+  const __half *src = (is_v ? v_full : k_full) + up * D;
+  const uint4 xv = *reinterpret_cast<const uint4 *>(src + 8 * t);
+  const int W = c.window;
+  if (p < T - W) {
+    const unsigned hmask = 0xFFFFu << (lane & 16);
+    uint8_t *codes = is_v ? c.v_codes : c.k_codes;
+    uint32_t *sz = reinterpret_cast<uint32_t *>(is_v ? c.v_sz : c.k_sz);
+    quantize_part(xv, t, hmask, codes + up * ROW_BYTES, sz + up * (SZ_BYTES / 4), c.dev_status);
+  } else {
+    __half *win = reinterpret_cast<__half *>(is_v ? c.win_v : c.win_k) + (u * W + p % W) * D;
+    *reinterpret_cast<uint4 *>(win + 8 * t) = xv;
+  }
+}
+
+// One block per batch b; 16 threads per (kv head, K|V) row, then the query
+// copy into the detector's ring.
+__global__ void append_kernel(hyq_cache c, const __half *__restrict__ k_new,
+                              const __half *__restrict__ v_new, const __half *__restrict__ q_new,
+                              __half *__restrict__ q_ring, int n_q) {
+  const int b = blockIdx.x;
+  const int T = c.seq_len[b];
+  __syncthreads();  // every thread has read seq_len[b] before it changes
+  if (T < 0 || T + 1 > c.capacity) {
+    if (threadIdx.x == 0) set_status(c.dev_status, HYQ_DEV_BADLEN);
+    return;
+  }
+  const int W = c.window;
+  const int slot = T % W;
+  const int n_rows = 2 * c.n_kv_heads;
+  const int row = threadIdx.x >> 4, t = threadIdx.x & 15;
+  const int lane = threadIdx.x & 31;
+  if (row < n_rows) {
+    const int h = row >> 1;
+    const bool is_v = row & 1;
+    const int64_t u = static_cast<int64_t>(b) * c.n_kv_heads + h;
+    __half *win = reinterpret_cast<__half *>(is_v ? c.win_v : c.win_k) + (u * W + slot) * D;
+    if (T >= W) {
+      const unsigned hmask = 0xFFFFu << (lane & 16);
+      const uint4 old = *reinterpret_cast<const uint4 *>(win + 8 * t);
+      const int64_t dst = u * c.capacity + (T - W);
+      uint8_t *codes = is_v ? c.v_codes : c.k_codes;
+      uint32_t *sz = reinterpret_cast<uint32_t *>(is_v ? c.v_sz : c.k_sz);
+      quantize_part(old, t, hmask, codes + dst * ROW_BYTES, sz + dst * (SZ_BYTES / 4), c.dev_status);
+    }
+    const __half *src = (is_v ? v_new : k_new) + u * D;
+    *reinterpret_cast<uint4 *>(win + 8 * t) = *reinterpret_cast<const uint4 *>(src + 8 * t);
+  }
+  if (q_new && q_ring) {
+    const int qs = T % n_q;
+    for (int i = threadIdx.x; i < c.n_q_heads * 16; i += blockDim.x) {
+      const int64_t hq = static_cast<int64_t>(b) * c.n_q_heads + (i >> 4);
+      const int part = i & 15;
+      *reinterpret_cast<uint4 *>(q_ring + (hq * n_q + qs) * D + 8 * part) =
+          *reinterpret_cast<const uint4 *>(q_new + hq * D + 8 * part);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) c.seq_len[b] = T + 1;
+}
+
+// ---------------------------------------------------------------- VL apply
+// One block per unit.  Shared memory: int32 [2][vl_capacity] (cache mode:
+// old slot and position of every kept row, in new-slot order).
+__device__ __forceinline__ int find_sorted(const int32_t *a, int n, int32_t key) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (a[mid] < key) lo = mid + 1; else hi = mid;
+  }
+  return (lo < n && a[lo] == key) ? lo : -1;
+}
+
+__global__ void __launch_bounds__(256) vl_apply_kernel(hyq_cache c, const int32_t *__restrict__ pos,
+                                                       int k, const __half *__restrict__ k_full,
+                                                       const __half *__restrict__ v_full,
+                                                       int32_t *n_unpromoted) {
+  extern __shared__ int32_t vl_list[];  // [2][vl_capacity]
+  __shared__ int red[32];
+  __shared__ int s_bad;
+  const int u = blockIdx.x;
+  const int b = u / c.n_kv_heads;
+  const int T = c.seq_len[b];
+  const int L4 = T - c.window;
+  const int32_t *np = pos + static_cast<int64_t>(u) * k;
+  int32_t *old = c.vl_pos + static_cast<int64_t>(u) * c.vl_capacity;
+  const int old_n = c.vl_count[u];
+  uint32_t *mask = c.vl_mask + static_cast<int64_t>(u) * (c.capacity / 32);
+  if (threadIdx.x == 0) s_bad = 0;
+  __syncthreads();
+  // validate the new list: ascending, within [0, T - window); old list sane
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    const int p = np[i];
+    if (p < 0 || p >= L4 || (i > 0 && np[i - 1] >= p)) s_bad = 1;
+  }
+  if (threadIdx.x == 0 && (old_n < 0 || old_n > c.vl_capacity)) s_bad = 1;
+  __syncthreads();
+  if (s_bad) {
+    if (threadIdx.x == 0) set_status(c.dev_status, HYQ_DEV_BADLEN);
+    return;
+  }
+  const int64_t row_base = static_cast<int64_t>(u) * c.vl_capacity;
+  __half *vk = reinterpret_cast<__half *>(c.vl_k);
+  __half *vv = reinterpret_cast<__half *>(c.vl_v);
+
+  if (k_full) {
+    // prefill: clear the old bits, gather the new rows, set the new bits
+    for (int i = threadIdx.x; i < old_n; i += blockDim.x) {
+      const int p = old[i];
+      if (p >= 0 && p < c.capacity) atomicAnd(&mask[p >> 5], ~(1u << (p & 31)));
+    }
+    __syncthreads();
+    const int64_t src_base = static_cast<int64_t>(u) * c.capacity;
+    for (int i = threadIdx.x; i < k * 16; i += blockDim.x) {
+      const int r = i >> 4, part = i & 15;
+      const int p = np[r];
+      const int64_t so = (src_base + p) * D + 8 * part;
+      const int64_t d = (row_base + r) * D + 8 * part;
+      *reinterpret_cast<uint4 *>(vk + d) = *reinterpret_cast<const uint4 *>(k_full + so);
+      *reinterpret_cast<uint4 *>(vv + d) = *reinterpret_cast<const uint4 *>(v_full + so);
+      if (part == 0) {
+        atomicOr(&mask[p >> 5], 1u << (p & 31));
+        old[r] = p;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) c.vl_count[u] = k;
+    return;
+  }
+
+  // cache mode: kept = new ∩ old, in ascending order.  kslot[r] = old slot
+  // of the r-th kept position, kpos[r] = that position.  Rows only move to
+  // lower slots (r <= kslot[r]), so the move is done in place in chunks.
+  int32_t *kslot = vl_list;
+  int32_t *kpos = vl_list + c.vl_capacity;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int n_kept = 0;
+  for (int base = 0; base < k; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const int j = (i < k) ? find_sorted(old, old_n, np[i]) : -1;
+    const bool kept = j >= 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, kept);
+    if (lane == 0) red[w] = __popc(bal);
+    __syncthreads();
+    int pre = 0, tot = 0;
+    for (int q = 0; q < nw; ++q) {
+      if (q < w) pre += red[q];
+      tot += red[q];
+    }
+    pre += __popc(bal & ((1u << lane) - 1u));
+    if (kept) {
+      kslot[n_kept + pre] = j;
+      kpos[n_kept + pre] = np[i];
+    }
+    n_kept += tot;
+    __syncthreads();
+  }
+  // dropped old positions fall back to their codes
+  for (int j = threadIdx.x; j < old_n; j += blockDim.x) {
+    const int p = old[j];
+    if (p >= 0 && p < c.capacity && find_sorted(np, k, p) < 0) atomicAnd(&mask[p >> 5], ~(1u << (p & 31)));
+  }
+  __syncthreads();
+  for (int base = 0; base < n_kept; base += 16) {
+    const int r = base + (threadIdx.x >> 4), part = threadIdx.x & 15;
+    const bool act = r < n_kept && (threadIdx.x >> 4) < 16;
+    uint4 rk = make_uint4(0, 0, 0, 0), rv = rk;
+    if (act) {
+      const int64_t so = (row_base + kslot[r]) * D + 8 * part;
+      rk = *reinterpret_cast<const uint4 *>(vk + so);
+      rv = *reinterpret_cast<const uint4 *>(vv + so);
+    }
+    __syncthreads();
+    if (act) {
+      const int64_t d = (row_base + r) * D + 8 * part;
+      *reinterpret_cast<uint4 *>(vk + d) = rk;
+      *reinterpret_cast<uint4 *>(vv + d) = rv;
+    }
+    __syncthreads();
+  }
+  for (int r = threadIdx.x; r < old_n || r < n_kept; r += blockDim.x)
+    old[r] = (r < n_kept) ? kpos[r] : -1;
+  if (threadIdx.x == 0) {
+    c.vl_count[u] = n_kept;
+    if (n_unpromoted) atomicAdd(n_unpromoted, k - n_kept);
+  }
+}
+
+}  // namespace hyq
+
+using namespace hyq;
+
+static inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+extern "C" hyq_status hyq_check_cache(const hyq_cache *c);  // hyq_api.cu
+
+extern "C" hyq_status hyq_pack(const void *x, int64_t n_rows, int64_t row_stride,
+                               const int64_t *dst_rows, uint8_t *codes, void *sz,
+                               uint32_t *dev_status, void *stream) {
+  if (n_rows < 0 || row_stride < D || (row_stride % 8) != 0) return HYQ_ERR_INVALID;
+  if (n_rows == 0) return HYQ_OK;
+  if (!x || !codes || !sz) return HYQ_ERR_INVALID;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(sz) || (dst_rows && !aligned16(dst_rows)))
+    return HYQ_ERR_ALIGN;
+  const int64_t threads = n_rows * 16;
+  const int64_t blocks = (threads + 255) / 256;
+  if (blocks > 0x7FFFFFFFll) return HYQ_ERR_INVALID;
+  pack_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __half *>(x), n_rows, row_stride, dst_rows, codes,
+      static_cast<uint32_t *>(sz), dev_status);
+  return cudaGetLastError() == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
+}
+
+extern "C" hyq_status hyq_prefill(const hyq_cache *c, const void *k_full, const void *v_full,
+                                  void *stream) {
+  hyq_status s = hyq_check_cache(c);
+  if (s != HYQ_OK) return s;
+  if (!k_full || !v_full) return HYQ_ERR_INVALID;
+  if (!aligned16(k_full) || !aligned16(v_full)) return HYQ_ERR_ALIGN;
+  const int64_t n_rows = static_cast<int64_t>(c->batch) * c->n_kv_heads * c->capacity * 2;
+  const int64_t blocks = (n_rows * 16 + 255) / 256;
+  if (blocks > 0x7FFFFFFFll) return HYQ_ERR_INVALID;
+  prefill_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      *c, static_cast<const __half *>(k_full), static_cast<const __half *>(v_full), n_rows);
+  return cudaGetLastError() == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
+}
+
+extern "C" hyq_status hyq_append(const hyq_cache *c, const void *k_new, const void *v_new,
+                                 const void *q_new, void *q_ring, int32_t n_q, void *stream) {
+  hyq_status s = hyq_check_cache(c);
+  if (s != HYQ_OK) return s;
+  if (!k_new || !v_new) return HYQ_ERR_INVALID;
+  if ((q_new == nullptr) != (q_ring == nullptr)) return HYQ_ERR_INVALID;
+  if (q_new && (n_q < 1 || n_q > 1024)) return HYQ_ERR_INVALID;
+  if (!aligned16(k_new) || !aligned16(v_new) || (q_new && (!aligned16(q_new) || !aligned16(q_ring))))
+    return HYQ_ERR_ALIGN;
+  if (c->n_kv_heads > 32) return HYQ_ERR_UNSUPPORTED;  // 2 rows x 16 threads per kv head
+  const int threads = 32 * c->n_kv_heads < 128 ? 128 : 32 * c->n_kv_heads;
+  append_kernel<<<c->batch, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      *c, static_cast<const __half *>(k_new), static_cast<const __half *>(v_new),
+      static_cast<const __half *>(q_new), static_cast<__half *>(q_ring), n_q);
+  return cudaGetLastError() == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
+}
+
+extern "C" hyq_status hyq_vl_apply(const hyq_cache *c, const int32_t *pos, int32_t k,
+                                   const void *k_full, const void *v_full,
+                                   int32_t *n_unpromoted, void *stream) {
+  hyq_status s = hyq_check_cache(c);
+  if (s != HYQ_OK) return s;
+  if (k < 0 || k > c->vl_capacity) return HYQ_ERR_INVALID;
+  if (k > 0 && !pos) return HYQ_ERR_INVALID;
+  if ((k_full == nullptr) != (v_full == nullptr)) return HYQ_ERR_INVALID;
+  if ((pos && !aligned16(pos)) || (k_full && (!aligned16(k_full) || !aligned16(v_full))))
+    return HYQ_ERR_ALIGN;
+  const size_t smem = 2 * sizeof(int32_t) * static_cast<size_t>(c->vl_capacity);
+  if (smem > 200 * 1024) return HYQ_ERR_UNSUPPORTED;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(vl_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    attr_set = true;
+  }
+  vl_apply_kernel<<<c->batch * c->n_kv_heads, 256, smem, static_cast<cudaStream_t>(stream)>>>(
+      *c, pos, k, static_cast<const __half *>(k_full), static_cast<const __half *>(v_full),
+      n_unpromoted);
+  return cudaGetLastError() == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
+}

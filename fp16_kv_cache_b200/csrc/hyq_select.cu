@@ -1,0 +1,569 @@
+// hyq_select.cu -- vertical-line detector: score the last n_q queries of a
+// unit's G query heads against its keys, softmax each query row, sum the
+// probabilities down every key column, keep the k largest column sums.
+//
+// Method: HyQuant.  wpnews.pro summary: the detector "accumulates query
+// vectors, runs a matrix multiplication every 64 tokens, and sums columns";
+// hotpaper.ai summary: vertical-line tokens are chosen by column-wise
+// attention score and are fewer than 5% of tokens; aifromscratch.in
+// explainer, "What to Watch For": a top-5% threshold.  Readings (the pages
+// are silent): the scores are post-softmax probabilities with scale
+// 1/sqrt(128); the column sum runs over the 64 queries and the G query heads
+// that share the KV head; query i sits at position T - n_q + i and sees keys
+// p <= T - n_q + i; candidates are positions older than the local window;
+// ties at the k-th value go to the lower position.
+//
+// Kernels (one launch each, stream ordered):
+//   1. row_stats  grid (key chunks, units): S = Q K^T on the tensor cores
+//      (mma.sync m16n8k16, query rows on M, keys on N, fp32 accumulate);
+//      per row the running max / sum of exp over the chunk's keys.
+//   2. stats_merge grid (units): log-sum-exp merge of the chunk partials in
+//      a fixed order -> (m_r, 1 / l_r).
+//   3. colsum     grid (key chunks, units): S again for candidate keys,
+//      P = exp2(S - m_r) / l_r, column sums over the rows with a fixed
+//      reduction order (no float atomics), so equal key columns give
+//      bitwise-equal sums.
+//   4. topk       grid (units): exact radix select on the fp32 bit patterns
+//      (non-negative floats order like their bits), ties to lower positions,
+//      output compacted in ascending position order.
+// Keys come from k_full (prefill) or from the cache as decode sees it: FP16
+// window and vertical-line rows, and INT4 rows dequantized as
+// zero + code * scale in fp32 and split into two fp16 terms hi + lo (both
+// multiplied on the tensor cores) so the dequantized key keeps ~22 bits.
+#include "hyq_common.cuh"
+
+namespace hyq {
+
+constexpr int SEL_SUB = 64;       // keys per shared-memory sub-tile
+constexpr int SEL_KC = 1024;      // keys per block (chunk)
+constexpr int SEL_MAX_ROWS = 512; // n_q * G
+constexpr int SEL_BLOCK_ROWS = 256;  // query rows per block (8 warps x 32)
+constexpr int TOPK_THREADS = 1024;
+constexpr float SEL_SCALE = 0.12751743082459868f;  // log2(e) / sqrt(128)
+
+struct SelectArgs {
+  int B, Hq, Hkv, G, n_q, q_ring, cap, W, vl_cap, U, R, k, n_chunks;
+  const __half *q;       // [B][Hq][n_q][128]
+  const __half *k_full;  // nullable [B][Hkv][cap][128]
+  const uint8_t *k_codes, *k_sz;
+  const __half *win_k, *vl_k;
+  const int32_t *vl_pos, *vl_count;
+  const uint32_t *vl_mask;
+  const int32_t *seq_len;
+  float2 *stats_part;  // [U][n_chunks][SEL_MAX_ROWS]
+  float2 *stats;       // [U][SEL_MAX_ROWS]  (m, 1/l)
+  float *colsum_part;  // [n_rb][U][cap]  per row block
+  float *colsum;       // [U][cap]  final column sums
+  int n_rb;            // row blocks: ceil(R / SEL_BLOCK_ROWS)
+  int32_t *out_pos;    // [U][k]
+  uint32_t *status;
+};
+
+// ldmatrix x4: four 8x8 b16 matrices, row addresses from lanes 0-7, 8-15, ...
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// Swizzled offset of 16-byte chunk c (0..15) of key row p in a [64][128] fp16
+// tile: chunk index XOR (p & 7) keeps ldmatrix row reads conflict free.
+__device__ __forceinline__ uint32_t tile_off(int p, int c) {
+  return static_cast<uint32_t>(p * 256 + ((c ^ (p & 7)) << 4));
+}
+
+__device__ __forceinline__ int sel_T(const SelectArgs &a, int u) { return a.seq_len[u / a.Hkv]; }
+
+// Fill sub-tile rows [key0, key0 + SEL_SUB) of unit u: hi (and lo in cache
+// mode) fp16 tiles.  Keys >= key_end are zero.
+template <bool CACHE>
+__device__ void fill_tile(const SelectArgs &a, int u, int T, int key0, int key_end, uint8_t *hi,
+                          uint8_t *lo, int *src_kind) {
+  const int nthr = blockDim.x;
+  if (!CACHE) {
+    const __half *base = a.k_full + static_cast<int64_t>(u) * a.cap * D;
+    for (int i = threadIdx.x; i < SEL_SUB * 16; i += nthr) {
+      const int p = i >> 4, c = i & 15;
+      const int key = key0 + p;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (key < key_end) v = *reinterpret_cast<const uint4 *>(base + static_cast<int64_t>(key) * D + 8 * c);
+      *reinterpret_cast<uint4 *>(hi + tile_off(p, c)) = v;
+    }
+    return;
+  }
+  // cache mode: src_kind[p] = -1 window, -2 INT4, >= 0 VL slot, -3 beyond
+  const int L4 = T - a.W;
+  for (int p = threadIdx.x; p < SEL_SUB; p += nthr) {
+    const int key = key0 + p;
+    int kind = -3;
+    if (key < key_end) {
+      if (key >= L4) {
+        kind = -1;
+      } else {
+        const uint32_t w = a.vl_mask[static_cast<int64_t>(u) * (a.cap / 32) + (key >> 5)];
+        kind = -2;
+        if ((w >> (key & 31)) & 1u) {
+          const int32_t *vp = a.vl_pos + static_cast<int64_t>(u) * a.vl_cap;
+          const int cnt = min(max(a.vl_count[u], 0), a.vl_cap);
+          int lo_ = 0, hi_ = cnt;
+          while (lo_ < hi_) {
+            const int mid = (lo_ + hi_) >> 1;
+            if (vp[mid] < key) lo_ = mid + 1; else hi_ = mid;
+          }
+          if (lo_ < cnt && vp[lo_] == key) kind = lo_;
+          else set_status(a.status, HYQ_DEV_OOB);
+        }
+      }
+    }
+    src_kind[p] = kind;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < SEL_SUB * 16; i += nthr) {
+    const int p = i >> 4, c = i & 15;
+    const int key = key0 + p;
+    const int kind = src_kind[p];
+    uint4 h = make_uint4(0, 0, 0, 0), l = h;
+    if (kind == -1) {
+      h = *reinterpret_cast<const uint4 *>(a.win_k + (static_cast<int64_t>(u) * a.W + key % a.W) * D + 8 * c);
+    } else if (kind >= 0) {
+      h = *reinterpret_cast<const uint4 *>(a.vl_k + (static_cast<int64_t>(u) * a.vl_cap + kind) * D + 8 * c);
+    } else if (kind == -2) {
+      // channels 8c..8c+7: group g = c / 4, pieces 2(c%4) and 2(c%4)+1
+      const int64_t row = static_cast<int64_t>(u) * a.cap + key;
+      const uint4 pc = *reinterpret_cast<const uint4 *>(a.k_codes + row * ROW_BYTES + 16 * (c & 3));
+      const int g = c >> 2, hh = g >> 1, ii = g & 1;
+      const uint32_t w0 = hh ? pc.y : pc.x;  // piece 2(c%4), word hh
+      const uint32_t w1 = hh ? pc.w : pc.z;  // piece 2(c%4)+1
+      const __half2 sz = u2h(*reinterpret_cast<const uint32_t *>(a.k_sz + row * SZ_BYTES + 4 * g));
+      const float sc = __low2float(sz), zr = __high2float(sz);
+      float x[8];
+      // byte 2j + ii of a word holds channels 2j (low) and 2j+1 (high)
+#pragma unroll
+      for (int s = 0; s < 2; ++s) {
+        const uint32_t w = s ? w1 : w0;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const uint32_t byte = (w >> (8 * (2 * j + ii))) & 0xFFu;
+          x[4 * s + 2 * j] = fmaf(static_cast<float>(byte & 15u), sc, zr);
+          x[4 * s + 2 * j + 1] = fmaf(static_cast<float>(byte >> 4), sc, zr);
+        }
+      }
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __half2 hv = __floats2half2_rn(x[2 * e], x[2 * e + 1]);
+        const float2 hf = __half22float2(hv);
+        hw[e] = h2u(hv);
+        lw[e] = h2u(__floats2half2_rn(x[2 * e] - hf.x, x[2 * e + 1] - hf.y));
+      }
+      h = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      l = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    *reinterpret_cast<uint4 *>(hi + tile_off(p, c)) = h;
+    *reinterpret_cast<uint4 *>(lo + tile_off(p, c)) = l;
+  }
+}
+
+// Q fragments of the warp's 32 rows (2 m-tiles x 8 k-steps x 4 regs).
+__device__ __forceinline__ void load_qa(const SelectArgs &a, int u, int T, int warp, int lane,
+                                        uint32_t (&qa)[2][8][4]) {
+  const int b = u / a.Hkv, kvh = u % a.Hkv;
+  const int gid = lane >> 2, t4 = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int row = 32 * warp + 16 * mt + gid + 8 * hr;
+      const __half *qr = nullptr;
+      if (row < a.R) {
+        const int hg = row / a.n_q, i = row % a.n_q;
+        int slot = i;
+        if (a.q_ring) slot = ((T - a.n_q + i) % a.n_q + a.n_q) % a.n_q;
+        qr = a.q + ((static_cast<int64_t>(b) * a.Hq + kvh * a.G + hg) * a.n_q + slot) * D;
+      }
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t v0 = 0, v1 = 0;
+        if (qr) {
+          v0 = *reinterpret_cast<const uint32_t *>(qr + 16 * ks + 2 * t4);
+          v1 = *reinterpret_cast<const uint32_t *>(qr + 16 * ks + 8 + 2 * t4);
+        }
+        qa[mt][ks][hr] = v0;      // a0 / a1: cols 2t, 2t+1
+        qa[mt][ks][2 + hr] = v1;  // a2 / a3: cols 2t+8, 2t+9
+      }
+    }
+}
+
+// S (log2 domain) for the warp's 32 rows x 64 keys of the sub-tile.
+template <bool CACHE>
+__device__ __forceinline__ void tile_scores(uint32_t hi, uint32_t lo, const uint32_t (&qa)[2][8][4],
+                                            int lane, float (&s)[2][8][4]) {
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[mt][nt][e] = 0.f;
+  // ldmatrix x4 row addresses: lanes 8j..8j+7 address key rows (nt*8 + lane%8)
+  // at chunk (2*kp + j) for matrices j = 0..3 (two k-steps per load)
+  const int kr = lane & 7, jm = lane >> 3;
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+    for (int kp = 0; kp < 4; ++kp) {
+      const int p = nt * 8 + kr, c = 4 * kp + jm;
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(hi + tile_off(p, c), b0, b1, b2, b3);
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        mma16816(s[mt][nt], qa[mt][2 * kp][0], qa[mt][2 * kp][1], qa[mt][2 * kp][2], qa[mt][2 * kp][3], b0, b1);
+        mma16816(s[mt][nt], qa[mt][2 * kp + 1][0], qa[mt][2 * kp + 1][1], qa[mt][2 * kp + 1][2],
+                 qa[mt][2 * kp + 1][3], b2, b3);
+      }
+      if (CACHE) {
+        ldsm_x4(lo + tile_off(p, c), b0, b1, b2, b3);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          mma16816(s[mt][nt], qa[mt][2 * kp][0], qa[mt][2 * kp][1], qa[mt][2 * kp][2], qa[mt][2 * kp][3], b0, b1);
+          mma16816(s[mt][nt], qa[mt][2 * kp + 1][0], qa[mt][2 * kp + 1][1], qa[mt][2 * kp + 1][2],
+                   qa[mt][2 * kp + 1][3], b2, b3);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[mt][nt][e] *= SEL_SCALE;
+}
+
+// PASS 1: per-row (max, sum exp) over the chunk; PASS 2: column sums.
+template <bool CACHE, int PASS>
+__global__ void __launch_bounds__(SEL_BLOCK_ROWS, 1) score_kernel(const SelectArgs a) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint8_t *hi = sm;
+  uint8_t *lo = sm + SEL_SUB * 256;
+  int *src_kind = reinterpret_cast<int *>(sm + 2 * SEL_SUB * 256);
+  float *cpart = reinterpret_cast<float *>(sm + 2 * SEL_SUB * 256 + SEL_SUB * 4);  // [warps][64]
+  const int u = blockIdx.y, chunk = blockIdx.x, rb = blockIdx.z;
+  const int T = sel_T(a, u);
+  const int warp = (threadIdx.x >> 5) + rb * (SEL_BLOCK_ROWS / 32), lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  if (T < a.n_q || T > a.cap || T - a.W < a.k) return;  // reported by the top-k kernel
+  const int key_end = (PASS == 1) ? T : T - a.W;
+  const int k0 = chunk * SEL_KC;
+  if (k0 >= key_end) {
+    if (PASS == 1) {
+      for (int r = threadIdx.x; r < SEL_BLOCK_ROWS; r += blockDim.x)
+        a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + rb * SEL_BLOCK_ROWS + r] =
+            make_float2(-INFINITY, 0.f);
+    }
+    return;
+  }
+  const int k1 = min(key_end, k0 + SEL_KC);
+  uint32_t qa[2][8][4];
+  load_qa(a, u, T, warp, lane, qa);
+  const int gid = lane >> 2, t4 = lane & 3;
+  // rows held by this lane: 32w + 16mt + gid + 8hr
+  float m[2][2], l[2][2], il[2][2];
+  int qpos[2][2];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int row = 32 * warp + 16 * mt + gid + 8 * hr;
+      m[mt][hr] = -INFINITY;
+      l[mt][hr] = 0.f;
+      qpos[mt][hr] = (row < a.R) ? T - a.n_q + row % a.n_q : -1;  // last visible key
+      il[mt][hr] = 0.f;
+      if (PASS == 2 && row < a.R) {
+        const float2 st = a.stats[static_cast<int64_t>(u) * SEL_MAX_ROWS + row];
+        m[mt][hr] = st.x;
+        il[mt][hr] = st.y;
+      }
+    }
+  const uint32_t hi_s = smem_u32(hi), lo_s = smem_u32(lo);
+  for (int key0 = k0; key0 < k1; key0 += SEL_SUB) {
+    __syncthreads();  // previous sub-tile fully consumed
+    fill_tile<CACHE>(a, u, T, key0, k1, hi, lo, src_kind);
+    __syncthreads();
+    float s[2][8][4];
+    tile_scores<CACHE>(hi_s, lo_s, qa, lane, s);
+    if (PASS == 1) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          float mx = -INFINITY;
+#pragma unroll
+          for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int key = key0 + nt * 8 + 2 * t4 + e;
+              const bool vis = key < k1 && key <= qpos[mt][hr];
+              float &x = s[mt][nt][2 * hr + e];
+              x = vis ? x : -INFINITY;
+              mx = fmaxf(mx, x);
+            }
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          const float mn = fmaxf(m[mt][hr], mx);
+          if (mn == -INFINITY) continue;
+          float sum = 0.f;
+#pragma unroll
+          for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) sum += fast_exp2(s[mt][nt][2 * hr + e] - mn);
+          l[mt][hr] = l[mt][hr] * fast_exp2(m[mt][hr] - mn) + sum;
+          m[mt][hr] = mn;
+        }
+    } else {
+      // probabilities, summed over this lane's 4 rows, then over the warp
+      float cs[8][2];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float acc = 0.f;
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr)
+              acc += (il[mt][hr] > 0.f) ? fast_exp2(s[mt][nt][2 * hr + e] - m[mt][hr]) * il[mt][hr] : 0.f;
+          acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+          acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+          acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+          cs[nt][e] = acc;
+        }
+      if (gid == 0) {
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) cpart[(threadIdx.x >> 5) * SEL_SUB + nt * 8 + 2 * t4 + e] = cs[nt][e];
+      }
+      __syncthreads();
+      for (int j = threadIdx.x; j < SEL_SUB; j += blockDim.x) {
+        const int key = key0 + j;
+        float tot = 0.f;
+        for (int w = 0; w < nwarps; ++w) tot += cpart[w * SEL_SUB + j];
+        if (key < k1) a.colsum_part[(static_cast<int64_t>(rb) * a.U + u) * a.cap + key] = tot;
+      }
+    }
+  }
+  if (PASS == 1) {
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        float lv = l[mt][hr];
+        lv += __shfl_xor_sync(0xffffffffu, lv, 1);
+        lv += __shfl_xor_sync(0xffffffffu, lv, 2);
+        const int row = 32 * warp + 16 * mt + gid + 8 * hr;
+        if (t4 == 0 && row < SEL_MAX_ROWS)
+          a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + row] =
+              make_float2(m[mt][hr], lv);
+      }
+  }
+}
+
+__global__ void stats_merge_kernel(const SelectArgs a) {
+  const int u = blockIdx.x;
+  const int T = sel_T(a, u);
+  if (T < a.n_q || T > a.cap) return;
+  const int nch = (T + SEL_KC - 1) / SEL_KC;
+  for (int r = threadIdx.x; r < a.R; r += blockDim.x) {
+    const float2 *p = a.stats_part + static_cast<int64_t>(u) * a.n_chunks * SEL_MAX_ROWS + r;
+    float M = -INFINITY;
+    for (int c = 0; c < nch; ++c) M = fmaxf(M, p[static_cast<int64_t>(c) * SEL_MAX_ROWS].x);
+    float L = 0.f;
+    for (int c = 0; c < nch; ++c) {
+      const float2 v = p[static_cast<int64_t>(c) * SEL_MAX_ROWS];
+      if (v.x != -INFINITY) L += v.y * fast_exp2(v.x - M);
+    }
+    a.stats[static_cast<int64_t>(u) * SEL_MAX_ROWS + r] = make_float2(M, L > 0.f ? 1.f / L : 0.f);
+  }
+}
+
+// Exact top-k of colsum[0, n) by (value desc, position asc), ascending output.
+__global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const SelectArgs a) {
+  __shared__ int hist[256];
+  __shared__ uint32_t s_prefix, s_mask;
+  __shared__ int s_need;
+  __shared__ int wsum[TOPK_THREADS / 32][2];
+  const int u = blockIdx.x;
+  const int T = sel_T(a, u);
+  const int k = a.k;
+  int32_t *out = a.out_pos + static_cast<int64_t>(u) * k;
+  if (T < a.n_q || T > a.cap || T - a.W < k) {
+    if (threadIdx.x == 0) set_status(a.status, HYQ_DEV_BADLEN);
+    for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = -1;
+    return;
+  }
+  const int n = T - a.W;
+  float *fin = a.colsum + static_cast<int64_t>(u) * a.cap;
+  if (a.n_rb > 1 || fin != a.colsum_part + static_cast<int64_t>(u) * a.cap) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      float v = 0.f;
+      for (int z = 0; z < a.n_rb; ++z) v += a.colsum_part[(static_cast<int64_t>(z) * a.U + u) * a.cap + i];
+      fin[i] = v;
+    }
+    __syncthreads();
+  }
+  const uint32_t *bits = reinterpret_cast<const uint32_t *>(fin);
+  if (threadIdx.x == 0) {
+    s_prefix = 0;
+    s_mask = 0;
+    s_need = k;
+  }
+  __syncthreads();
+  if (k > 0) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+      __syncthreads();
+      const uint32_t pre = s_prefix, msk = s_mask;
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const uint32_t b = bits[i];
+        if ((b & msk) == pre) atomicAdd(&hist[(b >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int need = s_need, cum = 0, d = 255;
+        for (; d > 0; --d) {
+          if (cum + hist[d] >= need) break;
+          cum += hist[d];
+        }
+        s_need = need - cum;
+        s_prefix = pre | (static_cast<uint32_t>(d) << shift);
+        s_mask = msk | (255u << shift);
+      }
+      __syncthreads();
+    }
+  }
+  // compaction in position order: contiguous chunk per thread
+  const uint32_t tau = s_prefix;
+  const int need_eq = (k > 0) ? s_need : 0;
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int beg = min(n, static_cast<int>(threadIdx.x) * per), end = min(n, beg + per);
+  int n_gt = 0, n_eq = 0;
+  if (k > 0)
+    for (int i = beg; i < end; ++i) {
+      const uint32_t b = bits[i];
+      n_gt += b > tau;
+      n_eq += b == tau;
+    }
+  // block exclusive scans of n_eq, then of the selected counts
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  auto block_excl = [&](int v, int which) {
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[w][which] = x;
+    __syncthreads();
+    int pre = 0;
+    for (int q = 0; q < w; ++q) pre += wsum[q][which];
+    return pre + x - v;
+  };
+  const int eq_before = block_excl(n_eq, 0);
+  const int take_eq = max(0, min(n_eq, need_eq - eq_before));
+  const int sel_before = block_excl(n_gt + take_eq, 1);
+  if (k > 0) {
+    int o = sel_before, eq_seen = 0;
+    for (int i = beg; i < end; ++i) {
+      const uint32_t b = bits[i];
+      bool take = b > tau;
+      if (b == tau) {
+        take = eq_seen < take_eq;
+        ++eq_seen;
+      }
+      if (take && o < k) out[o++] = i;
+    }
+  }
+}
+
+static cudaError_t select_launch(const SelectArgs &a, bool cache, cudaStream_t s) {
+  const int nw = a.R < SEL_BLOCK_ROWS ? (a.R + 31) / 32 : SEL_BLOCK_ROWS / 32;
+  const int threads = 32 * nw;
+  const size_t smem = 2 * SEL_SUB * 256 + SEL_SUB * 4 + static_cast<size_t>(nw) * SEL_SUB * 4;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(score_kernel<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+    cudaFuncSetAttribute(score_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+    cudaFuncSetAttribute(score_kernel<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+    cudaFuncSetAttribute(score_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+    attr = true;
+  }
+  const dim3 grid(a.n_chunks, a.U, a.n_rb);
+  if (cache) score_kernel<true, 1><<<grid, threads, smem, s>>>(a);
+  else score_kernel<false, 1><<<grid, threads, smem, s>>>(a);
+  stats_merge_kernel<<<a.U, 256, 0, s>>>(a);
+  if (cache) score_kernel<true, 2><<<grid, threads, smem, s>>>(a);
+  else score_kernel<false, 2><<<grid, threads, smem, s>>>(a);
+  topk_kernel<<<a.U, TOPK_THREADS, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace hyq
+
+using namespace hyq;
+
+extern "C" hyq_status hyq_check_cache(const hyq_cache *c);
+
+static inline bool al16s(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static size_t a256(size_t x) { return (x + 255) / 256 * 256; }
+
+extern "C" size_t hyq_select_vl_workspace(const hyq_cache *c, int32_t n_q) {
+  if (!c || c->n_kv_heads <= 0 || c->capacity <= 0 || n_q <= 0) return 0;
+  const size_t U = static_cast<size_t>(c->batch) * c->n_kv_heads;
+  const size_t nch = (static_cast<size_t>(c->capacity) + SEL_KC - 1) / SEL_KC;
+  const size_t n_rb = (static_cast<size_t>(n_q) * (c->n_q_heads / c->n_kv_heads) + SEL_BLOCK_ROWS - 1) / SEL_BLOCK_ROWS;
+  return a256(U * nch * SEL_MAX_ROWS * 8) + a256(U * SEL_MAX_ROWS * 8) + a256(U * c->capacity * 4) * (n_rb + 1);
+}
+
+extern "C" hyq_status hyq_select_vl(const hyq_cache *c, const void *q_sel, int32_t n_q,
+                                    int32_t q_is_ring, const void *k_full, int32_t k,
+                                    int32_t *out_pos, float *out_colsum, void *ws, size_t ws_bytes,
+                                    void *stream) {
+  hyq_status st = hyq_check_cache(c);
+  if (st != HYQ_OK) return st;
+  if (!q_sel || (k > 0 && !out_pos)) return HYQ_ERR_INVALID;
+  if (n_q < 1 || n_q > 64 || n_q > c->window) return HYQ_ERR_INVALID;
+  if (k < 0 || k > c->vl_capacity || k > c->capacity - c->window) return HYQ_ERR_INVALID;
+  const int G = c->n_q_heads / c->n_kv_heads;
+  if (n_q * G > SEL_MAX_ROWS) return HYQ_ERR_UNSUPPORTED;
+  if (!al16s(q_sel) || (k_full && !al16s(k_full)) || (out_pos && !al16s(out_pos)) ||
+      (out_colsum && !al16s(out_colsum)) || !al16s(ws))
+    return HYQ_ERR_ALIGN;
+  if (!ws || ws_bytes < hyq_select_vl_workspace(c, n_q)) return HYQ_ERR_WORKSPACE;
+  if (k == 0 && !out_colsum) return HYQ_OK;
+  SelectArgs a{};
+  a.B = c->batch; a.Hq = c->n_q_heads; a.Hkv = c->n_kv_heads; a.G = G; a.n_q = n_q;
+  a.q_ring = q_is_ring ? 1 : 0; a.cap = c->capacity; a.W = c->window; a.vl_cap = c->vl_capacity;
+  a.U = c->batch * c->n_kv_heads; a.R = n_q * G; a.k = k;
+  a.n_chunks = (c->capacity + SEL_KC - 1) / SEL_KC;
+  a.q = static_cast<const __half *>(q_sel);
+  a.k_full = static_cast<const __half *>(k_full);
+  a.k_codes = c->k_codes; a.k_sz = static_cast<const uint8_t *>(c->k_sz);
+  a.win_k = static_cast<const __half *>(c->win_k); a.vl_k = static_cast<const __half *>(c->vl_k);
+  a.vl_pos = c->vl_pos; a.vl_count = c->vl_count; a.vl_mask = c->vl_mask; a.seq_len = c->seq_len;
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  const size_t U = a.U;
+  a.stats_part = reinterpret_cast<float2 *>(w);
+  w += a256(U * a.n_chunks * SEL_MAX_ROWS * 8);
+  a.stats = reinterpret_cast<float2 *>(w);
+  w += a256(U * SEL_MAX_ROWS * 8);
+  a.n_rb = (a.R + SEL_BLOCK_ROWS - 1) / SEL_BLOCK_ROWS;
+  a.colsum_part = reinterpret_cast<float *>(w);
+  w += a256(U * c->capacity * 4) * a.n_rb;
+  a.colsum = out_colsum ? out_colsum : (a.n_rb == 1 ? a.colsum_part : reinterpret_cast<float *>(w));
+  a.out_pos = out_pos;
+  a.status = c->dev_status;
+  return select_launch(a, k_full == nullptr, static_cast<cudaStream_t>(stream)) == cudaSuccess ? HYQ_OK
+                                                                                                : HYQ_ERR_CUDA;
+}

@@ -1,0 +1,235 @@
+"""Thin Python binding of libhyq.so (the C ABI in include/hyq.h).
+
+Argument marshalling only: torch tensors supply device memory and streams,
+every computation runs in the library's CUDA kernels.  There is no CPU or
+PyTorch fallback: if the shared library is missing or no CUDA device is
+present, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+HEAD_DIM = 128
+GROUP = 32
+WINDOW = 128
+ROW_BYTES = 64
+
+DEV_NONFINITE = 0x1
+DEV_OOB = 0x2
+DEV_TIMEOUT = 0x4
+DEV_BADLEN = 0x8
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "pointer not 16-byte aligned",
+          4: "workspace missing or too small", 5: "CUDA launch error"}
+
+_lib = None
+
+
+class HyqError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(code, code)} (hyq status {code})")
+        self.code = code
+
+
+class hyq_cache(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("group", ctypes.c_int32), ("window", ctypes.c_int32),
+        ("capacity", ctypes.c_int32), ("vl_capacity", ctypes.c_int32),
+        ("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
+        ("k_sz", ctypes.c_void_p), ("v_sz", ctypes.c_void_p),
+        ("win_k", ctypes.c_void_p), ("win_v", ctypes.c_void_p),
+        ("vl_k", ctypes.c_void_p), ("vl_v", ctypes.c_void_p),
+        ("vl_pos", ctypes.c_void_p), ("vl_count", ctypes.c_void_p),
+        ("vl_mask", ctypes.c_void_p), ("seq_len", ctypes.c_void_p),
+        ("dev_status", ctypes.c_void_p),
+    ]
+
+
+# (name, restype, argtypes) of every exported entry point
+_P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_CP = ctypes.POINTER(hyq_cache)
+EXPORTS = [
+    ("hyq_pack", ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
+    ("hyq_prefill", ctypes.c_int, [_CP, _P, _P, _P]),
+    ("hyq_append", ctypes.c_int, [_CP, _P, _P, _P, _P, _I32, _P]),
+    ("hyq_select_vl_workspace", _SZ, [_CP, _I32]),
+    ("hyq_select_vl", ctypes.c_int, [_CP, _P, _I32, _I32, _P, _I32, _P, _P, _P, _SZ, _P]),
+    ("hyq_vl_apply", ctypes.c_int, [_CP, _P, _I32, _P, _P, _P, _P]),
+    ("hyq_decode_workspace", _SZ, [_CP, _I32]),
+    ("hyq_decode", ctypes.c_int, [_CP, _P, _P, _P, _I32, _P, _SZ, _P]),
+    ("hyq_decode_fp16_workspace", _SZ, [_I32, _I32, _I32, _I32]),
+    ("hyq_decode_fp16", ctypes.c_int, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _I32, _P, _SZ, _P, _P]),
+    ("hyq_status_string", ctypes.c_char_p, [ctypes.c_int]),
+    ("hyq_decode_default_ctas", _I32, []),
+    ("hyq_version", _I32, []),
+]
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def lib():
+    """Load libhyq.so (built in-tree by ``python -m fp16_kv_cache_b200.build``)."""
+    global _lib
+    if _lib is None:
+        path = lib_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is not built: run `python -m fp16_kv_cache_b200.build`")
+        L = ctypes.CDLL(path)
+        for name, res, args in EXPORTS:
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libhyq takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libhyq takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise HyqError(int(rc), what)
+
+
+# ------------------------------------------------------------------ cache
+class HybridCache:
+    """Device buffers of one layer's hybrid cache plus its C descriptor."""
+
+    def __init__(self, batch, n_q_heads, n_kv_heads, capacity, vl_capacity, device="cuda"):
+        if capacity % 128:
+            raise ValueError("capacity must be a multiple of 128")
+        B, Hkv = batch, n_kv_heads
+        dev = torch.device(device)
+        z = lambda *s, dt: torch.zeros(*s, dtype=dt, device=dev)  # noqa: E731
+        self.B, self.Hq, self.Hkv, self.cap, self.vl_cap = B, n_q_heads, Hkv, capacity, vl_capacity
+        self.k_codes = z(B, Hkv, capacity, ROW_BYTES, dt=torch.uint8)
+        self.v_codes = z(B, Hkv, capacity, ROW_BYTES, dt=torch.uint8)
+        self.k_sz = z(B, Hkv, capacity, 8, dt=torch.float16)
+        self.v_sz = z(B, Hkv, capacity, 8, dt=torch.float16)
+        self.win_k = z(B, Hkv, WINDOW, HEAD_DIM, dt=torch.float16)
+        self.win_v = z(B, Hkv, WINDOW, HEAD_DIM, dt=torch.float16)
+        self.vl_k = z(B, Hkv, vl_capacity, HEAD_DIM, dt=torch.float16)
+        self.vl_v = z(B, Hkv, vl_capacity, HEAD_DIM, dt=torch.float16)
+        self.vl_pos = z(B, Hkv, vl_capacity, dt=torch.int32)
+        self.vl_count = z(B, Hkv, dt=torch.int32)
+        self.vl_mask = z(B, Hkv, capacity // 32, dt=torch.int32)  # bit pattern of uint32 words
+        self.seq_len = z(B, dt=torch.int32)
+        self.dev_status = z(4, dt=torch.int32)
+        c = hyq_cache()
+        c.batch, c.n_q_heads, c.n_kv_heads = B, n_q_heads, Hkv
+        c.head_dim, c.group, c.window = HEAD_DIM, GROUP, WINDOW
+        c.capacity, c.vl_capacity = capacity, vl_capacity
+        for name in ("k_codes", "v_codes", "k_sz", "v_sz", "win_k", "win_v", "vl_k", "vl_v",
+                     "vl_pos", "vl_count", "vl_mask", "seq_len", "dev_status"):
+            setattr(c, name, getattr(self, name).data_ptr())
+        self.desc = c
+
+    def ref(self):
+        return ctypes.byref(self.desc)
+
+    def status(self) -> int:
+        return int(self.dev_status[0].item()) & 0xFFFFFFFF
+
+    def clear_status(self):
+        self.dev_status.zero_()
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (
+            self.k_codes, self.v_codes, self.k_sz, self.v_sz, self.win_k, self.win_v,
+            self.vl_k, self.vl_v, self.vl_pos, self.vl_count, self.vl_mask, self.seq_len))
+
+
+# ------------------------------------------------------------------ entry points
+def hyq_pack(x, codes, sz, dst_rows=None, dev_status=None, stream=None):
+    """x: fp16 [n][stride] (row-contiguous); codes u8 [*][64]; sz fp16 [*][8]."""
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit column stride")
+    n, stride = x.shape[0], x.stride(0)
+    if not x.is_cuda:
+        raise ValueError("libhyq takes device tensors")
+    rc = lib().hyq_pack(ctypes.c_void_p(x.data_ptr()), n, stride, _ptr(dst_rows), _ptr(codes),
+                        _ptr(sz), _ptr(dev_status), _stream(stream))
+    _check(rc, "hyq_pack")
+
+
+def hyq_prefill(cache: HybridCache, k_full, v_full, stream=None):
+    _check(lib().hyq_prefill(cache.ref(), _ptr(k_full), _ptr(v_full), _stream(stream)), "hyq_prefill")
+
+
+def hyq_append(cache: HybridCache, k_new, v_new, q_new=None, q_ring=None, stream=None):
+    n_q = 0 if q_ring is None else q_ring.shape[2]
+    _check(lib().hyq_append(cache.ref(), _ptr(k_new), _ptr(v_new), _ptr(q_new), _ptr(q_ring), n_q,
+                            _stream(stream)), "hyq_append")
+
+
+def hyq_select_vl_workspace(cache: HybridCache, n_q: int) -> int:
+    return int(lib().hyq_select_vl_workspace(cache.ref(), n_q))
+
+
+def hyq_select_vl(cache: HybridCache, q_sel, k, out_pos, ws, out_colsum=None, k_full=None,
+                  q_is_ring=False, stream=None):
+    n_q = q_sel.shape[2]
+    _check(lib().hyq_select_vl(cache.ref(), _ptr(q_sel), n_q, int(bool(q_is_ring)), _ptr(k_full), k,
+                               _ptr(out_pos), _ptr(out_colsum), _ptr(ws), ws.numel() * ws.element_size(),
+                               _stream(stream)), "hyq_select_vl")
+
+
+def hyq_vl_apply(cache: HybridCache, pos, k_full=None, v_full=None, n_unpromoted=None, stream=None):
+    k = pos.shape[-1]
+    _check(lib().hyq_vl_apply(cache.ref(), _ptr(pos), k, _ptr(k_full), _ptr(v_full),
+                              _ptr(n_unpromoted), _stream(stream)), "hyq_vl_apply")
+
+
+def hyq_decode_workspace(cache: HybridCache, n_ctas: int = 0) -> int:
+    return int(lib().hyq_decode_workspace(cache.ref(), n_ctas))
+
+
+def hyq_decode(cache: HybridCache, q, o, ws, lse=None, n_ctas: int = 0, stream=None):
+    _check(lib().hyq_decode(cache.ref(), _ptr(q), _ptr(o), _ptr(lse), n_ctas, _ptr(ws),
+                            ws.numel() * ws.element_size(), _stream(stream)), "hyq_decode")
+
+
+def hyq_decode_fp16_workspace(batch, n_q_heads, n_kv_heads, n_ctas: int = 0) -> int:
+    return int(lib().hyq_decode_fp16_workspace(batch, n_q_heads, n_kv_heads, n_ctas))
+
+
+def hyq_decode_fp16(q, k, v, seq_len, o, ws, lse=None, n_ctas: int = 0, dev_status=None, stream=None):
+    B, Hkv, cap, _ = k.shape
+    Hq = q.shape[1]
+    _check(lib().hyq_decode_fp16(_ptr(q), _ptr(k), _ptr(v), _ptr(seq_len), B, Hq, Hkv, cap, _ptr(o),
+                                 _ptr(lse), n_ctas, _ptr(ws), ws.numel() * ws.element_size(),
+                                 _ptr(dev_status), _stream(stream)), "hyq_decode_fp16")
+
+
+def hyq_decode_default_ctas() -> int:
+    return int(lib().hyq_decode_default_ctas())
+
+
+def hyq_version() -> int:
+    return int(lib().hyq_version())
+
+
+def workspace(nbytes: int, device="cuda"):
+    """A zero-filled byte workspace (16-byte aligned, as torch allocations are)."""
+    return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)

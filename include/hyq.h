@@ -1,0 +1,252 @@
+/*
+ * hyq.h -- C ABI of libhyq.so: decode-stage attention over a hybrid
+ * INT4/FP16 KV cache with fused dequantization (HyQuant), for NVIDIA B200
+ * (sm_100a).
+ *
+ * The method ("HyQuant: Hybrid-Precision Quantization for LLM Attention",
+ * arXiv 2608.27875): keys and values of most cached tokens are stored in
+ * 4-bit form; a small set of vertical-line tokens (< 5% of positions, chosen
+ * from column-summed attention scores of recent queries) and a local window
+ * of the last 128 tokens stay in FP16; decode dequantizes on the fly inside
+ * the attention kernel.  Sources: aifromscratch.in explainer, sections "How
+ * It Works" (three token classes) and "Two Operational Modes / Decode Stage"
+ * (fused dequantization); wpnews.pro summary (the detector accumulates
+ * queries, runs a matrix multiplication every 64 tokens and sums columns);
+ * hotpaper.ai summary (column-wise attention score, < 5% of tokens).
+ *
+ * Conventions for every entry point
+ *   - Memory: every pointer is DEVICE memory owned by the caller, unless the
+ *     argument says "host".  The library never allocates, frees or
+ *     synchronizes.  Scratch space is passed in as a workspace whose size the
+ *     matching *_workspace() query returns.
+ *   - Asynchrony: work is enqueued on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  A return other than HYQ_OK means nothing was
+ *     enqueued, except HYQ_ERR_CUDA, which reports a launch error.
+ *   - Validation is synchronous and host-side (shapes, alignment, null
+ *     pointers).  Conditions only the device can see (a sequence length out
+ *     of range, a non-finite input to the quantizer, a bounded wait that ran
+ *     out) are OR-ed into the optional device status word `dev_status`
+ *     (uint32, HYQ_DEV_* bits) which the caller reads after synchronizing.
+ *   - Alignment: every device pointer must be 16-byte aligned.
+ *   - Fixed sizes: head_dim 128, quantization group 32, window 128;
+ *     G = n_q_heads / n_kv_heads must be 1, 2, 4 or 8 (query head h reads
+ *     KV head h / G).
+ *   - Stateless and reentrant; the library caches the SM count per device.
+ */
+#ifndef HYQ_H
+#define HYQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HYQ_OK = 0,
+  HYQ_ERR_INVALID = 1,     /* bad argument: null pointer, shape, count */
+  HYQ_ERR_UNSUPPORTED = 2, /* head_dim/group/window/G outside the fixed set */
+  HYQ_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  HYQ_ERR_WORKSPACE = 4,   /* workspace missing or too small */
+  HYQ_ERR_CUDA = 5         /* the CUDA runtime reported an error at launch */
+} hyq_status;
+
+/* device status word bits */
+#define HYQ_DEV_NONFINITE 0x1u /* the quantizer saw Inf/NaN (codes undefined) */
+#define HYQ_DEV_OOB 0x2u       /* a device-side index check failed           */
+#define HYQ_DEV_TIMEOUT 0x4u   /* a bounded wait expired; outputs undefined   */
+#define HYQ_DEV_BADLEN 0x8u    /* seq_len / vl_count out of range; skipped    */
+
+#define HYQ_HEAD_DIM 128
+#define HYQ_GROUP 32
+#define HYQ_WINDOW 128
+#define HYQ_ROW_BYTES 64 /* packed INT4 codes per row (128 x 4 bit)        */
+#define HYQ_SZ_BYTES 16  /* fp16 (scale, zero) x 4 groups per row           */
+
+/*
+ * Packed INT4 row format (64 bytes per row of 128 channels).  Channel c is in
+ * group g = c / 32 at offset w = c % 32.  The row is 8 pieces of 8 bytes;
+ * piece p = w / 4 holds channels 4p..4p+3 of every group.  Inside a piece,
+ * byte 4*(g/2) + 2*j + (g%2), j = (w/2) % 2, holds channel w = 4p + 2j in its
+ * low nibble and w = 4p + 2j + 1 in its high nibble.  (Chosen so that one
+ * 16-byte load yields eight channels of every group and the nibble-to-fp16
+ * conversion pairs two channels of one group per 32-bit word.)
+ * Scale/zero row: fp16 {scale_0, zero_0, scale_1, zero_1, ..., zero_3}.
+ *
+ * Quantizer (the pages give only "4-bit for both keys and values"; this
+ * grid is fixed by the library): per group, mn/mx = min/max; scale =
+ * fp16(fp32(mx - mn) / 15) with fp32 IEEE round-to-nearest-even; zero = mn
+ * (a -0 minimum is stored as +0); code = 0 if scale == 0, else
+ * clamp(round_half_even(fp32(x - zero) / fp32(scale)), 0, 15), computed with
+ * IEEE fp32 subtraction and division (no FMA, no reciprocal).  Dequantized
+ * value: zero + code * scale.
+ */
+
+/*
+ * The hybrid cache of one layer.  All arrays are caller-owned device memory
+ * and must be zero-filled before first use.  Per unit u = b * n_kv_heads + h:
+ *   quantized majority  positions [0, T - window):  k_codes/v_codes
+ *                       [B][Hkv][capacity][64] u8, k_sz/v_sz
+ *                       [B][Hkv][capacity][8] fp16;
+ *   vertical-line rows  vl_k/vl_v [B][Hkv][vl_capacity][128] fp16, in the
+ *                       ascending order of vl_pos [B][Hkv][vl_capacity];
+ *                       vl_count [B][Hkv] rows are valid; vl_mask
+ *                       [B][Hkv][capacity/32] u32 has bit p%32 of word p/32
+ *                       set exactly for the positions held in vl_k/vl_v;
+ *   local window        win_k/win_v [B][Hkv][window][128] fp16, position p
+ *                       in slot p % window, positions [max(0, T-window), T);
+ *   seq_len [B] int32   T, the number of positions, newest token included.
+ */
+typedef struct {
+  int32_t batch, n_q_heads, n_kv_heads;
+  int32_t head_dim;    /* must be 128 */
+  int32_t group;       /* must be 32  */
+  int32_t window;      /* must be 128 */
+  int32_t capacity;    /* max positions per sequence, multiple of 64 */
+  int32_t vl_capacity; /* max vertical-line rows per unit, >= 1 */
+  uint8_t *k_codes, *v_codes;
+  void *k_sz, *v_sz;
+  void *win_k, *win_v;
+  void *vl_k, *vl_v;
+  int32_t *vl_pos;
+  int32_t *vl_count;
+  uint32_t *vl_mask;
+  int32_t *seq_len;
+  uint32_t *dev_status; /* nullable */
+} hyq_cache;
+
+/*
+ * hyq_pack -- quantize FP16 rows to packed INT4 codes and fp16 scale/zero
+ * (the KV-cache compression of the decode stage).
+ *   x          fp16 rows, row i at x + i*row_stride (elements), 128 values
+ *   n_rows     >= 0 (0 enqueues nothing)
+ *   row_stride >= 128, multiple of 8
+ *   dst_rows   nullable int64 [n_rows]: row i goes to output row dst_rows[i]
+ *              (scatter); NULL means row i -> row i
+ *   codes      u8 [*][64] output; sz fp16 [*][8] output
+ *   dev_status nullable; HYQ_DEV_NONFINITE is set for a row holding Inf/NaN
+ */
+hyq_status hyq_pack(const void *x, int64_t n_rows, int64_t row_stride,
+                    const int64_t *dst_rows, uint8_t *codes, void *sz,
+                    uint32_t *dev_status, void *stream);
+
+/*
+ * hyq_prefill -- build the cache from a prompt (end of prefill).  For every
+ * unit with T = seq_len[b] (device): rows [0, T - window) of k_full/v_full
+ * are quantized into the codes (as hyq_pack), rows [max(0, T - window), T)
+ * are copied into the window ring, and the vertical-line set is emptied
+ * (vl_count = 0, vl_mask cleared).
+ *   k_full, v_full  fp16 [B][Hkv][capacity][128]
+ * Sets HYQ_DEV_BADLEN (and skips the batch) when T is outside [0, capacity];
+ * HYQ_DEV_NONFINITE as hyq_pack.
+ */
+hyq_status hyq_prefill(const hyq_cache *c, const void *k_full, const void *v_full,
+                       void *stream);
+
+/*
+ * hyq_append -- add one token per sequence to the cache (decode step).
+ * For every batch b with T = seq_len[b]: the row leaving the window
+ * (position T - window, when T >= window) is packed into the codes, the new
+ * K/V row takes window slot T % window, and seq_len[b] becomes T + 1.
+ *   k_new, v_new  fp16 [B][Hkv][128]
+ *   q_new, q_ring nullable together: q_new fp16 [B][Hq][128] is copied to
+ *                 q_ring fp16 [B][Hq][n_q][128] at slot T % n_q (the ring of
+ *                 recent queries the vertical-line detector accumulates)
+ * Sets HYQ_DEV_BADLEN (and skips the batch) when T + 1 > capacity.
+ */
+hyq_status hyq_append(const hyq_cache *c, const void *k_new, const void *v_new,
+                      const void *q_new, void *q_ring, int32_t n_q, void *stream);
+
+/*
+ * hyq_select_vl -- vertical-line detector.  For every unit, the n_q most
+ * recent queries of each of its G query heads (R = n_q * G rows) are scored
+ * against the keys; query i sits at position T - n_q + i and sees keys
+ * p <= T - n_q + i.  Each row becomes a softmax over (q . k) / sqrt(128);
+ * the probabilities are summed down each key column; the k largest column
+ * sums among positions [0, T - window) are returned, ties to the lower
+ * position, in ascending order.
+ *   q_sel      fp16 [B][Hq][n_q][128]; q_is_ring = 0: row i at index i;
+ *              q_is_ring = 1: the row of position p at index p % n_q (the
+ *              layout hyq_append writes)
+ *   n_q        1..64 (64 in the method)
+ *   k_full     nullable fp16 [B][Hkv][capacity][128]: score these keys
+ *              (prefill); NULL scores the cache as decode sees it
+ *   k          number of positions to select, 0 <= k <= vl_capacity;
+ *              a unit whose T - window < k sets HYQ_DEV_BADLEN
+ *   out_pos    int32 [B][Hkv][k]
+ *   out_colsum nullable fp32 [B][Hkv][capacity] (non-candidates 0)
+ *   ws         workspace of hyq_select_vl_workspace(c, n_q) bytes
+ * Requires window >= n_q.
+ */
+size_t hyq_select_vl_workspace(const hyq_cache *c, int32_t n_q);
+hyq_status hyq_select_vl(const hyq_cache *c, const void *q_sel, int32_t n_q,
+                         int32_t q_is_ring, const void *k_full, int32_t k,
+                         int32_t *out_pos, float *out_colsum, void *ws,
+                         size_t ws_bytes, void *stream);
+
+/*
+ * hyq_vl_apply -- make `pos` the vertical-line set.
+ *   pos        int32 [B][Hkv][k], ascending, within [0, T - window)
+ *   k_full/v_full  non-NULL (prefill): the FP16 rows are gathered from
+ *              these [B][Hkv][capacity][128] arrays.  NULL (cache mode):
+ *              positions already held in FP16 keep their rows, positions
+ *              no longer selected fall back to their INT4 codes, and newly
+ *              selected positions, whose FP16 copy is gone, stay INT4 and
+ *              are counted in *n_unpromoted (nullable device int32,
+ *              accumulated with atomicAdd; zero it first).
+ * Rows move only towards lower slots, so the update is done in place.
+ */
+hyq_status hyq_vl_apply(const hyq_cache *c, const int32_t *pos, int32_t k,
+                        const void *k_full, const void *v_full,
+                        int32_t *n_unpromoted, void *stream);
+
+/*
+ * hyq_decode -- one decode step of GQA attention over the hybrid cache,
+ * INT4 dequantization fused into the attention (split-KV flash decoding:
+ * work is spread over n_ctas thread blocks by tile count, per-block partial
+ * (max, sum, accumulator) triples are merged by log-sum-exp in the last
+ * block to finish a unit).
+ *   q    fp16 [B][Hq][128]; o fp16 [B][Hq][128] output
+ *   lse  nullable fp32 [B][Hq]: natural-log sum of exp of the scaled logits
+ *   n_ctas  thread blocks; 0 = automatic (a multiple of the SM count)
+ *   ws   workspace of hyq_decode_workspace(c, n_ctas) bytes; zero-filled
+ *        before the first call, every completed call leaves it reusable
+ *        (re-zero it after a call that reported HYQ_DEV_TIMEOUT)
+ * Scale 1/sqrt(128); all softmax arithmetic in fp32.
+ */
+size_t hyq_decode_workspace(const hyq_cache *c, int32_t n_ctas);
+hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, float *lse,
+                      int32_t n_ctas, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * hyq_decode_fp16 -- the same decode kernel design over an all-FP16 cache
+ * (the full-precision comparator).
+ *   q fp16 [B][Hq][128]; k, v fp16 [B][Hkv][capacity][128]; seq_len int32 [B]
+ *   o fp16 [B][Hq][128]; lse nullable fp32 [B][Hq]
+ *   ws   workspace of hyq_decode_fp16_workspace(B, Hq, Hkv, n_ctas) bytes,
+ *        zero-filled before the first call
+ */
+size_t hyq_decode_fp16_workspace(int32_t batch, int32_t n_q_heads,
+                                 int32_t n_kv_heads, int32_t n_ctas);
+hyq_status hyq_decode_fp16(const void *q, const void *k, const void *v,
+                           const int32_t *seq_len, int32_t batch,
+                           int32_t n_q_heads, int32_t n_kv_heads,
+                           int32_t capacity, void *o, float *lse,
+                           int32_t n_ctas, void *ws, size_t ws_bytes,
+                           uint32_t *dev_status, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *hyq_status_string(hyq_status s);
+
+/* Number of thread blocks n_ctas = 0 selects for the decode kernels on the
+ * current device (host query; needs a current CUDA device). */
+int32_t hyq_decode_default_ctas(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int32_t hyq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HYQ_H */

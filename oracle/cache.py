@@ -46,12 +46,14 @@ class OracleCache:
         self.seq_len = np.zeros(B, np.int32)
 
     # ------------------------------------------------------------ prompt
-    def load_prompt(self, K, V, seq_len):
+    def load_prompt(self, K, V, seq_len, units=None):
         """K, V: [B][Hkv][>=T][128] fp16 (as uint16 bits or float16).
-        Packs [0, T-W) and fills the window with [max(0, T-W), T)."""
+        Packs [0, T-W) and fills the window with [max(0, T-W), T).  With
+        `units`, only those (b * Hkv + h) units are filled."""
         K = np.asarray(K).view(np.uint16)
         V = np.asarray(V).view(np.uint16)
         seq_len = np.asarray(seq_len, np.int32)
+        keep = None if units is None else set(int(u) for u in units)
         for b in range(self.B):
             T = int(seq_len[b])
             assert 0 <= T <= self.cap
@@ -59,6 +61,8 @@ class OracleCache:
             n_old = max(0, T - self.W)
             for h in range(self.Hkv):
                 u = b * self.Hkv + h
+                if keep is not None and u not in keep:
+                    continue
                 if n_old:
                     c, s, bad = pack(K[b, h, :n_old])
                     assert bad == 0
@@ -73,7 +77,7 @@ class OracleCache:
                 self.vl_pos[u] = -1
 
     # ------------------------------------------------------------ VL set
-    def apply_vl(self, pos, K_full=None, V_full=None):
+    def apply_vl(self, pos, K_full=None, V_full=None, units=None):
         """pos: [B][Hkv][k] ascending.  With K_full/V_full (prefill mode) the
         FP16 rows come from them; without (cache mode) only positions already
         held in FP16 stay FP16.  Returns the number of unpromoted positions."""
@@ -84,9 +88,12 @@ class OracleCache:
         if K_full is not None:
             K_full = np.asarray(K_full).view(np.uint16)
             V_full = np.asarray(V_full).view(np.uint16)
+        keep = None if units is None else set(int(u) for u in units)
         for b in range(self.B):
             for h in range(self.Hkv):
                 u = b * self.Hkv + h
+                if keep is not None and u not in keep:
+                    continue
                 new = [int(p) for p in pos[b, h]]
                 if K_full is not None:
                     rows_k = [K_full[b, h, p] for p in new]

@@ -1,0 +1,110 @@
+"""The C-ABI library: builds, loads, exports every entry point the header
+declares, and rejects bad arguments on the host without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp16_kv_cache_b200 import build as hbuild
+from fp16_kv_cache_b200 import hyq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hyq.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    hbuild.build()
+    return hyq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hyq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("hyq_pack", "hyq_prefill", "hyq_append", "hyq_select_vl", "hyq_vl_apply",
+              "hyq_decode", "hyq_decode_fp16", "hyq_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+    assert {n for n, _, _ in hyq.EXPORTS} == set(declared_functions())
+
+
+def test_version_and_status_strings(L):
+    assert L.hyq_version() == 100
+    for code, text in hyq.STATUS.items():
+        assert L.hyq_status_string(code).decode() == text
+
+
+def _desc(**over):
+    c = hyq.hyq_cache()
+    c.batch, c.n_q_heads, c.n_kv_heads = 1, 8, 2
+    c.head_dim, c.group, c.window, c.capacity, c.vl_capacity = 128, 32, 128, 4096, 64
+    fake = 0x10000  # aligned, never dereferenced: validation fails or stops first
+    for name in ("k_codes", "v_codes", "k_sz", "v_sz", "win_k", "win_v", "vl_k", "vl_v",
+                 "vl_pos", "vl_count", "vl_mask", "seq_len"):
+        setattr(c, name, fake)
+        fake += 0x10000
+    for k, v in over.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("head_dim", 64, 2), ("group", 64, 2), ("window", 256, 2), ("n_q_heads", 7, 1), ("n_q_heads", 6, 2),
+    ("n_q_heads", 24, 2), ("capacity", 4000, 1), ("capacity", 0, 1), ("vl_capacity", 0, 1),
+    ("batch", 0, 1), ("k_codes", 0, 1), ("vl_mask", 0x10008, 3), ("seq_len", None, 1),
+])
+def test_decode_rejects_bad_descriptors(L, field, value, code):
+    c = _desc(**{field: value})
+    rc = L.hyq_decode(ctypes.byref(c), 0x20000000, 0x30000000, None, 0, 0x40000000, 1 << 30, None)
+    assert rc == code
+
+
+def test_decode_requires_workspace(L):
+    c = _desc()
+    assert L.hyq_decode(ctypes.byref(c), 0x20000000, 0x30000000, None, 8, None, 0, None) == 4
+    need = L.hyq_decode_workspace(ctypes.byref(c), 8)
+    assert need > 0
+    assert L.hyq_decode(ctypes.byref(c), 0x20000000, 0x30000000, None, 8, 0x40000000, need - 1, None) == 4
+    assert L.hyq_decode(ctypes.byref(c), 0x20000008, 0x30000000, None, 8, 0x40000000, need, None) == 3
+
+
+def test_pack_argument_checks(L):
+    assert L.hyq_pack(0x1000, 0, 128, None, 0x2000, 0x3000, None, None) == 0   # nothing to do
+    assert L.hyq_pack(0x1000, -1, 128, None, 0x2000, 0x3000, None, None) == 1
+    assert L.hyq_pack(0x1000, 4, 100, None, 0x2000, 0x3000, None, None) == 1
+    assert L.hyq_pack(0x1000, 4, 132, None, 0x2000, 0x3000, None, None) == 1
+    assert L.hyq_pack(0x1004, 4, 128, None, 0x2000, 0x3000, None, None) == 3
+    assert L.hyq_pack(None, 4, 128, None, 0x2000, 0x3000, None, None) == 1
+
+
+def test_select_and_vl_apply_argument_checks(L):
+    c = _desc()
+    ws = L.hyq_select_vl_workspace(ctypes.byref(c), 64)
+    assert ws > 0
+    sel = L.hyq_select_vl
+    assert sel(ctypes.byref(c), 0x1000, 0, 0, None, 8, 0x2000, None, 0x4000, ws, None) == 1     # n_q
+    assert sel(ctypes.byref(c), 0x1000, 65, 0, None, 8, 0x2000, None, 0x4000, ws, None) == 1    # n_q
+    assert sel(ctypes.byref(c), 0x1000, 64, 0, None, 65, 0x2000, None, 0x4000, ws, None) == 1   # k > vl_cap
+    assert sel(ctypes.byref(c), 0x1000, 64, 0, None, 8, 0x2000, None, 0x4000, ws - 1, None) == 4
+    assert L.hyq_vl_apply(ctypes.byref(c), 0x1000, 65, None, None, None, None) == 1
+    assert L.hyq_vl_apply(ctypes.byref(c), 0x1000, 8, 0x2000, None, None, None) == 1  # k_full w/o v_full
+
+
+def test_append_and_prefill_argument_checks(L):
+    c = _desc()
+    assert L.hyq_append(ctypes.byref(c), None, 0x2000, None, None, 0, None) == 1
+    assert L.hyq_append(ctypes.byref(c), 0x1000, 0x2000, 0x3000, None, 64, None) == 1
+    assert L.hyq_append(ctypes.byref(c), 0x1008, 0x2000, None, None, 0, None) == 3
+    assert L.hyq_prefill(ctypes.byref(c), None, 0x2000, None) == 1
+    assert L.hyq_decode_fp16(0x1000, 0x2000, 0x3000, 0x4000, 1, 6, 2, 4096, 0x5000, None, 0,
+                             0x6000, 1 << 20, None, None) == 2
