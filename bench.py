@@ -212,7 +212,8 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     # capture K steps with events around every decode
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_steps)]
+    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+           for _ in range(K_steps)]
     g = torch.cuda.CUDAGraph()
     total_launches = 0
     seen = []  # (step, layer, T)
@@ -321,7 +322,8 @@ def fp16_comparator(torch, hyq, cfg, Kd, Vd, q_in, dev, copies=3, reps=60):
     for i in range(6):
         hyq.hyq_decode_fp16(q_in[i], Ks[i % copies], Vs[i % copies], seq, o, ws)
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+           for _ in range(reps)]
     g = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())

@@ -374,6 +374,107 @@ __device__ __forceinline__ int unit_of_tile(const int *ts, int U, int t) {
   return lo;
 }
 
+// Merge the partials of unit u written by the blocks that share it (run by
+// the last one to finish; 128 consumer threads).  Parts are taken in chunks
+// of MERGE_CHUNK: their (max, sum) pairs are loaded in parallel, per-head
+// weights 2^(m_p - M) live in shared memory, and every thread accumulates
+// float4 slices of the output with many loads in flight.
+constexpr int MERGE_CHUNK = 128;
+
+template <int G>
+__device__ __forceinline__ void merge_parts(const DecodeArgs &a, const Smem &sm, int u, int u0, int u1,
+                                            int64_t n_tiles, int64_t N, int64_t hbase, int tid) {
+  float *pw = sm.mo;                       // [MERGE_CHUNK][G] weights
+  float *pl = sm.mo + MERGE_CHUNK * G;     // [MERGE_CHUNK][G] sums
+  int *pid = sm.scan;                      // [MERGE_CHUNK] partial record index or -1
+  float *runM = sm.mm, *runL = sm.ml, *alpha = sm.mm + 8;
+  const int c_lo = cta_of_tile(u0, n_tiles, N), c_hi = cta_of_tile(u1 - 1, n_tiles, N);
+  constexpr int NV = (G * D / 4 + NCW * 32 - 1) / (NCW * 32);  // float4 outputs per thread
+  float4 acc[NV];
+#pragma unroll
+  for (int v = 0; v < NV; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (tid < G) {
+    runM[tid] = -INFINITY;
+    runL[tid] = 0.f;
+  }
+  for (int base = c_lo; base <= c_hi; base += MERGE_CHUNK) {
+    const int n = min(MERGE_CHUNK, c_hi - base + 1);
+    named_bar_sync(1, NCW * 32);
+    for (int j = tid; j < n; j += NCW * 32) {
+      const int64_t cc = base + j;
+      const int64_t f0 = cta_first_tile(cc, n_tiles, N), f1 = cta_first_tile(cc + 1, n_tiles, N);
+      pid[j] = (f0 == f1) ? -1 : static_cast<int>(cc * 2 + ((u0 >= f0) ? 0 : 1));
+    }
+    named_bar_sync(1, NCW * 32);
+    for (int e = tid; e < n * G; e += NCW * 32) {
+      const int j = e / G, h = e % G;
+      float m = -INFINITY, l = 0.f;
+      if (pid[j] >= 0) {
+        const float *pr = a.part + (static_cast<int64_t>(pid[j]) * G + h) * PART_STRIDE;
+        m = __ldcg(pr);
+        l = __ldcg(pr + 1);
+      }
+      pw[e] = m;
+      pl[e] = l;
+    }
+    named_bar_sync(1, NCW * 32);
+    if (tid < G) {
+      const int h = tid;
+      float cm = -INFINITY;
+      for (int j = 0; j < n; ++j) cm = fmaxf(cm, pw[j * G + h]);
+      const float M = fmaxf(runM[h], cm);
+      const float al = (runM[h] == -INFINITY) ? 0.f : fast_exp2(runM[h] - M);
+      float L = runL[h] * al;
+      for (int j = 0; j < n; ++j) {
+        const float m = pw[j * G + h];
+        const float w = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
+        pw[j * G + h] = w;
+        L += pl[j * G + h] * w;
+      }
+      runM[h] = M;
+      runL[h] = L;
+      alpha[h] = al;
+    }
+    named_bar_sync(1, NCW * 32);
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const int o4 = tid + v * NCW * 32;  // float4 index over [G][32]
+      if (o4 < G * D / 4) {
+        const int h = o4 / (D / 4), c4 = o4 % (D / 4);
+        const float al = alpha[h];
+        float4 s = make_float4(acc[v].x * al, acc[v].y * al, acc[v].z * al, acc[v].w * al);
+#pragma unroll 16
+        for (int j = 0; j < n; ++j) {
+          const int id = pid[j];
+          if (id < 0) continue;
+          const float w = pw[j * G + h];
+          const float4 x = __ldcg(reinterpret_cast<const float4 *>(
+              a.part + (static_cast<int64_t>(id) * G + h) * PART_STRIDE + 4 + 4 * c4));
+          s.x += w * x.x;
+          s.y += w * x.y;
+          s.z += w * x.z;
+          s.w += w * x.w;
+        }
+        acc[v] = s;
+      }
+    }
+  }
+  named_bar_sync(1, NCW * 32);
+#pragma unroll
+  for (int v = 0; v < NV; ++v) {
+    const int o4 = tid + v * NCW * 32;
+    if (o4 < G * D / 4) {
+      const int h = o4 / (D / 4), c4 = o4 % (D / 4);
+      const float inv = 1.f / runL[h];
+      __half2 lo = __floats2half2_rn(acc[v].x * inv, acc[v].y * inv);
+      __half2 hi = __floats2half2_rn(acc[v].z * inv, acc[v].w * inv);
+      uint2 pk = make_uint2(h2u(lo), h2u(hi));
+      *reinterpret_cast<uint2 *>(a.o + (hbase + h) * D + 4 * c4) = pk;
+      if (c4 == 0 && a.lse) a.lse[hbase + h] = (runM[h] + __log2f(runL[h])) * LN2;
+    }
+  }
+}
+
 template <int G, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -635,31 +736,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
       named_bar_sync(1, NCW * 32);
       if (*sm.last_flag) {
         __threadfence();
-        const int c_lo = cta_of_tile(u0, n_tiles, N), c_hi = cta_of_tile(u1 - 1, n_tiles, N);
-        for (int idx = tid; idx < G * D; idx += NCW * 32) {
-          const int h = idx / D, c = idx % D;
-          float M = -INFINITY;
-          for (int cc = c_lo; cc <= c_hi; ++cc) {
-            const int64_t f0 = cta_first_tile(cc, n_tiles, N), f1 = cta_first_tile(cc + 1, n_tiles, N);
-            if (f0 == f1) continue;
-            const int sid = (u0 >= f0) ? 0 : 1;
-            const float *pr = a.part + (static_cast<int64_t>(cc * 2 + sid) * G + h) * PART_STRIDE;
-            M = fmaxf(M, __ldcg(pr));
-          }
-          float L = 0.f, O = 0.f;
-          for (int cc = c_lo; cc <= c_hi; ++cc) {
-            const int64_t f0 = cta_first_tile(cc, n_tiles, N), f1 = cta_first_tile(cc + 1, n_tiles, N);
-            if (f0 == f1) continue;
-            const int sid = (u0 >= f0) ? 0 : 1;
-            const float *pr = a.part + (static_cast<int64_t>(cc * 2 + sid) * G + h) * PART_STRIDE;
-            const float mw = __ldcg(pr);
-            const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-            L += __ldcg(pr + 1) * f;
-            O += __ldcg(pr + 4 + c) * f;
-          }
-          a.o[(hbase + h) * D + c] = __float2half_rn(O / L);
-          if (c == 0 && a.lse) a.lse[hbase + h] = (M + __log2f(L)) * LN2;
-        }
+        merge_parts<G>(a, sm, u, u0, u1, n_tiles, N, hbase, tid);
         if (tid == 0) a.counters[u] = 0;
       }
     }

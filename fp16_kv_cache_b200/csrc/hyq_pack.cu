@@ -193,66 +193,81 @@ __device__ __forceinline__ int find_sorted(const int32_t *a, int n, int32_t key)
   return (lo < n && a[lo] == key) ? lo : -1;
 }
 
-__global__ void __launch_bounds__(256) vl_apply_kernel(hyq_cache c, const int32_t *__restrict__ pos,
-                                                       int k, const __half *__restrict__ k_full,
-                                                       const __half *__restrict__ v_full,
-                                                       int32_t *n_unpromoted) {
+// Prefill mode, step 1 (one block per unit): validate the new list, clear
+// the unit's bitmask, publish the count (0 when the list is invalid, which
+// turns step 2 into a no-op for the unit).
+__global__ void __launch_bounds__(256) vl_reset_kernel(hyq_cache c, const int32_t *__restrict__ pos, int k) {
+  __shared__ int s_bad;
+  const int u = blockIdx.x;
+  const int T = c.seq_len[u / c.n_kv_heads];
+  const int L4 = T - c.window;
+  const int32_t *np = pos + static_cast<int64_t>(u) * k;
+  if (threadIdx.x == 0) s_bad = (T < 0 || T > c.capacity);
+  __syncthreads();
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    const int p = np[i];
+    if (p < 0 || p >= L4 || (i > 0 && np[i - 1] >= p)) s_bad = 1;
+  }
+  uint32_t *mask = c.vl_mask + static_cast<int64_t>(u) * (c.capacity / 32);
+  for (int w = threadIdx.x; w < c.capacity / 32; w += blockDim.x) mask[w] = 0u;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (s_bad) set_status(c.dev_status, HYQ_DEV_BADLEN);
+    c.vl_count[u] = s_bad ? 0 : k;
+  }
+}
+
+// Prefill mode, step 2 (blocks of 32 rows x 16 lanes): gather the FP16 rows,
+// write the position list, set the bits.
+__global__ void __launch_bounds__(512) vl_gather_kernel(hyq_cache c, const int32_t *__restrict__ pos, int k,
+                                                        const __half *__restrict__ k_full,
+                                                        const __half *__restrict__ v_full) {
+  const int u = blockIdx.y;
+  if (c.vl_count[u] != k) return;  // invalid list: left empty by step 1
+  const int r = blockIdx.x * 32 + (threadIdx.x >> 4), part = threadIdx.x & 15;
+  if (r >= k) return;
+  const int p = pos[static_cast<int64_t>(u) * k + r];
+  const int64_t so = (static_cast<int64_t>(u) * c.capacity + p) * D + 8 * part;
+  const int64_t d = (static_cast<int64_t>(u) * c.vl_capacity + r) * D + 8 * part;
+  *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.vl_k) + d) = *reinterpret_cast<const uint4 *>(k_full + so);
+  *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.vl_v) + d) = *reinterpret_cast<const uint4 *>(v_full + so);
+  if (part == 0) {
+    atomicOr(&c.vl_mask[static_cast<int64_t>(u) * (c.capacity / 32) + (p >> 5)], 1u << (p & 31));
+    c.vl_pos[static_cast<int64_t>(u) * c.vl_capacity + r] = p;
+  }
+}
+
+// Cache mode (one block of 1024 threads per unit): kept = new ∩ old in
+// ascending order; kslot[r] = old slot of the r-th kept position, kpos[r] =
+// that position.  Rows only move to lower slots (r <= kslot[r]), so the move
+// is done in place, 64 rows per chunk, each chunk reading all its sources
+// before writing.
+__global__ void __launch_bounds__(1024) vl_recompact_kernel(hyq_cache c, const int32_t *__restrict__ pos, int k,
+                                                            int32_t *n_unpromoted) {
   extern __shared__ int32_t vl_list[];  // [2][vl_capacity]
   __shared__ int red[32];
   __shared__ int s_bad;
   const int u = blockIdx.x;
-  const int b = u / c.n_kv_heads;
-  const int T = c.seq_len[b];
+  const int T = c.seq_len[u / c.n_kv_heads];
   const int L4 = T - c.window;
   const int32_t *np = pos + static_cast<int64_t>(u) * k;
   int32_t *old = c.vl_pos + static_cast<int64_t>(u) * c.vl_capacity;
   const int old_n = c.vl_count[u];
   uint32_t *mask = c.vl_mask + static_cast<int64_t>(u) * (c.capacity / 32);
-  if (threadIdx.x == 0) s_bad = 0;
+  if (threadIdx.x == 0) s_bad = (old_n < 0 || old_n > c.vl_capacity);
   __syncthreads();
-  // validate the new list: ascending, within [0, T - window); old list sane
   for (int i = threadIdx.x; i < k; i += blockDim.x) {
     const int p = np[i];
     if (p < 0 || p >= L4 || (i > 0 && np[i - 1] >= p)) s_bad = 1;
   }
-  if (threadIdx.x == 0 && (old_n < 0 || old_n > c.vl_capacity)) s_bad = 1;
   __syncthreads();
   if (s_bad) {
     if (threadIdx.x == 0) set_status(c.dev_status, HYQ_DEV_BADLEN);
     return;
   }
-  const int64_t row_base = static_cast<int64_t>(u) * c.vl_capacity;
   __half *vk = reinterpret_cast<__half *>(c.vl_k);
   __half *vv = reinterpret_cast<__half *>(c.vl_v);
-
-  if (k_full) {
-    // prefill: clear the old bits, gather the new rows, set the new bits
-    for (int i = threadIdx.x; i < old_n; i += blockDim.x) {
-      const int p = old[i];
-      if (p >= 0 && p < c.capacity) atomicAnd(&mask[p >> 5], ~(1u << (p & 31)));
-    }
-    __syncthreads();
-    const int64_t src_base = static_cast<int64_t>(u) * c.capacity;
-    for (int i = threadIdx.x; i < k * 16; i += blockDim.x) {
-      const int r = i >> 4, part = i & 15;
-      const int p = np[r];
-      const int64_t so = (src_base + p) * D + 8 * part;
-      const int64_t d = (row_base + r) * D + 8 * part;
-      *reinterpret_cast<uint4 *>(vk + d) = *reinterpret_cast<const uint4 *>(k_full + so);
-      *reinterpret_cast<uint4 *>(vv + d) = *reinterpret_cast<const uint4 *>(v_full + so);
-      if (part == 0) {
-        atomicOr(&mask[p >> 5], 1u << (p & 31));
-        old[r] = p;
-      }
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) c.vl_count[u] = k;
-    return;
-  }
-
-  // cache mode: kept = new ∩ old, in ascending order.  kslot[r] = old slot
-  // of the r-th kept position, kpos[r] = that position.  Rows only move to
-  // lower slots (r <= kslot[r]), so the move is done in place in chunks.
+  const int64_t row_base = static_cast<int64_t>(u) * c.vl_capacity;
   int32_t *kslot = vl_list;
   int32_t *kpos = vl_list + c.vl_capacity;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -283,9 +298,10 @@ __global__ void __launch_bounds__(256) vl_apply_kernel(hyq_cache c, const int32_
     if (p >= 0 && p < c.capacity && find_sorted(np, k, p) < 0) atomicAnd(&mask[p >> 5], ~(1u << (p & 31)));
   }
   __syncthreads();
-  for (int base = 0; base < n_kept; base += 16) {
+  const int rows = blockDim.x / 16;
+  for (int base = 0; base < n_kept; base += rows) {
     const int r = base + (threadIdx.x >> 4), part = threadIdx.x & 15;
-    const bool act = r < n_kept && (threadIdx.x >> 4) < 16;
+    const bool act = r < n_kept && kslot[r] != r;
     uint4 rk = make_uint4(0, 0, 0, 0), rv = rk;
     if (act) {
       const int64_t so = (row_base + kslot[r]) * D + 8 * part;
@@ -374,15 +390,24 @@ extern "C" hyq_status hyq_vl_apply(const hyq_cache *c, const int32_t *pos, int32
   if ((k_full == nullptr) != (v_full == nullptr)) return HYQ_ERR_INVALID;
   if ((pos && !aligned16(pos)) || (k_full && (!aligned16(k_full) || !aligned16(v_full))))
     return HYQ_ERR_ALIGN;
-  const size_t smem = 2 * sizeof(int32_t) * static_cast<size_t>(c->vl_capacity);
-  if (smem > 200 * 1024) return HYQ_ERR_UNSUPPORTED;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(vl_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    attr_set = true;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int U = c->batch * c->n_kv_heads;
+  if (k_full) {
+    vl_reset_kernel<<<U, 256, 0, st>>>(*c, pos, k);
+    if (k > 0)
+      vl_gather_kernel<<<dim3((k + 31) / 32, U), 512, 0, st>>>(*c, pos, k, static_cast<const __half *>(k_full),
+                                                               static_cast<const __half *>(v_full));
+  } else {
+    const size_t smem = 2 * sizeof(int32_t) * static_cast<size_t>(c->vl_capacity);
+    if (smem > 200 * 1024) return HYQ_ERR_UNSUPPORTED;
+    static int attr_dev = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr_dev != dev) {
+      cudaFuncSetAttribute(vl_recompact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+      attr_dev = dev;
+    }
+    vl_recompact_kernel<<<U, 1024, smem, st>>>(*c, pos, k, n_unpromoted);
   }
-  vl_apply_kernel<<<c->batch * c->n_kv_heads, 256, smem, static_cast<cudaStream_t>(stream)>>>(
-      *c, pos, k, static_cast<const __half *>(k_full), static_cast<const __half *>(v_full),
-      n_unpromoted);
   return cudaGetLastError() == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
 }

@@ -32,10 +32,14 @@
 // multiplied on the tensor cores) so the dequantized key keeps ~22 bits.
 #include "hyq_common.cuh"
 
+extern "C" int32_t hyq_sm_count(void);  // hyq_api.cu
+
 namespace hyq {
 
+static int hyq_sm_count_dev() { return hyq_sm_count(); }
+
 constexpr int SEL_SUB = 64;       // keys per shared-memory sub-tile
-constexpr int SEL_KC = 1024;      // keys per block (chunk)
+constexpr int SEL_KC = 512;       // keys per work item (chunk)
 constexpr int SEL_MAX_ROWS = 512; // n_q * G
 constexpr int SEL_BLOCK_ROWS = 256;  // query rows per block (8 warps x 32)
 constexpr int TOPK_THREADS = 1024;
@@ -55,6 +59,7 @@ struct SelectArgs {
   float *colsum_part;  // [n_rb][U][cap]  per row block
   float *colsum;       // [U][cap]  final column sums
   int n_rb;            // row blocks: ceil(R / SEL_BLOCK_ROWS)
+  int32_t *rank_base;  // [U][cap/32]: vertical-line rows before each mask word
   int32_t *out_pos;    // [U][k]
   uint32_t *status;
 };
@@ -75,78 +80,93 @@ __device__ __forceinline__ uint32_t tile_off(int p, int c) {
 
 __device__ __forceinline__ int sel_T(const SelectArgs &a, int u) { return a.seq_len[u / a.Hkv]; }
 
-// Fill sub-tile rows [key0, key0 + SEL_SUB) of unit u: hi (and lo in cache
-// mode) fp16 tiles.  Keys >= key_end are zero.
-template <bool CACHE>
-__device__ void fill_tile(const SelectArgs &a, int u, int T, int key0, int key_end, uint8_t *hi,
-                          uint8_t *lo, int *src_kind) {
-  const int nthr = blockDim.x;
-  if (!CACHE) {
-    const __half *base = a.k_full + static_cast<int64_t>(u) * a.cap * D;
-    for (int i = threadIdx.x; i < SEL_SUB * 16; i += nthr) {
-      const int p = i >> 4, c = i & 15;
-      const int key = key0 + p;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (key < key_end) v = *reinterpret_cast<const uint4 *>(base + static_cast<int64_t>(key) * D + 8 * c);
-      *reinterpret_cast<uint4 *>(hi + tile_off(p, c)) = v;
-    }
-    return;
-  }
-  // cache mode: src_kind[p] = -1 window, -2 INT4, >= 0 VL slot, -3 beyond
-  const int L4 = T - a.W;
-  for (int p = threadIdx.x; p < SEL_SUB; p += nthr) {
-    const int key = key0 + p;
-    int kind = -3;
-    if (key < key_end) {
-      if (key >= L4) {
-        kind = -1;
-      } else {
-        const uint32_t w = a.vl_mask[static_cast<int64_t>(u) * (a.cap / 32) + (key >> 5)];
-        kind = -2;
-        if ((w >> (key & 31)) & 1u) {
-          const int32_t *vp = a.vl_pos + static_cast<int64_t>(u) * a.vl_cap;
-          const int cnt = min(max(a.vl_count[u], 0), a.vl_cap);
-          int lo_ = 0, hi_ = cnt;
-          while (lo_ < hi_) {
-            const int mid = (lo_ + hi_) >> 1;
-            if (vp[mid] < key) lo_ = mid + 1; else hi_ = mid;
-          }
-          if (lo_ < cnt && vp[lo_] == key) kind = lo_;
-          else set_status(a.status, HYQ_DEV_OOB);
-        }
-      }
-    }
-    src_kind[p] = kind;
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < SEL_SUB * 16; i += nthr) {
+// One block = 256 threads; a 64-key sub-tile is 1024 items (key, 16-byte
+// chunk), 4 per thread: item i = threadIdx.x + 256 j -> key i / 16, chunk i % 16.
+constexpr int SEL_THREADS = 256;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Prefill mode: FP16 keys straight into the swizzled tile (zero past key_end).
+__device__ __forceinline__ void issue_fp16(const SelectArgs &a, int u, int key0, int key_end, uint32_t hi) {
+  const __half *base = a.k_full + static_cast<int64_t>(u) * a.cap * D;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int i = threadIdx.x + SEL_THREADS * j;
     const int p = i >> 4, c = i & 15;
     const int key = key0 + p;
-    const int kind = src_kind[p];
-    uint4 h = make_uint4(0, 0, 0, 0), l = h;
-    if (kind == -1) {
-      h = *reinterpret_cast<const uint4 *>(a.win_k + (static_cast<int64_t>(u) * a.W + key % a.W) * D + 8 * c);
-    } else if (kind >= 0) {
-      h = *reinterpret_cast<const uint4 *>(a.vl_k + (static_cast<int64_t>(u) * a.vl_cap + kind) * D + 8 * c);
-    } else if (kind == -2) {
-      // channels 8c..8c+7: group g = c / 4, pieces 2(c%4) and 2(c%4)+1
-      const int64_t row = static_cast<int64_t>(u) * a.cap + key;
-      const uint4 pc = *reinterpret_cast<const uint4 *>(a.k_codes + row * ROW_BYTES + 16 * (c & 3));
+    const bool in = key < key_end;
+    cp_async16(hi + tile_off(p, c), base + static_cast<int64_t>(in ? key : 0) * D + 8 * c, in ? 16 : 0);
+  }
+  cp_async_commit();
+}
+
+// Cache mode: raw bytes of 4 items in registers (loaded before the current
+// sub-tile is computed, converted after).
+struct RawItems {
+  uint4 v[4];
+  uint32_t sz[4];
+  int kind[4];  // -1 FP16 row (window / vertical line), -2 INT4, -3 zero
+};
+
+__device__ __forceinline__ void issue_cache(const SelectArgs &a, int u, int T, int key0, int key_end,
+                                            const int *slot_of, int k0, RawItems &r) {
+  const int L4 = T - a.W;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int i = threadIdx.x + SEL_THREADS * j;
+    const int p = i >> 4, c = i & 15;
+    const int key = key0 + p;
+    r.v[j] = make_uint4(0, 0, 0, 0);
+    r.sz[j] = 0;
+    r.kind[j] = -3;
+    if (key >= key_end) continue;
+    if (key >= L4) {
+      r.kind[j] = -1;
+      r.v[j] = *reinterpret_cast<const uint4 *>(a.win_k + (static_cast<int64_t>(u) * a.W + key % a.W) * D + 8 * c);
+      continue;
+    }
+    const int slot = slot_of[key - k0];
+    if (slot >= 0) {
+      r.kind[j] = -1;
+      r.v[j] = *reinterpret_cast<const uint4 *>(a.vl_k + (static_cast<int64_t>(u) * a.vl_cap + slot) * D + 8 * c);
+      continue;
+    }
+    // channels 8c..8c+7: group c / 4, pieces 2(c%4) and 2(c%4)+1
+    const int64_t row = static_cast<int64_t>(u) * a.cap + key;
+    r.kind[j] = -2;
+    r.v[j] = *reinterpret_cast<const uint4 *>(a.k_codes + row * ROW_BYTES + 16 * (c & 3));
+    r.sz[j] = *reinterpret_cast<const uint32_t *>(a.k_sz + row * SZ_BYTES + 4 * (c >> 2));
+  }
+}
+
+// Convert the raw items to fp16 hi (+ lo) tiles.  INT4: x = zero + code*scale
+// in fp32 (one rounding), hi = fp16(x), lo = fp16(x - hi).
+__device__ __forceinline__ void store_cache(const RawItems &r, uint8_t *hi, uint8_t *lo) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int i = threadIdx.x + SEL_THREADS * j;
+    const int p = i >> 4, c = i & 15;
+    uint4 h = r.v[j], l = make_uint4(0, 0, 0, 0);
+    if (r.kind[j] == -2) {
       const int g = c >> 2, hh = g >> 1, ii = g & 1;
-      const uint32_t w0 = hh ? pc.y : pc.x;  // piece 2(c%4), word hh
-      const uint32_t w1 = hh ? pc.w : pc.z;  // piece 2(c%4)+1
-      const __half2 sz = u2h(*reinterpret_cast<const uint32_t *>(a.k_sz + row * SZ_BYTES + 4 * g));
+      const uint32_t w0 = hh ? r.v[j].y : r.v[j].x;  // piece 2(c%4), word hh
+      const uint32_t w1 = hh ? r.v[j].w : r.v[j].z;  // piece 2(c%4)+1
+      const __half2 sz = u2h(r.sz[j]);
       const float sc = __low2float(sz), zr = __high2float(sz);
       float x[8];
-      // byte 2j + ii of a word holds channels 2j (low) and 2j+1 (high)
 #pragma unroll
       for (int s = 0; s < 2; ++s) {
         const uint32_t w = s ? w1 : w0;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const uint32_t byte = (w >> (8 * (2 * j + ii))) & 0xFFu;
-          x[4 * s + 2 * j] = fmaf(static_cast<float>(byte & 15u), sc, zr);
-          x[4 * s + 2 * j + 1] = fmaf(static_cast<float>(byte >> 4), sc, zr);
+        for (int jj = 0; jj < 2; ++jj) {
+          const uint32_t byte = (w >> (8 * (2 * jj + ii))) & 0xFFu;  // channels 2jj (lo), 2jj+1 (hi)
+          x[4 * s + 2 * jj] = fmaf(static_cast<float>(byte & 15u), sc, zr);
+          x[4 * s + 2 * jj + 1] = fmaf(static_cast<float>(byte >> 4), sc, zr);
         }
       }
       uint32_t hw[4], lw[4];
@@ -240,132 +260,206 @@ __device__ __forceinline__ void tile_scores(uint32_t hi, uint32_t lo, const uint
       for (int e = 0; e < 4; ++e) s[mt][nt][e] *= SEL_SCALE;
 }
 
-// PASS 1: per-row (max, sum exp) over the chunk; PASS 2: column sums.
+// PASS 1: per-row (max, sum exp) over a chunk of keys; PASS 2: column sums.
+// Persistent: block b takes work items b, b + gridDim.x, ... of the
+// (unit, chunk) space; blockIdx.y is the row block (rows 256 y .. 256 y + 255).
+// Shared memory: 2 x (hi, lo) 64-key tiles, slot_of[SEL_KC], cpart[8][64].
 template <bool CACHE, int PASS>
-__global__ void __launch_bounds__(SEL_BLOCK_ROWS, 1) score_kernel(const SelectArgs a) {
+__global__ void __launch_bounds__(SEL_THREADS, 1) score_kernel(const SelectArgs a) {
   extern __shared__ __align__(128) uint8_t sm[];
-  uint8_t *hi = sm;
-  uint8_t *lo = sm + SEL_SUB * 256;
-  int *src_kind = reinterpret_cast<int *>(sm + 2 * SEL_SUB * 256);
-  float *cpart = reinterpret_cast<float *>(sm + 2 * SEL_SUB * 256 + SEL_SUB * 4);  // [warps][64]
-  const int u = blockIdx.y, chunk = blockIdx.x, rb = blockIdx.z;
-  const int T = sel_T(a, u);
-  const int warp = (threadIdx.x >> 5) + rb * (SEL_BLOCK_ROWS / 32), lane = threadIdx.x & 31;
-  const int nwarps = blockDim.x >> 5;
-  if (T < a.n_q || T > a.cap || T - a.W < a.k) return;  // reported by the top-k kernel
-  const int key_end = (PASS == 1) ? T : T - a.W;
-  const int k0 = chunk * SEL_KC;
-  if (k0 >= key_end) {
-    if (PASS == 1) {
-      for (int r = threadIdx.x; r < SEL_BLOCK_ROWS; r += blockDim.x)
-        a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + rb * SEL_BLOCK_ROWS + r] =
-            make_float2(-INFINITY, 0.f);
-    }
-    return;
-  }
-  const int k1 = min(key_end, k0 + SEL_KC);
-  uint32_t qa[2][8][4];
-  load_qa(a, u, T, warp, lane, qa);
+  constexpr int TILE = SEL_SUB * 256;
+  uint8_t *tiles = sm;  // buf b: hi at 2b*TILE, lo at (2b+1)*TILE
+  int *slot_of = reinterpret_cast<int *>(sm + 4 * TILE);
+  float *cpart = reinterpret_cast<float *>(sm + 4 * TILE + SEL_KC * 4);
+  const int rb = blockIdx.y;
+  const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = wl + rb * (SEL_BLOCK_ROWS / 32);  // global warp: rows 32 warp ..
+  const bool has_rows = 32 * warp < a.R;
   const int gid = lane >> 2, t4 = lane & 3;
-  // rows held by this lane: 32w + 16mt + gid + 8hr
-  float m[2][2], l[2][2], il[2][2];
-  int qpos[2][2];
+  const int n_items = a.U * a.n_chunks;
+  const uint32_t tiles_s = smem_u32(tiles);
+  uint32_t qa[2][8][4];
+  int q_unit = -1, q_T = -1;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int u = item / a.n_chunks, chunk = item % a.n_chunks;
+    const int T = sel_T(a, u);
+    if (T < a.n_q || T > a.cap || T - a.W < a.k) continue;  // reported by the top-k kernel
+    const int key_end = (PASS == 1) ? T : T - a.W;
+    const int k0 = chunk * SEL_KC;
+    if (k0 >= key_end) {
+      if (PASS == 1)
+        for (int r = threadIdx.x; r < SEL_BLOCK_ROWS; r += blockDim.x)
+          a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + rb * SEL_BLOCK_ROWS + r] =
+              make_float2(-INFINITY, 0.f);
+      continue;
+    }
+    const int k1 = min(key_end, k0 + SEL_KC);
+    const int nsub = (k1 - k0 + SEL_SUB - 1) / SEL_SUB;
+    __syncthreads();  // previous item fully done with shared memory
+    RawItems raw;
+    if (CACHE) {
+      // vertical-line slot of every key of the chunk: rank of its mask bit
+      const uint32_t *mrow = a.vl_mask + static_cast<int64_t>(u) * (a.cap / 32);
+      const int32_t *rbase = a.rank_base + static_cast<int64_t>(u) * (a.cap / 32);
+      for (int j = threadIdx.x; j < SEL_KC; j += blockDim.x) {
+        const int key = k0 + j;
+        int slot = -1;
+        if (key < k1 && key < T - a.W) {
+          const uint32_t w = mrow[key >> 5];
+          if ((w >> (key & 31)) & 1u) slot = rbase[key >> 5] + __popc(w & ((1u << (key & 31)) - 1u));
+        }
+        slot_of[j] = slot;
+      }
+      __syncthreads();
+      issue_cache(a, u, T, k0, k1, slot_of, k0, raw);
+    } else {
+      issue_fp16(a, u, k0, k1, tiles_s);
+    }
+    if (u != q_unit || T != q_T) {
+      load_qa(a, u, T, warp, lane, qa);
+      q_unit = u;
+      q_T = T;
+    }
+    float m[2][2], l[2][2], il[2][2];
+    int qpos[2][2];
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      const int row = 32 * warp + 16 * mt + gid + 8 * hr;
-      m[mt][hr] = -INFINITY;
-      l[mt][hr] = 0.f;
-      qpos[mt][hr] = (row < a.R) ? T - a.n_q + row % a.n_q : -1;  // last visible key
-      il[mt][hr] = 0.f;
-      if (PASS == 2 && row < a.R) {
-        const float2 st = a.stats[static_cast<int64_t>(u) * SEL_MAX_ROWS + row];
-        m[mt][hr] = st.x;
-        il[mt][hr] = st.y;
+      for (int hr = 0; hr < 2; ++hr) {
+        const int row = 32 * warp + 16 * mt + gid + 8 * hr;
+        m[mt][hr] = -INFINITY;
+        l[mt][hr] = 0.f;
+        il[mt][hr] = 0.f;
+        qpos[mt][hr] = (row < a.R) ? T - a.n_q + row % a.n_q : -1;  // last visible key
+        if (PASS == 2 && row < a.R) {
+          const float2 st = a.stats[static_cast<int64_t>(u) * SEL_MAX_ROWS + row];
+          m[mt][hr] = st.x;
+          il[mt][hr] = st.y;
+        }
+      }
+    if (CACHE) store_cache(raw, tiles, tiles + TILE);
+    for (int st = 0; st < nsub; ++st) {
+      const int cur = st & 1;
+      const int key0 = k0 + st * SEL_SUB;
+      const bool more = st + 1 < nsub;
+      if (more) {
+        if (CACHE) issue_cache(a, u, T, key0 + SEL_SUB, k1, slot_of, k0, raw);
+        else issue_fp16(a, u, key0 + SEL_SUB, k1, tiles_s + (cur ^ 1) * 2 * TILE);
+      }
+      if (!CACHE) {
+        if (more) cp_async_wait<1>(); else cp_async_wait<0>();
+      }
+      __syncthreads();
+      float s[2][8][4];
+      if (has_rows) {
+        tile_scores<CACHE>(tiles_s + cur * 2 * TILE, tiles_s + cur * 2 * TILE + TILE, qa, lane, s);
+        if (PASS == 1) {
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+              float mx = -INFINITY;
+#pragma unroll
+              for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const int key = key0 + nt * 8 + 2 * t4 + e;
+                  const bool vis = key < k1 && key <= qpos[mt][hr];
+                  float &x = s[mt][nt][2 * hr + e];
+                  x = vis ? x : -INFINITY;
+                  mx = fmaxf(mx, x);
+                }
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+              const float mn = fmaxf(m[mt][hr], mx);
+              if (mn == -INFINITY) continue;
+              float sum = 0.f;
+#pragma unroll
+              for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) sum += fast_exp2(s[mt][nt][2 * hr + e] - mn);
+              l[mt][hr] = l[mt][hr] * fast_exp2(m[mt][hr] - mn) + sum;
+              m[mt][hr] = mn;
+            }
+        } else {
+#pragma unroll
+          for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              float acc = 0.f;
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr)
+                  acc += (il[mt][hr] > 0.f) ? fast_exp2(s[mt][nt][2 * hr + e] - m[mt][hr]) * il[mt][hr] : 0.f;
+              acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+              acc += __shfl_xor_sync(0xffffffffu, acc, 8);
+              acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+              if (gid == 0) cpart[wl * SEL_SUB + nt * 8 + 2 * t4 + e] = acc;
+            }
+        }
+      } else if (PASS == 2) {
+        for (int j = lane; j < SEL_SUB; j += 32) cpart[wl * SEL_SUB + j] = 0.f;
+      }
+      if (CACHE && more) store_cache(raw, tiles + (cur ^ 1) * 2 * TILE, tiles + (cur ^ 1) * 2 * TILE + TILE);
+      __syncthreads();
+      if (PASS == 2) {
+        for (int j = threadIdx.x; j < SEL_SUB; j += blockDim.x) {
+          const int key = key0 + j;
+          float tot = 0.f;
+          for (int w = 0; w < SEL_BLOCK_ROWS / 32; ++w) tot += cpart[w * SEL_SUB + j];
+          if (key < k1) a.colsum_part[(static_cast<int64_t>(rb) * a.U + u) * a.cap + key] = tot;
+        }
+        __syncthreads();
       }
     }
-  const uint32_t hi_s = smem_u32(hi), lo_s = smem_u32(lo);
-  for (int key0 = k0; key0 < k1; key0 += SEL_SUB) {
-    __syncthreads();  // previous sub-tile fully consumed
-    fill_tile<CACHE>(a, u, T, key0, k1, hi, lo, src_kind);
-    __syncthreads();
-    float s[2][8][4];
-    tile_scores<CACHE>(hi_s, lo_s, qa, lane, s);
     if (PASS == 1) {
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
-          float mx = -INFINITY;
-#pragma unroll
-          for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int key = key0 + nt * 8 + 2 * t4 + e;
-              const bool vis = key < k1 && key <= qpos[mt][hr];
-              float &x = s[mt][nt][2 * hr + e];
-              x = vis ? x : -INFINITY;
-              mx = fmaxf(mx, x);
-            }
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-          const float mn = fmaxf(m[mt][hr], mx);
-          if (mn == -INFINITY) continue;
-          float sum = 0.f;
-#pragma unroll
-          for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) sum += fast_exp2(s[mt][nt][2 * hr + e] - mn);
-          l[mt][hr] = l[mt][hr] * fast_exp2(m[mt][hr] - mn) + sum;
-          m[mt][hr] = mn;
+          float lv = l[mt][hr];
+          lv += __shfl_xor_sync(0xffffffffu, lv, 1);
+          lv += __shfl_xor_sync(0xffffffffu, lv, 2);
+          const int row = 32 * warp + 16 * mt + gid + 8 * hr;
+          if (t4 == 0 && row < SEL_MAX_ROWS)
+            a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + row] =
+                make_float2(m[mt][hr], lv);
         }
-    } else {
-      // probabilities, summed over this lane's 4 rows, then over the warp
-      float cs[8][2];
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          float acc = 0.f;
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr)
-              acc += (il[mt][hr] > 0.f) ? fast_exp2(s[mt][nt][2 * hr + e] - m[mt][hr]) * il[mt][hr] : 0.f;
-          acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-          acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-          acc += __shfl_xor_sync(0xffffffffu, acc, 16);
-          cs[nt][e] = acc;
-        }
-      if (gid == 0) {
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) cpart[(threadIdx.x >> 5) * SEL_SUB + nt * 8 + 2 * t4 + e] = cs[nt][e];
-      }
-      __syncthreads();
-      for (int j = threadIdx.x; j < SEL_SUB; j += blockDim.x) {
-        const int key = key0 + j;
-        float tot = 0.f;
-        for (int w = 0; w < nwarps; ++w) tot += cpart[w * SEL_SUB + j];
-        if (key < k1) a.colsum_part[(static_cast<int64_t>(rb) * a.U + u) * a.cap + key] = tot;
-      }
     }
   }
-  if (PASS == 1) {
+}
+
+// Cache mode: rank_base[u][w] = vertical-line rows at positions < 32 w
+// (exclusive prefix popcount of the unit's mask), so the slot of a position
+// is one popcount away.
+__global__ void __launch_bounds__(1024) rank_kernel(const SelectArgs a) {
+  __shared__ int wsum[32];
+  const int u = blockIdx.x;
+  const int nw = a.cap / 32;
+  const uint32_t *mrow = a.vl_mask + static_cast<int64_t>(u) * nw;
+  int32_t *out = a.rank_base + static_cast<int64_t>(u) * nw;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int carry = 0;
+  for (int base = 0; base < nw; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const int v = (i < nw) ? __popc(mrow[i]) : 0;
+    int x = v;
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        float lv = l[mt][hr];
-        lv += __shfl_xor_sync(0xffffffffu, lv, 1);
-        lv += __shfl_xor_sync(0xffffffffu, lv, 2);
-        const int row = 32 * warp + 16 * mt + gid + 8 * hr;
-        if (t4 == 0 && row < SEL_MAX_ROWS)
-          a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + row] =
-              make_float2(m[mt][hr], lv);
-      }
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[w] = x;
+    __syncthreads();
+    int pre = 0, tot = 0;
+    for (int q = 0; q < (int)(blockDim.x >> 5); ++q) {
+      if (q < w) pre += wsum[q];
+      tot += wsum[q];
+    }
+    if (i < nw) out[i] = carry + pre + x - v;
+    carry += tot;
+    __syncthreads();
   }
 }
 
@@ -424,9 +518,17 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const SelectArgs a) 
       for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
       __syncthreads();
       const uint32_t pre = s_prefix, msk = s_mask;
-      for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const uint32_t b = bits[i];
-        if ((b & msk) == pre) atomicAdd(&hist[(b >> shift) & 255u], 1);
+      // warp-aggregated: one shared-memory atomic per distinct bin per warp
+      for (int base = 0; base < n; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        const uint32_t b = (i < n) ? bits[i] : 0u;
+        const bool act = (i < n) && ((b & msk) == pre);
+        const unsigned am = __ballot_sync(0xffffffffu, act);
+        if (act) {
+          const uint32_t bin = (b >> shift) & 255u;
+          const unsigned peers = __match_any_sync(am, bin);
+          if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+        }
       }
       __syncthreads();
       if (threadIdx.x == 0) {
@@ -487,23 +589,29 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const SelectArgs a) 
 }
 
 static cudaError_t select_launch(const SelectArgs &a, bool cache, cudaStream_t s) {
-  const int nw = a.R < SEL_BLOCK_ROWS ? (a.R + 31) / 32 : SEL_BLOCK_ROWS / 32;
-  const int threads = 32 * nw;
-  const size_t smem = 2 * SEL_SUB * 256 + SEL_SUB * 4 + static_cast<size_t>(nw) * SEL_SUB * 4;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(score_kernel<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-    cudaFuncSetAttribute(score_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-    cudaFuncSetAttribute(score_kernel<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-    cudaFuncSetAttribute(score_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-    attr = true;
+  const size_t smem = 4 * SEL_SUB * 256 + SEL_KC * 4 + (SEL_BLOCK_ROWS / 32) * SEL_SUB * 4;
+  static int attr_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_dev != dev) {
+    cudaFuncSetAttribute(score_kernel<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(score_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(score_kernel<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(score_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attr_dev = dev;
   }
-  const dim3 grid(a.n_chunks, a.U, a.n_rb);
-  if (cache) score_kernel<true, 1><<<grid, threads, smem, s>>>(a);
-  else score_kernel<false, 1><<<grid, threads, smem, s>>>(a);
+  const int n_items = a.U * a.n_chunks;
+  const int sms = hyq_sm_count_dev();
+  const dim3 grid(n_items < sms ? n_items : sms, a.n_rb);
+  if (cache) {
+    rank_kernel<<<a.U, 1024, 0, s>>>(a);
+    score_kernel<true, 1><<<grid, SEL_THREADS, smem, s>>>(a);
+  } else {
+    score_kernel<false, 1><<<grid, SEL_THREADS, smem, s>>>(a);
+  }
   stats_merge_kernel<<<a.U, 256, 0, s>>>(a);
-  if (cache) score_kernel<true, 2><<<grid, threads, smem, s>>>(a);
-  else score_kernel<false, 2><<<grid, threads, smem, s>>>(a);
+  if (cache) score_kernel<true, 2><<<grid, SEL_THREADS, smem, s>>>(a);
+  else score_kernel<false, 2><<<grid, SEL_THREADS, smem, s>>>(a);
   topk_kernel<<<a.U, TOPK_THREADS, 0, s>>>(a);
   return cudaGetLastError();
 }
@@ -523,7 +631,8 @@ extern "C" size_t hyq_select_vl_workspace(const hyq_cache *c, int32_t n_q) {
   const size_t U = static_cast<size_t>(c->batch) * c->n_kv_heads;
   const size_t nch = (static_cast<size_t>(c->capacity) + SEL_KC - 1) / SEL_KC;
   const size_t n_rb = (static_cast<size_t>(n_q) * (c->n_q_heads / c->n_kv_heads) + SEL_BLOCK_ROWS - 1) / SEL_BLOCK_ROWS;
-  return a256(U * nch * SEL_MAX_ROWS * 8) + a256(U * SEL_MAX_ROWS * 8) + a256(U * c->capacity * 4) * (n_rb + 1);
+  return a256(U * nch * SEL_MAX_ROWS * 8) + a256(U * SEL_MAX_ROWS * 8) + a256(U * c->capacity * 4) * (n_rb + 1) +
+         a256(U * (c->capacity / 32) * 4);
 }
 
 extern "C" hyq_status hyq_select_vl(const hyq_cache *c, const void *q_sel, int32_t n_q,
@@ -562,6 +671,8 @@ extern "C" hyq_status hyq_select_vl(const hyq_cache *c, const void *q_sel, int32
   a.colsum_part = reinterpret_cast<float *>(w);
   w += a256(U * c->capacity * 4) * a.n_rb;
   a.colsum = out_colsum ? out_colsum : (a.n_rb == 1 ? a.colsum_part : reinterpret_cast<float *>(w));
+  w += a256(U * c->capacity * 4);
+  a.rank_base = reinterpret_cast<int32_t *>(w);
   a.out_pos = out_pos;
   a.status = c->dev_status;
   return select_launch(a, k_full == nullptr, static_cast<cudaStream_t>(stream)) == cudaSuccess ? HYQ_OK

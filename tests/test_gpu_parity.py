@@ -321,7 +321,7 @@ def test_select_ties_lower_position_wins():
     dom = (8.0 * np.sqrt(128) * m / np.linalg.norm(m)).astype(np.float16)
     for p in (300, 17, 123):
         K[0, 0, p] = dom
-    case = Case(cfg, vl=np.zeros((1, 2, 0), np.int32), cap=640)
+    case = Case(cfg, vl=np.zeros((1, 2, 0), np.int32), cap=640, vl_cap=8)
     kf = dev(K)
     for k, want in ((2, [17, 123]), (3, [17, 123, 300])):
         pos_g, cs_g = _select_gpu(case, dev(qs), k, k_full=kf)
