@@ -879,3 +879,65 @@ extern "C" hyq_status hyq_decode_fp16(const void *q, const void *k, const void *
   return dispatch_decode<MODE_FP16>(G, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? HYQ_OK
                                                                                             : HYQ_ERR_CUDA;
 }
+
+// ---------------------------------------------------------------- no-alloc variant
+// hyq_decode_noalloc: the same decode for callers that cannot allocate
+// device memory or carry a workspace pointer.  Its scratch -- the per-unit
+// tile counters and the per-block partial records of the split merge -- is
+// this fixed array, which every GPU that loads the library keeps until the
+// process exits.  Layout as in hyq_decode: counters, then partials.
+namespace {
+constexpr int NOALLOC_MAX_UNITS = 4096;  // batch x kv heads
+constexpr int NOALLOC_MAX_CTAS = 320;    // thread blocks of one launch
+constexpr int NOALLOC_MAX_G = 8;
+constexpr size_t NOALLOC_BYTES = static_cast<size_t>(NOALLOC_MAX_UNITS) * 4 +
+                                 static_cast<size_t>(NOALLOC_MAX_CTAS) * 2 * NOALLOC_MAX_G * PART_STRIDE * 4;
+__device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_BYTES];
+void *g_noalloc_addr[64] = {nullptr};  // device address of the array, per device
+
+// Host code cannot pass g_noalloc_scratch itself (that name is a host-side
+// stand-in); look its device address up once per device, with the device
+// current, and reuse it.
+bool noalloc_address(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!g_noalloc_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return false;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return true;
+}
+}  // namespace
+
+extern "C" hyq_status hyq_decode_noalloc(const hyq_cache *c, const void *q, void *o, float *lse,
+                                         void *stream) {
+  hyq_status s = hyq_check_cache(c);
+  if (s != HYQ_OK) return s;
+  if (!q || !o) return HYQ_ERR_INVALID;
+  if (!al16(q) || !al16(o) || (lse && !al16(lse))) return HYQ_ERR_ALIGN;
+  const int G = c->n_q_heads / c->n_kv_heads;
+  const int U = c->batch * c->n_kv_heads;
+  const int N = resolve_ctas(0);
+  if (U > NOALLOC_MAX_UNITS || N > NOALLOC_MAX_CTAS || G > NOALLOC_MAX_G) return HYQ_ERR_UNSUPPORTED;
+  if (decode_ws_bytes(G, U, N) > NOALLOC_BYTES) return HYQ_ERR_UNSUPPORTED;
+  void *ws = nullptr;
+  if (!noalloc_address(&ws)) return HYQ_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the array keeps the last call's contents: the counters must start at 0
+  if (cudaMemsetAsync(ws, 0, static_cast<size_t>(U) * 4, st) != cudaSuccess) return HYQ_ERR_CUDA;
+  DecodeArgs a{};
+  a.B = c->batch; a.Hq = c->n_q_heads; a.Hkv = c->n_kv_heads; a.cap = c->capacity;
+  a.W = c->window; a.vl_cap = c->vl_capacity; a.U = U; a.n_ctas = N;
+  a.k_codes = c->k_codes; a.v_codes = c->v_codes;
+  a.k_sz = static_cast<const uint8_t *>(c->k_sz); a.v_sz = static_cast<const uint8_t *>(c->v_sz);
+  a.win_k = static_cast<const __half *>(c->win_k); a.win_v = static_cast<const __half *>(c->win_v);
+  a.vl_k = static_cast<const __half *>(c->vl_k); a.vl_v = static_cast<const __half *>(c->vl_v);
+  a.vl_count = c->vl_count; a.vl_mask = c->vl_mask; a.seq_len = c->seq_len;
+  a.q = static_cast<const __half *>(q); a.o = static_cast<__half *>(o); a.lse = lse;
+  a.counters = static_cast<int32_t *>(ws);
+  a.part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + (static_cast<size_t>(U) * 4 + 255) / 256 * 256);
+  a.status = c->dev_status;
+  return dispatch_decode<MODE_HYBRID>(G, a, st) == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
+}

@@ -63,6 +63,7 @@ EXPORTS = [
     ("hyq_vl_apply", ctypes.c_int, [_CP, _P, _I32, _P, _P, _P, _P]),
     ("hyq_decode_workspace", _SZ, [_CP, _I32]),
     ("hyq_decode", ctypes.c_int, [_CP, _P, _P, _P, _I32, _P, _SZ, _P]),
+    ("hyq_decode_noalloc", ctypes.c_int, [_CP, _P, _P, _P, _P]),
     ("hyq_decode_fp16_workspace", _SZ, [_I32, _I32, _I32, _I32]),
     ("hyq_decode_fp16", ctypes.c_int, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _I32, _P, _SZ, _P, _P]),
     ("hyq_status_string", ctypes.c_char_p, [ctypes.c_int]),
@@ -208,6 +209,14 @@ def hyq_decode_workspace(cache: HybridCache, n_ctas: int = 0) -> int:
 def hyq_decode(cache: HybridCache, q, o, ws, lse=None, n_ctas: int = 0, stream=None):
     _check(lib().hyq_decode(cache.ref(), _ptr(q), _ptr(o), _ptr(lse), n_ctas, _ptr(ws),
                             ws.numel() * ws.element_size(), _stream(stream)), "hyq_decode")
+
+
+def hyq_decode_noalloc(cache: HybridCache, q, o, lse=None, stream=None):
+    """hyq_decode with the library's built-in scratch array instead of a
+    caller workspace (for callers that cannot allocate device memory).  Calls
+    sharing a device must not overlap on the GPU."""
+    _check(lib().hyq_decode_noalloc(cache.ref(), _ptr(q), _ptr(o), _ptr(lse), _stream(stream)),
+           "hyq_decode_noalloc")
 
 
 def hyq_decode_fp16_workspace(batch, n_q_heads, n_kv_heads, n_ctas: int = 0) -> int:

@@ -220,6 +220,30 @@ hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, float *lse,
                       int32_t n_ctas, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * hyq_decode_noalloc -- hyq_decode without a workspace argument, for callers
+ * that cannot allocate device memory: for example a plugin inside a host
+ * application whose own allocator owns the whole GPU memory budget and does
+ * not let plugins call cudaMalloc, or a caller bound to a fixed C interface
+ * with no way to carry a workspace pointer.  There is no counterpart in the
+ * paper; this is a deployment convenience of the library.
+ *   Arguments as hyq_decode (n_ctas is the automatic choice).
+ *   Scratch: a fixed array compiled into the library (2,719,744 bytes), which
+ *   every GPU that loads the library keeps until the process exits.  Limits:
+ *   batch x n_kv_heads <= 4096, automatic block count <= 320, G <= 8;
+ *   larger shapes return HYQ_ERR_UNSUPPORTED without enqueuing anything.
+ *   The first call on a device looks up the array's device address (once
+ *   per device, with that device current); make that first call before any
+ *   stream capture.  Every call clears the array's counters
+ *   (cudaMemsetAsync on `stream`) and then launches the decode.
+ *   All calls share the one array: two calls whose work overlaps on the GPU
+ *   (different streams, or different host threads on one device) race and
+ *   give undefined results.  Serialize them on one stream.
+ *   Never allocates or frees memory.
+ */
+hyq_status hyq_decode_noalloc(const hyq_cache *c, const void *q, void *o, float *lse,
+                              void *stream);
+
+/*
  * hyq_decode_fp16 -- the same decode kernel design over an all-FP16 cache
  * (the full-precision comparator).
  *   q fp16 [B][Hq][128]; k, v fp16 [B][Hkv][capacity][128]; seq_len int32 [B]
