@@ -36,23 +36,33 @@
 
 namespace hyq {
 
-constexpr int NCW = 4;                    // consumer warps
-constexpr int NTHREADS = (NCW + 1) * 32;  // + 1 producer warp
-constexpr int NS = 8;                     // shared-memory ring slots
-constexpr int I4_TOK = 64;                // tokens per INT4 tile
-constexpr int F16_ROWS = 16;              // rows per FP16 tile
-constexpr int KF_STRIDE = 320;            // bytes between FP16 K rows in a slot
-constexpr int VF_STRIDE = 272;            // bytes between FP16 V rows in a slot
-constexpr int SLOT_KSZ = I4_TOK * ROW_BYTES;         // 4096
-constexpr int SLOT_VC = SLOT_KSZ + I4_TOK * SZ_BYTES;  // 5120
-constexpr int SLOT_VSZ = SLOT_VC + I4_TOK * ROW_BYTES;  // 9216
-constexpr int SLOT_MASK = SLOT_VSZ + I4_TOK * SZ_BYTES;  // 10240
-constexpr int SLOT_BYTES = SLOT_MASK + 64;                // 10304
+constexpr int NCW = 6;                    // compute warps per block, each fed by itself
+constexpr int NTHREADS = NCW * 32;
+constexpr int I4_TOK = 32;                // tokens per INT4 tile
+constexpr int F16_ROWS = 8;               // rows per FP16 tile
+constexpr int F16_ROW = D * 2;            // bytes of one FP16 K or V row
+constexpr int SLOT_F16V = F16_ROWS * F16_ROW;  // V rows of an FP16 tile start here
+constexpr int SLOT_KSZ = I4_TOK * ROW_BYTES;             // 2048
+constexpr int SLOT_VC = SLOT_KSZ + I4_TOK * SZ_BYTES;    // 2560
+constexpr int SLOT_VSZ = SLOT_VC + I4_TOK * ROW_BYTES;   // 4608
+constexpr int SLOT_MASK = SLOT_VSZ + I4_TOK * SZ_BYTES;  // 5120
+constexpr int SLOT_BYTES = SLOT_MASK + 32;               // 5152
 constexpr int PART_STRIDE = 132;  // floats per (partial, head): m, l, -, -, acc[128]
 constexpr float LOG2E_OVER_SQRT_D = 0.12751743082459868f;  // log2(e) / sqrt(128)
 constexpr float LN2 = 0.69314718055994531f;
 
-static_assert(F16_ROWS * (KF_STRIDE + VF_STRIDE) <= SLOT_MASK, "fp16 tile fits a slot");
+static_assert(2 * F16_ROWS * F16_ROW <= SLOT_MASK, "fp16 tile fits a slot");
+// Split-KV balance: a block's share is measured in these tile costs (bytes
+// read, in KiB: an INT4 tile moves 32 x 160 B, an FP16 tile 8 x 512 B).
+constexpr int COST4 = 5, COST16 = 4;
+static_assert(SLOT_BYTES % 16 == 0, "slots stay 16-byte aligned");
+
+// ring slots per compute warp: 3 (2 when 8 query heads share a KV head, so
+// that two blocks still fit one SM's shared memory)
+template <int G>
+struct Ring {
+  static constexpr int SPW = (G == 8) ? 2 : 3;
+};
 
 enum { MODE_HYBRID = 0, MODE_FP16 = 1 };
 
@@ -83,10 +93,9 @@ struct UnitShape {
 };
 
 template <int MODE>
-__device__ __forceinline__ UnitShape unit_shape(const DecodeArgs &a, int u, bool &bad) {
+__device__ __forceinline__ UnitShape shape_of(const DecodeArgs &a, int T, int vlc, bool &bad) {
   UnitShape s;
-  const int b = u / a.Hkv;
-  s.T = a.seq_len[b];
+  s.T = T;
   bad = false;
   if (s.T < 0 || s.T > a.cap) {
     bad = true;
@@ -102,7 +111,7 @@ __device__ __forceinline__ UnitShape unit_shape(const DecodeArgs &a, int u, bool
     return s;
   }
   s.L4 = s.T > a.W ? s.T - a.W : 0;
-  s.vlc = a.vl_count[u];
+  s.vlc = vlc;
   if (s.vlc < 0 || s.vlc > a.vl_cap || s.vlc > s.L4) {
     bad = true;
     s.vlc = 0;
@@ -114,6 +123,15 @@ __device__ __forceinline__ UnitShape unit_shape(const DecodeArgs &a, int u, bool
   return s;
 }
 
+// Shape of unit u from global state (prologue only; later reads use the
+// per-unit (T, vl_count) copies kept in shared memory).
+template <int MODE>
+__device__ __forceinline__ UnitShape unit_shape_global(const DecodeArgs &a, int u, bool &bad) {
+  const int T = a.seq_len[u / a.Hkv];
+  const int vlc = (MODE == MODE_FP16) ? 0 : a.vl_count[u];
+  return shape_of<MODE>(a, T, vlc, bad);
+}
+
 // Per-warp running state, in the accumulator layout of m16n8: lane (r, q)
 // holds query heads 2q and 2q+1 of the unit (heads >= G are padding).
 struct WarpState {
@@ -121,7 +139,7 @@ struct WarpState {
   float zs[2][NG];         // sum over tokens of p * vzero, per (head, group)
   float acc[NG][2][4];     // O^T accumulators: m-tile (group g, half j)
   uint32_t qf[NG][2][2];   // Q as the B operand: k-step (group g, piece s)
-  float qs[2][NG];         // log2(e)/sqrt(d) * sum of q over each group
+  float qs[2][NG];         // sum of q over each group (heads 2q, 2q+1)
 };
 
 __device__ __forceinline__ void state_reset(WarpState &st) {
@@ -167,7 +185,7 @@ __device__ __forceinline__ void load_q(WarpState &st, const DecodeArgs &a, int u
     }
     s += __shfl_xor_sync(0xffffffffu, s, 1);
     s += __shfl_xor_sync(0xffffffffu, s, 2);
-    part[g] = s * LOG2E_OVER_SQRT_D;  // lanes 4n..4n+3 hold head n
+    part[g] = s;  // lanes 4n..4n+3 hold head n
   }
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
@@ -176,12 +194,10 @@ __device__ __forceinline__ void load_q(WarpState &st, const DecodeArgs &a, int u
   }
 }
 
-// Online softmax over the 4 scores a lane holds: rows A (token sig(r)) and
-// B (sig(r)+8), heads 2q and 2q+1.  Returns the probabilities relative to the
-// running max; rescales the running state when the max grows.
-__device__ __forceinline__ void softmax_step(WarpState &st, float (&S)[4], bool vA, bool vB,
-                                             float (&p)[4]) {
-  float mx0 = fmaxf(S[0], S[2]), mx1 = fmaxf(S[1], S[3]);
+// Running-max update: when any lane sees a larger score for head 2q or
+// 2q+1, the warp reduces the new maxima over its token rows and rescales the
+// running sums and accumulators (exact max, so every p <= 1).
+__device__ __forceinline__ void rescale_if_needed(WarpState &st, float mx0, float mx1) {
   const bool need = (mx0 > st.m[0]) || (mx1 > st.m[1]);
   if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
@@ -209,6 +225,13 @@ __device__ __forceinline__ void softmax_step(WarpState &st, float (&S)[4], bool 
       }
     }
   }
+}
+
+// Online softmax over the 4 scores a lane holds in one 16-token block:
+// rows A (token sig(r)) and B (sig(r)+8), heads 2q and 2q+1.
+__device__ __forceinline__ void softmax_step(WarpState &st, float (&S)[4], bool vA, bool vB,
+                                             float (&p)[4]) {
+  rescale_if_needed(st, fmaxf(S[0], S[2]), fmaxf(S[1], S[3]));
   p[0] = vA ? fast_exp2(S[0] - st.m[0]) : 0.f;
   p[1] = vA ? fast_exp2(S[1] - st.m[1]) : 0.f;
   p[2] = vB ? fast_exp2(S[2] - st.m[0]) : 0.f;
@@ -217,57 +240,86 @@ __device__ __forceinline__ void softmax_step(WarpState &st, float (&S)[4], bool 
   st.l[1] += p[1] + p[3];
 }
 
-// One INT4 tile (up to 64 tokens) staged at `slot`.
-__device__ __forceinline__ void int4_tile(WarpState &st, uint32_t slot, int n_valid, uint64_t vlbits,
+// One INT4 tile (up to 32 tokens) staged at `slot`, in three phases so the
+// two 16-token MMA row blocks give independent work to overlap: Q.K of both
+// blocks, one online-softmax update over the 32 tokens, then P.V.
+// Invalid tokens (past the tile end, or held in the vertical-line segment)
+// get S = -inf and p = 0.  Their scale/zero bytes in shared memory are stale
+// but finite (the ring is zero-filled at start and only ever holds fp16
+// data), so p * scale stays 0 without a select.
+__device__ __forceinline__ void int4_tile(WarpState &st, uint32_t slot, int n_valid, uint32_t vlbits,
                                           int lane) {
   const int r = lane >> 2, q4 = lane & 3;
   const uint32_t kc = slot, ksz = slot + SLOT_KSZ, vc = slot + SLOT_VC, vsz = slot + SLOT_VSZ;
   const int s2q = sig(2 * q4), s2q1 = sig(2 * q4 + 1);
-#pragma unroll 1
-  for (int mt = 0; mt < I4_TOK / 16; ++mt) {
-    if (16 * mt >= n_valid) break;
+  const int nmt = (n_valid + 15) >> 4;
+  constexpr int NMT = I4_TOK / 16;
+  float S[NMT][4];
+  bool vA[NMT], vB[NMT];
+
+  // ---- phase 1: S = Q K^T per group on exact codes, per 16-token block
+#pragma unroll
+  for (int mt = 0; mt < NMT; ++mt) {
     const int tA = 16 * mt + sig(r), tB = tA + 8;
-    const bool vA = tA < n_valid && !((vlbits >> tA) & 1ull);
-    const bool vB = tB < n_valid && !((vlbits >> tB) & 1ull);
-
-    // ---- S = Q K^T per group on exact codes
-    const uint4 ka = lds128(kc + tA * ROW_BYTES + 16 * q4);
-    const uint4 kb = lds128(kc + tB * ROW_BYTES + 16 * q4);
-    float sg[NG][4];
+    vA[mt] = tA < n_valid && !((vlbits >> tA) & 1u);
+    vB[mt] = tB < n_valid && !((vlbits >> tB) & 1u);
 #pragma unroll
-    for (int g = 0; g < NG; ++g)
+    for (int e = 0; e < 4; ++e) S[mt][e] = 0.f;
+    if (mt < nmt) {
+      const uint4 ka = lds128(kc + tA * ROW_BYTES + 16 * q4);
+      const uint4 kb = lds128(kc + tB * ROW_BYTES + 16 * q4);
+      const uint4 za = lds128(ksz + tA * SZ_BYTES), zb = lds128(ksz + tB * SZ_BYTES);
+      const uint32_t zaw[4] = {za.x, za.y, za.z, za.w}, zbw[4] = {zb.x, zb.y, zb.z, zb.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sg[g][e] = 0.f;
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      const uint32_t wa0 = s ? ka.z : ka.x, wa1 = s ? ka.w : ka.y;
-      const uint32_t wb0 = s ? kb.z : kb.x, wb1 = s ? kb.w : kb.y;
-      mma16816(sg[0], nib_lo(wa0), nib_lo(wb0), nib_hi(wa0), nib_hi(wb0), st.qf[0][s][0], st.qf[0][s][1]);
-      mma16816(sg[1], nib_lo(wa0 >> 8), nib_lo(wb0 >> 8), nib_hi(wa0 >> 8), nib_hi(wb0 >> 8),
-               st.qf[1][s][0], st.qf[1][s][1]);
-      mma16816(sg[2], nib_lo(wa1), nib_lo(wb1), nib_hi(wa1), nib_hi(wb1), st.qf[2][s][0], st.qf[2][s][1]);
-      mma16816(sg[3], nib_lo(wa1 >> 8), nib_lo(wb1 >> 8), nib_hi(wa1 >> 8), nib_hi(wb1 >> 8),
-               st.qf[3][s][0], st.qf[3][s][1]);
+      for (int g = 0; g < NG; ++g) {
+        const uint32_t w0a = (g < 2) ? ka.x : ka.y, w1a = (g < 2) ? ka.z : ka.w;
+        const uint32_t w0b = (g < 2) ? kb.x : kb.y, w1b = (g < 2) ? kb.z : kb.w;
+        const int sh = (g & 1) ? 8 : 0;
+        float sg[4] = {0.f, 0.f, 0.f, 0.f};
+        mma16816(sg, nib_lo(w0a >> sh), nib_lo(w0b >> sh), nib_hi(w0a >> sh), nib_hi(w0b >> sh),
+                 st.qf[g][0][0], st.qf[g][0][1]);
+        mma16816(sg, nib_lo(w1a >> sh), nib_lo(w1b >> sh), nib_hi(w1a >> sh), nib_hi(w1b >> sh),
+                 st.qf[g][1][0], st.qf[g][1][1]);
+        const float2 fa = __half22float2(u2h(zaw[g]));  // (scale, zero) of row A
+        const float2 fb = __half22float2(u2h(zbw[g]));
+        S[mt][0] += fa.x * sg[0] + fa.y * st.qs[0][g];
+        S[mt][1] += fa.x * sg[1] + fa.y * st.qs[1][g];
+        S[mt][2] += fb.x * sg[2] + fb.y * st.qs[0][g];
+        S[mt][3] += fb.x * sg[3] + fb.y * st.qs[1][g];
+      }
     }
-    const uint4 za = lds128(ksz + tA * SZ_BYTES), zb = lds128(ksz + tB * SZ_BYTES);
-    const uint32_t zaw[4] = {za.x, za.y, za.z, za.w}, zbw[4] = {zb.x, zb.y, zb.z, zb.w};
-    float S[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int g = 0; g < NG; ++g) {
-      const float2 fa = __half22float2(u2h(zaw[g]));  // (scale, zero) of row A
-      const float2 fb = __half22float2(u2h(zbw[g]));
-      const float ca = fa.x * LOG2E_OVER_SQRT_D, cb = fb.x * LOG2E_OVER_SQRT_D;
-      S[0] += ca * sg[g][0] + fa.y * st.qs[0][g];
-      S[1] += ca * sg[g][1] + fa.y * st.qs[1][g];
-      S[2] += cb * sg[g][2] + fb.y * st.qs[0][g];
-      S[3] += cb * sg[g][3] + fb.y * st.qs[1][g];
-    }
-    if (!vA) S[0] = S[1] = -INFINITY;
-    if (!vB) S[2] = S[3] = -INFINITY;
-    float p[4];
-    softmax_step(st, S, vA, vB, p);
+    for (int e = 0; e < 4; ++e) S[mt][e] *= LOG2E_OVER_SQRT_D;
+    if (!vA[mt]) S[mt][0] = S[mt][1] = -INFINITY;
+    if (!vB[mt]) S[mt][2] = S[mt][3] = -INFINITY;
+  }
 
-    // ---- O += P V: scale folded into P per group, zero added separately
+  // ---- phase 2: one online-softmax update for the tile
+  {
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+    for (int mt = 0; mt < NMT; ++mt) {
+      mx0 = fmaxf(mx0, fmaxf(S[mt][0], S[mt][2]));
+      mx1 = fmaxf(mx1, fmaxf(S[mt][1], S[mt][3]));
+    }
+    rescale_if_needed(st, mx0, mx1);
+  }
+  float p[NMT][4];
+#pragma unroll
+  for (int mt = 0; mt < NMT; ++mt) {
+    p[mt][0] = vA[mt] ? fast_exp2(S[mt][0] - st.m[0]) : 0.f;
+    p[mt][1] = vA[mt] ? fast_exp2(S[mt][1] - st.m[1]) : 0.f;
+    p[mt][2] = vB[mt] ? fast_exp2(S[mt][2] - st.m[0]) : 0.f;
+    p[mt][3] = vB[mt] ? fast_exp2(S[mt][3] - st.m[1]) : 0.f;
+    st.l[0] += p[mt][0] + p[mt][2];
+    st.l[1] += p[mt][1] + p[mt][3];
+  }
+
+  // ---- phase 3: O += P V, scale folded into P per group, zero separately
+#pragma unroll
+  for (int mt = 0; mt < NMT; ++mt) {
+    if (mt >= nmt) break;
+    const int tA = 16 * mt + sig(r), tB = tA + 8;
     const uint4 wa = lds128(vsz + tA * SZ_BYTES), wb = lds128(vsz + tB * SZ_BYTES);
     const uint32_t waw[4] = {wa.x, wa.y, wa.z, wa.w}, wbw[4] = {wb.x, wb.y, wb.z, wb.w};
     uint32_t bq[NG][2];
@@ -275,12 +327,10 @@ __device__ __forceinline__ void int4_tile(WarpState &st, uint32_t slot, int n_va
     for (int g = 0; g < NG; ++g) {
       const float2 fa = __half22float2(u2h(waw[g]));
       const float2 fb = __half22float2(u2h(wbw[g]));
-      const float sa = vA ? fa.x : 0.f, sb = vB ? fb.x : 0.f;
-      const float za_ = vA ? fa.y : 0.f, zb_ = vB ? fb.y : 0.f;
-      st.zs[0][g] += p[0] * za_ + p[2] * zb_;
-      st.zs[1][g] += p[1] * za_ + p[3] * zb_;
-      bq[g][0] = movmatrix_t(pack_half2(p[0] * sa, p[1] * sa));
-      bq[g][1] = movmatrix_t(pack_half2(p[2] * sb, p[3] * sb));
+      st.zs[0][g] += p[mt][0] * fa.y + p[mt][2] * fb.y;
+      st.zs[1][g] += p[mt][1] * fa.y + p[mt][3] * fb.y;
+      bq[g][0] = movmatrix_t(pack_half2(p[mt][0] * fa.x, p[mt][1] * fa.x));
+      bq[g][1] = movmatrix_t(pack_half2(p[mt][2] * fb.x, p[mt][3] * fb.x));
     }
     const uint32_t vrow = vc + 8 * r;
     const uint2 x0 = lds64(vrow + (16 * mt + s2q) * ROW_BYTES);
@@ -304,190 +354,267 @@ __device__ __forceinline__ void int4_tile(WarpState &st, uint32_t slot, int n_va
   }
 }
 
-// One FP16 tile (up to 16 rows) staged at `slot` (K rows at KF_STRIDE, V rows
-// at VF_STRIDE).
+// One FP16 tile (up to 8 rows) staged at `slot`: K rows [8][256 B], then V
+// rows [8][256 B].  The MMA row block has 16 token rows; rows 8..15 are empty.
 __device__ __forceinline__ void f16_tile(WarpState &st, uint32_t slot, int n_valid, int lane) {
   const int r = lane >> 2, q4 = lane & 3;
-  const uint32_t kb_ = slot, vb_ = slot + F16_ROWS * KF_STRIDE;
-  const int tA = sig(r), tB = tA + 8;
-  const bool vA = tA < n_valid, vB = tB < n_valid;
+  const uint32_t kb_ = slot, vb_ = slot + SLOT_F16V;
+  const int tA = sig(r);
+  const bool vA = tA < n_valid;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
-    const uint4 ka = lds128(kb_ + tA * KF_STRIDE + 64 * g + 16 * q4);
-    const uint4 kb = lds128(kb_ + tB * KF_STRIDE + 64 * g + 16 * q4);
-    mma16816(acc, prmt(ka.x, ka.y, 0x5410u), prmt(kb.x, kb.y, 0x5410u), prmt(ka.x, ka.y, 0x7632u),
-             prmt(kb.x, kb.y, 0x7632u), st.qf[g][0][0], st.qf[g][0][1]);
-    mma16816(acc, prmt(ka.z, ka.w, 0x5410u), prmt(kb.z, kb.w, 0x5410u), prmt(ka.z, ka.w, 0x7632u),
-             prmt(kb.z, kb.w, 0x7632u), st.qf[g][1][0], st.qf[g][1][1]);
+    const uint4 ka = lds128(kb_ + tA * F16_ROW + 64 * g + 16 * q4);
+    mma16816(acc, prmt(ka.x, ka.y, 0x5410u), 0u, prmt(ka.x, ka.y, 0x7632u), 0u, st.qf[g][0][0], st.qf[g][0][1]);
+    mma16816(acc, prmt(ka.z, ka.w, 0x5410u), 0u, prmt(ka.z, ka.w, 0x7632u), 0u, st.qf[g][1][0], st.qf[g][1][1]);
   }
   float S[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) S[e] = acc[e] * LOG2E_OVER_SQRT_D;
   if (!vA) S[0] = S[1] = -INFINITY;
-  if (!vB) S[2] = S[3] = -INFINITY;
+  S[2] = S[3] = -INFINITY;
   float p[4];
-  softmax_step(st, S, vA, vB, p);
+  softmax_step(st, S, vA, false, p);
   const uint32_t b0 = movmatrix_t(pack_half2(p[0], p[1]));
-  const uint32_t b1 = movmatrix_t(pack_half2(p[2], p[3]));
   const int t0 = sig(2 * q4), t1 = sig(2 * q4 + 1);
-  const bool v0 = t0 < n_valid, v1 = t1 < n_valid, v2 = t0 + 8 < n_valid, v3 = t1 + 8 < n_valid;
+  const bool v0 = t0 < n_valid, v1 = t1 < n_valid;
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
     const uint32_t off = vb_ + 64 * g + 8 * r;
     const uint2 z2 = make_uint2(0, 0);
-    const uint2 A0 = v0 ? lds64(off + t0 * VF_STRIDE) : z2;
-    const uint2 A1 = v1 ? lds64(off + t1 * VF_STRIDE) : z2;
-    const uint2 B0 = v2 ? lds64(off + (t0 + 8) * VF_STRIDE) : z2;
-    const uint2 B1 = v3 ? lds64(off + (t1 + 8) * VF_STRIDE) : z2;
-    mma16816(st.acc[g][0], prmt(A0.x, A1.x, 0x5410u), prmt(A0.x, A1.x, 0x7632u), prmt(B0.x, B1.x, 0x5410u),
-             prmt(B0.x, B1.x, 0x7632u), b0, b1);
-    mma16816(st.acc[g][1], prmt(A0.y, A1.y, 0x5410u), prmt(A0.y, A1.y, 0x7632u), prmt(B0.y, B1.y, 0x5410u),
-             prmt(B0.y, B1.y, 0x7632u), b0, b1);
+    const uint2 A0 = v0 ? lds64(off + t0 * F16_ROW) : z2;
+    const uint2 A1 = v1 ? lds64(off + t1 * F16_ROW) : z2;
+    mma16816(st.acc[g][0], prmt(A0.x, A1.x, 0x5410u), prmt(A0.x, A1.x, 0x7632u), 0u, 0u, b0, 0u);
+    mma16816(st.acc[g][1], prmt(A0.y, A1.y, 0x5410u), prmt(A0.y, A1.y, 0x7632u), 0u, 0u, b0, 0u);
   }
 }
 
+__host__ __device__ __forceinline__ int U_of(const DecodeArgs &a) { return a.U; }
+
 struct Smem {
-  uint32_t slots;     // shared address of slot 0
-  uint64_t *full, *empty;
+  uint32_t slots;     // shared address of slot 0: [NCW][SPW][SLOT_BYTES]
+  uint64_t *full;     // [NCW][SPW] transaction barriers, one per slot
   int *abort_flag, *last_flag;
   float *mm, *ml, *mo;  // merge buffers: [NCW][8], [NCW][8], [NCW][G][128]
-  int *tile_start;      // [U + 1]
+  int *cost_start;      // [U + 1]: cost of the units before u
   int *scan;            // [NTHREADS]
+  int2 *unit_tv;        // [U]: (T, vl_count) as read at launch
 };
 
-__device__ __forceinline__ int64_t cta_first_tile(int64_t c, int64_t n_tiles, int64_t n_ctas) {
-  return c * n_tiles / n_ctas;
-}
-// CTA that owns global tile t: the largest c with first_tile(c) <= t.
-__device__ __forceinline__ int cta_of_tile(int64_t t, int64_t n_tiles, int64_t n_ctas) {
-  return static_cast<int>(((t + 1) * n_ctas - 1) / n_tiles);
+// Tiles of unit u: n4 INT4 tiles, then n16 FP16 tiles (vertical lines, window).
+template <int MODE>
+__device__ __forceinline__ void unit_tiles(const DecodeArgs &a, const Smem &sm, int u, int &n4, int &n16) {
+  bool bad;
+  const UnitShape s = shape_of<MODE>(a, sm.unit_tv[u].x, sm.unit_tv[u].y, bad);
+  n4 = s.n4;
+  n16 = s.nv + s.nw;
 }
 
-// last unit u with tile_start[u] <= t < tile_start[u+1]
-__device__ __forceinline__ int unit_of_tile(const int *ts, int U, int t) {
+// First tile of a unit (cost start cs, n4 + n16 tiles) whose start cost is >= x.
+__device__ __forceinline__ int first_tile_from(int64_t x, int64_t cs, int n4, int n16) {
+  const int64_t rel = x - cs;
+  if (rel <= 0) return 0;
+  const int64_t c4 = static_cast<int64_t>(COST4) * n4;
+  int64_t j;
+  if (rel <= c4) j = (rel + COST4 - 1) / COST4;
+  else j = n4 + (rel - c4 + COST16 - 1) / COST16;
+  return static_cast<int>(j < n4 + n16 ? j : n4 + n16);
+}
+
+// Start cost of tile j of a unit.
+__device__ __forceinline__ int64_t tile_cost(int64_t cs, int n4, int j) {
+  return j <= n4 ? cs + static_cast<int64_t>(COST4) * j
+                 : cs + static_cast<int64_t>(COST4) * n4 + static_cast<int64_t>(COST16) * (j - n4);
+}
+
+__device__ __forceinline__ int64_t cta_lo(int64_t c, int64_t total, int64_t n_ctas) { return c * total / n_ctas; }
+// block whose cost range holds x: the largest c with cta_lo(c) <= x
+__device__ __forceinline__ int cta_of_cost(int64_t x, int64_t total, int64_t n_ctas) {
+  return static_cast<int>(((x + 1) * n_ctas - 1) / total);
+}
+
+// last unit u with cost_start[u] <= x
+__device__ __forceinline__ int unit_of_cost(const int *cs, int U, int64_t x) {
   int lo = 0, hi = U - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (ts[mid] <= t) lo = mid; else hi = mid - 1;
+    if (cs[mid] <= x) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
 
+// A block's tiles of one unit: the segment [jb, je) of unit u, which holds
+// block-local tile indices [base, base + je - jb).
+struct Seg {
+  int u, jb, je, base;
+};
+
+// Next non-empty segment of this block at or after unit u (u = U: none).
+template <int MODE>
+__device__ __forceinline__ Seg seg_from(const DecodeArgs &a, const Smem &sm, int u, int base, int64_t lo, int64_t hi) {
+  Seg s{a.U, 0, 0, base};
+  for (; u < a.U && sm.cost_start[u] < hi; ++u) {
+    int n4, n16;
+    unit_tiles<MODE>(a, sm, u, n4, n16);
+    const int jb = first_tile_from(lo, sm.cost_start[u], n4, n16);
+    const int je = first_tile_from(hi, sm.cost_start[u], n4, n16);
+    if (jb < je) {
+      s.u = u;
+      s.jb = jb;
+      s.je = je;
+      return s;
+    }
+  }
+  return s;
+}
+
 // Merge the partials of unit u written by the blocks that share it (run by
-// the last one to finish; 128 consumer threads).  Parts are taken in chunks
-// of MERGE_CHUNK: their (max, sum) pairs are loaded in parallel, per-head
-// weights 2^(m_p - M) live in shared memory, and every thread accumulates
-// float4 slices of the output with many loads in flight.
+// the last block to finish, 128 consumer threads).  The ids of the partial
+// records go to shared memory first; then every thread owns float4 slices of
+// the output of one head and merges the records online, loading (max, sum,
+// slice) of MERGE_BATCH records at a time so their latencies overlap.
 constexpr int MERGE_CHUNK = 128;
+constexpr int MERGE_BATCH = 20;
 
 template <int G>
-__device__ __forceinline__ void merge_parts(const DecodeArgs &a, const Smem &sm, int u, int u0, int u1,
-                                            int64_t n_tiles, int64_t N, int64_t hbase, int tid) {
-  float *pw = sm.mo;                       // [MERGE_CHUNK][G] weights
-  float *pl = sm.mo + MERGE_CHUNK * G;     // [MERGE_CHUNK][G] sums
-  int *pid = sm.scan;                      // [MERGE_CHUNK] partial record index or -1
-  float *runM = sm.mm, *runL = sm.ml, *alpha = sm.mm + 8;
-  const int c_lo = cta_of_tile(u0, n_tiles, N), c_hi = cta_of_tile(u1 - 1, n_tiles, N);
+__device__ __forceinline__ void merge_parts(const DecodeArgs &a, const Smem &sm, int u, int n4, int n16,
+                                            int64_t total, int64_t N, int64_t hbase, int tid) {
+  int *pid = sm.scan;  // [MERGE_CHUNK] partial record index, or -1 for a block without tiles of u
+  const int64_t cs = sm.cost_start[u];
+  const int c_lo = cta_of_cost(cs, total, N), c_hi = cta_of_cost(tile_cost(cs, n4, n4 + n16 - 1), total, N);
   constexpr int NV = (G * D / 4 + NCW * 32 - 1) / (NCW * 32);  // float4 outputs per thread
   float4 acc[NV];
+  float M[NV], L[NV];
 #pragma unroll
-  for (int v = 0; v < NV; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (tid < G) {
-    runM[tid] = -INFINITY;
-    runL[tid] = 0.f;
+  for (int v = 0; v < NV; ++v) {
+    acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    M[v] = -INFINITY;
+    L[v] = 0.f;
   }
   for (int base = c_lo; base <= c_hi; base += MERGE_CHUNK) {
     const int n = min(MERGE_CHUNK, c_hi - base + 1);
     named_bar_sync(1, NCW * 32);
     for (int j = tid; j < n; j += NCW * 32) {
       const int64_t cc = base + j;
-      const int64_t f0 = cta_first_tile(cc, n_tiles, N), f1 = cta_first_tile(cc + 1, n_tiles, N);
-      pid[j] = (f0 == f1) ? -1 : static_cast<int>(cc * 2 + ((u0 >= f0) ? 0 : 1));
-    }
-    named_bar_sync(1, NCW * 32);
-    for (int e = tid; e < n * G; e += NCW * 32) {
-      const int j = e / G, h = e % G;
-      float m = -INFINITY, l = 0.f;
-      if (pid[j] >= 0) {
-        const float *pr = a.part + (static_cast<int64_t>(pid[j]) * G + h) * PART_STRIDE;
-        m = __ldcg(pr);
-        l = __ldcg(pr + 1);
-      }
-      pw[e] = m;
-      pl[e] = l;
-    }
-    named_bar_sync(1, NCW * 32);
-    if (tid < G) {
-      const int h = tid;
-      float cm = -INFINITY;
-      for (int j = 0; j < n; ++j) cm = fmaxf(cm, pw[j * G + h]);
-      const float M = fmaxf(runM[h], cm);
-      const float al = (runM[h] == -INFINITY) ? 0.f : fast_exp2(runM[h] - M);
-      float L = runL[h] * al;
-      for (int j = 0; j < n; ++j) {
-        const float m = pw[j * G + h];
-        const float w = (m == -INFINITY) ? 0.f : fast_exp2(m - M);
-        pw[j * G + h] = w;
-        L += pl[j * G + h] * w;
-      }
-      runM[h] = M;
-      runL[h] = L;
-      alpha[h] = al;
+      const int64_t lo = cta_lo(cc, total, N), hi = cta_lo(cc + 1, total, N);
+      const bool has = first_tile_from(lo, cs, n4, n16) < first_tile_from(hi, cs, n4, n16);
+      pid[j] = has ? static_cast<int>(cc * 2 + ((cs <= lo) ? 0 : 1)) : -1;
     }
     named_bar_sync(1, NCW * 32);
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
       const int o4 = tid + v * NCW * 32;  // float4 index over [G][32]
-      if (o4 < G * D / 4) {
-        const int h = o4 / (D / 4), c4 = o4 % (D / 4);
-        const float al = alpha[h];
-        float4 s = make_float4(acc[v].x * al, acc[v].y * al, acc[v].z * al, acc[v].w * al);
-#pragma unroll 16
-        for (int j = 0; j < n; ++j) {
-          const int id = pid[j];
-          if (id < 0) continue;
-          const float w = pw[j * G + h];
-          const float4 x = __ldcg(reinterpret_cast<const float4 *>(
-              a.part + (static_cast<int64_t>(id) * G + h) * PART_STRIDE + 4 + 4 * c4));
-          s.x += w * x.x;
-          s.y += w * x.y;
-          s.z += w * x.z;
-          s.w += w * x.w;
+      if (o4 >= G * D / 4) continue;
+      const int h = o4 / (D / 4), c4 = o4 % (D / 4);
+      for (int j0 = 0; j0 < n; j0 += MERGE_BATCH) {
+        float2 ml[MERGE_BATCH];
+        float4 x[MERGE_BATCH];
+#pragma unroll
+        for (int b = 0; b < MERGE_BATCH; ++b) {
+          const int id = (j0 + b < n) ? pid[j0 + b] : -1;
+          ml[b] = make_float2(-INFINITY, 0.f);
+          x[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (id >= 0) {
+            const float *pr = a.part + (static_cast<int64_t>(id) * G + h) * PART_STRIDE;
+            ml[b] = __ldcg(reinterpret_cast<const float2 *>(pr));
+            x[b] = __ldcg(reinterpret_cast<const float4 *>(pr + 4 + 4 * c4));
+          }
         }
-        acc[v] = s;
+        float bm = M[v];
+#pragma unroll
+        for (int b = 0; b < MERGE_BATCH; ++b) bm = fmaxf(bm, ml[b].x);
+        if (bm == -INFINITY) continue;
+        const float al = (M[v] == -INFINITY) ? 0.f : fast_exp2(M[v] - bm);
+        float4 s4 = make_float4(acc[v].x * al, acc[v].y * al, acc[v].z * al, acc[v].w * al);
+        float sl = L[v] * al;
+#pragma unroll
+        for (int b = 0; b < MERGE_BATCH; ++b) {
+          const float w = (ml[b].x == -INFINITY) ? 0.f : fast_exp2(ml[b].x - bm);
+          sl += w * ml[b].y;
+          s4.x += w * x[b].x;
+          s4.y += w * x[b].y;
+          s4.z += w * x[b].z;
+          s4.w += w * x[b].w;
+        }
+        acc[v] = s4;
+        M[v] = bm;
+        L[v] = sl;
       }
     }
   }
-  named_bar_sync(1, NCW * 32);
 #pragma unroll
   for (int v = 0; v < NV; ++v) {
     const int o4 = tid + v * NCW * 32;
     if (o4 < G * D / 4) {
       const int h = o4 / (D / 4), c4 = o4 % (D / 4);
-      const float inv = 1.f / runL[h];
+      const float inv = 1.f / L[v];
       __half2 lo = __floats2half2_rn(acc[v].x * inv, acc[v].y * inv);
       __half2 hi = __floats2half2_rn(acc[v].z * inv, acc[v].w * inv);
-      uint2 pk = make_uint2(h2u(lo), h2u(hi));
-      *reinterpret_cast<uint2 *>(a.o + (hbase + h) * D + 4 * c4) = pk;
-      if (c4 == 0 && a.lse) a.lse[hbase + h] = (runM[h] + __log2f(runL[h])) * LN2;
+      *reinterpret_cast<uint2 *>(a.o + (hbase + h) * D + 4 * c4) = make_uint2(h2u(lo), h2u(hi));
+      if (c4 == 0 && a.lse) a.lse[hbase + h] = (M[v] + __log2f(L[v])) * LN2;
     }
   }
 }
 
+// Issue the bulk copies of tile j of unit u into one ring slot (lane 0 arms
+// the barrier and copies; an FP16 tile is two contiguous runs of rows).
+template <int MODE>
+__device__ __forceinline__ void issue_tile(const DecodeArgs &a, const Smem &sm, int u, int j, uint32_t dst,
+                                           uint32_t bar, int lane) {
+  bool bad;
+  const UnitShape us = shape_of<MODE>(a, sm.unit_tv[u].x, sm.unit_tv[u].y, bad);
+  if (lane != 0) return;
+  if (MODE == MODE_HYBRID && j < us.n4) {
+    const int t0 = j * I4_TOK;
+    const int n = min(I4_TOK, us.L4 - t0);
+    const int64_t row = static_cast<int64_t>(u) * a.cap + t0;
+    mbar_arrive_expect_tx(bar, n * 160 + 16);
+    bulk_g2s(dst, a.k_codes + row * ROW_BYTES, n * ROW_BYTES, bar);
+    bulk_g2s(dst + SLOT_KSZ, a.k_sz + row * SZ_BYTES, n * SZ_BYTES, bar);
+    bulk_g2s(dst + SLOT_VC, a.v_codes + row * ROW_BYTES, n * ROW_BYTES, bar);
+    bulk_g2s(dst + SLOT_VSZ, a.v_sz + row * SZ_BYTES, n * SZ_BYTES, bar);
+    const uint32_t *mrow = a.vl_mask + static_cast<int64_t>(u) * (a.cap / 32);
+    bulk_g2s(dst + SLOT_MASK, mrow + ((t0 / 32) & ~3), 16, bar);
+    return;
+  }
+  const __half *sk, *sv;
+  int n;
+  if (MODE == MODE_FP16) {
+    const int r0 = j * F16_ROWS;
+    n = min(F16_ROWS, us.T - r0);
+    const int64_t base = (static_cast<int64_t>(u) * a.cap + r0) * D;
+    sk = a.k16 + base;
+    sv = a.v16 + base;
+  } else if (j < us.n4 + us.nv) {
+    const int r0 = (j - us.n4) * F16_ROWS;
+    n = min(F16_ROWS, us.vlc - r0);
+    const int64_t base = (static_cast<int64_t>(u) * a.vl_cap + r0) * D;
+    sk = a.vl_k + base;
+    sv = a.vl_v + base;
+  } else {
+    const int r0 = (j - us.n4 - us.nv) * F16_ROWS;
+    n = min(F16_ROWS, us.nwin - r0);
+    const int64_t base = (static_cast<int64_t>(u) * a.W + r0) * D;
+    sk = a.win_k + base;
+    sv = a.win_v + base;
+  }
+  mbar_arrive_expect_tx(bar, n * 2 * F16_ROW);
+  bulk_g2s(dst, sk, n * F16_ROW, bar);
+  bulk_g2s(dst + SLOT_F16V, sv, n * F16_ROW, bar);
+}
+
 template <int G, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a) {
+  constexpr int SPW = Ring<G>::SPW;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   Smem sm;
   {
     uint8_t *p = smem_raw;
     sm.slots = smem_u32(p);
-    p += NS * SLOT_BYTES;
+    p += NCW * SPW * SLOT_BYTES;
     sm.full = reinterpret_cast<uint64_t *>(p);
-    p += NS * 8;
-    sm.empty = reinterpret_cast<uint64_t *>(p);
-    p += NS * 8;
+    p += NCW * SPW * 8;
     sm.abort_flag = reinterpret_cast<int *>(p);
     sm.last_flag = sm.abort_flag + 1;
     p += 16;
@@ -499,22 +626,30 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
     p += NCW * G * D * 4;
     sm.scan = reinterpret_cast<int *>(p);
     p += NTHREADS * 4;
-    sm.tile_start = reinterpret_cast<int *>(p);
+    sm.cost_start = reinterpret_cast<int *>(p);
+    p += ((U_of(a) + 1) * 4 + 15) / 16 * 16;
+    sm.unit_tv = reinterpret_cast<int2 *>(p);
   }
   const int U = a.U;
 
-  // ---- schedule: tile_start[u] = tiles of units before u
+  // ---- prologue: zero the ring, read every unit's (T, vl_count), cost prefix
   {
+    // the ring starts as zeros, so stale bytes read as scale/zero are finite
+    for (int i = tid; i < NCW * SPW * SLOT_BYTES / 16; i += NTHREADS)
+      *reinterpret_cast<uint4 *>(smem_raw + 16 * i) = make_uint4(0, 0, 0, 0);
+    // order these generic-proxy stores before the bulk copies (async proxy)
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     const int per = (U + NTHREADS - 1) / NTHREADS;
     const int beg = min(U, tid * per), end = min(U, beg + per);
     int local = 0;
     for (int u = beg; u < end; ++u) {
       bool bad;
-      const UnitShape s = unit_shape<MODE>(a, u, bad);
-      local += s.n4 + s.nv + s.nw;
+      const UnitShape s = unit_shape_global<MODE>(a, u, bad);
+      sm.unit_tv[u] = make_int2(s.T, s.vlc);
+      local += COST4 * s.n4 + COST16 * (s.nv + s.nw);
+      if (bad && (u % a.n_ctas) == static_cast<int>(blockIdx.x)) set_status(a.status, HYQ_DEV_BADLEN);
     }
-    // block exclusive scan of `local`
-    int v = local;
+    int v = local;  // block exclusive scan of `local`
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, v, off);
@@ -523,10 +658,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
     if (lane == 31) sm.scan[warp] = v;
     if (tid == 0) {
       *sm.abort_flag = 0;
-      for (int s = 0; s < NS; ++s) {
-        mbar_init(smem_u32(&sm.full[s]), 1);
-        mbar_init(smem_u32(&sm.empty[s]), 1);
-      }
+      for (int s = 0; s < NCW * SPW; ++s) mbar_init(smem_u32(&sm.full[s]), 1);
       fence_barrier_init();
     }
     __syncthreads();
@@ -534,121 +666,71 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
     for (int w = 0; w < warp; ++w) wpre += sm.scan[w];
     int acc = wpre + v - local;
     for (int u = beg; u < end; ++u) {
-      bool bad;
-      const UnitShape s = unit_shape<MODE>(a, u, bad);
-      sm.tile_start[u] = acc;
-      acc += s.n4 + s.nv + s.nw;
-      if (bad && (u % a.n_ctas) == static_cast<int>(blockIdx.x)) set_status(a.status, HYQ_DEV_BADLEN);
+      int n4, n16;
+      unit_tiles<MODE>(a, sm, u, n4, n16);
+      sm.cost_start[u] = acc;
+      acc += COST4 * n4 + COST16 * n16;
     }
-    if (tid == NTHREADS - 1) sm.tile_start[U] = acc;
+    if (tid == NTHREADS - 1) sm.cost_start[U] = acc;
     __syncthreads();
   }
-  const int64_t n_tiles = sm.tile_start[U];
+  const int64_t total = sm.cost_start[U];
   const int64_t N = a.n_ctas;
   const int cta = blockIdx.x;
-  const int t_begin = static_cast<int>(cta_first_tile(cta, n_tiles, N));
-  const int t_end = static_cast<int>(cta_first_tile(cta + 1, n_tiles, N));
+  const int64_t lo = total ? cta_lo(cta, total, N) : 0, hi = total ? cta_lo(cta + 1, total, N) : 0;
   volatile int *abort_flag = sm.abort_flag;
+  const int u_first = (lo < hi) ? unit_of_cost(sm.cost_start, U, lo) : U;
 
-  if (warp == NCW) {
-    // ================= producer
-    int i = 0;
-    bool ok = true;
-    for (int t = t_begin; t < t_end && ok;) {
-      const int u = unit_of_tile(sm.tile_start, U, t);
-      const int u0 = sm.tile_start[u], u1 = sm.tile_start[u + 1];
-      const int seg_end = min(t_end, u1);
-      bool bad;
-      const UnitShape us = unit_shape<MODE>(a, u, bad);
-      for (; t < seg_end; ++t, ++i) {
-        const int s = i % NS;
-        const uint32_t ph = (i / NS) & 1;
-        if (i >= NS && !mbar_wait_bounded(smem_u32(&sm.empty[s]), ph ^ 1u, abort_flag, a.status)) {
-          ok = false;
-          break;
-        }
-        const uint32_t dst = sm.slots + s * SLOT_BYTES;
-        const uint32_t bar = smem_u32(&sm.full[s]);
-        const int j = t - u0;
-        if (MODE == MODE_HYBRID && j < us.n4) {
-          const int t0 = j * I4_TOK;
-          const int n = min(I4_TOK, us.L4 - t0);
-          if (lane == 0) {
-            const int64_t row = static_cast<int64_t>(u) * a.cap + t0;
-            mbar_arrive_expect_tx(bar, n * 160 + 16);
-            bulk_g2s(dst, a.k_codes + row * ROW_BYTES, n * ROW_BYTES, bar);
-            bulk_g2s(dst + SLOT_KSZ, a.k_sz + row * SZ_BYTES, n * SZ_BYTES, bar);
-            bulk_g2s(dst + SLOT_VC, a.v_codes + row * ROW_BYTES, n * ROW_BYTES, bar);
-            bulk_g2s(dst + SLOT_VSZ, a.v_sz + row * SZ_BYTES, n * SZ_BYTES, bar);
-            const uint32_t *mrow = a.vl_mask + static_cast<int64_t>(u) * (a.cap / 32);
-            bulk_g2s(dst + SLOT_MASK, mrow + ((t0 / 32) & ~3), 16, bar);
-          }
-        } else {
-          const __half *sk, *sv;
-          int r0, n;
-          if (MODE == MODE_FP16) {
-            r0 = j * F16_ROWS;
-            n = min(F16_ROWS, us.T - r0);
-            const int64_t base = (static_cast<int64_t>(u) * a.cap + r0) * D;
-            sk = a.k16 + base;
-            sv = a.v16 + base;
-          } else if (j < us.n4 + us.nv) {
-            r0 = (j - us.n4) * F16_ROWS;
-            n = min(F16_ROWS, us.vlc - r0);
-            const int64_t base = (static_cast<int64_t>(u) * a.vl_cap + r0) * D;
-            sk = a.vl_k + base;
-            sv = a.vl_v + base;
-          } else {
-            r0 = (j - us.n4 - us.nv) * F16_ROWS;
-            n = min(F16_ROWS, us.nwin - r0);
-            const int64_t base = (static_cast<int64_t>(u) * a.W + r0) * D;
-            sk = a.win_k + base;
-            sv = a.win_v + base;
-          }
-          if (lane == 0) mbar_arrive_expect_tx(bar, n * 2 * D * 2);
-          __syncwarp();
-          if (lane < n) {
-            bulk_g2s(dst + lane * KF_STRIDE, sk + lane * D, D * 2, bar);
-            bulk_g2s(dst + F16_ROWS * KF_STRIDE + lane * VF_STRIDE, sv + lane * D, D * 2, bar);
-          }
-        }
-        __syncwarp();
-      }
-      (void)u1;
-    }
-    if (!ok) {
-      // let copies already issued land before the block can exit
-      for (int k = (i > NS ? i - NS : 0); k < i; ++k)
-        mbar_wait_bounded(smem_u32(&sm.full[k % NS]), (k / NS) & 1, abort_flag, a.status, 500000000ull);
-    }
-    return;
-  }
+  // This warp's tiles are the block-local tiles warp, warp + NCW, ...; its
+  // k-th tile lives in ring slot k % SPW.  The warp issues its own copies:
+  // SPW tiles ahead at the start, then tile k + SPW once tile k is read.
+  const uint32_t my_slots = sm.slots + warp * SPW * SLOT_BYTES;
+  const uint32_t my_bars = smem_u32(&sm.full[warp * SPW]);
+  int k_issued = 0, k_done = 0, first_fail = -1;
+  Seg ic = seg_from<MODE>(a, sm, u_first, 0, lo, hi);  // issue cursor
+  auto issue_next = [&]() {
+    const int i = warp + NCW * k_issued;  // block-local tile index
+    while (ic.u < U && i >= ic.base + ic.je - ic.jb)
+      ic = seg_from<MODE>(a, sm, ic.u + 1, ic.base + ic.je - ic.jb, lo, hi);
+    const int stop = __shfl_sync(0xffffffffu, *abort_flag, 0);  // one decision per warp
+    if (ic.u >= U || stop) return;
+    const int sl = k_issued % SPW;
+    issue_tile<MODE>(a, sm, ic.u, ic.jb + (i - ic.base), my_slots + sl * SLOT_BYTES, my_bars + sl * 8, lane);
+    __syncwarp();
+    ++k_issued;
+  };
+  for (int k = 0; k < SPW; ++k) issue_next();
 
-  // ================= consumers
   WarpState st;
-  int i = 0;
-  for (int t = t_begin; t < t_end;) {
-    const int u = unit_of_tile(sm.tile_start, U, t);
-    const int u0 = sm.tile_start[u], u1 = sm.tile_start[u + 1];
-    const int seg_beg = t, seg_end = min(t_end, u1);
+  for (Seg sg = seg_from<MODE>(a, sm, u_first, 0, lo, hi); sg.u < U;
+       sg = seg_from<MODE>(a, sm, sg.u + 1, sg.base + sg.je - sg.jb, lo, hi)) {
+    const int u = sg.u;
     bool bad;
-    const UnitShape us = unit_shape<MODE>(a, u, bad);
+    const UnitShape us = shape_of<MODE>(a, sm.unit_tv[u].x, sm.unit_tv[u].y, bad);
+    const int n_unit = us.n4 + us.nv + us.nw;
     state_reset(st);
     load_q<G>(st, a, u, lane);
-    for (; t < seg_end; ++t, ++i) {
-      if (i % NCW != warp) continue;
-      const int s = i % NS;
-      const uint32_t ph = (i / NS) & 1;
-      if (!mbar_wait_bounded(smem_u32(&sm.full[s]), ph, abort_flag, a.status)) continue;
-      const uint32_t slot = sm.slots + s * SLOT_BYTES;
-      const int j = t - u0;
+    // my tiles inside this segment: block-local i = base .. base + je - jb - 1
+    int i = sg.base + (warp - sg.base % NCW + NCW) % NCW;
+    for (; i < sg.base + sg.je - sg.jb; i += NCW) {
+      const int kk = k_done;
+      const int sl = kk % SPW;
+      const uint32_t slot = my_slots + sl * SLOT_BYTES;
+      ++k_done;
+      bool landed = first_fail < 0 && mbar_wait_bounded(my_bars + sl * 8, (kk / SPW) & 1, abort_flag, a.status);
+      landed = __all_sync(0xffffffffu, landed);  // the warp computes together or not at all
+      if (!landed) {
+        if (first_fail < 0) first_fail = kk;
+        continue;
+      }
+      const int j = sg.jb + (i - sg.base);
       if (MODE == MODE_HYBRID && j < us.n4) {
         const int t0 = j * I4_TOK;
         const int n = min(I4_TOK, us.L4 - t0);
         const uint4 mw = lds128(slot + SLOT_MASK);
-        const int wsel = (t0 / 32) & 3;  // 0 or 2
-        const uint32_t lo = wsel ? mw.z : mw.x, hi = wsel ? mw.w : mw.y;
-        int4_tile(st, slot, n, (static_cast<uint64_t>(hi) << 32) | lo, lane);
+        const int wsel = (t0 / 32) & 3;
+        const uint32_t bits = wsel == 0 ? mw.x : wsel == 1 ? mw.y : wsel == 2 ? mw.z : mw.w;
+        int4_tile(st, slot, n, bits, lane);
       } else {
         int n;
         if (MODE == MODE_FP16)
@@ -659,8 +741,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
           n = min(F16_ROWS, us.nwin - (j - us.n4 - us.nv) * F16_ROWS);
         f16_tile(st, slot, n, lane);
       }
+      // the slot has been read: order those reads before the next bulk copy
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm.empty[s]));
+      issue_next();
     }
 
     // ---- segment end: reduce the warp's state over token rows
@@ -693,14 +777,14 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
           }
       }
     }
-    named_bar_sync(1, NCW * 32);
+    named_bar_sync(1, NTHREADS);
 
-    // ---- merge the consumer warps
-    const bool complete = (seg_beg == u0) && (seg_end == u1);
-    const int slot_id = (u0 >= t_begin) ? 0 : 1;  // 1: the unit began in an earlier block
+    // ---- merge the warps of the block
+    const bool complete = (sg.jb == 0) && (sg.je == n_unit);
+    const int slot_id = (sm.cost_start[u] <= lo) ? 0 : 1;  // 1: the unit began after this block's start
     const int b = u / a.Hkv, kvh = u % a.Hkv;
     const int64_t hbase = static_cast<int64_t>(b) * a.Hq + kvh * G;
-    for (int idx = tid; idx < G * D; idx += NCW * 32) {
+    for (int idx = tid; idx < G * D; idx += NTHREADS) {
       const int h = idx / D, c = idx % D;
       float M = -INFINITY;
 #pragma unroll
@@ -727,29 +811,32 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
     }
     if (!complete) {
       __threadfence();
-      named_bar_sync(1, NCW * 32);
+      named_bar_sync(1, NTHREADS);
       if (tid == 0) {
-        const int mine = seg_end - seg_beg;
+        const int mine = sg.je - sg.jb;
         const int old = atomicAdd(&a.counters[u], mine);
-        *sm.last_flag = (old + mine == u1 - u0);
+        *sm.last_flag = (old + mine == n_unit);
       }
-      named_bar_sync(1, NCW * 32);
+      named_bar_sync(1, NTHREADS);
       if (*sm.last_flag) {
         __threadfence();
-        merge_parts<G>(a, sm, u, u0, u1, n_tiles, N, hbase, tid);
+        merge_parts<G>(a, sm, u, us.n4, us.nv + us.nw, total, N, hbase, tid);
         if (tid == 0) a.counters[u] = 0;
       }
     }
-    named_bar_sync(1, NCW * 32);
-    t = seg_end;
+    named_bar_sync(1, NTHREADS);
   }
+
+  // copies still in flight (only after an abort): let them land before exit
+  for (int kk = (first_fail >= 0 ? first_fail : k_done); kk < k_issued; ++kk)
+    mbar_drain(my_bars + (kk % SPW) * 8, (kk / SPW) & 1, 500000000ull);
 
   // units without any position: o = 0, lse = -inf (one block each)
   for (int u = cta; u < U; u += a.n_ctas) {
-    if (sm.tile_start[u] != sm.tile_start[u + 1]) continue;
+    if (sm.cost_start[u] != sm.cost_start[u + 1]) continue;
     const int b = u / a.Hkv, kvh = u % a.Hkv;
     const int64_t hbase = static_cast<int64_t>(b) * a.Hq + kvh * G;
-    for (int idx = tid; idx < G * D; idx += NCW * 32) {
+    for (int idx = tid; idx < G * D; idx += NTHREADS) {
       a.o[(hbase + idx / D) * D + idx % D] = __float2half_rn(0.f);
       if (idx % D == 0 && a.lse) a.lse[hbase + idx / D] = -INFINITY;
     }
@@ -758,8 +845,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
 
 // ---------------------------------------------------------------- host side
 static size_t decode_smem_bytes(int G, int U) {
-  return static_cast<size_t>(NS) * SLOT_BYTES + NS * 16 + 16 + NCW * 8 * 4 * 2 +
-         static_cast<size_t>(NCW) * G * D * 4 + NTHREADS * 4 + static_cast<size_t>(U + 1) * 4;
+  const int spw = (G == 8) ? 2 : 3;
+  return static_cast<size_t>(NCW) * spw * SLOT_BYTES + NCW * spw * 8 + 16 + NCW * 8 * 4 * 2 +
+         static_cast<size_t>(NCW) * G * D * 4 + NTHREADS * 4 + (static_cast<size_t>(U + 1) * 4 + 15) / 16 * 16 +
+         static_cast<size_t>(U) * 8;
 }
 
 static size_t decode_ws_bytes(int G, int U, int n_ctas) {
