@@ -17,8 +17,8 @@ extern "C" hyq_status hyq_check_cache(const hyq_cache *c) {
   if (G != 1 && G != 2 && G != 4 && G != 8) return HYQ_ERR_UNSUPPORTED;
   if (c->capacity <= 0 || (c->capacity % 128) != 0) return HYQ_ERR_INVALID;
   if (c->vl_capacity <= 0) return HYQ_ERR_INVALID;
-  const void *ptrs[] = {c->k_codes, c->v_codes, c->k_sz,     c->v_sz,    c->win_k,  c->win_v,
-                        c->vl_k,    c->vl_v,    c->vl_pos,   c->vl_count, c->vl_mask, c->seq_len};
+  const void *ptrs[] = {c->blocks, c->win_k,  c->win_v,    c->vl_k,
+                        c->vl_v,   c->vl_pos, c->vl_count, c->seq_len};
   for (const void *p : ptrs) {
     if (!p) return HYQ_ERR_INVALID;
     if (!al16(p)) return HYQ_ERR_ALIGN;

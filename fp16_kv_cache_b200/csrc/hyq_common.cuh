@@ -21,6 +21,30 @@ constexpr int WIN = 128;
 constexpr int ROW_BYTES = 64;
 constexpr int SZ_BYTES = 16;
 constexpr int MAX_UNITS = 4096;  // units (batch x kv heads) one launch schedules
+constexpr int BLK_TOK = HYQ_BLOCK_TOKENS;
+constexpr int BLK_BYTES = HYQ_BLOCK_BYTES;
+
+// Quantized-majority block of position p of unit u, and the byte offsets of
+// that position's K/V codes and scale/zero rows inside the cache's blocks.
+__host__ __device__ __forceinline__ int64_t blk_base(int64_t u, int64_t p, int cap) {
+  return (u * (cap / BLK_TOK) + p / BLK_TOK) * BLK_BYTES;
+}
+__host__ __device__ __forceinline__ int64_t kcode_off(int64_t u, int64_t p, int cap) {
+  return blk_base(u, p, cap) + HYQ_BLK_KCODES + (p % BLK_TOK) * ROW_BYTES;
+}
+__host__ __device__ __forceinline__ int64_t ksz_off(int64_t u, int64_t p, int cap) {
+  return blk_base(u, p, cap) + HYQ_BLK_KSZ + (p % BLK_TOK) * SZ_BYTES;
+}
+__host__ __device__ __forceinline__ int64_t vcode_off(int64_t u, int64_t p, int cap) {
+  return blk_base(u, p, cap) + HYQ_BLK_VCODES + (p % BLK_TOK) * ROW_BYTES;
+}
+__host__ __device__ __forceinline__ int64_t vsz_off(int64_t u, int64_t p, int cap) {
+  return blk_base(u, p, cap) + HYQ_BLK_VSZ + (p % BLK_TOK) * SZ_BYTES;
+}
+// the vertical-line bitmask word covering position p (bit p % 32)
+__device__ __forceinline__ uint32_t *mask_word(uint8_t *blocks, int64_t u, int64_t p, int cap) {
+  return reinterpret_cast<uint32_t *>(blocks + blk_base(u, p, cap) + HYQ_BLK_MASK);
+}
 
 // ---------------------------------------------------------------- status
 __device__ __forceinline__ void set_status(uint32_t *st, uint32_t bits) {

@@ -42,11 +42,12 @@ constexpr int I4_TOK = 32;                // tokens per INT4 tile
 constexpr int F16_ROWS = 8;               // rows per FP16 tile
 constexpr int F16_ROW = D * 2;            // bytes of one FP16 K or V row
 constexpr int SLOT_F16V = F16_ROWS * F16_ROW;  // V rows of an FP16 tile start here
-constexpr int SLOT_KSZ = I4_TOK * ROW_BYTES;             // 2048
-constexpr int SLOT_VC = SLOT_KSZ + I4_TOK * SZ_BYTES;    // 2560
-constexpr int SLOT_VSZ = SLOT_VC + I4_TOK * ROW_BYTES;   // 4608
-constexpr int SLOT_MASK = SLOT_VSZ + I4_TOK * SZ_BYTES;  // 5120
-constexpr int SLOT_BYTES = SLOT_MASK + 32;               // 5152
+// An INT4 tile is one quantized-majority block of the cache, copied whole.
+constexpr int SLOT_KSZ = HYQ_BLK_KSZ;    // 2048
+constexpr int SLOT_VC = HYQ_BLK_VCODES;  // 2560
+constexpr int SLOT_VSZ = HYQ_BLK_VSZ;    // 4608
+constexpr int SLOT_MASK = HYQ_BLK_MASK;  // 5120
+constexpr int SLOT_BYTES = BLK_BYTES;    // 5136
 constexpr int PART_STRIDE = 132;  // floats per (partial, head): m, l, -, -, acc[128]
 constexpr float LOG2E_OVER_SQRT_D = 0.12751743082459868f;  // log2(e) / sqrt(128)
 constexpr float LN2 = 0.69314718055994531f;
@@ -56,6 +57,7 @@ static_assert(2 * F16_ROWS * F16_ROW <= SLOT_MASK, "fp16 tile fits a slot");
 // read, in KiB: an INT4 tile moves 32 x 160 B, an FP16 tile 8 x 512 B).
 constexpr int COST4 = 5, COST16 = 4;
 static_assert(SLOT_BYTES % 16 == 0, "slots stay 16-byte aligned");
+static_assert(I4_TOK == BLK_TOK, "an INT4 tile is one cache block");
 
 // ring slots per compute warp: 3 (2 when 8 query heads share a KV head, so
 // that two blocks still fit one SM's shared memory)
@@ -68,10 +70,9 @@ enum { MODE_HYBRID = 0, MODE_FP16 = 1 };
 
 struct DecodeArgs {
   int B, Hq, Hkv, cap, W, vl_cap, U, n_ctas;
-  const uint8_t *k_codes, *v_codes, *k_sz, *v_sz;
+  const uint8_t *blocks;  // quantized majority + bitmask, [U][cap/32][BLK_BYTES]
   const __half *win_k, *win_v, *vl_k, *vl_v;
   const int32_t *vl_count;
-  const uint32_t *vl_mask;
   const int32_t *seq_len;
   const __half *k16, *v16;  // comparator cache [B][Hkv][cap][128]
   const __half *q;
@@ -565,16 +566,8 @@ __device__ __forceinline__ void issue_tile(const DecodeArgs &a, const Smem &sm, 
   const UnitShape us = shape_of<MODE>(a, sm.unit_tv[u].x, sm.unit_tv[u].y, bad);
   if (lane != 0) return;
   if (MODE == MODE_HYBRID && j < us.n4) {
-    const int t0 = j * I4_TOK;
-    const int n = min(I4_TOK, us.L4 - t0);
-    const int64_t row = static_cast<int64_t>(u) * a.cap + t0;
-    mbar_arrive_expect_tx(bar, n * 160 + 16);
-    bulk_g2s(dst, a.k_codes + row * ROW_BYTES, n * ROW_BYTES, bar);
-    bulk_g2s(dst + SLOT_KSZ, a.k_sz + row * SZ_BYTES, n * SZ_BYTES, bar);
-    bulk_g2s(dst + SLOT_VC, a.v_codes + row * ROW_BYTES, n * ROW_BYTES, bar);
-    bulk_g2s(dst + SLOT_VSZ, a.v_sz + row * SZ_BYTES, n * SZ_BYTES, bar);
-    const uint32_t *mrow = a.vl_mask + static_cast<int64_t>(u) * (a.cap / 32);
-    bulk_g2s(dst + SLOT_MASK, mrow + ((t0 / 32) & ~3), 16, bar);
+    mbar_arrive_expect_tx(bar, BLK_BYTES);
+    bulk_g2s(dst, a.blocks + blk_base(u, static_cast<int64_t>(j) * I4_TOK, a.cap), BLK_BYTES, bar);
     return;
   }
   const __half *sk, *sv;
@@ -727,9 +720,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
       if (MODE == MODE_HYBRID && j < us.n4) {
         const int t0 = j * I4_TOK;
         const int n = min(I4_TOK, us.L4 - t0);
-        const uint4 mw = lds128(slot + SLOT_MASK);
-        const int wsel = (t0 / 32) & 3;
-        const uint32_t bits = wsel == 0 ? mw.x : wsel == 1 ? mw.y : wsel == 2 ? mw.z : mw.w;
+        uint32_t bits;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bits) : "r"(slot + SLOT_MASK));
         int4_tile(st, slot, n, bits, lane);
       } else {
         int n;
@@ -927,11 +919,10 @@ extern "C" hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, flo
   DecodeArgs a{};
   a.B = c->batch; a.Hq = c->n_q_heads; a.Hkv = c->n_kv_heads; a.cap = c->capacity;
   a.W = c->window; a.vl_cap = c->vl_capacity; a.U = U; a.n_ctas = N;
-  a.k_codes = c->k_codes; a.v_codes = c->v_codes;
-  a.k_sz = static_cast<const uint8_t *>(c->k_sz); a.v_sz = static_cast<const uint8_t *>(c->v_sz);
+  a.blocks = c->blocks;
   a.win_k = static_cast<const __half *>(c->win_k); a.win_v = static_cast<const __half *>(c->win_v);
   a.vl_k = static_cast<const __half *>(c->vl_k); a.vl_v = static_cast<const __half *>(c->vl_v);
-  a.vl_count = c->vl_count; a.vl_mask = c->vl_mask; a.seq_len = c->seq_len;
+  a.vl_count = c->vl_count; a.seq_len = c->seq_len;
   a.q = static_cast<const __half *>(q); a.o = static_cast<__half *>(o); a.lse = lse;
   a.counters = static_cast<int32_t *>(ws);
   a.part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + (static_cast<size_t>(U) * 4 + 255) / 256 * 256);
@@ -1019,11 +1010,10 @@ extern "C" hyq_status hyq_decode_noalloc(const hyq_cache *c, const void *q, void
   DecodeArgs a{};
   a.B = c->batch; a.Hq = c->n_q_heads; a.Hkv = c->n_kv_heads; a.cap = c->capacity;
   a.W = c->window; a.vl_cap = c->vl_capacity; a.U = U; a.n_ctas = N;
-  a.k_codes = c->k_codes; a.v_codes = c->v_codes;
-  a.k_sz = static_cast<const uint8_t *>(c->k_sz); a.v_sz = static_cast<const uint8_t *>(c->v_sz);
+  a.blocks = c->blocks;
   a.win_k = static_cast<const __half *>(c->win_k); a.win_v = static_cast<const __half *>(c->win_v);
   a.vl_k = static_cast<const __half *>(c->vl_k); a.vl_v = static_cast<const __half *>(c->vl_v);
-  a.vl_count = c->vl_count; a.vl_mask = c->vl_mask; a.seq_len = c->seq_len;
+  a.vl_count = c->vl_count; a.seq_len = c->seq_len;
   a.q = static_cast<const __half *>(q); a.o = static_cast<__half *>(o); a.lse = lse;
   a.counters = static_cast<int32_t *>(ws);
   a.part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + (static_cast<size_t>(U) * 4 + 255) / 256 * 256);

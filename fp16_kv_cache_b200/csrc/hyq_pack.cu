@@ -117,8 +117,8 @@ __global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half 
     if (p == 0 && t == 0 && !is_v && (u % c.n_kv_heads) == 0) set_status(c.dev_status, HYQ_DEV_BADLEN);
     return;
   }
-  // clear this unit's vertical-line set (bitmask words and count)
-  if (!is_v && t == 0 && p < c.capacity / 32) c.vl_mask[u * (c.capacity / 32) + p] = 0u;
+  // clear this unit's vertical-line set (block bitmask words and count)
+  if (!is_v && t == 0 && (p % BLK_TOK) == 0) *mask_word(c.blocks, u, p, c.capacity) = 0u;
   if (!is_v && t == 0 && p == 0) c.vl_count[u] = 0;
   if (p >= T) return;
   const __half *src = (is_v ? v_full : k_full) + up * D;
@@ -126,9 +126,9 @@ __global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half 
   const int W = c.window;
   if (p < T - W) {
     const unsigned hmask = 0xFFFFu << (lane & 16);
-    uint8_t *codes = is_v ? c.v_codes : c.k_codes;
-    uint32_t *sz = reinterpret_cast<uint32_t *>(is_v ? c.v_sz : c.k_sz);
-    quantize_part(xv, t, hmask, codes + up * ROW_BYTES, sz + up * (SZ_BYTES / 4), c.dev_status);
+    const int64_t co = is_v ? vcode_off(u, p, c.capacity) : kcode_off(u, p, c.capacity);
+    const int64_t so = is_v ? vsz_off(u, p, c.capacity) : ksz_off(u, p, c.capacity);
+    quantize_part(xv, t, hmask, c.blocks + co, reinterpret_cast<uint32_t *>(c.blocks + so), c.dev_status);
   } else {
     __half *win = reinterpret_cast<__half *>(is_v ? c.win_v : c.win_k) + (u * W + p % W) * D;
     *reinterpret_cast<uint4 *>(win + 8 * t) = xv;
@@ -160,10 +160,10 @@ __global__ void append_kernel(hyq_cache c, const __half *__restrict__ k_new,
     if (T >= W) {
       const unsigned hmask = 0xFFFFu << (lane & 16);
       const uint4 old = *reinterpret_cast<const uint4 *>(win + 8 * t);
-      const int64_t dst = u * c.capacity + (T - W);
-      uint8_t *codes = is_v ? c.v_codes : c.k_codes;
-      uint32_t *sz = reinterpret_cast<uint32_t *>(is_v ? c.v_sz : c.k_sz);
-      quantize_part(old, t, hmask, codes + dst * ROW_BYTES, sz + dst * (SZ_BYTES / 4), c.dev_status);
+      const int64_t p = T - W;
+      const int64_t co = is_v ? vcode_off(u, p, c.capacity) : kcode_off(u, p, c.capacity);
+      const int64_t so = is_v ? vsz_off(u, p, c.capacity) : ksz_off(u, p, c.capacity);
+      quantize_part(old, t, hmask, c.blocks + co, reinterpret_cast<uint32_t *>(c.blocks + so), c.dev_status);
     }
     const __half *src = (is_v ? v_new : k_new) + u * D;
     *reinterpret_cast<uint4 *>(win + 8 * t) = *reinterpret_cast<const uint4 *>(src + 8 * t);
@@ -208,8 +208,8 @@ __global__ void __launch_bounds__(256) vl_reset_kernel(hyq_cache c, const int32_
     const int p = np[i];
     if (p < 0 || p >= L4 || (i > 0 && np[i - 1] >= p)) s_bad = 1;
   }
-  uint32_t *mask = c.vl_mask + static_cast<int64_t>(u) * (c.capacity / 32);
-  for (int w = threadIdx.x; w < c.capacity / 32; w += blockDim.x) mask[w] = 0u;
+  for (int w = threadIdx.x; w < c.capacity / BLK_TOK; w += blockDim.x)
+    *mask_word(c.blocks, u, static_cast<int64_t>(w) * BLK_TOK, c.capacity) = 0u;
   __syncthreads();
   if (threadIdx.x == 0) {
     if (s_bad) set_status(c.dev_status, HYQ_DEV_BADLEN);
@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(512) vl_gather_kernel(hyq_cache c, const int32
   *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.vl_k) + d) = *reinterpret_cast<const uint4 *>(k_full + so);
   *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.vl_v) + d) = *reinterpret_cast<const uint4 *>(v_full + so);
   if (part == 0) {
-    atomicOr(&c.vl_mask[static_cast<int64_t>(u) * (c.capacity / 32) + (p >> 5)], 1u << (p & 31));
+    atomicOr(mask_word(c.blocks, u, p, c.capacity), 1u << (p & 31));
     c.vl_pos[static_cast<int64_t>(u) * c.vl_capacity + r] = p;
   }
 }
@@ -253,7 +253,6 @@ __global__ void __launch_bounds__(1024) vl_recompact_kernel(hyq_cache c, const i
   const int32_t *np = pos + static_cast<int64_t>(u) * k;
   int32_t *old = c.vl_pos + static_cast<int64_t>(u) * c.vl_capacity;
   const int old_n = c.vl_count[u];
-  uint32_t *mask = c.vl_mask + static_cast<int64_t>(u) * (c.capacity / 32);
   if (threadIdx.x == 0) s_bad = (old_n < 0 || old_n > c.vl_capacity);
   __syncthreads();
   for (int i = threadIdx.x; i < k; i += blockDim.x) {
@@ -295,7 +294,8 @@ __global__ void __launch_bounds__(1024) vl_recompact_kernel(hyq_cache c, const i
   // dropped old positions fall back to their codes
   for (int j = threadIdx.x; j < old_n; j += blockDim.x) {
     const int p = old[j];
-    if (p >= 0 && p < c.capacity && find_sorted(np, k, p) < 0) atomicAnd(&mask[p >> 5], ~(1u << (p & 31)));
+    if (p >= 0 && p < c.capacity && find_sorted(np, k, p) < 0)
+      atomicAnd(mask_word(c.blocks, u, p, c.capacity), ~(1u << (p & 31)));
   }
   __syncthreads();
   const int rows = blockDim.x / 16;

@@ -49,10 +49,9 @@ struct SelectArgs {
   int B, Hq, Hkv, G, n_q, q_ring, cap, W, vl_cap, U, R, k, n_chunks;
   const __half *q;       // [B][Hq][n_q][128]
   const __half *k_full;  // nullable [B][Hkv][cap][128]
-  const uint8_t *k_codes, *k_sz;
+  const uint8_t *blocks;  // quantized majority + bitmask, [U][cap/32][BLK_BYTES]
   const __half *win_k, *vl_k;
   const int32_t *vl_pos, *vl_count;
-  const uint32_t *vl_mask;
   const int32_t *seq_len;
   float2 *stats_part;  // [U][n_chunks][SEL_MAX_ROWS]
   float2 *stats;       // [U][SEL_MAX_ROWS]  (m, 1/l)
@@ -137,10 +136,9 @@ __device__ __forceinline__ void issue_cache(const SelectArgs &a, int u, int T, i
       continue;
     }
     // channels 8c..8c+7: group c / 4, pieces 2(c%4) and 2(c%4)+1
-    const int64_t row = static_cast<int64_t>(u) * a.cap + key;
     r.kind[j] = -2;
-    r.v[j] = *reinterpret_cast<const uint4 *>(a.k_codes + row * ROW_BYTES + 16 * (c & 3));
-    r.sz[j] = *reinterpret_cast<const uint32_t *>(a.k_sz + row * SZ_BYTES + 4 * (c >> 2));
+    r.v[j] = *reinterpret_cast<const uint4 *>(a.blocks + kcode_off(u, key, a.cap) + 16 * (c & 3));
+    r.sz[j] = *reinterpret_cast<const uint32_t *>(a.blocks + ksz_off(u, key, a.cap) + 4 * (c >> 2));
   }
 }
 
@@ -299,13 +297,12 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) score_kernel(const SelectArgs 
     RawItems raw;
     if (CACHE) {
       // vertical-line slot of every key of the chunk: rank of its mask bit
-      const uint32_t *mrow = a.vl_mask + static_cast<int64_t>(u) * (a.cap / 32);
       const int32_t *rbase = a.rank_base + static_cast<int64_t>(u) * (a.cap / 32);
       for (int j = threadIdx.x; j < SEL_KC; j += blockDim.x) {
         const int key = k0 + j;
         int slot = -1;
         if (key < k1 && key < T - a.W) {
-          const uint32_t w = mrow[key >> 5];
+          const uint32_t w = *reinterpret_cast<const uint32_t *>(a.blocks + blk_base(u, key, a.cap) + HYQ_BLK_MASK);
           if ((w >> (key & 31)) & 1u) slot = rbase[key >> 5] + __popc(w & ((1u << (key & 31)) - 1u));
         }
         slot_of[j] = slot;
@@ -437,13 +434,14 @@ __global__ void __launch_bounds__(1024) rank_kernel(const SelectArgs a) {
   __shared__ int wsum[32];
   const int u = blockIdx.x;
   const int nw = a.cap / 32;
-  const uint32_t *mrow = a.vl_mask + static_cast<int64_t>(u) * nw;
   int32_t *out = a.rank_base + static_cast<int64_t>(u) * nw;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   int carry = 0;
   for (int base = 0; base < nw; base += blockDim.x) {
     const int i = base + threadIdx.x;
-    const int v = (i < nw) ? __popc(mrow[i]) : 0;
+    const int v = (i < nw) ? __popc(*reinterpret_cast<const uint32_t *>(
+                                 a.blocks + blk_base(u, static_cast<int64_t>(i) * 32, a.cap) + HYQ_BLK_MASK))
+                           : 0;
     int x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -658,9 +656,9 @@ extern "C" hyq_status hyq_select_vl(const hyq_cache *c, const void *q_sel, int32
   a.n_chunks = (c->capacity + SEL_KC - 1) / SEL_KC;
   a.q = static_cast<const __half *>(q_sel);
   a.k_full = static_cast<const __half *>(k_full);
-  a.k_codes = c->k_codes; a.k_sz = static_cast<const uint8_t *>(c->k_sz);
+  a.blocks = c->blocks;
   a.win_k = static_cast<const __half *>(c->win_k); a.vl_k = static_cast<const __half *>(c->vl_k);
-  a.vl_pos = c->vl_pos; a.vl_count = c->vl_count; a.vl_mask = c->vl_mask; a.seq_len = c->seq_len;
+  a.vl_pos = c->vl_pos; a.vl_count = c->vl_count; a.seq_len = c->seq_len;
   uint8_t *w = static_cast<uint8_t *>(ws);
   const size_t U = a.U;
   a.stats_part = reinterpret_cast<float2 *>(w);

@@ -18,6 +18,9 @@ HEAD_DIM = 128
 GROUP = 32
 WINDOW = 128
 ROW_BYTES = 64
+BLOCK_TOKENS = 32
+BLOCK_BYTES = 5136
+BLK_KCODES, BLK_KSZ, BLK_VCODES, BLK_VSZ, BLK_MASK = 0, 2048, 2560, 4608, 5120
 
 DEV_NONFINITE = 0x1
 DEV_OOB = 0x2
@@ -41,12 +44,11 @@ class hyq_cache(ctypes.Structure):
         ("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
         ("head_dim", ctypes.c_int32), ("group", ctypes.c_int32), ("window", ctypes.c_int32),
         ("capacity", ctypes.c_int32), ("vl_capacity", ctypes.c_int32),
-        ("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
-        ("k_sz", ctypes.c_void_p), ("v_sz", ctypes.c_void_p),
+        ("blocks", ctypes.c_void_p),
         ("win_k", ctypes.c_void_p), ("win_v", ctypes.c_void_p),
         ("vl_k", ctypes.c_void_p), ("vl_v", ctypes.c_void_p),
         ("vl_pos", ctypes.c_void_p), ("vl_count", ctypes.c_void_p),
-        ("vl_mask", ctypes.c_void_p), ("seq_len", ctypes.c_void_p),
+        ("seq_len", ctypes.c_void_p),
         ("dev_status", ctypes.c_void_p),
     ]
 
@@ -124,25 +126,21 @@ class HybridCache:
         dev = torch.device(device)
         z = lambda *s, dt: torch.zeros(*s, dtype=dt, device=dev)  # noqa: E731
         self.B, self.Hq, self.Hkv, self.cap, self.vl_cap = B, n_q_heads, Hkv, capacity, vl_capacity
-        self.k_codes = z(B, Hkv, capacity, ROW_BYTES, dt=torch.uint8)
-        self.v_codes = z(B, Hkv, capacity, ROW_BYTES, dt=torch.uint8)
-        self.k_sz = z(B, Hkv, capacity, 8, dt=torch.float16)
-        self.v_sz = z(B, Hkv, capacity, 8, dt=torch.float16)
+        self.blocks = z(B, Hkv, capacity // BLOCK_TOKENS, BLOCK_BYTES, dt=torch.uint8)
         self.win_k = z(B, Hkv, WINDOW, HEAD_DIM, dt=torch.float16)
         self.win_v = z(B, Hkv, WINDOW, HEAD_DIM, dt=torch.float16)
         self.vl_k = z(B, Hkv, vl_capacity, HEAD_DIM, dt=torch.float16)
         self.vl_v = z(B, Hkv, vl_capacity, HEAD_DIM, dt=torch.float16)
         self.vl_pos = z(B, Hkv, vl_capacity, dt=torch.int32)
         self.vl_count = z(B, Hkv, dt=torch.int32)
-        self.vl_mask = z(B, Hkv, capacity // 32, dt=torch.int32)  # bit pattern of uint32 words
         self.seq_len = z(B, dt=torch.int32)
         self.dev_status = z(4, dt=torch.int32)
         c = hyq_cache()
         c.batch, c.n_q_heads, c.n_kv_heads = B, n_q_heads, Hkv
         c.head_dim, c.group, c.window = HEAD_DIM, GROUP, WINDOW
         c.capacity, c.vl_capacity = capacity, vl_capacity
-        for name in ("k_codes", "v_codes", "k_sz", "v_sz", "win_k", "win_v", "vl_k", "vl_v",
-                     "vl_pos", "vl_count", "vl_mask", "seq_len", "dev_status"):
+        for name in ("blocks", "win_k", "win_v", "vl_k", "vl_v", "vl_pos", "vl_count", "seq_len",
+                     "dev_status"):
             setattr(c, name, getattr(self, name).data_ptr())
         self.desc = c
 
@@ -157,8 +155,24 @@ class HybridCache:
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in (
-            self.k_codes, self.v_codes, self.k_sz, self.v_sz, self.win_k, self.win_v,
-            self.vl_k, self.vl_v, self.vl_pos, self.vl_count, self.vl_mask, self.seq_len))
+            self.blocks, self.win_k, self.win_v, self.vl_k, self.vl_v, self.vl_pos, self.vl_count,
+            self.seq_len))
+
+    def unpack_blocks(self):
+        """Host views of the block records as per-position rows: (k_codes
+        [B][Hkv][cap][64] u8, k_sz [B][Hkv][cap][8] u16, v_codes, v_sz,
+        mask [B][Hkv][cap/32] u32).  A copy; for inspection and tests."""
+        b = self.blocks.cpu().numpy()
+        B, H, nb, _ = b.shape
+        cap = nb * BLOCK_TOKENS
+        def field(off, width):
+            return b[..., off:off + BLOCK_TOKENS * width].reshape(B, H, cap, width)
+        kc = field(BLK_KCODES, ROW_BYTES)
+        ks = field(BLK_KSZ, 16).copy().view("<u2")
+        vc = field(BLK_VCODES, ROW_BYTES)
+        vs = field(BLK_VSZ, 16).copy().view("<u2")
+        mask = b[..., BLK_MASK:BLK_MASK + 4].copy().view("<u4").reshape(B, H, nb)
+        return kc, ks, vc, vs, mask
 
 
 # ------------------------------------------------------------------ entry points

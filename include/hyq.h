@@ -84,16 +84,35 @@ typedef enum {
  */
 
 /*
+ * Quantized-majority blocks.  The INT4 part of a unit is stored in blocks of
+ * 32 consecutive positions, each one contiguous HYQ_BLOCK_BYTES record, so a
+ * decode tile is a single bulk copy:
+ *   offset    0: K codes   [32][64]  (packed rows, format above)
+ *   offset 2048: K scale/zero [32][8] fp16
+ *   offset 2560: V codes   [32][64]
+ *   offset 4608: V scale/zero [32][8] fp16
+ *   offset 5120: uint32 vertical-line bitmask: bit i set exactly when
+ *                position 32*b + i is held in FP16 in the vertical-line rows
+ *   offset 5124: 12 bytes of padding (keeps records 16-byte aligned)
+ */
+#define HYQ_BLOCK_TOKENS 32
+#define HYQ_BLOCK_BYTES 5136
+#define HYQ_BLK_KCODES 0
+#define HYQ_BLK_KSZ 2048
+#define HYQ_BLK_VCODES 2560
+#define HYQ_BLK_VSZ 4608
+#define HYQ_BLK_MASK 5120
+
+/*
  * The hybrid cache of one layer.  All arrays are caller-owned device memory
  * and must be zero-filled before first use.  Per unit u = b * n_kv_heads + h:
- *   quantized majority  positions [0, T - window):  k_codes/v_codes
- *                       [B][Hkv][capacity][64] u8, k_sz/v_sz
- *                       [B][Hkv][capacity][8] fp16;
+ *   quantized majority  positions [0, T - window): blocks
+ *                       [B][Hkv][capacity/32][HYQ_BLOCK_BYTES], position p
+ *                       in block p / 32, slot p % 32;
  *   vertical-line rows  vl_k/vl_v [B][Hkv][vl_capacity][128] fp16, in the
  *                       ascending order of vl_pos [B][Hkv][vl_capacity];
- *                       vl_count [B][Hkv] rows are valid; vl_mask
- *                       [B][Hkv][capacity/32] u32 has bit p%32 of word p/32
- *                       set exactly for the positions held in vl_k/vl_v;
+ *                       vl_count [B][Hkv] rows are valid, and the block
+ *                       bitmasks mark exactly these positions;
  *   local window        win_k/win_v [B][Hkv][window][128] fp16, position p
  *                       in slot p % window, positions [max(0, T-window), T);
  *   seq_len [B] int32   T, the number of positions, newest token included.
@@ -103,22 +122,20 @@ typedef struct {
   int32_t head_dim;    /* must be 128 */
   int32_t group;       /* must be 32  */
   int32_t window;      /* must be 128 */
-  int32_t capacity;    /* max positions per sequence, multiple of 64 */
+  int32_t capacity;    /* max positions per sequence, multiple of 128 */
   int32_t vl_capacity; /* max vertical-line rows per unit, >= 1 */
-  uint8_t *k_codes, *v_codes;
-  void *k_sz, *v_sz;
+  uint8_t *blocks;
   void *win_k, *win_v;
   void *vl_k, *vl_v;
   int32_t *vl_pos;
   int32_t *vl_count;
-  uint32_t *vl_mask;
   int32_t *seq_len;
   uint32_t *dev_status; /* nullable */
 } hyq_cache;
 
 /*
  * hyq_pack -- quantize FP16 rows to packed INT4 codes and fp16 scale/zero
- * (the KV-cache compression of the decode stage).
+ * (the KV-cache compression of the decode stage), into plain row arrays.
  *   x          fp16 rows, row i at x + i*row_stride (elements), 128 values
  *   n_rows     >= 0 (0 enqueues nothing)
  *   row_stride >= 128, multiple of 8
@@ -134,9 +151,9 @@ hyq_status hyq_pack(const void *x, int64_t n_rows, int64_t row_stride,
 /*
  * hyq_prefill -- build the cache from a prompt (end of prefill).  For every
  * unit with T = seq_len[b] (device): rows [0, T - window) of k_full/v_full
- * are quantized into the codes (as hyq_pack), rows [max(0, T - window), T)
+ * are quantized into the blocks (as hyq_pack), rows [max(0, T - window), T)
  * are copied into the window ring, and the vertical-line set is emptied
- * (vl_count = 0, vl_mask cleared).
+ * (vl_count = 0, every block bitmask cleared).
  *   k_full, v_full  fp16 [B][Hkv][capacity][128]
  * Sets HYQ_DEV_BADLEN (and skips the batch) when T is outside [0, capacity];
  * HYQ_DEV_NONFINITE as hyq_pack.

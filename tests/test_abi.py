@@ -49,8 +49,7 @@ def _desc(**over):
     c.batch, c.n_q_heads, c.n_kv_heads = 1, 8, 2
     c.head_dim, c.group, c.window, c.capacity, c.vl_capacity = 128, 32, 128, 4096, 64
     fake = 0x10000  # aligned, never dereferenced: validation fails or stops first
-    for name in ("k_codes", "v_codes", "k_sz", "v_sz", "win_k", "win_v", "vl_k", "vl_v",
-                 "vl_pos", "vl_count", "vl_mask", "seq_len"):
+    for name in ("blocks", "win_k", "win_v", "vl_k", "vl_v", "vl_pos", "vl_count", "seq_len"):
         setattr(c, name, fake)
         fake += 0x10000
     for k, v in over.items():
@@ -61,7 +60,7 @@ def _desc(**over):
 @pytest.mark.parametrize("field,value,code", [
     ("head_dim", 64, 2), ("group", 64, 2), ("window", 256, 2), ("n_q_heads", 7, 1), ("n_q_heads", 6, 2),
     ("n_q_heads", 24, 2), ("capacity", 4000, 1), ("capacity", 0, 1), ("vl_capacity", 0, 1),
-    ("batch", 0, 1), ("k_codes", 0, 1), ("vl_mask", 0x10008, 3), ("seq_len", None, 1),
+    ("batch", 0, 1), ("blocks", 0, 1), ("vl_pos", 0x10008, 3), ("seq_len", None, 1),
 ])
 def test_decode_rejects_bad_descriptors(L, field, value, code):
     c = _desc(**{field: value})

@@ -88,16 +88,15 @@ def _assert_cache_equal(case, units=None):
     units = range(U) if units is None else units
     T = cfg.T
     n_old = max(0, T - cfg.W)
-    kc = host(g.k_codes).reshape(U, case.cap, 64)
-    vc = host(g.v_codes).reshape(U, case.cap, 64)
-    ks = host(g.k_sz).view(np.uint16).reshape(U, case.cap, 8)
-    vs = host(g.v_sz).view(np.uint16).reshape(U, case.cap, 8)
+    kc, ks, vc, vs, mask = g.unpack_blocks()
+    kc, vc = kc.reshape(U, case.cap, 64), vc.reshape(U, case.cap, 64)
+    ks, vs = ks.reshape(U, case.cap, 8), vs.reshape(U, case.cap, 8)
+    mask = mask.reshape(U, case.cap // 32)
     wk = host(g.win_k).view(np.uint16).reshape(U, 128, 128)
     wv = host(g.win_v).view(np.uint16).reshape(U, 128, 128)
     vlk = host(g.vl_k).view(np.uint16).reshape(U, case.vl_cap, 128)
     vpos = host(g.vl_pos).reshape(U, case.vl_cap)
     vcnt = host(g.vl_count).reshape(U)
-    mask = host(g.vl_mask).view(np.uint32).reshape(U, case.cap // 32)
     nw = min(T, cfg.W)
     for u in units:
         assert np.array_equal(kc[u, :n_old], o.k_codes[u, :n_old])
