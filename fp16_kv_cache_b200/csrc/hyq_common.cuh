@@ -2,8 +2,8 @@
 //
 // Inline PTX wrappers for the asynchronous bulk-copy engine (cp.async.bulk +
 // mbarrier transaction counts), warp-level tensor-core MMA, the 8x8 b16
-// register transpose, and the nibble -> fp16 conversion used to feed packed
-// INT4 codes to the tensor cores without a trip through shared memory.
+// register transpose, and the nibble -> fp16 subnormal view used to feed
+// packed INT4 codes to the tensor cores.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -196,18 +196,14 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
 
-// Nibbles in bits 0-3 and 16-19 of w -> half2 holding those two integers.
-// An fp16 with exponent field 25 (bits 0x6400) and a 4-bit fraction n is
-// exactly 1024 + n; subtracting 1024 leaves n exactly.
-__device__ __forceinline__ uint32_t nib_lo(uint32_t w) {
-  uint32_t x = lop3_and_or(w, 0x000F000Fu, 0x64006400u);
-  return h2u(__hsub2(u2h(x), u2h(0x64006400u)));
-}
-// Nibbles in bits 4-7 and 20-23: the half is 1024 + 16 n; n = x / 16 - 64.
-__device__ __forceinline__ uint32_t nib_hi(uint32_t w) {
-  uint32_t x = lop3_and_or(w, 0x00F000F0u, 0x64006400u);
-  return h2u(__hfma2(u2h(x), u2h(0x2C002C00u) /* 1/16 */, u2h(0xD400D400u) /* -64 */));
-}
+// Nibbles in bits 0-3 / 4-7 and 16-19 / 20-23 of w as a half2 of fp16
+// subnormals, one AND each: a half whose exponent field is zero and whose
+// fraction is f has the value f * 2^-24 exactly (IEEE 754 binary16), so
+// bits 0-3 give n * 2^-24 and bits 4-7 give 16 n * 2^-24.  The tensor core
+// multiplies these exactly; the caller undoes the power-of-two factors in
+// fp32.
+__device__ __forceinline__ uint32_t code_lo(uint32_t w) { return w & 0x000F000Fu; }
+__device__ __forceinline__ uint32_t code_hi(uint32_t w) { return w & 0x00F000F0u; }
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;

@@ -36,7 +36,7 @@
 
 namespace hyq {
 
-constexpr int NCW = 6;                    // compute warps per block, each fed by itself
+constexpr int NCW = 12;                   // compute warps per block (one block per SM), each fed by itself
 constexpr int NTHREADS = NCW * 32;
 constexpr int I4_TOK = 32;                // tokens per INT4 tile
 constexpr int F16_ROWS = 8;               // rows per FP16 tile
@@ -50,6 +50,7 @@ constexpr int SLOT_MASK = HYQ_BLK_MASK;  // 5120
 constexpr int SLOT_BYTES = BLK_BYTES;    // 5136
 constexpr int PART_STRIDE = 132;  // floats per (partial, head): m, l, -, -, acc[128]
 constexpr float LOG2E_OVER_SQRT_D = 0.12751743082459868f;  // log2(e) / sqrt(128)
+constexpr float TWO24 = 16777216.f, TWO20 = 1048576.f, TWO_M24 = 1.f / 16777216.f;
 constexpr float LN2 = 0.69314718055994531f;
 
 static_assert(2 * F16_ROWS * F16_ROW <= SLOT_MASK, "fp16 tile fits a slot");
@@ -59,11 +60,13 @@ constexpr int COST4 = 5, COST16 = 4;
 static_assert(SLOT_BYTES % 16 == 0, "slots stay 16-byte aligned");
 static_assert(I4_TOK == BLK_TOK, "an INT4 tile is one cache block");
 
-// ring slots per compute warp: 3 (2 when 8 query heads share a KV head, so
-// that two blocks still fit one SM's shared memory)
+// Ring slots per compute warp: 2 (one being read, one in flight), so one
+// SM holds 24 tiles in flight, about 120 KB, enough to cover the memory
+// latency at full bandwidth while leaving shared memory for the merge
+// buffers and per-unit tables of up to 4096 units.
 template <int G>
 struct Ring {
-  static constexpr int SPW = (G == 8) ? 2 : 3;
+  static constexpr int SPW = 2;
 };
 
 enum { MODE_HYBRID = 0, MODE_FP16 = 1 };
@@ -135,21 +138,45 @@ __device__ __forceinline__ UnitShape unit_shape_global(const DecodeArgs &a, int 
 
 // Per-warp running state, in the accumulator layout of m16n8: lane (r, q)
 // holds query heads 2q and 2q+1 of the unit (heads >= G are padding).
+//
+// INT4 codes enter the MMAs as fp16 subnormals (code_lo / code_hi), so
+// while a warp sweeps INT4 tiles its accumulator rows carry power-of-two
+// factors: rows r (elements 0, 1) hold 2^-24 O and rows r + 8 (elements 2,
+// 3) hold 2^-20 O.  unscale_acc removes them before FP16 rows are added and
+// before the state leaves the warp.
+//
+// The zero-point terms are MMAs too.  Keys: sum_g zero_g * qsum_g, with
+// A = the token rows' four zeros (the same pair in every lane of a row) and
+// B = qz, the per-group sums of q split into fp16 hi + lo parts (k rows 0-3
+// and 8-11; the rest zero).  Values: zacc = Vzero^T P, groups on M (lane
+// row r < 4 holds group r), heads on N.
 struct WarpState {
   float m[2], l[2];
-  float zs[2][NG];         // sum over tokens of p * vzero, per (head, group)
+  float zacc[2];           // sum over tokens of p * vzero: group r, heads 2q, 2q+1
   float acc[NG][2][4];     // O^T accumulators: m-tile (group g, half j)
-  uint32_t qf[NG][2][2];   // Q as the B operand: k-step (group g, piece s)
-  float qs[2][NG];         // sum of q over each group (heads 2q, 2q+1)
+  uint32_t qf[NG][2][2];   // Q as the B operand: k-step (group g, piece s);
+                           // piece [.][.][1] (high-nibble channels) is q / 16
+  uint32_t qz[2];          // B operand of the key zero term
 };
+
+__device__ __forceinline__ void unscale_acc(WarpState &st) {
+#pragma unroll
+  for (int g = 0; g < NG; ++g)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      st.acc[g][j][0] *= TWO24;
+      st.acc[g][j][1] *= TWO24;
+      st.acc[g][j][2] *= TWO20;
+      st.acc[g][j][3] *= TWO20;
+    }
+}
 
 __device__ __forceinline__ void state_reset(WarpState &st) {
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     st.m[e] = -INFINITY;
     st.l[e] = 0.f;
-#pragma unroll
-    for (int g = 0; g < NG; ++g) st.zs[e][g] = 0.f;
+    st.zacc[e] = 0.f;
   }
 #pragma unroll
   for (int g = 0; g < NG; ++g)
@@ -162,11 +189,14 @@ __device__ __forceinline__ void state_reset(WarpState &st) {
 // Query fragments of unit u.  Channel order inside a k-step matches the
 // packed INT4 row: k-step (g, s) lane q carries channels
 // 32g + 8q + 4s + {0, 2} (slots 2q, 2q+1) and {1, 3} (slots 2q+8, 2q+9).
+// The odd channels meet high nibbles (16 x the code as a subnormal), so
+// their q is stored divided by 16: exact for |q| >= 2^-10, and off by at
+// most 2^-25 below that.
 template <int G>
 __device__ __forceinline__ void load_q(WarpState &st, const DecodeArgs &a, int u, int lane) {
   const int n = lane >> 2, q4 = lane & 3;
   const int b = u / a.Hkv, kvh = u % a.Hkv;
-  float part[NG];
+  __half hi[NG], lo[NG];
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
     uint4 x = make_uint4(0, 0, 0, 0);
@@ -177,6 +207,8 @@ __device__ __forceinline__ void load_q(WarpState &st, const DecodeArgs &a, int u
     st.qf[g][0][1] = prmt(x.x, x.y, 0x7632u);
     st.qf[g][1][0] = prmt(x.z, x.w, 0x5410u);
     st.qf[g][1][1] = prmt(x.z, x.w, 0x7632u);
+    st.qf[g][0][1] = h2u(__hmul2(u2h(st.qf[g][0][1]), u2h(0x2C002C00u)));  // x 1/16
+    st.qf[g][1][1] = h2u(__hmul2(u2h(st.qf[g][1][1]), u2h(0x2C002C00u)));
     float s = 0.f;
     const __half2 *h = reinterpret_cast<const __half2 *>(&x);
 #pragma unroll
@@ -186,13 +218,16 @@ __device__ __forceinline__ void load_q(WarpState &st, const DecodeArgs &a, int u
     }
     s += __shfl_xor_sync(0xffffffffu, s, 1);
     s += __shfl_xor_sync(0xffffffffu, s, 2);
-    part[g] = s;  // lanes 4n..4n+3 hold head n
+    // lanes 4n..4n+3 hold head n's group sum; keep it as hi + lo fp16
+    // (relative error 2^-22)
+    hi[g] = __float2half_rn(s);
+    lo[g] = __float2half_rn(s - __half2float(hi[g]));
   }
-#pragma unroll
-  for (int g = 0; g < NG; ++g) {
-    st.qs[0][g] = __shfl_sync(0xffffffffu, part[g], (2 * q4) * 4);
-    st.qs[1][g] = __shfl_sync(0xffffffffu, part[g], (2 * q4 + 1) * 4);
-  }
+  // B fragment rows k = 2q, 2q+1 (and 8 + 2q, 9 + 2q) of column n = head:
+  // lane q = 0 carries the hi parts of groups (0, 1) / (2, 3), lane q = 1
+  // the lo parts, lanes 2 and 3 zeros.
+  st.qz[0] = (q4 == 0) ? h2u(__halves2half2(hi[0], hi[1])) : (q4 == 1) ? h2u(__halves2half2(lo[0], lo[1])) : 0u;
+  st.qz[1] = (q4 == 0) ? h2u(__halves2half2(hi[2], hi[3])) : (q4 == 1) ? h2u(__halves2half2(lo[2], lo[3])) : 0u;
 }
 
 // Running-max update: when any lane sees a larger score for head 2q or
@@ -213,10 +248,10 @@ __device__ __forceinline__ void rescale_if_needed(WarpState &st, float mx0, floa
     st.m[1] = n1;
     st.l[0] *= a0;
     st.l[1] *= a1;
+    st.zacc[0] *= a0;
+    st.zacc[1] *= a1;
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
-      st.zs[0][g] *= a0;
-      st.zs[1][g] *= a1;
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         st.acc[g][j][0] *= a0;
@@ -245,9 +280,10 @@ __device__ __forceinline__ void softmax_step(WarpState &st, float (&S)[4], bool 
 // two 16-token MMA row blocks give independent work to overlap: Q.K of both
 // blocks, one online-softmax update over the 32 tokens, then P.V.
 // Invalid tokens (past the tile end, or held in the vertical-line segment)
-// get S = -inf and p = 0.  Their scale/zero bytes in shared memory are stale
-// but finite (the ring is zero-filled at start and only ever holds fp16
-// data), so p * scale stays 0 without a select.
+// get S = -inf and p = 0.  Their codes and scale/zero rows come with the
+// rest of the block record, which holds zeros or earlier quantizer output
+// (the cache starts zero-filled), so p * scale and p * zero stay 0 without
+// a select.
 __device__ __forceinline__ void int4_tile(WarpState &st, uint32_t slot, int n_valid, uint32_t vlbits,
                                           int lane) {
   const int r = lane >> 2, q4 = lane & 3;
@@ -271,26 +307,33 @@ __device__ __forceinline__ void int4_tile(WarpState &st, uint32_t slot, int n_va
       const uint4 kb = lds128(kc + tB * ROW_BYTES + 16 * q4);
       const uint4 za = lds128(ksz + tA * SZ_BYTES), zb = lds128(ksz + tB * SZ_BYTES);
       const uint32_t zaw[4] = {za.x, za.y, za.z, za.w}, zbw[4] = {zb.x, zb.y, zb.z, zb.w};
+      // zero term: A row = (zero_0, zero_1 | zero_2, zero_3) of the row's token
+      mma16816(S[mt], prmt(za.x, za.y, 0x7632u), prmt(zb.x, zb.y, 0x7632u), prmt(za.z, za.w, 0x7632u),
+               prmt(zb.z, zb.w, 0x7632u), st.qz[0], st.qz[1]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) S[mt][e] *= TWO_M24;
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
         const uint32_t w0a = (g < 2) ? ka.x : ka.y, w1a = (g < 2) ? ka.z : ka.w;
         const uint32_t w0b = (g < 2) ? kb.x : kb.y, w1b = (g < 2) ? kb.z : kb.w;
         const int sh = (g & 1) ? 8 : 0;
         float sg[4] = {0.f, 0.f, 0.f, 0.f};
-        mma16816(sg, nib_lo(w0a >> sh), nib_lo(w0b >> sh), nib_hi(w0a >> sh), nib_hi(w0b >> sh),
+        // sg = 2^-24 (q . code): low nibbles n 2^-24 against q, high
+        // nibbles 16 n 2^-24 against q / 16
+        mma16816(sg, code_lo(w0a >> sh), code_lo(w0b >> sh), code_hi(w0a >> sh), code_hi(w0b >> sh),
                  st.qf[g][0][0], st.qf[g][0][1]);
-        mma16816(sg, nib_lo(w1a >> sh), nib_lo(w1b >> sh), nib_hi(w1a >> sh), nib_hi(w1b >> sh),
+        mma16816(sg, code_lo(w1a >> sh), code_lo(w1b >> sh), code_hi(w1a >> sh), code_hi(w1b >> sh),
                  st.qf[g][1][0], st.qf[g][1][1]);
-        const float2 fa = __half22float2(u2h(zaw[g]));  // (scale, zero) of row A
-        const float2 fb = __half22float2(u2h(zbw[g]));
-        S[mt][0] += fa.x * sg[0] + fa.y * st.qs[0][g];
-        S[mt][1] += fa.x * sg[1] + fa.y * st.qs[1][g];
-        S[mt][2] += fb.x * sg[2] + fb.y * st.qs[0][g];
-        S[mt][3] += fb.x * sg[3] + fb.y * st.qs[1][g];
+        const float sa = __low2float(u2h(zaw[g]));  // scales of rows A and B
+        const float sb = __low2float(u2h(zbw[g]));
+        S[mt][0] += sa * sg[0];
+        S[mt][1] += sa * sg[1];
+        S[mt][2] += sb * sg[2];
+        S[mt][3] += sb * sg[3];
       }
     }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) S[mt][e] *= LOG2E_OVER_SQRT_D;
+    for (int e = 0; e < 4; ++e) S[mt][e] *= LOG2E_OVER_SQRT_D * TWO24;
     if (!vA[mt]) S[mt][0] = S[mt][1] = -INFINITY;
     if (!vB[mt]) S[mt][2] = S[mt][3] = -INFINITY;
   }
@@ -323,15 +366,28 @@ __device__ __forceinline__ void int4_tile(WarpState &st, uint32_t slot, int n_va
     const int tA = 16 * mt + sig(r), tB = tA + 8;
     const uint4 wa = lds128(vsz + tA * SZ_BYTES), wb = lds128(vsz + tB * SZ_BYTES);
     const uint32_t waw[4] = {wa.x, wa.y, wa.z, wa.w}, wbw[4] = {wb.x, wb.y, wb.z, wb.w};
+    {
+      // zero term: A = Vzero^T (group r&3 of the tokens of k rows 2q, 2q+1,
+      // 8 + 2q, 9 + 2q), B = P^T unscaled
+      const uint32_t zrow = vsz + 4 * (r & 3);
+      uint32_t z0, z1, z2, z3;
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(z0) : "r"(zrow + (16 * mt + s2q) * SZ_BYTES));
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(z1) : "r"(zrow + (16 * mt + s2q1) * SZ_BYTES));
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(z2) : "r"(zrow + (16 * mt + s2q + 8) * SZ_BYTES));
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(z3) : "r"(zrow + (16 * mt + s2q1 + 8) * SZ_BYTES));
+      float z4[4] = {st.zacc[0], st.zacc[1], 0.f, 0.f};
+      mma16816(z4, prmt(z0, z1, 0x7632u), 0u, prmt(z2, z3, 0x7632u), 0u,
+               movmatrix_t(pack_half2(p[mt][0], p[mt][1])), movmatrix_t(pack_half2(p[mt][2], p[mt][3])));
+      st.zacc[0] = z4[0];
+      st.zacc[1] = z4[1];
+    }
     uint32_t bq[NG][2];
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
-      const float2 fa = __half22float2(u2h(waw[g]));
-      const float2 fb = __half22float2(u2h(wbw[g]));
-      st.zs[0][g] += p[mt][0] * fa.y + p[mt][2] * fb.y;
-      st.zs[1][g] += p[mt][1] * fa.y + p[mt][3] * fb.y;
-      bq[g][0] = movmatrix_t(pack_half2(p[mt][0] * fa.x, p[mt][1] * fa.x));
-      bq[g][1] = movmatrix_t(pack_half2(p[mt][2] * fb.x, p[mt][3] * fb.x));
+      const float sa = __low2float(u2h(waw[g]));
+      const float sb = __low2float(u2h(wbw[g]));
+      bq[g][0] = movmatrix_t(pack_half2(p[mt][0] * sa, p[mt][1] * sa));
+      bq[g][1] = movmatrix_t(pack_half2(p[mt][2] * sb, p[mt][3] * sb));
     }
     const uint32_t vrow = vc + 8 * r;
     const uint2 x0 = lds64(vrow + (16 * mt + s2q) * ROW_BYTES);
@@ -345,11 +401,12 @@ __device__ __forceinline__ void int4_tile(WarpState &st, uint32_t slot, int n_va
       const uint32_t xa = prmt(A0, A1, 0x5410u), ya = prmt(A0, A1, 0x7632u);
       const uint32_t xb = prmt(B0, B1, 0x5410u), yb = prmt(B0, B1, 0x7632u);
       const int g0 = 2 * hh, g1 = 2 * hh + 1;
-      mma16816(st.acc[g0][0], nib_lo(xa), nib_hi(xa), nib_lo(xb), nib_hi(xb), bq[g0][0], bq[g0][1]);
-      mma16816(st.acc[g0][1], nib_lo(ya), nib_hi(ya), nib_lo(yb), nib_hi(yb), bq[g0][0], bq[g0][1]);
-      mma16816(st.acc[g1][0], nib_lo(xa >> 8), nib_hi(xa >> 8), nib_lo(xb >> 8), nib_hi(xb >> 8),
+      // rows r take low nibbles (2^-24 O), rows r + 8 high nibbles (2^-20 O)
+      mma16816(st.acc[g0][0], code_lo(xa), code_hi(xa), code_lo(xb), code_hi(xb), bq[g0][0], bq[g0][1]);
+      mma16816(st.acc[g0][1], code_lo(ya), code_hi(ya), code_lo(yb), code_hi(yb), bq[g0][0], bq[g0][1]);
+      mma16816(st.acc[g1][0], code_lo(xa >> 8), code_hi(xa >> 8), code_lo(xb >> 8), code_hi(xb >> 8),
                bq[g1][0], bq[g1][1]);
-      mma16816(st.acc[g1][1], nib_lo(ya >> 8), nib_hi(ya >> 8), nib_lo(yb >> 8), nib_hi(yb >> 8),
+      mma16816(st.acc[g1][1], code_lo(ya >> 8), code_hi(ya >> 8), code_lo(yb >> 8), code_hi(yb >> 8),
                bq[g1][0], bq[g1][1]);
     }
   }
@@ -366,8 +423,11 @@ __device__ __forceinline__ void f16_tile(WarpState &st, uint32_t slot, int n_val
 #pragma unroll
   for (int g = 0; g < NG; ++g) {
     const uint4 ka = lds128(kb_ + tA * F16_ROW + 64 * g + 16 * q4);
-    mma16816(acc, prmt(ka.x, ka.y, 0x5410u), 0u, prmt(ka.x, ka.y, 0x7632u), 0u, st.qf[g][0][0], st.qf[g][0][1]);
-    mma16816(acc, prmt(ka.z, ka.w, 0x5410u), 0u, prmt(ka.z, ka.w, 0x7632u), 0u, st.qf[g][1][0], st.qf[g][1][1]);
+    // the odd channels' q is held divided by 16 (for the INT4 tiles)
+    const uint32_t q01 = h2u(__hmul2(u2h(st.qf[g][0][1]), u2h(0x4C004C00u)));  // x 16
+    const uint32_t q11 = h2u(__hmul2(u2h(st.qf[g][1][1]), u2h(0x4C004C00u)));
+    mma16816(acc, prmt(ka.x, ka.y, 0x5410u), 0u, prmt(ka.x, ka.y, 0x7632u), 0u, st.qf[g][0][0], q01);
+    mma16816(acc, prmt(ka.z, ka.w, 0x5410u), 0u, prmt(ka.z, ka.w, 0x7632u), 0u, st.qf[g][1][0], q11);
   }
   float S[4];
 #pragma unroll
@@ -412,30 +472,36 @@ __device__ __forceinline__ void unit_tiles(const DecodeArgs &a, const Smem &sm, 
 }
 
 // First tile of a unit (cost start cs, n4 + n16 tiles) whose start cost is >= x.
-__device__ __forceinline__ int first_tile_from(int64_t x, int64_t cs, int n4, int n16) {
-  const int64_t rel = x - cs;
+// Costs are int32: the host rejects launches whose total cost reaches 2^31.
+__device__ __forceinline__ int first_tile_from(int x, int cs, int n4, int n16) {
+  const int rel = x - cs;
   if (rel <= 0) return 0;
-  const int64_t c4 = static_cast<int64_t>(COST4) * n4;
-  int64_t j;
-  if (rel <= c4) j = (rel + COST4 - 1) / COST4;
-  else j = n4 + (rel - c4 + COST16 - 1) / COST16;
-  return static_cast<int>(j < n4 + n16 ? j : n4 + n16);
+  const int c4 = COST4 * n4;
+  const int j = (rel <= c4) ? (rel + COST4 - 1) / COST4 : n4 + (rel - c4 + COST16 - 1) / COST16;
+  return j < n4 + n16 ? j : n4 + n16;
 }
 
 // Start cost of tile j of a unit.
-__device__ __forceinline__ int64_t tile_cost(int64_t cs, int n4, int j) {
-  return j <= n4 ? cs + static_cast<int64_t>(COST4) * j
-                 : cs + static_cast<int64_t>(COST4) * n4 + static_cast<int64_t>(COST16) * (j - n4);
+__device__ __forceinline__ int tile_cost(int cs, int n4, int j) {
+  return j <= n4 ? cs + COST4 * j : cs + COST4 * n4 + COST16 * (j - n4);
 }
 
-__device__ __forceinline__ int64_t cta_lo(int64_t c, int64_t total, int64_t n_ctas) { return c * total / n_ctas; }
-// block whose cost range holds x: the largest c with cta_lo(c) <= x
-__device__ __forceinline__ int cta_of_cost(int64_t x, int64_t total, int64_t n_ctas) {
-  return static_cast<int>(((x + 1) * n_ctas - 1) / total);
-}
+// Balanced split of the total cost over the launch's blocks: block c owns
+// [lo(c), lo(c + 1)) with lo(c) = c * per + min(c, rem), i.e. the first rem
+// blocks take per + 1 and the others per.
+struct Split {
+  int per, rem;
+  __device__ __forceinline__ Split(int total, int n) : per(total / n), rem(total % n) {}
+  __device__ __forceinline__ int lo(int c) const { return c * per + min(c, rem); }
+  // the block whose (non-empty) range holds cost x, for 0 <= x < total
+  __device__ __forceinline__ int of(int x) const {
+    const int big = rem * (per + 1);
+    return x < big ? x / (per + 1) : rem + (x - big) / per;
+  }
+};
 
 // last unit u with cost_start[u] <= x
-__device__ __forceinline__ int unit_of_cost(const int *cs, int U, int64_t x) {
+__device__ __forceinline__ int unit_of_cost(const int *cs, int U, int x) {
   int lo = 0, hi = U - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -452,7 +518,7 @@ struct Seg {
 
 // Next non-empty segment of this block at or after unit u (u = U: none).
 template <int MODE>
-__device__ __forceinline__ Seg seg_from(const DecodeArgs &a, const Smem &sm, int u, int base, int64_t lo, int64_t hi) {
+__device__ __forceinline__ Seg seg_from(const DecodeArgs &a, const Smem &sm, int u, int base, int lo, int hi) {
   Seg s{a.U, 0, 0, base};
   for (; u < a.U && sm.cost_start[u] < hi; ++u) {
     int n4, n16;
@@ -469,91 +535,110 @@ __device__ __forceinline__ Seg seg_from(const DecodeArgs &a, const Smem &sm, int
   return s;
 }
 
-// Merge the partials of unit u written by the blocks that share it (run by
-// the last block to finish, 128 consumer threads).  The ids of the partial
-// records go to shared memory first; then every thread owns float4 slices of
-// the output of one head and merges the records online, loading (max, sum,
-// slice) of MERGE_BATCH records at a time so their latencies overlap.
-constexpr int MERGE_CHUNK = 128;
-constexpr int MERGE_BATCH = 20;
+// Log-sum-exp combine of the NCW per-warp states in shared memory (sm.mm,
+// sm.ml, sm.mo) for output element idx of [G][D]: returns the merged max,
+// sum and unnormalized output.
+template <int G>
+__device__ __forceinline__ void combine_warps(const Smem &sm, int idx, float &M, float &L, float &O) {
+  const int h = idx / D, c = idx % D;
+  M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < NCW; ++w) M = fmaxf(M, sm.mm[w * 8 + h]);
+  L = 0.f;
+  O = 0.f;
+#pragma unroll
+  for (int w = 0; w < NCW; ++w) {
+    const float mw = sm.mm[w * 8 + h];
+    const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+    L += sm.ml[w * 8 + h] * f;
+    O += sm.mo[(w * G + h) * D + c] * f;
+  }
+}
 
+// Merge the partial records of unit u written by the blocks that share it
+// (run by the last block to finish).  Warp w takes the records of candidate
+// blocks c_lo + w, c_lo + w + NCW, ...; lane l holds channels 4l..4l+3 of
+// every head.  A batch of RB records is loaded at once (one round trip to
+// L2 per batch, most warps need one batch), merged online in registers, and
+// the NCW warp states are then combined through shared memory like the
+// warps of one block.
 template <int G>
 __device__ __forceinline__ void merge_parts(const DecodeArgs &a, const Smem &sm, int u, int n4, int n16,
-                                            int64_t total, int64_t N, int64_t hbase, int tid) {
-  int *pid = sm.scan;  // [MERGE_CHUNK] partial record index, or -1 for a block without tiles of u
-  const int64_t cs = sm.cost_start[u];
-  const int c_lo = cta_of_cost(cs, total, N), c_hi = cta_of_cost(tile_cost(cs, n4, n4 + n16 - 1), total, N);
-  constexpr int NV = (G * D / 4 + NCW * 32 - 1) / (NCW * 32);  // float4 outputs per thread
-  float4 acc[NV];
-  float M[NV], L[NV];
+                                            const Split &sp, int64_t hbase, int tid) {
+  constexpr int RB = (G >= 8) ? 1 : 16 / G;  // records per batch (bounded by registers)
+  const int warp = tid >> 5, lane = tid & 31;
+  const int cs = sm.cost_start[u];
+  const int c_lo = sp.of(cs), c_hi = sp.of(tile_cost(cs, n4, n4 + n16 - 1));
+  float M[G], L[G];
+  float4 acc[G];
 #pragma unroll
-  for (int v = 0; v < NV; ++v) {
-    acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-    M[v] = -INFINITY;
-    L[v] = 0.f;
+  for (int h = 0; h < G; ++h) {
+    M[h] = -INFINITY;
+    L[h] = 0.f;
+    acc[h] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  for (int base = c_lo; base <= c_hi; base += MERGE_CHUNK) {
-    const int n = min(MERGE_CHUNK, c_hi - base + 1);
-    named_bar_sync(1, NCW * 32);
-    for (int j = tid; j < n; j += NCW * 32) {
-      const int64_t cc = base + j;
-      const int64_t lo = cta_lo(cc, total, N), hi = cta_lo(cc + 1, total, N);
-      const bool has = first_tile_from(lo, cs, n4, n16) < first_tile_from(hi, cs, n4, n16);
-      pid[j] = has ? static_cast<int>(cc * 2 + ((cs <= lo) ? 0 : 1)) : -1;
-    }
-    named_bar_sync(1, NCW * 32);
+  for (int c0 = c_lo + warp; c0 <= c_hi; c0 += RB * NCW) {
+    float2 ml[RB][G];
+    float4 x[RB][G];
 #pragma unroll
-    for (int v = 0; v < NV; ++v) {
-      const int o4 = tid + v * NCW * 32;  // float4 index over [G][32]
-      if (o4 >= G * D / 4) continue;
-      const int h = o4 / (D / 4), c4 = o4 % (D / 4);
-      for (int j0 = 0; j0 < n; j0 += MERGE_BATCH) {
-        float2 ml[MERGE_BATCH];
-        float4 x[MERGE_BATCH];
+    for (int b = 0; b < RB; ++b) {
+      const int cc = c0 + b * NCW;
+      int id = -1;  // record of block cc for unit u, if cc has tiles of u
+      if (cc <= c_hi) {
+        const int lo = sp.lo(cc), hi = sp.lo(cc + 1);
+        if (first_tile_from(lo, cs, n4, n16) < first_tile_from(hi, cs, n4, n16)) id = cc * 2 + ((cs <= lo) ? 0 : 1);
+      }
 #pragma unroll
-        for (int b = 0; b < MERGE_BATCH; ++b) {
-          const int id = (j0 + b < n) ? pid[j0 + b] : -1;
-          ml[b] = make_float2(-INFINITY, 0.f);
-          x[b] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (id >= 0) {
-            const float *pr = a.part + (static_cast<int64_t>(id) * G + h) * PART_STRIDE;
-            ml[b] = __ldcg(reinterpret_cast<const float2 *>(pr));
-            x[b] = __ldcg(reinterpret_cast<const float4 *>(pr + 4 + 4 * c4));
-          }
+      for (int h = 0; h < G; ++h) {
+        ml[b][h] = make_float2(-INFINITY, 0.f);
+        x[b][h] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (id >= 0) {
+          const float *pr = a.part + (static_cast<int64_t>(id) * G + h) * PART_STRIDE;
+          ml[b][h] = __ldcg(reinterpret_cast<const float2 *>(pr));
+          x[b][h] = __ldcg(reinterpret_cast<const float4 *>(pr + 4 + 4 * lane));
         }
-        float bm = M[v];
-#pragma unroll
-        for (int b = 0; b < MERGE_BATCH; ++b) bm = fmaxf(bm, ml[b].x);
-        if (bm == -INFINITY) continue;
-        const float al = (M[v] == -INFINITY) ? 0.f : fast_exp2(M[v] - bm);
-        float4 s4 = make_float4(acc[v].x * al, acc[v].y * al, acc[v].z * al, acc[v].w * al);
-        float sl = L[v] * al;
-#pragma unroll
-        for (int b = 0; b < MERGE_BATCH; ++b) {
-          const float w = (ml[b].x == -INFINITY) ? 0.f : fast_exp2(ml[b].x - bm);
-          sl += w * ml[b].y;
-          s4.x += w * x[b].x;
-          s4.y += w * x[b].y;
-          s4.z += w * x[b].z;
-          s4.w += w * x[b].w;
-        }
-        acc[v] = s4;
-        M[v] = bm;
-        L[v] = sl;
       }
     }
-  }
 #pragma unroll
-  for (int v = 0; v < NV; ++v) {
-    const int o4 = tid + v * NCW * 32;
-    if (o4 < G * D / 4) {
-      const int h = o4 / (D / 4), c4 = o4 % (D / 4);
-      const float inv = 1.f / L[v];
-      __half2 lo = __floats2half2_rn(acc[v].x * inv, acc[v].y * inv);
-      __half2 hi = __floats2half2_rn(acc[v].z * inv, acc[v].w * inv);
-      *reinterpret_cast<uint2 *>(a.o + (hbase + h) * D + 4 * c4) = make_uint2(h2u(lo), h2u(hi));
-      if (c4 == 0 && a.lse) a.lse[hbase + h] = (M[v] + __log2f(L[v])) * LN2;
+    for (int h = 0; h < G; ++h) {
+      float bm = M[h];
+#pragma unroll
+      for (int b = 0; b < RB; ++b) bm = fmaxf(bm, ml[b][h].x);
+      if (bm == -INFINITY) continue;
+      const float al = (M[h] == -INFINITY) ? 0.f : fast_exp2(M[h] - bm);
+      float4 s4 = make_float4(acc[h].x * al, acc[h].y * al, acc[h].z * al, acc[h].w * al);
+      float sl = L[h] * al;
+#pragma unroll
+      for (int b = 0; b < RB; ++b) {
+        const float w = (ml[b][h].x == -INFINITY) ? 0.f : fast_exp2(ml[b][h].x - bm);
+        sl += w * ml[b][h].y;
+        s4.x += w * x[b][h].x;
+        s4.y += w * x[b][h].y;
+        s4.z += w * x[b][h].z;
+        s4.w += w * x[b][h].w;
+      }
+      acc[h] = s4;
+      M[h] = bm;
+      L[h] = sl;
     }
+  }
+  // the block's own per-warp buffers are free again (the caller has passed
+  // the barriers after its block merge)
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    if (lane == 0) {
+      sm.mm[warp * 8 + h] = M[h];
+      sm.ml[warp * 8 + h] = L[h];
+    }
+    *reinterpret_cast<float4 *>(sm.mo + (warp * G + h) * D + 4 * lane) = acc[h];
+  }
+  named_bar_sync(1, NTHREADS);
+  for (int idx = tid; idx < G * D; idx += NTHREADS) {
+    float Mx, Lx, Ox;
+    combine_warps<G>(sm, idx, Mx, Lx, Ox);
+    const int h = idx / D, c = idx % D;
+    a.o[(hbase + h) * D + c] = __float2half_rn(Ox / Lx);
+    if (c == 0 && a.lse) a.lse[hbase + h] = (Mx + __log2f(Lx)) * LN2;
   }
 }
 
@@ -597,7 +682,7 @@ __device__ __forceinline__ void issue_tile(const DecodeArgs &a, const Smem &sm, 
 }
 
 template <int G, int MODE>
-__global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a) {
   constexpr int SPW = Ring<G>::SPW;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -625,13 +710,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
   }
   const int U = a.U;
 
-  // ---- prologue: zero the ring, read every unit's (T, vl_count), cost prefix
+  // ---- prologue: read every unit's (T, vl_count), cost prefix
   {
-    // the ring starts as zeros, so stale bytes read as scale/zero are finite
-    for (int i = tid; i < NCW * SPW * SLOT_BYTES / 16; i += NTHREADS)
-      *reinterpret_cast<uint4 *>(smem_raw + 16 * i) = make_uint4(0, 0, 0, 0);
-    // order these generic-proxy stores before the bulk copies (async proxy)
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     const int per = (U + NTHREADS - 1) / NTHREADS;
     const int beg = min(U, tid * per), end = min(U, beg + per);
     int local = 0;
@@ -667,10 +747,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
     if (tid == NTHREADS - 1) sm.cost_start[U] = acc;
     __syncthreads();
   }
-  const int64_t total = sm.cost_start[U];
-  const int64_t N = a.n_ctas;
+  const int total = sm.cost_start[U];
+  const Split sp(total, a.n_ctas);
   const int cta = blockIdx.x;
-  const int64_t lo = total ? cta_lo(cta, total, N) : 0, hi = total ? cta_lo(cta + 1, total, N) : 0;
+  const int lo = sp.lo(cta), hi = sp.lo(cta + 1);
   volatile int *abort_flag = sm.abort_flag;
   const int u_first = (lo < hi) ? unit_of_cost(sm.cost_start, U, lo) : U;
 
@@ -705,6 +785,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
     load_q<G>(st, a, u, lane);
     // my tiles inside this segment: block-local i = base .. base + je - jb - 1
     int i = sg.base + (warp - sg.base % NCW + NCW) % NCW;
+    bool scaled = false;  // acc holds the INT4 sweep's power-of-two factors
     for (; i < sg.base + sg.je - sg.jb; i += NCW) {
       const int kk = k_done;
       const int sl = kk % SPW;
@@ -723,7 +804,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
         uint32_t bits;
         asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bits) : "r"(slot + SLOT_MASK));
         int4_tile(st, slot, n, bits, lane);
+        scaled = true;
       } else {
+        if (scaled) unscale_acc(st);
+        scaled = false;
         int n;
         if (MODE == MODE_FP16)
           n = min(F16_ROWS, us.T - j * F16_ROWS);
@@ -740,16 +824,18 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
     }
 
     // ---- segment end: reduce the warp's state over token rows
+    if (scaled) unscale_acc(st);
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        st.l[e] += __shfl_xor_sync(0xffffffffu, st.l[e], off);
-#pragma unroll
-        for (int g = 0; g < NG; ++g) st.zs[e][g] += __shfl_xor_sync(0xffffffffu, st.zs[e][g], off);
-      }
+      for (int e = 0; e < 2; ++e) st.l[e] += __shfl_xor_sync(0xffffffffu, st.l[e], off);
     }
     const int r = lane >> 2, q4 = lane & 3;
+    float zs[2][NG];  // value zero term of heads 2q, 2q+1: held by lane (g, q)
+#pragma unroll
+    for (int g = 0; g < NG; ++g)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) zs[e][g] = __shfl_sync(0xffffffffu, st.zacc[e], 4 * g + q4);
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int h = 2 * q4 + e;
@@ -764,8 +850,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
             const int ch = 32 * g + 4 * r + 2 * j;
-            orow[ch] = st.acc[g][j][e] + st.zs[e][g];
-            orow[ch + 1] = st.acc[g][j][2 + e] + st.zs[e][g];
+            orow[ch] = st.acc[g][j][e] + zs[e][g];
+            orow[ch + 1] = st.acc[g][j][2 + e] + zs[e][g];
           }
       }
     }
@@ -778,17 +864,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
     const int64_t hbase = static_cast<int64_t>(b) * a.Hq + kvh * G;
     for (int idx = tid; idx < G * D; idx += NTHREADS) {
       const int h = idx / D, c = idx % D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) M = fmaxf(M, sm.mm[w * 8 + h]);
-      float L = 0.f, O = 0.f;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) {
-        const float mw = sm.mm[w * 8 + h];
-        const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-        L += sm.ml[w * 8 + h] * f;
-        O += sm.mo[(w * G + h) * D + c] * f;
-      }
+      float M, L, O;
+      combine_warps<G>(sm, idx, M, L, O);
       if (complete) {
         a.o[(hbase + h) * D + c] = __float2half_rn(O / L);
         if (c == 0 && a.lse) a.lse[hbase + h] = (M + __log2f(L)) * LN2;
@@ -812,7 +889,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
       named_bar_sync(1, NTHREADS);
       if (*sm.last_flag) {
         __threadfence();
-        merge_parts<G>(a, sm, u, us.n4, us.nv + us.nw, total, N, hbase, tid);
+        merge_parts<G>(a, sm, u, us.n4, us.nv + us.nw, sp, hbase, tid);
         if (tid == 0) a.counters[u] = 0;
       }
     }
@@ -837,7 +914,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_kernel(const DecodeArgs a)
 
 // ---------------------------------------------------------------- host side
 static size_t decode_smem_bytes(int G, int U) {
-  const int spw = (G == 8) ? 2 : 3;
+  const int spw = Ring<1>::SPW;
+  static_assert(Ring<1>::SPW == Ring<8>::SPW, "one ring depth for every G");
   return static_cast<size_t>(NCW) * spw * SLOT_BYTES + NCW * spw * 8 + 16 + NCW * 8 * 4 * 2 +
          static_cast<size_t>(NCW) * G * D * 4 + NTHREADS * 4 + (static_cast<size_t>(U + 1) * 4 + 15) / 16 * 16 +
          static_cast<size_t>(U) * 8;
@@ -886,7 +964,7 @@ static inline bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) 
 
 static int resolve_ctas(int32_t n_ctas) {
   if (n_ctas > 0) return n_ctas;
-  return 2 * hyq_sm_count();
+  return hyq_sm_count();
 }
 
 extern "C" int32_t hyq_decode_default_ctas(void) { return resolve_ctas(0); }
@@ -904,6 +982,15 @@ extern "C" size_t hyq_decode_fp16_workspace(int32_t batch, int32_t n_q_heads, in
 
 static bool g_supported(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
 
+// The kernels split the work in int32 cost units; bound the total.
+static bool cost_fits(int U, int cap, int vl_cap, int mode) {
+  const int64_t per_unit = (mode == MODE_FP16)
+                               ? static_cast<int64_t>(COST16) * ((cap + F16_ROWS - 1) / F16_ROWS)
+                               : static_cast<int64_t>(COST4) * ((cap + I4_TOK - 1) / I4_TOK) +
+                                     static_cast<int64_t>(COST16) * ((vl_cap + F16_ROWS - 1) / F16_ROWS + WIN / F16_ROWS);
+  return static_cast<int64_t>(U) * per_unit < (static_cast<int64_t>(1) << 31) - 1;
+}
+
 extern "C" hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, float *lse,
                                  int32_t n_ctas, void *ws, size_t ws_bytes, void *stream) {
   hyq_status s = hyq_check_cache(c);
@@ -913,7 +1000,7 @@ extern "C" hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, flo
   if (n_ctas < 0) return HYQ_ERR_INVALID;
   const int G = c->n_q_heads / c->n_kv_heads;
   const int U = c->batch * c->n_kv_heads;
-  if (U > MAX_UNITS) return HYQ_ERR_UNSUPPORTED;
+  if (U > MAX_UNITS || !cost_fits(U, c->capacity, c->vl_capacity, MODE_HYBRID)) return HYQ_ERR_UNSUPPORTED;
   const int N = resolve_ctas(n_ctas);
   if (!ws || ws_bytes < decode_ws_bytes(G, U, N)) return HYQ_ERR_WORKSPACE;
   DecodeArgs a{};
@@ -945,7 +1032,7 @@ extern "C" hyq_status hyq_decode_fp16(const void *q, const void *k, const void *
     return HYQ_ERR_ALIGN;
   const int G = n_q_heads / n_kv_heads;
   const int U = batch * n_kv_heads;
-  if (U > MAX_UNITS) return HYQ_ERR_UNSUPPORTED;
+  if (U > MAX_UNITS || !cost_fits(U, capacity, 0, MODE_FP16)) return HYQ_ERR_UNSUPPORTED;
   const int N = resolve_ctas(n_ctas);
   if (!ws || ws_bytes < decode_ws_bytes(G, U, N)) return HYQ_ERR_WORKSPACE;
   DecodeArgs a{};
@@ -1001,6 +1088,7 @@ extern "C" hyq_status hyq_decode_noalloc(const hyq_cache *c, const void *q, void
   const int U = c->batch * c->n_kv_heads;
   const int N = resolve_ctas(0);
   if (U > NOALLOC_MAX_UNITS || N > NOALLOC_MAX_CTAS || G > NOALLOC_MAX_G) return HYQ_ERR_UNSUPPORTED;
+  if (!cost_fits(U, c->capacity, c->vl_capacity, MODE_HYBRID)) return HYQ_ERR_UNSUPPORTED;
   if (decode_ws_bytes(G, U, N) > NOALLOC_BYTES) return HYQ_ERR_UNSUPPORTED;
   void *ws = nullptr;
   if (!noalloc_address(&ws)) return HYQ_ERR_CUDA;

@@ -221,16 +221,19 @@ hyq_status hyq_vl_apply(const hyq_cache *c, const int32_t *pos, int32_t k,
 /*
  * hyq_decode -- one decode step of GQA attention over the hybrid cache,
  * INT4 dequantization fused into the attention (split-KV flash decoding:
- * work is spread over n_ctas thread blocks by tile count, per-block partial
+ * work is spread over n_ctas thread blocks by bytes read, per-block partial
  * (max, sum, accumulator) triples are merged by log-sum-exp in the last
  * block to finish a unit).
  *   q    fp16 [B][Hq][128]; o fp16 [B][Hq][128] output
  *   lse  nullable fp32 [B][Hq]: natural-log sum of exp of the scaled logits
- *   n_ctas  thread blocks; 0 = automatic (a multiple of the SM count)
+ *   n_ctas  thread blocks; 0 = automatic (one per SM)
  *   ws   workspace of hyq_decode_workspace(c, n_ctas) bytes; zero-filled
  *        before the first call, every completed call leaves it reusable
  *        (re-zero it after a call that reported HYQ_DEV_TIMEOUT)
  * Scale 1/sqrt(128); all softmax arithmetic in fp32.
+ * HYQ_ERR_UNSUPPORTED when batch x n_kv_heads > 4096, or when the launch's
+ * work, counted as 5 per 32 capacity positions plus 4 per 8 rows of
+ * vl_capacity and window, reaches 2^31 over all units.
  */
 size_t hyq_decode_workspace(const hyq_cache *c, int32_t n_ctas);
 hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, float *lse,
@@ -267,6 +270,8 @@ hyq_status hyq_decode_noalloc(const hyq_cache *c, const void *q, void *o, float 
  *   o fp16 [B][Hq][128]; lse nullable fp32 [B][Hq]
  *   ws   workspace of hyq_decode_fp16_workspace(B, Hq, Hkv, n_ctas) bytes,
  *        zero-filled before the first call
+ * HYQ_ERR_UNSUPPORTED when batch x n_kv_heads > 4096 or when
+ * batch x n_kv_heads x 4 x ceil(capacity / 8) reaches 2^31.
  */
 size_t hyq_decode_fp16_workspace(int32_t batch, int32_t n_q_heads,
                                  int32_t n_kv_heads, int32_t n_ctas);
