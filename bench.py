@@ -41,18 +41,31 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decode-attention effective HBM GB/s (% of B200 peak); µs/step at 32K ctx"
-N_LAYERS = 8
+L2_DEFEAT_BYTES = 360e6  # rotate layer caches until a pass over them is ~3x the 126 MB L2
 RESELECT = 64
 N_Q = 64
 
 
+EV_EVERY = 8  # decodes timed with events: one in every EV_EVERY steps
+
+
 def algorithmic_bytes(B, Hq, Hkv, T, k, W=128):
-    """Bytes one decode step must move: packed INT4 K/V + scale/zero (160 B
-    per token per unit), FP16 K/V of vertical-line and window tokens (512 B),
-    Q in and O out (fp16)."""
+    """Bytes one decode must move at length T: packed INT4 K/V + scale/zero
+    (160 B per token per unit), FP16 K/V of vertical-line and window tokens
+    (512 B), Q in and O out (fp16).  k: vertical-line rows, one count for
+    every unit or a list with one count per unit."""
     n_old = max(0, T - W)
-    per_unit = (n_old - k) * 160 + k * 512 + min(T, W) * 512
-    return B * Hkv * per_unit + B * Hq * 128 * 2 * 2
+    ks = [k] * (B * Hkv) if isinstance(k, int) else list(k)
+    return sum((n_old - ku) * 160 + ku * 512 + min(T, W) * 512 for ku in ks) + B * Hq * 128 * 2 * 2
+
+
+def step_bytes(B, Hq, Hkv, T, k, W=128):
+    """Bytes of one fused step that ends at length T: the decode's, plus the
+    append's per unit (new K/V rows in, the leaving window row in, its INT4
+    codes and scale/zero out, the new rows into the window) and the query
+    into the detector ring."""
+    append = (2 * 256 + 2 * 256 + 160 + 2 * 256) if T - 1 >= W else (2 * 256 + 2 * 256)
+    return algorithmic_bytes(B, Hq, Hkv, T, k, W) + B * Hkv * append + B * Hq * 256
 
 
 def decode_traffic():
@@ -64,7 +77,7 @@ def decode_traffic():
     with open(p) as f:
         d = json.load(f)
     h = hashlib.sha256()
-    for name in ("hyq_decode.cu", "hyq_common.cuh"):
+    for name in ("hyq_decode.cu", "hyq_common.cuh", "hyq_quant.cuh"):
         with open(os.path.join(ROOT, "fp16_kv_cache_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return int(d["bytes_per_launch"]) if h.hexdigest() == d.get("source_sha256") else None
@@ -89,6 +102,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4],
+                    help="workload (2: the headline Llama-3.1-8B 32K batch-1 decode; 3 and 4 for profiling)")
     return ap.parse_args()
 
 
@@ -174,11 +189,13 @@ def run_ours(args):
         dist.init_process_group("nccl", device_id=torch.device("cuda", local),
                                 timeout=__import__("datetime").timedelta(seconds=120))
     build.build()
-    cfg = synth.config(2)
+    cfg = synth.config(args.config)
     K_steps, W_steps = args.steps, args.warmup
-    per_layer_tokens = (K_steps + W_steps + args.e2e_steps) // N_LAYERS + 2
+    # enough layer caches that consecutive steps never find their data in L2
+    n_layers = int(min(8, max(2, math.ceil(L2_DEFEAT_BYTES / algorithmic_bytes(cfg.B, cfg.Hq, cfg.Hkv, cfg.T, cfg.k)))))
+    per_layer_tokens = (K_steps + W_steps + args.e2e_steps) // n_layers + 2
     cap = ((cfg.T + per_layer_tokens + 127) // 128) * 128
-    layers, Kd, Vd = setup_layers(torch, hyq, synth, cfg, cap, N_LAYERS)
+    layers, Kd, Vd = setup_layers(torch, hyq, synth, cfg, cap, n_layers)
     B, Hq, Hkv = cfg.B, cfg.Hq, cfg.Hkv
     dev = torch.device("cuda", local)
 
@@ -192,34 +209,36 @@ def run_ours(args):
     out = torch.empty(B, Hq, 128, dtype=torch.float16, device=dev)
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
     n_ctas = hyq.hyq_decode_default_ctas()
-    dws = [hyq.workspace(hyq.hyq_decode_workspace(c, n_ctas)) for c in layers]
+    dws = [hyq.workspace(hyq.hyq_decode_step_workspace(c, n_ctas)) for c in layers]
     sws = hyq.workspace(hyq.hyq_select_vl_workspace(layers[0], N_Q))
     sel_pos = torch.zeros(B, Hkv, cfg.k, dtype=torch.int32, device=dev)
     nunp = torch.zeros(1, dtype=torch.int32, device=dev)
-    tokens = [cfg.T] * N_LAYERS        # host mirror of each layer's length
-    appended = [0] * N_LAYERS
+    tokens = [cfg.T] * n_layers        # host mirror of each layer's length
+    appended = [0] * n_layers
 
-    resel_at = {}  # layer -> index of the step whose decode first sees the new VL set
+    resel_at = {}  # layer -> step after which its first re-selection ran
 
     def step(s, ev=None):
-        """Enqueue step s; returns (launches, layer, T seen by the decode)."""
-        li = s % N_LAYERS
+        """Enqueue step s; returns (launches, layer, T after the step's append)."""
+        li = s % n_layers
         c = layers[li]
         i = s % 64
-        hyq.hyq_append(c, k_in[i], v_in[i], q_in[i], rings[li])
+        if ev is not None:
+            ev[0].record()
+        hyq.hyq_decode_step(c, q_in[i], k_in[i], v_in[i], out, dws[li], q_ring=rings[li], lse=lse,
+                            n_ctas=n_ctas)
+        if ev is not None:
+            ev[1].record()
         tokens[li] += 1
         appended[li] += 1
-        launches = 2
+        launches = 1
         if appended[li] % RESELECT == 0:
+            # the 64 queries of the ring are scored; the next decode of the
+            # layer sees the new vertical-line set
             hyq.hyq_select_vl(c, rings[li], cfg.k, sel_pos, sws, q_is_ring=True)
             hyq.hyq_vl_apply(c, sel_pos, n_unpromoted=nunp)
             resel_at.setdefault(li, s)
             launches += 6  # select (cache mode): 5 kernels; vl_apply (cache mode): 1
-        if ev is not None:
-            ev[0].record()
-        hyq.hyq_decode(c, q_in[i], out, dws[li], lse=lse, n_ctas=n_ctas)
-        if ev is not None:
-            ev[1].record()
         return launches, li, tokens[li]
 
     # warm-up (eager, untimed) -- also sets kernel attributes before capture
@@ -227,9 +246,9 @@ def run_ours(args):
         step(s)
     torch.cuda.synchronize()
 
-    # capture K steps with events around every decode
+    # capture K steps; every EV_EVERY-th step's launch is bracketed by events
     evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
-           for _ in range(K_steps)]
+           if j % EV_EVERY == 0 else None for j in range(K_steps)]
     g = torch.cuda.CUDAGraph()
     total_launches = 0
     seen = []  # (step, layer, T)
@@ -266,24 +285,28 @@ def run_ours(args):
         elapsed_ms = float(t.item())
     # algorithmic bytes of every timed decode, with the VL count it saw
     # (a cache-mode re-selection keeps only rows still held in FP16)
-    k_after = [int(c.vl_count.min().item()) for c in layers]
-    k_after_max = [int(c.vl_count.max().item()) for c in layers]
+    k_after = [c.vl_count.flatten().tolist() for c in layers]  # per unit, after the re-selection
     total_bytes = 0
-    for s_, li, T in seen:
-        kk = cfg.k if (li not in resel_at or s_ < resel_at[li]) else k_after[li]
-        total_bytes += algorithmic_bytes(B, Hq, Hkv, T, kk)
-    dec_ms = [a.elapsed_time(b) for a, b in evs]
+    ev_bytes = []
+    for j, (s_, li, T) in enumerate(seen):
+        kk = cfg.k if (li not in resel_at or s_ <= resel_at[li]) else k_after[li]
+        nb = step_bytes(B, Hq, Hkv, T, kk)
+        total_bytes += nb
+        if evs[j] is not None:
+            ev_bytes.append(nb)
+    dec_ms = [e[0].elapsed_time(e[1]) for e in evs if e is not None]
     dec_avg_ms = float(np.mean(dec_ms))
     status = max(c.status() for c in layers)
 
     # roofline of the decode kernel (the dominant launch)
     peak, peak_kind = measured_peaks()
-    bytes_per_decode = total_bytes / K_steps
+    bytes_per_decode = float(np.mean(ev_bytes))
     achieved = bytes_per_decode / (dec_avg_ms * 1e-3) / 1e9
     value = world * total_bytes / (elapsed_ms * 1e-3) / 1e9
 
     # FP16 comparator (same kernel design over an all-FP16 cache), 3 copies > L2
-    fp16 = fp16_comparator(torch, hyq, cfg, Kd, Vd, q_in, dev)
+    # (the comparator needs 3 FP16 copies of the cache: headline workload only)
+    fp16 = fp16_comparator(torch, hyq, cfg, Kd, Vd, q_in, dev) if args.config == 2 else None
 
     # end to end through the public API with host buffers (eager loop)
     e2e = run_e2e(torch, hyq, cfg, layers, rings, dws, sws, sel_pos, nunp, n_ctas, tokens, appended,
@@ -296,24 +319,26 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
         "data": "synthetic (seeded N(0,1) fp16 Q/K/V, 4 K outlier channels x8, planted vertical lines)",
         "config": {
-            "workload": "llama3.1-8b-32k-b1: decode attention, B=1/GPU, Hq=32, Hkv=8, d=128, T=32768, "
-                        "window 128, VL 3% (983), INT4 g32",
-            "step": "hyq_append + hyq_decode on one of 8 layer caches; hyq_select_vl(cache)+hyq_vl_apply "
-                    "every 64 tokens of a layer",
-            "l2": "inputs larger than L2: 8 rotating layer caches (~360 MB) per GPU",
+            "workload": f"{cfg.name}: decode attention, B={cfg.B}/GPU, Hq={cfg.Hq}, Hkv={cfg.Hkv}, d=128, "
+                        f"T={cfg.T}, window 128, VL {cfg.k}, INT4 g32",
+            "step": f"hyq_decode_step (append + decode in one launch) on one of {n_layers} layer caches; "
+                    "hyq_select_vl(cache) + hyq_vl_apply after every 64 tokens of a layer",
+            "l2": f"inputs larger than L2: {n_layers} rotating layer caches (~{n_layers * total_bytes / K_steps / 1e6:.0f} MB) "
+                  "per GPU",
             "us_per_step": round(1000 * elapsed_ms / K_steps, 3),
             "decode_us_avg": round(1000 * dec_avg_ms, 3),
+            "decode_timed": f"CUDA events around {len(dec_ms)} of the {K_steps} timed launches",
             "decode_bytes_per_step": int(bytes_per_decode),
             "pct_of_peak_step": round(100 * value / world / peak, 1),
             "n_ctas": n_ctas,
             "fp16_comparator": fp16,
             "dev_status": status,
-            "vl_rows_after_reselect": [min(k_after), max(k_after_max)],
+            "vl_rows_after_reselect": [min(min(k) for k in k_after), max(max(k) for k in k_after)],
             "parallelism": f"replicas x{world} (independent sequences, no collective)",
         },
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": decode_traffic(),
-                     "kernel": "hyq::decode_kernel<4,0>", "peak_source": f"{peak_kind} hbm_gbs",
+                     "kernel": "hyq::decode_kernel<G,2> (hyq_decode_step)", "peak_source": f"{peak_kind} hbm_gbs",
                      "bytes_per_launch": int(bytes_per_decode)},
         "e2e": e2e,
         "gpu_launches": total_launches,
@@ -371,7 +396,9 @@ def run_e2e(torch, hyq, cfg, layers, rings, dws, sws, sel_pos, nunp, n_ctas, tok
     dk = torch.empty(B, Hkv, 128, dtype=torch.float16, device=dev)
     dv = torch.empty(B, Hkv, 128, dtype=torch.float16, device=dev)
     do = torch.empty(B, Hq, 128, dtype=torch.float16, device=dev)
-    total = 0
+    k_before = [c.vl_count.flatten().tolist() for c in layers]  # vertical-line rows per unit
+    seen = []  # (layer, T after the step, whether the layer has re-selected during this loop)
+    resel = set()
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
@@ -382,18 +409,20 @@ def run_e2e(torch, hyq, cfg, layers, rings, dws, sws, sel_pos, nunp, n_ctas, tok
         dq.copy_(hq[s], non_blocking=True)
         dk.copy_(hk[s], non_blocking=True)
         dv.copy_(hv[s], non_blocking=True)
-        hyq.hyq_append(c, dk, dv, dq, rings[li])
+        hyq.hyq_decode_step(c, dq, dk, dv, do, dws[li], q_ring=rings[li], n_ctas=n_ctas)
+        ho[s].copy_(do, non_blocking=True)
         tokens[li] += 1
         appended[li] += 1
+        seen.append((li, tokens[li], li in resel))
         if appended[li] % RESELECT == 0:
             hyq.hyq_select_vl(c, rings[li], cfg.k, sel_pos, sws, q_is_ring=True)
             hyq.hyq_vl_apply(c, sel_pos, n_unpromoted=nunp)
-        hyq.hyq_decode(c, dq, do, dws[li], n_ctas=n_ctas)
-        ho[s].copy_(do, non_blocking=True)
-        total += algorithmic_bytes(B, Hq, Hkv, tokens[li], cfg.k)
+            resel.add(li)
     t1.record()
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
+    k_after = [c.vl_count.flatten().tolist() for c in layers]
+    total = sum(step_bytes(B, Hq, Hkv, T, k_after[li] if late else k_before[li]) for li, T, late in seen)
     return {"value": round(world * total / (ms * 1e-3) / 1e9, 1), "unit": "GB/s",
             "h2d_bytes_per_step": (B * Hq + 2 * B * Hkv) * 256, "d2h_bytes_per_step": B * Hq * 256,
             "us_per_step": round(1000 * ms / n, 3), "steps": n,

@@ -10,6 +10,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/hyq.h"
 
 namespace hyq {
@@ -213,6 +215,33 @@ __device__ __forceinline__ float fast_exp2(float x) {
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return h2u(__floats2half2_rn(lo, hi));
+}
+
+// ---------------------------------------------------------------- launches
+// Programmatic dependent launch: every library kernel is launched with
+// programmatic stream serialization, so it may be scheduled while the
+// previous kernel on the stream is still running.  Each kernel calls
+// pdl_trigger() early (the next kernel may then be scheduled once every
+// block of this one has started) and pdl_wait() before it touches global
+// memory: the wait returns when the previous grid has completed and its
+// writes are visible, so stream order is kept.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+static inline cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                 Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace hyq

@@ -33,6 +33,7 @@
 //     writes its (max, sum, acc) partial and the last block to finish the
 //     unit (atomic tile counter) merges the partials by log-sum-exp.
 #include "hyq_common.cuh"
+#include "hyq_quant.cuh"
 
 namespace hyq {
 
@@ -69,14 +70,17 @@ struct Ring {
   static constexpr int SPW = 2;
 };
 
-enum { MODE_HYBRID = 0, MODE_FP16 = 1 };
+// MODE_STEP: the hybrid decode with the token append of the same step fused
+// in (hyq_decode_step): the cache is decoded as it is after the append.
+enum { MODE_HYBRID = 0, MODE_FP16 = 1, MODE_STEP = 2 };
 
 struct DecodeArgs {
   int B, Hq, Hkv, cap, W, vl_cap, U, n_ctas;
-  const uint8_t *blocks;  // quantized majority + bitmask, [U][cap/32][BLK_BYTES]
-  const __half *win_k, *win_v, *vl_k, *vl_v;
+  uint8_t *blocks;        // quantized majority + bitmask, [U][cap/32][BLK_BYTES]
+  __half *win_k, *win_v;  // written only by the fused step
+  const __half *vl_k, *vl_v;
   const int32_t *vl_count;
-  const int32_t *seq_len;
+  int32_t *seq_len;       // written only by the fused step
   const __half *k16, *v16;  // comparator cache [B][Hkv][cap][128]
   const __half *q;
   __half *o;
@@ -84,6 +88,12 @@ struct DecodeArgs {
   float *part;        // [n_ctas][2][G][PART_STRIDE]
   int32_t *counters;  // [U]
   uint32_t *status;
+  // fused step only: the new token's K/V rows [B][Hkv][128], the detector's
+  // query ring [B][Hq][n_q][128] (nullable), and a block counter
+  const __half *k_new, *v_new;
+  __half *q_ring;
+  int n_q;
+  int32_t *grid_counter;
 };
 
 // Token order inside a 16-token MMA block: row r of the block holds token
@@ -131,7 +141,8 @@ __device__ __forceinline__ UnitShape shape_of(const DecodeArgs &a, int T, int vl
 // per-unit (T, vl_count) copies kept in shared memory).
 template <int MODE>
 __device__ __forceinline__ UnitShape unit_shape_global(const DecodeArgs &a, int u, bool &bad) {
-  const int T = a.seq_len[u / a.Hkv];
+  int T = a.seq_len[u / a.Hkv];
+  if (MODE == MODE_STEP) T = (T < 0) ? -1 : T + 1;  // the length after the append
   const int vlc = (MODE == MODE_FP16) ? 0 : a.vl_count[u];
   return shape_of<MODE>(a, T, vlc, bad);
 }
@@ -642,6 +653,93 @@ __device__ __forceinline__ void merge_parts(const DecodeArgs &a, const Smem &sm,
   }
 }
 
+// ---------------------------------------------------------------- fused step
+// The append of hyq_append done inside the decode of the same step, so that
+// the result equals hyq_append followed by hyq_decode:
+//  * the row at position T_old - W (the oldest window row, slot T_old % W)
+//    is quantized by the warp that owns the unit's last INT4 tile; it
+//    patches the tile in shared memory, writes the codes to the cache block
+//    and then puts the new token into that window slot (every other reader
+//    of the slot takes the new token from k_new / v_new);
+//  * the warp that owns the window tile holding slot T_old % W patches that
+//    row from k_new / v_new (and writes the slot when T_old < W, where no
+//    row leaves the window);
+//  * the query goes to ring slot T_old % n_q, rows spread over the blocks;
+//  * seq_len = T_old + 1 is written by the last block to pass the prologue,
+//    when every block has read the old lengths.
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+// Lanes 0-15 handle the K row, lanes 16-31 the V row (8 channels each).
+__device__ __forceinline__ void step_exit_row(const DecodeArgs &a, int u, int T_old, uint32_t slot, int lane) {
+  const int t = lane & 15;
+  const bool is_v = lane >= 16;
+  const unsigned hmask = 0xFFFFu << (lane & 16);
+  const int px = T_old - a.W;
+  __half *wrow = (is_v ? a.win_v : a.win_k) + (static_cast<int64_t>(u) * a.W + T_old % a.W) * D;
+  const uint4 old = *reinterpret_cast<const uint4 *>(wrow + 8 * t);
+  const QuantShare q = quantize_share(old, t, hmask, a.status);
+  const int row = px % I4_TOK;
+  const uint32_t code_s = slot + (is_v ? SLOT_VC : 0) + row * ROW_BYTES;
+  const uint32_t sz_s = slot + (is_v ? SLOT_VSZ : SLOT_KSZ) + row * SZ_BYTES;
+  uint8_t *code_g = a.blocks + (is_v ? vcode_off(u, px, a.cap) : kcode_off(u, px, a.cap));
+  uint32_t *sz_g = reinterpret_cast<uint32_t *>(a.blocks + (is_v ? vsz_off(u, px, a.cap) : ksz_off(u, px, a.cap)));
+  if (q.has_codes) {
+    sts32(code_s + q.off0, q.w0);
+    sts32(code_s + q.off1, q.w1);
+    *reinterpret_cast<uint32_t *>(code_g + q.off0) = q.w0;
+    *reinterpret_cast<uint32_t *>(code_g + q.off1) = q.w1;
+  }
+  if (q.has_sz) {
+    sts32(sz_s + 4 * q.g, q.sz);
+    sz_g[q.g] = q.sz;
+  }
+  // the old row has been read (its value is consumed above): the new token
+  // takes its slot
+  const __half *nrow = (is_v ? a.v_new : a.k_new) + static_cast<int64_t>(u) * D;
+  *reinterpret_cast<uint4 *>(wrow + 8 * t) = *reinterpret_cast<const uint4 *>(nrow + 8 * t);
+  __syncwarp();
+}
+
+__device__ __forceinline__ void step_new_row(const DecodeArgs &a, int u, int s_new, int row, bool write_slot,
+                                             uint32_t slot, int lane) {
+  const int t = lane & 15;
+  const bool is_v = lane >= 16;
+  const uint4 x = *reinterpret_cast<const uint4 *>((is_v ? a.v_new : a.k_new) + static_cast<int64_t>(u) * D + 8 * t);
+  sts128(slot + (is_v ? SLOT_F16V : 0) + row * F16_ROW + 16 * t, x);
+  if (write_slot)
+    *reinterpret_cast<uint4 *>((is_v ? a.win_v : a.win_k) + (static_cast<int64_t>(u) * a.W + s_new) * D + 8 * t) = x;
+  __syncwarp();
+}
+
+// After the prologue (unit lengths in shared memory are T_old + 1).
+__device__ __forceinline__ void step_prologue(const DecodeArgs &a, const Smem &sm, int tid) {
+  if (a.q_ring) {
+    const int64_t items = static_cast<int64_t>(a.B) * a.Hq * 16;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * NTHREADS + tid; i < items;
+         i += static_cast<int64_t>(a.n_ctas) * NTHREADS) {
+      const int64_t row = i >> 4;  // b * Hq + query head
+      const int part = static_cast<int>(i & 15), b = static_cast<int>(row / a.Hq);
+      const int T = sm.unit_tv[b * a.Hkv].x;  // T_old + 1
+      if (T < 1 || T > a.cap) continue;
+      *reinterpret_cast<uint4 *>(a.q_ring + (row * a.n_q + (T - 1) % a.n_q) * D + 8 * part) =
+          *reinterpret_cast<const uint4 *>(a.q + row * D + 8 * part);
+    }
+  }
+  if (tid == 0 && atomicAdd(a.grid_counter, 1) == a.n_ctas - 1) {
+    // every block has read seq_len (each increments after its prologue)
+    for (int b = 0; b < a.B; ++b) {
+      const int T = sm.unit_tv[b * a.Hkv].x;
+      if (T >= 1 && T <= a.cap) a.seq_len[b] = T;
+    }
+    *a.grid_counter = 0;
+  }
+}
+
 // Issue the bulk copies of tile j of unit u into one ring slot (lane 0 arms
 // the barrier and copies; an FP16 tile is two contiguous runs of rows).
 template <int MODE>
@@ -650,7 +748,7 @@ __device__ __forceinline__ void issue_tile(const DecodeArgs &a, const Smem &sm, 
   bool bad;
   const UnitShape us = shape_of<MODE>(a, sm.unit_tv[u].x, sm.unit_tv[u].y, bad);
   if (lane != 0) return;
-  if (MODE == MODE_HYBRID && j < us.n4) {
+  if (MODE != MODE_FP16 && j < us.n4) {
     mbar_arrive_expect_tx(bar, BLK_BYTES);
     bulk_g2s(dst, a.blocks + blk_base(u, static_cast<int64_t>(j) * I4_TOK, a.cap), BLK_BYTES, bar);
     return;
@@ -709,6 +807,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
     sm.unit_tv = reinterpret_cast<int2 *>(p);
   }
   const int U = a.U;
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream (an append) is complete and visible
 
   // ---- prologue: read every unit's (T, vl_count), cost prefix
   {
@@ -746,6 +846,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
     }
     if (tid == NTHREADS - 1) sm.cost_start[U] = acc;
     __syncthreads();
+    if (MODE == MODE_STEP) step_prologue(a, sm, tid);
   }
   const int total = sm.cost_start[U];
   const Split sp(total, a.n_ctas);
@@ -798,9 +899,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
         continue;
       }
       const int j = sg.jb + (i - sg.base);
-      if (MODE == MODE_HYBRID && j < us.n4) {
+      if (MODE != MODE_FP16 && j < us.n4) {
         const int t0 = j * I4_TOK;
         const int n = min(I4_TOK, us.L4 - t0);
+        // fused step: the row leaving the window is the unit's last INT4 position
+        if (MODE == MODE_STEP && j == us.n4 - 1 && us.T > a.W) step_exit_row(a, u, us.T - 1, slot, lane);
         uint32_t bits;
         asm volatile("ld.shared.u32 %0, [%1];" : "=r"(bits) : "r"(slot + SLOT_MASK));
         int4_tile(st, slot, n, bits, lane);
@@ -815,6 +918,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
           n = min(F16_ROWS, us.vlc - (j - us.n4) * F16_ROWS);
         else
           n = min(F16_ROWS, us.nwin - (j - us.n4 - us.nv) * F16_ROWS);
+        if (MODE == MODE_STEP && j >= us.n4 + us.nv) {
+          // fused step: the new token's window row
+          const int r0 = (j - us.n4 - us.nv) * F16_ROWS, s_new = (us.T - 1) % a.W;
+          if (s_new >= r0 && s_new < r0 + n) step_new_row(a, u, s_new, s_new - r0, us.T - 1 < a.W, slot, lane);
+        }
         f16_tile(st, slot, n, lane);
       }
       // the slot has been read: order those reads before the next bulk copy
@@ -938,8 +1046,7 @@ static cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  decode_kernel<G, MODE><<<a.n_ctas, NTHREADS, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch(decode_kernel<G, MODE>, dim3(a.n_ctas), dim3(NTHREADS), smem, s, a);
 }
 
 template <int MODE>
@@ -1007,7 +1114,7 @@ extern "C" hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, flo
   a.B = c->batch; a.Hq = c->n_q_heads; a.Hkv = c->n_kv_heads; a.cap = c->capacity;
   a.W = c->window; a.vl_cap = c->vl_capacity; a.U = U; a.n_ctas = N;
   a.blocks = c->blocks;
-  a.win_k = static_cast<const __half *>(c->win_k); a.win_v = static_cast<const __half *>(c->win_v);
+  a.win_k = static_cast<__half *>(c->win_k); a.win_v = static_cast<__half *>(c->win_v);
   a.vl_k = static_cast<const __half *>(c->vl_k); a.vl_v = static_cast<const __half *>(c->vl_v);
   a.vl_count = c->vl_count; a.seq_len = c->seq_len;
   a.q = static_cast<const __half *>(q); a.o = static_cast<__half *>(o); a.lse = lse;
@@ -1016,6 +1123,48 @@ extern "C" hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, flo
   a.status = c->dev_status;
   return dispatch_decode<MODE_HYBRID>(G, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? HYQ_OK
                                                                                               : HYQ_ERR_CUDA;
+}
+
+// Fused append + decode: the workspace of hyq_decode plus 256 bytes for the
+// block counter of the seq_len update.
+extern "C" size_t hyq_decode_step_workspace(const hyq_cache *c, int32_t n_ctas) {
+  const size_t base = hyq_decode_workspace(c, n_ctas);
+  return base ? base + 256 : 0;
+}
+
+extern "C" hyq_status hyq_decode_step(const hyq_cache *c, const void *q, const void *k_new, const void *v_new,
+                                      void *q_ring, int32_t n_q, void *o, float *lse, int32_t n_ctas, void *ws,
+                                      size_t ws_bytes, void *stream) {
+  hyq_status s = hyq_check_cache(c);
+  if (s != HYQ_OK) return s;
+  if (!q || !o || !k_new || !v_new) return HYQ_ERR_INVALID;
+  if (q_ring && (n_q < 1 || n_q > 1024)) return HYQ_ERR_INVALID;
+  if (!al16(q) || !al16(o) || !al16(k_new) || !al16(v_new) || (q_ring && !al16(q_ring)) || (lse && !al16(lse)) ||
+      !al16(ws))
+    return HYQ_ERR_ALIGN;
+  if (n_ctas < 0) return HYQ_ERR_INVALID;
+  const int G = c->n_q_heads / c->n_kv_heads;
+  const int U = c->batch * c->n_kv_heads;
+  if (U > MAX_UNITS || !cost_fits(U, c->capacity, c->vl_capacity, MODE_STEP)) return HYQ_ERR_UNSUPPORTED;
+  const int N = resolve_ctas(n_ctas);
+  const size_t dws = decode_ws_bytes(G, U, N);
+  if (!ws || ws_bytes < dws + 256) return HYQ_ERR_WORKSPACE;
+  DecodeArgs a{};
+  a.B = c->batch; a.Hq = c->n_q_heads; a.Hkv = c->n_kv_heads; a.cap = c->capacity;
+  a.W = c->window; a.vl_cap = c->vl_capacity; a.U = U; a.n_ctas = N;
+  a.blocks = c->blocks;
+  a.win_k = static_cast<__half *>(c->win_k); a.win_v = static_cast<__half *>(c->win_v);
+  a.vl_k = static_cast<const __half *>(c->vl_k); a.vl_v = static_cast<const __half *>(c->vl_v);
+  a.vl_count = c->vl_count; a.seq_len = c->seq_len;
+  a.q = static_cast<const __half *>(q); a.o = static_cast<__half *>(o); a.lse = lse;
+  a.counters = static_cast<int32_t *>(ws);
+  a.part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + (static_cast<size_t>(U) * 4 + 255) / 256 * 256);
+  a.status = c->dev_status;
+  a.k_new = static_cast<const __half *>(k_new); a.v_new = static_cast<const __half *>(v_new);
+  a.q_ring = static_cast<__half *>(q_ring); a.n_q = n_q;
+  a.grid_counter = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + dws);
+  return dispatch_decode<MODE_STEP>(G, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? HYQ_OK
+                                                                                            : HYQ_ERR_CUDA;
 }
 
 extern "C" hyq_status hyq_decode_fp16(const void *q, const void *k, const void *v,
@@ -1037,7 +1186,7 @@ extern "C" hyq_status hyq_decode_fp16(const void *q, const void *k, const void *
   if (!ws || ws_bytes < decode_ws_bytes(G, U, N)) return HYQ_ERR_WORKSPACE;
   DecodeArgs a{};
   a.B = batch; a.Hq = n_q_heads; a.Hkv = n_kv_heads; a.cap = capacity; a.W = WIN; a.vl_cap = 0;
-  a.U = U; a.n_ctas = N; a.seq_len = seq_len;
+  a.U = U; a.n_ctas = N; a.seq_len = const_cast<int32_t *>(seq_len);  // read only in this mode
   a.k16 = static_cast<const __half *>(k); a.v16 = static_cast<const __half *>(v);
   a.q = static_cast<const __half *>(q); a.o = static_cast<__half *>(o); a.lse = lse;
   a.counters = static_cast<int32_t *>(ws);
@@ -1099,7 +1248,7 @@ extern "C" hyq_status hyq_decode_noalloc(const hyq_cache *c, const void *q, void
   a.B = c->batch; a.Hq = c->n_q_heads; a.Hkv = c->n_kv_heads; a.cap = c->capacity;
   a.W = c->window; a.vl_cap = c->vl_capacity; a.U = U; a.n_ctas = N;
   a.blocks = c->blocks;
-  a.win_k = static_cast<const __half *>(c->win_k); a.win_v = static_cast<const __half *>(c->win_v);
+  a.win_k = static_cast<__half *>(c->win_k); a.win_v = static_cast<__half *>(c->win_v);
   a.vl_k = static_cast<const __half *>(c->vl_k); a.vl_v = static_cast<const __half *>(c->vl_v);
   a.vl_count = c->vl_count; a.seq_len = c->seq_len;
   a.q = static_cast<const __half *>(q); a.o = static_cast<__half *>(o); a.lse = lse;

@@ -11,84 +11,19 @@
 // quantization grid is the library's (see include/hyq.h): the pages do not
 // give one.
 //
-// One row of 128 channels is handled by 16 threads; thread t of the row owns
-// channels 8t..8t+7, i.e. group g = t/4, pieces 2(t%4) and 2(t%4)+1 of the
-// packed format.  The group min/max is a 4-lane shuffle reduction; all
-// arithmetic that decides a code is IEEE fp32 with explicit round-to-nearest
-// intrinsics (no contraction into FMA, no reciprocal).
+// One row of 128 channels is handled by 16 threads (hyq_quant.cuh).
 #include "hyq_common.cuh"
+#include "hyq_quant.cuh"
 
 namespace hyq {
-
-// Quantize this thread's 8 channels (x = 16 bytes of fp16) and write its
-// share of the packed row.  `hmask` = the 16 lanes that own this row.
-__device__ __forceinline__ void quantize_part(uint4 x, int t, unsigned hmask, uint8_t *codes_row,
-                                              uint32_t *sz_row, uint32_t *status) {
-  float v[8];
-  const __half2 *hx = reinterpret_cast<const __half2 *>(&x);
-  bool finite = true;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 f = __half22float2(hx[i]);
-    v[2 * i] = f.x;
-    v[2 * i + 1] = f.y;
-  }
-  float mn = v[0], mx = v[0];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    finite = finite && isfinite(v[i]);
-    mn = fminf(mn, v[i]);
-    mx = fmaxf(mx, v[i]);
-  }
-  mn = fminf(mn, __shfl_xor_sync(hmask, mn, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 1));
-  mn = fminf(mn, __shfl_xor_sync(hmask, mn, 2));
-  mx = fmaxf(mx, __shfl_xor_sync(hmask, mx, 2));
-  if (!finite) set_status(status, HYQ_DEV_NONFINITE);
-
-  const float s32 = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-  const __half sh = __float2half_rn(s32);
-  __half zh = __float2half_rn(mn);  // exact: mn is an fp16 value
-  if (mn == 0.0f) zh = __ushort_as_half(0);
-  const float sf = __half2float(sh);
-  const float zf = __half2float(zh);
-
-  uint32_t c[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int q = 0;
-    if (sf != 0.0f) {
-      q = __float2int_rn(__fdiv_rn(__fsub_rn(v[i], zf), sf));  // ties to even
-      q = min(max(q, 0), 15);
-    }
-    c[i] = static_cast<uint32_t>(q);
-  }
-  // my bytes: piece p0 = 2(t%4): (j0, j1), piece p1 = p0 + 1: (j0, j1)
-  const uint32_t mine = (c[0] | (c[1] << 4)) | ((c[2] | (c[3] << 4)) << 8) |
-                        ((c[4] | (c[5] << 4)) << 16) | ((c[6] | (c[7] << 4)) << 24);
-  // the odd group of the pair (g = 2h+1) sits 4 lanes above the even one
-  const uint32_t other = __shfl_down_sync(hmask, mine, 4);
-  const int g = t >> 2, sub = t & 3;
-  if ((g & 1) == 0) {
-    const int h = g >> 1;
-    const int p0 = 2 * sub;
-    // word (p, h) = {g2h.j0, g2h+1.j0, g2h.j1, g2h+1.j1}
-    const uint32_t w0 = prmt(mine, other, 0x5140u);
-    const uint32_t w1 = prmt(mine, other, 0x7362u);
-    *reinterpret_cast<uint32_t *>(codes_row + 8 * p0 + 4 * h) = w0;
-    *reinterpret_cast<uint32_t *>(codes_row + 8 * (p0 + 1) + 4 * h) = w1;
-  }
-  if (sub == 0) {
-    __half2 szv = __halves2half2(sh, zh);
-    sz_row[g] = h2u(szv);
-  }
-}
 
 __global__ void __launch_bounds__(256) pack_kernel(const __half *__restrict__ x, int64_t n_rows,
                                                    int64_t stride,
                                                    const int64_t *__restrict__ dst_rows,
                                                    uint8_t *__restrict__ codes,
                                                    uint32_t *__restrict__ sz, uint32_t *status) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream is complete and visible
   const int lane = threadIdx.x & 31;
   const int t = lane & 15;
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
@@ -103,6 +38,8 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half *__restrict__ x,
 __global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half *__restrict__ k_full,
                                                       const __half *__restrict__ v_full,
                                                       int64_t n_rows) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream is complete and visible
   const int lane = threadIdx.x & 31;
   const int t = lane & 15;
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
@@ -140,6 +77,8 @@ __global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half 
 __global__ void append_kernel(hyq_cache c, const __half *__restrict__ k_new,
                               const __half *__restrict__ v_new, const __half *__restrict__ q_new,
                               __half *__restrict__ q_ring, int n_q) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream is complete and visible
   const int b = blockIdx.x;
   const int T = c.seq_len[b];
   __syncthreads();  // every thread has read seq_len[b] before it changes
@@ -197,6 +136,8 @@ __device__ __forceinline__ int find_sorted(const int32_t *a, int n, int32_t key)
 // the unit's bitmask, publish the count (0 when the list is invalid, which
 // turns step 2 into a no-op for the unit).
 __global__ void __launch_bounds__(256) vl_reset_kernel(hyq_cache c, const int32_t *__restrict__ pos, int k) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream is complete and visible
   __shared__ int s_bad;
   const int u = blockIdx.x;
   const int T = c.seq_len[u / c.n_kv_heads];
@@ -222,6 +163,8 @@ __global__ void __launch_bounds__(256) vl_reset_kernel(hyq_cache c, const int32_
 __global__ void __launch_bounds__(512) vl_gather_kernel(hyq_cache c, const int32_t *__restrict__ pos, int k,
                                                         const __half *__restrict__ k_full,
                                                         const __half *__restrict__ v_full) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream is complete and visible
   const int u = blockIdx.y;
   if (c.vl_count[u] != k) return;  // invalid list: left empty by step 1
   const int r = blockIdx.x * 32 + (threadIdx.x >> 4), part = threadIdx.x & 15;
@@ -244,6 +187,8 @@ __global__ void __launch_bounds__(512) vl_gather_kernel(hyq_cache c, const int32
 // before writing.
 __global__ void __launch_bounds__(1024) vl_recompact_kernel(hyq_cache c, const int32_t *__restrict__ pos, int k,
                                                             int32_t *n_unpromoted) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream is complete and visible
   extern __shared__ int32_t vl_list[];  // [2][vl_capacity]
   __shared__ int red[32];
   __shared__ int s_bad;
@@ -343,10 +288,10 @@ extern "C" hyq_status hyq_pack(const void *x, int64_t n_rows, int64_t row_stride
   const int64_t threads = n_rows * 16;
   const int64_t blocks = (threads + 255) / 256;
   if (blocks > 0x7FFFFFFFll) return HYQ_ERR_INVALID;
-  pack_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __half *>(x), n_rows, row_stride, dst_rows, codes,
-      static_cast<uint32_t *>(sz), dev_status);
-  return cudaGetLastError() == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
+  const cudaError_t e = launch(pack_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                                static_cast<cudaStream_t>(stream), static_cast<const __half *>(x), n_rows,
+                                row_stride, dst_rows, codes, static_cast<uint32_t *>(sz), dev_status);
+  return e == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
 }
 
 extern "C" hyq_status hyq_prefill(const hyq_cache *c, const void *k_full, const void *v_full,
@@ -358,9 +303,10 @@ extern "C" hyq_status hyq_prefill(const hyq_cache *c, const void *k_full, const 
   const int64_t n_rows = static_cast<int64_t>(c->batch) * c->n_kv_heads * c->capacity * 2;
   const int64_t blocks = (n_rows * 16 + 255) / 256;
   if (blocks > 0x7FFFFFFFll) return HYQ_ERR_INVALID;
-  prefill_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      *c, static_cast<const __half *>(k_full), static_cast<const __half *>(v_full), n_rows);
-  return cudaGetLastError() == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
+  const cudaError_t e = launch(prefill_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                                static_cast<cudaStream_t>(stream), *c, static_cast<const __half *>(k_full),
+                                static_cast<const __half *>(v_full), n_rows);
+  return e == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
 }
 
 extern "C" hyq_status hyq_append(const hyq_cache *c, const void *k_new, const void *v_new,
@@ -374,10 +320,10 @@ extern "C" hyq_status hyq_append(const hyq_cache *c, const void *k_new, const vo
     return HYQ_ERR_ALIGN;
   if (c->n_kv_heads > 32) return HYQ_ERR_UNSUPPORTED;  // 2 rows x 16 threads per kv head
   const int threads = 32 * c->n_kv_heads < 128 ? 128 : 32 * c->n_kv_heads;
-  append_kernel<<<c->batch, threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      *c, static_cast<const __half *>(k_new), static_cast<const __half *>(v_new),
-      static_cast<const __half *>(q_new), static_cast<__half *>(q_ring), n_q);
-  return cudaGetLastError() == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
+  const cudaError_t e = launch(append_kernel, dim3(c->batch), dim3(threads), 0, static_cast<cudaStream_t>(stream),
+                                *c, static_cast<const __half *>(k_new), static_cast<const __half *>(v_new),
+                                static_cast<const __half *>(q_new), static_cast<__half *>(q_ring), n_q);
+  return e == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
 }
 
 extern "C" hyq_status hyq_vl_apply(const hyq_cache *c, const int32_t *pos, int32_t k,
@@ -392,11 +338,12 @@ extern "C" hyq_status hyq_vl_apply(const hyq_cache *c, const int32_t *pos, int32
     return HYQ_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int U = c->batch * c->n_kv_heads;
+  cudaError_t e = cudaSuccess;
   if (k_full) {
-    vl_reset_kernel<<<U, 256, 0, st>>>(*c, pos, k);
-    if (k > 0)
-      vl_gather_kernel<<<dim3((k + 31) / 32, U), 512, 0, st>>>(*c, pos, k, static_cast<const __half *>(k_full),
-                                                               static_cast<const __half *>(v_full));
+    e = launch(vl_reset_kernel, dim3(U), dim3(256), 0, st, *c, pos, k);
+    if (e == cudaSuccess && k > 0)
+      e = launch(vl_gather_kernel, dim3((k + 31) / 32, U), dim3(512), 0, st, *c, pos, k,
+                 static_cast<const __half *>(k_full), static_cast<const __half *>(v_full));
   } else {
     const size_t smem = 2 * sizeof(int32_t) * static_cast<size_t>(c->vl_capacity);
     if (smem > 200 * 1024) return HYQ_ERR_UNSUPPORTED;
@@ -407,7 +354,7 @@ extern "C" hyq_status hyq_vl_apply(const hyq_cache *c, const int32_t *pos, int32
       cudaFuncSetAttribute(vl_recompact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
       attr_dev = dev;
     }
-    vl_recompact_kernel<<<U, 1024, smem, st>>>(*c, pos, k, n_unpromoted);
+    e = launch(vl_recompact_kernel, dim3(U), dim3(1024), smem, st, *c, pos, k, n_unpromoted);
   }
-  return cudaGetLastError() == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
+  return e == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
 }

@@ -264,6 +264,8 @@ __device__ __forceinline__ void tile_scores(uint32_t hi, uint32_t lo, const uint
 // Shared memory: 2 x (hi, lo) 64-key tiles, slot_of[SEL_KC], cpart[8][64].
 template <bool CACHE, int PASS>
 __global__ void __launch_bounds__(SEL_THREADS, 1) score_kernel(const SelectArgs a) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream is complete and visible
   extern __shared__ __align__(128) uint8_t sm[];
   constexpr int TILE = SEL_SUB * 256;
   uint8_t *tiles = sm;  // buf b: hi at 2b*TILE, lo at (2b+1)*TILE
@@ -431,6 +433,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) score_kernel(const SelectArgs 
 // (exclusive prefix popcount of the unit's mask), so the slot of a position
 // is one popcount away.
 __global__ void __launch_bounds__(1024) rank_kernel(const SelectArgs a) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream is complete and visible
   __shared__ int wsum[32];
   const int u = blockIdx.x;
   const int nw = a.cap / 32;
@@ -462,6 +466,8 @@ __global__ void __launch_bounds__(1024) rank_kernel(const SelectArgs a) {
 }
 
 __global__ void stats_merge_kernel(const SelectArgs a) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream is complete and visible
   const int u = blockIdx.x;
   const int T = sel_T(a, u);
   if (T < a.n_q || T > a.cap) return;
@@ -481,6 +487,8 @@ __global__ void stats_merge_kernel(const SelectArgs a) {
 
 // Exact top-k of colsum[0, n) by (value desc, position asc), ascending output.
 __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const SelectArgs a) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream is complete and visible
   __shared__ int hist[256];
   __shared__ uint32_t s_prefix, s_mask;
   __shared__ int s_need;
@@ -601,17 +609,17 @@ static cudaError_t select_launch(const SelectArgs &a, bool cache, cudaStream_t s
   const int n_items = a.U * a.n_chunks;
   const int sms = hyq_sm_count_dev();
   const dim3 grid(n_items < sms ? n_items : sms, a.n_rb);
+  cudaError_t e;
   if (cache) {
-    rank_kernel<<<a.U, 1024, 0, s>>>(a);
-    score_kernel<true, 1><<<grid, SEL_THREADS, smem, s>>>(a);
+    e = launch(rank_kernel, dim3(a.U), dim3(1024), 0, s, a);
+    if (e == cudaSuccess) e = launch(score_kernel<true, 1>, grid, dim3(SEL_THREADS), smem, s, a);
   } else {
-    score_kernel<false, 1><<<grid, SEL_THREADS, smem, s>>>(a);
+    e = launch(score_kernel<false, 1>, grid, dim3(SEL_THREADS), smem, s, a);
   }
-  stats_merge_kernel<<<a.U, 256, 0, s>>>(a);
-  if (cache) score_kernel<true, 2><<<grid, SEL_THREADS, smem, s>>>(a);
-  else score_kernel<false, 2><<<grid, SEL_THREADS, smem, s>>>(a);
-  topk_kernel<<<a.U, TOPK_THREADS, 0, s>>>(a);
-  return cudaGetLastError();
+  if (e == cudaSuccess) e = launch(stats_merge_kernel, dim3(a.U), dim3(256), 0, s, a);
+  if (e == cudaSuccess) e = launch(cache ? score_kernel<true, 2> : score_kernel<false, 2>, grid, dim3(SEL_THREADS), smem, s, a);
+  if (e == cudaSuccess) e = launch(topk_kernel, dim3(a.U), dim3(TOPK_THREADS), 0, s, a);
+  return e;
 }
 
 }  // namespace hyq

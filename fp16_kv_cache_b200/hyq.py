@@ -65,6 +65,8 @@ EXPORTS = [
     ("hyq_vl_apply", ctypes.c_int, [_CP, _P, _I32, _P, _P, _P, _P]),
     ("hyq_decode_workspace", _SZ, [_CP, _I32]),
     ("hyq_decode", ctypes.c_int, [_CP, _P, _P, _P, _I32, _P, _SZ, _P]),
+    ("hyq_decode_step_workspace", _SZ, [_CP, _I32]),
+    ("hyq_decode_step", ctypes.c_int, [_CP, _P, _P, _P, _P, _I32, _P, _P, _I32, _P, _SZ, _P]),
     ("hyq_decode_noalloc", ctypes.c_int, [_CP, _P, _P, _P, _P]),
     ("hyq_decode_fp16_workspace", _SZ, [_I32, _I32, _I32, _I32]),
     ("hyq_decode_fp16", ctypes.c_int, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _I32, _P, _SZ, _P, _P]),
@@ -223,6 +225,20 @@ def hyq_decode_workspace(cache: HybridCache, n_ctas: int = 0) -> int:
 def hyq_decode(cache: HybridCache, q, o, ws, lse=None, n_ctas: int = 0, stream=None):
     _check(lib().hyq_decode(cache.ref(), _ptr(q), _ptr(o), _ptr(lse), n_ctas, _ptr(ws),
                             ws.numel() * ws.element_size(), _stream(stream)), "hyq_decode")
+
+
+def hyq_decode_step_workspace(cache: HybridCache, n_ctas: int = 0) -> int:
+    return int(lib().hyq_decode_step_workspace(cache.ref(), n_ctas))
+
+
+def hyq_decode_step(cache: HybridCache, q, k_new, v_new, o, ws, q_ring=None, lse=None, n_ctas: int = 0,
+                    stream=None):
+    """hyq_append(cache, k_new, v_new, q, q_ring) and hyq_decode(cache, q) in
+    one launch."""
+    n_q = int(q_ring.shape[2]) if q_ring is not None else 0
+    _check(lib().hyq_decode_step(cache.ref(), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_ring), n_q, _ptr(o),
+                                 _ptr(lse), n_ctas, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "hyq_decode_step")
 
 
 def hyq_decode_noalloc(cache: HybridCache, q, o, lse=None, stream=None):

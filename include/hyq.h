@@ -240,6 +240,32 @@ hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, float *lse,
                       int32_t n_ctas, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * hyq_decode_step -- one whole decode step in a single launch: the append of
+ * hyq_append(c, k_new, v_new, q, q_ring, n_q) fused into hyq_decode(c, q,
+ * o, lse).  Results (o, lse, and the cache, ring and seq_len after the
+ * call) are identical to the two calls in sequence.  Method: HyQuant,
+ * "Two Operational Modes / Decode Stage" (the token leaving the local window
+ * is compressed to 4 bits as decoding proceeds) and "How It Works" (the
+ * decode attention over K_Q, K_VL and K_Win).
+ *   q      fp16 [B][Hq][128]: the new token's queries (decoded and, when
+ *          q_ring is non-NULL, stored in ring slot T % n_q)
+ *   k_new, v_new  fp16 [B][Hkv][128]: the new token's key and value rows
+ *   q_ring nullable fp16 [B][Hq][n_q][128]; n_q in [1, 1024] when non-NULL
+ *   o, lse, n_ctas as hyq_decode
+ *   ws     workspace of hyq_decode_step_workspace(c, n_ctas) bytes, zero-
+ *          filled before the first call and left reusable by every
+ *          completed call
+ * A sequence whose length would pass capacity is not appended: its rows get
+ * o = 0, lse = -inf and HYQ_DEV_BADLEN is raised (hyq_append leaves such a
+ * sequence unchanged too).  Errors as hyq_decode.
+ */
+size_t hyq_decode_step_workspace(const hyq_cache *c, int32_t n_ctas);
+hyq_status hyq_decode_step(const hyq_cache *c, const void *q, const void *k_new,
+                           const void *v_new, void *q_ring, int32_t n_q, void *o,
+                           float *lse, int32_t n_ctas, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/*
  * hyq_decode_noalloc -- hyq_decode without a workspace argument, for callers
  * that cannot allocate device memory: for example a plugin inside a host
  * application whose own allocator owns the whole GPU memory budget and does

@@ -1,0 +1,123 @@
+"""hyq_decode_step: the append and the decode of one step in a single launch.
+
+Its results must be identical, bit for bit, to hyq_append followed by
+hyq_decode on the same cache: the outputs, the log-sum-exp, and everything
+the append leaves behind (INT4 blocks, window, query ring, seq_len).  The
+fused path is also checked against the oracle directly.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_cases import Case, compare_decode, dev, host
+from fp16_kv_cache_b200 import hyq
+
+pytestmark = pytest.mark.gpu
+
+
+def _clone_cache(c):
+    d = hyq.HybridCache(c.B, c.Hq, c.Hkv, c.cap, c.vl_cap)
+    for name in ("blocks", "win_k", "win_v", "vl_k", "vl_v", "vl_pos", "vl_count", "seq_len"):
+        getattr(d, name).copy_(getattr(c, name))
+    return d
+
+
+def _state(c, ring):
+    torch.cuda.synchronize()
+    return {name: host(getattr(c, name)).view(np.uint8).copy()
+            for name in ("blocks", "win_k", "win_v", "vl_pos", "vl_count", "seq_len")} | \
+        {"ring": None if ring is None else host(ring).view(np.uint8).copy()}
+
+
+def _run_both(case, steps, n_q=64, seed_q=500, with_ring=True, n_ctas=0):
+    """Advance two copies of the cache: A by append + decode, B by the fused
+    step; compare every step's outputs and the final state."""
+    cfg = case.cfg
+    a_cache, b_cache = case.g, _clone_cache(case.g)
+    ring_a = ring_b = None
+    if with_ring:
+        ring_a = torch.zeros(cfg.B, cfg.Hq, n_q, 128, dtype=torch.float16, device="cuda")
+        ring_b = ring_a.clone()
+    ws_a = hyq.workspace(hyq.hyq_decode_workspace(a_cache, n_ctas))
+    ws_b = hyq.workspace(hyq.hyq_decode_step_workspace(b_cache, n_ctas))
+    for step in range(steps):
+        kn, vn = synth.step_kv(cfg, step)
+        q = dev(synth.q(cfg, seed_q + step))
+        kd, vd = dev(kn), dev(vn)
+        o_a = torch.full_like(q, float("nan"))
+        o_b = torch.full_like(q, float("nan"))
+        l_a = torch.full((cfg.B, cfg.Hq), float("nan"), dtype=torch.float32, device="cuda")
+        l_b = l_a.clone()
+        hyq.hyq_append(a_cache, kd, vd, q if with_ring else None, ring_a)
+        hyq.hyq_decode(a_cache, q, o_a, ws_a, lse=l_a, n_ctas=n_ctas)
+        hyq.hyq_decode_step(b_cache, q, kd, vd, o_b, ws_b, q_ring=ring_b, lse=l_b, n_ctas=n_ctas)
+        torch.cuda.synchronize()
+        assert torch.equal(o_a.view(torch.int16), o_b.view(torch.int16)), f"step {step}: outputs differ"
+        assert torch.equal(l_a.view(torch.int32), l_b.view(torch.int32)), f"step {step}: lse differs"
+    sa, sb = _state(a_cache, ring_a), _state(b_cache, ring_b)
+    for k in sa:
+        if sa[k] is not None:
+            assert np.array_equal(sa[k], sb[k]), f"{k} differs after {steps} steps"
+    assert a_cache.status() == 0 and b_cache.status() == 0
+    return b_cache
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,k,steps,n_ctas", [
+    (1, 8, 2, 100, 0, 40, 0),      # window filling: T_old < 128 for the first 28 steps
+    (2, 16, 4, 200, 12, 70, 0),    # exiting rows cross a 32-token block boundary
+    (1, 32, 8, 4096, 64, 33, 0),   # tiny-4k shape
+    (3, 32, 8, 1000, 30, 20, 7),   # several units per block, odd block count
+    (2, 8, 1, 517, 9, 12, 1000),   # more blocks than work
+    (1, 64, 8, 700, 20, 10, 0),    # G = 8
+])
+def test_step_equals_append_then_decode(B, Hq, Hkv, T, k, steps, n_ctas):
+    cfg = synth.custom(B, Hq, Hkv, T, k, seed=T + 7 * k, steps=steps)
+    case = Case(cfg)
+    _run_both(case, steps, n_ctas=n_ctas)
+
+
+def test_step_without_ring():
+    cfg = synth.custom(2, 16, 4, 300, 8, seed=5, steps=6)
+    _run_both(Case(cfg), 6, with_ring=False)
+
+
+def test_step_stream_matches_oracle():
+    cfg = synth.custom(2, 16, 4, 150, 10, seed=23, steps=60)
+    case = Case(cfg)
+    ring = torch.zeros(cfg.B, cfg.Hq, 64, 128, dtype=torch.float16, device="cuda")
+    ws = hyq.workspace(hyq.hyq_decode_step_workspace(case.g))
+    for step in range(cfg.steps):
+        kn, vn = synth.step_kv(cfg, step)
+        qn = synth.q(cfg, 2000 + step)
+        q = dev(qn)
+        o = torch.empty_like(q)
+        lse = torch.empty(cfg.B, cfg.Hq, dtype=torch.float32, device="cuda")
+        hyq.hyq_decode_step(case.g, q, dev(kn), dev(vn), o, ws, q_ring=ring, lse=lse)
+        case.o.append(kn, vn)
+        if step % 11 == 0 or step == cfg.steps - 1:
+            torch.cuda.synchronize()
+            oo, lo = oracle.decode(case.o, qn)
+            compare_decode(host(o.float()).astype(np.float64), host(lse).astype(np.float64), oo, lo)
+    assert np.array_equal(host(case.g.seq_len), case.o.seq_len)
+    assert case.g.status() == 0
+
+
+def test_step_past_capacity_sets_status():
+    cfg = synth.custom(1, 8, 2, 128, 0, seed=1)
+    case = Case(cfg)  # capacity 128, T = 128: no room for one more token
+    before = _state(case.g, None)
+    kn, vn = synth.step_kv(cfg, 0)
+    q = dev(synth.q(cfg, 3))
+    o = torch.full_like(q, float("nan"))
+    lse = torch.zeros(cfg.B, cfg.Hq, dtype=torch.float32, device="cuda")
+    ws = hyq.workspace(hyq.hyq_decode_step_workspace(case.g))
+    hyq.hyq_decode_step(case.g, q, dev(kn), dev(vn), o, ws, lse=lse)
+    torch.cuda.synchronize()
+    assert case.g.status() & hyq.DEV_BADLEN
+    after = _state(case.g, None)
+    for k in before:
+        if before[k] is not None:
+            assert np.array_equal(before[k], after[k]), k
+    assert torch.all(o == 0) and torch.all(torch.isinf(lse)) and torch.all(lse < 0)
