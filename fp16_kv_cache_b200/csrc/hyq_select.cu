@@ -142,50 +142,51 @@ __device__ __forceinline__ void issue_cache(const SelectArgs &a, int u, int T, i
   }
 }
 
-// Convert the raw items to fp16 hi (+ lo) tiles.  INT4: x = zero + code*scale
-// in fp32 (one rounding), hi = fp16(x), lo = fp16(x - hi).
-__device__ __forceinline__ void store_cache(const RawItems &r, uint8_t *hi, uint8_t *lo) {
+// Convert the raw items into the sub-tile: every key row holds 128 fp16
+// values, the INT4 codes as exact small integers (an INT4 key is zero_g +
+// scale_g * code, applied after the MMA) and FP16 keys as they are.  The
+// per-key tables (in the sub-tile's second 16 KB) hold scale_g as fp32
+// [4][64] at byte 0 and zero_g as fp16 [64][4] at byte 1024; FP16 and
+// padding keys get scale 1, zero 0.
+constexpr int TAB_ZERO = 1024;
+__device__ __forceinline__ void store_cache(const RawItems &r, uint8_t *hi, uint8_t *tab) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int i = threadIdx.x + SEL_THREADS * j;
     const int p = i >> 4, c = i & 15;
-    uint4 h = r.v[j], l = make_uint4(0, 0, 0, 0);
+    const int g = c >> 2;
+    uint4 h = r.v[j];
+    __half2 sz = __floats2half2_rn(1.f, 0.f);
     if (r.kind[j] == -2) {
-      const int g = c >> 2, hh = g >> 1, ii = g & 1;
+      const int hh = g >> 1, ii = g & 1;
       const uint32_t w0 = hh ? r.v[j].y : r.v[j].x;  // piece 2(c%4), word hh
       const uint32_t w1 = hh ? r.v[j].w : r.v[j].z;  // piece 2(c%4)+1
-      const __half2 sz = u2h(r.sz[j]);
-      const float sc = __low2float(sz), zr = __high2float(sz);
-      float x[8];
+      uint32_t hw[4];
 #pragma unroll
-      for (int s = 0; s < 2; ++s) {
-        const uint32_t w = s ? w1 : w0;
+      for (int s2 = 0; s2 < 2; ++s2) {
+        const uint32_t w = s2 ? w1 : w0;
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
           const uint32_t byte = (w >> (8 * (2 * jj + ii))) & 0xFFu;  // channels 2jj (lo), 2jj+1 (hi)
-          x[4 * s + 2 * jj] = fmaf(static_cast<float>(byte & 15u), sc, zr);
-          x[4 * s + 2 * jj + 1] = fmaf(static_cast<float>(byte >> 4), sc, zr);
+          hw[2 * s2 + jj] = h2u(__floats2half2_rn(static_cast<float>(byte & 15u), static_cast<float>(byte >> 4)));
         }
       }
-      uint32_t hw[4], lw[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const __half2 hv = __floats2half2_rn(x[2 * e], x[2 * e + 1]);
-        const float2 hf = __half22float2(hv);
-        hw[e] = h2u(hv);
-        lw[e] = h2u(__floats2half2_rn(x[2 * e] - hf.x, x[2 * e + 1] - hf.y));
-      }
       h = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      l = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      sz = u2h(r.sz[j]);
+    } else if (r.kind[j] == -3) {
+      h = make_uint4(0, 0, 0, 0);
     }
     *reinterpret_cast<uint4 *>(hi + tile_off(p, c)) = h;
-    *reinterpret_cast<uint4 *>(lo + tile_off(p, c)) = l;
+    if ((c & 3) == 0) {
+      reinterpret_cast<float *>(tab)[g * SEL_SUB + p] = __low2float(sz);
+      reinterpret_cast<__half *>(tab + TAB_ZERO)[p * 4 + g] = __high2half(sz);
+    }
   }
 }
 
 // Q fragments of the warp's 32 rows (2 m-tiles x 8 k-steps x 4 regs).
 __device__ __forceinline__ void load_qa(const SelectArgs &a, int u, int T, int warp, int lane,
-                                        uint32_t (&qa)[2][8][4]) {
+                                        uint32_t (&qa)[2][8][4], uint32_t (&qz)[2][4]) {
   const int b = u / a.Hkv, kvh = u % a.Hkv;
   const int gid = lane >> 2, t4 = lane & 3;
 #pragma unroll
@@ -211,36 +212,85 @@ __device__ __forceinline__ void load_qa(const SelectArgs &a, int u, int T, int w
         qa[mt][ks][2 + hr] = v1;  // a2 / a3: cols 2t+8, 2t+9
       }
     }
-}
-
-// S (log2 domain) for the warp's 32 rows x 64 keys of the sub-tile.
-template <bool CACHE>
-__device__ __forceinline__ void tile_scores(uint32_t hi, uint32_t lo, const uint32_t (&qa)[2][8][4],
-                                            int lane, float (&s)[2][8][4]) {
+  // Zero-term A fragments: row r's per-group sums of q split hi + lo in
+  // fp16, at k = 0,1 (hi of groups 0,1), 2,3 (lo), 8,9 (hi of 2,3), 10,11
+  // (lo); lanes t = 0 and 1 carry them, lanes 2 and 3 zeros.
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int hr = 0; hr < 2; ++hr) {
+      float gs[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s[mt][nt][e] = 0.f;
+      for (int g = 0; g < 4; ++g) {
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float2 f0 = __half22float2(u2h(qa[mt][2 * g + e][hr]));
+          const float2 f1 = __half22float2(u2h(qa[mt][2 * g + e][2 + hr]));
+          s += (f0.x + f0.y) + (f1.x + f1.y);
+        }
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        gs[g] = s;
+      }
+      __half hi[4], lo[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        hi[g] = __float2half_rn(gs[g]);
+        lo[g] = __float2half_rn(gs[g] - __half2float(hi[g]));
+      }
+      qz[mt][hr] = (t4 == 0) ? h2u(__halves2half2(hi[0], hi[1])) : (t4 == 1) ? h2u(__halves2half2(lo[0], lo[1])) : 0u;
+      qz[mt][2 + hr] = (t4 == 0) ? h2u(__halves2half2(hi[2], hi[3])) : (t4 == 1) ? h2u(__halves2half2(lo[2], lo[3])) : 0u;
+    }
+}
+
+// S (log2 domain) for the warp's 32 rows x 64 keys of the sub-tile.
+// Prefill mode: the tile holds FP16 keys, S = Q K^T.  Cache mode: per group
+// g of 32 channels, S += scale_g * (Q_g . tile_g) with the scale applied in
+// fp32 per key, plus sum_g zero_g * qsum_g as one more MMA per 16 rows.
+template <bool CACHE>
+__device__ __forceinline__ void tile_scores(uint32_t hi, uint32_t tab, const uint32_t (&qa)[2][8][4],
+                                            const uint32_t (&qz)[2][4], int lane, float (&s)[2][8][4]) {
   // ldmatrix x4 row addresses: lanes 8j..8j+7 address key rows (nt*8 + lane%8)
   // at chunk (2*kp + j) for matrices j = 0..3 (two k-steps per load)
   const int kr = lane & 7, jm = lane >> 3;
+  const int gid = lane >> 2, t4 = lane & 3;
 #pragma unroll
   for (int nt = 0; nt < 8; ++nt) {
 #pragma unroll
-    for (int kp = 0; kp < 4; ++kp) {
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s[mt][nt][e] = 0.f;
+    if (CACHE) {
+      const uint2 z = lds64(tab + TAB_ZERO + (nt * 8 + gid) * 8);  // zeros of key nt*8 + gid
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) mma16816(s[mt][nt], qz[mt][0], qz[mt][1], qz[mt][2], qz[mt][3], z.x, z.y);
+    }
+#pragma unroll
+    for (int kp = 0; kp < 4; ++kp) {  // kp = group g: channels 32g .. 32g + 31
       const int p = nt * 8 + kr, c = 4 * kp + jm;
       uint32_t b0, b1, b2, b3;
       ldsm_x4(hi + tile_off(p, c), b0, b1, b2, b3);
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        mma16816(s[mt][nt], qa[mt][2 * kp][0], qa[mt][2 * kp][1], qa[mt][2 * kp][2], qa[mt][2 * kp][3], b0, b1);
-        mma16816(s[mt][nt], qa[mt][2 * kp + 1][0], qa[mt][2 * kp + 1][1], qa[mt][2 * kp + 1][2],
-                 qa[mt][2 * kp + 1][3], b2, b3);
-      }
       if (CACHE) {
-        ldsm_x4(lo + tile_off(p, c), b0, b1, b2, b3);
+        float sg[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          mma16816(sg[mt], qa[mt][2 * kp][0], qa[mt][2 * kp][1], qa[mt][2 * kp][2], qa[mt][2 * kp][3], b0, b1);
+          mma16816(sg[mt], qa[mt][2 * kp + 1][0], qa[mt][2 * kp + 1][1], qa[mt][2 * kp + 1][2],
+                   qa[mt][2 * kp + 1][3], b2, b3);
+        }
+        // scales of the lane's two key columns nt*8 + 2t, nt*8 + 2t + 1
+        float2 sc;
+        asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(sc.x), "=f"(sc.y)
+                     : "r"(tab + (kp * SEL_SUB + nt * 8 + 2 * t4) * 4));
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          s[mt][nt][0] += sc.x * sg[mt][0];
+          s[mt][nt][1] += sc.y * sg[mt][1];
+          s[mt][nt][2] += sc.x * sg[mt][2];
+          s[mt][nt][3] += sc.y * sg[mt][3];
+        }
+      } else {
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
           mma16816(s[mt][nt], qa[mt][2 * kp][0], qa[mt][2 * kp][1], qa[mt][2 * kp][2], qa[mt][2 * kp][3], b0, b1);
@@ -268,7 +318,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) score_kernel(const SelectArgs 
   pdl_wait();     // earlier work on the stream is complete and visible
   extern __shared__ __align__(128) uint8_t sm[];
   constexpr int TILE = SEL_SUB * 256;
-  uint8_t *tiles = sm;  // buf b: hi at 2b*TILE, lo at (2b+1)*TILE
+  uint8_t *tiles = sm;  // buf b: keys at 2b*TILE, cache-mode scale/zero tables at (2b+1)*TILE
   int *slot_of = reinterpret_cast<int *>(sm + 4 * TILE);
   float *cpart = reinterpret_cast<float *>(sm + 4 * TILE + SEL_KC * 4);
   const int rb = blockIdx.y;
@@ -278,7 +328,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) score_kernel(const SelectArgs 
   const int gid = lane >> 2, t4 = lane & 3;
   const int n_items = a.U * a.n_chunks;
   const uint32_t tiles_s = smem_u32(tiles);
-  uint32_t qa[2][8][4];
+  uint32_t qa[2][8][4], qz[2][4];
   int q_unit = -1, q_T = -1;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
     const int u = item / a.n_chunks, chunk = item % a.n_chunks;
@@ -315,7 +365,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) score_kernel(const SelectArgs 
       issue_fp16(a, u, k0, k1, tiles_s);
     }
     if (u != q_unit || T != q_T) {
-      load_qa(a, u, T, warp, lane, qa);
+      load_qa(a, u, T, warp, lane, qa, qz);
       q_unit = u;
       q_T = T;
     }
@@ -351,7 +401,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) score_kernel(const SelectArgs 
       __syncthreads();
       float s[2][8][4];
       if (has_rows) {
-        tile_scores<CACHE>(tiles_s + cur * 2 * TILE, tiles_s + cur * 2 * TILE + TILE, qa, lane, s);
+        tile_scores<CACHE>(tiles_s + cur * 2 * TILE, tiles_s + cur * 2 * TILE + TILE, qa, qz, lane, s);
         if (PASS == 1) {
 #pragma unroll
           for (int mt = 0; mt < 2; ++mt)
@@ -472,125 +522,192 @@ __global__ void stats_merge_kernel(const SelectArgs a) {
   const int T = sel_T(a, u);
   if (T < a.n_q || T > a.cap) return;
   const int nch = (T + SEL_KC - 1) / SEL_KC;
+  constexpr int MB = 8;  // chunk partials loaded at once
   for (int r = threadIdx.x; r < a.R; r += blockDim.x) {
     const float2 *p = a.stats_part + static_cast<int64_t>(u) * a.n_chunks * SEL_MAX_ROWS + r;
-    float M = -INFINITY;
-    for (int c = 0; c < nch; ++c) M = fmaxf(M, p[static_cast<int64_t>(c) * SEL_MAX_ROWS].x);
-    float L = 0.f;
-    for (int c = 0; c < nch; ++c) {
-      const float2 v = p[static_cast<int64_t>(c) * SEL_MAX_ROWS];
-      if (v.x != -INFINITY) L += v.y * fast_exp2(v.x - M);
+    // log-sum-exp merge of the chunk partials in chunk order, MB loads in flight
+    float M = -INFINITY, L = 0.f;
+    for (int c0 = 0; c0 < nch; c0 += MB) {
+      float2 v[MB];
+#pragma unroll
+      for (int j = 0; j < MB; ++j)
+        v[j] = (c0 + j < nch) ? p[static_cast<int64_t>(c0 + j) * SEL_MAX_ROWS] : make_float2(-INFINITY, 0.f);
+      float bm = M;
+#pragma unroll
+      for (int j = 0; j < MB; ++j) bm = fmaxf(bm, v[j].x);
+      if (bm == -INFINITY) continue;
+      L = (M == -INFINITY) ? 0.f : L * fast_exp2(M - bm);
+#pragma unroll
+      for (int j = 0; j < MB; ++j)
+        if (v[j].x != -INFINITY) L += v[j].y * fast_exp2(v[j].x - bm);
+      M = bm;
     }
     a.stats[static_cast<int64_t>(u) * SEL_MAX_ROWS + r] = make_float2(M, L > 0.f ? 1.f / L : 0.f);
   }
 }
 
 // Exact top-k of colsum[0, n) by (value desc, position asc), ascending output.
+// One block of TOPK_THREADS per unit.  The column sums (non-negative floats,
+// which order like their bit patterns) are staged in shared memory when they
+// fit.  A radix select over the bit patterns, one byte per pass from the
+// top, finds the k-th largest value tau and how many of the values equal to
+// tau are taken (lowest positions first).  Counts go to one private 256-bin
+// histogram per warp (the values crowd into a few bins, so block-wide atomics
+// would serialize); after the first byte only the candidates (values whose
+// top byte is the selected digit) are visited again.  Each warp then owns a
+// contiguous run of positions: it counts, the counts are scanned once, and
+// it writes its selected positions in order.
+constexpr int TOPK_SMEM_VALS = 32768;  // values staged in shared memory (128 KB; positions fit uint16)
+constexpr int TOPK_WARPS = TOPK_THREADS / 32;
+
 __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const SelectArgs a) {
   pdl_trigger();  // the next kernel may be scheduled
   pdl_wait();     // earlier work on the stream is complete and visible
+  extern __shared__ uint32_t tk_smem[];  // [TOPK_SMEM_VALS] values, then [TOPK_SMEM_VALS] uint16 candidates
+  __shared__ int whist[TOPK_WARPS][256];
   __shared__ int hist[256];
-  __shared__ uint32_t s_prefix, s_mask;
-  __shared__ int s_need;
-  __shared__ int wsum[TOPK_THREADS / 32][2];
-  const int u = blockIdx.x;
+  __shared__ int wcnt[TOPK_WARPS][2];
+  __shared__ int s_digit, s_need, s_ncand;
+  const int u = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int T = sel_T(a, u);
   const int k = a.k;
   int32_t *out = a.out_pos + static_cast<int64_t>(u) * k;
   if (T < a.n_q || T > a.cap || T - a.W < k) {
-    if (threadIdx.x == 0) set_status(a.status, HYQ_DEV_BADLEN);
-    for (int i = threadIdx.x; i < k; i += blockDim.x) out[i] = -1;
+    if (tid == 0) set_status(a.status, HYQ_DEV_BADLEN);
+    for (int i = tid; i < k; i += blockDim.x) out[i] = -1;
     return;
   }
   const int n = T - a.W;
   float *fin = a.colsum + static_cast<int64_t>(u) * a.cap;
-  if (a.n_rb > 1 || fin != a.colsum_part + static_cast<int64_t>(u) * a.cap) {
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      float v = 0.f;
+  const bool reduce = a.n_rb > 1 || fin != a.colsum_part + static_cast<int64_t>(u) * a.cap;
+  const bool staged = n <= TOPK_SMEM_VALS;
+  for (int i = tid; i < n; i += blockDim.x) {
+    float v;
+    if (reduce) {
+      v = 0.f;
       for (int z = 0; z < a.n_rb; ++z) v += a.colsum_part[(static_cast<int64_t>(z) * a.U + u) * a.cap + i];
       fin[i] = v;
+    } else {
+      v = fin[i];
+    }
+    if (staged) tk_smem[i] = __float_as_uint(v);
+  }
+  if (tid == 0) s_ncand = 0;
+  __syncthreads();
+  if (k == 0) return;
+  const uint32_t *vals = staged ? tk_smem : reinterpret_cast<const uint32_t *>(fin);
+  uint16_t *cand = reinterpret_cast<uint16_t *>(tk_smem + TOPK_SMEM_VALS);  // candidate positions (< 2^15)
+  const bool use_cand = staged;
+
+  uint32_t prefix = 0, mask = 0;
+  int need = k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = lane; i < 256; i += 32) whist[w][i] = 0;
+    __syncwarp();
+    const int ncand = s_ncand;
+    const bool from_cand = pass > 0 && use_cand;
+    const int m = from_cand ? ncand : n;
+    for (int base = 0; base < m; base += blockDim.x) {  // whole warps iterate together
+      const int j = base + tid;
+      uint32_t b = 0;
+      bool act = false;
+      if (j < m) {
+        b = vals[from_cand ? cand[j] : j];
+        act = (b & mask) == prefix;
+      }
+      const unsigned am = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const uint32_t bin = (b >> shift) & 255u;
+        const unsigned peers = __match_any_sync(am, bin);
+        if (lane == __ffs(peers) - 1) atomicAdd(&whist[w][bin], __popc(peers));  // private to the warp: no contention
+      }
     }
     __syncthreads();
+    if (tid < 256) {
+      int c = 0;
+#pragma unroll 8
+      for (int q = 0; q < TOPK_WARPS; ++q) c += whist[q][tid];
+      hist[tid] = c;
+    }
+    __syncthreads();
+    if (w == 0) {
+      // suffix counts over bins 255 .. 0: lane l holds bins 255 - 8l .. 248 - 8l
+      int h[8], sum = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        h[e] = hist[255 - 8 * lane - e];
+        sum += h[e];
+      }
+      int x = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      int run = x - sum;  // count of bins above this lane's first bin
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (run < need && run + h[e] >= need) {
+          s_digit = 255 - 8 * lane - e;
+          s_need = need - run;
+        }
+        run += h[e];
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(s_digit) << shift;
+    mask |= 255u << shift;
+    need = s_need;
+    if (pass == 0 && use_cand) {
+      // candidates for the lower bytes: values whose top byte is the digit
+      for (int base = 0; base < n; base += blockDim.x) {
+        const int j = base + tid;
+        const bool c = j < n && (vals[j] & mask) == prefix;
+        const unsigned bal = __ballot_sync(0xffffffffu, c);
+        int slot0 = 0;
+        if (lane == 0 && bal) slot0 = atomicAdd(&s_ncand, __popc(bal));
+        slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+        if (c) cand[slot0 + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(j);
+      }
+    }
+    __syncthreads();  // s_digit, s_need, s_ncand, whist and hist are reused
   }
-  const uint32_t *bits = reinterpret_cast<const uint32_t *>(fin);
-  if (threadIdx.x == 0) {
-    s_prefix = 0;
-    s_mask = 0;
-    s_need = k;
+  // tau = prefix: take every value > tau and the first `need` values == tau.
+  // Warp w owns positions [w * per, (w + 1) * per).
+  const uint32_t tau = prefix;
+  const int per = ((n + TOPK_WARPS - 1) / TOPK_WARPS + 31) / 32 * 32;
+  const int beg = min(n, w * per), end = min(n, beg + per);
+  int n_gt = 0, n_eq = 0;
+  for (int j = beg + lane; j < beg + per; j += 32) {  // per is a multiple of 32: whole warps iterate
+    const bool in = j < end;
+    const uint32_t b = in ? vals[j] : 0u;
+    n_gt += __popc(__ballot_sync(0xffffffffu, in && b > tau));
+    n_eq += __popc(__ballot_sync(0xffffffffu, in && b == tau));
+  }
+  if (lane == 0) {
+    wcnt[w][0] = n_gt;
+    wcnt[w][1] = n_eq;
   }
   __syncthreads();
-  if (k > 0) {
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-      __syncthreads();
-      const uint32_t pre = s_prefix, msk = s_mask;
-      // warp-aggregated: one shared-memory atomic per distinct bin per warp
-      for (int base = 0; base < n; base += blockDim.x) {
-        const int i = base + threadIdx.x;
-        const uint32_t b = (i < n) ? bits[i] : 0u;
-        const bool act = (i < n) && ((b & msk) == pre);
-        const unsigned am = __ballot_sync(0xffffffffu, act);
-        if (act) {
-          const uint32_t bin = (b >> shift) & 255u;
-          const unsigned peers = __match_any_sync(am, bin);
-          if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
-        }
-      }
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        int need = s_need, cum = 0, d = 255;
-        for (; d > 0; --d) {
-          if (cum + hist[d] >= need) break;
-          cum += hist[d];
-        }
-        s_need = need - cum;
-        s_prefix = pre | (static_cast<uint32_t>(d) << shift);
-        s_mask = msk | (255u << shift);
-      }
-      __syncthreads();
-    }
+  int gt_before = 0, eq_before = 0;
+  for (int q = 0; q < w; ++q) {
+    gt_before += wcnt[q][0];
+    eq_before += wcnt[q][1];
   }
-  // compaction in position order: contiguous chunk per thread
-  const uint32_t tau = s_prefix;
-  const int need_eq = (k > 0) ? s_need : 0;
-  const int per = (n + blockDim.x - 1) / blockDim.x;
-  const int beg = min(n, static_cast<int>(threadIdx.x) * per), end = min(n, beg + per);
-  int n_gt = 0, n_eq = 0;
-  if (k > 0)
-    for (int i = beg; i < end; ++i) {
-      const uint32_t b = bits[i];
-      n_gt += b > tau;
-      n_eq += b == tau;
-    }
-  // block exclusive scans of n_eq, then of the selected counts
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  auto block_excl = [&](int v, int which) {
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == 31) wsum[w][which] = x;
-    __syncthreads();
-    int pre = 0;
-    for (int q = 0; q < w; ++q) pre += wsum[q][which];
-    return pre + x - v;
-  };
-  const int eq_before = block_excl(n_eq, 0);
-  const int take_eq = max(0, min(n_eq, need_eq - eq_before));
-  const int sel_before = block_excl(n_gt + take_eq, 1);
-  if (k > 0) {
-    int o = sel_before, eq_seen = 0;
-    for (int i = beg; i < end; ++i) {
-      const uint32_t b = bits[i];
-      bool take = b > tau;
-      if (b == tau) {
-        take = eq_seen < take_eq;
-        ++eq_seen;
-      }
-      if (take && o < k) out[o++] = i;
-    }
+  const int take_eq_before = min(eq_before, need);  // equal values taken by the warps before this one
+  int o = gt_before + take_eq_before, eq_seen = eq_before;
+  for (int j = beg + lane; j < beg + per; j += 32) {
+    const bool in = j < end;
+    const uint32_t b = in ? vals[j] : 0u;
+    const bool gt = in && b > tau, eq = in && b == tau;
+    const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && eq_seen + __popc(eqb & ((1u << lane) - 1u)) < need);
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    const int pos = o + __popc(tb & ((1u << lane) - 1u));
+    if (take && pos < k) out[pos] = j;
+    o += __popc(tb);
+    eq_seen += __popc(eqb);
   }
 }
 
@@ -604,6 +721,8 @@ static cudaError_t select_launch(const SelectArgs &a, bool cache, cudaStream_t s
     cudaFuncSetAttribute(score_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     cudaFuncSetAttribute(score_kernel<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     cudaFuncSetAttribute(score_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(TOPK_SMEM_VALS * (sizeof(uint32_t) + sizeof(uint16_t))));
     attr_dev = dev;
   }
   const int n_items = a.U * a.n_chunks;
@@ -618,7 +737,7 @@ static cudaError_t select_launch(const SelectArgs &a, bool cache, cudaStream_t s
   }
   if (e == cudaSuccess) e = launch(stats_merge_kernel, dim3(a.U), dim3(256), 0, s, a);
   if (e == cudaSuccess) e = launch(cache ? score_kernel<true, 2> : score_kernel<false, 2>, grid, dim3(SEL_THREADS), smem, s, a);
-  if (e == cudaSuccess) e = launch(topk_kernel, dim3(a.U), dim3(TOPK_THREADS), 0, s, a);
+  if (e == cudaSuccess) e = launch(topk_kernel, dim3(a.U), dim3(TOPK_THREADS), TOPK_SMEM_VALS * (sizeof(uint32_t) + sizeof(uint16_t)), s, a);
   return e;
 }
 
