@@ -83,6 +83,18 @@ def decode_traffic():
     return int(d["bytes_per_launch"]) if h.hexdigest() == d.get("source_sha256") else None
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The job's time is the slowest rank's: MAX all-reduce over the process
+    group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -278,11 +290,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     clk = clocks.stop() if clocks else None
-    elapsed_ms = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), dev)
     # algorithmic bytes of every timed decode, with the VL count it saw
     # (a cache-mode re-selection keeps only rows still held in FP16)
     k_after = [c.vl_count.flatten().tolist() for c in layers]  # per unit, after the re-selection

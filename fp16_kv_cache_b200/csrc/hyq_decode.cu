@@ -9,29 +9,34 @@
 // full-precision comparator.
 //
 // Design (B200, sm_100a)
-//   * Work: per unit (batch, kv head) the positions are cut into tiles -- INT4
-//     tiles of 64 tokens (160 B per token: 64 B K codes, 16 B K scale/zero,
-//     64 B V codes, 16 B V scale/zero) and FP16 tiles of 16 rows (512 B per
-//     row).  All tiles of all units are concatenated and the launch's blocks
-//     take equal contiguous runs of tiles (split-KV with the split points
-//     chosen by tile count, so any batch/length mix keeps every SM busy).
-//   * Pipeline: one producer warp streams tiles into an 8-slot shared-memory
-//     ring with 1-D bulk copies (cp.async.bulk, no multicast) completing on
-//     mbarriers; tile i is consumed by consumer warp i % 4.
+//   * Work: per unit (batch, kv head) the positions are cut into tiles --
+//     INT4 tiles of 32 tokens (one 5136-byte cache block record: K codes, K
+//     scale/zero, V codes, V scale/zero, vertical-line bitmask) and FP16
+//     tiles of 8 rows (vertical lines, then the window).  All tiles of all
+//     units are concatenated and split over the launch's blocks by bytes
+//     read (cost 5 per INT4 tile, 4 per FP16 tile), so any batch/length mix
+//     fills every SM (split-KV, stream-K style).
+//   * One block per SM, 12 compute warps.  Block-local tile i belongs to
+//     warp i % 12, which issues its own 1-D bulk copies (cp.async.bulk, no
+//     multicast) into a private 2-slot ring with mbarrier transaction counts;
+//     every wait is bounded by %globaltimer.
 //   * Math: Q.K and P.V run on the tensor cores (mma.sync m16n8k16, fp16 in,
 //     fp32 accumulate), tokens on the M side so a 16-token slice is one MMA
 //     row block and the G <= 8 query heads of the unit fill N.  INT4 codes
-//     enter the MMA as exact small integers (nibble -> fp16 by exponent
-//     bias); the per-(token, group) scale and zero are applied in fp32:
-//       s = sum_g scale_g * (q_g . code_g) + zero_g * sum(q_g)
+//     enter the MMA as exact fp16 subnormals; the per-(token, group) scale is
+//     applied in fp32 and both zero-point terms are one more MMA each:
+//       s = sum_g scale_g * (q_g . code_g) + sum_g zero_g * sum(q_g)
 //       o += sum_t (p_t * vscale_tg) * vcode_t + sum_t p_t * vzero_tg.
 //     The softmax is fp32 online (running max / sum, exp2 domain), reduced
 //     across lanes with warp shuffles; scores of skipped or padded tokens are
 //     -inf.  Positions held in the vertical-line segment are skipped in the
-//     INT4 sweep through the cache's bitmask.
-//   * Combine: a block that finishes a unit writes O directly; otherwise it
-//     writes its (max, sum, acc) partial and the last block to finish the
-//     unit (atomic tile counter) merges the partials by log-sum-exp.
+//     INT4 sweep through the record's bitmask.
+//   * Combine: the 12 warps of a block merge through shared memory; a block
+//     that finishes a unit writes O directly; otherwise it writes its
+//     (max, sum, acc) partial and the last block to finish the unit (atomic
+//     tile counter) merges the partials by log-sum-exp.
+//   * MODE_STEP (hyq_decode_step) fuses the append of the new token into the
+//     same launch (see "fused step" below).
 #include "hyq_common.cuh"
 #include "hyq_quant.cuh"
 

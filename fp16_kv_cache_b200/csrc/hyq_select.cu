@@ -2,11 +2,11 @@
 // unit's G query heads against its keys, softmax each query row, sum the
 // probabilities down every key column, keep the k largest column sums.
 //
-// Method: HyQuant.  wpnews.pro summary: the detector "accumulates query
-// vectors, runs a matrix multiplication every 64 tokens, and sums columns";
-// hotpaper.ai summary: vertical-line tokens are chosen by column-wise
-// attention score and are fewer than 5% of tokens; aifromscratch.in
-// explainer, "What to Watch For": a top-5% threshold.  Readings (the pages
+// Method: HyQuant.  wpnews.pro summary: the detector collects the recent
+// queries and, every 64 tokens, multiplies them against the keys and adds
+// up each key's column; hotpaper.ai summary: the vertical-line tokens, under
+// 5% of all, are the keys with the largest column totals of attention;
+// aifromscratch.in explainer, "What to Watch For": a top-5% cut.  Readings (the pages
 // are silent): the scores are post-softmax probabilities with scale
 // 1/sqrt(128); the column sum runs over the 64 queries and the G query heads
 // that share the KV head; query i sits at position T - n_q + i and sees keys

@@ -10,9 +10,10 @@
  * of the last 128 tokens stay in FP16; decode dequantizes on the fly inside
  * the attention kernel.  Sources: aifromscratch.in explainer, sections "How
  * It Works" (three token classes) and "Two Operational Modes / Decode Stage"
- * (fused dequantization); wpnews.pro summary (the detector accumulates
- * queries, runs a matrix multiplication every 64 tokens and sums columns);
- * hotpaper.ai summary (column-wise attention score, < 5% of tokens).
+ * (fused dequantization); wpnews.pro summary (the detector keeps recent
+ * queries and every 64 tokens scores them against the keys, totalling each
+ * key's column); hotpaper.ai summary (selection by column totals of
+ * attention, under 5% of tokens).
  *
  * Conventions for every entry point
  *   - Memory: every pointer is DEVICE memory owned by the caller, unless the
@@ -74,8 +75,8 @@ typedef enum {
  * conversion pairs two channels of one group per 32-bit word.)
  * Scale/zero row: fp16 {scale_0, zero_0, scale_1, zero_1, ..., zero_3}.
  *
- * Quantizer (the pages give only "4-bit for both keys and values"; this
- * grid is fixed by the library): per group, mn/mx = min/max; scale =
+ * Quantizer (the pages fix only the bit width, 4 bits for keys and for
+ * values; this grid is fixed by the library): per group, mn/mx = min/max; scale =
  * fp16(fp32(mx - mn) / 15) with fp32 IEEE round-to-nearest-even; zero = mn
  * (a -0 minimum is stored as +0); code = 0 if scale == 0, else
  * clamp(round_half_even(fp32(x - zero) / fp32(scale)), 0, 15), computed with

@@ -59,7 +59,7 @@ uint16_t hyqo_float_to_half(float f) {
 static float half_to_float(uint16_t h) { return (float)hyqo_half_to_double(h); }
 
 /* ------------------------------------------------------------------------
- * Quantizer.  The pages only say "4-bit for both keys and values"; the grid
+ * Quantizer.  The pages fix only the bit width (4 bits, keys and values); the grid
  * used here is asymmetric min/max over groups of 32 contiguous channels of
  * one token, fp16 scale = (max-min)/15 and fp16 zero = min, codes by
  * round-half-to-even of (x - zero)/scale clamped to [0, 15], decided in fp32.
@@ -341,9 +341,9 @@ int hyqo_decode_fp16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 /* ------------------------------------------------------------------------
  * Vertical-line selection.  Reading of the detector description: the last
  * n_q queries of every query head of the group are scored against all keys
- * (the "matrix multiplication"), each query row is turned into attention
- * probabilities by a causal softmax, and the probabilities are summed down
- * each key column ("sums columns" / "column-wise attention score").  The k
+ * (the pages' periodic matrix product), each query row is turned into
+ * attention probabilities by a causal softmax, and the probabilities are
+ * summed down each key column (the pages' column totals).  The k
  * largest column sums among positions older than the window are kept.
  * ---------------------------------------------------------------------- */
 typedef struct {

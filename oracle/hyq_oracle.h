@@ -9,10 +9,10 @@
  *   - aifromscratch.in explainer, "How It Works" (three token classes: K_VL,
  *     K_Win = last 128 tokens, K_Q = 4-bit keys and values) and
  *     "Two Operational Modes / Decode Stage" (fused dequant + attention);
- *   - wpnews.pro summary (the vertical-line detector accumulates queries,
- *     runs a matmul every 64 tokens and sums columns);
- *   - hotpaper.ai summary (vertical lines chosen by column-wise attention
- *     score, < 5% of tokens).
+ *   - wpnews.pro summary (the vertical-line detector keeps recent queries and
+ *     every 64 tokens scores them against the keys, totalling each column);
+ *   - hotpaper.ai summary (vertical lines chosen by column totals of
+ *     attention, under 5% of tokens).
  * Where the pages leave a step open (quantizer grid, scale format, softmax
  * before the column sum, GQA grouping, re-selection semantics) the reading
  * used is stated at each function below.
