@@ -361,3 +361,31 @@ def test_vl_apply_cache_mode_matches_oracle():
     og, lg = case.decode_gpu(q)
     oo, lo = oracle.decode(case.o, q)
     compare_decode(og, lg, oo, lo)
+
+
+def test_select_long_context_global_path():
+    """More candidates than the top-k stages in shared memory (n > 32768):
+    the radix passes read the column sums from global memory."""
+    cfg = synth.custom(1, 8, 2, 40000, 100, seed=41)
+    case = Case(cfg)
+    qs = synth.qsel(cfg, 0)[None]
+    pos_g, cs_g = _select_gpu(case, dev(qs), cfg.k, k_full=case.Kd)
+    pos_o, cs_o, margin = oracle.select_vl(case.o, qs, cfg.k, k_full=case.K)
+    _check_selection(pos_g, cs_g, pos_o, cs_o, margin, cfg.T, 128, [(0, 0), (0, 1)])
+
+
+@pytest.mark.parametrize("k", [1, 50, 472])
+def test_select_mass_ties_take_lowest_positions(k):
+    """Every key identical and visible to every selection query: all column
+    sums are equal (fixed summation order), so the k lowest positions win;
+    k = 472 takes every candidate."""
+    cfg = synth.custom(1, 8, 2, 600, 0, seed=9)
+    K, V, _ = synth.kv_full(cfg, 640)
+    K[:, :, :600] = K[0, 0, 5]
+    case = Case(cfg, vl=np.zeros((1, 2, 0), np.int32), cap=640, vl_cap=472)
+    qs = synth.qsel(cfg, 0)[None]
+    pos_g, cs_g = _select_gpu(case, dev(qs), k, k_full=dev(K))
+    n = 600 - 128
+    for h in range(2):
+        assert np.all(cs_g[0, h, :n] == cs_g[0, h, 0])
+        assert list(pos_g[0, h]) == list(range(k))
