@@ -30,6 +30,8 @@
 // window and vertical-line rows, and INT4 rows dequantized as
 // zero + code * scale in fp32 and split into two fp16 terms hi + lo (both
 // multiplied on the tensor cores) so the dequantized key keeps ~22 bits.
+#include <algorithm>
+
 #include "hyq_common.cuh"
 
 extern "C" int32_t hyq_sm_count(void);  // hyq_api.cu
@@ -38,10 +40,9 @@ namespace hyq {
 
 static int hyq_sm_count_dev() { return hyq_sm_count(); }
 
-constexpr int SEL_SUB = 64;       // keys per shared-memory sub-tile
 constexpr int SEL_KC = 512;       // keys per work item (chunk)
 constexpr int SEL_MAX_ROWS = 512; // n_q * G
-constexpr int SEL_BLOCK_ROWS = 256;  // query rows per block (8 warps x 32)
+constexpr int SEL_BLOCK_ROWS = SEL_MAX_ROWS;  // every query row of a unit in one block
 constexpr int TOPK_THREADS = 1024;
 constexpr float SEL_SCALE = 0.12751743082459868f;  // log2(e) / sqrt(128)
 
@@ -63,274 +64,247 @@ struct SelectArgs {
   uint32_t *status;
 };
 
-// ldmatrix x4: four 8x8 b16 matrices, row addresses from lanes 0-7, 8-15, ...
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
-                                        uint32_t &r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-// Swizzled offset of 16-byte chunk c (0..15) of key row p in a [64][128] fp16
-// tile: chunk index XOR (p & 7) keeps ldmatrix row reads conflict free.
-__device__ __forceinline__ uint32_t tile_off(int p, int c) {
-  return static_cast<uint32_t>(p * 256 + ((c ^ (p & 7)) << 4));
-}
-
 __device__ __forceinline__ int sel_T(const SelectArgs &a, int u) { return a.seq_len[u / a.Hkv]; }
 
-// One block = 256 threads; a 64-key sub-tile is 1024 items (key, 16-byte
-// chunk), 4 per thread: item i = threadIdx.x + 256 j -> key i / 16, chunk i % 16.
-constexpr int SEL_THREADS = 256;
+// ---------------------------------------------------------------- scorer
+// S = Q K^T on the 5th-generation tensor cores (tcgen05, fp16 in, fp32
+// accumulate in tensor memory).  One block of 8 warps per SM walks the
+// (unit, 512-key chunk) items.  Per unit the R query rows sit in shared
+// memory as row blocks of 128 (the MMA's M); per sub-tile of 128 keys (the
+// MMA's N) the keys are written to shared memory as fp16 -- in cache mode an
+// INT4 key is dequantized as zero + code * scale in fp32 and stored as
+// hi + lo fp16 (both multiplied, so the key keeps ~22 bits), FP16 keys as
+// they are -- and one thread issues the MMAs into the accumulators (one per
+// row block, 128 columns each) and commits them to an mbarrier.  Both
+// operands are K-major with the 128-byte swizzle.  The epilogue reads the
+// accumulators with tcgen05.ld: warp w owns rows 32 (w % 4) .. + 31 of each
+// row block and columns 64 (w / 4) .. + 63 of the sub-tile.
+constexpr int TC_THREADS = 256;
+constexpr int TC_NK = 128;               // keys per sub-tile
+constexpr int TC_TILE = TC_NK * 256;     // bytes of a [128][128] fp16 tile
+constexpr int TC_MAX_RB = SEL_MAX_ROWS / 128;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+// Byte offset of element (row r, channel k) in a [128][128] fp16 K-major tile
+// with the 128-byte swizzle: channels 0-63 and 64-127 form two 16 KB halves;
+// within a half, row r is 128 bytes at r * 128 and its 16-byte chunk c sits
+// at position c ^ (r % 8).
+__device__ __forceinline__ uint32_t sw128_off(int r, int k) {
+  const int kb = k >> 6, chunk = (k & 63) >> 3;
+  return kb * (TC_NK * 128) + r * 128 + ((chunk ^ (r & 7)) << 4) + (k & 7) * 2;
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// Shared-memory matrix descriptor of k-step ks (16 channels) of such a tile:
+// start address, leading offset 16 B (unused with the swizzle), stride 1024 B
+// between 8-row groups, descriptor version 1, 128-byte swizzle.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t tile, int ks) {
+  const uint32_t start = tile + (ks >> 2) * (TC_NK * 128) + (ks & 3) * 32;
+  return static_cast<uint64_t>((start >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+// Instruction descriptor: fp32 accumulate, fp16 A and B, both K-major,
+// N = 128, M = 128.
+constexpr uint32_t TC_IDESC = (1u << 4) | ((uint32_t)(TC_NK >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 
-// Prefill mode: FP16 keys straight into the swizzled tile (zero past key_end).
-__device__ __forceinline__ void issue_fp16(const SelectArgs &a, int u, int key0, int key_end, uint32_t hi) {
-  const __half *base = a.k_full + static_cast<int64_t>(u) * a.cap * D;
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t ad, uint64_t bd, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n}" ::"r"(d),
+      "l"(ad), "l"(bd), "r"(TC_IDESC), "r"(accumulate), "r"(0u));
+}
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int i = threadIdx.x + SEL_THREADS * j;
-    const int p = i >> 4, c = i & 15;
-    const int key = key0 + p;
-    const bool in = key < key_end;
-    cp_async16(hi + tile_off(p, c), base + static_cast<int64_t>(in ? key : 0) * D + 8 * c, in ? 16 : 0);
-  }
-  cp_async_commit();
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// Cache mode: raw bytes of 4 items in registers (loaded before the current
-// sub-tile is computed, converted after).
-struct RawItems {
-  uint4 v[4];
-  uint32_t sz[4];
-  int kind[4];  // -1 FP16 row (window / vertical line), -2 INT4, -3 zero
+// Raw bytes of one thread's half key row (64 channels) for the next sub-tile:
+// FP16 (window, vertical line, prefill) as 8 x 16 B, INT4 as the 4 x 16 B
+// packed row plus the 16-byte scale/zero row.
+struct KeyRaw {
+  uint4 v[8];
+  int kind;  // 0 zero, 1 FP16, 2 INT4
 };
 
-__device__ __forceinline__ void issue_cache(const SelectArgs &a, int u, int T, int key0, int key_end,
-                                            const int *slot_of, int k0, RawItems &r) {
-  const int L4 = T - a.W;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int i = threadIdx.x + SEL_THREADS * j;
-    const int p = i >> 4, c = i & 15;
-    const int key = key0 + p;
-    r.v[j] = make_uint4(0, 0, 0, 0);
-    r.sz[j] = 0;
-    r.kind[j] = -3;
-    if (key >= key_end) continue;
-    if (key >= L4) {
-      r.kind[j] = -1;
-      r.v[j] = *reinterpret_cast<const uint4 *>(a.win_k + (static_cast<int64_t>(u) * a.W + key % a.W) * D + 8 * c);
-      continue;
-    }
+// Thread t loads key (t % 128) of the sub-tile, channels 64 (t / 128) .. + 63.
+template <bool CACHE>
+__device__ __forceinline__ void key_load(const SelectArgs &a, int u, int T, int key, int key_end, const int *slot_of,
+                                         int k0, int hf, KeyRaw &r) {
+  r.kind = 0;
+  if (key >= key_end) return;
+  const __half *row = nullptr;
+  if (!CACHE) {
+    row = a.k_full + (static_cast<int64_t>(u) * a.cap + key) * D;
+  } else if (key >= T - a.W) {
+    row = a.win_k + (static_cast<int64_t>(u) * a.W + key % a.W) * D;
+  } else {
     const int slot = slot_of[key - k0];
-    if (slot >= 0) {
-      r.kind[j] = -1;
-      r.v[j] = *reinterpret_cast<const uint4 *>(a.vl_k + (static_cast<int64_t>(u) * a.vl_cap + slot) * D + 8 * c);
-      continue;
-    }
-    // channels 8c..8c+7: group c / 4, pieces 2(c%4) and 2(c%4)+1
-    r.kind[j] = -2;
-    r.v[j] = *reinterpret_cast<const uint4 *>(a.blocks + kcode_off(u, key, a.cap) + 16 * (c & 3));
-    r.sz[j] = *reinterpret_cast<const uint32_t *>(a.blocks + ksz_off(u, key, a.cap) + 4 * (c >> 2));
+    if (slot >= 0) row = a.vl_k + (static_cast<int64_t>(u) * a.vl_cap + slot) * D;
   }
+  if (row) {
+    r.kind = 1;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) r.v[c] = *reinterpret_cast<const uint4 *>(row + 64 * hf + 8 * c);
+    return;
+  }
+  r.kind = 2;
+  const uint4 *codes = reinterpret_cast<const uint4 *>(a.blocks + kcode_off(u, key, a.cap));
+#pragma unroll
+  for (int c = 0; c < 4; ++c) r.v[c] = codes[c];
+  r.v[4] = *reinterpret_cast<const uint4 *>(a.blocks + ksz_off(u, key, a.cap));
 }
 
-// Convert the raw items into the sub-tile: every key row holds 128 fp16
-// values, the INT4 codes as exact small integers (an INT4 key is zero_g +
-// scale_g * code, applied after the MMA) and FP16 keys as they are.  The
-// per-key tables (in the sub-tile's second 16 KB) hold scale_g as fp32
-// [4][64] at byte 0 and zero_g as fp16 [64][4] at byte 1024; FP16 and
-// padding keys get scale 1, zero 0.
-constexpr int TAB_ZERO = 1024;
-__device__ __forceinline__ void store_cache(const RawItems &r, uint8_t *hi, uint8_t *tab) {
+// Write the thread's 8 chunks of key row kk as fp16 (hi) and, in cache mode,
+// the fp16 remainder (lo).  INT4: x = zero + code * scale in fp32 (one
+// rounding), hi = fp16(x), lo = fp16(x - hi).
+template <bool CACHE>
+__device__ __forceinline__ void key_store(const KeyRaw &r, int kk, int hf, uint8_t *hi, uint8_t *lo) {
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int i = threadIdx.x + SEL_THREADS * j;
-    const int p = i >> 4, c = i & 15;
-    const int g = c >> 2;
-    uint4 h = r.v[j];
-    __half2 sz = __floats2half2_rn(1.f, 0.f);
-    if (r.kind[j] == -2) {
-      const int hh = g >> 1, ii = g & 1;
-      const uint32_t w0 = hh ? r.v[j].y : r.v[j].x;  // piece 2(c%4), word hh
-      const uint32_t w1 = hh ? r.v[j].w : r.v[j].z;  // piece 2(c%4)+1
-      uint32_t hw[4];
+  for (int cc = 0; cc < 8; ++cc) {
+    const int c = 8 * hf + cc;  // 16-byte chunk = channels 8c .. 8c+7
+    uint4 h = make_uint4(0, 0, 0, 0), l = make_uint4(0, 0, 0, 0);
+    if (r.kind == 1) {
+      h = r.v[cc];
+    } else if (CACHE && r.kind == 2) {
+      // channels 8c .. 8c+7 are group g = c / 4, pieces 2 (c % 4) and
+      // 2 (c % 4) + 1, i.e. the 16 bytes at 16 (c % 4); word g / 2 of each
+      // 8-byte piece, byte (g % 2) of each of its channel pairs
+      const int g = c >> 2, hh = g >> 1, ii = g & 1, pc = c & 3;
+      const uint4 vv = r.v[pc];
+      const uint32_t wp0 = hh ? vv.y : vv.x;  // piece 2pc, word hh
+      const uint32_t wp1 = hh ? vv.w : vv.z;  // piece 2pc + 1, word hh
+      const uint32_t szw = (g == 0) ? r.v[4].x : (g == 1) ? r.v[4].y : (g == 2) ? r.v[4].z : r.v[4].w;
+      const __half2 sz = u2h(szw);
+      const float sc = __low2float(sz), zr = __high2float(sz);
+      uint32_t hw[4], lw[4];
 #pragma unroll
       for (int s2 = 0; s2 < 2; ++s2) {
-        const uint32_t w = s2 ? w1 : w0;
+        const uint32_t w = s2 ? wp1 : wp0;
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
           const uint32_t byte = (w >> (8 * (2 * jj + ii))) & 0xFFu;  // channels 2jj (lo), 2jj+1 (hi)
-          hw[2 * s2 + jj] = h2u(__floats2half2_rn(static_cast<float>(byte & 15u), static_cast<float>(byte >> 4)));
+          const float x0 = fmaf(static_cast<float>(byte & 15u), sc, zr);
+          const float x1 = fmaf(static_cast<float>(byte >> 4), sc, zr);
+          const __half2 hv = __floats2half2_rn(x0, x1);
+          const float2 hf2 = __half22float2(hv);
+          hw[2 * s2 + jj] = h2u(hv);
+          lw[2 * s2 + jj] = h2u(__floats2half2_rn(x0 - hf2.x, x1 - hf2.y));
         }
       }
       h = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      sz = u2h(r.sz[j]);
-    } else if (r.kind[j] == -3) {
-      h = make_uint4(0, 0, 0, 0);
+      l = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
-    *reinterpret_cast<uint4 *>(hi + tile_off(p, c)) = h;
-    if ((c & 3) == 0) {
-      reinterpret_cast<float *>(tab)[g * SEL_SUB + p] = __low2float(sz);
-      reinterpret_cast<__half *>(tab + TAB_ZERO)[p * 4 + g] = __high2half(sz);
-    }
+    const uint32_t off = sw128_off(kk, 8 * c);
+    *reinterpret_cast<uint4 *>(hi + off) = h;
+    if (CACHE) *reinterpret_cast<uint4 *>(lo + off) = l;
   }
 }
 
-// Q fragments of the warp's 32 rows (2 m-tiles x 8 k-steps x 4 regs).
-__device__ __forceinline__ void load_qa(const SelectArgs &a, int u, int T, int warp, int lane,
-                                        uint32_t (&qa)[2][8][4], uint32_t (&qz)[2][4]) {
-  const int b = u / a.Hkv, kvh = u % a.Hkv;
-  const int gid = lane >> 2, t4 = lane & 3;
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      const int row = 32 * warp + 16 * mt + gid + 8 * hr;
-      const __half *qr = nullptr;
-      if (row < a.R) {
-        const int hg = row / a.n_q, i = row % a.n_q;
-        int slot = i;
-        if (a.q_ring) slot = ((T - a.n_q + i) % a.n_q + a.n_q) % a.n_q;
-        qr = a.q + ((static_cast<int64_t>(b) * a.Hq + kvh * a.G + hg) * a.n_q + slot) * D;
-      }
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        uint32_t v0 = 0, v1 = 0;
-        if (qr) {
-          v0 = *reinterpret_cast<const uint32_t *>(qr + 16 * ks + 2 * t4);
-          v1 = *reinterpret_cast<const uint32_t *>(qr + 16 * ks + 8 + 2 * t4);
-        }
-        qa[mt][ks][hr] = v0;      // a0 / a1: cols 2t, 2t+1
-        qa[mt][ks][2 + hr] = v1;  // a2 / a3: cols 2t+8, 2t+9
-      }
-    }
-  // Zero-term A fragments: row r's per-group sums of q split hi + lo in
-  // fp16, at k = 0,1 (hi of groups 0,1), 2,3 (lo), 8,9 (hi of 2,3), 10,11
-  // (lo); lanes t = 0 and 1 carry them, lanes 2 and 3 zeros.
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      float gs[4];
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        float s = 0.f;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float2 f0 = __half22float2(u2h(qa[mt][2 * g + e][hr]));
-          const float2 f1 = __half22float2(u2h(qa[mt][2 * g + e][2 + hr]));
-          s += (f0.x + f0.y) + (f1.x + f1.y);
-        }
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        gs[g] = s;
-      }
-      __half hi[4], lo[4];
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        hi[g] = __float2half_rn(gs[g]);
-        lo[g] = __float2half_rn(gs[g] - __half2float(hi[g]));
-      }
-      qz[mt][hr] = (t4 == 0) ? h2u(__halves2half2(hi[0], hi[1])) : (t4 == 1) ? h2u(__halves2half2(lo[0], lo[1])) : 0u;
-      qz[mt][2 + hr] = (t4 == 0) ? h2u(__halves2half2(hi[2], hi[3])) : (t4 == 1) ? h2u(__halves2half2(lo[2], lo[3])) : 0u;
-    }
-}
-
-// S (log2 domain) for the warp's 32 rows x 64 keys of the sub-tile.
-// Prefill mode: the tile holds FP16 keys, S = Q K^T.  Cache mode: per group
-// g of 32 channels, S += scale_g * (Q_g . tile_g) with the scale applied in
-// fp32 per key, plus sum_g zero_g * qsum_g as one more MMA per 16 rows.
-template <bool CACHE>
-__device__ __forceinline__ void tile_scores(uint32_t hi, uint32_t tab, const uint32_t (&qa)[2][8][4],
-                                            const uint32_t (&qz)[2][4], int lane, float (&s)[2][8][4]) {
-  // ldmatrix x4 row addresses: lanes 8j..8j+7 address key rows (nt*8 + lane%8)
-  // at chunk (2*kp + j) for matrices j = 0..3 (two k-steps per load)
-  const int kr = lane & 7, jm = lane >> 3;
-  const int gid = lane >> 2, t4 = lane & 3;
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[mt][nt][e] = 0.f;
-    if (CACHE) {
-      const uint2 z = lds64(tab + TAB_ZERO + (nt * 8 + gid) * 8);  // zeros of key nt*8 + gid
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) mma16816(s[mt][nt], qz[mt][0], qz[mt][1], qz[mt][2], qz[mt][3], z.x, z.y);
-    }
-#pragma unroll
-    for (int kp = 0; kp < 4; ++kp) {  // kp = group g: channels 32g .. 32g + 31
-      const int p = nt * 8 + kr, c = 4 * kp + jm;
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(hi + tile_off(p, c), b0, b1, b2, b3);
-      if (CACHE) {
-        float sg[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          mma16816(sg[mt], qa[mt][2 * kp][0], qa[mt][2 * kp][1], qa[mt][2 * kp][2], qa[mt][2 * kp][3], b0, b1);
-          mma16816(sg[mt], qa[mt][2 * kp + 1][0], qa[mt][2 * kp + 1][1], qa[mt][2 * kp + 1][2],
-                   qa[mt][2 * kp + 1][3], b2, b3);
-        }
-        // scales of the lane's two key columns nt*8 + 2t, nt*8 + 2t + 1
-        float2 sc;
-        asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(sc.x), "=f"(sc.y)
-                     : "r"(tab + (kp * SEL_SUB + nt * 8 + 2 * t4) * 4));
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          s[mt][nt][0] += sc.x * sg[mt][0];
-          s[mt][nt][1] += sc.y * sg[mt][1];
-          s[mt][nt][2] += sc.x * sg[mt][2];
-          s[mt][nt][3] += sc.y * sg[mt][3];
-        }
-      } else {
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          mma16816(s[mt][nt], qa[mt][2 * kp][0], qa[mt][2 * kp][1], qa[mt][2 * kp][2], qa[mt][2 * kp][3], b0, b1);
-          mma16816(s[mt][nt], qa[mt][2 * kp + 1][0], qa[mt][2 * kp + 1][1], qa[mt][2 * kp + 1][2],
-                   qa[mt][2 * kp + 1][3], b2, b3);
-        }
-      }
+// Wait (bounded) for the MMAs committed to `bar` to complete phase `parity`.
+__device__ __forceinline__ void tc_wait(uint32_t bar, uint32_t parity, const SelectArgs &a, int *abort) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > 2000000000ull) {
+      set_status(a.status, HYQ_DEV_TIMEOUT);
+      *abort = 1;
+      return;
     }
   }
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[mt][nt][e] *= SEL_SCALE;
 }
 
 // PASS 1: per-row (max, sum exp) over a chunk of keys; PASS 2: column sums.
-// Persistent: block b takes work items b, b + gridDim.x, ... of the
-// (unit, chunk) space; blockIdx.y is the row block (rows 256 y .. 256 y + 255).
-// Shared memory: 2 x (hi, lo) 64-key tiles, slot_of[SEL_KC], cpart[8][64].
+// Block b takes a contiguous run of (unit, 512-key chunk) items, so the
+// query rows are loaded once per unit.  With up to 256 query rows the key
+// tiles and the accumulators are double-buffered: the MMAs of sub-tile t+1
+// run while the epilogue of t and the dequantization of t+2 proceed.
 template <bool CACHE, int PASS>
-__global__ void __launch_bounds__(SEL_THREADS, 1) score_kernel(const SelectArgs a) {
+__global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a) {
   pdl_trigger();  // the next kernel may be scheduled
-  pdl_wait();     // earlier work on the stream is complete and visible
-  extern __shared__ __align__(128) uint8_t sm[];
-  constexpr int TILE = SEL_SUB * 256;
-  uint8_t *tiles = sm;  // buf b: keys at 2b*TILE, cache-mode scale/zero tables at (2b+1)*TILE
-  int *slot_of = reinterpret_cast<int *>(sm + 4 * TILE);
-  float *cpart = reinterpret_cast<float *>(sm + 4 * TILE + SEL_KC * 4);
-  const int rb = blockIdx.y;
-  const int wl = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int warp = wl + rb * (SEL_BLOCK_ROWS / 32);  // global warp: rows 32 warp ..
-  const bool has_rows = 32 * warp < a.R;
-  const int gid = lane >> 2, t4 = lane & 3;
+  pdl_wait();     // earlier work on the stream is complete and visible (and its tensor memory freed)
+  extern __shared__ __align__(1024) uint8_t sm_raw[];
+  __shared__ uint32_t tmem_base;
+  __shared__ __align__(8) uint64_t mbar[2];
+  __shared__ int s_abort;
+  // 128-byte swizzled tiles must start on a 1024-byte boundary
+  uint8_t *sm = sm_raw + ((1024u - (smem_u32(sm_raw) & 1023u)) & 1023u);
+  const int n_rbt = (a.R + 127) / 128;
+  const int nbuf = (n_rbt <= 2) ? 2 : 1;
+  constexpr int KT = CACHE ? 2 * TC_TILE : TC_TILE;     // one key buffer: hi (+ lo)
+  uint8_t *sQ = sm;                                      // [n_rbt][32 KB]
+  uint8_t *sK = sQ + n_rbt * TC_TILE;                    // [nbuf][KT]
+  int *slot_of = reinterpret_cast<int *>(sK + nbuf * KT);               // [SEL_KC]
+  float *csum = reinterpret_cast<float *>(slot_of + SEL_KC);            // [4][128]
+  float2 *pst = reinterpret_cast<float2 *>(csum + 4 * TC_NK);           // [TC_MAX_RB][128]
+  float *moff = reinterpret_cast<float *>(pst + TC_MAX_RB * 128);       // [SEL_MAX_ROWS] pass 2: m_r - log2(1/l_r)
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, hfw = warp >> 2;  // TMEM lane quadrant, column half
+  const uint32_t acc_cols = static_cast<uint32_t>(n_rbt) * TC_NK;      // one accumulator set
+  const uint32_t need = acc_cols * nbuf;
+  const uint32_t ncols = (need <= 128) ? 128u : (need <= 256) ? 256u : 512u;
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_base)),
+                 "r"(ncols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (tid == 0) {
+    mbar_init(smem_u32(&mbar[0]), 1);
+    mbar_init(smem_u32(&mbar[1]), 1);
+    fence_barrier_init();
+    s_abort = 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_base;
+  uint32_t phase[2] = {0u, 0u};
   const int n_items = a.U * a.n_chunks;
-  const uint32_t tiles_s = smem_u32(tiles);
-  uint32_t qa[2][8][4], qz[2][4];
+  const int per = (n_items + gridDim.x - 1) / gridDim.x;
+  const int it0 = min(n_items, static_cast<int>(blockIdx.x) * per), it1 = min(n_items, it0 + per);
   int q_unit = -1, q_T = -1;
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+  const int kk = tid & 127, hfk = tid >> 7;  // key row and channel half this thread stages
+
+  // one sub-tile's MMAs into accumulator set `buf` from key buffer `buf`
+  auto issue = [&](int buf) {
+    if (tid == 0) {
+      const uint32_t kh = smem_u32(sK + buf * KT), kl = kh + TC_TILE;
+      for (int rb = 0; rb < n_rbt; ++rb)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t ad = sw128_desc(smem_u32(sQ) + rb * TC_TILE, ks);
+          const uint32_t d = tbase + buf * acc_cols + rb * TC_NK;
+          if (PASS == 1) {  // rows on M, keys on N
+            tc_mma(d, ad, sw128_desc(kh, ks), ks > 0);
+            if (CACHE) tc_mma(d, ad, sw128_desc(kl, ks), 1u);
+          } else {          // keys on M, rows on N: each TMEM lane is one key column
+            tc_mma(d, sw128_desc(kh, ks), ad, ks > 0);
+            if (CACHE) tc_mma(d, sw128_desc(kl, ks), ad, 1u);
+          }
+        }
+      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                       smem_u32(&mbar[buf]))
+                   : "memory");
+    }
+  };
+  // hand the staged tile to the tensor core (generic writes -> async proxy)
+  auto publish = [&]() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  };
+
+  for (int item = it0; item < it1 && !s_abort; ++item) {
     const int u = item / a.n_chunks, chunk = item % a.n_chunks;
     const int T = sel_T(a, u);
     if (T < a.n_q || T > a.cap || T - a.W < a.k) continue;  // reported by the top-k kernel
@@ -338,19 +312,19 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) score_kernel(const SelectArgs 
     const int k0 = chunk * SEL_KC;
     if (k0 >= key_end) {
       if (PASS == 1)
-        for (int r = threadIdx.x; r < SEL_BLOCK_ROWS; r += blockDim.x)
-          a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + rb * SEL_BLOCK_ROWS + r] =
-              make_float2(-INFINITY, 0.f);
+        for (int r = tid; r < a.R; r += TC_THREADS)
+          a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + r] = make_float2(-INFINITY, 0.f);
       continue;
     }
     const int k1 = min(key_end, k0 + SEL_KC);
-    const int nsub = (k1 - k0 + SEL_SUB - 1) / SEL_SUB;
-    __syncthreads();  // previous item fully done with shared memory
-    RawItems raw;
+    const int nsub = (k1 - k0 + TC_NK - 1) / TC_NK;
+    tc_fence_before();
+    __syncthreads();  // the previous item is done with shared and tensor memory
+    tc_fence_after();
     if (CACHE) {
       // vertical-line slot of every key of the chunk: rank of its mask bit
       const int32_t *rbase = a.rank_base + static_cast<int64_t>(u) * (a.cap / 32);
-      for (int j = threadIdx.x; j < SEL_KC; j += blockDim.x) {
+      for (int j = tid; j < SEL_KC; j += TC_THREADS) {
         const int key = k0 + j;
         int slot = -1;
         if (key < k1 && key < T - a.W) {
@@ -359,129 +333,152 @@ __global__ void __launch_bounds__(SEL_THREADS, 1) score_kernel(const SelectArgs 
         }
         slot_of[j] = slot;
       }
-      __syncthreads();
-      issue_cache(a, u, T, k0, k1, slot_of, k0, raw);
-    } else {
-      issue_fp16(a, u, k0, k1, tiles_s);
     }
     if (u != q_unit || T != q_T) {
-      load_qa(a, u, T, warp, lane, qa, qz);
+      // the unit's query rows into the swizzled row blocks (zeros past R)
+      const int b = u / a.Hkv, kvh = u % a.Hkv;
+      for (int i = tid; i < n_rbt * 128 * 16; i += TC_THREADS) {
+        const int r = i >> 4, c = i & 15;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < a.R) {
+          const int hg = r / a.n_q, ii = r % a.n_q;
+          const int slot = a.q_ring ? ((T - a.n_q + ii) % a.n_q + a.n_q) % a.n_q : ii;
+          v = *reinterpret_cast<const uint4 *>(a.q + ((static_cast<int64_t>(b) * a.Hq + kvh * a.G + hg) * a.n_q + slot) * D +
+                                               8 * c);
+        }
+        *reinterpret_cast<uint4 *>(sQ + (r >> 7) * TC_TILE + sw128_off(r & 127, 8 * c)) = v;
+      }
+      if (PASS == 2)
+        // p = exp2(s - m_r) / l_r = exp2(s - (m_r - log2(1 / l_r))); rows
+        // without keys (or past R) get +inf, i.e. p = 0
+        for (int r = tid; r < n_rbt * 128; r += TC_THREADS) {
+          float mo = INFINITY;
+          if (r < a.R) {
+            const float2 st = a.stats[static_cast<int64_t>(u) * SEL_MAX_ROWS + r];
+            if (st.y > 0.f) mo = st.x - __log2f(st.y);
+          }
+          moff[r] = mo;
+        }
       q_unit = u;
       q_T = T;
     }
-    float m[2][2], l[2][2], il[2][2];
-    int qpos[2][2];
+    __syncthreads();  // slot_of is written
+    float rm[TC_MAX_RB], rl[TC_MAX_RB];  // pass 1: running (max, sum) of this thread's rows over its columns
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const int row = 32 * warp + 16 * mt + gid + 8 * hr;
-        m[mt][hr] = -INFINITY;
-        l[mt][hr] = 0.f;
-        il[mt][hr] = 0.f;
-        qpos[mt][hr] = (row < a.R) ? T - a.n_q + row % a.n_q : -1;  // last visible key
-        if (PASS == 2 && row < a.R) {
-          const float2 st = a.stats[static_cast<int64_t>(u) * SEL_MAX_ROWS + row];
-          m[mt][hr] = st.x;
-          il[mt][hr] = st.y;
-        }
-      }
-    if (CACHE) store_cache(raw, tiles, tiles + TILE);
+    for (int rb = 0; rb < TC_MAX_RB; ++rb) {
+      rm[rb] = -INFINITY;
+      rl[rb] = 0.f;
+    }
+    KeyRaw raw;
+    key_load<CACHE>(a, u, T, k0 + kk, k1, slot_of, k0, hfk, raw);
+    key_store<CACHE>(raw, kk, hfk, sK, sK + TC_TILE);
+    publish();
+    issue(0);
+    if (nsub > 1) key_load<CACHE>(a, u, T, k0 + TC_NK + kk, k1, slot_of, k0, hfk, raw);
     for (int st = 0; st < nsub; ++st) {
-      const int cur = st & 1;
-      const int key0 = k0 + st * SEL_SUB;
-      const bool more = st + 1 < nsub;
-      if (more) {
-        if (CACHE) issue_cache(a, u, T, key0 + SEL_SUB, k1, slot_of, k0, raw);
-        else issue_fp16(a, u, key0 + SEL_SUB, k1, tiles_s + (cur ^ 1) * 2 * TILE);
+      const int buf = (nbuf == 2) ? (st & 1) : 0;
+      const int key0 = k0 + st * TC_NK;
+      if (nbuf == 2 && st + 1 < nsub) {
+        // next tile into the other buffer (its last reader, sub-tile st-1, is done)
+        key_store<CACHE>(raw, kk, hfk, sK + (buf ^ 1) * KT, sK + (buf ^ 1) * KT + TC_TILE);
+        publish();
+        issue(buf ^ 1);
+        if (st + 2 < nsub) key_load<CACHE>(a, u, T, key0 + 2 * TC_NK + kk, k1, slot_of, k0, hfk, raw);
       }
-      if (!CACHE) {
-        if (more) cp_async_wait<1>(); else cp_async_wait<0>();
-      }
-      __syncthreads();
-      float s[2][8][4];
-      if (has_rows) {
-        tile_scores<CACHE>(tiles_s + cur * 2 * TILE, tiles_s + cur * 2 * TILE + TILE, qa, qz, lane, s);
-        if (PASS == 1) {
+      tc_wait(smem_u32(&mbar[buf]), phase[buf], a, &s_abort);
+      phase[buf] ^= 1u;
+      tc_fence_after();
+      if (PASS == 1) {
+        // epilogue: this thread's row of each row block, 64 key columns
+        const bool all_visible = key0 + TC_NK <= k1 && key0 + TC_NK - 1 <= T - a.n_q;
 #pragma unroll
-          for (int mt = 0; mt < 2; ++mt)
+        for (int rb = 0; rb < TC_MAX_RB; ++rb) {
+          if (rb >= n_rbt) break;
+          const int r = 128 * rb + 32 * qd + lane;
+          const bool row_ok = r < a.R;
+          const int qpos = row_ok ? T - a.n_q + r % a.n_q : -1;  // last key this query sees
 #pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-              float mx = -INFINITY;
+          for (int cb = 0; cb < 2; ++cb) {
+            float v[32];
+            // every lane of the warp takes part in the tensor-memory load
+            tc_ld32(tbase + (static_cast<uint32_t>(32 * qd) << 16) + buf * acc_cols + rb * TC_NK + 64 * hfw + 32 * cb, v);
+            const int kb = key0 + 64 * hfw + 32 * cb;  // key of v[0]
+            if (!(all_visible && row_ok))
 #pragma unroll
-              for (int nt = 0; nt < 8; ++nt)
+              for (int j = 0; j < 32; ++j)
+                if (!(kb + j < k1 && kb + j <= qpos)) v[j] = -INFINITY;
+            float mx = -INFINITY;
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                  const int key = key0 + nt * 8 + 2 * t4 + e;
-                  const bool vis = key < k1 && key <= qpos[mt][hr];
-                  float &x = s[mt][nt][2 * hr + e];
-                  x = vis ? x : -INFINITY;
-                  mx = fmaxf(mx, x);
-                }
-              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-              const float mn = fmaxf(m[mt][hr], mx);
-              if (mn == -INFINITY) continue;
+            for (int j = 0; j < 32; ++j) mx = fmaxf(mx, v[j]);
+            const float mn = fmaxf(rm[rb], mx * SEL_SCALE);  // the scale is positive
+            if (mn != -INFINITY) {
               float sum = 0.f;
 #pragma unroll
-              for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) sum += fast_exp2(s[mt][nt][2 * hr + e] - mn);
-              l[mt][hr] = l[mt][hr] * fast_exp2(m[mt][hr] - mn) + sum;
-              m[mt][hr] = mn;
+              for (int j = 0; j < 32; ++j) sum += fast_exp2(fmaf(v[j], SEL_SCALE, -mn));
+              rl[rb] = rl[rb] * fast_exp2(rm[rb] - mn) + sum;
+              rm[rb] = mn;
             }
-        } else {
-#pragma unroll
-          for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              float acc = 0.f;
-#pragma unroll
-              for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr)
-                  acc += (il[mt][hr] > 0.f) ? fast_exp2(s[mt][nt][2 * hr + e] - m[mt][hr]) * il[mt][hr] : 0.f;
-              acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-              acc += __shfl_xor_sync(0xffffffffu, acc, 8);
-              acc += __shfl_xor_sync(0xffffffffu, acc, 16);
-              if (gid == 0) cpart[wl * SEL_SUB + nt * 8 + 2 * t4 + e] = acc;
-            }
+          }
         }
-      } else if (PASS == 2) {
-        for (int j = lane; j < SEL_SUB; j += 32) cpart[wl * SEL_SUB + j] = 0.f;
-      }
-      if (CACHE && more) store_cache(raw, tiles + (cur ^ 1) * 2 * TILE, tiles + (cur ^ 1) * 2 * TILE + TILE);
-      __syncthreads();
-      if (PASS == 2) {
-        for (int j = threadIdx.x; j < SEL_SUB; j += blockDim.x) {
-          const int key = key0 + j;
-          float tot = 0.f;
-          for (int w = 0; w < SEL_BLOCK_ROWS / 32; ++w) tot += cpart[w * SEL_SUB + j];
-          if (key < k1) a.colsum_part[(static_cast<int64_t>(rb) * a.U + u) * a.cap + key] = tot;
+      } else {
+        // epilogue: this thread is key column 32 (w % 4) + lane of the
+        // sub-tile; it sums p over its half of the rows (every candidate
+        // key is visible to every selection query)
+        float acc = 0.f;
+#pragma unroll
+        for (int rb = 0; rb < TC_MAX_RB; ++rb) {
+          if (rb >= n_rbt) break;
+#pragma unroll
+          for (int cb = 0; cb < 2; ++cb) {
+            float v[32];
+            tc_ld32(tbase + (static_cast<uint32_t>(32 * qd) << 16) + buf * acc_cols + rb * TC_NK + 64 * hfw + 32 * cb, v);
+            const float *mo = moff + rb * TC_NK + 64 * hfw + 32 * cb;  // row of v[0]
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc += fast_exp2(fmaf(v[j], SEL_SCALE, -mo[j]));
+          }
         }
-        __syncthreads();
+        csum[hfw * TC_NK + 32 * qd + lane] = acc;
       }
+      tc_fence_before();
+      __syncthreads();  // accumulator set `buf` is free again
+      tc_fence_after();
+      if (PASS == 2 && tid < TC_NK) {
+        const int key = key0 + tid;
+        if (key < k1) a.colsum_part[static_cast<int64_t>(u) * a.cap + key] = csum[tid] + csum[TC_NK + tid];
+      }
+      if (nbuf == 1 && st + 1 < nsub) {
+        key_store<CACHE>(raw, kk, hfk, sK, sK + TC_TILE);
+        publish();
+        issue(0);
+        if (st + 2 < nsub) key_load<CACHE>(a, u, T, key0 + 2 * TC_NK + kk, k1, slot_of, k0, hfk, raw);
+      }
+      if (s_abort) break;
     }
     if (PASS == 1) {
+      // merge the two column halves of every row, then write the chunk partial
+      if (hfw == 1)
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
+        for (int rb = 0; rb < TC_MAX_RB; ++rb)
+          if (rb < n_rbt) pst[rb * 128 + 32 * qd + lane] = make_float2(rm[rb], rl[rb]);
+      __syncthreads();
+      if (hfw == 0)
 #pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          float lv = l[mt][hr];
-          lv += __shfl_xor_sync(0xffffffffu, lv, 1);
-          lv += __shfl_xor_sync(0xffffffffu, lv, 2);
-          const int row = 32 * warp + 16 * mt + gid + 8 * hr;
-          if (t4 == 0 && row < SEL_MAX_ROWS)
-            a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + row] =
-                make_float2(m[mt][hr], lv);
+        for (int rb = 0; rb < TC_MAX_RB; ++rb) {
+          const int r = 128 * rb + 32 * qd + lane;
+          if (rb >= n_rbt || r >= a.R) continue;
+          const float2 o = pst[rb * 128 + 32 * qd + lane];
+          const float M = fmaxf(rm[rb], o.x);
+          float L = 0.f;
+          if (M != -INFINITY) L = rl[rb] * fast_exp2(rm[rb] - M) + o.y * fast_exp2(o.x - M);
+          a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + r] = make_float2(M, L);
         }
     }
   }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(ncols));
 }
 
-// Cache mode: rank_base[u][w] = vertical-line rows at positions < 32 w
-// (exclusive prefix popcount of the unit's mask), so the slot of a position
-// is one popcount away.
 __global__ void __launch_bounds__(1024) rank_kernel(const SelectArgs a) {
   pdl_trigger();  // the next kernel may be scheduled
   pdl_wait();     // earlier work on the stream is complete and visible
@@ -711,32 +708,40 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const SelectArgs a) 
   }
 }
 
+static size_t score_smem_bytes(int R, bool cache) {
+  const int n_rbt = (R + 127) / 128;
+  const int nbuf = (n_rbt <= 2) ? 2 : 1;
+  return 1024 /* alignment */ + static_cast<size_t>(n_rbt) * TC_TILE + static_cast<size_t>(nbuf) * (cache ? 2 : 1) * TC_TILE +
+         SEL_KC * 4 + 4 * TC_NK * 4 + TC_MAX_RB * 128 * 8 + SEL_MAX_ROWS * 4;
+}
+
 static cudaError_t select_launch(const SelectArgs &a, bool cache, cudaStream_t s) {
-  const size_t smem = 4 * SEL_SUB * 256 + SEL_KC * 4 + (SEL_BLOCK_ROWS / 32) * SEL_SUB * 4;
+  const size_t smem = score_smem_bytes(a.R, cache);
   static int attr_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_dev != dev) {
-    cudaFuncSetAttribute(score_kernel<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(score_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(score_kernel<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(score_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int mx = static_cast<int>(std::max(score_smem_bytes(SEL_MAX_ROWS, true), score_smem_bytes(256, true)));
+    cudaFuncSetAttribute(score_kernel<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+    cudaFuncSetAttribute(score_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+    cudaFuncSetAttribute(score_kernel<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
+    cudaFuncSetAttribute(score_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
     cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(TOPK_SMEM_VALS * (sizeof(uint32_t) + sizeof(uint16_t))));
     attr_dev = dev;
   }
   const int n_items = a.U * a.n_chunks;
   const int sms = hyq_sm_count_dev();
-  const dim3 grid(n_items < sms ? n_items : sms, a.n_rb);
+  const dim3 grid(n_items < sms ? n_items : sms);
   cudaError_t e;
   if (cache) {
     e = launch(rank_kernel, dim3(a.U), dim3(1024), 0, s, a);
-    if (e == cudaSuccess) e = launch(score_kernel<true, 1>, grid, dim3(SEL_THREADS), smem, s, a);
+    if (e == cudaSuccess) e = launch(score_kernel<true, 1>, grid, dim3(TC_THREADS), smem, s, a);
   } else {
-    e = launch(score_kernel<false, 1>, grid, dim3(SEL_THREADS), smem, s, a);
+    e = launch(score_kernel<false, 1>, grid, dim3(TC_THREADS), smem, s, a);
   }
   if (e == cudaSuccess) e = launch(stats_merge_kernel, dim3(a.U), dim3(256), 0, s, a);
-  if (e == cudaSuccess) e = launch(cache ? score_kernel<true, 2> : score_kernel<false, 2>, grid, dim3(SEL_THREADS), smem, s, a);
+  if (e == cudaSuccess) e = launch(cache ? score_kernel<true, 2> : score_kernel<false, 2>, grid, dim3(TC_THREADS), smem, s, a);
   if (e == cudaSuccess) e = launch(topk_kernel, dim3(a.U), dim3(TOPK_THREADS), TOPK_SMEM_VALS * (sizeof(uint32_t) + sizeof(uint16_t)), s, a);
   return e;
 }
