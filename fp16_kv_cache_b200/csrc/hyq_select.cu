@@ -138,8 +138,7 @@ struct KeyRaw {
 
 // Thread t loads key (t % 128) of the sub-tile, channels 64 (t / 128) .. + 63.
 template <bool CACHE>
-__device__ __forceinline__ void key_load(const SelectArgs &a, int u, int T, int key, int key_end, const int *slot_of,
-                                         int k0, int hf, KeyRaw &r) {
+__device__ __forceinline__ void key_load(const SelectArgs &a, int u, int T, int key, int key_end, int hf, KeyRaw &r) {
   r.kind = 0;
   if (key >= key_end) return;
   const __half *row = nullptr;
@@ -148,8 +147,13 @@ __device__ __forceinline__ void key_load(const SelectArgs &a, int u, int T, int 
   } else if (key >= T - a.W) {
     row = a.win_k + (static_cast<int64_t>(u) * a.W + key % a.W) * D;
   } else {
-    const int slot = slot_of[key - k0];
-    if (slot >= 0) row = a.vl_k + (static_cast<int64_t>(u) * a.vl_cap + slot) * D;
+    // a vertical line: its row is the rank of its bit among the unit's set bits
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(a.blocks + blk_base(u, key, a.cap) + HYQ_BLK_MASK);
+    if ((w >> (key & 31)) & 1u) {
+      const int slot = a.rank_base[static_cast<int64_t>(u) * (a.cap / 32) + (key >> 5)] +
+                       __popc(w & ((1u << (key & 31)) - 1u));
+      row = a.vl_k + (static_cast<int64_t>(u) * a.vl_cap + slot) * D;
+    }
   }
   if (row) {
     r.kind = 1;
@@ -243,8 +247,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
   constexpr int KT = CACHE ? 2 * TC_TILE : TC_TILE;     // one key buffer: hi (+ lo)
   uint8_t *sQ = sm;                                      // [n_rbt][32 KB]
   uint8_t *sK = sQ + n_rbt * TC_TILE;                    // [nbuf][KT]
-  int *slot_of = reinterpret_cast<int *>(sK + nbuf * KT);               // [SEL_KC]
-  float *csum = reinterpret_cast<float *>(slot_of + SEL_KC);            // [4][128]
+  float *csum = reinterpret_cast<float *>(sK + nbuf * KT);              // [4][128]
   float2 *pst = reinterpret_cast<float2 *>(csum + 4 * TC_NK);           // [TC_MAX_RB][128]
   float *moff = reinterpret_cast<float *>(pst + TC_MAX_RB * 128);       // [SEL_MAX_ROWS] pass 2: m_r - log2(1/l_r)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -273,6 +276,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
   const int it0 = min(n_items, static_cast<int>(blockIdx.x) * per), it1 = min(n_items, it0 + per);
   int q_unit = -1, q_T = -1;
   const int kk = tid & 127, hfk = tid >> 7;  // key row and channel half this thread stages
+  KeyRaw raw;
+  bool have_next = false;  // raw holds the first tile of the next item
 
   // one sub-tile's MMAs into accumulator set `buf` from key buffer `buf`
   auto issue = [&](int buf) {
@@ -321,19 +326,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
     tc_fence_before();
     __syncthreads();  // the previous item is done with shared and tensor memory
     tc_fence_after();
-    if (CACHE) {
-      // vertical-line slot of every key of the chunk: rank of its mask bit
-      const int32_t *rbase = a.rank_base + static_cast<int64_t>(u) * (a.cap / 32);
-      for (int j = tid; j < SEL_KC; j += TC_THREADS) {
-        const int key = k0 + j;
-        int slot = -1;
-        if (key < k1 && key < T - a.W) {
-          const uint32_t w = *reinterpret_cast<const uint32_t *>(a.blocks + blk_base(u, key, a.cap) + HYQ_BLK_MASK);
-          if ((w >> (key & 31)) & 1u) slot = rbase[key >> 5] + __popc(w & ((1u << (key & 31)) - 1u));
-        }
-        slot_of[j] = slot;
-      }
-    }
     if (u != q_unit || T != q_T) {
       // the unit's query rows into the swizzled row blocks (zeros past R)
       const int b = u / a.Hkv, kvh = u % a.Hkv;
@@ -361,20 +353,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
         }
       q_unit = u;
       q_T = T;
+      __syncthreads();  // stage arrays written
     }
-    __syncthreads();  // slot_of is written
     float rm[TC_MAX_RB], rl[TC_MAX_RB];  // pass 1: running (max, sum) of this thread's rows over its columns
 #pragma unroll
     for (int rb = 0; rb < TC_MAX_RB; ++rb) {
       rm[rb] = -INFINITY;
       rl[rb] = 0.f;
     }
-    KeyRaw raw;
-    key_load<CACHE>(a, u, T, k0 + kk, k1, slot_of, k0, hfk, raw);
+    if (!have_next) key_load<CACHE>(a, u, T, k0 + kk, k1, hfk, raw);
+    have_next = false;
     key_store<CACHE>(raw, kk, hfk, sK, sK + TC_TILE);
     publish();
     issue(0);
-    if (nsub > 1) key_load<CACHE>(a, u, T, k0 + TC_NK + kk, k1, slot_of, k0, hfk, raw);
+    if (nsub > 1) key_load<CACHE>(a, u, T, k0 + TC_NK + kk, k1, hfk, raw);
     for (int st = 0; st < nsub; ++st) {
       const int buf = (nbuf == 2) ? (st & 1) : 0;
       const int key0 = k0 + st * TC_NK;
@@ -383,7 +375,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
         key_store<CACHE>(raw, kk, hfk, sK + (buf ^ 1) * KT, sK + (buf ^ 1) * KT + TC_TILE);
         publish();
         issue(buf ^ 1);
-        if (st + 2 < nsub) key_load<CACHE>(a, u, T, key0 + 2 * TC_NK + kk, k1, slot_of, k0, hfk, raw);
+        if (st + 2 < nsub) key_load<CACHE>(a, u, T, key0 + 2 * TC_NK + kk, k1, hfk, raw);
+      }
+      if (st + 1 == nsub && item + 1 < it1 && (item + 1) / a.n_chunks == u) {
+        // the next item's first tile (same unit) loads during this epilogue
+        const int k0n = k0 + SEL_KC;
+        if (k0n < key_end) {
+          key_load<CACHE>(a, u, T, k0n + kk, min(key_end, k0n + SEL_KC), hfk, raw);
+          have_next = true;
+        }
       }
       tc_wait(smem_u32(&mbar[buf]), phase[buf], a, &s_abort);
       phase[buf] ^= 1u;
@@ -450,7 +450,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
         key_store<CACHE>(raw, kk, hfk, sK, sK + TC_TILE);
         publish();
         issue(0);
-        if (st + 2 < nsub) key_load<CACHE>(a, u, T, key0 + 2 * TC_NK + kk, k1, slot_of, k0, hfk, raw);
+        if (st + 2 < nsub) key_load<CACHE>(a, u, T, key0 + 2 * TC_NK + kk, k1, hfk, raw);
       }
       if (s_abort) break;
     }
