@@ -16,8 +16,9 @@ working set (~360 MB) exceeds the 126 MB L2 between successive steps.
 Metric: effective decode-attention HBM GB/s = algorithmic bytes of the
 decode steps (packed codes + scales + FP16 vertical-line/window K/V + Q/O) /
 time.  The timed region is one CUDA-graph replay of K steps, bracketed by
-a barrier and synchronize; per-launch decode durations come from CUDA
-events captured around every decode inside the graph.
+a barrier and synchronize; the decode kernel's average launch time comes
+from CUDA events captured inside the graph around each run of back-to-back
+step launches between two re-selections.
 
 --impl reference times the CPU oracle (fp64, plain C) on a bounded sample of
 the same workload, on the host cores.
@@ -44,9 +45,6 @@ METRIC = "decode-attention effective HBM GB/s (% of B200 peak); µs/step at 32K 
 L2_DEFEAT_BYTES = 360e6  # rotate layer caches until a pass over them is ~3x the 126 MB L2
 RESELECT = 64
 N_Q = 64
-
-
-EV_EVERY = 8  # decodes timed with events: one in every EV_EVERY steps
 
 
 def algorithmic_bytes(B, Hq, Hkv, T, k, W=128):
@@ -230,20 +228,21 @@ def run_ours(args):
 
     resel_at = {}  # layer -> step after which its first re-selection ran
 
-    def step(s, ev=None):
-        """Enqueue step s; returns (launches, layer, T after the step's append)."""
+    def step(s, before=None, after=None):
+        """Enqueue step s; returns (launches, layer, T after the step's append).
+        before() runs before the decode launch, after(reselect) after it."""
         li = s % n_layers
         c = layers[li]
         i = s % 64
-        if ev is not None:
-            ev[0].record()
+        if before is not None:
+            before()
         hyq.hyq_decode_step(c, q_in[i], k_in[i], v_in[i], out, dws[li], q_ring=rings[li], lse=lse,
                             n_ctas=n_ctas)
-        if ev is not None:
-            ev[1].record()
         tokens[li] += 1
         appended[li] += 1
         launches = 1
+        if after is not None:
+            after(appended[li] % RESELECT == 0)
         if appended[li] % RESELECT == 0:
             # the 64 queries of the ring are scored; the next decode of the
             # layer sees the new vertical-line set
@@ -258,9 +257,22 @@ def run_ours(args):
         step(s)
     torch.cuda.synchronize()
 
-    # capture K steps; every EV_EVERY-th step's launch is bracketed by events
-    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
-           if j % EV_EVERY == 0 else None for j in range(K_steps)]
+    # capture K steps; each run of back-to-back decode launches between two
+    # re-selections is bracketed by one pair of events, so the launches inside
+    # a run keep their programmatic overlap with the launch before them
+    runs = []  # [start event, end event, [indices into `seen`]]
+
+    def run_open():
+        if not runs or runs[-1][1] is not None:
+            e = torch.cuda.Event(enable_timing=True, external=True)
+            e.record()
+            runs.append([e, None, []])
+
+    def run_close():
+        e = torch.cuda.Event(enable_timing=True, external=True)
+        e.record()
+        runs[-1][1] = e
+
     g = torch.cuda.CUDAGraph()
     total_launches = 0
     seen = []  # (step, layer, T)
@@ -269,7 +281,14 @@ def run_ours(args):
     with torch.cuda.stream(side):
         with torch.cuda.graph(g, stream=side):
             for j in range(K_steps):
-                nl, li, T = step(W_steps + j, evs[j])
+                last = j == K_steps - 1
+
+                def after(resel, j=j, last=last):
+                    runs[-1][2].append(j)
+                    if resel or last:
+                        run_close()
+
+                nl, li, T = step(W_steps + j, run_open, after)
                 total_launches += nl
                 seen.append((W_steps + j, li, T))
     torch.cuda.synchronize()
@@ -295,15 +314,16 @@ def run_ours(args):
     # (a cache-mode re-selection keeps only rows still held in FP16)
     k_after = [c.vl_count.flatten().tolist() for c in layers]  # per unit, after the re-selection
     total_bytes = 0
-    ev_bytes = []
+    nbytes = []
     for j, (s_, li, T) in enumerate(seen):
         kk = cfg.k if (li not in resel_at or s_ <= resel_at[li]) else k_after[li]
         nb = step_bytes(B, Hq, Hkv, T, kk)
         total_bytes += nb
-        if evs[j] is not None:
-            ev_bytes.append(nb)
-    dec_ms = [e[0].elapsed_time(e[1]) for e in evs if e is not None]
-    dec_avg_ms = float(np.mean(dec_ms))
+        nbytes.append(nb)
+    run_ms = sum(r[0].elapsed_time(r[1]) for r in runs)
+    run_n = sum(len(r[2]) for r in runs)
+    dec_avg_ms = run_ms / run_n
+    ev_bytes = [nbytes[j] for r in runs for j in r[2]]
     status = max(c.status() for c in layers)
 
     # roofline of the decode kernel (the dominant launch)
@@ -335,7 +355,8 @@ def run_ours(args):
                   "per GPU",
             "us_per_step": round(1000 * elapsed_ms / K_steps, 3),
             "decode_us_avg": round(1000 * dec_avg_ms, 3),
-            "decode_timed": f"CUDA events around {len(dec_ms)} of the {K_steps} timed launches",
+            "decode_timed": f"CUDA events around {len(runs)} runs of back-to-back step launches "
+                            f"({run_n} launches, re-selections outside the runs)",
             "decode_bytes_per_step": int(bytes_per_decode),
             "pct_of_peak_step": round(100 * value / world / peak, 1),
             "n_ctas": n_ctas,
@@ -371,21 +392,22 @@ def fp16_comparator(torch, hyq, cfg, Kd, Vd, q_in, dev, copies=3, reps=60):
     for i in range(6):
         hyq.hyq_decode_fp16(q_in[i], Ks[i % copies], Vs[i % copies], seq, o, ws)
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
-           for _ in range(reps)]
+    # timed like the hybrid step: one pair of events around back-to-back launches
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
     g = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
         with torch.cuda.graph(g, stream=side):
+            e0.record()
             for i in range(reps):
-                evs[i][0].record()
                 hyq.hyq_decode_fp16(q_in[i % 64], Ks[i % copies], Vs[i % copies], seq, o, ws)
-                evs[i][1].record()
+            e1.record()
     torch.cuda.synchronize()
     g.replay()
     torch.cuda.synchronize()
-    ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    ms = e0.elapsed_time(e1) / reps
     nbytes = cfg.B * cfg.Hkv * cfg.T * 512 + cfg.B * cfg.Hq * 128 * 4
     del g
     return {"us": round(1000 * ms, 3), "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1), "bytes": nbytes}

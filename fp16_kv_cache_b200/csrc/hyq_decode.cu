@@ -15,7 +15,9 @@
 //     tiles of 8 rows (vertical lines, then the window).  All tiles of all
 //     units are concatenated and split over the launch's blocks by bytes
 //     read (cost 5 per INT4 tile, 4 per FP16 tile), so any batch/length mix
-//     fills every SM (split-KV, stream-K style).
+//     fills every SM (split-KV, stream-K style).  With few long units the
+//     split is aligned to units (whole blocks per unit).  The split is
+//     planned before the wait on the previous launch and checked after it.
 //   * One block per SM, 12 compute warps.  Block-local tile i belongs to
 //     warp i % 12, which issues its own 1-D bulk copies (cp.async.bulk, no
 //     multicast) into a private 2-slot ring with mbarrier transaction counts;
@@ -144,12 +146,24 @@ __device__ __forceinline__ UnitShape shape_of(const DecodeArgs &a, int T, int vl
 
 // Shape of unit u from global state (prologue only; later reads use the
 // per-unit (T, vl_count) copies kept in shared memory).
+// (seq_len, vl_count) of unit u as stored.  L2-only loads: the first read
+// may precede the wait on the previous launch, and no stale copy of it may
+// stay in L1 for the re-read after it.
+template <int MODE>
+__device__ __forceinline__ int2 raw_lengths(const DecodeArgs &a, int u) {
+  return make_int2(__ldcg(a.seq_len + u / a.Hkv), (MODE == MODE_FP16) ? 0 : __ldcg(a.vl_count + u));
+}
+
+template <int MODE>
+__device__ __forceinline__ UnitShape shape_from_raw(const DecodeArgs &a, int2 raw, bool &bad) {
+  int T = raw.x;
+  if (MODE == MODE_STEP) T = (T < 0) ? -1 : T + 1;  // the length after the append
+  return shape_of<MODE>(a, T, raw.y, bad);
+}
+
 template <int MODE>
 __device__ __forceinline__ UnitShape unit_shape_global(const DecodeArgs &a, int u, bool &bad) {
-  int T = a.seq_len[u / a.Hkv];
-  if (MODE == MODE_STEP) T = (T < 0) ? -1 : T + 1;  // the length after the append
-  const int vlc = (MODE == MODE_FP16) ? 0 : a.vl_count[u];
-  return shape_of<MODE>(a, T, vlc, bad);
+  return shape_from_raw<MODE>(a, raw_lengths<MODE>(a, u), bad);
 }
 
 // Per-warp running state, in the accumulator layout of m16n8: lane (r, q)
@@ -475,6 +489,8 @@ struct Smem {
   float *mm, *ml, *mo;  // merge buffers: [NCW][8], [NCW][8], [NCW][G][128]
   int *cost_start;      // [U + 1]: cost of the units before u
   int *scan;            // [NTHREADS]
+  int *blk_start;       // [ALIGN_MAX_U + 1]: first block of each unit (aligned split)
+  int *blk_lo;          // [ALIGN_MAX_CTAS + 1]: start cost of each block (aligned split)
   int2 *unit_tv;        // [U]: (T, vl_count) as read at launch
 };
 
@@ -502,17 +518,38 @@ __device__ __forceinline__ int tile_cost(int cs, int n4, int j) {
   return j <= n4 ? cs + COST4 * j : cs + COST4 * n4 + COST16 * (j - n4);
 }
 
-// Balanced split of the total cost over the launch's blocks: block c owns
-// [lo(c), lo(c + 1)) with lo(c) = c * per + min(c, rem), i.e. the first rem
-// blocks take per + 1 and the others per.
+// Split of the total cost over the launch's blocks.
+//  * Contiguous: block c owns [lo(c), lo(c + 1)) with lo(c) = c * per +
+//    min(c, rem), i.e. the first rem blocks take per + 1 and the others per;
+//    a block may hold the end of one unit and the start of the next.
+//  * Aligned (few long units): unit u owns the whole blocks [bs[u],
+//    bs[u + 1]), bs[u] = round(n * cost_start[u] / total), and its cost is
+//    spread evenly over them, so no block pays for two unit ends (two block
+//    merges and two partial records).  Chosen only when every non-empty unit
+//    gets a block and no block carries more than 9/8 of the mean cost; the
+//    blocks' start costs are tabulated once per launch (sm.blk_lo).
+constexpr int ALIGN_MAX_U = 32, ALIGN_MIN_BPU = 8, ALIGN_MAX_CTAS = 1024;
+constexpr int BLK_TABLE_BYTES = ((ALIGN_MAX_U + 1) * 4 + 15) / 16 * 16 + ((ALIGN_MAX_CTAS + 1) * 4 + 15) / 16 * 16;
+
 struct Split {
   int per, rem;
-  __device__ __forceinline__ Split(int total, int n) : per(total / n), rem(total % n) {}
-  __device__ __forceinline__ int lo(int c) const { return c * per + min(c, rem); }
+  bool aligned;
+  __device__ __forceinline__ Split(int total, int n, bool al) : per(total / n), rem(total % n), aligned(al) {}
+  __device__ __forceinline__ int lo(const Smem &sm, int U, int c) const {
+    return aligned ? sm.blk_lo[c] : c * per + min(c, rem);
+  }
   // the block whose (non-empty) range holds cost x, for 0 <= x < total
-  __device__ __forceinline__ int of(int x) const {
-    const int big = rem * (per + 1);
-    return x < big ? x / (per + 1) : rem + (x - big) / per;
+  __device__ __forceinline__ int of(const Smem &sm, int U, int x) const {
+    if (!aligned) {
+      const int big = rem * (per + 1);
+      return x < big ? x / (per + 1) : rem + (x - big) / per;
+    }
+    int l = 0, h = sm.blk_start[U] - 1;  // last block c with blk_lo[c] <= x
+    while (l < h) {
+      const int mid = (l + h + 1) >> 1;
+      if (sm.blk_lo[mid] <= x) l = mid; else h = mid - 1;
+    }
+    return l;
   }
 };
 
@@ -584,7 +621,7 @@ __device__ __forceinline__ void merge_parts(const DecodeArgs &a, const Smem &sm,
   constexpr int RB = (G >= 8) ? 1 : 16 / G;  // records per batch (bounded by registers)
   const int warp = tid >> 5, lane = tid & 31;
   const int cs = sm.cost_start[u];
-  const int c_lo = sp.of(cs), c_hi = sp.of(tile_cost(cs, n4, n4 + n16 - 1));
+  const int c_lo = sp.of(sm, a.U, cs), c_hi = sp.of(sm, a.U, tile_cost(cs, n4, n4 + n16 - 1));
   float M[G], L[G];
   float4 acc[G];
 #pragma unroll
@@ -601,7 +638,7 @@ __device__ __forceinline__ void merge_parts(const DecodeArgs &a, const Smem &sm,
       const int cc = c0 + b * NCW;
       int id = -1;  // record of block cc for unit u, if cc has tiles of u
       if (cc <= c_hi) {
-        const int lo = sp.lo(cc), hi = sp.lo(cc + 1);
+        const int lo = sp.lo(sm, a.U, cc), hi = sp.lo(sm, a.U, cc + 1);
         if (first_tile_from(lo, cs, n4, n16) < first_tile_from(hi, cs, n4, n16)) id = cc * 2 + ((cs <= lo) ? 0 : 1);
       }
 #pragma unroll
@@ -745,19 +782,19 @@ __device__ __forceinline__ void step_prologue(const DecodeArgs &a, const Smem &s
   }
 }
 
-// Issue the bulk copies of tile j of unit u into one ring slot (lane 0 arms
-// the barrier and copies; an FP16 tile is two contiguous runs of rows).
+// Global source of tile j of unit u: one run (an INT4 block record) or two
+// runs of `bytes` each (the K rows and the V rows of an FP16 tile).
+struct TileSrc {
+  const void *k, *v;
+  uint32_t bytes;
+};
+
 template <int MODE>
-__device__ __forceinline__ void issue_tile(const DecodeArgs &a, const Smem &sm, int u, int j, uint32_t dst,
-                                           uint32_t bar, int lane) {
+__device__ __forceinline__ TileSrc tile_src(const DecodeArgs &a, const Smem &sm, int u, int j) {
   bool bad;
   const UnitShape us = shape_of<MODE>(a, sm.unit_tv[u].x, sm.unit_tv[u].y, bad);
-  if (lane != 0) return;
-  if (MODE != MODE_FP16 && j < us.n4) {
-    mbar_arrive_expect_tx(bar, BLK_BYTES);
-    bulk_g2s(dst, a.blocks + blk_base(u, static_cast<int64_t>(j) * I4_TOK, a.cap), BLK_BYTES, bar);
-    return;
-  }
+  if (MODE != MODE_FP16 && j < us.n4)
+    return {a.blocks + blk_base(u, static_cast<int64_t>(j) * I4_TOK, a.cap), nullptr, BLK_BYTES};
   const __half *sk, *sv;
   int n;
   if (MODE == MODE_FP16) {
@@ -779,9 +816,121 @@ __device__ __forceinline__ void issue_tile(const DecodeArgs &a, const Smem &sm, 
     sk = a.win_k + base;
     sv = a.win_v + base;
   }
-  mbar_arrive_expect_tx(bar, n * 2 * F16_ROW);
-  bulk_g2s(dst, sk, n * F16_ROW, bar);
-  bulk_g2s(dst + SLOT_F16V, sv, n * F16_ROW, bar);
+  return {sk, sv, static_cast<uint32_t>(n * F16_ROW)};
+}
+
+// Issue the bulk copies of tile j of unit u into one ring slot (lane 0 arms
+// the barrier and copies; an FP16 tile is two contiguous runs of rows).
+template <int MODE>
+__device__ __forceinline__ void issue_tile(const DecodeArgs &a, const Smem &sm, int u, int j, uint32_t dst,
+                                           uint32_t bar, int lane) {
+  if (lane != 0) return;
+  const TileSrc t = tile_src<MODE>(a, sm, u, j);
+  if (t.v == nullptr) {
+    mbar_arrive_expect_tx(bar, t.bytes);
+    bulk_g2s(dst, t.k, t.bytes, bar);
+    return;
+  }
+  mbar_arrive_expect_tx(bar, 2 * t.bytes);
+  bulk_g2s(dst, t.k, t.bytes, bar);
+  bulk_g2s(dst + SLOT_F16V, t.v, t.bytes, bar);
+}
+
+// Read every unit's (T, vl_count) from global memory into shared memory and
+// build the cost prefix sm.cost_start (and, for few units, the aligned
+// split's block table).  Returns whether the split is aligned (the same in
+// every thread).  Status bits for malformed lengths are raised only when
+// `report` is set.
+template <int MODE>
+__device__ __forceinline__ bool plan_units(const DecodeArgs &a, const Smem &sm, int tid, bool report) {
+  const int U = a.U, warp = tid >> 5, lane = tid & 31;
+  const int per = (U + NTHREADS - 1) / NTHREADS;
+  const int beg = min(U, tid * per), end = min(U, beg + per);
+  int local = 0;
+  for (int u = beg; u < end; ++u) {
+    bool bad;
+    const UnitShape s = unit_shape_global<MODE>(a, u, bad);
+    sm.unit_tv[u] = make_int2(s.T, s.vlc);
+    local += COST4 * s.n4 + COST16 * (s.nv + s.nw);
+    if (report && bad && (u % a.n_ctas) == static_cast<int>(blockIdx.x)) set_status(a.status, HYQ_DEV_BADLEN);
+  }
+  int v = local;  // block exclusive scan of `local`
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += y;
+  }
+  if (lane == 31) sm.scan[warp] = v;
+  __syncthreads();
+  int wpre = 0;
+  for (int w = 0; w < warp; ++w) wpre += sm.scan[w];
+  int acc = wpre + v - local;
+  for (int u = beg; u < end; ++u) {
+    int n4, n16;
+    unit_tiles<MODE>(a, sm, u, n4, n16);
+    sm.cost_start[u] = acc;
+    acc += COST4 * n4 + COST16 * n16;
+  }
+  if (tid == NTHREADS - 1) sm.cost_start[U] = acc;
+  __syncthreads();
+  const int n = a.n_ctas;
+  if (U > ALIGN_MAX_U || U * ALIGN_MIN_BPU > n || n > ALIGN_MAX_CTAS) return false;
+  const int total = sm.cost_start[U];
+  if (total <= 0) return false;
+  if (tid <= U)
+    sm.blk_start[tid] = static_cast<int>((2 * static_cast<int64_t>(n) * sm.cost_start[tid] + total) /
+                                         (2 * static_cast<int64_t>(total)));
+  __syncthreads();
+  int unfit = 0;
+  if (tid < U) {
+    const int C = sm.cost_start[tid + 1] - sm.cost_start[tid], k = sm.blk_start[tid + 1] - sm.blk_start[tid];
+    unfit = C > 0 && (k == 0 || static_cast<int64_t>(C) * n * 8 > static_cast<int64_t>(total) * k * 9);
+  }
+  if (__syncthreads_or(unfit)) return false;
+  // block c of unit u (k blocks, cost C) starts at cost_start[u] + floor(j C / k),
+  // j = c - blk_start[u], evaluated exactly in 32 bits as j (C / k) + j (C % k) / k
+  for (int c = tid; c <= n; c += NTHREADS) {
+    int v = total;
+    if (c < n) {
+      int l = 0, h = U - 1;  // last unit whose first block is <= c (a non-empty one)
+      while (l < h) {
+        const int mid = (l + h + 1) >> 1;
+        if (sm.blk_start[mid] <= c) l = mid; else h = mid - 1;
+      }
+      const int k = sm.blk_start[l + 1] - sm.blk_start[l], C = sm.cost_start[l + 1] - sm.cost_start[l];
+      const int j = c - sm.blk_start[l];
+      v = sm.cost_start[l] + j * (C / k) + j * (C % k) / k;
+    }
+    sm.blk_lo[c] = v;
+  }
+  __syncthreads();
+  return true;
+}
+
+// After the wait on the previous launch: true (in every thread) when some
+// unit's (T, vl_count) differs from the plan built before the wait.  Raises
+// the status bits of malformed lengths.  `first` holds the raw lengths of
+// the thread's first unit, read by first_lengths before the first copies
+// were issued (so that read does not queue behind them).
+template <int MODE>
+__device__ __forceinline__ int2 first_lengths(const DecodeArgs &a, int tid) {
+  const int per = (a.U + NTHREADS - 1) / NTHREADS, beg = tid * per;
+  return beg < a.U ? raw_lengths<MODE>(a, beg) : make_int2(0, 0);
+}
+
+template <int MODE>
+__device__ __forceinline__ bool plan_stale(const DecodeArgs &a, const Smem &sm, int tid, int2 first) {
+  const int U = a.U;
+  const int per = (U + NTHREADS - 1) / NTHREADS;
+  const int beg = min(U, tid * per), end = min(U, beg + per);
+  int changed = 0;
+  for (int u = beg; u < end; ++u) {
+    bool bad;
+    const UnitShape s = shape_from_raw<MODE>(a, u == beg ? first : raw_lengths<MODE>(a, u), bad);
+    if (s.T != sm.unit_tv[u].x || s.vlc != sm.unit_tv[u].y) changed = 1;
+    if (bad && (u % a.n_ctas) == static_cast<int>(blockIdx.x)) set_status(a.status, HYQ_DEV_BADLEN);
+  }
+  return __syncthreads_or(changed) != 0;
 }
 
 template <int G, int MODE>
@@ -807,58 +956,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
     p += NCW * G * D * 4;
     sm.scan = reinterpret_cast<int *>(p);
     p += NTHREADS * 4;
+    sm.blk_start = reinterpret_cast<int *>(p);
+    sm.blk_lo = sm.blk_start + ((ALIGN_MAX_U + 1) * 4 + 15) / 16 * 4;
+    p += BLK_TABLE_BYTES;
     sm.cost_start = reinterpret_cast<int *>(p);
     p += ((U_of(a) + 1) * 4 + 15) / 16 * 16;
     sm.unit_tv = reinterpret_cast<int2 *>(p);
   }
   const int U = a.U;
   pdl_trigger();  // the next kernel may be scheduled
-  pdl_wait();     // earlier work on the stream (an append) is complete and visible
-
-  // ---- prologue: read every unit's (T, vl_count), cost prefix
-  {
-    const int per = (U + NTHREADS - 1) / NTHREADS;
-    const int beg = min(U, tid * per), end = min(U, beg + per);
-    int local = 0;
-    for (int u = beg; u < end; ++u) {
-      bool bad;
-      const UnitShape s = unit_shape_global<MODE>(a, u, bad);
-      sm.unit_tv[u] = make_int2(s.T, s.vlc);
-      local += COST4 * s.n4 + COST16 * (s.nv + s.nw);
-      if (bad && (u % a.n_ctas) == static_cast<int>(blockIdx.x)) set_status(a.status, HYQ_DEV_BADLEN);
-    }
-    int v = local;  // block exclusive scan of `local`
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, v, off);
-      if (lane >= off) v += y;
-    }
-    if (lane == 31) sm.scan[warp] = v;
-    if (tid == 0) {
-      *sm.abort_flag = 0;
-      for (int s = 0; s < NCW * SPW; ++s) mbar_init(smem_u32(&sm.full[s]), 1);
-      fence_barrier_init();
-    }
-    __syncthreads();
-    int wpre = 0;
-    for (int w = 0; w < warp; ++w) wpre += sm.scan[w];
-    int acc = wpre + v - local;
-    for (int u = beg; u < end; ++u) {
-      int n4, n16;
-      unit_tiles<MODE>(a, sm, u, n4, n16);
-      sm.cost_start[u] = acc;
-      acc += COST4 * n4 + COST16 * n16;
-    }
-    if (tid == NTHREADS - 1) sm.cost_start[U] = acc;
-    __syncthreads();
-    if (MODE == MODE_STEP) step_prologue(a, sm, tid);
+  if (tid == 0) {
+    *sm.abort_flag = 0;
+    for (int s = 0; s < NCW * SPW; ++s) mbar_init(smem_u32(&sm.full[s]), 1);
+    fence_barrier_init();
   }
-  const int total = sm.cost_start[U];
-  const Split sp(total, a.n_ctas);
+  // Plan from the lengths as they stand, which the previous launch on the
+  // stream may still be changing: the plan is made while that launch drains
+  // and only checked after the wait.
+  bool aligned = plan_units<MODE>(a, sm, tid, false);
+  pdl_wait();  // earlier work on the stream (an append) is complete and visible
+
   const int cta = blockIdx.x;
-  const int lo = sp.lo(cta), hi = sp.lo(cta + 1);
+  Split sp(sm.cost_start[U], a.n_ctas, aligned);
+  int lo = sp.lo(sm, U, cta), hi = sp.lo(sm, U, cta + 1);
   volatile int *abort_flag = sm.abort_flag;
-  const int u_first = (lo < hi) ? unit_of_cost(sm.cost_start, U, lo) : U;
+  int u_first = (lo < hi) ? unit_of_cost(sm.cost_start, U, lo) : U;
 
   // This warp's tiles are the block-local tiles warp, warp + NCW, ...; its
   // k-th tile lives in ring slot k % SPW.  The warp issues its own copies:
@@ -866,9 +988,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
   const uint32_t my_slots = sm.slots + warp * SPW * SLOT_BYTES;
   const uint32_t my_bars = smem_u32(&sm.full[warp * SPW]);
   int k_issued = 0, k_done = 0, first_fail = -1;
+  int k_skip = 0;  // copies drained unused (a stale plan): not tiles of this plan
   Seg ic = seg_from<MODE>(a, sm, u_first, 0, lo, hi);  // issue cursor
   auto issue_next = [&]() {
-    const int i = warp + NCW * k_issued;  // block-local tile index
+    const int i = warp + NCW * (k_issued - k_skip);  // block-local tile index
     while (ic.u < U && i >= ic.base + ic.je - ic.jb)
       ic = seg_from<MODE>(a, sm, ic.u + 1, ic.base + ic.je - ic.jb, lo, hi);
     const int stop = __shfl_sync(0xffffffffu, *abort_flag, 0);  // one decision per warp
@@ -878,7 +1001,28 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
     __syncwarp();
     ++k_issued;
   };
+  // The first copies follow the plan made before the wait; the lengths are
+  // read again meanwhile (loads issued ahead of the copies).  If they changed
+  // (the previous launch appended to this cache), those copies land unused
+  // and the block plans again.
+  const int2 first = first_lengths<MODE>(a, tid);
   for (int k = 0; k < SPW; ++k) issue_next();
+  if (plan_stale<MODE>(a, sm, tid, first)) {
+    for (; k_done < k_issued; ++k_done) {
+      const bool ok = first_fail < 0 &&
+                      mbar_wait_bounded(my_bars + (k_done % SPW) * 8, (k_done / SPW) & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok) && first_fail < 0) first_fail = k_done;
+    }
+    aligned = plan_units<MODE>(a, sm, tid, false);
+    sp = Split(sm.cost_start[U], a.n_ctas, aligned);
+    lo = sp.lo(sm, U, cta);
+    hi = sp.lo(sm, U, cta + 1);
+    u_first = (lo < hi) ? unit_of_cost(sm.cost_start, U, lo) : U;
+    k_skip = k_issued;
+    ic = seg_from<MODE>(a, sm, u_first, 0, lo, hi);
+    for (int k = 0; k < SPW; ++k) issue_next();
+  }
+  if (MODE == MODE_STEP) step_prologue(a, sm, tid);
 
   WarpState st;
   for (Seg sg = seg_from<MODE>(a, sm, u_first, 0, lo, hi); sg.u < U;
@@ -1030,7 +1174,8 @@ static size_t decode_smem_bytes(int G, int U) {
   const int spw = Ring<1>::SPW;
   static_assert(Ring<1>::SPW == Ring<8>::SPW, "one ring depth for every G");
   return static_cast<size_t>(NCW) * spw * SLOT_BYTES + NCW * spw * 8 + 16 + NCW * 8 * 4 * 2 +
-         static_cast<size_t>(NCW) * G * D * 4 + NTHREADS * 4 + (static_cast<size_t>(U + 1) * 4 + 15) / 16 * 16 +
+         static_cast<size_t>(NCW) * G * D * 4 + NTHREADS * 4 + BLK_TABLE_BYTES +
+         (static_cast<size_t>(U + 1) * 4 + 15) / 16 * 16 +
          static_cast<size_t>(U) * 8;
 }
 
