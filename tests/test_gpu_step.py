@@ -121,3 +121,94 @@ def test_step_past_capacity_sets_status():
         if before[k] is not None:
             assert np.array_equal(before[k], after[k]), k
     assert torch.all(o == 0) and torch.all(torch.isinf(lse)) and torch.all(lse < 0)
+
+
+def _graph(fn):
+    """Capture fn() in a CUDA graph on a side stream, replay it once."""
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            fn()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    del g
+
+
+def _step_inputs(cfg, steps, seed_q):
+    kv = [synth.step_kv(cfg, s) for s in range(steps)]
+    return ([dev(k) for k, _ in kv], [dev(v) for _, v in kv], [dev(synth.q(cfg, seed_q + s)) for s in range(steps)])
+
+
+def test_graph_append_then_decode_equals_fused_step():
+    """Inside one CUDA graph a decode starts while the append before it (same
+    cache) is still running, so the plan it made from the lengths before the
+    wait is stale and is made again; the results must still equal the fused
+    step's, bit for bit, step by step."""
+    cfg = synth.custom(2, 16, 4, 300, 10, seed=41, steps=24)
+    case = Case(cfg)
+    a_cache, b_cache, warm = case.g, _clone_cache(case.g), _clone_cache(case.g)
+    B, Hq, steps = cfg.B, cfg.Hq, cfg.steps
+    rings = [torch.zeros(B, Hq, 64, 128, dtype=torch.float16, device="cuda") for _ in range(3)]
+    ws_a = hyq.workspace(hyq.hyq_decode_workspace(a_cache))
+    ws_b = hyq.workspace(hyq.hyq_decode_step_workspace(b_cache))
+    ws_w = hyq.workspace(hyq.hyq_decode_step_workspace(warm))
+    ks, vs, qs = _step_inputs(cfg, steps, 700)
+    o_a = [torch.full_like(q, float("nan")) for q in qs]
+    o_b = [torch.full_like(q, float("nan")) for q in qs]
+    l_a = [torch.full((B, Hq), float("nan"), dtype=torch.float32, device="cuda") for _ in qs]
+    l_b = [x.clone() for x in l_a]
+    # every kernel once outside the capture (launch attributes), on a scratch copy
+    hyq.hyq_append(warm, ks[0], vs[0], qs[0], rings[2])
+    hyq.hyq_decode(warm, qs[0], o_a[0], ws_w, lse=l_a[0])
+    hyq.hyq_decode_step(warm, qs[0], ks[0], vs[0], o_b[0], ws_w, q_ring=rings[2], lse=l_b[0])
+    torch.cuda.synchronize()
+
+    def body():
+        for s in range(steps):
+            hyq.hyq_append(a_cache, ks[s], vs[s], qs[s], rings[0])
+            hyq.hyq_decode(a_cache, qs[s], o_a[s], ws_a, lse=l_a[s])
+            hyq.hyq_decode_step(b_cache, qs[s], ks[s], vs[s], o_b[s], ws_b, q_ring=rings[1], lse=l_b[s])
+
+    _graph(body)
+    for s in range(steps):
+        assert torch.equal(o_a[s].view(torch.int16), o_b[s].view(torch.int16)), f"step {s}: outputs differ"
+        assert torch.equal(l_a[s].view(torch.int32), l_b[s].view(torch.int32)), f"step {s}: lse differs"
+    sa, sb = _state(a_cache, rings[0]), _state(b_cache, rings[1])
+    for k in sa:
+        assert np.array_equal(sa[k], sb[k]), f"{k} differs after {steps} steps"
+    assert a_cache.status() == 0 and b_cache.status() == 0
+
+
+@pytest.mark.parametrize("n_ctas", [7, 0])
+def test_graph_consecutive_steps_equal_eager(n_ctas):
+    """Fused steps on one cache back to back inside a CUDA graph (with 7
+    blocks the next launch starts on idle SMs before the previous one has
+    written seq_len) equal the same steps launched one by one."""
+    cfg = synth.custom(1, 32, 8, 700, 20, seed=43, steps=20)
+    case = Case(cfg)
+    g_cache, e_cache = case.g, _clone_cache(case.g)
+    B, Hq, steps = cfg.B, cfg.Hq, cfg.steps
+    rings = [torch.zeros(B, Hq, 64, 128, dtype=torch.float16, device="cuda") for _ in range(2)]
+    ws_g = hyq.workspace(hyq.hyq_decode_step_workspace(g_cache, n_ctas))
+    ws_e = hyq.workspace(hyq.hyq_decode_step_workspace(e_cache, n_ctas))
+    ks, vs, qs = _step_inputs(cfg, steps, 900)
+    o_g = [torch.full_like(q, float("nan")) for q in qs]
+    o_e = [torch.full_like(q, float("nan")) for q in qs]
+    for s in range(steps):
+        hyq.hyq_decode_step(e_cache, qs[s], ks[s], vs[s], o_e[s], ws_e, q_ring=rings[1], n_ctas=n_ctas)
+        torch.cuda.synchronize()
+
+    def body():
+        for s in range(steps):
+            hyq.hyq_decode_step(g_cache, qs[s], ks[s], vs[s], o_g[s], ws_g, q_ring=rings[0], n_ctas=n_ctas)
+
+    _graph(body)
+    for s in range(steps):
+        assert torch.equal(o_g[s].view(torch.int16), o_e[s].view(torch.int16)), f"step {s}: outputs differ"
+    sg, se = _state(g_cache, rings[0]), _state(e_cache, rings[1])
+    for k in sg:
+        assert np.array_equal(sg[k], se[k]), f"{k} differs after {steps} steps"
+    assert g_cache.status() == 0 and e_cache.status() == 0
