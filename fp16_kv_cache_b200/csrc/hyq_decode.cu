@@ -79,7 +79,10 @@ struct Ring {
 
 // MODE_STEP: the hybrid decode with the token append of the same step fused
 // in (hyq_decode_step): the cache is decoded as it is after the append.
-enum { MODE_HYBRID = 0, MODE_FP16 = 1, MODE_STEP = 2 };
+// MODE_VLONLY: the vertical-only ablation (hyq_decode_vl_only): the same
+// cache with its INT4 majority left out, i.e. attention over the vertical
+// lines and the window alone.
+enum { MODE_HYBRID = 0, MODE_FP16 = 1, MODE_STEP = 2, MODE_VLONLY = 3 };
 
 struct DecodeArgs {
   int B, Hq, Hkv, cap, W, vl_cap, U, n_ctas;
@@ -138,7 +141,7 @@ __device__ __forceinline__ UnitShape shape_of(const DecodeArgs &a, int T, int vl
     s.vlc = 0;
   }
   s.nwin = s.T < a.W ? s.T : a.W;
-  s.n4 = (s.L4 + I4_TOK - 1) / I4_TOK;
+  s.n4 = (MODE == MODE_VLONLY) ? 0 : (s.L4 + I4_TOK - 1) / I4_TOK;
   s.nv = (s.vlc + F16_ROWS - 1) / F16_ROWS;
   s.nw = (s.nwin + F16_ROWS - 1) / F16_ROWS;
   return s;
@@ -1248,8 +1251,9 @@ static bool cost_fits(int U, int cap, int vl_cap, int mode) {
   return static_cast<int64_t>(U) * per_unit < (static_cast<int64_t>(1) << 31) - 1;
 }
 
-extern "C" hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, float *lse,
-                                 int32_t n_ctas, void *ws, size_t ws_bytes, void *stream) {
+template <int MODE>
+static hyq_status decode_entry(const hyq_cache *c, const void *q, void *o, float *lse, int32_t n_ctas, void *ws,
+                               size_t ws_bytes, void *stream) {
   hyq_status s = hyq_check_cache(c);
   if (s != HYQ_OK) return s;
   if (!q || !o) return HYQ_ERR_INVALID;
@@ -1271,8 +1275,17 @@ extern "C" hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, flo
   a.counters = static_cast<int32_t *>(ws);
   a.part = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + (static_cast<size_t>(U) * 4 + 255) / 256 * 256);
   a.status = c->dev_status;
-  return dispatch_decode<MODE_HYBRID>(G, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? HYQ_OK
-                                                                                              : HYQ_ERR_CUDA;
+  return dispatch_decode<MODE>(G, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
+}
+
+extern "C" hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, float *lse,
+                                 int32_t n_ctas, void *ws, size_t ws_bytes, void *stream) {
+  return decode_entry<MODE_HYBRID>(c, q, o, lse, n_ctas, ws, ws_bytes, stream);
+}
+
+extern "C" hyq_status hyq_decode_vl_only(const hyq_cache *c, const void *q, void *o, float *lse,
+                                         int32_t n_ctas, void *ws, size_t ws_bytes, void *stream) {
+  return decode_entry<MODE_VLONLY>(c, q, o, lse, n_ctas, ws, ws_bytes, stream);
 }
 
 // Fused append + decode: the workspace of hyq_decode plus 256 bytes for the

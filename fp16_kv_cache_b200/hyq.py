@@ -65,6 +65,7 @@ EXPORTS = [
     ("hyq_vl_apply", ctypes.c_int, [_CP, _P, _I32, _P, _P, _P, _P]),
     ("hyq_decode_workspace", _SZ, [_CP, _I32]),
     ("hyq_decode", ctypes.c_int, [_CP, _P, _P, _P, _I32, _P, _SZ, _P]),
+    ("hyq_decode_vl_only", ctypes.c_int, [_CP, _P, _P, _P, _I32, _P, _SZ, _P]),
     ("hyq_decode_step_workspace", _SZ, [_CP, _I32]),
     ("hyq_decode_step", ctypes.c_int, [_CP, _P, _P, _P, _P, _I32, _P, _P, _I32, _P, _SZ, _P]),
     ("hyq_decode_noalloc", ctypes.c_int, [_CP, _P, _P, _P, _P]),
@@ -225,6 +226,13 @@ def hyq_decode_workspace(cache: HybridCache, n_ctas: int = 0) -> int:
 def hyq_decode(cache: HybridCache, q, o, ws, lse=None, n_ctas: int = 0, stream=None):
     _check(lib().hyq_decode(cache.ref(), _ptr(q), _ptr(o), _ptr(lse), n_ctas, _ptr(ws),
                             ws.numel() * ws.element_size(), _stream(stream)), "hyq_decode")
+
+
+def hyq_decode_vl_only(cache: HybridCache, q, o, ws, lse=None, n_ctas: int = 0, stream=None):
+    """The vertical-only ablation: attention over the vertical-line rows and
+    the window alone (workspace of hyq_decode_workspace)."""
+    _check(lib().hyq_decode_vl_only(cache.ref(), _ptr(q), _ptr(o), _ptr(lse), n_ctas, _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)), "hyq_decode_vl_only")
 
 
 def hyq_decode_step_workspace(cache: HybridCache, n_ctas: int = 0) -> int:

@@ -241,6 +241,21 @@ hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, float *lse,
                       int32_t n_ctas, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * hyq_decode_vl_only -- the vertical-only ablation of hyq_decode: attention
+ * over the cache's vertical-line rows and local window alone, with the INT4
+ * majority left out (the sparse-attention variant that drops the long-tail
+ * positions).  Method: AI Radio episode "HyQuant: Hybrid-Precision
+ * Quantization for LLM Attention", "Paper Summary" (vertical-only variants
+ * discard the long-tail positions that HyQuant keeps in low precision) and
+ * "Improvements and Ablation Studies" (Table twelve compares the two).
+ * Arguments, workspace (hyq_decode_workspace) and errors as hyq_decode; the
+ * cache is only read.  A unit with no vertical line and an empty window
+ * gets o = 0, lse = -inf.
+ */
+hyq_status hyq_decode_vl_only(const hyq_cache *c, const void *q, void *o, float *lse,
+                              int32_t n_ctas, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * hyq_decode_step -- one whole decode step in a single launch: the append of
  * hyq_append(c, k_new, v_new, q, q_ring, n_q) fused into hyq_decode(c, q,
  * o, lse).  Results (o, lse, and the cache, ring and seq_len after the

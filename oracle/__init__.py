@@ -79,6 +79,8 @@ def lib():
         L.hyqo_dequant_row.argtypes = [P, P, P]
         L.hyqo_decode.restype = ctypes.c_int
         L.hyqo_decode.argtypes = [ctypes.POINTER(_Cache), P, P, ctypes.c_int32, P, P]
+        L.hyqo_decode_vl_only.restype = ctypes.c_int
+        L.hyqo_decode_vl_only.argtypes = [ctypes.POINTER(_Cache), P, P, ctypes.c_int32, P, P]
         L.hyqo_decode_fp16.restype = ctypes.c_int
         L.hyqo_decode_fp16.argtypes = [P, P, P, P, ctypes.c_int32, ctypes.c_int32,
                                        ctypes.c_int32, ctypes.c_int32, P,
@@ -170,20 +172,32 @@ def _cache_struct(c):
     return s
 
 
-def decode(cache, q, units=None):
-    """fp64 decode over the oracle's hybrid cache.  q: [B][Hq][128] fp16.
-    Returns (o [B][Hq][128] f64, lse [B][Hq] f64); rows of units not listed
-    are NaN."""
+def _decode(fn, what, cache, q, units):
     q = _c16(q)
     o = np.full((cache.B, cache.Hq, D), np.nan)
     lse = np.full((cache.B, cache.Hq), np.nan)
     u = None if units is None else np.ascontiguousarray(units, np.int32)
     s = _cache_struct(cache)
-    rc = lib().hyqo_decode(ctypes.byref(s), _ptr(q), _ptr(u),
-                           0 if u is None else len(u), _ptr(o), _ptr(lse))
+    rc = fn(ctypes.byref(s), _ptr(q), _ptr(u), 0 if u is None else len(u), _ptr(o), _ptr(lse))
     if rc != 0:
-        raise ValueError(f"oracle decode: inconsistent cache (code {rc})")
+        raise ValueError(f"oracle {what}: inconsistent cache (code {rc})")
     return o, lse
+
+
+def decode(cache, q, units=None):
+    """fp64 decode over the oracle's hybrid cache.  q: [B][Hq][128] fp16.
+    Returns (o [B][Hq][128] f64, lse [B][Hq] f64); rows of units not listed
+    are NaN."""
+    return _decode(lib().hyqo_decode, "decode", cache, q, units)
+
+
+def decode_vl_only(cache, q, units=None):
+    """The vertical-only ablation (AI Radio episode "HyQuant: Hybrid-Precision
+    Quantization for LLM Attention", "Improvements and Ablation Studies",
+    Table twelve): attention over the cache's vertical-line rows and window
+    alone, the quantized majority left out.  Same arguments and results as
+    decode."""
+    return _decode(lib().hyqo_decode_vl_only, "decode_vl_only", cache, q, units)
 
 
 def decode_fp16(q, k, v, seq_len, Hq, units=None):

@@ -225,32 +225,45 @@ static void view_row(const unit_view *u, int32_t p, double k[HYQO_D], double v[H
   }
 }
 
-/* softmax(q . k_p / sqrt(d)) weighted sum of v_p over positions [0, T).
- * Two plain passes: logits and their max, then weights and the sum. */
-static void attend_one_head(const unit_view *u, const double *qd, double *o, double *lse) {
+/* Whether position p is in the unit's key/value multiset: every position of
+ * [0, T) for the hybrid decode; for the vertical-only ablation only the
+ * vertical-line positions and the window. */
+static int in_multiset(const unit_view *u, int32_t p, int vl_only) {
+  if (!vl_only) return 1;
+  return p >= u->T - u->c->window || u->slot_of[p] >= 0;
+}
+
+/* softmax(q . k_p / sqrt(d)) weighted sum of v_p over the positions of the
+ * multiset.  Two plain passes: logits and their max, then weights and the
+ * sum. */
+static void attend_one_head(const unit_view *u, const double *qd, int vl_only, double *o, double *lse) {
   int32_t T = u->T;
   double scale = 1.0 / sqrt((double)HYQO_D);
   double *logit = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
   double k[HYQO_D], v[HYQO_D];
   double m = -INFINITY;
+  int32_t n = 0; /* positions in the multiset */
   for (int32_t p = 0; p < T; ++p) {
+    if (!in_multiset(u, p, vl_only)) continue;
     view_row(u, p, k, v);
     double s = 0.0;
     for (int d = 0; d < HYQO_D; ++d) s += qd[d] * k[d];
     logit[p] = s * scale;
     if (logit[p] > m) m = logit[p];
+    ++n;
   }
   double l = 0.0;
   double acc[HYQO_D];
   for (int d = 0; d < HYQO_D; ++d) acc[d] = 0.0;
   for (int32_t p = 0; p < T; ++p) {
+    if (!in_multiset(u, p, vl_only)) continue;
     view_row(u, p, k, v);
     double w = exp(logit[p] - m);
     l += w;
     for (int d = 0; d < HYQO_D; ++d) acc[d] += w * v[d];
   }
-  for (int d = 0; d < HYQO_D; ++d) o[d] = (T > 0) ? acc[d] / l : 0.0;
-  *lse = (T > 0) ? m + log(l) : -INFINITY;
+  for (int d = 0; d < HYQO_D; ++d) o[d] = (n > 0) ? acc[d] / l : 0.0;
+  *lse = (n > 0) ? m + log(l) : -INFINITY;
   free(logit);
 }
 
@@ -258,8 +271,8 @@ static int64_t n_units_of(const hyqo_cache *c) {
   return (int64_t)c->batch * c->n_kv_heads;
 }
 
-int hyqo_decode(const hyqo_cache *c, const uint16_t *q, const int32_t *units,
-                int32_t n_units, double *o, double *lse) {
+static int decode_units(const hyqo_cache *c, const uint16_t *q, const int32_t *units,
+                        int32_t n_units, int vl_only, double *o, double *lse) {
   if (c->n_q_heads % c->n_kv_heads != 0) return -1;
   int G = c->n_q_heads / c->n_kv_heads;
   int64_t total = units ? n_units : n_units_of(c);
@@ -279,7 +292,7 @@ int hyqo_decode(const hyqo_cache *c, const uint16_t *q, const int32_t *units,
       int64_t h = (int64_t)u.b * c->n_q_heads + (int64_t)u.kvh * G + hg;
       double qd[HYQO_D], od[HYQO_D], l;
       for (int d = 0; d < HYQO_D; ++d) qd[d] = hyqo_half_to_double(q[h * HYQO_D + d]);
-      attend_one_head(&u, qd, od, &l);
+      attend_one_head(&u, qd, vl_only, od, &l);
       if (o)
         for (int d = 0; d < HYQO_D; ++d) o[h * HYQO_D + d] = od[d];
       if (lse) lse[h] = l;
@@ -287,6 +300,16 @@ int hyqo_decode(const hyqo_cache *c, const uint16_t *q, const int32_t *units,
     view_close(&u);
   }
   return err;
+}
+
+int hyqo_decode(const hyqo_cache *c, const uint16_t *q, const int32_t *units,
+                int32_t n_units, double *o, double *lse) {
+  return decode_units(c, q, units, n_units, 0, o, lse);
+}
+
+int hyqo_decode_vl_only(const hyqo_cache *c, const uint16_t *q, const int32_t *units,
+                        int32_t n_units, double *o, double *lse) {
+  return decode_units(c, q, units, n_units, 1, o, lse);
 }
 
 int hyqo_decode_fp16(const uint16_t *q, const uint16_t *k, const uint16_t *v,

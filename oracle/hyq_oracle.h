@@ -88,6 +88,14 @@ typedef struct {
 int hyqo_decode(const hyqo_cache *c, const uint16_t *q, const int32_t *units,
                 int32_t n_units, double *o, double *lse);
 
+/* The vertical-only ablation (AI Radio episode "HyQuant: Hybrid-Precision
+ * Quantization for LLM Attention", "Paper Summary" and "Improvements and
+ * Ablation Studies", Table twelve): hyqo_decode with the quantized majority
+ * left out, i.e. attention over the VL rows and the window rows alone.  A
+ * unit whose multiset is empty gets o = 0 and lse = -inf. */
+int hyqo_decode_vl_only(const hyqo_cache *c, const uint16_t *q, const int32_t *units,
+                        int32_t n_units, double *o, double *lse);
+
 /* Attention over an all-FP16 cache k, v: [B][Hkv][cap][128], T = seq_len[b]. */
 int hyqo_decode_fp16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const int32_t *seq_len, int32_t B, int32_t Hq, int32_t Hkv,

@@ -65,12 +65,14 @@ class Case:
             out += [(b, h * G + i) for i in range(G)]
         return out
 
-    def decode_gpu(self, q, n_ctas=0):
+    def decode_gpu(self, q, n_ctas=0, decode=None):
+        """hyq_decode (or another entry with its arguments, e.g. the
+        vertical-only hyq_decode_vl_only) on the GPU cache."""
         qd = dev(q)
         o = torch.empty_like(qd)
         lse = torch.empty(qd.shape[:2], dtype=torch.float32, device="cuda")
         ws = hyq.workspace(hyq.hyq_decode_workspace(self.g, n_ctas))
-        hyq.hyq_decode(self.g, qd, o, ws, lse=lse, n_ctas=n_ctas)
+        (decode or hyq.hyq_decode)(self.g, qd, o, ws, lse=lse, n_ctas=n_ctas)
         torch.cuda.synchronize()
         return host(o.float()).astype(np.float64), host(lse).astype(np.float64)
 

@@ -291,6 +291,73 @@ def test_decode_gqa_groups_read_their_own_kv_head():
         assert np.allclose(o[0, h], ro[0], atol=1e-12)
 
 
+# ------------------------------------------------ vertical-only ablation
+@pytest.mark.parametrize("T,k", [(700, 17), (300, 0), (100, 0), (1, 0)])
+def test_decode_vl_only_is_attention_over_vertical_lines_and_window(T, k):
+    """The ablation's multiset, gathered here from the raw fp16 inputs: the
+    selected positions plus the last W positions, nothing quantized."""
+    cfg = synth.custom(2, 8, 2, T, k, seed=13)
+    c, K, V, vl = _build(cfg)
+    qv = synth.q(cfg, 4)
+    o, lse = oracle.decode_vl_only(c, qv)
+    for b in range(cfg.B):
+        for h in range(cfg.Hkv):
+            keep = sorted(set(vl[b, h, :k].tolist()) | set(range(max(0, T - 128), T)))
+            ro, rl = _sdpa(qv[b, h * 4:(h + 1) * 4], K[b, h, keep].astype(np.float64),
+                           V[b, h, keep].astype(np.float64), 4)
+            assert np.allclose(o[b, h * 4:(h + 1) * 4], ro, rtol=0, atol=1e-12)
+            assert np.allclose(lse[b, h * 4:(h + 1) * 4], rl, rtol=0, atol=1e-11)
+
+
+def test_decode_vl_only_with_every_old_position_selected_equals_hybrid():
+    cfg = synth.custom(1, 8, 2, 600, 600 - 128, seed=9)
+    allpos = np.broadcast_to(np.arange(600 - 128, dtype=np.int32), (1, 2, 472)).copy()
+    c, K, V, _ = _build(cfg, vl=allpos)
+    qv = synth.q(cfg, 5)
+    o, lse = oracle.decode_vl_only(c, qv)
+    o2, lse2 = oracle.decode(c, qv)
+    assert np.allclose(o, o2, rtol=0, atol=1e-12) and np.allclose(lse, lse2, rtol=0, atol=1e-11)
+
+
+def test_decode_vl_only_drops_exactly_the_quantized_positions():
+    """Moving one position from the quantized majority into the vertical
+    lines changes the ablation's result and leaves the set of the others."""
+    cfg = synth.custom(1, 4, 1, 400, 8, seed=21)
+    c, K, V, vl = _build(cfg)
+    qv = synth.q(cfg, 6)
+    o1, _ = oracle.decode_vl_only(c, qv)
+    extra = next(p for p in range(400 - 128) if p not in set(vl[0, 0].tolist()))
+    vl2 = np.sort(np.append(vl[0, 0], extra)).astype(np.int32)[None, None]
+    c2 = oracle.OracleCache(1, 4, 1, cfg.capacity, 9)
+    c2.load_prompt(K, V, [400])
+    c2.apply_vl(vl2, K, V)
+    o2, _ = oracle.decode_vl_only(c2, qv)
+    keep = sorted(set(vl2[0, 0].tolist()) | set(range(400 - 128, 400)))
+    ro, _ = _sdpa(qv[0], K[0, 0, keep].astype(np.float64), V[0, 0, keep].astype(np.float64), 4)
+    assert np.allclose(o2[0], ro, rtol=0, atol=1e-12)
+    assert not np.allclose(o1, o2, rtol=0, atol=1e-9)
+
+
+def test_ablation_keeping_the_quantized_tail_cuts_the_error():
+    """The ablation the pages discuss (Table twelve: dropping the long-tail
+    positions costs accuracy), reproduced on the synthetic workload: against
+    exact FP16 attention, the hybrid cache's error is a small fraction of the
+    vertical-only variant's, for random decode queries and for queries drawn
+    like the selection queries."""
+    cfg = synth.config(1)
+    K, V, planted = synth.kv_full(cfg)
+    c = oracle.OracleCache(cfg.B, cfg.Hq, cfg.Hkv, cfg.capacity, cfg.k)
+    c.load_prompt(K, V, [cfg.T] * cfg.B)
+    c.apply_vl(planted, K, V)
+    for q in (synth.q(cfg, 100), synth.qsel(cfg, 0)[None, :, cfg.n_q - 1]):
+        ref, _ = oracle.decode_fp16(q, K, V, [cfg.T], cfg.Hq)
+        err = {}
+        for name, fn in (("hybrid", oracle.decode), ("vl_only", oracle.decode_vl_only)):
+            o, _ = fn(c, q)
+            err[name] = np.linalg.norm(o - ref) / np.linalg.norm(ref)
+        assert 5 * err["hybrid"] < err["vl_only"], err
+
+
 # --------------------------------------------------------------- selection
 def _select_by_torch(q_rows, kk, T, n_cand, k, n_q, G):
     """Brute force: full fp64 causal softmax, column sums, stable sort."""
