@@ -102,6 +102,43 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense fp16/bf16 tensor TFLOP/s (burst): measured, else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
+def prefill_kernels(cfg, t_ms):
+    """Rooflines of the prompt-side calls timed while the layer caches are
+    built: hyq_prefill (HBM: per unit T rows of K and V in, 160 B of codes
+    and scale/zero out per packed row, the window rows out), hyq_select_vl in
+    prefill mode (tensor: 2 passes of 2*128 flop per causal (query row, key)
+    pair) and hyq_vl_apply in prefill mode (HBM: 1028 B per selected row)."""
+    U, G, T, W, k = cfg.B * cfg.Hkv, cfg.Hq // cfg.Hkv, cfg.T, 128, cfg.k
+    hbm, hbm_kind = measured_peaks()
+    tc, tc_kind = measured_tensor_peak()
+    n_old, nwin = max(0, T - W), min(T, W)
+    b_prefill = U * (T * 512 + n_old * 160 + nwin * 512)
+    pairs = G * sum(max(0, T - 63 + i) for i in range(64))  # causal (row, key) pairs per unit
+    f_select = 2 * 2 * 128 * pairs * U
+    b_apply = U * k * 1028
+    out = {}
+    for name, ms, amount, unit, peak, kind in (
+            ("hyq_prefill", t_ms[0], b_prefill, "GB/s", hbm, hbm_kind),
+            ("hyq_select_vl (prefill mode)", t_ms[1], f_select, "TFLOP/s", tc, tc_kind),
+            ("hyq_vl_apply (prefill mode)", t_ms[2], b_apply, "GB/s", hbm, hbm_kind)):
+        rate = amount / (ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
+        out[name] = {"us": round(1000 * ms, 2), "achieved": round(rate, 1 if unit == "GB/s" else 2),
+                     "unit": unit, "per_launch": int(amount), "peak": peak,
+                     "frac": round(rate / peak, 4), "peak_source": kind}
+    return out
+
+
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -165,23 +202,36 @@ class ClockSampler:
 # --------------------------------------------------------------- setup
 def setup_layers(torch, hyq, synth, cfg, cap, n_layers):
     """Build n_layers hybrid caches from the workload's prompt, entirely with
-    the library: prefill -> select_vl (prefill mode) -> vl_apply."""
+    the library: prefill -> select_vl (prefill mode) -> vl_apply.  Returns the
+    caches, the prompt's K/V on the device, and the CUDA-event times (ms) of
+    the last layer's three calls (every kernel has run before by then)."""
     K, V, _ = synth.kv_full(cfg, cap)
     Kd = torch.from_numpy(K).cuda()
     Vd = torch.from_numpy(V).cuda()
     qs = torch.from_numpy(np.stack([synth.qsel(cfg, b) for b in range(cfg.B)])).cuda()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     layers = []
-    for _ in range(n_layers):
+    for li in range(n_layers):
+        timed = li == n_layers - 1
         c = hyq.HybridCache(cfg.B, cfg.Hq, cfg.Hkv, cap, cfg.k)
         c.seq_len.fill_(cfg.T)
-        hyq.hyq_prefill(c, Kd, Vd)
         pos = torch.zeros(cfg.B, cfg.Hkv, cfg.k, dtype=torch.int32, device="cuda")
         ws = hyq.workspace(hyq.hyq_select_vl_workspace(c, N_Q))
+        if timed:
+            ev[0].record()
+        hyq.hyq_prefill(c, Kd, Vd)
+        if timed:
+            ev[1].record()
         hyq.hyq_select_vl(c, qs, cfg.k, pos, ws, k_full=Kd)
+        if timed:
+            ev[2].record()
         hyq.hyq_vl_apply(c, pos, Kd, Vd)
+        if timed:
+            ev[3].record()
         layers.append(c)
     torch.cuda.synchronize()
-    return layers, Kd, Vd
+    t_ms = [ev[i].elapsed_time(ev[i + 1]) for i in range(3)]
+    return layers, Kd, Vd, t_ms
 
 
 def run_ours(args):
@@ -205,7 +255,7 @@ def run_ours(args):
     n_layers = int(min(8, max(2, math.ceil(L2_DEFEAT_BYTES / algorithmic_bytes(cfg.B, cfg.Hq, cfg.Hkv, cfg.T, cfg.k)))))
     per_layer_tokens = (K_steps + W_steps + args.e2e_steps) // n_layers + 2
     cap = ((cfg.T + per_layer_tokens + 127) // 128) * 128
-    layers, Kd, Vd = setup_layers(torch, hyq, synth, cfg, cap, n_layers)
+    layers, Kd, Vd, t_setup = setup_layers(torch, hyq, synth, cfg, cap, n_layers)
     B, Hq, Hkv = cfg.B, cfg.Hq, cfg.Hkv
     dev = torch.device("cuda", local)
 
@@ -371,6 +421,7 @@ def run_ours(args):
                      "bytes_per_launch": int(bytes_per_decode)},
         "e2e": e2e,
         "gpu_launches": total_launches,
+        "other_kernels": prefill_kernels(cfg, t_setup),
     }
     if clk:
         line["clocks"] = clk
