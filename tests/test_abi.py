@@ -107,3 +107,37 @@ def test_append_and_prefill_argument_checks(L):
     assert L.hyq_prefill(ctypes.byref(c), None, 0x2000, None) == 1
     assert L.hyq_decode_fp16(0x1000, 0x2000, 0x3000, 0x4000, 1, 6, 2, 4096, 0x5000, None, 0,
                              0x6000, 1 << 20, None, None) == 2
+
+
+@pytest.mark.parametrize("field,value,code", [("head_dim", 64, 2), ("n_q_heads", 7, 1), ("blocks", 0, 1),
+                                              ("vl_pos", 0x10008, 3)])
+def test_decode_vl_only_checks_like_decode(L, field, value, code):
+    c = _desc(**{field: value})
+    args = (0x20000000, 0x30000000, None, 0, 0x40000000, 1 << 30, None)
+    assert L.hyq_decode_vl_only(ctypes.byref(c), *args) == code == L.hyq_decode(ctypes.byref(c), *args)
+
+
+def test_decode_vl_only_requires_workspace(L):
+    c = _desc()
+    need = L.hyq_decode_workspace(ctypes.byref(c), 8)
+    assert L.hyq_decode_vl_only(ctypes.byref(c), 0x20000000, 0x30000000, None, 8, None, 0, None) == 4
+    assert L.hyq_decode_vl_only(ctypes.byref(c), 0x20000000, 0x30000000, None, 8, 0x40000000, need - 1, None) == 4
+    assert L.hyq_decode_vl_only(ctypes.byref(c), 0x20000000, 0x30000008, None, 8, 0x40000000, need, None) == 3
+    assert L.hyq_decode_vl_only(ctypes.byref(c), None, 0x30000000, None, 8, 0x40000000, need, None) == 1
+
+
+def test_decode_step_argument_checks(L):
+    c = _desc()
+    step = L.hyq_decode_step
+    need = L.hyq_decode_step_workspace(ctypes.byref(c), 8)
+    assert need == L.hyq_decode_workspace(ctypes.byref(c), 8) + 256
+    q, kn, vn, ring, o, ws = 0x20000000, 0x21000000, 0x22000000, 0x23000000, 0x30000000, 0x40000000
+    assert step(ctypes.byref(c), q, None, vn, ring, 64, o, None, 8, ws, need, None) == 1        # k_new
+    assert step(ctypes.byref(c), q, kn, vn, ring, 0, o, None, 8, ws, need, None) == 1           # n_q
+    assert step(ctypes.byref(c), q, kn, vn, ring, 1025, o, None, 8, ws, need, None) == 1        # n_q
+    assert step(ctypes.byref(c), q, kn + 8, vn, ring, 64, o, None, 8, ws, need, None) == 3      # alignment
+    assert step(ctypes.byref(c), q, kn, vn, ring + 8, 64, o, None, 8, ws, need, None) == 3
+    assert step(ctypes.byref(c), q, kn, vn, ring, 64, o, None, -1, ws, need, None) == 1         # n_ctas
+    assert step(ctypes.byref(c), q, kn, vn, ring, 64, o, None, 8, ws, need - 1, None) == 4      # workspace
+    assert step(ctypes.byref(c), q, kn, vn, None, 0, o, None, 8, ws, need - 1, None) == 4       # no ring: n_q free
+    assert step(ctypes.byref(_desc(window=256)), q, kn, vn, ring, 64, o, None, 8, ws, need, None) == 2
