@@ -132,10 +132,10 @@ def prefill_kernels(cfg, t_ms):
             ("hyq_prefill", t_ms[0], b_prefill, "GB/s", hbm, hbm_kind),
             ("hyq_select_vl (prefill mode)", t_ms[1], f_select, "TFLOP/s", tc, tc_kind),
             ("hyq_vl_apply (prefill mode)", t_ms[2], b_apply, "GB/s", hbm, hbm_kind)):
-        rate = amount / (ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
-        out[name] = {"us": round(1000 * ms, 2), "achieved": round(rate, 1 if unit == "GB/s" else 2),
+        rate = amount / (ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12) if ms > 0 else None
+        out[name] = {"us": round(1000 * ms, 2), "achieved": None if rate is None else round(rate, 2),
                      "unit": unit, "per_launch": int(amount), "peak": peak,
-                     "frac": round(rate / peak, 4), "peak_source": kind}
+                     "frac": None if rate is None else round(rate / peak, 4), "peak_source": kind}
     return out
 
 
