@@ -20,6 +20,9 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "hyq_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
+# A library built elsewhere from a modified copy of the source: the pin tests
+# run against it to show that a planted mistake makes a pin fail.
+_LIB_OVERRIDE = os.environ.get("HYQ_ORACLE_LIB")
 _lib = None
 
 D = 128
@@ -28,18 +31,27 @@ NG = 4
 ROW_BYTES = 64
 
 
+def compile_to(src: str, out: str) -> str:
+    """Compile an oracle source file (its header beside it) with IEEE
+    fp32/fp64 semantics: no FMA contraction, no fast-math."""
+    cmd = [
+        "gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+        "-ffp-contract=off", "-fno-fast-math", "-frounding-math",
+        "-o", out, src, "-lm",
+    ]
+    subprocess.check_call(cmd, cwd=os.path.dirname(os.path.abspath(src)))
+    return out
+
+
 def build(force: bool = False) -> str:
-    """Compile the oracle with IEEE fp32/fp64 semantics (no FMA contraction,
-    no fast-math) into ``oracle/liboracle.so``."""
+    """Compile the oracle into ``oracle/liboracle.so`` (or return the
+    library named by HYQ_ORACLE_LIB, built by its maker)."""
+    if _LIB_OVERRIDE:
+        return _LIB_OVERRIDE
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < max(
         os.path.getmtime(_SRC), os.path.getmtime(os.path.join(_HERE, "hyq_oracle.h"))
     ):
-        cmd = [
-            "gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
-            "-ffp-contract=off", "-fno-fast-math", "-frounding-math",
-            "-o", _LIB, _SRC, "-lm",
-        ]
-        subprocess.check_call(cmd, cwd=_HERE)
+        compile_to(_SRC, _LIB)
     return _LIB
 
 
@@ -60,8 +72,7 @@ class _Cache(ctypes.Structure):
 def lib():
     global _lib
     if _lib is None:
-        build()
-        L = ctypes.CDLL(_LIB)
+        L = ctypes.CDLL(build())
         P = ctypes.c_void_p
         L.hyqo_half_to_double.restype = ctypes.c_double
         L.hyqo_half_to_double.argtypes = [ctypes.c_uint16]

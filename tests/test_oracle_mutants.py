@@ -1,0 +1,72 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of the C oracle (a text substitution),
+builds the copy with the oracle's own flags, and runs the pins expected to
+notice it in a child process pointed at the mutant library (HYQ_ORACLE_LIB).
+The pins must fail.  The unmodified source built the same way must pass them,
+which also shows that the child really loads the library it is given.
+"""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "hyq_oracle.c")
+HDR = os.path.join(ROOT, "oracle", "hyq_oracle.h")
+
+# (mistake, text in hyq_oracle.c, replacement, pins that must fail: a -k expression)
+MUTANTS = [
+    ("softmax scale 1/d instead of 1/sqrt(d)",
+     "double scale = 1.0 / sqrt((double)HYQO_D);", "double scale = 1.0 / (double)HYQO_D;",
+     "decode_matches_torch"),
+    ("codes rounded half away from zero",
+     "float ri = rintf(r);", "float ri = roundf(r);", "quantizer_hand_vectors"),
+    ("scale = range / 16",
+     "float s32 = diff / 15.0f;", "float s32 = diff / 16.0f;", "quantizer_hand_vectors"),
+    ("zero point dropped in the dequantization",
+     "out[c] = z + (double)code[c] * s;", "out[c] = (double)code[c] * s;", "dequant_error"),
+    ("query head reads the wrong KV head",
+     "(int64_t)u.kvh * G + hg;", "(int64_t)hg * c->n_kv_heads + u.kvh;", "gqa_groups"),
+    ("window boundary off by one",
+     "if (p >= u->T - W) {", "if (p > u->T - W) {", "decode_matches_torch"),
+    ("selection without the causal mask",
+     "int32_t last = T - n_q + i; /* causal: keys 0..last */", "int32_t last = T - 1;",
+     "select_matches_bruteforce"),
+    ("ties go to the higher position",
+     "return (x->p < y->p) ? -1 : (x->p > y->p);", "return (x->p > y->p) ? -1 : (x->p < y->p);",
+     "ties_go_to_the_lower"),
+    ("vertical-only variant keeps the quantized positions",
+     "return p >= u->T - u->c->window || u->slot_of[p] >= 0;", "return 1;", "vl_only"),
+]
+
+
+def _run_pins(tmp_path, source, pins):
+    d = tmp_path / "src"
+    d.mkdir()
+    (d / "hyq_oracle.c").write_text(source)
+    shutil.copy(HDR, d / "hyq_oracle.h")
+    lib = oracle.compile_to(str(d / "hyq_oracle.c"), str(tmp_path / "liboracle_variant.so"))
+    env = dict(os.environ, HYQ_ORACLE_LIB=lib, OMP_NUM_THREADS="4")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"), "-k", pins],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    return r.returncode, r.stdout[-2000:]
+
+
+def test_unmodified_oracle_passes_the_selected_pins(tmp_path):
+    pins = " or ".join(sorted({m[3] for m in MUTANTS}))
+    rc, out = _run_pins(tmp_path, open(SRC).read(), pins)
+    assert rc == 0, out
+
+
+@pytest.mark.parametrize("what,old,new,pins", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_a_planted_mistake_fails_a_pin(tmp_path, what, old, new, pins):
+    src = open(SRC).read()
+    assert old in src, f"mutation site not found: {old}"
+    rc, out = _run_pins(tmp_path, src.replace(old, new), pins)
+    assert rc == 1, f"{what}: no pin failed (pytest exit {rc})\n{out}"
