@@ -19,6 +19,13 @@ Readings where the pages are silent:
   * re-selection from the cache keeps FP16 rows only for positions selected
     again; newly selected positions have no FP16 source left and stay INT4
     ("unpromoted"); dropped positions fall back to their codes.
+
+Staged promotion (optional, ``stage`` > 0; the pages say nothing about it):
+the FP16 rows of the ``stage`` most recently quantized positions, [T - W -
+stage, T - W), are also kept in a ring (slot = p % stage), filled from the
+prompt and by every append with the row leaving the window.  A cache-mode
+re-selection then promotes a newly selected position from that ring when it
+lies in the staged range; only older new positions stay unpromoted.
 """
 from __future__ import annotations
 
@@ -28,11 +35,14 @@ from . import D, ROW_BYTES, pack
 
 
 class OracleCache:
-    def __init__(self, B, Hq, Hkv, cap, vl_cap, W=128):
+    def __init__(self, B, Hq, Hkv, cap, vl_cap, W=128, stage=0):
         assert Hq % Hkv == 0
         vl_cap = max(int(vl_cap), 1)
         self.B, self.Hq, self.Hkv, self.cap, self.vl_cap, self.W = B, Hq, Hkv, cap, vl_cap, W
         U = B * Hkv
+        self.stage = int(stage)
+        self.stage_k = np.zeros((U, max(self.stage, 1), D), np.uint16)
+        self.stage_v = np.zeros((U, max(self.stage, 1), D), np.uint16)
         self.k_codes = np.zeros((U, cap, ROW_BYTES), np.uint8)
         self.v_codes = np.zeros((U, cap, ROW_BYTES), np.uint8)
         self.k_sz = np.zeros((U, cap, 8), np.uint16)
@@ -73,8 +83,16 @@ class OracleCache:
                 for p in range(n_old, T):
                     self.win_k[u, p % self.W] = K[b, h, p]
                     self.win_v[u, p % self.W] = V[b, h, p]
+                for p in range(max(0, n_old - self.stage), n_old):
+                    self.stage_k[u, p % self.stage] = K[b, h, p]
+                    self.stage_v[u, p % self.stage] = V[b, h, p]
                 self.vl_count[u] = 0
                 self.vl_pos[u] = -1
+
+    def staged(self, b, p):
+        """Whether position p of batch b has its FP16 rows in the staging ring."""
+        n_old = int(self.seq_len[b]) - self.W
+        return self.stage > 0 and max(0, n_old - self.stage) <= p < n_old
 
     # ------------------------------------------------------------ VL set
     def apply_vl(self, pos, K_full=None, V_full=None, units=None):
@@ -101,10 +119,18 @@ class OracleCache:
                     kept = new
                 else:
                     old = {int(self.vl_pos[u, i]): i for i in range(self.vl_count[u])}
-                    kept = [p for p in new if p in old]
+                    kept, rows_k, rows_v = [], [], []
+                    for p in new:
+                        if p in old:
+                            src_k, src_v = self.vl_k[u, old[p]], self.vl_v[u, old[p]]
+                        elif self.staged(b, p):
+                            src_k, src_v = self.stage_k[u, p % self.stage], self.stage_v[u, p % self.stage]
+                        else:
+                            continue
+                        kept.append(p)
+                        rows_k.append(src_k.copy())
+                        rows_v.append(src_v.copy())
                     unpromoted += len(new) - len(kept)
-                    rows_k = [self.vl_k[u, old[p]].copy() for p in kept]
-                    rows_v = [self.vl_v[u, old[p]].copy() for p in kept]
                 self.vl_pos[u] = -1
                 for i, p in enumerate(kept):
                     self.vl_pos[u, i] = p
@@ -127,6 +153,9 @@ class OracleCache:
                 u = b * self.Hkv + h
                 if T >= self.W:
                     p_out = T - self.W
+                    if self.stage:
+                        self.stage_k[u, p_out % self.stage] = self.win_k[u, slot]
+                        self.stage_v[u, p_out % self.stage] = self.win_v[u, slot]
                     c, s, bad = pack(self.win_k[u, slot])
                     assert bad == 0
                     self.k_codes[u, p_out], self.k_sz[u, p_out] = c[0], s[0]

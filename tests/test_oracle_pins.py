@@ -461,3 +461,49 @@ def test_cache_mode_reselection_keeps_only_known_fp16_rows():
     assert n == 3
     assert list(c.vl_pos[0, :c.vl_count[0]]) == [10, 60, 250]
     assert np.array_equal(c.vl_k[0, 1], K[0, 0, 60].view(np.uint16))
+
+
+def test_staging_ring_holds_the_most_recently_quantized_rows():
+    """With staging, the ring holds the FP16 rows of [T - W - 64, T - W):
+    the same after streaming 140 -> 300 as after loading the 300 prompt, and
+    equal to the raw input rows."""
+    cfg = synth.custom(2, 8, 2, 300, 0, seed=52)
+    K, V, _ = synth.kv_full(cfg)
+    a = oracle.OracleCache(2, 8, 2, 320, 1, stage=64)
+    a.load_prompt(K, V, [140, 140])
+    for t in range(140, 300):
+        a.append(K[:, :, t], V[:, :, t])
+    b_ = oracle.OracleCache(2, 8, 2, 320, 1, stage=64)
+    b_.load_prompt(K, V, [300, 300])
+    for name in ("stage_k", "stage_v", "k_codes", "win_k"):
+        assert np.array_equal(getattr(a, name), getattr(b_, name)), name
+    for b in range(2):
+        for h in range(2):
+            for p in range(300 - 128 - 64, 300 - 128):
+                assert np.array_equal(a.stage_k[b * 2 + h, p % 64], K[b, h, p].view(np.uint16))
+                assert np.array_equal(a.stage_v[b * 2 + h, p % 64], V[b, h, p].view(np.uint16))
+                assert a.staged(b, p)
+            assert not a.staged(b, 300 - 128 - 65) and not a.staged(b, 300 - 128)
+
+
+@pytest.mark.parametrize("stage,kept,unpromoted", [
+    (64, [10, 60, 230, 250, 260], 2),   # 230, 260 lie in the staged range [208, 272)
+    (0, [10, 60, 250], 4),              # without staging only known FP16 rows stay
+])
+def test_cache_mode_reselection_promotes_staged_positions(stage, kept, unpromoted):
+    cfg = synth.custom(1, 4, 1, 400, 6, seed=62)
+    K, V, _ = synth.kv_full(cfg)
+    c = oracle.OracleCache(1, 4, 1, 400, 8, stage=stage)
+    c.load_prompt(K, V, [400])
+    c.apply_vl(np.array([[[3, 10, 50, 60, 200, 250]]]), K, V)
+    n = c.apply_vl(np.array([[[10, 11, 60, 201, 230, 250, 260]]]))
+    assert n == unpromoted
+    assert list(c.vl_pos[0, :c.vl_count[0]]) == kept
+    for i, p in enumerate(kept):
+        assert np.array_equal(c.vl_k[0, i], K[0, 0, p].view(np.uint16))
+        assert np.array_equal(c.vl_v[0, i], V[0, 0, p].view(np.uint16))
+    qv = synth.q(cfg, 7)
+    o, _ = oracle.decode(c, qv)
+    kk, vv = _materialize(c, K, V, 0, 0)
+    ro, _ = _sdpa(qv[0], kk, vv, 4)
+    assert np.allclose(o[0], ro, rtol=0, atol=1e-12)
