@@ -23,7 +23,7 @@ BLOCK_BYTES = 5136
 BLK_KCODES, BLK_KSZ, BLK_VCODES, BLK_VSZ, BLK_MASK = 0, 2048, 2560, 4608, 5120
 
 DEV_NONFINITE = 0x1
-DEV_OOB = 0x2
+DEV_OOB = 0x2  # reserved: no kernel raises it
 DEV_TIMEOUT = 0x4
 DEV_BADLEN = 0x8
 

@@ -55,7 +55,7 @@ typedef enum {
 
 /* device status word bits */
 #define HYQ_DEV_NONFINITE 0x1u /* the quantizer saw Inf/NaN (codes undefined) */
-#define HYQ_DEV_OOB 0x2u       /* a device-side index check failed           */
+#define HYQ_DEV_OOB 0x2u       /* reserved (index checks); never raised now   */
 #define HYQ_DEV_TIMEOUT 0x4u   /* a bounded wait expired; outputs undefined   */
 #define HYQ_DEV_BADLEN 0x8u    /* seq_len / vl_count out of range; skipped    */
 
