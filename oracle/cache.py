@@ -25,7 +25,10 @@ the FP16 rows of the ``stage`` most recently quantized positions, [T - W -
 stage, T - W), are also kept in a ring (slot = p % stage), filled from the
 prompt and by every append with the row leaving the window.  A cache-mode
 re-selection then promotes a newly selected position from that ring when it
-lies in the staged range; only older new positions stay unpromoted.
+lies in the staged range and is newer than every position kept from the
+previous set (promoted rows follow the kept rows, which then only move to
+lower slots); other new positions stay unpromoted.  With re-selection every
+64 tokens every staged position is newer than the whole previous set.
 """
 from __future__ import annotations
 
@@ -119,11 +122,12 @@ class OracleCache:
                     kept = new
                 else:
                     old = {int(self.vl_pos[u, i]): i for i in range(self.vl_count[u])}
+                    last_kept = max([p for p in new if p in old], default=-1)
                     kept, rows_k, rows_v = [], [], []
                     for p in new:
                         if p in old:
                             src_k, src_v = self.vl_k[u, old[p]], self.vl_v[u, old[p]]
-                        elif self.staged(b, p):
+                        elif self.staged(b, p) and p > last_kept:
                             src_k, src_v = self.stage_k[u, p % self.stage], self.stage_v[u, p % self.stage]
                         else:
                             continue

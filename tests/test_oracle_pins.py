@@ -487,7 +487,9 @@ def test_staging_ring_holds_the_most_recently_quantized_rows():
 
 
 @pytest.mark.parametrize("stage,kept,unpromoted", [
-    (64, [10, 60, 230, 250, 260], 2),   # 230, 260 lie in the staged range [208, 272)
+    # staged range [208, 272): 260 is promoted; 230 is staged but older than
+    # the kept 250, so it stays INT4 (promoted rows follow the kept rows)
+    (64, [10, 60, 250, 260], 3),
     (0, [10, 60, 250], 4),              # without staging only known FP16 rows stay
 ])
 def test_cache_mode_reselection_promotes_staged_positions(stage, kept, unpromoted):
@@ -507,3 +509,21 @@ def test_cache_mode_reselection_promotes_staged_positions(stage, kept, unpromote
     kk, vv = _materialize(c, K, V, 0, 0)
     ro, _ = _sdpa(qv[0], kk, vv, 4)
     assert np.allclose(o[0], ro, rtol=0, atol=1e-12)
+
+
+def test_staged_promotion_at_the_method_cadence_promotes_every_recent_pick():
+    """Re-selecting every 64 appends: every newly selected position that left
+    the window since the previous selection is promoted (none unpromoted)."""
+    cfg = synth.custom(1, 4, 1, 600, 0, seed=63)
+    K, V, _ = synth.kv_full(cfg)
+    c = oracle.OracleCache(1, 4, 1, 640, 16, stage=64)
+    c.load_prompt(K, V, [400])
+    c.apply_vl(np.array([[[5, 40, 90, 150, 260]]], np.int32), K, V)   # all < 400 - 128 = 272
+    for t in range(400, 464):
+        c.append(K[:, :, t], V[:, :, t])
+    # T = 464: the 64 positions [272, 336) left the window since the selection
+    new = np.array([[[5, 90, 260, 280, 300, 335]]], np.int32)
+    assert c.apply_vl(new) == 0
+    assert list(c.vl_pos[0, :c.vl_count[0]]) == [5, 90, 260, 280, 300, 335]
+    for i, p in enumerate([5, 90, 260, 280, 300, 335]):
+        assert np.array_equal(c.vl_k[0, i], K[0, 0, p].view(np.uint16))
