@@ -96,6 +96,9 @@ def lib():
         L.hyqo_decode_fp16.argtypes = [P, P, P, P, ctypes.c_int32, ctypes.c_int32,
                                        ctypes.c_int32, ctypes.c_int32, P,
                                        ctypes.c_int32, P, P]
+        L.hyqo_prefill_attention.restype = ctypes.c_int
+        L.hyqo_prefill_attention.argtypes = [P, P, P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                             ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_int32, P, P]
         L.hyqo_select_vl.restype = ctypes.c_int
         L.hyqo_select_vl.argtypes = [ctypes.POINTER(_Cache), P, ctypes.c_int32, P,
                                      ctypes.c_int32, P, ctypes.c_int32, P, P, P]
@@ -209,6 +212,33 @@ def decode_vl_only(cache, q, units=None):
     alone, the quantized majority left out.  Same arguments and results as
     decode."""
     return _decode(lib().hyqo_decode_vl_only, "decode_vl_only", cache, q, units)
+
+
+def prefill_attention(q, k, v, seq_len, vl=None, W=128):
+    """Prefill hybrid-precision attention (explainer "Two Operational Modes /
+    Prefill Stage"): causal attention in which a (query row i, key j) pair is
+    computed from FP16 q, k, v when j is a vertical line or j > i - W, and
+    from the INT4-dequantized q, k, v otherwise.  q [B][Hq][cap][128], k/v
+    [B][Hkv][cap][128] fp16, vl [B][Hkv][n] ascending positions (or None).
+    Returns (o [B][Hq][cap][128] f64, lse [B][Hq][cap] f64); rows >= T are
+    NaN."""
+    q, k, v = _c16(q), _c16(k), _c16(v)
+    B, Hq, cap, _ = q.shape
+    Hkv = k.shape[1]
+    seq_len = np.ascontiguousarray(seq_len, np.int32)
+    o = np.full((B, Hq, cap, D), np.nan)
+    lse = np.full((B, Hq, cap), np.nan)
+    pos = cnt = None
+    stride = 0
+    if vl is not None:
+        pos = np.ascontiguousarray(vl, np.int32).reshape(B * Hkv, -1)
+        stride = pos.shape[1]
+        cnt = np.full(B * Hkv, stride, np.int32)
+    rc = lib().hyqo_prefill_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(seq_len), B, Hq, Hkv, cap, W,
+                                      _ptr(pos), _ptr(cnt), stride, _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle prefill_attention: bad arguments (code {rc})")
+    return o, lse
 
 
 def decode_fp16(q, k, v, seq_len, Hq, units=None):

@@ -468,3 +468,106 @@ int hyqo_select_vl(const hyqo_cache *c, const uint16_t *q_sel, int32_t n_q,
   }
   return err;
 }
+
+/* ------------------------------------------------------------------------
+ * Prefill hybrid-precision attention (the prefill operator).  Reading of
+ * the pages (explainer "Two Operational Modes / Prefill Stage": the quantized
+ * majority is computed first and the high-precision vertical lines and
+ * local window are overlaid; wpnews: the bulk of query, key and value is
+ * quantized): causal attention in which the pair (query row i, key j <= i)
+ * is high precision when j is a vertical line or lies in the query's
+ * sliding window (j > i - W), and then uses the FP16 q_i, k_j, v_j;
+ * otherwise it uses the INT4-dequantized q_i, k_j, v_j (the cache's grid).
+ * One softmax over all keys j <= i, scale 1/sqrt(128), in fp64.
+ * ---------------------------------------------------------------------- */
+static int quant_dequant(const uint16_t *x, double out[HYQO_D]) {
+  uint8_t code[HYQO_D];
+  uint16_t s[HYQO_NG], z[HYQO_NG];
+  if (hyqo_quantize_row(x, code, s, z) != 0) return -1;
+  for (int c = 0; c < HYQO_D; ++c) {
+    int g = c / HYQO_GROUP;
+    out[c] = hyqo_half_to_double(z[g]) + (double)code[c] * hyqo_half_to_double(s[g]);
+  }
+  return 0;
+}
+
+int hyqo_prefill_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           const int32_t *seq_len, int32_t B, int32_t Hq, int32_t Hkv,
+                           int32_t cap, int32_t W, const int32_t *vl_pos,
+                           const int32_t *vl_count, int32_t vl_stride, double *o,
+                           double *lse) {
+  if (Hkv <= 0 || Hq % Hkv != 0 || W < 0) return -1;
+  int G = Hq / Hkv;
+  double scale = 1.0 / sqrt((double)HYQO_D);
+  int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t uh = 0; uh < (int64_t)B * Hq; ++uh) {
+    int b = (int)(uh / Hq), h = (int)(uh % Hq), kvh = h / G;
+    int64_t unit = (int64_t)b * Hkv + kvh;
+    int32_t T = seq_len[b];
+    if (T < 0 || T > cap) {
+#pragma omp atomic write
+      err = -2;
+      continue;
+    }
+    int32_t n = T > 0 ? T : 1;
+    char *is_vl = (char *)calloc((size_t)n, 1);
+    double *kq = (double *)malloc(sizeof(double) * (size_t)n * HYQO_D);
+    double *vq = (double *)malloc(sizeof(double) * (size_t)n * HYQO_D);
+    double *w = (double *)malloc(sizeof(double) * (size_t)n);
+    int bad = 0;
+    if (vl_pos && vl_count) {
+      int32_t cnt = vl_count[unit];
+      for (int32_t i = 0; i < cnt; ++i) {
+        int32_t p = vl_pos[unit * vl_stride + i];
+        if (p < 0 || p >= T) bad = 1;
+        else is_vl[p] = 1;
+      }
+    }
+    const uint16_t *ku = k + unit * (int64_t)cap * HYQO_D, *vu = v + unit * (int64_t)cap * HYQO_D;
+    for (int32_t j = 0; j < T && !bad; ++j)
+      if (quant_dequant(ku + (int64_t)j * HYQO_D, kq + (int64_t)j * HYQO_D) ||
+          quant_dequant(vu + (int64_t)j * HYQO_D, vq + (int64_t)j * HYQO_D))
+        bad = 1;
+    const uint16_t *qh = q + ((int64_t)b * Hq + h) * (int64_t)cap * HYQO_D;
+    for (int32_t i = 0; i < T && !bad; ++i) {
+      double qf[HYQO_D], qq[HYQO_D];
+      for (int d = 0; d < HYQO_D; ++d) qf[d] = hyqo_half_to_double(qh[(int64_t)i * HYQO_D + d]);
+      if (quant_dequant(qh + (int64_t)i * HYQO_D, qq)) {
+        bad = 1;
+        break;
+      }
+      double m = -INFINITY;
+      for (int32_t j = 0; j <= i; ++j) {
+        int high = is_vl[j] || j > i - W;
+        double sdot = 0.0;
+        for (int d = 0; d < HYQO_D; ++d)
+          sdot += high ? qf[d] * hyqo_half_to_double(ku[(int64_t)j * HYQO_D + d])
+                       : qq[d] * kq[(int64_t)j * HYQO_D + d];
+        w[j] = sdot * scale;
+        if (w[j] > m) m = w[j];
+      }
+      double l = 0.0, acc[HYQO_D];
+      for (int d = 0; d < HYQO_D; ++d) acc[d] = 0.0;
+      for (int32_t j = 0; j <= i; ++j) {
+        int high = is_vl[j] || j > i - W;
+        double e = exp(w[j] - m);
+        l += e;
+        for (int d = 0; d < HYQO_D; ++d)
+          acc[d] += e * (high ? hyqo_half_to_double(vu[(int64_t)j * HYQO_D + d]) : vq[(int64_t)j * HYQO_D + d]);
+      }
+      double *orow = o + (((int64_t)b * Hq + h) * cap + i) * HYQO_D;
+      for (int d = 0; d < HYQO_D; ++d) orow[d] = acc[d] / l;
+      if (lse) lse[((int64_t)b * Hq + h) * cap + i] = m + log(l);
+    }
+    if (bad) {
+#pragma omp atomic write
+      err = -3;
+    }
+    free(is_vl);
+    free(kq);
+    free(vq);
+    free(w);
+  }
+  return err;
+}

@@ -96,6 +96,21 @@ int hyqo_decode(const hyqo_cache *c, const uint16_t *q, const int32_t *units,
 int hyqo_decode_vl_only(const hyqo_cache *c, const uint16_t *q, const int32_t *units,
                         int32_t n_units, double *o, double *lse);
 
+/* Prefill hybrid-precision attention (explainer "Two Operational Modes /
+ * Prefill Stage"; wpnews: the bulk of query, key and value is quantized).
+ * Causal attention; the pair (query row i, key j <= i) uses FP16 q, k, v
+ * when j is a vertical line (vl_pos[unit][0..vl_count[unit]), NULL = none)
+ * or j > i - W, and the INT4-dequantized q, k, v (the cache's quantizer)
+ * otherwise.  q [B][Hq][cap][128], k/v [B][Hkv][cap][128] fp16, rows [0, T)
+ * used; o [B][Hq][cap][128] fp64 and lse [B][Hq][cap] (nullable) written for
+ * rows [0, T).  Returns 0, -1 (shapes), -2 (a length) or -3 (a vertical
+ * line outside [0, T) or a non-finite row). */
+int hyqo_prefill_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                           const int32_t *seq_len, int32_t B, int32_t Hq, int32_t Hkv,
+                           int32_t cap, int32_t W, const int32_t *vl_pos,
+                           const int32_t *vl_count, int32_t vl_stride, double *o,
+                           double *lse);
+
 /* Attention over an all-FP16 cache k, v: [B][Hkv][cap][128], T = seq_len[b]. */
 int hyqo_decode_fp16(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                      const int32_t *seq_len, int32_t B, int32_t Hq, int32_t Hkv,

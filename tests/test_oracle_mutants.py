@@ -42,6 +42,11 @@ MUTANTS = [
      "ties_go_to_the_lower"),
     ("vertical-only variant keeps the quantized positions",
      "return p >= u->T - u->c->window || u->slot_of[p] >= 0;", "return 1;", "vl_only"),
+    ("prefill sliding window one key too wide",
+     "int high = is_vl[j] || j > i - W;", "int high = is_vl[j] || j >= i - W;", "prefill_row_with_grid"),
+    ("prefill high-precision pairs use the quantized query",
+     "sdot += high ? qf[d] * hyqo_half_to_double(", "sdot += high ? qq[d] * hyqo_half_to_double(",
+     "prefill_rows_inside_the_window"),
 ]
 
 

@@ -358,6 +358,81 @@ def test_ablation_keeping_the_quantized_tail_cuts_the_error():
         assert 5 * err["hybrid"] < err["vl_only"], err
 
 
+# ------------------------------------------------------- prefill operator
+def _causal_sdpa(Q, K, V, T, G):
+    """torch fp64 causal attention for one unit: Q [G][T][128], K/V [T][128]."""
+    qt = torch.from_numpy(Q[:, :T].astype(np.float64))[None]
+    kt = torch.from_numpy(K[:T].astype(np.float64))[None, None].expand(1, G, -1, -1)
+    vt = torch.from_numpy(V[:T].astype(np.float64))[None, None].expand(1, G, -1, -1)
+    o = F.scaled_dot_product_attention(qt, kt, vt, is_causal=True)[0]
+    s_ = (qt[0] @ kt[0, 0].T) / math.sqrt(D)
+    s_ = s_.masked_fill(torch.triu(torch.ones(T, T, dtype=torch.bool), 1), -math.inf)
+    return o.numpy(), torch.logsumexp(s_, dim=-1).numpy()
+
+
+def _prefill_inputs(T, k, seed, grid_q=False):
+    cfg = synth.custom(1, 4, 1, T, k, seed=seed)
+    K, V, vl = synth.kv_full(cfg)
+    rng = np.random.default_rng(seed)
+    if grid_q:   # every group holds 0 and 15 * 0.25: quantizing q is lossless
+        c = rng.integers(0, 16, (1, 4, K.shape[2], D))
+        c[..., 0::32], c[..., 1::32] = 0, 15
+        Q = (c * 0.25).astype(np.float16)
+    else:
+        Q = rng.standard_normal((1, 4, K.shape[2], D)).astype(np.float16)
+    return cfg, Q, K, V, vl
+
+
+def test_prefill_rows_inside_the_window_are_exact_causal_attention():
+    T = 300
+    cfg, Q, K, V, vl = _prefill_inputs(T, 8, seed=71)
+    o, lse = oracle.prefill_attention(Q, K, V, [T], vl)
+    ro, rl = _causal_sdpa(Q[0], K[0, 0], V[0, 0], T, 4)
+    assert np.allclose(o[0, :, :128], ro[:, :128], rtol=0, atol=1e-12)
+    assert np.allclose(lse[0, :, :128], rl[:, :128], rtol=0, atol=1e-11)
+    assert np.abs(o[0, :, 200:T] - ro[:, 200:]).max() > 1e-6   # the quantized majority is in effect
+
+
+def test_prefill_with_every_old_position_selected_is_exact_causal_attention():
+    T = 260
+    cfg, Q, K, V, _ = _prefill_inputs(T, 0, seed=72)
+    allpos = np.arange(T - 128, dtype=np.int32)[None, None]
+    o, lse = oracle.prefill_attention(Q, K, V, [T], allpos)
+    ro, rl = _causal_sdpa(Q[0], K[0, 0], V[0, 0], T, 4)
+    assert np.allclose(o[0, :, :T], ro, rtol=0, atol=1e-12)
+    assert np.allclose(lse[0, :, :T], rl, rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("i", [130, 260, 371, 499])
+def test_prefill_row_with_grid_queries_equals_decode_of_the_prefix(i):
+    """With q on the INT4 grid, row i is the decode of the cache holding the
+    first i + 1 positions (same vertical lines, window = the last W of them)."""
+    T = 500
+    cfg, Q, K, V, vl = _prefill_inputs(T, 16, seed=73, grid_q=True)
+    o, lse = oracle.prefill_attention(Q, K, V, [T], vl)
+    Ti = i + 1
+    c = oracle.OracleCache(1, 4, 1, cfg.capacity, 16)
+    c.load_prompt(K, V, [Ti])
+    pre = vl[0, 0][vl[0, 0] < Ti - 128]
+    if len(pre):
+        c.apply_vl(pre[None, None].astype(np.int32), K, V)
+    od, ld = oracle.decode(c, Q[:, :, i])
+    assert np.allclose(o[0, :, i], od[0], rtol=0, atol=1e-12)
+    assert np.allclose(lse[0, :, i], ld[0], rtol=0, atol=1e-11)
+
+
+def test_prefill_is_causal():
+    T = 400
+    cfg, Q, K, V, vl = _prefill_inputs(T, 8, seed=74)
+    o1, _ = oracle.prefill_attention(Q, K, V, [T], vl)
+    K2, V2 = K.copy(), V.copy()
+    K2[:, :, 301:T] = -K2[:, :, 301:T]
+    V2[:, :, 301:T] = V2[:, :, 301:T] * np.float16(2)
+    o2, _ = oracle.prefill_attention(Q, K2, V2, [T], vl)
+    assert np.array_equal(o1[:, :, :301], o2[:, :, :301])
+    assert not np.allclose(o1[:, :, 301:T], o2[:, :, 301:T])
+
+
 # --------------------------------------------------------------- selection
 def _select_by_torch(q_rows, kk, T, n_cand, k, n_q, G):
     """Brute force: full fp64 causal softmax, column sums, stable sort."""
