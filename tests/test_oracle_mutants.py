@@ -42,6 +42,15 @@ MUTANTS = [
      "ties_go_to_the_lower"),
     ("vertical-only variant keeps the quantized positions",
      "return p >= u->T - u->c->window || u->slot_of[p] >= 0;", "return 1;", "vl_only"),
+    ("a -0 minimum stored as -0",
+     "if (zh == 0x8000u) zh = 0;", "/* no canonical zero */", "quantizer"),
+    ("codes clamped at 16",
+     "if (ri > 15.0f) ri = 15.0f;", "if (ri > 16.0f) ri = 16.0f;", "quantizer"),
+    ("scale and zero swapped in the dequantization",
+     "double s = hyqo_half_to_double(sz[2 * g]);", "double s = hyqo_half_to_double(sz[2 * g + 1]);",
+     "dequant_error"),
+    ("selection candidates include the window",
+     "int32_t n_cand = T - c->window;", "int32_t n_cand = T;", "select_matches_bruteforce"),
     ("prefill sliding window one key too wide",
      "int high = is_vl[j] || j > i - W;", "int high = is_vl[j] || j >= i - W;", "prefill_row_with_grid"),
     ("prefill high-precision pairs use the quantized query",

@@ -78,6 +78,21 @@ def test_quantizer_constant_negative_group_and_extremes():
     assert code[32] == 0 and code[63] == 15
 
 
+def test_quantizer_stores_a_negative_zero_minimum_as_plus_zero():
+    """Reading of the grid: a -0 minimum is stored as +0, so the bytes do not
+    depend on the sign of a zero (group 0 here: -0 then values up to 1.5;
+    group 1: all -0, a constant group)."""
+    x = np.zeros(D, np.float16)
+    x[0] = np.float16(-0.0)
+    x[1:32] = np.linspace(0.0, 1.5, 31).astype(np.float16)
+    x[32:64] = np.float16(-0.0)
+    code, s, z, rc = oracle.quantize_row(x)
+    assert rc == 0
+    assert z[0] == 0x0000 and z[1] == 0x0000
+    assert s[0] == np.float16(np.float32(1.5) / np.float32(15)).view(np.uint16) and s[1] == 0
+    assert code[0] == 0 and code[31] == 15
+
+
 def test_quantizer_subnormal_scale_clamps_to_15():
     x = np.zeros(D, np.float16)
     x[1] = np.float16(2.0 ** -20)            # max; (2^-20)/15 -> one fp16 ulp 2^-24
