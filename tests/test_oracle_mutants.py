@@ -51,6 +51,19 @@ MUTANTS = [
      "dequant_error"),
     ("selection candidates include the window",
      "int32_t n_cand = T - c->window;", "int32_t n_cand = T;", "select_matches_bruteforce"),
+    ("low and high nibbles swapped in the packed layout",
+     "*high_nibble = w % 2;", "*high_nibble = 1 - w % 2;", "packed_layout"),
+    ("decode log-sum-exp in base 2",
+     "*lse = (n > 0) ? m + log(l) : -INFINITY;", "*lse = (n > 0) ? m + log2(l) : -INFINITY;",
+     "decode_matches_torch"),
+    ("selection sums logits instead of probabilities",
+     "cs[p] += exp(s[p] - m) / l;", "cs[p] += s[p];", "select_matches_bruteforce"),
+    ("codes decided with the unrounded fp32 scale",
+     "float sf = half_to_float(sh);", "float sf = s32;", "quantizer"),
+    ("codes by reciprocal multiply instead of division",
+     "float r = num / sf;", "float r = num * (1.0f / sf);", "quantizer"),
+    ("vertical-line rows read from the next slot",
+     "u->slot_of[pos[i]] = i;", "u->slot_of[pos[i]] = (i + 1) % cnt;", "select_cache_mode"),
     ("prefill sliding window one key too wide",
      "int high = is_vl[j] || j > i - W;", "int high = is_vl[j] || j >= i - W;", "prefill_row_with_grid"),
     ("prefill high-precision pairs use the quantized query",

@@ -93,6 +93,20 @@ def test_quantizer_stores_a_negative_zero_minimum_as_plus_zero():
     assert code[0] == 0 and code[31] == 15
 
 
+def test_quantizer_divides_instead_of_multiplying_by_the_reciprocal():
+    """Codes use an IEEE fp32 division.  Group 0 spans [0, 1.640625], so the
+    scale is 1.640625 / 15 = 0.109375 exactly, and 0.7109375, 1.3671875,
+    1.5859375 divide to exactly 6.5, 12.5, 14.5: ties to even give 6, 12, 14
+    (multiplying by the fp32 reciprocal of the scale lands just above the
+    ties and would give 7, 13, 15)."""
+    x = np.zeros(D, np.float16)
+    x[:5] = [0.0, 1.640625, 0.7109375, 1.3671875, 1.5859375]
+    code, s, z, rc = oracle.quantize_row(x)
+    assert rc == 0
+    assert s[0] == np.float16(0.109375).view(np.uint16) and z[0] == 0
+    assert list(code[:5]) == [0, 15, 6, 12, 14]
+
+
 def test_quantizer_subnormal_scale_clamps_to_15():
     x = np.zeros(D, np.float16)
     x[1] = np.float16(2.0 ** -20)            # max; (2^-20)/15 -> one fp16 ulp 2^-24
