@@ -10,8 +10,8 @@ import os
 import shutil
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
-import pytest
 
 import oracle
 
@@ -72,28 +72,34 @@ MUTANTS = [
 ]
 
 
-def _run_pins(tmp_path, source, pins):
-    d = tmp_path / "src"
-    d.mkdir()
+def _run_pins(workdir, source, pins):
+    d = workdir / "src"
+    d.mkdir(parents=True)
     (d / "hyq_oracle.c").write_text(source)
     shutil.copy(HDR, d / "hyq_oracle.h")
-    lib = oracle.compile_to(str(d / "hyq_oracle.c"), str(tmp_path / "liboracle_variant.so"))
-    env = dict(os.environ, HYQ_ORACLE_LIB=lib, OMP_NUM_THREADS="4")
+    lib = oracle.compile_to(str(d / "hyq_oracle.c"), str(workdir / "liboracle_variant.so"))
+    env = dict(os.environ, HYQ_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py"), "-k", pins],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    return r.returncode, r.stdout[-2000:]
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    return r.returncode, r.stdout[-1500:]
 
 
-def test_unmodified_oracle_passes_the_selected_pins(tmp_path):
-    pins = " or ".join(sorted({m[3] for m in MUTANTS}))
-    rc, out = _run_pins(tmp_path, open(SRC).read(), pins)
-    assert rc == 0, out
-
-
-@pytest.mark.parametrize("what,old,new,pins", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_a_planted_mistake_fails_a_pin(tmp_path, what, old, new, pins):
+def test_every_planted_mistake_fails_a_pin(tmp_path):
+    """The unmodified source passes the union of the pins; every mutant makes
+    its pins fail.  The cases run in parallel child processes."""
     src = open(SRC).read()
-    assert old in src, f"mutation site not found: {old}"
-    rc, out = _run_pins(tmp_path, src.replace(old, new), pins)
-    assert rc == 1, f"{what}: no pin failed (pytest exit {rc})\n{out}"
+    jobs = [("unmodified source", src, " or ".join(sorted({m[3] for m in MUTANTS})), 0)]
+    for what, old, new, pins in MUTANTS:
+        assert old in src, f"mutation site not found: {old}"
+        jobs.append((what, src.replace(old, new), pins, 1))
+
+    def run(job):
+        n, (what, source, pins, want) = job
+        rc, out = _run_pins(tmp_path / f"case{n}", source, pins)
+        return what, want, rc, out
+
+    with ThreadPoolExecutor(max_workers=max(2, min(8, os.cpu_count() or 2))) as ex:
+        results = list(ex.map(run, enumerate(jobs)))
+    bad = [f"{what}: pytest exit {rc}, expected {want}\n{out}" for what, want, rc, out in results if rc != want]
+    assert not bad, "\n\n".join(bad)
