@@ -103,3 +103,61 @@ def test_every_planted_mistake_fails_a_pin(tmp_path):
         results = list(ex.map(run, enumerate(jobs)))
     bad = [f"{what}: pytest exit {rc}, expected {want}\n{out}" for what, want, rc, out in results if rc != want]
     assert not bad, "\n\n".join(bad)
+
+
+# (mistake, text in oracle/cache.py, replacement, pins that must fail)
+BOOKKEEPING_MUTANTS = [
+    ("the new row packed instead of the row leaving the window",
+     "c, s, bad = pack(self.win_k[u, slot])", "c, s, bad = pack(k_new[b, h][None])", "append_equals"),
+    ("the leaving position off by one",
+     "p_out = T - self.W\n", "p_out = T - self.W + 1\n", "append_equals"),
+    ("K and V swapped when vertical lines are gathered",
+     "rows_k = [K_full[b, h, p] for p in new]", "rows_k = [V_full[b, h, p] for p in new]",
+     "decode_matches_torch"),
+    ("the window filled from one row late",
+     "for p in range(n_old, T):", "for p in range(n_old + 1, T):", "decode_matches_torch"),
+    ("staged positions promoted without the order rule",
+     "elif self.staged(b, p) and p > last_kept:", "elif self.staged(b, p):", "promotes_staged"),
+    ("the staging ring filled one row short",
+     "for p in range(max(0, n_old - self.stage), n_old):", "for p in range(max(0, n_old - self.stage + 1), n_old):",
+     "staging_ring"),
+    ("re-selection keeps no earlier rows",
+     "                        if p in old:\n", "                        if False:\n", "reselection"),
+]
+
+
+def _run_pins_with_package(workdir, cache_source, pins):
+    """Copies of tests/, synth/ and oracle/ (cache.py replaced) under a
+    scratch root; the copied conftest puts that root first on sys.path."""
+    for name in ("tests", "synth", "oracle"):
+        shutil.copytree(os.path.join(ROOT, name), workdir / name,
+                        ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    (workdir / "oracle" / "cache.py").write_text(cache_source)
+    shutil.copy(os.path.join(ROOT, "pytest.ini"), workdir / "pytest.ini")
+    env = dict(os.environ, OMP_NUM_THREADS="2")
+    env.pop("HYQ_ORACLE_LIB", None)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider",
+                        str(workdir / "tests" / "test_oracle_pins.py"), "-k", pins],
+                       cwd=str(workdir), env=env, capture_output=True, text=True, timeout=900)
+    return r.returncode, r.stdout[-1500:]
+
+
+def test_every_planted_bookkeeping_mistake_fails_a_pin(tmp_path):
+    """The same check for the host-side bookkeeping of the oracle cache."""
+    src = open(os.path.join(ROOT, "oracle", "cache.py")).read()
+    jobs = [("unmodified cache.py", src, " or ".join(sorted({m[3] for m in BOOKKEEPING_MUTANTS})), 0)]
+    for what, old, new, pins in BOOKKEEPING_MUTANTS:
+        assert src.count(old) == 1, f"mutation site not found once: {old!r}"
+        jobs.append((what, src.replace(old, new), pins, 1))
+
+    def run(job):
+        n, (what, source, pins, want) = job
+        d = tmp_path / f"pkg{n}"
+        d.mkdir()
+        rc, out = _run_pins_with_package(d, source, pins)
+        return what, want, rc, out
+
+    with ThreadPoolExecutor(max_workers=max(2, min(8, os.cpu_count() or 2))) as ex:
+        results = list(ex.map(run, enumerate(jobs)))
+    bad = [f"{what}: pytest exit {rc}, expected {want}\n{out}" for what, want, rc, out in results if rc != want]
+    assert not bad, "\n\n".join(bad)
