@@ -64,6 +64,21 @@ MUTANTS = [
      "float r = num / sf;", "float r = num * (1.0f / sf);", "quantizer"),
     ("vertical-line rows read from the next slot",
      "u->slot_of[pos[i]] = i;", "u->slot_of[pos[i]] = (i + 1) % cnt;", "select_cache_mode"),
+    ("FP16 comparator reads the wrong KV head",
+     "int64_t h = (int64_t)b * Hq + (int64_t)kvh * G + hg;", "int64_t h = (int64_t)b * Hq + (int64_t)hg * Hkv + kvh;",
+     "decode_all_fp16"),
+    ("selection query i sees one key too few",
+     "int32_t last = T - n_q + i; /* causal: keys 0..last */", "int32_t last = T - n_q + i - 1;",
+     "select_matches_bruteforce"),
+    ("selection margin relative to the k+1-th sum",
+     "margin[unit] = (cand[k - 1].cs - cand[k].cs) / cand[k - 1].cs;",
+     "margin[unit] = (cand[k - 1].cs - cand[k].cs) / cand[k].cs;", "margin"),
+    ("prefill high-precision pairs use the quantized value",
+     "acc[d] += e * (high ? hyqo_half_to_double(vu[(int64_t)j * HYQO_D + d]) : vq[(int64_t)j * HYQO_D + d]);",
+     "acc[d] += e * vq[(int64_t)j * HYQO_D + d];", "prefill_rows_inside_the_window"),
+    ("vertical-only window one position short",
+     "return p >= u->T - u->c->window || u->slot_of[p] >= 0;", "return p > u->T - u->c->window || u->slot_of[p] >= 0;",
+     "vl_only"),
     ("prefill sliding window one key too wide",
      "int high = is_vl[j] || j > i - W;", "int high = is_vl[j] || j >= i - W;", "prefill_row_with_grid"),
     ("prefill high-precision pairs use the quantized query",
