@@ -45,6 +45,7 @@ METRIC = "decode-attention effective HBM GB/s (% of B200 peak); µs/step at 32K 
 L2_DEFEAT_BYTES = 360e6  # rotate layer caches until a pass over them is ~3x the 126 MB L2
 RESELECT = 64
 N_Q = 64
+RESELECT_REPS = 4  # cache-mode re-selections timed on their own (the first untimed)
 
 
 def algorithmic_bytes(B, Hq, Hkv, T, k, W=128):
@@ -66,10 +67,11 @@ def step_bytes(B, Hq, Hkv, T, k, W=128):
     return algorithmic_bytes(B, Hq, Hkv, T, k, W) + B * Hkv * append + B * Hq * 256
 
 
-def decode_traffic():
-    """DRAM bytes per decode launch from the committed ncu capture, or None
-    once the decode kernel's sources differ from the captured ones."""
-    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+def decode_traffic(cid=2):
+    """DRAM bytes per decode launch of workload `cid` from the committed ncu
+    capture, or None once the decode kernel's sources differ from the
+    captured ones."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json" if cid == 2 else f"decode_traffic_c{cid}.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
@@ -113,6 +115,36 @@ def measured_tensor_peak():
     return 1590.0, "fallback"
 
 
+def prefill_attention_leg(torch, hyq, synth, cfg, layer, Kd, Vd):
+    """hyq_prefill_attention over the workload's prompt (the layer's cache
+    gives T and the vertical lines), timed with CUDA events after one
+    untimed call.  Algorithmic work: 4 * 128 flop per causal (query row,
+    key) pair and query head (Q K^T and P V), against the measured dense
+    fp16/bf16 tensor peak."""
+    B, Hq, T = cfg.B, cfg.Hq, cfg.T
+    cap = layer.cap
+    g = torch.Generator(device="cuda").manual_seed(cfg.seed & 0xFFFF)
+    q = torch.randn(B, Hq, cap, 128, device="cuda", generator=g, dtype=torch.float32).to(torch.float16)
+    o = torch.empty(B, Hq, cap, 128, dtype=torch.float32, device="cuda")
+    ws = hyq.workspace(hyq.hyq_prefill_attention_workspace(layer))
+    hyq.hyq_prefill_attention(layer, q, Kd, Vd, o, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    hyq.hyq_prefill_attention(layer, q, Kd, Vd, o, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    flops = 4 * 128 * B * Hq * T * (T + 1) / 2
+    tc, tc_kind = measured_tensor_peak()
+    rate = flops / (ms * 1e-3) / 1e12
+    del q, o, ws
+    torch.cuda.empty_cache()
+    return {"us": round(1000 * ms, 1), "achieved": round(rate, 2), "unit": "TFLOP/s", "per_launch": int(flops),
+            "peak": tc, "frac": round(rate / tc, 4), "peak_source": tc_kind,
+            "how": "prepass (quantize + dequantize Q/K/V, transpose V) and the tcgen05 attention kernel, one call"}
+
+
 def prefill_kernels(cfg, t_ms):
     """Rooflines of the prompt-side calls timed while the layer caches are
     built: hyq_prefill (HBM: per unit T rows of K and V in, 160 B of codes
@@ -151,6 +183,10 @@ def parse_args():
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4],
                     help="workload (2: the headline Llama-3.1-8B 32K batch-1 decode; 3 and 4 for profiling)")
+    ap.add_argument("--no-prefill-attention", action="store_true",
+                    help="skip timing hyq_prefill_attention over the prompt")
+    ap.add_argument("--no-batched", action="store_true",
+                    help="skip the batched 32K workload (batch 16) that the default run adds under 'batched'")
     return ap.parse_args()
 
 
@@ -234,38 +270,32 @@ def setup_layers(torch, hyq, synth, cfg, cap, n_layers):
     return layers, Kd, Vd, t_ms
 
 
-def run_ours(args):
-    import torch
-    import torch.distributed as dist
-
-    import synth
-    from fp16_kv_cache_b200 import build, hyq
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
-                                timeout=__import__("datetime").timedelta(seconds=120))
-    build.build()
-    cfg = synth.config(args.config)
-    K_steps, W_steps = args.steps, args.warmup
+def bench_workload(torch, hyq, synth, cfg, K_steps, W_steps, e2e_steps, world, dev, clocks_on, fp16_on,
+                   prefill_attn_on=False):
+    """Build the workload's layer caches, capture K_steps fused steps in one
+    CUDA graph and replay it (timed), time one cache-mode re-selection on
+    its own, then the FP16 comparator and the end-to-end loop.  Returns the
+    measurements; the caller composes the JSON line."""
     # enough layer caches that consecutive steps never find their data in L2
     n_layers = int(min(8, max(2, math.ceil(L2_DEFEAT_BYTES / algorithmic_bytes(cfg.B, cfg.Hq, cfg.Hkv, cfg.T, cfg.k)))))
-    per_layer_tokens = (K_steps + W_steps + args.e2e_steps) // n_layers + 2
+    per_layer_tokens = (K_steps + W_steps + e2e_steps) // n_layers + 2 + RESELECT_REPS
     cap = ((cfg.T + per_layer_tokens + 127) // 128) * 128
     layers, Kd, Vd, t_setup = setup_layers(torch, hyq, synth, cfg, cap, n_layers)
     B, Hq, Hkv = cfg.B, cfg.Hq, cfg.Hkv
-    dev = torch.device("cuda", local)
+    pa = prefill_attention_leg(torch, hyq, synth, cfg, layers[-1], Kd, Vd) if prefill_attn_on else None
 
     # per-step inputs (device) and detector rings / workspaces
-    n_total = W_steps + K_steps
     q_in = torch.from_numpy(np.stack([synth.q(cfg, 10 + s) for s in range(64)])).to(dev)
     kv = [synth.step_kv(cfg, s) for s in range(64)]
     k_in = torch.from_numpy(np.stack([a for a, _ in kv])).to(dev)
     v_in = torch.from_numpy(np.stack([b for _, b in kv])).to(dev)
-    rings = [torch.zeros(B, Hq, N_Q, 128, dtype=torch.float16, device=dev) for _ in layers]
+    # the detector's ring holds the last 64 queries of each layer: at the end
+    # of the prompt these are the prompt's own last 64 (slot = position % 64)
+    qs = np.stack([synth.qsel(cfg, b) for b in range(B)])
+    ring0 = np.zeros_like(qs)
+    for i in range(N_Q):
+        ring0[:, :, (cfg.T - N_Q + i) % N_Q] = qs[:, :, i]
+    rings = [torch.from_numpy(ring0).to(dev) for _ in layers]
     out = torch.empty(B, Hq, 128, dtype=torch.float16, device=dev)
     lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
     n_ctas = hyq.hyq_decode_default_ctas()
@@ -274,13 +304,18 @@ def run_ours(args):
     sel_pos = torch.zeros(B, Hkv, cfg.k, dtype=torch.int32, device=dev)
     nunp = torch.zeros(1, dtype=torch.int32, device=dev)
     tokens = [cfg.T] * n_layers        # host mirror of each layer's length
-    appended = [0] * n_layers
+    # Every layer re-selects after every 64 of its tokens.  The layers'
+    # phases are staggered evenly (as if each had started decoding at a
+    # different time), so that over a long run the re-selections are spread
+    # through it at the steady-state rate instead of arriving together.
+    appended = [(li * RESELECT) // n_layers for li in range(n_layers)]
 
     resel_at = {}  # layer -> step after which its first re-selection ran
 
     def step(s, before=None, after=None):
-        """Enqueue step s; returns (launches, layer, T after the step's append).
-        before() runs before the decode launch, after(reselect) after it."""
+        """Enqueue step s; returns (launches, layer, T after the step's append,
+        whether a re-selection followed).  before() runs before the decode
+        launch, after(reselect) after it."""
         li = s % n_layers
         c = layers[li]
         i = s % 64
@@ -291,16 +326,17 @@ def run_ours(args):
         tokens[li] += 1
         appended[li] += 1
         launches = 1
+        resel = appended[li] % RESELECT == 0
         if after is not None:
-            after(appended[li] % RESELECT == 0)
-        if appended[li] % RESELECT == 0:
+            after(resel)
+        if resel:
             # the 64 queries of the ring are scored; the next decode of the
             # layer sees the new vertical-line set
             hyq.hyq_select_vl(c, rings[li], cfg.k, sel_pos, sws, q_is_ring=True)
             hyq.hyq_vl_apply(c, sel_pos, n_unpromoted=nunp)
             resel_at.setdefault(li, s)
             launches += 6  # select (cache mode): 5 kernels; vl_apply (cache mode): 1
-        return launches, li, tokens[li]
+        return launches, li, tokens[li], resel
 
     # warm-up (eager, untimed) -- also sets kernel attributes before capture
     for s in range(W_steps):
@@ -325,6 +361,7 @@ def run_ours(args):
 
     g = torch.cuda.CUDAGraph()
     total_launches = 0
+    n_resel_timed = 0
     seen = []  # (step, layer, T)
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -338,13 +375,15 @@ def run_ours(args):
                     if resel or last:
                         run_close()
 
-                nl, li, T = step(W_steps + j, run_open, after)
+                nl, li, T, resel = step(W_steps + j, run_open, after)
                 total_launches += nl
+                n_resel_timed += int(resel)
                 seen.append((W_steps + j, li, T))
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(local) if not args.no_clocks else None
+    clocks = ClockSampler(dev.index or 0) if clocks_on else None
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     if clocks:
@@ -374,57 +413,133 @@ def run_ours(args):
     run_n = sum(len(r[2]) for r in runs)
     dec_avg_ms = run_ms / run_n
     ev_bytes = [nbytes[j] for r in runs for j in r[2]]
+    del g
+
+    # one cache-mode re-selection (hyq_select_vl over the cache from the ring
+    # + hyq_vl_apply), timed on its own with CUDA events, a few times
+    resel_ms = []
+    for r in range(RESELECT_REPS):
+        c = layers[r % n_layers]
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        hyq.hyq_select_vl(c, rings[r % n_layers], cfg.k, sel_pos, sws, q_is_ring=True)
+        hyq.hyq_vl_apply(c, sel_pos, n_unpromoted=nunp)
+        e1.record()
+        torch.cuda.synchronize()
+        resel_ms.append(e0.elapsed_time(e1))
+    resel_us = 1000 * float(np.median(resel_ms[1:] if len(resel_ms) > 1 else resel_ms))
     status = max(c.status() for c in layers)
 
-    # roofline of the decode kernel (the dominant launch)
-    peak, peak_kind = measured_peaks()
-    bytes_per_decode = float(np.mean(ev_bytes))
-    achieved = bytes_per_decode / (dec_avg_ms * 1e-3) / 1e9
-    value = world * total_bytes / (elapsed_ms * 1e-3) / 1e9
-
     # FP16 comparator (same kernel design over an all-FP16 cache), 3 copies > L2
-    # (the comparator needs 3 FP16 copies of the cache: headline workload only)
-    fp16 = fp16_comparator(torch, hyq, cfg, Kd, Vd, q_in, dev) if args.config == 2 else None
+    fp16 = fp16_comparator(torch, hyq, cfg, Kd, Vd, q_in, dev) if fp16_on else None
 
     # end to end through the public API with host buffers (eager loop)
     e2e = run_e2e(torch, hyq, cfg, layers, rings, dws, sws, sel_pos, nunp, n_ctas, tokens, appended,
-                  args.e2e_steps, world, dev)
+                  e2e_steps, world, dev) if e2e_steps else None
 
-    del g
+    peak, peak_kind = measured_peaks()
+    bytes_per_decode = float(np.mean(ev_bytes))
+    achieved = bytes_per_decode / (dec_avg_ms * 1e-3) / 1e9
+    us_step = 1000 * elapsed_ms / K_steps
+    return {
+        "cfg": cfg, "n_layers": n_layers, "n_ctas": n_ctas, "elapsed_ms": elapsed_ms,
+        "total_bytes": total_bytes, "value": world * total_bytes / (elapsed_ms * 1e-3) / 1e9,
+        "us_per_step": us_step, "dec_avg_ms": dec_avg_ms, "runs": len(runs), "run_n": run_n,
+        "bytes_per_decode": bytes_per_decode, "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+        "n_resel_timed": n_resel_timed, "resel_us": resel_us, "k_after": k_after, "status": status,
+        "fp16": fp16, "e2e": e2e, "clk": clk, "launches": total_launches, "t_setup": t_setup, "prefill_attn": pa,
+        # the detector at the pages' cadence: one re-selection per 64 decode
+        # steps of a layer, against 64 steps of this workload's decode
+        "detector_share": resel_us / (64 * 1000 * dec_avg_ms + resel_us),
+    }
+
+
+def workload_summary(r, world):
+    """The per-workload keys of the JSON line."""
+    cfg = r["cfg"]
+    return {
+        "workload": f"{cfg.name}: decode attention, B={cfg.B}/GPU, Hq={cfg.Hq}, Hkv={cfg.Hkv}, d=128, "
+                    f"T={cfg.T}, window 128, VL {cfg.k}, INT4 g32",
+        "step": f"hyq_decode_step (append + decode in one launch) on one of {r['n_layers']} layer caches; "
+                f"every 64 tokens of a layer hyq_select_vl(cache) + hyq_vl_apply; "
+                f"{r['n_resel_timed']} re-selections ran inside the timed region",
+        "l2": f"inputs larger than L2: {r['n_layers']} rotating layer caches "
+              f"(~{r['n_layers'] * r['bytes_per_decode'] / 1e6:.0f} MB) per GPU",
+        "us_per_step": round(r["us_per_step"], 3),
+        "decode_us_avg": round(1000 * r["dec_avg_ms"], 3),
+        "decode_timed": f"CUDA events around {r['runs']} runs of back-to-back step launches "
+                        f"({r['run_n']} launches, re-selections outside the runs)",
+        "decode_bytes_per_step": int(r["bytes_per_decode"]),
+        "pct_of_peak_step": round(100 * r["value"] / world / r["peak"], 1),
+        "reselect": {"us": round(r["resel_us"], 1),
+                     "how": "one cache-mode hyq_select_vl (from the 64-query ring) + hyq_vl_apply, CUDA events, "
+                            f"median of {RESELECT_REPS - 1} after one untimed",
+                     "share_at_64_token_cadence": round(r["detector_share"], 4)},
+        "n_ctas": r["n_ctas"],
+        "fp16_comparator": r["fp16"],
+        "dev_status": r["status"],
+        "vl_rows_after_reselect": [min(min(k) for k in r["k_after"]), max(max(k) for k in r["k_after"])],
+        "parallelism": f"replicas x{world} (independent sequences, no collective)",
+    }
+
+
+def roofline_of(r):
+    return {"bound": "hbm", "achieved": round(r["achieved"], 1), "peak": r["peak"], "unit": "GB/s",
+            "frac": round(r["achieved"] / r["peak"], 4), "traffic": decode_traffic(r["cfg"].cid),
+            "kernel": "hyq::decode_kernel<G,2> (hyq_decode_step)", "peak_source": f"{r['peak_kind']} hbm_gbs",
+            "bytes_per_launch": int(r["bytes_per_decode"])}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    from fp16_kv_cache_b200 import build, hyq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=120))
+    build.build()
+    dev = torch.device("cuda", local)
+    cfg = synth.config(args.config)
+    r = bench_workload(torch, hyq, synth, cfg, args.steps, args.warmup, args.e2e_steps, world, dev,
+                       not args.no_clocks, args.config == 2, prefill_attn_on=not args.no_prefill_attention)
+    batched = None
+    if args.config == 2 and not args.no_batched:
+        # the batched long-context workload (batch 16, 32K each): its own
+        # caches, graph and events, in the same run
+        rb = bench_workload(torch, hyq, synth, synth.config(3), max(8, min(args.steps, 48)),
+                            max(3, min(args.warmup, 8)), 0, world, dev, not args.no_clocks, False)
+        batched = workload_summary(rb, world)
+        batched.update({"value": round(rb["value"], 1), "unit": "GB/s", "steps": max(8, min(args.steps, 48)),
+                        "roofline": roofline_of(rb), "gpu_launches": rb["launches"]})
+        if rb["clk"]:
+            batched["clocks"] = rb["clk"]
+        torch.cuda.empty_cache()
+    K_steps, W_steps = args.steps, args.warmup
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
-        "steps": K_steps, "warmup": W_steps, "ms_per_step": round(elapsed_ms / K_steps, 6),
+        "metric": METRIC, "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world,
+        "steps": K_steps, "warmup": W_steps, "ms_per_step": round(r["elapsed_ms"] / K_steps, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
         "data": "synthetic (seeded N(0,1) fp16 Q/K/V, 4 K outlier channels x8, planted vertical lines)",
-        "config": {
-            "workload": f"{cfg.name}: decode attention, B={cfg.B}/GPU, Hq={cfg.Hq}, Hkv={cfg.Hkv}, d=128, "
-                        f"T={cfg.T}, window 128, VL {cfg.k}, INT4 g32",
-            "step": f"hyq_decode_step (append + decode in one launch) on one of {n_layers} layer caches; "
-                    "hyq_select_vl(cache) + hyq_vl_apply after every 64 tokens of a layer",
-            "l2": f"inputs larger than L2: {n_layers} rotating layer caches (~{n_layers * total_bytes / K_steps / 1e6:.0f} MB) "
-                  "per GPU",
-            "us_per_step": round(1000 * elapsed_ms / K_steps, 3),
-            "decode_us_avg": round(1000 * dec_avg_ms, 3),
-            "decode_timed": f"CUDA events around {len(runs)} runs of back-to-back step launches "
-                            f"({run_n} launches, re-selections outside the runs)",
-            "decode_bytes_per_step": int(bytes_per_decode),
-            "pct_of_peak_step": round(100 * value / world / peak, 1),
-            "n_ctas": n_ctas,
-            "fp16_comparator": fp16,
-            "dev_status": status,
-            "vl_rows_after_reselect": [min(min(k) for k in k_after), max(max(k) for k in k_after)],
-            "parallelism": f"replicas x{world} (independent sequences, no collective)",
-        },
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": decode_traffic(),
-                     "kernel": "hyq::decode_kernel<G,2> (hyq_decode_step)", "peak_source": f"{peak_kind} hbm_gbs",
-                     "bytes_per_launch": int(bytes_per_decode)},
-        "e2e": e2e,
-        "gpu_launches": total_launches,
-        "other_kernels": prefill_kernels(cfg, t_setup),
+        "config": workload_summary(r, world),
+        "roofline": roofline_of(r),
+        "e2e": r["e2e"],
+        "gpu_launches": r["launches"],
+        "other_kernels": prefill_kernels(cfg, r["t_setup"]),
     }
-    if clk:
-        line["clocks"] = clk
+    if r["prefill_attn"] is not None:
+        line["other_kernels"]["hyq_prefill_attention"] = r["prefill_attn"]
+    if batched is not None:
+        line["batched"] = batched
+    if r["clk"]:
+        line["clocks"] = r["clk"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0:

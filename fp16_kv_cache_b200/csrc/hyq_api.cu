@@ -24,6 +24,11 @@ extern "C" hyq_status hyq_check_cache(const hyq_cache *c) {
     if (!al16(p)) return HYQ_ERR_ALIGN;
   }
   if (c->dev_status && (reinterpret_cast<uintptr_t>(c->dev_status) & 3u)) return HYQ_ERR_ALIGN;
+  if (c->stage_rows < 0 || c->stage_rows > 1024) return HYQ_ERR_INVALID;
+  if (c->stage_rows > 0) {
+    if (!c->stage_k || !c->stage_v) return HYQ_ERR_INVALID;
+    if (!al16(c->stage_k) || !al16(c->stage_v)) return HYQ_ERR_ALIGN;
+  }
   return HYQ_OK;
 }
 

@@ -100,6 +100,12 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// Complete the current phase of a barrier armed for one arrival without
+// waiting for any bytes (a copy that is not issued).
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}" ::"r"(bar) : "memory");
+}
+
 // Bounded wait on an mbarrier phase.  Gives up after `limit_ns` of wall time
 // (or as soon as *abort is raised by another warp), raising *abort and
 // HYQ_DEV_TIMEOUT in the status word.  Returns true when the phase completed.

@@ -39,6 +39,10 @@
 //     tile counter) merges the partials by log-sum-exp.
 //   * MODE_STEP (hyq_decode_step) fuses the append of the new token into the
 //     same launch (see "fused step" below).
+#include <cuda.h>  // driver types of the context query in hyq_decode_noalloc
+
+#include <mutex>
+
 #include "hyq_common.cuh"
 #include "hyq_quant.cuh"
 
@@ -72,9 +76,12 @@ static_assert(I4_TOK == BLK_TOK, "an INT4 tile is one cache block");
 // SM holds 24 tiles in flight, about 120 KB, enough to cover the memory
 // latency at full bandwidth while leaving shared memory for the merge
 // buffers and per-unit tables of up to 4096 units.
+#ifndef HYQ_DECODE_SPW
+#define HYQ_DECODE_SPW 2
+#endif
 template <int G>
 struct Ring {
-  static constexpr int SPW = 2;
+  static constexpr int SPW = HYQ_DECODE_SPW;
 };
 
 // MODE_STEP: the hybrid decode with the token append of the same step fused
@@ -83,6 +90,31 @@ struct Ring {
 // cache with its INT4 majority left out, i.e. attention over the vertical
 // lines and the window alone.
 enum { MODE_HYBRID = 0, MODE_FP16 = 1, MODE_STEP = 2, MODE_VLONLY = 3 };
+
+// Debug builds (-DHYQ_DEBUG, built as libhyq_debug.so): the limit of the
+// tile waits is a device variable the host may set (hyq_debug_set_wait), and
+// a second one makes every warp's first tile wait a wait on a barrier that
+// nothing completes, so that a test can make the bounded waits run out and
+// check that the launch still returns, with HYQ_DEV_TIMEOUT; and the indexes
+// the kernel derives (the block's share of the split, every tile's source
+// rows, the partial records merged, the row leaving the window) are checked
+// against the arrays they address: a failed check raises HYQ_DEV_OOB and the
+// access is skipped.  Release builds compile all of it away.
+#ifdef HYQ_DEBUG
+__device__ unsigned long long g_debug_wait_ns = 2000000000ull;
+__device__ int g_debug_stall = 0;
+__device__ __forceinline__ uint64_t tile_wait_limit() {
+  return *reinterpret_cast<volatile unsigned long long *>(&g_debug_wait_ns);
+}
+__device__ __forceinline__ bool dbg_check(bool ok, uint32_t *status) {
+  if (!ok) set_status(status, HYQ_DEV_OOB);
+  return ok;
+}
+#define DBG_OK(cond, status) dbg_check((cond), (status))
+#else
+__device__ __forceinline__ uint64_t tile_wait_limit() { return 2000000000ull; }
+#define DBG_OK(cond, status) true
+#endif
 
 struct DecodeArgs {
   int B, Hq, Hkv, cap, W, vl_cap, U, n_ctas;
@@ -104,6 +136,9 @@ struct DecodeArgs {
   __half *q_ring;
   int n_q;
   int32_t *grid_counter;
+  // staging ring of the most recently quantized rows (stage_rows = 0: none)
+  __half *stage_k, *stage_v;
+  int stage_rows;
 };
 
 // Token order inside a 16-token MMA block: row r of the block holds token
@@ -489,6 +524,7 @@ struct Smem {
   uint32_t slots;     // shared address of slot 0: [NCW][SPW][SLOT_BYTES]
   uint64_t *full;     // [NCW][SPW] transaction barriers, one per slot
   int *abort_flag, *last_flag;
+  uint64_t *never;    // a barrier nothing completes (the debug build's stall test)
   float *mm, *ml, *mo;  // merge buffers: [NCW][8], [NCW][8], [NCW][G][128]
   int *cost_start;      // [U + 1]: cost of the units before u
   int *scan;            // [NTHREADS]
@@ -643,6 +679,7 @@ __device__ __forceinline__ void merge_parts(const DecodeArgs &a, const Smem &sm,
       if (cc <= c_hi) {
         const int lo = sp.lo(sm, a.U, cc), hi = sp.lo(sm, a.U, cc + 1);
         if (first_tile_from(lo, cs, n4, n16) < first_tile_from(hi, cs, n4, n16)) id = cc * 2 + ((cs <= lo) ? 0 : 1);
+        if (id >= 0 && !DBG_OK(id < 2 * a.n_ctas, lane == 0 ? a.status : nullptr)) id = -1;
       }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
@@ -725,9 +762,13 @@ __device__ __forceinline__ void step_exit_row(const DecodeArgs &a, int u, int T_
   const bool is_v = lane >= 16;
   const unsigned hmask = 0xFFFFu << (lane & 16);
   const int px = T_old - a.W;
+  if (!DBG_OK(0 <= px && px < a.cap, lane == 0 ? a.status : nullptr)) return;
   __half *wrow = (is_v ? a.win_v : a.win_k) + (static_cast<int64_t>(u) * a.W + T_old % a.W) * D;
   const uint4 old = *reinterpret_cast<const uint4 *>(wrow + 8 * t);
   const QuantShare q = quantize_share(old, t, hmask, a.status);
+  if (a.stage_rows > 0)  // the leaving row also enters the staging ring
+    *reinterpret_cast<uint4 *>((is_v ? a.stage_v : a.stage_k) +
+                               (static_cast<int64_t>(u) * a.stage_rows + px % a.stage_rows) * D + 8 * t) = old;
   const int row = px % I4_TOK;
   const uint32_t code_s = slot + (is_v ? SLOT_VC : 0) + row * ROW_BYTES;
   const uint32_t sz_s = slot + (is_v ? SLOT_VSZ : SLOT_KSZ) + row * SZ_BYTES;
@@ -822,12 +863,34 @@ __device__ __forceinline__ TileSrc tile_src(const DecodeArgs &a, const Smem &sm,
   return {sk, sv, static_cast<uint32_t>(n * F16_ROW)};
 }
 
+// Whether tile j of unit u addresses rows inside the cache's arrays: a
+// quantized block below capacity, vertical-line rows below vl_capacity,
+// window rows below the window, comparator rows below capacity.
+template <int MODE>
+__device__ __forceinline__ bool tile_in_bounds(const DecodeArgs &a, const Smem &sm, int u, int j) {
+  if (u < 0 || u >= a.U || j < 0) return false;
+  bool bad;
+  const UnitShape us = shape_of<MODE>(a, sm.unit_tv[u].x, sm.unit_tv[u].y, bad);
+  if (MODE == MODE_FP16) return j < us.nw && j * F16_ROWS < us.T && us.T <= a.cap;
+  if (j < us.n4) return (j + 1) * I4_TOK <= a.cap;
+  if (j < us.n4 + us.nv) {
+    const int r0 = (j - us.n4) * F16_ROWS;
+    return r0 < us.vlc && min(r0 + F16_ROWS, us.vlc) <= a.vl_cap;
+  }
+  const int r0 = (j - us.n4 - us.nv) * F16_ROWS;
+  return j < us.n4 + us.nv + us.nw && r0 < us.nwin && min(r0 + F16_ROWS, us.nwin) <= a.W;
+}
+
 // Issue the bulk copies of tile j of unit u into one ring slot (lane 0 arms
 // the barrier and copies; an FP16 tile is two contiguous runs of rows).
 template <int MODE>
 __device__ __forceinline__ void issue_tile(const DecodeArgs &a, const Smem &sm, int u, int j, uint32_t dst,
                                            uint32_t bar, int lane) {
   if (lane != 0) return;
+  if (!DBG_OK(tile_in_bounds<MODE>(a, sm, u, j), a.status)) {
+    mbar_arrive(bar);  // the slot's phase completes with no copy
+    return;
+  }
   const TileSrc t = tile_src<MODE>(a, sm, u, j);
   if (t.v == nullptr) {
     mbar_arrive_expect_tx(bar, t.bytes);
@@ -950,6 +1013,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
     p += NCW * SPW * 8;
     sm.abort_flag = reinterpret_cast<int *>(p);
     sm.last_flag = sm.abort_flag + 1;
+    sm.never = reinterpret_cast<uint64_t *>(sm.abort_flag + 2);  // debug builds only
     p += 16;
     sm.mm = reinterpret_cast<float *>(p);
     p += NCW * 8 * 4;
@@ -971,6 +1035,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
   if (tid == 0) {
     *sm.abort_flag = 0;
     for (int s = 0; s < NCW * SPW; ++s) mbar_init(smem_u32(&sm.full[s]), 1);
+#ifdef HYQ_DEBUG
+    mbar_init(smem_u32(sm.never), 1);
+#endif
     fence_barrier_init();
   }
   // Plan from the lengths as they stand, which the previous launch on the
@@ -982,6 +1049,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
   const int cta = blockIdx.x;
   Split sp(sm.cost_start[U], a.n_ctas, aligned);
   int lo = sp.lo(sm, U, cta), hi = sp.lo(sm, U, cta + 1);
+  if (!DBG_OK(0 <= lo && lo <= hi && hi <= sm.cost_start[U], tid == 0 ? a.status : nullptr)) lo = hi = 0;
   volatile int *abort_flag = sm.abort_flag;
   int u_first = (lo < hi) ? unit_of_cost(sm.cost_start, U, lo) : U;
 
@@ -1013,13 +1081,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
   if (plan_stale<MODE>(a, sm, tid, first)) {
     for (; k_done < k_issued; ++k_done) {
       const bool ok = first_fail < 0 &&
-                      mbar_wait_bounded(my_bars + (k_done % SPW) * 8, (k_done / SPW) & 1, abort_flag, a.status);
+                      mbar_wait_bounded(my_bars + (k_done % SPW) * 8, (k_done / SPW) & 1, abort_flag, a.status,
+                                        tile_wait_limit());
       if (!__all_sync(0xffffffffu, ok) && first_fail < 0) first_fail = k_done;
     }
     aligned = plan_units<MODE>(a, sm, tid, false);
     sp = Split(sm.cost_start[U], a.n_ctas, aligned);
     lo = sp.lo(sm, U, cta);
     hi = sp.lo(sm, U, cta + 1);
+    if (!DBG_OK(0 <= lo && lo <= hi && hi <= sm.cost_start[U], tid == 0 ? a.status : nullptr)) lo = hi = 0;
     u_first = (lo < hi) ? unit_of_cost(sm.cost_start, U, lo) : U;
     k_skip = k_issued;
     ic = seg_from<MODE>(a, sm, u_first, 0, lo, hi);
@@ -1044,7 +1114,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
       const int sl = kk % SPW;
       const uint32_t slot = my_slots + sl * SLOT_BYTES;
       ++k_done;
-      bool landed = first_fail < 0 && mbar_wait_bounded(my_bars + sl * 8, (kk / SPW) & 1, abort_flag, a.status);
+      uint32_t wait_bar = my_bars + sl * 8, wait_parity = (kk / SPW) & 1;
+#ifdef HYQ_DEBUG
+      if (kk == k_skip && *reinterpret_cast<volatile int *>(&g_debug_stall)) {
+        wait_bar = smem_u32(sm.never);  // the stall test: a phase that never completes
+        wait_parity = 0;
+      }
+#endif
+      bool landed = first_fail < 0 &&
+                    mbar_wait_bounded(wait_bar, wait_parity, abort_flag, a.status, tile_wait_limit());
       landed = __all_sync(0xffffffffu, landed);  // the warp computes together or not at all
       if (!landed) {
         if (first_fail < 0) first_fail = kk;
@@ -1325,6 +1403,8 @@ extern "C" hyq_status hyq_decode_step(const hyq_cache *c, const void *q, const v
   a.status = c->dev_status;
   a.k_new = static_cast<const __half *>(k_new); a.v_new = static_cast<const __half *>(v_new);
   a.q_ring = static_cast<__half *>(q_ring); a.n_q = n_q;
+  a.stage_k = static_cast<__half *>(c->stage_k); a.stage_v = static_cast<__half *>(c->stage_v);
+  a.stage_rows = c->stage_rows;
   a.grid_counter = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + dws);
   return dispatch_decode<MODE_STEP>(G, a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? HYQ_OK
                                                                                             : HYQ_ERR_CUDA;
@@ -1372,20 +1452,66 @@ constexpr int NOALLOC_MAX_G = 8;
 constexpr size_t NOALLOC_BYTES = static_cast<size_t>(NOALLOC_MAX_UNITS) * 4 +
                                  static_cast<size_t>(NOALLOC_MAX_CTAS) * 2 * NOALLOC_MAX_G * PART_STRIDE * 4;
 __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_BYTES];
-void *g_noalloc_addr[64] = {nullptr};  // device address of the array, per device
 
 // Host code cannot pass g_noalloc_scratch itself (that name is a host-side
-// stand-in); look its device address up once per device, with the device
-// current, and reuse it.
+// stand-in); its device address is looked up with cudaGetSymbolAddress, with
+// the device current, once per device and CUDA context, and reused.  The
+// context's unique id is part of the key: after cudaDeviceReset the runtime
+// makes a new primary context and loads the module again, which may place
+// the array elsewhere, so the next call looks it up again.  The driver calls
+// that give the id are found through the runtime's entry-point query, so the
+// library does not link the driver library itself.
+struct NoallocSlot {
+  unsigned long long ctx_id;
+  void *addr;
+};
+NoallocSlot g_noalloc_slot[64] = {};
+std::mutex g_noalloc_mu;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Unique id of the current context (false when none is current or the query
+// is unavailable).  Called with g_noalloc_mu held.
+bool current_ctx_id(unsigned long long *id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (!get_current || !get_id) {
+    void *f1 = nullptr, *f2 = nullptr;
+    cudaDriverEntryPointQueryResult r1 = cudaDriverEntryPointSymbolNotFound, r2 = r1;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f1, 12000, cudaEnableDefault, &r1) != cudaSuccess ||
+        r1 != cudaDriverEntryPointSuccess || !f1)
+      return false;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f2, 12000, cudaEnableDefault, &r2) != cudaSuccess ||
+        r2 != cudaDriverEntryPointSuccess || !f2)
+      return false;
+    get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 bool noalloc_address(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  if (!g_noalloc_addr[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return false;
-    g_noalloc_addr[dev] = p;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  unsigned long long id = 0;
+  const bool have_id = current_ctx_id(&id);
+  NoallocSlot &slot = g_noalloc_slot[dev];
+  if (have_id && slot.addr && slot.ctx_id == id) {
+    *out = slot.addr;
+    return true;
   }
-  *out = g_noalloc_addr[dev];
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return false;
+  // the lookup makes the device's primary context current if it was not
+  if (have_id || current_ctx_id(&id)) {
+    slot.ctx_id = id;
+    slot.addr = p;
+  }
+  *out = p;
   return true;
 }
 }  // namespace
@@ -1420,3 +1546,14 @@ extern "C" hyq_status hyq_decode_noalloc(const hyq_cache *c, const void *q, void
   a.status = c->dev_status;
   return dispatch_decode<MODE_HYBRID>(G, a, st) == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
 }
+
+#ifdef HYQ_DEBUG
+// Debug library only: the decode kernels' tile-wait limit and the stall
+// switch on the current device.  Synchronous.
+extern "C" hyq_status hyq_debug_set_wait(uint64_t limit_ns, int32_t stall_first_wait) {
+  if (limit_ns < 1000 || limit_ns > 10000000000ull) return HYQ_ERR_INVALID;
+  const int st = stall_first_wait ? 1 : 0;
+  if (cudaMemcpyToSymbol(g_debug_wait_ns, &limit_ns, sizeof(limit_ns)) != cudaSuccess) return HYQ_ERR_CUDA;
+  return cudaMemcpyToSymbol(g_debug_stall, &st, sizeof(st)) == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
+}
+#endif

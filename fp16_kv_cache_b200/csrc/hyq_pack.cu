@@ -66,6 +66,10 @@ __global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half 
     const int64_t co = is_v ? vcode_off(u, p, c.capacity) : kcode_off(u, p, c.capacity);
     const int64_t so = is_v ? vsz_off(u, p, c.capacity) : ksz_off(u, p, c.capacity);
     quantize_part(xv, t, hmask, c.blocks + co, reinterpret_cast<uint32_t *>(c.blocks + so), c.dev_status);
+    if (c.stage_rows > 0 && p >= T - W - c.stage_rows) {  // staging ring: the most recent quantized rows
+      __half *st = reinterpret_cast<__half *>(is_v ? c.stage_v : c.stage_k) + (u * c.stage_rows + p % c.stage_rows) * D;
+      *reinterpret_cast<uint4 *>(st + 8 * t) = xv;
+    }
   } else {
     __half *win = reinterpret_cast<__half *>(is_v ? c.win_v : c.win_k) + (u * W + p % W) * D;
     *reinterpret_cast<uint4 *>(win + 8 * t) = xv;
@@ -103,6 +107,11 @@ __global__ void append_kernel(hyq_cache c, const __half *__restrict__ k_new,
       const int64_t co = is_v ? vcode_off(u, p, c.capacity) : kcode_off(u, p, c.capacity);
       const int64_t so = is_v ? vsz_off(u, p, c.capacity) : ksz_off(u, p, c.capacity);
       quantize_part(old, t, hmask, c.blocks + co, reinterpret_cast<uint32_t *>(c.blocks + so), c.dev_status);
+      if (c.stage_rows > 0) {  // the leaving row also enters the staging ring
+        __half *st = reinterpret_cast<__half *>(is_v ? c.stage_v : c.stage_k) +
+                     (u * c.stage_rows + p % c.stage_rows) * D;
+        *reinterpret_cast<uint4 *>(st + 8 * t) = old;
+      }
     }
     const __half *src = (is_v ? v_new : k_new) + u * D;
     *reinterpret_cast<uint4 *>(win + 8 * t) = *reinterpret_cast<const uint4 *>(src + 8 * t);
@@ -191,7 +200,7 @@ __global__ void __launch_bounds__(1024) vl_recompact_kernel(hyq_cache c, const i
   pdl_wait();     // earlier work on the stream is complete and visible
   extern __shared__ int32_t vl_list[];  // [2][vl_capacity]
   __shared__ int red[32];
-  __shared__ int s_bad;
+  __shared__ int s_bad, s_prom;
   const int u = blockIdx.x;
   const int T = c.seq_len[u / c.n_kv_heads];
   const int L4 = T - c.window;
@@ -261,11 +270,46 @@ __global__ void __launch_bounds__(1024) vl_recompact_kernel(hyq_cache c, const i
     }
     __syncthreads();
   }
-  for (int r = threadIdx.x; r < old_n || r < n_kept; r += blockDim.x)
-    old[r] = (r < n_kept) ? kpos[r] : -1;
+  // Staged promotion: the new positions newer than every kept one and still
+  // in the staging ring, [T - window - stage_rows, T - window), take their
+  // rows from the ring.  They are a suffix of the ascending list and go
+  // after the kept rows (whose moves above are complete).
+  int n_prom = 0;
+  if (c.stage_rows > 0) {
+    const int last_kept = (n_kept > 0) ? kpos[n_kept - 1] : -1;
+    const int thr = max(last_kept + 1, L4 - c.stage_rows);
+    if (threadIdx.x == 0) s_prom = 0;
+    __syncthreads();
+    int cnt = 0;
+    for (int i = threadIdx.x; i < k; i += blockDim.x) cnt += (np[i] >= thr);
+    if (cnt) atomicAdd(&s_prom, cnt);
+    __syncthreads();
+    n_prom = s_prom;
+    const int first = k - n_prom;
+    const __half *sk = reinterpret_cast<const __half *>(c.stage_k);
+    const __half *sv = reinterpret_cast<const __half *>(c.stage_v);
+    for (int base = 0; base < n_prom; base += rows) {
+      const int r = base + (threadIdx.x >> 4), part = threadIdx.x & 15;
+      if (r < n_prom) {
+        const int p = np[first + r];
+        const int64_t so = (static_cast<int64_t>(u) * c.stage_rows + p % c.stage_rows) * D + 8 * part;
+        const int64_t d = (row_base + n_kept + r) * D + 8 * part;
+        *reinterpret_cast<uint4 *>(vk + d) = *reinterpret_cast<const uint4 *>(sk + so);
+        *reinterpret_cast<uint4 *>(vv + d) = *reinterpret_cast<const uint4 *>(sv + so);
+        if (part == 0) {
+          atomicOr(mask_word(c.blocks, u, p, c.capacity), 1u << (p & 31));
+          kpos[n_kept + r] = p;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const int n_new = n_kept + n_prom;
+  for (int r = threadIdx.x; r < old_n || r < n_new; r += blockDim.x)
+    old[r] = (r < n_new) ? kpos[r] : -1;
   if (threadIdx.x == 0) {
-    c.vl_count[u] = n_kept;
-    if (n_unpromoted) atomicAdd(n_unpromoted, k - n_kept);
+    c.vl_count[u] = n_new;
+    if (n_unpromoted) atomicAdd(n_unpromoted, k - n_new);
   }
 }
 

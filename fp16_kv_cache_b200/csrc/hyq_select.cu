@@ -14,18 +14,22 @@
 // ties at the k-th value go to the lower position.
 //
 // Kernels (one launch each, stream ordered):
-//   1. row_stats  grid (key chunks, units): S = Q K^T on the tensor cores
-//      (mma.sync m16n8k16, query rows on M, keys on N, fp32 accumulate);
-//      per row the running max / sum of exp over the chunk's keys.
-//   2. stats_merge grid (units): log-sum-exp merge of the chunk partials in
-//      a fixed order -> (m_r, 1 / l_r).
-//   3. colsum     grid (key chunks, units): S again for candidate keys,
-//      P = exp2(S - m_r) / l_r, column sums over the rows with a fixed
-//      reduction order (no float atomics), so equal key columns give
-//      bitwise-equal sums.
-//   4. topk       grid (units): exact radix select on the fp32 bit patterns
-//      (non-negative floats order like their bits), ties to lower positions,
-//      output compacted in ascending position order.
+//   0. rank_kernel       (cache mode only) grid (units): per bitmask word of
+//      the unit, the number of vertical-line rows before it, so the scorer
+//      finds the FP16 row of a vertical-line key without a search.
+//   1. score_kernel<.,1> persistent, one block per SM over (unit, 512-key
+//      chunk) items: S = Q K^T on the tcgen05 tensor cores (fp16 operands in
+//      shared memory, fp32 accumulators in tensor memory), query rows on M;
+//      per row the running max / sum of exp over the chunk's causal keys.
+//   2. stats_merge_kernel grid (units): log-sum-exp merge of the chunk
+//      partials in a fixed order -> (m_r, 1 / l_r).
+//   3. score_kernel<.,2> the same walk with keys on M: S again for candidate
+//      keys, P = exp2(S - m_r) / l_r, each thread sums one key column over
+//      the rows in a fixed order (no float atomics), so equal key columns
+//      give bitwise-equal sums.
+//   4. topk_kernel       grid (units): exact radix select on the fp32 bit
+//      patterns (non-negative floats order like their bits), ties to lower
+//      positions, output compacted in ascending position order.
 // Keys come from k_full (prefill) or from the cache as decode sees it: FP16
 // window and vertical-line rows, and INT4 rows dequantized as
 // zero + code * scale in fp32 and split into two fp16 terms hi + lo (both

@@ -7,6 +7,7 @@ present, the calls raise.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -23,7 +24,7 @@ BLOCK_BYTES = 5136
 BLK_KCODES, BLK_KSZ, BLK_VCODES, BLK_VSZ, BLK_MASK = 0, 2048, 2560, 4608, 5120
 
 DEV_NONFINITE = 0x1
-DEV_OOB = 0x2  # reserved: no kernel raises it
+DEV_OOB = 0x2  # raised by the index checks of the debug build only
 DEV_TIMEOUT = 0x4
 DEV_BADLEN = 0x8
 
@@ -31,6 +32,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "pointer no
           4: "workspace missing or too small", 5: "CUDA launch error"}
 
 _lib = None
+_debug_lib = None
+_active = None  # the library the wrappers below call (None: libhyq.so)
 
 
 class HyqError(RuntimeError):
@@ -50,6 +53,8 @@ class hyq_cache(ctypes.Structure):
         ("vl_pos", ctypes.c_void_p), ("vl_count", ctypes.c_void_p),
         ("seq_len", ctypes.c_void_p),
         ("dev_status", ctypes.c_void_p),
+        ("stage_k", ctypes.c_void_p), ("stage_v", ctypes.c_void_p),
+        ("stage_rows", ctypes.c_int32),
     ]
 
 
@@ -71,6 +76,8 @@ EXPORTS = [
     ("hyq_decode_noalloc", ctypes.c_int, [_CP, _P, _P, _P, _P]),
     ("hyq_decode_fp16_workspace", _SZ, [_I32, _I32, _I32, _I32]),
     ("hyq_decode_fp16", ctypes.c_int, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _I32, _P, _SZ, _P, _P]),
+    ("hyq_prefill_attention_workspace", _SZ, [_CP]),
+    ("hyq_prefill_attention", ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     ("hyq_status_string", ctypes.c_char_p, [ctypes.c_int]),
     ("hyq_decode_default_ctas", _I32, []),
     ("hyq_version", _I32, []),
@@ -95,6 +102,42 @@ def lib():
             f.argtypes = args
         _lib = L
     return _lib
+
+
+# extra entry point of the debug build (include/hyq_debug.h)
+DEBUG_EXPORTS = [("hyq_debug_set_wait", ctypes.c_int, [ctypes.c_uint64, ctypes.c_int32])]
+
+
+def debug_lib():
+    """Load libhyq_debug.so: the same entry points built with device-side
+    index checks (HYQ_DEV_OOB) and a settable decode wait limit."""
+    global _debug_lib
+    if _debug_lib is None:
+        path = _build.DEBUG_LIB
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is not built: run `python -m fp16_kv_cache_b200.build`")
+        L = ctypes.CDLL(path)
+        for name, res, args in EXPORTS + DEBUG_EXPORTS:
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _debug_lib = L
+    return _debug_lib
+
+
+@contextlib.contextmanager
+def using_debug_library():
+    """Route the wrappers below to libhyq_debug.so inside the block."""
+    global _active
+    prev, _active = _active, debug_lib()
+    try:
+        yield _active
+    finally:
+        _active = prev
+
+
+def _L():
+    return _active if _active is not None else lib()
 
 
 def _ptr(t):
@@ -122,7 +165,7 @@ def _check(rc, what):
 class HybridCache:
     """Device buffers of one layer's hybrid cache plus its C descriptor."""
 
-    def __init__(self, batch, n_q_heads, n_kv_heads, capacity, vl_capacity, device="cuda"):
+    def __init__(self, batch, n_q_heads, n_kv_heads, capacity, vl_capacity, device="cuda", stage_rows=0):
         if capacity % 128:
             raise ValueError("capacity must be a multiple of 128")
         B, Hkv = batch, n_kv_heads
@@ -138,6 +181,9 @@ class HybridCache:
         self.vl_count = z(B, Hkv, dt=torch.int32)
         self.seq_len = z(B, dt=torch.int32)
         self.dev_status = z(4, dt=torch.int32)
+        self.stage_rows = int(stage_rows)
+        self.stage_k = z(B, Hkv, max(self.stage_rows, 1), HEAD_DIM, dt=torch.float16)
+        self.stage_v = z(B, Hkv, max(self.stage_rows, 1), HEAD_DIM, dt=torch.float16)
         c = hyq_cache()
         c.batch, c.n_q_heads, c.n_kv_heads = B, n_q_heads, Hkv
         c.head_dim, c.group, c.window = HEAD_DIM, GROUP, WINDOW
@@ -145,6 +191,8 @@ class HybridCache:
         for name in ("blocks", "win_k", "win_v", "vl_k", "vl_v", "vl_pos", "vl_count", "seq_len",
                      "dev_status"):
             setattr(c, name, getattr(self, name).data_ptr())
+        if self.stage_rows:
+            c.stage_k, c.stage_v, c.stage_rows = self.stage_k.data_ptr(), self.stage_v.data_ptr(), self.stage_rows
         self.desc = c
 
     def ref(self):
@@ -186,57 +234,57 @@ def hyq_pack(x, codes, sz, dst_rows=None, dev_status=None, stream=None):
     n, stride = x.shape[0], x.stride(0)
     if not x.is_cuda:
         raise ValueError("libhyq takes device tensors")
-    rc = lib().hyq_pack(ctypes.c_void_p(x.data_ptr()), n, stride, _ptr(dst_rows), _ptr(codes),
+    rc = _L().hyq_pack(ctypes.c_void_p(x.data_ptr()), n, stride, _ptr(dst_rows), _ptr(codes),
                         _ptr(sz), _ptr(dev_status), _stream(stream))
     _check(rc, "hyq_pack")
 
 
 def hyq_prefill(cache: HybridCache, k_full, v_full, stream=None):
-    _check(lib().hyq_prefill(cache.ref(), _ptr(k_full), _ptr(v_full), _stream(stream)), "hyq_prefill")
+    _check(_L().hyq_prefill(cache.ref(), _ptr(k_full), _ptr(v_full), _stream(stream)), "hyq_prefill")
 
 
 def hyq_append(cache: HybridCache, k_new, v_new, q_new=None, q_ring=None, stream=None):
     n_q = 0 if q_ring is None else q_ring.shape[2]
-    _check(lib().hyq_append(cache.ref(), _ptr(k_new), _ptr(v_new), _ptr(q_new), _ptr(q_ring), n_q,
+    _check(_L().hyq_append(cache.ref(), _ptr(k_new), _ptr(v_new), _ptr(q_new), _ptr(q_ring), n_q,
                             _stream(stream)), "hyq_append")
 
 
 def hyq_select_vl_workspace(cache: HybridCache, n_q: int) -> int:
-    return int(lib().hyq_select_vl_workspace(cache.ref(), n_q))
+    return int(_L().hyq_select_vl_workspace(cache.ref(), n_q))
 
 
 def hyq_select_vl(cache: HybridCache, q_sel, k, out_pos, ws, out_colsum=None, k_full=None,
                   q_is_ring=False, stream=None):
     n_q = q_sel.shape[2]
-    _check(lib().hyq_select_vl(cache.ref(), _ptr(q_sel), n_q, int(bool(q_is_ring)), _ptr(k_full), k,
+    _check(_L().hyq_select_vl(cache.ref(), _ptr(q_sel), n_q, int(bool(q_is_ring)), _ptr(k_full), k,
                                _ptr(out_pos), _ptr(out_colsum), _ptr(ws), ws.numel() * ws.element_size(),
                                _stream(stream)), "hyq_select_vl")
 
 
 def hyq_vl_apply(cache: HybridCache, pos, k_full=None, v_full=None, n_unpromoted=None, stream=None):
     k = pos.shape[-1]
-    _check(lib().hyq_vl_apply(cache.ref(), _ptr(pos), k, _ptr(k_full), _ptr(v_full),
+    _check(_L().hyq_vl_apply(cache.ref(), _ptr(pos), k, _ptr(k_full), _ptr(v_full),
                               _ptr(n_unpromoted), _stream(stream)), "hyq_vl_apply")
 
 
 def hyq_decode_workspace(cache: HybridCache, n_ctas: int = 0) -> int:
-    return int(lib().hyq_decode_workspace(cache.ref(), n_ctas))
+    return int(_L().hyq_decode_workspace(cache.ref(), n_ctas))
 
 
 def hyq_decode(cache: HybridCache, q, o, ws, lse=None, n_ctas: int = 0, stream=None):
-    _check(lib().hyq_decode(cache.ref(), _ptr(q), _ptr(o), _ptr(lse), n_ctas, _ptr(ws),
+    _check(_L().hyq_decode(cache.ref(), _ptr(q), _ptr(o), _ptr(lse), n_ctas, _ptr(ws),
                             ws.numel() * ws.element_size(), _stream(stream)), "hyq_decode")
 
 
 def hyq_decode_vl_only(cache: HybridCache, q, o, ws, lse=None, n_ctas: int = 0, stream=None):
     """The vertical-only ablation: attention over the vertical-line rows and
     the window alone (workspace of hyq_decode_workspace)."""
-    _check(lib().hyq_decode_vl_only(cache.ref(), _ptr(q), _ptr(o), _ptr(lse), n_ctas, _ptr(ws),
+    _check(_L().hyq_decode_vl_only(cache.ref(), _ptr(q), _ptr(o), _ptr(lse), n_ctas, _ptr(ws),
                                     ws.numel() * ws.element_size(), _stream(stream)), "hyq_decode_vl_only")
 
 
 def hyq_decode_step_workspace(cache: HybridCache, n_ctas: int = 0) -> int:
-    return int(lib().hyq_decode_step_workspace(cache.ref(), n_ctas))
+    return int(_L().hyq_decode_step_workspace(cache.ref(), n_ctas))
 
 
 def hyq_decode_step(cache: HybridCache, q, k_new, v_new, o, ws, q_ring=None, lse=None, n_ctas: int = 0,
@@ -244,7 +292,7 @@ def hyq_decode_step(cache: HybridCache, q, k_new, v_new, o, ws, q_ring=None, lse
     """hyq_append(cache, k_new, v_new, q, q_ring) and hyq_decode(cache, q) in
     one launch."""
     n_q = int(q_ring.shape[2]) if q_ring is not None else 0
-    _check(lib().hyq_decode_step(cache.ref(), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_ring), n_q, _ptr(o),
+    _check(_L().hyq_decode_step(cache.ref(), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_ring), n_q, _ptr(o),
                                  _ptr(lse), n_ctas, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "hyq_decode_step")
 
@@ -253,28 +301,41 @@ def hyq_decode_noalloc(cache: HybridCache, q, o, lse=None, stream=None):
     """hyq_decode with the library's built-in scratch array instead of a
     caller workspace (for callers that cannot allocate device memory).  Calls
     sharing a device must not overlap on the GPU."""
-    _check(lib().hyq_decode_noalloc(cache.ref(), _ptr(q), _ptr(o), _ptr(lse), _stream(stream)),
+    _check(_L().hyq_decode_noalloc(cache.ref(), _ptr(q), _ptr(o), _ptr(lse), _stream(stream)),
            "hyq_decode_noalloc")
 
 
 def hyq_decode_fp16_workspace(batch, n_q_heads, n_kv_heads, n_ctas: int = 0) -> int:
-    return int(lib().hyq_decode_fp16_workspace(batch, n_q_heads, n_kv_heads, n_ctas))
+    return int(_L().hyq_decode_fp16_workspace(batch, n_q_heads, n_kv_heads, n_ctas))
 
 
 def hyq_decode_fp16(q, k, v, seq_len, o, ws, lse=None, n_ctas: int = 0, dev_status=None, stream=None):
     B, Hkv, cap, _ = k.shape
     Hq = q.shape[1]
-    _check(lib().hyq_decode_fp16(_ptr(q), _ptr(k), _ptr(v), _ptr(seq_len), B, Hq, Hkv, cap, _ptr(o),
+    _check(_L().hyq_decode_fp16(_ptr(q), _ptr(k), _ptr(v), _ptr(seq_len), B, Hq, Hkv, cap, _ptr(o),
                                  _ptr(lse), n_ctas, _ptr(ws), ws.numel() * ws.element_size(),
                                  _ptr(dev_status), _stream(stream)), "hyq_decode_fp16")
 
 
+def hyq_prefill_attention_workspace(cache: HybridCache) -> int:
+    return int(_L().hyq_prefill_attention_workspace(cache.ref()))
+
+
+def hyq_prefill_attention(cache: HybridCache, q, k_full, v_full, o, ws, lse=None, stream=None):
+    """Prefill hybrid-precision attention of the prompt: q fp16 [B][Hq][cap][128],
+    k_full/v_full fp16 [B][Hkv][cap][128], o fp32 [B][Hq][cap][128] (output),
+    lse optional fp32 [B][Hq][cap]; the cache gives T and the vertical lines."""
+    _check(_L().hyq_prefill_attention(cache.ref(), _ptr(q), _ptr(k_full), _ptr(v_full), _ptr(o), _ptr(lse),
+                                      _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "hyq_prefill_attention")
+
+
 def hyq_decode_default_ctas() -> int:
-    return int(lib().hyq_decode_default_ctas())
+    return int(_L().hyq_decode_default_ctas())
 
 
 def hyq_version() -> int:
-    return int(lib().hyq_version())
+    return int(_L().hyq_version())
 
 
 def workspace(nbytes: int, device="cuda"):

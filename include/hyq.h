@@ -55,7 +55,7 @@ typedef enum {
 
 /* device status word bits */
 #define HYQ_DEV_NONFINITE 0x1u /* the quantizer saw Inf/NaN (codes undefined) */
-#define HYQ_DEV_OOB 0x2u       /* reserved (index checks); never raised now   */
+#define HYQ_DEV_OOB 0x2u       /* an index check failed (debug build only)    */
 #define HYQ_DEV_TIMEOUT 0x4u   /* a bounded wait expired; outputs undefined   */
 #define HYQ_DEV_BADLEN 0x8u    /* seq_len / vl_count out of range; skipped    */
 
@@ -132,11 +132,25 @@ typedef struct {
   int32_t *vl_count;
   int32_t *seq_len;
   uint32_t *dev_status; /* nullable */
+  /* Staged promotion (optional): the FP16 K/V rows of the stage_rows most
+   * recently quantized positions [T - window - stage_rows, T - window) of
+   * every unit, [B][Hkv][stage_rows][128] fp16, position p in slot
+   * p % stage_rows.  hyq_prefill fills it from the prompt; hyq_append and
+   * hyq_decode_step write the row leaving the window; a cache-mode
+   * hyq_vl_apply promotes newly selected positions from it.  stage_rows = 0
+   * turns it off (stage_k / stage_v may then be NULL). */
+  void *stage_k, *stage_v;
+  int32_t stage_rows; /* 0, or 1..1024 */
 } hyq_cache;
 
 /*
  * hyq_pack -- quantize FP16 rows to packed INT4 codes and fp16 scale/zero
  * (the KV-cache compression of the decode stage), into plain row arrays.
+ * Method: aifromscratch.in explainer, "How It Works" (keys and values of the
+ * long-tail tokens are kept in 4 bits) and "Two Operational Modes / Decode
+ * Stage" (the cache is compressed to 4 bits as decoding proceeds); the grid
+ * itself is the library's (quantizer above), since the pages fix only the
+ * bit width.
  *   x          fp16 rows, row i at x + i*row_stride (elements), 128 values
  *   n_rows     >= 0 (0 enqueues nothing)
  *   row_stride >= 128, multiple of 8
@@ -150,7 +164,11 @@ hyq_status hyq_pack(const void *x, int64_t n_rows, int64_t row_stride,
                     uint32_t *dev_status, void *stream);
 
 /*
- * hyq_prefill -- build the cache from a prompt (end of prefill).  For every
+ * hyq_prefill -- build the cache from a prompt (end of prefill).  Method:
+ * aifromscratch.in explainer, "How It Works" (three token classes: the
+ * quantized majority, the vertical lines and the local window of the last
+ * 128 tokens, kept in FP16) and "Two Operational Modes / Prefill Stage".
+ * For every
  * unit with T = seq_len[b] (device): rows [0, T - window) of k_full/v_full
  * are quantized into the blocks (as hyq_pack), rows [max(0, T - window), T)
  * are copied into the window ring, and the vertical-line set is emptied
@@ -164,6 +182,10 @@ hyq_status hyq_prefill(const hyq_cache *c, const void *k_full, const void *v_ful
 
 /*
  * hyq_append -- add one token per sequence to the cache (decode step).
+ * Method: aifromscratch.in explainer, "Two Operational Modes / Decode Stage"
+ * (the token that leaves the local window is compressed to 4 bits as
+ * decoding proceeds); wpnews.pro summary (the detector accumulates the
+ * recent queries it scores every 64 tokens).
  * For every batch b with T = seq_len[b]: the row leaving the window
  * (position T - window, when T >= window) is packed into the codes, the new
  * K/V row takes window slot T % window, and seq_len[b] becomes T + 1.
@@ -177,7 +199,12 @@ hyq_status hyq_append(const hyq_cache *c, const void *k_new, const void *v_new,
                       const void *q_new, void *q_ring, int32_t n_q, void *stream);
 
 /*
- * hyq_select_vl -- vertical-line detector.  For every unit, the n_q most
+ * hyq_select_vl -- vertical-line detector.  Method: wpnews.pro summary (the
+ * recent queries are kept and, every 64 tokens, multiplied against the keys,
+ * after which each key's column is totalled); hotpaper.ai summary (the
+ * vertical-line tokens, under 5% of positions, are those with the largest
+ * column totals of attention); aifromscratch.in explainer, "What to Watch
+ * For" (a top-5% cut).  For every unit, the n_q most
  * recent queries of each of its G query heads (R = n_q * G rows) are scored
  * against the keys; query i sits at position T - n_q + i and sees keys
  * p <= T - n_q + i.  Each row becomes a softmax over (q . k) / sqrt(128);
@@ -204,7 +231,9 @@ hyq_status hyq_select_vl(const hyq_cache *c, const void *q_sel, int32_t n_q,
                          size_t ws_bytes, void *stream);
 
 /*
- * hyq_vl_apply -- make `pos` the vertical-line set.
+ * hyq_vl_apply -- make `pos` the vertical-line set.  Method: aifromscratch.in
+ * explainer, "How It Works" (the vertical-line tokens keep their keys and
+ * values in FP16); wpnews.pro summary (the set is re-chosen every 64 tokens).
  *   pos        int32 [B][Hkv][k], ascending, within [0, T - window)
  *   k_full/v_full  non-NULL (prefill): the FP16 rows are gathered from
  *              these [B][Hkv][capacity][128] arrays.  NULL (cache mode):
@@ -212,7 +241,11 @@ hyq_status hyq_select_vl(const hyq_cache *c, const void *q_sel, int32_t n_q,
  *              no longer selected fall back to their INT4 codes, and newly
  *              selected positions, whose FP16 copy is gone, stay INT4 and
  *              are counted in *n_unpromoted (nullable device int32,
- *              accumulated with atomicAdd; zero it first).
+ *              accumulated with atomicAdd; zero it first).  With staging
+ *              (stage_rows > 0), a newly selected position still in the
+ *              staging ring and newer than every position kept from the
+ *              previous set is promoted with its staged FP16 rows (the
+ *              promoted rows follow the kept rows).
  * Rows move only towards lower slots, so the update is done in place.
  */
 hyq_status hyq_vl_apply(const hyq_cache *c, const int32_t *pos, int32_t k,
@@ -220,8 +253,12 @@ hyq_status hyq_vl_apply(const hyq_cache *c, const int32_t *pos, int32_t k,
                         int32_t *n_unpromoted, void *stream);
 
 /*
- * hyq_decode -- one decode step of GQA attention over the hybrid cache,
- * INT4 dequantization fused into the attention (split-KV flash decoding:
+ * hyq_decode -- one decode step of GQA attention over the hybrid cache.
+ * Method: aifromscratch.in explainer, "Two Operational Modes / Decode Stage"
+ * (the 4-bit cache is decompressed inside the attention computation, with
+ * no FP16 copy written back) and "How It Works" (attention over the
+ * quantized keys, the vertical lines and the window together).  INT4
+ * dequantization is fused into the attention (split-KV flash decoding:
  * work is spread over n_ctas thread blocks by bytes read, per-block partial
  * (max, sum, accumulator) triples are merged by log-sum-exp in the last
  * block to finish a unit).
@@ -307,7 +344,9 @@ hyq_status hyq_decode_noalloc(const hyq_cache *c, const void *q, void *o, float 
 
 /*
  * hyq_decode_fp16 -- the same decode kernel design over an all-FP16 cache
- * (the full-precision comparator).
+ * (the full-precision comparator).  Method: aifromscratch.in explainer, "Key
+ * Results & Benchmarks" (HyQuant's decode kernel is measured against a
+ * full-precision FlashAttention-2 baseline).
  *   q fp16 [B][Hq][128]; k, v fp16 [B][Hkv][capacity][128]; seq_len int32 [B]
  *   o fp16 [B][Hq][128]; lse nullable fp32 [B][Hq]
  *   ws   workspace of hyq_decode_fp16_workspace(B, Hq, Hkv, n_ctas) bytes,
@@ -323,6 +362,43 @@ hyq_status hyq_decode_fp16(const void *q, const void *k, const void *v,
                            int32_t capacity, void *o, float *lse,
                            int32_t n_ctas, void *ws, size_t ws_bytes,
                            uint32_t *dev_status, void *stream);
+
+/*
+ * hyq_prefill_attention -- the prefill-stage hybrid-precision attention
+ * operator: causal GQA attention of a prompt over itself in which most
+ * (query, key) pairs are computed from INT4-quantized queries, keys and
+ * values while the vertical-line keys and each query's local window stay in
+ * FP16, in one softmax per query row.  Method: aifromscratch.in explainer,
+ * "Two Operational Modes / Prefill Stage" (a fused operator computes the
+ * quantized majority and overlays the high-precision vertical lines and
+ * local window into the same result); wpnews.pro summary (the bulk of the
+ * query, key and value tensors is quantized, vertical-line tokens and a
+ * local sliding window stay in full precision); kipquest.com abstract (the
+ * prefill stage's hybrid-precision quantized attention operator).
+ * Definition used (the pages give no formula): for query row i and key
+ * j <= i, the pair is high precision when j is one of the unit's vertical
+ * lines or j > i - window, and then uses the FP16 q_i, k_j, v_j; otherwise
+ * it uses q_i, k_j, v_j quantized on the grid above and dequantized.  Scale
+ * 1/sqrt(128), natural-log LSE.
+ *   q       fp16 [B][Hq][capacity][128]: the prompt's queries, row p =
+ *           position p
+ *   k_full, v_full  fp16 [B][Hkv][capacity][128]: the prompt's keys, values
+ *   o       fp32 [B][Hq][capacity][128] output (rows >= T untouched)
+ *   lse     nullable fp32 [B][Hq][capacity]
+ *   ws      workspace of hyq_prefill_attention_workspace(c) bytes (the
+ *           dequantized operands: about (2 Hq + 8 Hkv) x capacity x 128
+ *           bytes per sequence; no zeroing needed)
+ * The cache supplies T = seq_len[b] and the vertical-line set (vl_pos,
+ * vl_count and the block bitmasks as hyq_prefill + hyq_vl_apply leave
+ * them); it is only read.  Device-side: HYQ_DEV_BADLEN for T outside
+ * [0, capacity] or a bad vl_count (the sequence or its set is skipped),
+ * HYQ_DEV_NONFINITE for a non-finite input row, HYQ_DEV_TIMEOUT if a wait
+ * for the tensor cores runs out (outputs undefined).
+ */
+size_t hyq_prefill_attention_workspace(const hyq_cache *c);
+hyq_status hyq_prefill_attention(const hyq_cache *c, const void *q, const void *k_full,
+                                 const void *v_full, float *o, float *lse, void *ws,
+                                 size_t ws_bytes, void *stream);
 
 /* Human-readable name of a status code (static storage). */
 const char *hyq_status_string(hyq_status s);

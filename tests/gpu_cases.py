@@ -91,3 +91,67 @@ def compare_decode(o_gpu, lse_gpu, o_ref, lse_ref, heads=None):
     assert rel <= REL_L2, f"rel L2 {rel:.3g} > {REL_L2}"
     assert lerr <= LSE_ABS, f"lse abs {lerr:.3g} > {LSE_ABS}"
     return err, rel
+
+
+def assert_cache_equal(case, units=None):
+    """Bit-exact comparison of the GPU cache with the oracle's on `units`
+    (all by default): INT4 codes, scale/zero bits, window rows, vertical-line
+    rows, positions and count, and the block bitmask."""
+    g, o, cfg = case.g, case.o, case.cfg
+    U = cfg.units
+    units = range(U) if units is None else units
+    T = cfg.T
+    n_old = max(0, T - cfg.W)
+    kc, ks, vc, vs, mask = g.unpack_blocks()
+    kc, vc = kc.reshape(U, case.cap, 64), vc.reshape(U, case.cap, 64)
+    ks, vs = ks.reshape(U, case.cap, 8), vs.reshape(U, case.cap, 8)
+    mask = mask.reshape(U, case.cap // 32)
+    wk = host(g.win_k).view(np.uint16).reshape(U, 128, 128)
+    wv = host(g.win_v).view(np.uint16).reshape(U, 128, 128)
+    vlk = host(g.vl_k).view(np.uint16).reshape(U, case.vl_cap, 128)
+    vlv = host(g.vl_v).view(np.uint16).reshape(U, case.vl_cap, 128)
+    vpos = host(g.vl_pos).reshape(U, case.vl_cap)
+    vcnt = host(g.vl_count).reshape(U)
+    nw = min(T, cfg.W)
+    for u in units:
+        assert np.array_equal(kc[u, :n_old], o.k_codes[u, :n_old])
+        assert np.array_equal(vc[u, :n_old], o.v_codes[u, :n_old])
+        assert np.array_equal(ks[u, :n_old], o.k_sz[u, :n_old])
+        assert np.array_equal(vs[u, :n_old], o.v_sz[u, :n_old])
+        slots = [p % cfg.W for p in range(T - nw, T)]
+        assert np.array_equal(wk[u, slots], o.win_k[u, slots])
+        assert np.array_equal(wv[u, slots], o.win_v[u, slots])
+        c = int(o.vl_count[u])
+        assert vcnt[u] == c
+        assert np.array_equal(vpos[u, :c], o.vl_pos[u, :c])
+        assert np.array_equal(vlk[u, :c], o.vl_k[u, :c])
+        assert np.array_equal(vlv[u, :c], o.vl_v[u, :c])
+        bits = np.unpackbits(mask[u].view(np.uint8), bitorder="little")
+        assert np.array_equal(np.flatnonzero(bits), np.sort(o.vl_pos[u, :c]))
+
+
+def select_gpu(case, q_sel, k, k_full=None, ring=False):
+    cfg = case.cfg
+    pos = torch.full((cfg.B, cfg.Hkv, max(k, 1)), -7, dtype=torch.int32, device="cuda")[..., :k].contiguous()
+    cs = torch.zeros(cfg.B, cfg.Hkv, case.cap, dtype=torch.float32, device="cuda")
+    ws = hyq.workspace(hyq.hyq_select_vl_workspace(case.g, q_sel.shape[2]))
+    hyq.hyq_select_vl(case.g, q_sel, k, pos, ws, out_colsum=cs, k_full=k_full, q_is_ring=ring)
+    torch.cuda.synchronize()
+    return host(pos), host(cs).astype(np.float64)
+
+
+def check_selection(pos_g, cs_g, pos_o, cs_o, margin, T, W, units, min_margin=1e-4):
+    """Column sums to fp32 accuracy and the selected positions bit for bit.
+    The inputs must leave the k-th column sum clear of the (k+1)-th by more
+    than `min_margin` (relative) on every checked unit, so that the fp32
+    GPU sums cannot reorder the boundary: that is asserted, not assumed."""
+    n = T - W
+    for u in units:
+        b, h = u
+        ref = cs_o[b, h, :n]
+        got = cs_g[b, h, :n]
+        assert np.allclose(got, ref, rtol=2e-4, atol=1e-6 * ref.max())
+        assert margin[b, h] > min_margin, f"unit {u}: oracle top-k margin {margin[b, h]:.3g} is a near-tie"
+        assert len(pos_g[b, h]) == len(pos_o[b, h])
+        assert np.array_equal(pos_g[b, h], pos_o[b, h]), (u, margin[b, h])
+        assert np.all(np.diff(pos_g[b, h]) > 0)

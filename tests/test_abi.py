@@ -11,6 +11,7 @@ from fp16_kv_cache_b200 import hyq
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "hyq.h")
+DEBUG_HEADER = os.path.join(ROOT, "include", "hyq_debug.h")
 
 
 @pytest.fixture(scope="module")
@@ -19,8 +20,8 @@ def L():
     return hyq.lib()
 
 
-def declared_functions():
-    text = open(HEADER).read()
+def declared_functions(header=HEADER):
+    text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(hyq_[a-z0-9_]+)\s*\(", text)))
 
@@ -36,6 +37,19 @@ def test_library_exports_every_declared_symbol(L):
     for n in declared_functions():
         assert hasattr(L, n), n
     assert {n for n, _, _ in hyq.EXPORTS} == set(declared_functions())
+
+
+def test_debug_library_exports_both_headers():
+    hbuild.build_debug()
+    D = hyq.debug_lib()
+    extra = declared_functions(DEBUG_HEADER)
+    assert extra == ["hyq_debug_set_wait"]
+    for n in declared_functions() + extra:
+        assert hasattr(D, n), n
+    assert {n for n, _, _ in hyq.DEBUG_EXPORTS} == set(extra)
+    # the release library has no debug entry point
+    assert not hasattr(hyq.lib(), "hyq_debug_set_wait")
+    assert D.hyq_debug_set_wait(10, 0) == 1  # limit below 1 us: rejected on the host
 
 
 def test_version_and_status_strings(L):
@@ -141,3 +155,13 @@ def test_decode_step_argument_checks(L):
     assert step(ctypes.byref(c), q, kn, vn, ring, 64, o, None, 8, ws, need - 1, None) == 4      # workspace
     assert step(ctypes.byref(c), q, kn, vn, None, 0, o, None, 8, ws, need - 1, None) == 4       # no ring: n_q free
     assert step(ctypes.byref(_desc(window=256)), q, kn, vn, ring, 64, o, None, 8, ws, need, None) == 2
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(stage_rows=-1), 1), (dict(stage_rows=2000), 1), (dict(stage_rows=64), 1),
+    (dict(stage_rows=64, stage_k=0x50008, stage_v=0x60000), 3),
+    (dict(stage_rows=64, stage_k=0x50000, stage_v=0x60000), 4),   # valid: stops at the workspace
+])
+def test_staging_fields_are_checked(L, over, code):
+    c = _desc(**over)
+    assert L.hyq_decode(ctypes.byref(c), 0x20000000, 0x30000000, None, 8, None, 0, None) == code

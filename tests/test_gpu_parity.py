@@ -14,6 +14,9 @@ import synth
 from fp16_kv_cache_b200 import hyq
 
 from gpu_cases import Case, compare_decode, dev, host
+from gpu_cases import assert_cache_equal as _assert_cache_equal
+from gpu_cases import check_selection as _check_selection
+from gpu_cases import select_gpu as _select_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -82,38 +85,6 @@ def test_pack_flags_non_finite_rows():
 
 
 # ------------------------------------------------------------------ cache build
-def _assert_cache_equal(case, units=None):
-    g, o, cfg = case.g, case.o, case.cfg
-    U = cfg.units
-    units = range(U) if units is None else units
-    T = cfg.T
-    n_old = max(0, T - cfg.W)
-    kc, ks, vc, vs, mask = g.unpack_blocks()
-    kc, vc = kc.reshape(U, case.cap, 64), vc.reshape(U, case.cap, 64)
-    ks, vs = ks.reshape(U, case.cap, 8), vs.reshape(U, case.cap, 8)
-    mask = mask.reshape(U, case.cap // 32)
-    wk = host(g.win_k).view(np.uint16).reshape(U, 128, 128)
-    wv = host(g.win_v).view(np.uint16).reshape(U, 128, 128)
-    vlk = host(g.vl_k).view(np.uint16).reshape(U, case.vl_cap, 128)
-    vpos = host(g.vl_pos).reshape(U, case.vl_cap)
-    vcnt = host(g.vl_count).reshape(U)
-    nw = min(T, cfg.W)
-    for u in units:
-        assert np.array_equal(kc[u, :n_old], o.k_codes[u, :n_old])
-        assert np.array_equal(vc[u, :n_old], o.v_codes[u, :n_old])
-        assert np.array_equal(ks[u, :n_old], o.k_sz[u, :n_old])
-        assert np.array_equal(vs[u, :n_old], o.v_sz[u, :n_old])
-        slots = [p % cfg.W for p in range(T - nw, T)]
-        assert np.array_equal(wk[u, slots], o.win_k[u, slots])
-        assert np.array_equal(wv[u, slots], o.win_v[u, slots])
-        c = int(o.vl_count[u])
-        assert vcnt[u] == c
-        assert np.array_equal(vpos[u, :c], o.vl_pos[u, :c])
-        assert np.array_equal(vlk[u, :c], o.vl_k[u, :c])
-        bits = np.unpackbits(mask[u].view(np.uint8), bitorder="little")
-        assert np.array_equal(np.flatnonzero(bits), np.sort(o.vl_pos[u, :c]))
-
-
 @pytest.mark.parametrize("T,k", [(1, 0), (100, 0), (128, 0), (129, 1), (700, 40), (4096, 64)])
 def test_prefill_and_vl_apply_bitexact(T, k):
     cfg = synth.custom(2, 8, 2, T, k, seed=T * 7 + k)
@@ -155,16 +126,6 @@ def test_decode_config2_full():
         og, lg = case.decode_gpu(q)
         oo, lo = oracle.decode(case.o, q)
         compare_decode(og, lg, oo, lo)
-
-
-@pytest.mark.parametrize("cid,units", [(3, [0, 17, 64, 127]), (4, [0, 13, 31])])
-def test_decode_full_size_sampled_units(cid, units):
-    cfg = synth.config(cid)
-    case = Case(cfg, oracle_units=units)
-    q = synth.q(cfg)
-    og, lg = case.decode_gpu(q)
-    oo, lo = oracle.decode(case.o, q, units=units)
-    compare_decode(og, lg, oo, lo, heads=case.heads_of(units))
 
 
 def test_decode_with_every_old_position_fp16_equals_fp16_kernel():
@@ -256,33 +217,6 @@ def test_append_past_capacity_sets_status():
 
 
 # ------------------------------------------------------------------ selection
-def _select_gpu(case, q_sel, k, k_full=None, ring=False):
-    cfg = case.cfg
-    pos = torch.full((cfg.B, cfg.Hkv, max(k, 1)), -7, dtype=torch.int32, device="cuda")[..., :k].contiguous()
-    cs = torch.zeros(cfg.B, cfg.Hkv, case.cap, dtype=torch.float32, device="cuda")
-    ws = hyq.workspace(hyq.hyq_select_vl_workspace(case.g, q_sel.shape[2]))
-    hyq.hyq_select_vl(case.g, q_sel, k, pos, ws, out_colsum=cs, k_full=k_full, q_is_ring=ring)
-    torch.cuda.synchronize()
-    return host(pos), host(cs).astype(np.float64)
-
-
-def _check_selection(pos_g, cs_g, pos_o, cs_o, margin, T, W, units, min_margin=1e-4):
-    n = T - W
-    for u in units:
-        b, h = u
-        # column sums agree to fp32 accuracy
-        ref = cs_o[b, h, :n]
-        got = cs_g[b, h, :n]
-        assert np.allclose(got, ref, rtol=2e-4, atol=1e-6 * ref.max())
-        if margin[b, h] > min_margin:
-            assert np.array_equal(pos_g[b, h], pos_o[b, h]), (u, margin[b, h])
-        else:  # near-tie at the boundary: the GPU set must still be a valid top-k
-            sel = set(pos_g[b, h].tolist())
-            thr = np.sort(ref)[::-1][len(sel) - 1]
-            assert all(ref[p] >= thr * (1 - 1e-3) for p in sel)
-        assert np.all(np.diff(pos_g[b, h]) > 0)
-
-
 @pytest.mark.parametrize("B,Hq,Hkv,T,k,n_q", [
     (1, 8, 2, 4096, 64, 64), (2, 16, 8, 700, 20, 64), (1, 8, 1, 300, 10, 64),
     (1, 64, 8, 2000, 40, 64), (1, 4, 4, 500, 16, 8), (2, 32, 8, 1200, 0, 64),
@@ -328,16 +262,14 @@ def test_select_ties_lower_position_wins():
         assert list(pos_g[0, 0]) == want
 
 
-def test_select_config1_and_config2_sampled():
-    for cid, units in ((1, None), (2, [0, 5])):
-        cfg = synth.config(cid)
-        case = Case(cfg, oracle_units=units)
-        qs = np.stack([synth.qsel(cfg, b) for b in range(cfg.B)])
-        pos_g, cs_g = _select_gpu(case, dev(qs), cfg.k, k_full=case.Kd)
-        pos_o, cs_o, margin = oracle.select_vl(case.o, qs, cfg.k, k_full=case.K, units=units)
-        us = units if units is not None else range(cfg.units)
-        _check_selection(pos_g, cs_g, pos_o, cs_o, margin, cfg.T, 128,
-                         [divmod(int(u), cfg.Hkv) for u in us])
+def test_select_config1_all_units():
+    cfg = synth.config(1)
+    case = Case(cfg)
+    qs = np.stack([synth.qsel(cfg, b) for b in range(cfg.B)])
+    pos_g, cs_g = _select_gpu(case, dev(qs), cfg.k, k_full=case.Kd)
+    pos_o, cs_o, margin = oracle.select_vl(case.o, qs, cfg.k, k_full=case.K)
+    _check_selection(pos_g, cs_g, pos_o, cs_o, margin, cfg.T, 128,
+                     [divmod(u, cfg.Hkv) for u in range(cfg.units)])
 
 
 # ------------------------------------------------------------------ VL apply, cache mode

@@ -2,8 +2,8 @@
 decode steps that append as they go (hyq_decode_step), with the detector
 re-selecting every 64 tokens in cache mode from the ring of the last 64
 decode queries.  Sampled units are checked against the oracle, which follows
-the same steps: selection indices (bit-exact where the boundary margin
-allows), the vertical-line rows after each cache-mode apply, the count of
+the same steps: selection indices (bit-exact, on units whose oracle top-k
+margin is asserted to exceed 1e-4), the vertical-line rows after each cache-mode apply, the count of
 unpromoted positions, and decode outputs along the way."""
 import numpy as np
 import pytest
@@ -21,12 +21,12 @@ STEPS = 130      # two re-selections (after steps 63 and 127)
 
 
 def _selection_ok(pos_g, pos_o, cs_o, margin, b, h, n):
-    if margin[b, h] > 1e-4:
-        assert np.array_equal(pos_g[b, h], pos_o[b, h]), (b, h, margin[b, h])
-    else:  # near-tie at the k-th value: the GPU set must still be a top-k
-        ref = cs_o[b, h, :n]
-        thr = np.sort(ref)[::-1][len(pos_g[b, h]) - 1]
-        assert all(ref[p] >= thr * (1 - 1e-3) for p in pos_g[b, h])
+    """Bit-exact selection on a unit whose oracle top-k margin exceeds 1e-4
+    (asserted: the sampled units keep margins of 5e-4 or more at both
+    re-selections)."""
+    assert margin[b, h] > 1e-4, (b, h, margin[b, h])
+    assert len(pos_g[b, h]) == len(pos_o[b, h])
+    assert np.array_equal(pos_g[b, h], pos_o[b, h]), (b, h, margin[b, h])
     assert np.all(np.diff(pos_g[b, h]) > 0)
 
 
