@@ -1217,16 +1217,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
       }
     }
     if (!complete) {
-      __threadfence();
+      // Publish the partial: after the block barrier, one acquire-release
+      // atomic by thread 0 orders the block's record writes (observed
+      // through the barrier) before the count, and, in the block that
+      // completes the unit, the other blocks' records before the merge
+      // (the barrier after it passes the acquire on to every thread).
       named_bar_sync(1, NTHREADS);
       if (tid == 0) {
         const int mine = sg.je - sg.jb;
-        const int old = atomicAdd(&a.counters[u], mine);
+        int old;
+        asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;"
+                     : "=r"(old)
+                     : "l"(a.counters + u), "r"(mine)
+                     : "memory");
         *sm.last_flag = (old + mine == n_unit);
       }
       named_bar_sync(1, NTHREADS);
       if (*sm.last_flag) {
-        __threadfence();
         merge_parts<G>(a, sm, u, us.n4, us.nv + us.nw, sp, hbase, tid);
         if (tid == 0) a.counters[u] = 0;
       }

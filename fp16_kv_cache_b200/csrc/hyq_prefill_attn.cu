@@ -154,7 +154,12 @@ __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::
 __device__ __forceinline__ void cp16(uint32_t dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void st_zero16(uint32_t dst) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(dst), "r"(0u) : "memory");
 }
@@ -305,8 +310,8 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   __shared__ uint32_t tmem_base;
   __shared__ __align__(8) uint64_t bars[2];  // [0] S MMAs, [1] P V MMAs
   __shared__ int s_abort;
-  __shared__ uint32_t s_vlmask[2];           // bitmask words of the current 64-key tile
-  __shared__ int s_vlpos[KT];                // positions of the current vertical-line tile
+  __shared__ uint32_t s_vlmask[2][2];        // bitmask words of a 64-key tile (two jobs in flight)
+  __shared__ int s_vlpos[2][KT];             // positions of a vertical-line tile
   const int tid = threadIdx.x, warp = tid >> 5;
   const int BH = a.B * a.Hq;
   const int n_qt = a.cap / QT;
@@ -381,13 +386,19 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   const __half *khb = a.kh + static_cast<int64_t>(u) * a.cap * D;
   const __half *klb = a.kl + static_cast<int64_t>(u) * a.cap * D;
 
-  for (int job = 0; job < n_jobs && !*abort; ++job) {
+  // Job j: the vertical-line tile j (j < n_vlt) or key tile j - n_vlt.
+  auto job_kind = [&](int job, int &kt) {
     const bool is_vl = job < n_vlt;
-    const int kt = is_vl ? job : job - n_vlt;
-    const int kind = is_vl ? JOB_VL : (kt >= band0 ? JOB_BAND : JOB_OFF);
-    const int j0 = kt * KT;
-    // ---- stage the tile's operands
-    for (int c = tid; c < KT * 16; c += THREADS) {  // key rows
+    kt = is_vl ? job : job - n_vlt;
+    return is_vl ? JOB_VL : (kt >= band0 ? JOB_BAND : JOB_OFF);
+  };
+  // Loads of a job's key rows (and the tile's vertical-line bitmask or
+  // positions, into mask buffer mb) as one cp.async group, and of its value
+  // tiles as another.  Rows past the end are zero-filled.
+  auto load_keys = [&](int job, int mb) {
+    int kt;
+    const int kind = job_kind(job, kt), j0 = kt * KT;
+    for (int c = tid; c < KT * 16; c += THREADS) {
       const int r = c >> 4, cc = c & 15;
       const uint32_t off = swz(KT, r, 8 * cc);
       if (kind == JOB_VL) {
@@ -406,7 +417,24 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
         }
       }
     }
-    for (int c = tid; c < D * 8; c += THREADS) {  // value tiles [128 ch][64 keys], zeros past the end
+    if (kind == JOB_VL && tid < KT) {
+      if (j0 + tid < n_vl)
+        cp4(smem_u32(&s_vlpos[mb][tid]), a.vl_pos + static_cast<int64_t>(u) * a.vl_cap + j0 + tid);
+      else
+        s_vlpos[mb][tid] = INT_MAX;
+    }
+    if (kind != JOB_VL && tid < 2) {
+      if (j0 + 32 * tid < T)
+        cp4(smem_u32(&s_vlmask[mb][tid]), a.blocks + blk_base(u, j0 + 32 * tid, a.cap) + HYQ_BLK_MASK);
+      else
+        s_vlmask[mb][tid] = 0u;
+    }
+    cp_commit();
+  };
+  auto load_values = [&](int job) {
+    int kt;
+    const int kind = job_kind(job, kt);
+    for (int c = tid; c < D * 8; c += THREADS) {  // [128 ch][64 keys], zeros past the end
       const int r = c >> 3, cc = c & 7;
       const uint32_t off = swz(D, r, 8 * cc);
       if (kind == JOB_VL) {
@@ -417,13 +445,19 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
         if (kind == JOB_BAND) cp16(s0 + OFF_VF + off, a.vft + (tb + r) * KT + 8 * cc);
       }
     }
-    if (kind == JOB_VL && tid < KT)
-      s_vlpos[tid] = (j0 + tid < n_vl) ? a.vl_pos[static_cast<int64_t>(u) * a.vl_cap + j0 + tid] : INT_MAX;
-    if (kind != JOB_VL && tid < 2)
-      s_vlmask[tid] = (j0 + 32 * tid < T)
-                          ? *reinterpret_cast<const uint32_t *>(a.blocks + blk_base(u, j0 + 32 * tid, a.cap) + HYQ_BLK_MASK)
-                          : 0u;
-    cp_wait_all();
+    cp_commit();
+  };
+  // Software pipeline over the single key and value buffers: the keys of
+  // job + 1 load while job's epilogue and P V run, its values while the
+  // next S and epilogue run.  cp.async groups complete in order.
+  if (n_jobs > 0) {
+    load_keys(0, 0);
+    load_values(0);
+  }
+  for (int job = 0; job < n_jobs && !*abort; ++job) {
+    int kt;
+    const int kind = job_kind(job, kt), j0 = kt * KT, mb = job & 1;
+    cp_wait_group<1>();  // this job's keys (its values may still be in flight)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
@@ -444,13 +478,15 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
     mma_wait(smem_u32(&bars[0]), ph_s, a, abort);
     ph_s ^= 1u;
     tc_fence_after();
+    // the key buffer is free: the next job's keys load during this epilogue
+    if (job + 1 < n_jobs) load_keys(job + 1, mb ^ 1); else cp_commit();
     // ---- epilogue: this thread's row, 64 key columns, in two passes over
     // 32-column chunks read from tensor memory (max, then exp2 and P)
     auto chunk = [&](int cb, float (&x)[32], uint32_t &hmask32) {
       float lo_v[32], hi_v[32];
       if (kind != JOB_VL) tm_ld32(tm_row + TM_SLO + 32 * cb, lo_v);
       if (kind != JOB_OFF) tm_ld32(tm_row + TM_SHI + 32 * cb, hi_v);
-      const uint32_t vlw = (kind != JOB_VL) ? s_vlmask[cb] : 0u;
+      const uint32_t vlw = (kind != JOB_VL) ? s_vlmask[mb][cb] : 0u;
       hmask32 = 0u;
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) {
@@ -459,7 +495,7 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
         if (kind == JOB_VL) {
           // vertical line j of the unit: counted here when it lies outside
           // the query's window (inside it, the band tile has it)
-          if (j < n_vl && s_vlpos[c] <= i - a.W) {
+          if (j < n_vl && s_vlpos[mb][c] <= i - a.W) {
             v = hi_v[jj];
             hmask32 |= 1u << jj;
           }
@@ -543,6 +579,7 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
       }
     }
     l_run += lsum;
+    cp_wait_group<1>();  // this job's values (the next job's keys may still be in flight)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
@@ -568,7 +605,10 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
     tc_fence_before();
     __syncthreads();  // every thread saw the MMAs complete: shared tiles and O are free
     tc_fence_after();
+    // the value buffer is free: the next job's values load during its S and epilogue
+    if (job + 1 < n_jobs) load_values(job + 1); else cp_commit();
   }
+  cp_wait_group<0>();  // nothing may land in shared memory after the block exits
 
   // ---- O / l and the log-sum-exp of row i
   if (!*abort && o_started) {  // uniform: the tensor-memory loads take the whole warp

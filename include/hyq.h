@@ -331,8 +331,9 @@ hyq_status hyq_decode_step(const hyq_cache *c, const void *q, const void *k_new,
  *   batch x n_kv_heads <= 4096, automatic block count <= 320, G <= 8;
  *   larger shapes return HYQ_ERR_UNSUPPORTED without enqueuing anything.
  *   The first call on a device looks up the array's device address (once
- *   per device, with that device current); make that first call before any
- *   stream capture.  Every call clears the array's counters
+ *   per device and CUDA context, with that device current; a
+ *   cudaDeviceReset makes the next call look it up again); make that first
+ *   call before any stream capture.  Every call clears the array's counters
  *   (cudaMemsetAsync on `stream`) and then launches the decode.
  *   All calls share the one array: two calls whose work overlaps on the GPU
  *   (different streams, or different host threads on one device) race and
@@ -386,7 +387,7 @@ hyq_status hyq_decode_fp16(const void *q, const void *k, const void *v,
  *   o       fp32 [B][Hq][capacity][128] output (rows >= T untouched)
  *   lse     nullable fp32 [B][Hq][capacity]
  *   ws      workspace of hyq_prefill_attention_workspace(c) bytes (the
- *           dequantized operands: about (2 Hq + 8 Hkv) x capacity x 128
+ *           dequantized operands: about (4 Hq + 8 Hkv) x capacity x 128
  *           bytes per sequence; no zeroing needed)
  * The cache supplies T = seq_len[b] and the vertical-line set (vl_pos,
  * vl_count and the block bitmasks as hyq_prefill + hyq_vl_apply leave
