@@ -431,6 +431,10 @@ def bench_workload(torch, hyq, synth, cfg, K_steps, W_steps, e2e_steps, world, d
     resel_us = 1000 * float(np.median(resel_ms[1:] if len(resel_ms) > 1 else resel_ms))
     status = max(c.status() for c in layers)
 
+    # hyq_decode alone (no fused append) over the same rotating caches,
+    # back-to-back launches in one CUDA graph between one pair of events
+    dec_only = decode_only_leg(torch, hyq, cfg, layers, q_in, out, lse, tokens, dev)
+
     # FP16 comparator (same kernel design over an all-FP16 cache), 3 copies > L2
     fp16 = fp16_comparator(torch, hyq, cfg, Kd, Vd, q_in, dev) if fp16_on else None
 
@@ -452,6 +456,7 @@ def bench_workload(torch, hyq, synth, cfg, K_steps, W_steps, e2e_steps, world, d
         # the detector at the pages' cadence: one re-selection per 64 decode
         # steps of a layer, against 64 steps of this workload's decode
         "detector_share": resel_us / (64 * 1000 * dec_avg_ms + resel_us),
+        "decode_only": dec_only,
     }
 
 
@@ -477,6 +482,7 @@ def workload_summary(r, world):
                             f"median of {RESELECT_REPS - 1} after one untimed",
                      "share_at_64_token_cadence": round(r["detector_share"], 4)},
         "n_ctas": r["n_ctas"],
+        "decode_only": r["decode_only"],
         "fp16_comparator": r["fp16"],
         "dev_status": r["status"],
         "vl_rows_after_reselect": [min(min(k) for k in r["k_after"]), max(max(k) for k in r["k_after"])],
@@ -547,6 +553,42 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def decode_only_leg(torch, hyq, cfg, layers, q_in, out, lse, tokens, dev, reps=None):
+    """hyq_decode (the decode without the fused append) timed like the step:
+    back-to-back launches over the rotating layer caches in one CUDA graph,
+    one pair of CUDA events around them.  The caches are only read."""
+    n = len(layers)
+    reps = reps or max(4 * n, 32 if cfg.B == 1 else 16)
+    n_ctas = hyq.hyq_decode_default_ctas()
+    ws = [hyq.workspace(hyq.hyq_decode_workspace(c, n_ctas)) for c in layers]
+    for i in range(n):
+        hyq.hyq_decode(layers[i], q_in[i % 64], out, ws[i], lse=lse, n_ctas=n_ctas)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            e0.record()
+            for i in range(reps):
+                hyq.hyq_decode(layers[i % n], q_in[i % 64], out, ws[i % n], lse=lse, n_ctas=n_ctas)
+            e1.record()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    del g
+    ks = [c.vl_count.flatten().tolist() for c in layers]
+    nbytes = float(np.mean([algorithmic_bytes(cfg.B, cfg.Hq, cfg.Hkv, tokens[i % n], ks[i % n]) for i in range(reps)]))
+    peak, kind = measured_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"us": round(1000 * ms, 3), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4), "bytes": int(nbytes),
+            "launches": reps, "peak_source": f"{kind} hbm_gbs",
+            "how": "hyq_decode alone (no fused append), back-to-back launches over the rotating caches, CUDA events"}
 
 
 def fp16_comparator(torch, hyq, cfg, Kd, Vd, q_in, dev, copies=3, reps=60):

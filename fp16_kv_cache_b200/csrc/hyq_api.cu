@@ -24,6 +24,10 @@ extern "C" hyq_status hyq_check_cache(const hyq_cache *c) {
     if (!al16(p)) return HYQ_ERR_ALIGN;
   }
   if (c->dev_status && (reinterpret_cast<uintptr_t>(c->dev_status) & 3u)) return HYQ_ERR_ALIGN;
+  if (c->block_table) {
+    if (c->n_pages < 1) return HYQ_ERR_INVALID;
+    if (reinterpret_cast<uintptr_t>(c->block_table) & 3u) return HYQ_ERR_ALIGN;
+  }
   if (c->stage_rows < 0 || c->stage_rows > 1024) return HYQ_ERR_INVALID;
   if (c->stage_rows > 0) {
     if (!c->stage_k || !c->stage_v) return HYQ_ERR_INVALID;

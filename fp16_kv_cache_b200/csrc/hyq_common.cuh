@@ -26,32 +26,49 @@ constexpr int MAX_UNITS = 4096;  // units (batch x kv heads) one launch schedule
 constexpr int BLK_TOK = HYQ_BLOCK_TOKENS;
 constexpr int BLK_BYTES = HYQ_BLOCK_BYTES;
 
-// Quantized-majority block of position p of unit u, and the byte offsets of
-// that position's K/V codes and scale/zero rows inside the cache's blocks.
-__host__ __device__ __forceinline__ int64_t blk_base(int64_t u, int64_t p, int cap) {
-  return (u * (cap / BLK_TOK) + p / BLK_TOK) * BLK_BYTES;
-}
-__host__ __device__ __forceinline__ int64_t kcode_off(int64_t u, int64_t p, int cap) {
-  return blk_base(u, p, cap) + HYQ_BLK_KCODES + (p % BLK_TOK) * ROW_BYTES;
-}
-__host__ __device__ __forceinline__ int64_t ksz_off(int64_t u, int64_t p, int cap) {
-  return blk_base(u, p, cap) + HYQ_BLK_KSZ + (p % BLK_TOK) * SZ_BYTES;
-}
-__host__ __device__ __forceinline__ int64_t vcode_off(int64_t u, int64_t p, int cap) {
-  return blk_base(u, p, cap) + HYQ_BLK_VCODES + (p % BLK_TOK) * ROW_BYTES;
-}
-__host__ __device__ __forceinline__ int64_t vsz_off(int64_t u, int64_t p, int cap) {
-  return blk_base(u, p, cap) + HYQ_BLK_VSZ + (p % BLK_TOK) * SZ_BYTES;
-}
-// the vertical-line bitmask word covering position p (bit p % 32)
-__device__ __forceinline__ uint32_t *mask_word(uint8_t *blocks, int64_t u, int64_t p, int cap) {
-  return reinterpret_cast<uint32_t *>(blocks + blk_base(u, p, cap) + HYQ_BLK_MASK);
-}
-
 // ---------------------------------------------------------------- status
 __device__ __forceinline__ void set_status(uint32_t *st, uint32_t bits) {
   if (st) atomicOr(st, bits);
 }
+
+// Quantized-majority block of position p of unit u, and the byte offsets of
+// that position's K/V codes and scale/zero rows inside the cache's blocks
+// (contiguous layout: each unit owns capacity / 32 consecutive records).
+__host__ __device__ __forceinline__ int64_t blk_base(int64_t u, int64_t p, int cap) {
+  return (u * (cap / BLK_TOK) + p / BLK_TOK) * BLK_BYTES;
+}
+
+// Where the record of (unit u, position p) lives.  Contiguous layout (no
+// block table): blk_base.  Paged layout: sequence b = u / Hkv maps its
+// logical block p / 32 to page table[b * (cap / 32) + p / 32] of a pool of
+// n_pages pages, and a page holds the records of the Hkv KV heads in order,
+// so the record is page * Hkv + u % Hkv.  A table entry outside [0,
+// n_pages) raises HYQ_DEV_BADLEN; reads then go to page 0 (in bounds) and
+// writers skip the access (rec() < 0).
+struct RecMap {
+  const int32_t *table;  // nullable
+  int Hkv, cap, n_pages;
+  uint32_t *status;
+  __device__ __forceinline__ int64_t rec(int64_t u, int64_t p) const {
+    if (!table) return blk_base(u, p, cap);
+    const int64_t pg = table[(u / Hkv) * (cap / BLK_TOK) + p / BLK_TOK];
+    if (pg < 0 || pg >= n_pages) {
+      set_status(status, HYQ_DEV_BADLEN);
+      return -1;
+    }
+    return (pg * Hkv + u % Hkv) * BLK_BYTES;
+  }
+  // for reads: an invalid entry reads page 0
+  __device__ __forceinline__ int64_t rec_rd(int64_t u, int64_t p) const {
+    const int64_t r = rec(u, p);
+    return r < 0 ? 0 : r;
+  }
+};
+__host__ __device__ __forceinline__ int64_t rec_kcode(int64_t rec, int64_t p) { return rec + HYQ_BLK_KCODES + (p % BLK_TOK) * ROW_BYTES; }
+__host__ __device__ __forceinline__ int64_t rec_ksz(int64_t rec, int64_t p) { return rec + HYQ_BLK_KSZ + (p % BLK_TOK) * SZ_BYTES; }
+__host__ __device__ __forceinline__ int64_t rec_vcode(int64_t rec, int64_t p) { return rec + HYQ_BLK_VCODES + (p % BLK_TOK) * ROW_BYTES; }
+__host__ __device__ __forceinline__ int64_t rec_vsz(int64_t rec, int64_t p) { return rec + HYQ_BLK_VSZ + (p % BLK_TOK) * SZ_BYTES; }
+__host__ __device__ __forceinline__ int64_t rec_mask(int64_t rec) { return rec + HYQ_BLK_MASK; }
 
 // ---------------------------------------------------------------- smem
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

@@ -118,7 +118,8 @@ __device__ __forceinline__ uint64_t tile_wait_limit() { return 2000000000ull; }
 
 struct DecodeArgs {
   int B, Hq, Hkv, cap, W, vl_cap, U, n_ctas;
-  uint8_t *blocks;        // quantized majority + bitmask, [U][cap/32][BLK_BYTES]
+  uint8_t *blocks;        // quantized majority + bitmask, [U][cap/32][BLK_BYTES] or a page pool
+  RecMap rm;              // record addresses (contiguous or through the block table)
   __half *win_k, *win_v;  // written only by the fused step
   const __half *vl_k, *vl_v;
   const int32_t *vl_count;
@@ -772,17 +773,28 @@ __device__ __forceinline__ void step_exit_row(const DecodeArgs &a, int u, int T_
   const int row = px % I4_TOK;
   const uint32_t code_s = slot + (is_v ? SLOT_VC : 0) + row * ROW_BYTES;
   const uint32_t sz_s = slot + (is_v ? SLOT_VSZ : SLOT_KSZ) + row * SZ_BYTES;
-  uint8_t *code_g = a.blocks + (is_v ? vcode_off(u, px, a.cap) : kcode_off(u, px, a.cap));
-  uint32_t *sz_g = reinterpret_cast<uint32_t *>(a.blocks + (is_v ? vsz_off(u, px, a.cap) : ksz_off(u, px, a.cap)));
+  const int64_t rec = a.rm.rec(u, px);  // < 0: a bad block-table entry; the cache write is skipped
+  uint8_t *code_g = a.blocks + (is_v ? rec_vcode(rec, px) : rec_kcode(rec, px));
+  uint32_t *sz_g = reinterpret_cast<uint32_t *>(a.blocks + (is_v ? rec_vsz(rec, px) : rec_ksz(rec, px)));
   if (q.has_codes) {
     sts32(code_s + q.off0, q.w0);
     sts32(code_s + q.off1, q.w1);
-    *reinterpret_cast<uint32_t *>(code_g + q.off0) = q.w0;
-    *reinterpret_cast<uint32_t *>(code_g + q.off1) = q.w1;
+    if (rec >= 0) {
+      *reinterpret_cast<uint32_t *>(code_g + q.off0) = q.w0;
+      *reinterpret_cast<uint32_t *>(code_g + q.off1) = q.w1;
+    }
   }
   if (q.has_sz) {
     sts32(sz_s + 4 * q.g, q.sz);
-    sz_g[q.g] = q.sz;
+    if (rec >= 0) sz_g[q.g] = q.sz;
+  }
+  if (row == 0 && lane == 0) {
+    // the first row quantized into this record: none of its positions is a
+    // vertical line yet (they lie below T - W), so its bitmask starts clear
+    // -- in the cache and in the staged copy of the tile -- whatever the
+    // record held before
+    sts32(slot + SLOT_MASK, 0u);
+    if (rec >= 0) *reinterpret_cast<uint32_t *>(a.blocks + rec_mask(rec)) = 0u;
   }
   // the old row has been read (its value is consumed above): the new token
   // takes its slot
@@ -838,7 +850,7 @@ __device__ __forceinline__ TileSrc tile_src(const DecodeArgs &a, const Smem &sm,
   bool bad;
   const UnitShape us = shape_of<MODE>(a, sm.unit_tv[u].x, sm.unit_tv[u].y, bad);
   if (MODE != MODE_FP16 && j < us.n4)
-    return {a.blocks + blk_base(u, static_cast<int64_t>(j) * I4_TOK, a.cap), nullptr, BLK_BYTES};
+    return {a.blocks + a.rm.rec_rd(u, static_cast<int64_t>(j) * I4_TOK), nullptr, BLK_BYTES};
   const __half *sk, *sv;
   int n;
   if (MODE == MODE_FP16) {
@@ -1353,6 +1365,7 @@ static hyq_status decode_entry(const hyq_cache *c, const void *q, void *o, float
   a.B = c->batch; a.Hq = c->n_q_heads; a.Hkv = c->n_kv_heads; a.cap = c->capacity;
   a.W = c->window; a.vl_cap = c->vl_capacity; a.U = U; a.n_ctas = N;
   a.blocks = c->blocks;
+  a.rm = RecMap{c->block_table, c->n_kv_heads, c->capacity, c->n_pages, c->dev_status};
   a.win_k = static_cast<__half *>(c->win_k); a.win_v = static_cast<__half *>(c->win_v);
   a.vl_k = static_cast<const __half *>(c->vl_k); a.vl_v = static_cast<const __half *>(c->vl_v);
   a.vl_count = c->vl_count; a.seq_len = c->seq_len;
@@ -1401,6 +1414,7 @@ extern "C" hyq_status hyq_decode_step(const hyq_cache *c, const void *q, const v
   a.B = c->batch; a.Hq = c->n_q_heads; a.Hkv = c->n_kv_heads; a.cap = c->capacity;
   a.W = c->window; a.vl_cap = c->vl_capacity; a.U = U; a.n_ctas = N;
   a.blocks = c->blocks;
+  a.rm = RecMap{c->block_table, c->n_kv_heads, c->capacity, c->n_pages, c->dev_status};
   a.win_k = static_cast<__half *>(c->win_k); a.win_v = static_cast<__half *>(c->win_v);
   a.vl_k = static_cast<const __half *>(c->vl_k); a.vl_v = static_cast<const __half *>(c->vl_v);
   a.vl_count = c->vl_count; a.seq_len = c->seq_len;
@@ -1544,6 +1558,7 @@ extern "C" hyq_status hyq_decode_noalloc(const hyq_cache *c, const void *q, void
   a.B = c->batch; a.Hq = c->n_q_heads; a.Hkv = c->n_kv_heads; a.cap = c->capacity;
   a.W = c->window; a.vl_cap = c->vl_capacity; a.U = U; a.n_ctas = N;
   a.blocks = c->blocks;
+  a.rm = RecMap{c->block_table, c->n_kv_heads, c->capacity, c->n_pages, c->dev_status};
   a.win_k = static_cast<__half *>(c->win_k); a.win_v = static_cast<__half *>(c->win_v);
   a.vl_k = static_cast<const __half *>(c->vl_k); a.vl_v = static_cast<const __half *>(c->vl_v);
   a.vl_count = c->vl_count; a.seq_len = c->seq_len;

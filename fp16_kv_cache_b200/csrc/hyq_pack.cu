@@ -17,6 +17,16 @@
 
 namespace hyq {
 
+__device__ __forceinline__ RecMap recmap(const hyq_cache &c) {
+  return RecMap{c.block_table, c.n_kv_heads, c.capacity, c.n_pages, c.dev_status};
+}
+// The bitmask word of the record holding position p (nullptr: a bad
+// block-table entry, already reported).
+__device__ __forceinline__ uint32_t *mask_of(const hyq_cache &c, int64_t u, int64_t p) {
+  const int64_t r = recmap(c).rec(u, p);
+  return r < 0 ? nullptr : reinterpret_cast<uint32_t *>(c.blocks + rec_mask(r));
+}
+
 __global__ void __launch_bounds__(256) pack_kernel(const __half *__restrict__ x, int64_t n_rows,
                                                    int64_t stride,
                                                    const int64_t *__restrict__ dst_rows,
@@ -54,18 +64,23 @@ __global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half 
     if (p == 0 && t == 0 && !is_v && (u % c.n_kv_heads) == 0) set_status(c.dev_status, HYQ_DEV_BADLEN);
     return;
   }
-  // clear this unit's vertical-line set (block bitmask words and count)
-  if (!is_v && t == 0 && (p % BLK_TOK) == 0) *mask_word(c.blocks, u, p, c.capacity) = 0u;
+  // clear this unit's vertical-line set (the bitmask words of the records
+  // holding its positions, and the count)
   if (!is_v && t == 0 && p == 0) c.vl_count[u] = 0;
   if (p >= T) return;
+  if (!is_v && t == 0 && (p % BLK_TOK) == 0) {
+    uint32_t *m = mask_of(c, u, p);
+    if (m) *m = 0u;
+  }
   const __half *src = (is_v ? v_full : k_full) + up * D;
   const uint4 xv = *reinterpret_cast<const uint4 *>(src + 8 * t);
   const int W = c.window;
   if (p < T - W) {
     const unsigned hmask = 0xFFFFu << (lane & 16);
-    const int64_t co = is_v ? vcode_off(u, p, c.capacity) : kcode_off(u, p, c.capacity);
-    const int64_t so = is_v ? vsz_off(u, p, c.capacity) : ksz_off(u, p, c.capacity);
-    quantize_part(xv, t, hmask, c.blocks + co, reinterpret_cast<uint32_t *>(c.blocks + so), c.dev_status);
+    const int64_t rec = recmap(c).rec(u, p);
+    if (rec >= 0)  // uniform over the row's 16 lanes
+      quantize_part(xv, t, hmask, c.blocks + (is_v ? rec_vcode(rec, p) : rec_kcode(rec, p)),
+                    reinterpret_cast<uint32_t *>(c.blocks + (is_v ? rec_vsz(rec, p) : rec_ksz(rec, p))), c.dev_status);
     if (c.stage_rows > 0 && p >= T - W - c.stage_rows) {  // staging ring: the most recent quantized rows
       __half *st = reinterpret_cast<__half *>(is_v ? c.stage_v : c.stage_k) + (u * c.stage_rows + p % c.stage_rows) * D;
       *reinterpret_cast<uint4 *>(st + 8 * t) = xv;
@@ -104,9 +119,16 @@ __global__ void append_kernel(hyq_cache c, const __half *__restrict__ k_new,
       const unsigned hmask = 0xFFFFu << (lane & 16);
       const uint4 old = *reinterpret_cast<const uint4 *>(win + 8 * t);
       const int64_t p = T - W;
-      const int64_t co = is_v ? vcode_off(u, p, c.capacity) : kcode_off(u, p, c.capacity);
-      const int64_t so = is_v ? vsz_off(u, p, c.capacity) : ksz_off(u, p, c.capacity);
-      quantize_part(old, t, hmask, c.blocks + co, reinterpret_cast<uint32_t *>(c.blocks + so), c.dev_status);
+      const int64_t rec = recmap(c).rec(u, p);
+      if (rec >= 0) {  // uniform over the row's 16 lanes
+        quantize_part(old, t, hmask, c.blocks + (is_v ? rec_vcode(rec, p) : rec_kcode(rec, p)),
+                      reinterpret_cast<uint32_t *>(c.blocks + (is_v ? rec_vsz(rec, p) : rec_ksz(rec, p))),
+                      c.dev_status);
+        // the first row quantized into a record: no position of it is a
+        // vertical line yet (they lie below T - W), so its bitmask starts
+        // clear, whatever the record held before
+        if (!is_v && t == 0 && (p % BLK_TOK) == 0) *reinterpret_cast<uint32_t *>(c.blocks + rec_mask(rec)) = 0u;
+      }
       if (c.stage_rows > 0) {  // the leaving row also enters the staging ring
         __half *st = reinterpret_cast<__half *>(is_v ? c.stage_v : c.stage_k) +
                      (u * c.stage_rows + p % c.stage_rows) * D;
@@ -158,8 +180,11 @@ __global__ void __launch_bounds__(256) vl_reset_kernel(hyq_cache c, const int32_
     const int p = np[i];
     if (p < 0 || p >= L4 || (i > 0 && np[i - 1] >= p)) s_bad = 1;
   }
-  for (int w = threadIdx.x; w < c.capacity / BLK_TOK; w += blockDim.x)
-    *mask_word(c.blocks, u, static_cast<int64_t>(w) * BLK_TOK, c.capacity) = 0u;
+  // the bitmask words of the records holding quantized positions [0, L4)
+  for (int w = threadIdx.x; w < (max(L4, 0) + BLK_TOK - 1) / BLK_TOK; w += blockDim.x) {
+    uint32_t *m = mask_of(c, u, static_cast<int64_t>(w) * BLK_TOK);
+    if (m) *m = 0u;
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
     if (s_bad) set_status(c.dev_status, HYQ_DEV_BADLEN);
@@ -184,7 +209,8 @@ __global__ void __launch_bounds__(512) vl_gather_kernel(hyq_cache c, const int32
   *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.vl_k) + d) = *reinterpret_cast<const uint4 *>(k_full + so);
   *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.vl_v) + d) = *reinterpret_cast<const uint4 *>(v_full + so);
   if (part == 0) {
-    atomicOr(mask_word(c.blocks, u, p, c.capacity), 1u << (p & 31));
+    uint32_t *m = mask_of(c, u, p);
+    if (m) atomicOr(m, 1u << (p & 31));
     c.vl_pos[static_cast<int64_t>(u) * c.vl_capacity + r] = p;
   }
 }
@@ -249,7 +275,7 @@ __global__ void __launch_bounds__(1024) vl_recompact_kernel(hyq_cache c, const i
   for (int j = threadIdx.x; j < old_n; j += blockDim.x) {
     const int p = old[j];
     if (p >= 0 && p < c.capacity && find_sorted(np, k, p) < 0)
-      atomicAnd(mask_word(c.blocks, u, p, c.capacity), ~(1u << (p & 31)));
+      if (uint32_t *m = mask_of(c, u, p)) atomicAnd(m, ~(1u << (p & 31)));
   }
   __syncthreads();
   const int rows = blockDim.x / 16;
@@ -297,7 +323,7 @@ __global__ void __launch_bounds__(1024) vl_recompact_kernel(hyq_cache c, const i
         *reinterpret_cast<uint4 *>(vk + d) = *reinterpret_cast<const uint4 *>(sk + so);
         *reinterpret_cast<uint4 *>(vv + d) = *reinterpret_cast<const uint4 *>(sv + so);
         if (part == 0) {
-          atomicOr(mask_word(c.blocks, u, p, c.capacity), 1u << (p & 31));
+          if (uint32_t *m = mask_of(c, u, p)) atomicOr(m, 1u << (p & 31));
           kpos[n_kept + r] = p;
         }
       }

@@ -26,8 +26,10 @@
 //      rows, and writes the tile transposed ([128 channels][64 keys]) twice,
 //      dequantized and in FP16, through shared memory; the same for the
 //      unit's vertical-line value rows (FP16).
-//   3. pa_attn_kernel  one block of 4 warps per (batch, query head, 128-row
-//      query tile), the longest tiles first.  Thread t owns query row t.
+//   3. pa_attn_kernel  one block of 8 warps per (batch, query head, 128-row
+//      query tile), the longest tiles first.  Two threads own each query
+//      row, each with half of the key columns of a tile and half of the
+//      output columns.
 //      The 5th-generation tensor cores (tcgen05, fp16 operands in shared
 //      memory with the 128-byte swizzle, fp32 accumulators in tensor memory)
 //      compute, per 64-key tile,
@@ -60,7 +62,7 @@ namespace pa {
 
 constexpr int QT = 128;      // query rows per tile (the MMA's M)
 constexpr int KT = 64;       // keys per tile (N of Q K^T, K of P V)
-constexpr int THREADS = 128;
+constexpr int THREADS = 256;  // two threads per query row
 constexpr float SCALE_LOG2 = 0.12751743082459868f;  // log2(e) / sqrt(128)
 constexpr float LN2 = 0.69314718055994531f;
 constexpr float RAISE = 8.f;  // raise the running max only past this margin (exp2 domain)
@@ -81,6 +83,7 @@ struct Args {
   int B, Hq, Hkv, G, cap, W, vl_cap, U;
   const __half *q, *k, *v;  // [B][Hq][cap][128], [B][Hkv][cap][128] x 2
   const uint8_t *blocks;    // the cache's block records (vertical-line bitmask)
+  RecMap rm;                // record addresses (contiguous or through the block table)
   const __half *vl_k, *vl_v;
   const int32_t *vl_pos, *vl_count, *seq_len;
   __half *qh, *ql, *kh, *kl;  // workspace: dequantized rows (hi, lo)
@@ -105,6 +108,9 @@ __device__ __forceinline__ uint64_t desc(uint32_t tile, int R, int ks) {
          (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
          (static_cast<uint64_t>(2) << 61);
 }
+// desc(tile, R, ks) - desc(tile, R, 0), in the start-address field (16-byte
+// units; tiles lie below 256 KB, so the field never carries).
+__device__ __forceinline__ uint32_t koff(int R, int ks) { return (ks >> 2) * (R * 8) + (ks & 3) * 2; }
 // Instruction descriptor: fp32 accumulate, fp16 A and B, both K-major, M = 128.
 __host__ __device__ constexpr uint32_t idesc(int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
@@ -312,6 +318,7 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   __shared__ int s_abort;
   __shared__ uint32_t s_vlmask[2][2];        // bitmask words of a 64-key tile (two jobs in flight)
   __shared__ int s_vlpos[2][KT];             // positions of a vertical-line tile
+  __shared__ float s_red[2][QT];             // the two halves' tile max (and, at the end, row sums)
   const int tid = threadIdx.x, warp = tid >> 5;
   const int BH = a.B * a.Hq;
   const int n_qt = a.cap / QT;
@@ -368,10 +375,17 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = tmem_base;
-  const uint32_t tm_row = tm + (static_cast<uint32_t>(32 * warp) << 16);  // this warp's lane quadrant
+  // Thread (warp w, lane l) owns query row rr = 32 (w % 4) + l -- the tensor
+  // memory lanes its warp may access -- and half hf = w / 4 of the columns:
+  // key columns 32 hf .. 32 hf + 31 of each tile's scores, and output
+  // columns 64 hf .. 64 hf + 63.  The two threads of a row keep the same
+  // running max (the tile max is exchanged through shared memory) and their
+  // own partial sums.
+  const int rq = warp & 3, hf = warp >> 2, rr = 32 * rq + (tid & 31);
+  const uint32_t tm_row = tm + (static_cast<uint32_t>(32 * rq) << 16);
   volatile int *abort = &s_abort;
 
-  const int i = q0 + tid;  // this thread's query row
+  const int i = q0 + rr;  // this thread's query row
   float m_run = -INFINITY, l_run = 0.f;
   bool o_started = false;   // the first P V MMA overwrites O
   uint32_t ph_s = 0, ph_o = 0;
@@ -425,7 +439,7 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
     }
     if (kind != JOB_VL && tid < 2) {
       if (j0 + 32 * tid < T)
-        cp4(smem_u32(&s_vlmask[mb][tid]), a.blocks + blk_base(u, j0 + 32 * tid, a.cap) + HYQ_BLK_MASK);
+        cp4(smem_u32(&s_vlmask[mb][tid]), a.blocks + rec_mask(a.rm.rec_rd(u, j0 + 32 * tid)));
       else
         s_vlmask[mb][tid] = 0u;
     }
@@ -464,14 +478,19 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
     tc_fence_after();
     // ---- S = Q K^T
     if (tid == 0) {
+      // k-step ks of a tile = its descriptor advanced by koff(R, ks) (the
+      // start-address field counts 16-byte units)
+      const uint64_t dqh = desc(s0 + OFF_QH, QT, 0), dql = desc(s0 + OFF_QL, QT, 0), dqf = desc(s0 + OFF_QF, QT, 0);
+      const uint64_t dkh = desc(s0 + OFF_KH, KT, 0), dkl = desc(s0 + OFF_KL, KT, 0), dkf = desc(s0 + OFF_KF, KT, 0);
+#pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
+        const uint32_t oq = koff(QT, ks), ok = koff(KT, ks);
         if (kind != JOB_VL) {
-          const uint64_t aq = desc(s0 + OFF_QH, QT, ks), bk = desc(s0 + OFF_KH, KT, ks);
-          mma(tm + TM_SLO, aq, bk, idesc(KT), ks > 0);
-          mma(tm + TM_SLO, aq, desc(s0 + OFF_KL, KT, ks), idesc(KT), 1u);
-          mma(tm + TM_SLO, desc(s0 + OFF_QL, QT, ks), bk, idesc(KT), 1u);
+          mma(tm + TM_SLO, dqh + oq, dkh + ok, idesc(KT), ks > 0);
+          mma(tm + TM_SLO, dqh + oq, dkl + ok, idesc(KT), 1u);
+          mma(tm + TM_SLO, dql + oq, dkh + ok, idesc(KT), 1u);
         }
-        if (kind != JOB_OFF) mma(tm + TM_SHI, desc(s0 + OFF_QF, QT, ks), desc(s0 + OFF_KF, KT, ks), idesc(KT), ks > 0);
+        if (kind != JOB_OFF) mma(tm + TM_SHI, dqf + oq, dkf + ok, idesc(KT), ks > 0);
       }
       commit(smem_u32(&bars[0]));
     }
@@ -513,14 +532,16 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
       }
     };
     float mx = -INFINITY;
-#pragma unroll 1
-    for (int cb = 0; cb < 2; ++cb) {
+    {
       float x[32];
       uint32_t hm;
-      chunk(cb, x, hm);
+      chunk(hf, x, hm);
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) mx = fmaxf(mx, x[jj]);
     }
+    s_red[hf][rr] = mx;
+    __syncthreads();
+    mx = fmaxf(s_red[0][rr], s_red[1][rr]);  // the same in both threads of the row
     // raise the running max only when this tile exceeds it by more than
     // RAISE (p stays <= 2^RAISE); O and l are rescaled then
     float alpha = 1.f;
@@ -540,7 +561,7 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
     if (__any_sync(0xffffffffu, rescale)) {
       const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
-      for (int cb = 0; cb < D / 32; ++cb) {
+      for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {  // this thread's half of the row
         float ov[32];
         tm_ld32(tm_row + TM_O + 32 * cb, ov);
 #pragma unroll
@@ -548,10 +569,10 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
         tm_st32(tm_row + TM_O + 32 * cb, ov);
       }
     }
-    // P as fp16 into P_lo / P_hi, row tid
+    // P as fp16 into P_lo / P_hi: row rr, this thread's 32 columns
     float lsum = 0.f;
-#pragma unroll 1
-    for (int cb = 0; cb < 2; ++cb) {
+    {
+      const int cb = hf;
       float x[32];
       uint32_t hm;
       chunk(cb, x, hm);
@@ -569,7 +590,7 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
           wh[e] = pk & keep_hi;
           wl[e] = pk & ~keep_hi;
         }
-        const uint32_t off = swz(QT, tid, 32 * cb + 8 * cc);
+        const uint32_t off = swz(QT, rr, 32 * cb + 8 * cc);
         if (kind != JOB_VL)
           asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PL + off), "r"(wl[0]), "r"(wl[1]),
                        "r"(wl[2]), "r"(wl[3]) : "memory");
@@ -587,13 +608,17 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
     // ---- O += P_lo V^ + P_hi V
     if (tid == 0) {
       uint32_t acc = o_started ? 1u : 0u;
+      const uint64_t dpl = desc(s0 + OFF_PL, QT, 0), dph = desc(s0 + OFF_PH, QT, 0);
+      const uint64_t dvq = desc(s0 + OFF_VQ, D, 0), dvf = desc(s0 + OFF_VF, D, 0);
+#pragma unroll
       for (int ks = 0; ks < KT / 16; ++ks) {
+        const uint32_t op = koff(QT, ks), ov = koff(D, ks);
         if (kind != JOB_VL) {
-          mma(tm + TM_O, desc(s0 + OFF_PL, QT, ks), desc(s0 + OFF_VQ, D, ks), idesc(D), acc);
+          mma(tm + TM_O, dpl + op, dvq + ov, idesc(D), acc);
           acc = 1u;
         }
         if (kind != JOB_OFF) {
-          mma(tm + TM_O, desc(s0 + OFF_PH, QT, ks), desc(s0 + OFF_VF, D, ks), idesc(D), acc);
+          mma(tm + TM_O, dph + op, dvf + ov, idesc(D), acc);
           acc = 1u;
         }
       }
@@ -610,12 +635,15 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   }
   cp_wait_group<0>();  // nothing may land in shared memory after the block exits
 
-  // ---- O / l and the log-sum-exp of row i
+  // ---- O / l and the log-sum-exp of row i (the row's sum is the two halves')
+  s_red[hf][rr] = l_run;
+  __syncthreads();
+  l_run = s_red[0][rr] + s_red[1][rr];
   if (!*abort && o_started) {  // uniform: the tensor-memory loads take the whole warp
     const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
     float *orow = a.o + (static_cast<int64_t>(bh) * a.cap + i) * D;
 #pragma unroll
-    for (int cb = 0; cb < D / 32; ++cb) {
+    for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
       float ov[32];
       tm_ld32(tm_row + TM_O + 32 * cb, ov);
       if (i < T)
@@ -624,7 +652,7 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
           *reinterpret_cast<float4 *>(orow + 32 * cb + jj) =
               make_float4(ov[jj] * inv, ov[jj + 1] * inv, ov[jj + 2] * inv, ov[jj + 3] * inv);
     }
-    if (a.lse && i < T) a.lse[static_cast<int64_t>(bh) * a.cap + i] = (m_run + __log2f(l_run)) * LN2;
+    if (a.lse && i < T && hf == 0) a.lse[static_cast<int64_t>(bh) * a.cap + i] = (m_run + __log2f(l_run)) * LN2;
   } else if (o_started && i < T) {
     // a wait ran out: the row is undefined; leave a recognisable value
     if (a.lse) a.lse[static_cast<int64_t>(bh) * a.cap + i] = __int_as_float(0x7fc00000);
@@ -692,6 +720,7 @@ extern "C" hyq_status hyq_prefill_attention(const hyq_cache *c, const void *q, c
   a.k = static_cast<const __half *>(k_full);
   a.v = static_cast<const __half *>(v_full);
   a.blocks = c->blocks;
+  a.rm = RecMap{c->block_table, c->n_kv_heads, c->capacity, c->n_pages, c->dev_status};
   a.vl_k = static_cast<const __half *>(c->vl_k);
   a.vl_v = static_cast<const __half *>(c->vl_v);
   a.vl_pos = c->vl_pos; a.vl_count = c->vl_count; a.seq_len = c->seq_len;

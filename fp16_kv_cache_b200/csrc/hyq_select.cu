@@ -54,7 +54,8 @@ struct SelectArgs {
   int B, Hq, Hkv, G, n_q, q_ring, cap, W, vl_cap, U, R, k, n_chunks;
   const __half *q;       // [B][Hq][n_q][128]
   const __half *k_full;  // nullable [B][Hkv][cap][128]
-  const uint8_t *blocks;  // quantized majority + bitmask, [U][cap/32][BLK_BYTES]
+  const uint8_t *blocks;  // quantized majority + bitmask, [U][cap/32][BLK_BYTES] or a page pool
+  RecMap rm;              // record addresses (contiguous or through the block table)
   const __half *win_k, *vl_k;
   const int32_t *vl_pos, *vl_count;
   const int32_t *seq_len;
@@ -152,7 +153,8 @@ __device__ __forceinline__ void key_load(const SelectArgs &a, int u, int T, int 
     row = a.win_k + (static_cast<int64_t>(u) * a.W + key % a.W) * D;
   } else {
     // a vertical line: its row is the rank of its bit among the unit's set bits
-    const uint32_t w = *reinterpret_cast<const uint32_t *>(a.blocks + blk_base(u, key, a.cap) + HYQ_BLK_MASK);
+    const int64_t rec = a.rm.rec_rd(u, key);
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(a.blocks + rec_mask(rec));
     if ((w >> (key & 31)) & 1u) {
       const int slot = a.rank_base[static_cast<int64_t>(u) * (a.cap / 32) + (key >> 5)] +
                        __popc(w & ((1u << (key & 31)) - 1u));
@@ -166,10 +168,11 @@ __device__ __forceinline__ void key_load(const SelectArgs &a, int u, int T, int 
     return;
   }
   r.kind = 2;
-  const uint4 *codes = reinterpret_cast<const uint4 *>(a.blocks + kcode_off(u, key, a.cap));
+  const int64_t rec = a.rm.rec_rd(u, key);
+  const uint4 *codes = reinterpret_cast<const uint4 *>(a.blocks + rec_kcode(rec, key));
 #pragma unroll
   for (int c = 0; c < 4; ++c) r.v[c] = codes[c];
-  r.v[4] = *reinterpret_cast<const uint4 *>(a.blocks + ksz_off(u, key, a.cap));
+  r.v[4] = *reinterpret_cast<const uint4 *>(a.blocks + rec_ksz(rec, key));
 }
 
 // Write the thread's 8 chunks of key row kk as fp16 (hi) and, in cache mode,
@@ -491,11 +494,14 @@ __global__ void __launch_bounds__(1024) rank_kernel(const SelectArgs a) {
   const int nw = a.cap / 32;
   int32_t *out = a.rank_base + static_cast<int64_t>(u) * nw;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  // records holding quantized positions [0, T - W); the words after them count 0
+  const int T = sel_T(a, u);
+  const int nq = (T >= 0 && T <= a.cap) ? (max(T - a.W, 0) + 31) / 32 : 0;
   int carry = 0;
   for (int base = 0; base < nw; base += blockDim.x) {
     const int i = base + threadIdx.x;
-    const int v = (i < nw) ? __popc(*reinterpret_cast<const uint32_t *>(
-                                 a.blocks + blk_base(u, static_cast<int64_t>(i) * 32, a.cap) + HYQ_BLK_MASK))
+    const int v = (i < nq) ? __popc(*reinterpret_cast<const uint32_t *>(
+                                 a.blocks + rec_mask(a.rm.rec_rd(u, static_cast<int64_t>(i) * 32))))
                            : 0;
     int x = v;
 #pragma unroll
@@ -793,6 +799,7 @@ extern "C" hyq_status hyq_select_vl(const hyq_cache *c, const void *q_sel, int32
   a.q = static_cast<const __half *>(q_sel);
   a.k_full = static_cast<const __half *>(k_full);
   a.blocks = c->blocks;
+  a.rm = RecMap{c->block_table, c->n_kv_heads, c->capacity, c->n_pages, c->dev_status};
   a.win_k = static_cast<const __half *>(c->win_k); a.vl_k = static_cast<const __half *>(c->vl_k);
   a.vl_pos = c->vl_pos; a.vl_count = c->vl_count; a.seq_len = c->seq_len;
   uint8_t *w = static_cast<uint8_t *>(ws);

@@ -11,6 +11,8 @@ import contextlib
 import ctypes
 import os
 
+import numpy as np
+
 import torch
 
 from . import build as _build
@@ -55,6 +57,7 @@ class hyq_cache(ctypes.Structure):
         ("dev_status", ctypes.c_void_p),
         ("stage_k", ctypes.c_void_p), ("stage_v", ctypes.c_void_p),
         ("stage_rows", ctypes.c_int32),
+        ("block_table", ctypes.c_void_p), ("n_pages", ctypes.c_int32),
     ]
 
 
@@ -165,14 +168,26 @@ def _check(rc, what):
 class HybridCache:
     """Device buffers of one layer's hybrid cache plus its C descriptor."""
 
-    def __init__(self, batch, n_q_heads, n_kv_heads, capacity, vl_capacity, device="cuda", stage_rows=0):
+    def __init__(self, batch, n_q_heads, n_kv_heads, capacity, vl_capacity, device="cuda", stage_rows=0,
+                 block_table=None, n_pages=0):
+        """block_table (int32 [B][capacity/32]) and n_pages: the quantized
+        majority lives in a pool of n_pages pages of n_kv_heads records, and
+        sequence b's 32-position block j in page block_table[b][j]."""
         if capacity % 128:
             raise ValueError("capacity must be a multiple of 128")
         B, Hkv = batch, n_kv_heads
         dev = torch.device(device)
         z = lambda *s, dt: torch.zeros(*s, dtype=dt, device=dev)  # noqa: E731
         self.B, self.Hq, self.Hkv, self.cap, self.vl_cap = B, n_q_heads, Hkv, capacity, vl_capacity
-        self.blocks = z(B, Hkv, capacity // BLOCK_TOKENS, BLOCK_BYTES, dt=torch.uint8)
+        self.block_table = None
+        if block_table is not None:
+            self.block_table = torch.as_tensor(block_table, dtype=torch.int32).reshape(B, capacity // BLOCK_TOKENS)
+            self.block_table = self.block_table.to(dev).contiguous()
+            self.n_pages = int(n_pages)
+            self.blocks = z(self.n_pages, Hkv, BLOCK_BYTES, dt=torch.uint8)
+        else:
+            self.n_pages = 0
+            self.blocks = z(B, Hkv, capacity // BLOCK_TOKENS, BLOCK_BYTES, dt=torch.uint8)
         self.win_k = z(B, Hkv, WINDOW, HEAD_DIM, dt=torch.float16)
         self.win_v = z(B, Hkv, WINDOW, HEAD_DIM, dt=torch.float16)
         self.vl_k = z(B, Hkv, vl_capacity, HEAD_DIM, dt=torch.float16)
@@ -193,6 +208,8 @@ class HybridCache:
             setattr(c, name, getattr(self, name).data_ptr())
         if self.stage_rows:
             c.stage_k, c.stage_v, c.stage_rows = self.stage_k.data_ptr(), self.stage_v.data_ptr(), self.stage_rows
+        if self.block_table is not None:
+            c.block_table, c.n_pages = self.block_table.data_ptr(), self.n_pages
         self.desc = c
 
     def ref(self):
@@ -214,6 +231,10 @@ class HybridCache:
         [B][Hkv][cap][64] u8, k_sz [B][Hkv][cap][8] u16, v_codes, v_sz,
         mask [B][Hkv][cap/32] u32).  A copy; for inspection and tests."""
         b = self.blocks.cpu().numpy()
+        if self.block_table is not None:  # gather the sequences' logical blocks from the pool
+            tab = self.block_table.cpu().numpy()
+            ok = (tab >= 0) & (tab < self.n_pages)
+            b = np.where(ok[:, None, :, None], b[np.where(ok, tab, 0)].transpose(0, 2, 1, 3), 0).astype(np.uint8)
         B, H, nb, _ = b.shape
         cap = nb * BLOCK_TOKENS
         def field(off, width):

@@ -141,6 +141,16 @@ typedef struct {
    * turns it off (stage_k / stage_v may then be NULL). */
   void *stage_k, *stage_v;
   int32_t stage_rows; /* 0, or 1..1024 */
+  /* Paged quantized majority (optional).  NULL: `blocks` holds each unit's
+   * capacity/32 records contiguously (layout above).  Non-NULL: `blocks` is
+   * a pool of n_pages pages of n_kv_heads records each (page g, KV head h
+   * at record g * n_kv_heads + h), and sequence b's positions
+   * [32 j, 32 j + 32) live in page block_table[b * (capacity/32) + j]
+   * (int32 [B][capacity/32], device; pages may be shared only by sequences
+   * that never write them).  An entry outside [0, n_pages) that a kernel
+   * needs raises HYQ_DEV_BADLEN: reads go to page 0, writes are skipped. */
+  int32_t *block_table;
+  int32_t n_pages; /* >= 1 when block_table is set */
 } hyq_cache;
 
 /*
