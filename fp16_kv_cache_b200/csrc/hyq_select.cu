@@ -84,7 +84,7 @@ __device__ __forceinline__ int sel_T(const SelectArgs &a, int u) { return a.seq_
 // operands are K-major with the 128-byte swizzle.  The epilogue reads the
 // accumulators with tcgen05.ld: warp w owns rows 32 (w % 4) .. + 31 of each
 // row block and columns 64 (w / 4) .. + 63 of the sub-tile.
-constexpr int TC_THREADS = 256;
+constexpr int TC_THREADS = 512;  // 16 warps: 4 lane quadrants x 4 column quarters
 constexpr int TC_NK = 128;               // keys per sub-tile
 constexpr int TC_TILE = TC_NK * 256;     // bytes of a [128][128] fp16 tile
 constexpr int TC_MAX_RB = SEL_MAX_ROWS / 128;
@@ -106,6 +106,8 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t tile, int ks) {
          (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
          (static_cast<uint64_t>(2) << 61);
 }
+// sw128_desc(tile, ks) - sw128_desc(tile, 0) in the start-address field.
+__device__ __forceinline__ uint32_t sw128_koff(int ks) { return (ks >> 2) * (TC_NK * 128 / 16) + (ks & 3) * 2; }
 // Instruction descriptor: fp32 accumulate, fp16 A and B, both K-major,
 // N = 128, M = 128.
 constexpr uint32_t TC_IDESC = (1u << 4) | ((uint32_t)(TC_NK >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
@@ -133,15 +135,16 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// Raw bytes of one thread's half key row (64 channels) for the next sub-tile:
-// FP16 (window, vertical line, prefill) as 8 x 16 B, INT4 as the 4 x 16 B
-// packed row plus the 16-byte scale/zero row.
+// Raw bytes of one thread's quarter key row (32 channels, one quantization
+// group) for the next sub-tile: FP16 (window, vertical line, prefill) as
+// 4 x 16 B, INT4 as the 4 x 16 B packed row plus the group's (scale, zero).
 struct KeyRaw {
-  uint4 v[8];
+  uint4 v[4];
+  uint32_t sz;
   int kind;  // 0 zero, 1 FP16, 2 INT4
 };
 
-// Thread t loads key (t % 128) of the sub-tile, channels 64 (t / 128) .. + 63.
+// Thread t loads key (t % 128) of the sub-tile, channels 32 (t / 128) .. + 31.
 template <bool CACHE>
 __device__ __forceinline__ void key_load(const SelectArgs &a, int u, int T, int key, int key_end, int hf, KeyRaw &r) {
   r.kind = 0;
@@ -164,7 +167,7 @@ __device__ __forceinline__ void key_load(const SelectArgs &a, int u, int T, int 
   if (row) {
     r.kind = 1;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) r.v[c] = *reinterpret_cast<const uint4 *>(row + 64 * hf + 8 * c);
+    for (int c = 0; c < 4; ++c) r.v[c] = *reinterpret_cast<const uint4 *>(row + 32 * hf + 8 * c);
     return;
   }
   r.kind = 2;
@@ -172,17 +175,17 @@ __device__ __forceinline__ void key_load(const SelectArgs &a, int u, int T, int 
   const uint4 *codes = reinterpret_cast<const uint4 *>(a.blocks + rec_kcode(rec, key));
 #pragma unroll
   for (int c = 0; c < 4; ++c) r.v[c] = codes[c];
-  r.v[4] = *reinterpret_cast<const uint4 *>(a.blocks + rec_ksz(rec, key));
+  r.sz = *reinterpret_cast<const uint32_t *>(a.blocks + rec_ksz(rec, key) + 4 * hf);
 }
 
-// Write the thread's 8 chunks of key row kk as fp16 (hi) and, in cache mode,
+// Write the thread's 4 chunks of key row kk as fp16 (hi) and, in cache mode,
 // the fp16 remainder (lo).  INT4: x = zero + code * scale in fp32 (one
 // rounding), hi = fp16(x), lo = fp16(x - hi).
 template <bool CACHE>
 __device__ __forceinline__ void key_store(const KeyRaw &r, int kk, int hf, uint8_t *hi, uint8_t *lo) {
 #pragma unroll
-  for (int cc = 0; cc < 8; ++cc) {
-    const int c = 8 * hf + cc;  // 16-byte chunk = channels 8c .. 8c+7
+  for (int cc = 0; cc < 4; ++cc) {
+    const int c = 4 * hf + cc;  // 16-byte chunk = channels 8c .. 8c+7, group hf
     uint4 h = make_uint4(0, 0, 0, 0), l = make_uint4(0, 0, 0, 0);
     if (r.kind == 1) {
       h = r.v[cc];
@@ -194,8 +197,7 @@ __device__ __forceinline__ void key_store(const KeyRaw &r, int kk, int hf, uint8
       const uint4 vv = r.v[pc];
       const uint32_t wp0 = hh ? vv.y : vv.x;  // piece 2pc, word hh
       const uint32_t wp1 = hh ? vv.w : vv.z;  // piece 2pc + 1, word hh
-      const uint32_t szw = (g == 0) ? r.v[4].x : (g == 1) ? r.v[4].y : (g == 2) ? r.v[4].z : r.v[4].w;
-      const __half2 sz = u2h(szw);
+      const __half2 sz = u2h(r.sz);  // group g == hf
       const float sc = __low2float(sz), zr = __high2float(sz);
       uint32_t hw[4], lw[4];
 #pragma unroll
@@ -255,10 +257,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
   uint8_t *sQ = sm;                                      // [n_rbt][32 KB]
   uint8_t *sK = sQ + n_rbt * TC_TILE;                    // [nbuf][KT]
   float *csum = reinterpret_cast<float *>(sK + nbuf * KT);              // [4][128]
-  float2 *pst = reinterpret_cast<float2 *>(csum + 4 * TC_NK);           // [TC_MAX_RB][128]
-  float *moff = reinterpret_cast<float *>(pst + TC_MAX_RB * 128);       // [SEL_MAX_ROWS] pass 2: m_r - log2(1/l_r)
+  float2 *pst = reinterpret_cast<float2 *>(csum + 4 * TC_NK);           // [3][TC_MAX_RB][128]
+  float *moff = reinterpret_cast<float *>(pst + 3 * TC_MAX_RB * 128);   // [SEL_MAX_ROWS] pass 2: m_r - log2(1/l_r)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qd = warp & 3, hfw = warp >> 2;  // TMEM lane quadrant, column half
+  const int qd = warp & 3, hfw = warp >> 2;  // TMEM lane quadrant, column quarter
   const uint32_t acc_cols = static_cast<uint32_t>(n_rbt) * TC_NK;      // one accumulator set
   const uint32_t need = acc_cols * nbuf;
   const uint32_t ncols = (need <= 128) ? 128u : (need <= 256) ? 256u : 512u;
@@ -282,27 +284,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
   const int per = (n_items + gridDim.x - 1) / gridDim.x;
   const int it0 = min(n_items, static_cast<int>(blockIdx.x) * per), it1 = min(n_items, it0 + per);
   int q_unit = -1, q_T = -1;
-  const int kk = tid & 127, hfk = tid >> 7;  // key row and channel half this thread stages
+  const int kk = tid & 127, hfk = tid >> 7;  // key row and channel quarter (quantization group) this thread stages
   KeyRaw raw;
   bool have_next = false;  // raw holds the first tile of the next item
 
   // one sub-tile's MMAs into accumulator set `buf` from key buffer `buf`
   auto issue = [&](int buf) {
     if (tid == 0) {
+      // descriptors of k-step 0; k-step ks adds sw128_koff(ks) to the
+      // start-address field (16-byte units; tiles lie below 256 KB)
       const uint32_t kh = smem_u32(sK + buf * KT), kl = kh + TC_TILE;
-      for (int rb = 0; rb < n_rbt; ++rb)
+      const uint64_t dkh = sw128_desc(kh, 0), dkl = sw128_desc(kl, 0);
+      for (int rb = 0; rb < n_rbt; ++rb) {
+        const uint64_t dq = sw128_desc(smem_u32(sQ) + rb * TC_TILE, 0);
+        const uint32_t d = tbase + buf * acc_cols + rb * TC_NK;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t ad = sw128_desc(smem_u32(sQ) + rb * TC_TILE, ks);
-          const uint32_t d = tbase + buf * acc_cols + rb * TC_NK;
+          const uint32_t o = sw128_koff(ks);
           if (PASS == 1) {  // rows on M, keys on N
-            tc_mma(d, ad, sw128_desc(kh, ks), ks > 0);
-            if (CACHE) tc_mma(d, ad, sw128_desc(kl, ks), 1u);
+            tc_mma(d, dq + o, dkh + o, ks > 0);
+            if (CACHE) tc_mma(d, dq + o, dkl + o, 1u);
           } else {          // keys on M, rows on N: each TMEM lane is one key column
-            tc_mma(d, sw128_desc(kh, ks), ad, ks > 0);
-            if (CACHE) tc_mma(d, sw128_desc(kl, ks), ad, 1u);
+            tc_mma(d, dkh + o, dq + o, ks > 0);
+            if (CACHE) tc_mma(d, dkl + o, dq + o, 1u);
           }
         }
+      }
       asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                        smem_u32(&mbar[buf]))
                    : "memory");
@@ -396,7 +403,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
       phase[buf] ^= 1u;
       tc_fence_after();
       if (PASS == 1) {
-        // epilogue: this thread's row of each row block, 64 key columns
+        // epilogue: this thread's row of each row block, 32 key columns
         const bool all_visible = key0 + TC_NK <= k1 && key0 + TC_NK - 1 <= T - a.n_q;
 #pragma unroll
         for (int rb = 0; rb < TC_MAX_RB; ++rb) {
@@ -404,12 +411,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
           const int r = 128 * rb + 32 * qd + lane;
           const bool row_ok = r < a.R;
           const int qpos = row_ok ? T - a.n_q + r % a.n_q : -1;  // last key this query sees
-#pragma unroll
-          for (int cb = 0; cb < 2; ++cb) {
+          {
             float v[32];
             // every lane of the warp takes part in the tensor-memory load
-            tc_ld32(tbase + (static_cast<uint32_t>(32 * qd) << 16) + buf * acc_cols + rb * TC_NK + 64 * hfw + 32 * cb, v);
-            const int kb = key0 + 64 * hfw + 32 * cb;  // key of v[0]
+            tc_ld32(tbase + (static_cast<uint32_t>(32 * qd) << 16) + buf * acc_cols + rb * TC_NK + 32 * hfw, v);
+            const int kb = key0 + 32 * hfw;  // key of v[0]
             if (!(all_visible && row_ok))
 #pragma unroll
               for (int j = 0; j < 32; ++j)
@@ -429,20 +435,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
         }
       } else {
         // epilogue: this thread is key column 32 (w % 4) + lane of the
-        // sub-tile; it sums p over its half of the rows (every candidate
+        // sub-tile; it sums p over its quarter of the rows (every candidate
         // key is visible to every selection query)
         float acc = 0.f;
 #pragma unroll
         for (int rb = 0; rb < TC_MAX_RB; ++rb) {
           if (rb >= n_rbt) break;
+          float v[32];
+          tc_ld32(tbase + (static_cast<uint32_t>(32 * qd) << 16) + buf * acc_cols + rb * TC_NK + 32 * hfw, v);
+          const float *mo = moff + rb * TC_NK + 32 * hfw;  // row of v[0]
 #pragma unroll
-          for (int cb = 0; cb < 2; ++cb) {
-            float v[32];
-            tc_ld32(tbase + (static_cast<uint32_t>(32 * qd) << 16) + buf * acc_cols + rb * TC_NK + 64 * hfw + 32 * cb, v);
-            const float *mo = moff + rb * TC_NK + 64 * hfw + 32 * cb;  // row of v[0]
-#pragma unroll
-            for (int j = 0; j < 32; ++j) acc += fast_exp2(fmaf(v[j], SEL_SCALE, -mo[j]));
-          }
+          for (int j = 0; j < 32; ++j) acc += fast_exp2(fmaf(v[j], SEL_SCALE, -mo[j]));
         }
         csum[hfw * TC_NK + 32 * qd + lane] = acc;
       }
@@ -451,7 +454,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
       tc_fence_after();
       if (PASS == 2 && tid < TC_NK) {
         const int key = key0 + tid;
-        if (key < k1) a.colsum_part[static_cast<int64_t>(u) * a.cap + key] = csum[tid] + csum[TC_NK + tid];
+        // fixed order: ((q0 + q1) + q2) + q3, the same for every key
+        if (key < k1)
+          a.colsum_part[static_cast<int64_t>(u) * a.cap + key] =
+              ((csum[tid] + csum[TC_NK + tid]) + csum[2 * TC_NK + tid]) + csum[3 * TC_NK + tid];
       }
       if (nbuf == 1 && st + 1 < nsub) {
         key_store<CACHE>(raw, kk, hfk, sK, sK + TC_TILE);
@@ -462,21 +468,30 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
       if (s_abort) break;
     }
     if (PASS == 1) {
-      // merge the two column halves of every row, then write the chunk partial
-      if (hfw == 1)
+      // merge the four column quarters of every row, then write the chunk partial
+      if (hfw > 0)
 #pragma unroll
         for (int rb = 0; rb < TC_MAX_RB; ++rb)
-          if (rb < n_rbt) pst[rb * 128 + 32 * qd + lane] = make_float2(rm[rb], rl[rb]);
+          if (rb < n_rbt) pst[((hfw - 1) * TC_MAX_RB + rb) * 128 + 32 * qd + lane] = make_float2(rm[rb], rl[rb]);
       __syncthreads();
       if (hfw == 0)
 #pragma unroll
         for (int rb = 0; rb < TC_MAX_RB; ++rb) {
           const int r = 128 * rb + 32 * qd + lane;
           if (rb >= n_rbt || r >= a.R) continue;
-          const float2 o = pst[rb * 128 + 32 * qd + lane];
-          const float M = fmaxf(rm[rb], o.x);
+          float2 o[3];
+          float M = rm[rb];
+#pragma unroll
+          for (int qq = 0; qq < 3; ++qq) {
+            o[qq] = pst[(qq * TC_MAX_RB + rb) * 128 + 32 * qd + lane];
+            M = fmaxf(M, o[qq].x);
+          }
           float L = 0.f;
-          if (M != -INFINITY) L = rl[rb] * fast_exp2(rm[rb] - M) + o.y * fast_exp2(o.x - M);
+          if (M != -INFINITY) {
+            L = rl[rb] * fast_exp2(rm[rb] - M);
+#pragma unroll
+            for (int qq = 0; qq < 3; ++qq) L += o[qq].y * fast_exp2(o[qq].x - M);
+          }
           a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + r] = make_float2(M, L);
         }
     }
@@ -722,7 +737,7 @@ static size_t score_smem_bytes(int R, bool cache) {
   const int n_rbt = (R + 127) / 128;
   const int nbuf = (n_rbt <= 2) ? 2 : 1;
   return 1024 /* alignment */ + static_cast<size_t>(n_rbt) * TC_TILE + static_cast<size_t>(nbuf) * (cache ? 2 : 1) * TC_TILE +
-         SEL_KC * 4 + 4 * TC_NK * 4 + TC_MAX_RB * 128 * 8 + SEL_MAX_ROWS * 4;
+         SEL_KC * 4 + 4 * TC_NK * 4 + 3 * TC_MAX_RB * 128 * 8 + SEL_MAX_ROWS * 4;
 }
 
 static cudaError_t select_launch(const SelectArgs &a, bool cache, cudaStream_t s) {
