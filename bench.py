@@ -181,8 +181,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
-    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4],
-                    help="workload (2: the headline Llama-3.1-8B 32K batch-1 decode; 3 and 4 for profiling)")
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4],
+                    help="workload (2: the headline Llama-3.1-8B 32K batch-1 decode; 1, 3 and 4 for profiling)")
     ap.add_argument("--no-prefill-attention", action="store_true",
                     help="skip timing hyq_prefill_attention over the prompt")
     ap.add_argument("--no-batched", action="store_true",

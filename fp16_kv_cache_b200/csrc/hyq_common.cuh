@@ -8,6 +8,7 @@
 
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include <utility>
@@ -15,6 +16,17 @@
 #include "../../include/hyq.h"
 
 namespace hyq {
+
+// Host-side NVTX range named after the entry point, open for the whole call
+// (argument checks, launches).  NVTX is header-only: without a tool attached
+// to the process the push and pop return at once.
+struct CallRange {
+  explicit CallRange(const char *name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange &) = delete;
+  CallRange &operator=(const CallRange &) = delete;
+};
+#define HYQ_RANGE(name) const ::hyq::CallRange hyq_call_range_(name)
 
 constexpr int D = 128;
 constexpr int GROUP = 32;

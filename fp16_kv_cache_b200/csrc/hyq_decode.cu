@@ -435,6 +435,9 @@ __device__ __forceinline__ void int4_tile(WarpState &st, uint32_t slot, int n_va
     const int tA = 16 * mt + sig(r), tB = tA + 8;
     const uint4 wa = lds128(vsz + tA * SZ_BYTES), wb = lds128(vsz + tB * SZ_BYTES);
     const uint32_t waw[4] = {wa.x, wa.y, wa.z, wa.w}, wbw[4] = {wb.x, wb.y, wb.z, wb.w};
+    // P of rows A and B as fp16 pairs (heads 2q, 2q+1), shared by the zero
+    // term and, scaled per group, by the code MMAs
+    const uint32_t pa2 = pack_half2(p[mt][0], p[mt][1]), pb2 = pack_half2(p[mt][2], p[mt][3]);
     {
       // zero term: A = Vzero^T (group r&3 of the tokens of k rows 2q, 2q+1,
       // 8 + 2q, 9 + 2q), B = P^T unscaled
@@ -445,18 +448,18 @@ __device__ __forceinline__ void int4_tile(WarpState &st, uint32_t slot, int n_va
       asm volatile("ld.shared.u32 %0, [%1];" : "=r"(z2) : "r"(zrow + (16 * mt + s2q + 8) * SZ_BYTES));
       asm volatile("ld.shared.u32 %0, [%1];" : "=r"(z3) : "r"(zrow + (16 * mt + s2q1 + 8) * SZ_BYTES));
       float z4[4] = {st.zacc[0], st.zacc[1], 0.f, 0.f};
-      mma16816(z4, prmt(z0, z1, 0x7632u), 0u, prmt(z2, z3, 0x7632u), 0u,
-               movmatrix_t(pack_half2(p[mt][0], p[mt][1])), movmatrix_t(pack_half2(p[mt][2], p[mt][3])));
+      mma16816(z4, prmt(z0, z1, 0x7632u), 0u, prmt(z2, z3, 0x7632u), 0u, movmatrix_t(pa2), movmatrix_t(pb2));
       st.zacc[0] = z4[0];
       st.zacc[1] = z4[1];
     }
+    // p * vscale in fp16 (one rounding of the fp16 p): the row's scale of
+    // group g duplicated into both halves, one packed multiply per row
     uint32_t bq[NG][2];
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
-      const float sa = __low2float(u2h(waw[g]));
-      const float sb = __low2float(u2h(wbw[g]));
-      bq[g][0] = movmatrix_t(pack_half2(p[mt][0] * sa, p[mt][1] * sa));
-      bq[g][1] = movmatrix_t(pack_half2(p[mt][2] * sb, p[mt][3] * sb));
+      const uint32_t sa2 = prmt(waw[g], 0u, 0x1010u), sb2 = prmt(wbw[g], 0u, 0x1010u);
+      bq[g][0] = movmatrix_t(h2u(__hmul2(u2h(pa2), u2h(sa2))));
+      bq[g][1] = movmatrix_t(h2u(__hmul2(u2h(pb2), u2h(sb2))));
     }
     const uint32_t vrow = vc + 8 * r;
     const uint2 x0 = lds64(vrow + (16 * mt + s2q) * ROW_BYTES);
@@ -1378,11 +1381,13 @@ static hyq_status decode_entry(const hyq_cache *c, const void *q, void *o, float
 
 extern "C" hyq_status hyq_decode(const hyq_cache *c, const void *q, void *o, float *lse,
                                  int32_t n_ctas, void *ws, size_t ws_bytes, void *stream) {
+  HYQ_RANGE("hyq_decode");
   return decode_entry<MODE_HYBRID>(c, q, o, lse, n_ctas, ws, ws_bytes, stream);
 }
 
 extern "C" hyq_status hyq_decode_vl_only(const hyq_cache *c, const void *q, void *o, float *lse,
                                          int32_t n_ctas, void *ws, size_t ws_bytes, void *stream) {
+  HYQ_RANGE("hyq_decode_vl_only");
   return decode_entry<MODE_VLONLY>(c, q, o, lse, n_ctas, ws, ws_bytes, stream);
 }
 
@@ -1396,6 +1401,7 @@ extern "C" size_t hyq_decode_step_workspace(const hyq_cache *c, int32_t n_ctas) 
 extern "C" hyq_status hyq_decode_step(const hyq_cache *c, const void *q, const void *k_new, const void *v_new,
                                       void *q_ring, int32_t n_q, void *o, float *lse, int32_t n_ctas, void *ws,
                                       size_t ws_bytes, void *stream) {
+  HYQ_RANGE("hyq_decode_step");
   hyq_status s = hyq_check_cache(c);
   if (s != HYQ_OK) return s;
   if (!q || !o || !k_new || !v_new) return HYQ_ERR_INVALID;
@@ -1436,6 +1442,7 @@ extern "C" hyq_status hyq_decode_fp16(const void *q, const void *k, const void *
                                       int32_t n_kv_heads, int32_t capacity, void *o, float *lse,
                                       int32_t n_ctas, void *ws, size_t ws_bytes,
                                       uint32_t *dev_status, void *stream) {
+  HYQ_RANGE("hyq_decode_fp16");
   if (!q || !k || !v || !seq_len || !o) return HYQ_ERR_INVALID;
   if (batch <= 0 || n_kv_heads <= 0 || n_q_heads <= 0 || capacity <= 0 || n_ctas < 0)
     return HYQ_ERR_INVALID;
@@ -1539,6 +1546,7 @@ bool noalloc_address(void **out) {
 
 extern "C" hyq_status hyq_decode_noalloc(const hyq_cache *c, const void *q, void *o, float *lse,
                                          void *stream) {
+  HYQ_RANGE("hyq_decode_noalloc");
   hyq_status s = hyq_check_cache(c);
   if (s != HYQ_OK) return s;
   if (!q || !o) return HYQ_ERR_INVALID;

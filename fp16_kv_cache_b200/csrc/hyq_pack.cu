@@ -350,6 +350,7 @@ extern "C" hyq_status hyq_check_cache(const hyq_cache *c);  // hyq_api.cu
 extern "C" hyq_status hyq_pack(const void *x, int64_t n_rows, int64_t row_stride,
                                const int64_t *dst_rows, uint8_t *codes, void *sz,
                                uint32_t *dev_status, void *stream) {
+  HYQ_RANGE("hyq_pack");
   if (n_rows < 0 || row_stride < D || (row_stride % 8) != 0) return HYQ_ERR_INVALID;
   if (n_rows == 0) return HYQ_OK;
   if (!x || !codes || !sz) return HYQ_ERR_INVALID;
@@ -366,6 +367,7 @@ extern "C" hyq_status hyq_pack(const void *x, int64_t n_rows, int64_t row_stride
 
 extern "C" hyq_status hyq_prefill(const hyq_cache *c, const void *k_full, const void *v_full,
                                   void *stream) {
+  HYQ_RANGE("hyq_prefill");
   hyq_status s = hyq_check_cache(c);
   if (s != HYQ_OK) return s;
   if (!k_full || !v_full) return HYQ_ERR_INVALID;
@@ -381,6 +383,7 @@ extern "C" hyq_status hyq_prefill(const hyq_cache *c, const void *k_full, const 
 
 extern "C" hyq_status hyq_append(const hyq_cache *c, const void *k_new, const void *v_new,
                                  const void *q_new, void *q_ring, int32_t n_q, void *stream) {
+  HYQ_RANGE("hyq_append");
   hyq_status s = hyq_check_cache(c);
   if (s != HYQ_OK) return s;
   if (!k_new || !v_new) return HYQ_ERR_INVALID;
@@ -399,6 +402,7 @@ extern "C" hyq_status hyq_append(const hyq_cache *c, const void *k_new, const vo
 extern "C" hyq_status hyq_vl_apply(const hyq_cache *c, const int32_t *pos, int32_t k,
                                    const void *k_full, const void *v_full,
                                    int32_t *n_unpromoted, void *stream) {
+  HYQ_RANGE("hyq_vl_apply");
   hyq_status s = hyq_check_cache(c);
   if (s != HYQ_OK) return s;
   if (k < 0 || k > c->vl_capacity) return HYQ_ERR_INVALID;

@@ -699,6 +699,7 @@ extern "C" size_t hyq_prefill_attention_workspace(const hyq_cache *c) {
 extern "C" hyq_status hyq_prefill_attention(const hyq_cache *c, const void *q, const void *k_full,
                                             const void *v_full, float *o, float *lse, void *ws,
                                             size_t ws_bytes, void *stream) {
+  HYQ_RANGE("hyq_prefill_attention");
   hyq_status s = hyq_check_cache(c);
   if (s != HYQ_OK) return s;
   if (!q || !k_full || !v_full || !o) return HYQ_ERR_INVALID;

@@ -603,16 +603,30 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const SelectArgs a) 
   float *fin = a.colsum + static_cast<int64_t>(u) * a.cap;
   const bool reduce = a.n_rb > 1 || fin != a.colsum_part + static_cast<int64_t>(u) * a.cap;
   const bool staged = n <= TOPK_SMEM_VALS;
-  for (int i = tid; i < n; i += blockDim.x) {
-    float v;
-    if (reduce) {
-      v = 0.f;
-      for (int z = 0; z < a.n_rb; ++z) v += a.colsum_part[(static_cast<int64_t>(z) * a.U + u) * a.cap + i];
-      fin[i] = v;
-    } else {
-      v = fin[i];
+  // the column sums, 8 loads in flight per thread
+  constexpr int LB = 8;
+  for (int i0 = tid; i0 < n; i0 += LB * static_cast<int>(blockDim.x)) {
+    float v[LB];
+#pragma unroll
+    for (int b = 0; b < LB; ++b) {
+      const int i = i0 + b * static_cast<int>(blockDim.x);
+      v[b] = 0.f;
+      if (i < n) {
+        if (reduce) {
+          for (int z = 0; z < a.n_rb; ++z) v[b] += __ldcg(a.colsum_part + (static_cast<int64_t>(z) * a.U + u) * a.cap + i);
+        } else {
+          v[b] = __ldcg(fin + i);
+        }
+      }
     }
-    if (staged) tk_smem[i] = __float_as_uint(v);
+#pragma unroll
+    for (int b = 0; b < LB; ++b) {
+      const int i = i0 + b * static_cast<int>(blockDim.x);
+      if (i < n) {
+        if (reduce) fin[i] = v[b];
+        if (staged) tk_smem[i] = __float_as_uint(v[b]);
+      }
+    }
   }
   if (tid == 0) s_ncand = 0;
   __syncthreads();
@@ -794,6 +808,7 @@ extern "C" hyq_status hyq_select_vl(const hyq_cache *c, const void *q_sel, int32
                                     int32_t q_is_ring, const void *k_full, int32_t k,
                                     int32_t *out_pos, float *out_colsum, void *ws, size_t ws_bytes,
                                     void *stream) {
+  HYQ_RANGE("hyq_select_vl");
   hyq_status st = hyq_check_cache(c);
   if (st != HYQ_OK) return st;
   if (!q_sel || (k > 0 && !out_pos)) return HYQ_ERR_INVALID;
