@@ -48,8 +48,11 @@
 
 namespace hyq {
 
-constexpr int NCW = 12;                   // compute warps per block (one block per SM), each fed by itself
-constexpr int NTHREADS = NCW * 32;
+// Compute warps per block (one block per SM, each warp fed by itself): 16
+// (at most 128 registers per thread) when the rings, the per-warp merge
+// buffers of G heads and the per-unit tables fit in shared memory, else 12
+// (168 registers).  The kernel is built for both; the host picks per launch.
+constexpr int NCW_WIDE = 16, NCW_NARROW = 12;
 constexpr int I4_TOK = 32;                // tokens per INT4 tile
 constexpr int F16_ROWS = 8;               // rows per FP16 tile
 constexpr int F16_ROW = D * 2;            // bytes of one FP16 K or V row
@@ -73,9 +76,10 @@ static_assert(SLOT_BYTES % 16 == 0, "slots stay 16-byte aligned");
 static_assert(I4_TOK == BLK_TOK, "an INT4 tile is one cache block");
 
 // Ring slots per compute warp: 2 (one being read, one in flight), so one
-// SM holds 24 tiles in flight, about 120 KB, enough to cover the memory
-// latency at full bandwidth while leaving shared memory for the merge
-// buffers and per-unit tables of up to 4096 units.
+// SM holds 24 or 32 tiles in flight (12 or 16 warps, about 120 or 160 KB),
+// enough to cover the memory latency at full bandwidth while leaving shared
+// memory for the merge buffers and per-unit tables (up to 4096 units with
+// 12 warps).
 #ifndef HYQ_DECODE_SPW
 #define HYQ_DECODE_SPW 2
 #endif
@@ -634,7 +638,7 @@ __device__ __forceinline__ Seg seg_from(const DecodeArgs &a, const Smem &sm, int
 // Log-sum-exp combine of the NCW per-warp states in shared memory (sm.mm,
 // sm.ml, sm.mo) for output element idx of [G][D]: returns the merged max,
 // sum and unnormalized output.
-template <int G>
+template <int G, int NCW>
 __device__ __forceinline__ void combine_warps(const Smem &sm, int idx, float &M, float &L, float &O) {
   const int h = idx / D, c = idx % D;
   M = -INFINITY;
@@ -658,10 +662,12 @@ __device__ __forceinline__ void combine_warps(const Smem &sm, int idx, float &M,
 // L2 per batch, most warps need one batch), merged online in registers, and
 // the NCW warp states are then combined through shared memory like the
 // warps of one block.
-template <int G>
+template <int G, int NCW>
 __device__ __forceinline__ void merge_parts(const DecodeArgs &a, const Smem &sm, int u, int n4, int n16,
                                             const Split &sp, int64_t hbase, int tid) {
-  constexpr int RB = (G >= 8) ? 1 : 16 / G;  // records per batch (bounded by registers)
+  constexpr int NTHREADS = NCW * 32;
+  // records per batch (bounded by registers: 168 per thread at 12 warps, 128 at 16)
+  constexpr int RB = (G >= 8) ? 1 : ((NCW > NCW_NARROW) ? 8 : 16) / G;
   const int warp = tid >> 5, lane = tid & 31;
   const int cs = sm.cost_start[u];
   const int c_lo = sp.of(sm, a.U, cs), c_hi = sp.of(sm, a.U, tile_cost(cs, n4, n4 + n16 - 1));
@@ -732,7 +738,7 @@ __device__ __forceinline__ void merge_parts(const DecodeArgs &a, const Smem &sm,
   named_bar_sync(1, NTHREADS);
   for (int idx = tid; idx < G * D; idx += NTHREADS) {
     float Mx, Lx, Ox;
-    combine_warps<G>(sm, idx, Mx, Lx, Ox);
+    combine_warps<G, NCW>(sm, idx, Mx, Lx, Ox);
     const int h = idx / D, c = idx % D;
     a.o[(hbase + h) * D + c] = __float2half_rn(Ox / Lx);
     if (c == 0 && a.lse) a.lse[hbase + h] = (Mx + __log2f(Lx)) * LN2;
@@ -751,7 +757,7 @@ __device__ __forceinline__ void merge_parts(const DecodeArgs &a, const Smem &sm,
 //    row from k_new / v_new (and writes the slot when T_old < W, where no
 //    row leaves the window);
 //  * the query goes to ring slot T_old % n_q, rows spread over the blocks;
-//  * seq_len = T_old + 1 is written by the last block to pass the prologue,
+//  * seq_len = T_old + 1 is written, as it ends, by the last block to pass the prologue,
 //    when every block has read the old lengths.
 __device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
@@ -817,8 +823,12 @@ __device__ __forceinline__ void step_new_row(const DecodeArgs &a, int u, int s_n
   __syncwarp();
 }
 
-// After the prologue (unit lengths in shared memory are T_old + 1).
-__device__ __forceinline__ void step_prologue(const DecodeArgs &a, const Smem &sm, int tid) {
+// After the prologue (unit lengths in shared memory are T_old + 1).  Thread
+// 0 counts the block in once every thread has read the lengths; the count
+// it gets back is only looked at when the block ends (step_epilogue), so the
+// round trip of the atomic overlaps the block's tiles.
+template <int NTHREADS>
+__device__ __forceinline__ int step_prologue(const DecodeArgs &a, const Smem &sm, int tid) {
   if (a.q_ring) {
     const int64_t items = static_cast<int64_t>(a.B) * a.Hq * 16;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * NTHREADS + tid; i < items;
@@ -831,8 +841,14 @@ __device__ __forceinline__ void step_prologue(const DecodeArgs &a, const Smem &s
           *reinterpret_cast<const uint4 *>(a.q + row * D + 8 * part);
     }
   }
-  if (tid == 0 && atomicAdd(a.grid_counter, 1) == a.n_ctas - 1) {
-    // every block has read seq_len (each increments after its prologue)
+  return (tid == 0) ? atomicAdd(a.grid_counter, 1) : -1;
+}
+
+// The block that was counted in last writes seq_len = T_old + 1: by then
+// every block has read the old lengths.  (The next launch on the stream
+// reads them only after this grid has completed.)
+__device__ __forceinline__ void step_epilogue(const DecodeArgs &a, const Smem &sm, int tid, int arrived) {
+  if (tid == 0 && arrived == a.n_ctas - 1) {
     for (int b = 0; b < a.B; ++b) {
       const int T = sm.unit_tv[b * a.Hkv].x;
       if (T >= 1 && T <= a.cap) a.seq_len[b] = T;
@@ -922,7 +938,7 @@ __device__ __forceinline__ void issue_tile(const DecodeArgs &a, const Smem &sm, 
 // split's block table).  Returns whether the split is aligned (the same in
 // every thread).  Status bits for malformed lengths are raised only when
 // `report` is set.
-template <int MODE>
+template <int MODE, int NTHREADS>
 __device__ __forceinline__ bool plan_units(const DecodeArgs &a, const Smem &sm, int tid, bool report) {
   const int U = a.U, warp = tid >> 5, lane = tid & 31;
   const int per = (U + NTHREADS - 1) / NTHREADS;
@@ -993,13 +1009,13 @@ __device__ __forceinline__ bool plan_units(const DecodeArgs &a, const Smem &sm, 
 // the status bits of malformed lengths.  `first` holds the raw lengths of
 // the thread's first unit, read by first_lengths before the first copies
 // were issued (so that read does not queue behind them).
-template <int MODE>
+template <int MODE, int NTHREADS>
 __device__ __forceinline__ int2 first_lengths(const DecodeArgs &a, int tid) {
   const int per = (a.U + NTHREADS - 1) / NTHREADS, beg = tid * per;
   return beg < a.U ? raw_lengths<MODE>(a, beg) : make_int2(0, 0);
 }
 
-template <int MODE>
+template <int MODE, int NTHREADS>
 __device__ __forceinline__ bool plan_stale(const DecodeArgs &a, const Smem &sm, int tid, int2 first) {
   const int U = a.U;
   const int per = (U + NTHREADS - 1) / NTHREADS;
@@ -1014,9 +1030,10 @@ __device__ __forceinline__ bool plan_stale(const DecodeArgs &a, const Smem &sm, 
   return __syncthreads_or(changed) != 0;
 }
 
-template <int G, int MODE>
-__global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a) {
+template <int G, int MODE, int NCW>
+__global__ void __launch_bounds__(NCW * 32, 1) decode_kernel(const DecodeArgs a) {
   constexpr int SPW = Ring<G>::SPW;
+  constexpr int NTHREADS = NCW * 32;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   Smem sm;
@@ -1058,7 +1075,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
   // Plan from the lengths as they stand, which the previous launch on the
   // stream may still be changing: the plan is made while that launch drains
   // and only checked after the wait.
-  bool aligned = plan_units<MODE>(a, sm, tid, false);
+  bool aligned = plan_units<MODE, NTHREADS>(a, sm, tid, false);
   pdl_wait();  // earlier work on the stream (an append) is complete and visible
 
   const int cta = blockIdx.x;
@@ -1091,16 +1108,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
   // read again meanwhile (loads issued ahead of the copies).  If they changed
   // (the previous launch appended to this cache), those copies land unused
   // and the block plans again.
-  const int2 first = first_lengths<MODE>(a, tid);
+  const int2 first = first_lengths<MODE, NTHREADS>(a, tid);
   for (int k = 0; k < SPW; ++k) issue_next();
-  if (plan_stale<MODE>(a, sm, tid, first)) {
+  if (plan_stale<MODE, NTHREADS>(a, sm, tid, first)) {
     for (; k_done < k_issued; ++k_done) {
       const bool ok = first_fail < 0 &&
                       mbar_wait_bounded(my_bars + (k_done % SPW) * 8, (k_done / SPW) & 1, abort_flag, a.status,
                                         tile_wait_limit());
       if (!__all_sync(0xffffffffu, ok) && first_fail < 0) first_fail = k_done;
     }
-    aligned = plan_units<MODE>(a, sm, tid, false);
+    aligned = plan_units<MODE, NTHREADS>(a, sm, tid, false);
     sp = Split(sm.cost_start[U], a.n_ctas, aligned);
     lo = sp.lo(sm, U, cta);
     hi = sp.lo(sm, U, cta + 1);
@@ -1110,7 +1127,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
     ic = seg_from<MODE>(a, sm, u_first, 0, lo, hi);
     for (int k = 0; k < SPW; ++k) issue_next();
   }
-  if (MODE == MODE_STEP) step_prologue(a, sm, tid);
+  const int arrived = (MODE == MODE_STEP) ? step_prologue<NTHREADS>(a, sm, tid) : -1;
 
   WarpState st;
   for (Seg sg = seg_from<MODE>(a, sm, u_first, 0, lo, hi); sg.u < U;
@@ -1218,7 +1235,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
     for (int idx = tid; idx < G * D; idx += NTHREADS) {
       const int h = idx / D, c = idx % D;
       float M, L, O;
-      combine_warps<G>(sm, idx, M, L, O);
+      combine_warps<G, NCW>(sm, idx, M, L, O);
       if (complete) {
         a.o[(hbase + h) * D + c] = __float2half_rn(O / L);
         if (c == 0 && a.lse) a.lse[hbase + h] = (M + __log2f(L)) * LN2;
@@ -1249,7 +1266,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
       }
       named_bar_sync(1, NTHREADS);
       if (*sm.last_flag) {
-        merge_parts<G>(a, sm, u, us.n4, us.nv + us.nw, sp, hbase, tid);
+        merge_parts<G, NCW>(a, sm, u, us.n4, us.nv + us.nw, sp, hbase, tid);
         if (tid == 0) a.counters[u] = 0;
       }
     }
@@ -1259,6 +1276,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
   // copies still in flight (only after an abort): let them land before exit
   for (int kk = (first_fail >= 0 ? first_fail : k_done); kk < k_issued; ++kk)
     mbar_drain(my_bars + (kk % SPW) * 8, (kk / SPW) & 1, 500000000ull);
+  if (MODE == MODE_STEP) step_epilogue(a, sm, tid, arrived);
 
   // units without any position: o = 0, lse = -inf (one block each)
   for (int u = cta; u < U; u += a.n_ctas) {
@@ -1273,13 +1291,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) decode_kernel(const DecodeArgs a)
 }
 
 // ---------------------------------------------------------------- host side
-static size_t decode_smem_bytes(int G, int U) {
+constexpr size_t DECODE_SMEM_MAX = 227 * 1024;
+
+static size_t decode_smem_bytes(int G, int U, int ncw) {
   const int spw = Ring<1>::SPW;
   static_assert(Ring<1>::SPW == Ring<8>::SPW, "one ring depth for every G");
-  return static_cast<size_t>(NCW) * spw * SLOT_BYTES + NCW * spw * 8 + 16 + NCW * 8 * 4 * 2 +
-         static_cast<size_t>(NCW) * G * D * 4 + NTHREADS * 4 + BLK_TABLE_BYTES +
+  return static_cast<size_t>(ncw) * spw * SLOT_BYTES + ncw * spw * 8 + 16 + ncw * 8 * 4 * 2 +
+         static_cast<size_t>(ncw) * G * D * 4 + ncw * 32 * 4 + BLK_TABLE_BYTES +
          (static_cast<size_t>(U + 1) * 4 + 15) / 16 * 16 +
          static_cast<size_t>(U) * 8;
+}
+
+// 16 compute warps for launches with many tiles per block (at least
+// WIDE_MIN_TILES quantized-tile slots of capacity per block: batched or long
+// contexts, where the INT4 tile arithmetic sets the pace and more warps hide
+// its latency), when their shared memory fits (G <= 4 and, at G = 4, up to
+// about 2300 units); 12 otherwise (few tiles per warp, where the block's
+// fixed costs set the pace and 168 registers per thread serve better).
+constexpr int64_t WIDE_MIN_TILES = 128;
+static int decode_ncw(int G, int U, int cap, int n_ctas) {
+  if (G >= 8 || decode_smem_bytes(G, U, NCW_WIDE) > DECODE_SMEM_MAX) return NCW_NARROW;
+  return static_cast<int64_t>(U) * (cap / I4_TOK) >= WIDE_MIN_TILES * n_ctas ? NCW_WIDE : NCW_NARROW;
 }
 
 static size_t decode_ws_bytes(int G, int U, int n_ctas) {
@@ -1287,28 +1319,38 @@ static size_t decode_ws_bytes(int G, int U, int n_ctas) {
   return cnt + static_cast<size_t>(n_ctas) * 2 * G * PART_STRIDE * 4;
 }
 
-template <int G, int MODE>
+template <int G, int MODE, int NCW>
 static cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
-  const size_t smem = decode_smem_bytes(G, a.U);
+  const size_t smem = decode_smem_bytes(G, a.U, NCW);
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<G, MODE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<G, MODE, NCW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(DECODE_SMEM_MAX));
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  return launch(decode_kernel<G, MODE>, dim3(a.n_ctas), dim3(NTHREADS), smem, s, a);
+  return launch(decode_kernel<G, MODE, NCW>, dim3(a.n_ctas), dim3(NCW * 32), smem, s, a);
+}
+
+template <int G, int MODE>
+static cudaError_t launch_decode_g(const DecodeArgs &a, cudaStream_t s) {
+  if constexpr (G >= 8) {
+    return launch_decode<G, MODE, NCW_NARROW>(a, s);
+  } else {
+    return decode_ncw(G, a.U, a.cap, a.n_ctas) == NCW_WIDE ? launch_decode<G, MODE, NCW_WIDE>(a, s)
+                                                           : launch_decode<G, MODE, NCW_NARROW>(a, s);
+  }
 }
 
 template <int MODE>
 static cudaError_t dispatch_decode(int G, const DecodeArgs &a, cudaStream_t s) {
   switch (G) {
-    case 1: return launch_decode<1, MODE>(a, s);
-    case 2: return launch_decode<2, MODE>(a, s);
-    case 4: return launch_decode<4, MODE>(a, s);
-    case 8: return launch_decode<8, MODE>(a, s);
+    case 1: return launch_decode_g<1, MODE>(a, s);
+    case 2: return launch_decode_g<2, MODE>(a, s);
+    case 4: return launch_decode_g<4, MODE>(a, s);
+    case 8: return launch_decode_g<8, MODE>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }

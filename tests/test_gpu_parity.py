@@ -109,6 +109,25 @@ def test_decode_small_shapes(B, Hq, Hkv, T, k, n_ctas):
     assert case.g.status() == 0
 
 
+@pytest.mark.parametrize("B,n_ctas", [(250, 7), (300, 7), (250, 0), (300, 1000)])
+def test_decode_many_units_both_block_widths(B, n_ctas):
+    """G = 4 with many short units.  2000 units on 7 blocks take the 16-warp
+    build (many tiles per block, shared memory fits); 2400 units do not fit
+    beside 16 warps' tile rings and take the 12-warp build, as do 2000 units
+    on 148 blocks (few tiles per block).  Sampled units (first, last, and
+    units inside) against the oracle, plus a bit-exact cache check on them."""
+    cfg = synth.custom(B, 32, 8, 200, 8, seed=4000 + B)
+    U = cfg.units
+    units = [0, 1, U // 3, U // 2 + 5, U - 2, U - 1]
+    case = Case(cfg, oracle_units=units)
+    q = synth.q(cfg)
+    og, lg = case.decode_gpu(q, n_ctas)
+    oo, lo = oracle.decode(case.o, q, units=units)
+    compare_decode(og, lg, oo, lo, heads=case.heads_of(units))
+    _assert_cache_equal(case, units)
+    assert case.g.status() == 0
+
+
 def test_decode_config1_full():
     cfg = synth.config(1)
     case = Case(cfg)
