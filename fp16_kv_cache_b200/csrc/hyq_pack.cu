@@ -12,8 +12,6 @@
 // give one.
 //
 // One row of 128 channels is handled by 16 threads (hyq_quant.cuh).
-#include <algorithm>
-
 #include "hyq_common.cuh"
 #include "hyq_quant.cuh"
 
@@ -46,21 +44,39 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half *__restrict__ x,
   quantize_part(xv, t, hmask, codes + dst * ROW_BYTES, sz + dst * (SZ_BYTES / 4), status);
 }
 
-// Prefill: row r = 2 (unit * capacity + position) + (0: K, 1: V) of the
-// prompt goes to one 16-thread group.  Each group takes PF_ROWS rows spaced
-// by the number of groups in the grid and issues their loads together before
-// quantizing any of them, so that a thread keeps PF_ROWS x 16 bytes in flight
-// and the division chains of the rows overlap; the grid is sized to the SMs.
-constexpr int PF_ROWS = 4;
-
-__device__ __forceinline__ void prefill_row(const hyq_cache &c, int64_t row, int T, uint4 xv, int t,
-                                            unsigned hmask) {
+// Prefill: one 16-thread group per (unit, position, K|V) row of the prompt.
+__global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half *__restrict__ k_full,
+                                                      const __half *__restrict__ v_full,
+                                                      int64_t n_rows) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream is complete and visible
+  const int lane = threadIdx.x & 31;
+  const int t = lane & 15;
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+  if (row >= n_rows) return;
   const bool is_v = row & 1;
   const int64_t up = row >> 1;  // unit * capacity + position
   const int p = static_cast<int>(up % c.capacity);
   const int64_t u = up / c.capacity;
+  const int b = static_cast<int>(u / c.n_kv_heads);
+  const int T = c.seq_len[b];
+  if (T < 0 || T > c.capacity) {
+    if (p == 0 && t == 0 && !is_v && (u % c.n_kv_heads) == 0) set_status(c.dev_status, HYQ_DEV_BADLEN);
+    return;
+  }
+  // clear this unit's vertical-line set (the bitmask words of the records
+  // holding its positions, and the count)
+  if (!is_v && t == 0 && p == 0) c.vl_count[u] = 0;
+  if (p >= T) return;
+  if (!is_v && t == 0 && (p % BLK_TOK) == 0) {
+    uint32_t *m = mask_of(c, u, p);
+    if (m) *m = 0u;
+  }
+  const __half *src = (is_v ? v_full : k_full) + up * D;
+  const uint4 xv = *reinterpret_cast<const uint4 *>(src + 8 * t);
   const int W = c.window;
   if (p < T - W) {
+    const unsigned hmask = 0xFFFFu << (lane & 16);
     const int64_t rec = recmap(c).rec(u, p);
     if (rec >= 0)  // uniform over the row's 16 lanes
       quantize_part(xv, t, hmask, c.blocks + (is_v ? rec_vcode(rec, p) : rec_kcode(rec, p)),
@@ -72,50 +88,6 @@ __device__ __forceinline__ void prefill_row(const hyq_cache &c, int64_t row, int
   } else {
     __half *win = reinterpret_cast<__half *>(is_v ? c.win_v : c.win_k) + (u * W + p % W) * D;
     *reinterpret_cast<uint4 *>(win + 8 * t) = xv;
-  }
-}
-
-__global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half *__restrict__ k_full,
-                                                      const __half *__restrict__ v_full,
-                                                      int64_t n_rows) {
-  pdl_trigger();  // the next kernel may be scheduled
-  pdl_wait();     // earlier work on the stream is complete and visible
-  const int lane = threadIdx.x & 31;
-  const int t = lane & 15;
-  const unsigned hmask = 0xFFFFu << (lane & 16);
-  const int64_t n_groups = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
-  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4; base < n_rows;
-       base += PF_ROWS * n_groups) {
-    uint4 xv[PF_ROWS];
-    int T[PF_ROWS];
-#pragma unroll
-    for (int k = 0; k < PF_ROWS; ++k) {
-      const int64_t row = base + k * n_groups;
-      T[k] = -1;  // -1: nothing to load (past the rows, past the prompt, or a bad length)
-      if (row >= n_rows) continue;
-      const bool is_v = row & 1;
-      const int64_t up = row >> 1;
-      const int p = static_cast<int>(up % c.capacity);
-      const int64_t u = up / c.capacity;
-      const int Tb = c.seq_len[u / c.n_kv_heads];
-      if (Tb < 0 || Tb > c.capacity) {
-        if (p == 0 && t == 0 && !is_v && (u % c.n_kv_heads) == 0) set_status(c.dev_status, HYQ_DEV_BADLEN);
-        continue;
-      }
-      // clear this unit's vertical-line set (the bitmask words of the records
-      // holding its positions, and the count)
-      if (!is_v && t == 0 && p == 0) c.vl_count[u] = 0;
-      if (p >= Tb) continue;
-      if (!is_v && t == 0 && (p % BLK_TOK) == 0) {
-        uint32_t *m = mask_of(c, u, p);
-        if (m) *m = 0u;
-      }
-      T[k] = Tb;
-      xv[k] = __ldg(reinterpret_cast<const uint4 *>((is_v ? v_full : k_full) + up * D + 8 * t));
-    }
-#pragma unroll
-    for (int k = 0; k < PF_ROWS; ++k)
-      if (T[k] >= 0) prefill_row(c, base + k * n_groups, T[k], xv[k], t, hmask);
   }
 }
 
@@ -374,7 +346,6 @@ using namespace hyq;
 static inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 extern "C" hyq_status hyq_check_cache(const hyq_cache *c);  // hyq_api.cu
-extern "C" int32_t hyq_sm_count(void);                      // hyq_api.cu
 
 extern "C" hyq_status hyq_pack(const void *x, int64_t n_rows, int64_t row_stride,
                                const int64_t *dst_rows, uint8_t *codes, void *sz,
@@ -402,13 +373,8 @@ extern "C" hyq_status hyq_prefill(const hyq_cache *c, const void *k_full, const 
   if (!k_full || !v_full) return HYQ_ERR_INVALID;
   if (!aligned16(k_full) || !aligned16(v_full)) return HYQ_ERR_ALIGN;
   const int64_t n_rows = static_cast<int64_t>(c->batch) * c->n_kv_heads * c->capacity * 2;
-  // one wave of resident blocks (fewer for small prompts)
-  static int per_sm = 0;
-  if (per_sm == 0 && cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefill_kernel, 256, 0) != cudaSuccess)
-    return HYQ_ERR_CUDA;
-  const int64_t want = (n_rows * 16 + 255) / 256;
-  const int64_t blocks = std::min<int64_t>(want, static_cast<int64_t>(hyq_sm_count()) * std::max(per_sm, 1));
-  if (blocks <= 0) return HYQ_OK;
+  const int64_t blocks = (n_rows * 16 + 255) / 256;
+  if (blocks > 0x7FFFFFFFll) return HYQ_ERR_INVALID;
   const cudaError_t e = launch(prefill_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
                                 static_cast<cudaStream_t>(stream), *c, static_cast<const __half *>(k_full),
                                 static_cast<const __half *>(v_full), n_rows);
