@@ -27,9 +27,12 @@
 //      keys, P = exp2(S - m_r) / l_r, each thread sums one key column over
 //      the rows in a fixed order (no float atomics), so equal key columns
 //      give bitwise-equal sums.
-//   4. topk_kernel       grid (units): exact radix select on the fp32 bit
-//      patterns (non-negative floats order like their bits), ties to lower
-//      positions, output compacted in ascending position order.
+//   4. topk_cluster_kernel  one cluster of 8 blocks per unit (each block a
+//      slice of the positions): exact radix select on the fp32 bit patterns
+//      (non-negative floats order like their bits), histograms and counts
+//      combined through distributed shared memory, ties to lower positions,
+//      output compacted in ascending position order; topk_kernel (one block
+//      per unit) does the same when a slice would not fit shared memory.
 // Keys come from k_full (prefill) or from the cache as decode sees it: FP16
 // window and vertical-line rows, and INT4 rows dequantized as
 // zero + code * scale in fp32 and split into two fp16 terms hi + lo (both
@@ -73,7 +76,7 @@ __device__ __forceinline__ int sel_T(const SelectArgs &a, int u) { return a.seq_
 
 // ---------------------------------------------------------------- scorer
 // S = Q K^T on the 5th-generation tensor cores (tcgen05, fp16 in, fp32
-// accumulate in tensor memory).  One block of 8 warps per SM walks the
+// accumulate in tensor memory).  One block of 16 warps per SM walks the
 // (unit, 512-key chunk) items.  Per unit the R query rows sit in shared
 // memory as row blocks of 128 (the MMA's M); per sub-tile of 128 keys (the
 // MMA's N) the keys are written to shared memory as fp16 -- in cache mode an
@@ -747,6 +750,276 @@ __global__ void __launch_bounds__(TOPK_THREADS) topk_kernel(const SelectArgs a) 
   }
 }
 
+// The same selection with the column sums of one unit spread over the TKC
+// blocks of a thread-block cluster (used while every block's share fits in
+// its shared memory; topk_kernel above serves longer contexts).  Block r
+// stages positions [r S, r S + S), S = n / TKC rounded up to a multiple of
+// 32.  In each radix pass a block counts its own values (or, after the first
+// byte, its own candidates) into a 256-bin histogram; after a cluster
+// barrier every block adds the TKC histograms through distributed shared
+// memory and picks the same digit.  At the end each block counts its values
+// above tau and equal to it, reads the counts of the blocks before it, and
+// writes its selected positions at their place in the ascending output; the
+// positions equal to tau are taken lowest first across the whole unit.
+constexpr int TKC = 8;                // blocks per unit: one cluster (the portable maximum size)
+constexpr int TKC_THREADS = 512;
+constexpr int TKC_WARPS = TKC_THREADS / 32;
+constexpr int TKC_MAX_VALS = 32768;   // values per block (block-local positions fit uint16)
+
+__device__ __forceinline__ int cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return static_cast<int>(r);
+}
+__device__ __forceinline__ int cluster_index() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return static_cast<int>(r);
+}
+// Every thread of every block of the cluster arrives; shared-memory writes
+// before it are visible to the cluster's reads after it.
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Read an int at the same shared-memory offset in block `rank` of the cluster.
+__device__ __forceinline__ int ld_cluster_s32(const int *p, int rank) {
+  uint32_t remote;
+  int v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(rank));
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(TKC_THREADS) topk_cluster_kernel(const SelectArgs a) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // earlier work on the stream is complete and visible
+  extern __shared__ uint32_t tkc_smem[];  // [S] values, then [S] uint16 block-local candidate positions
+  __shared__ int whist[TKC_WARPS][256];
+  __shared__ int bhist[2][256];  // this block's histogram of the even / odd passes (read by the cluster)
+  __shared__ int ghist[256];     // the cluster's histogram of the pass
+  __shared__ int bcnt[2];        // this block's values above tau and equal to it (read by later blocks)
+  __shared__ int wcnt[TKC_WARPS][2];
+  __shared__ int s_digit, s_need, s_ncand, s_gt_before, s_eq_before;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int r = cluster_rank(), u = cluster_index();
+  const int T = sel_T(a, u);
+  const int k = a.k;
+  int32_t *out = a.out_pos + static_cast<int64_t>(u) * k;
+  if (T < a.n_q || T > a.cap || T - a.W < k) {  // the same decision in every block of the cluster
+    if (r == 0) {
+      if (tid == 0) set_status(a.status, HYQ_DEV_BADLEN);
+      for (int i = tid; i < k; i += TKC_THREADS) out[i] = -1;
+    }
+    return;
+  }
+  const int n = T - a.W;
+  const int S = ((n + TKC - 1) / TKC + 31) / 32 * 32;
+  const int beg = min(n, r * S), m = min(n, beg + S) - beg;  // this block's positions [beg, beg + m)
+  float *fin = a.colsum + static_cast<int64_t>(u) * a.cap;
+  const bool reduce = a.n_rb > 1 || fin != a.colsum_part + static_cast<int64_t>(u) * a.cap;
+  uint32_t *vals = tkc_smem;
+  uint16_t *cand = reinterpret_cast<uint16_t *>(tkc_smem + S);
+  constexpr int LB = 8;  // loads in flight per thread
+  for (int i0 = tid; i0 < m; i0 += LB * TKC_THREADS) {
+    float v[LB];
+#pragma unroll
+    for (int b = 0; b < LB; ++b) {
+      const int i = i0 + b * TKC_THREADS;
+      v[b] = 0.f;
+      if (i < m) {
+        if (reduce) {
+          for (int z = 0; z < a.n_rb; ++z)
+            v[b] += __ldcg(a.colsum_part + (static_cast<int64_t>(z) * a.U + u) * a.cap + beg + i);
+        } else {
+          v[b] = __ldcg(fin + beg + i);
+        }
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < LB; ++b) {
+      const int i = i0 + b * TKC_THREADS;
+      if (i < m) {
+        if (reduce) fin[beg + i] = v[b];
+        vals[i] = __float_as_uint(v[b]);
+      }
+    }
+  }
+  if (tid == 0) s_ncand = 0;
+  __syncthreads();
+  if (k == 0) return;  // k is the same for every block: no block waits at a cluster barrier
+
+  uint32_t prefix = 0, mask = 0;
+  int need = k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = lane; i < 256; i += 32) whist[w][i] = 0;
+    __syncwarp();
+    const int mc = pass > 0 ? s_ncand : m;
+    for (int base = 0; base < mc; base += TKC_THREADS) {  // whole warps iterate together
+      const int j = base + tid;
+      uint32_t b = 0;
+      bool act = false;
+      if (j < mc) {
+        b = vals[pass > 0 ? cand[j] : j];
+        act = (b & mask) == prefix;
+      }
+      const unsigned am = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const uint32_t bin = (b >> shift) & 255u;
+        const unsigned peers = __match_any_sync(am, bin);
+        if (lane == __ffs(peers) - 1) atomicAdd(&whist[w][bin], __popc(peers));
+      }
+    }
+    __syncthreads();
+    if (tid < 256) {
+      int c = 0;
+#pragma unroll
+      for (int q = 0; q < TKC_WARPS; ++q) c += whist[q][tid];
+      bhist[pass & 1][tid] = c;
+    }
+    // Every block's histogram of this pass is complete.  (A block rewrites
+    // bhist[pass & 1] two passes later, after the next barrier, which no
+    // block reaches before it has read this pass's histograms.)
+    cluster_barrier();
+    if (tid < 256) {
+      int c = 0;
+#pragma unroll
+      for (int q = 0; q < TKC; ++q) c += ld_cluster_s32(&bhist[pass & 1][tid], q);
+      ghist[tid] = c;
+    }
+    __syncthreads();
+    if (w == 0) {
+      // suffix counts over bins 255 .. 0: lane l holds bins 255 - 8l .. 248 - 8l
+      int h[8], sum = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        h[e] = ghist[255 - 8 * lane - e];
+        sum += h[e];
+      }
+      int x = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      int run = x - sum;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (run < need && run + h[e] >= need) {
+          s_digit = 255 - 8 * lane - e;
+          s_need = need - run;
+        }
+        run += h[e];
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(s_digit) << shift;
+    mask |= 255u << shift;
+    need = s_need;
+    if (pass == 0) {
+      // this block's candidates for the lower bytes
+      for (int base = 0; base < m; base += TKC_THREADS) {
+        const int j = base + tid;
+        const bool c = j < m && (vals[j] & mask) == prefix;
+        const unsigned bal = __ballot_sync(0xffffffffu, c);
+        int slot0 = 0;
+        if (lane == 0 && bal) slot0 = atomicAdd(&s_ncand, __popc(bal));
+        slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+        if (c) cand[slot0 + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(j);
+      }
+    }
+    __syncthreads();  // s_digit, s_need, s_ncand, whist and ghist are reused
+  }
+  // tau = prefix: take every value > tau and the first `need` values == tau
+  // of the unit.  Warp w of this block owns block-local positions
+  // [w * per, (w + 1) * per).
+  const uint32_t tau = prefix;
+  const int per = ((m + TKC_WARPS - 1) / TKC_WARPS + 31) / 32 * 32;
+  const int wb = min(m, w * per), we = min(m, wb + per);
+  int n_gt = 0, n_eq = 0;
+  for (int j = wb + lane; j < wb + per; j += 32) {  // per is a multiple of 32: whole warps iterate
+    const bool in = j < we;
+    const uint32_t b = in ? vals[j] : 0u;
+    n_gt += __popc(__ballot_sync(0xffffffffu, in && b > tau));
+    n_eq += __popc(__ballot_sync(0xffffffffu, in && b == tau));
+  }
+  if (lane == 0) {
+    wcnt[w][0] = n_gt;
+    wcnt[w][1] = n_eq;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int g = 0, e = 0;
+    for (int q = 0; q < TKC_WARPS; ++q) {
+      g += wcnt[q][0];
+      e += wcnt[q][1];
+    }
+    bcnt[0] = g;
+    bcnt[1] = e;
+  }
+  cluster_barrier();  // every block's counts are complete
+  if (tid == 0) {
+    int g = 0, e = 0;
+    for (int q = 0; q < r; ++q) {
+      g += ld_cluster_s32(&bcnt[0], q);
+      e += ld_cluster_s32(&bcnt[1], q);
+    }
+    s_gt_before = g;
+    s_eq_before = e;
+  }
+  __syncthreads();
+  int gt_before = s_gt_before, eq_before = s_eq_before;
+  for (int q = 0; q < w; ++q) {
+    gt_before += wcnt[q][0];
+    eq_before += wcnt[q][1];
+  }
+  const int take_eq_before = min(eq_before, need);  // equal values taken before this warp's positions
+  int o = gt_before + take_eq_before, eq_seen = eq_before;
+  for (int j = wb + lane; j < wb + per; j += 32) {
+    const bool in = j < we;
+    const uint32_t b = in ? vals[j] : 0u;
+    const bool gt = in && b > tau, eq = in && b == tau;
+    const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+    const bool take = gt || (eq && eq_seen + __popc(eqb & ((1u << lane) - 1u)) < need);
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    const int pos = o + __popc(tb & ((1u << lane) - 1u));
+    if (take && pos < k) out[pos] = beg + j;
+    o += __popc(tb);
+    eq_seen += __popc(eqb);
+  }
+  cluster_barrier();  // no block leaves while another may still read its shared memory
+}
+
+// Values per block of the cluster top-k for a cache, or 0 when topk_kernel
+// (one block per unit) is used instead: when a block's share would not fit
+// its shared memory, or when the clusters would fill more than two waves of
+// the SMs (many units: one block per unit already spreads over the GPU, and
+// measured faster at 128 units).
+static int topk_cluster_vals(const SelectArgs &a, int sms) {
+  const int n_max = a.cap - a.W;
+  const int S = ((n_max + TKC - 1) / TKC + 31) / 32 * 32;
+  if (S > TKC_MAX_VALS || static_cast<int64_t>(a.U) * TKC > 2 * static_cast<int64_t>(sms)) return 0;
+  return std::max(S, 32);
+}
+
+static cudaError_t launch_topk_cluster(const SelectArgs &a, int S, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.U * TKC));
+  cfg.blockDim = dim3(TKC_THREADS);
+  cfg.dynamicSmemBytes = static_cast<size_t>(S) * (sizeof(uint32_t) + sizeof(uint16_t));
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = TKC;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, a);
+}
+
 static size_t score_smem_bytes(int R, bool cache) {
   const int n_rbt = (R + 127) / 128;
   const int nbuf = (n_rbt <= 2) ? 2 : 1;
@@ -767,6 +1040,8 @@ static cudaError_t select_launch(const SelectArgs &a, bool cache, cudaStream_t s
     cudaFuncSetAttribute(score_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx);
     cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          static_cast<int>(TOPK_SMEM_VALS * (sizeof(uint32_t) + sizeof(uint16_t))));
+    cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(TKC_MAX_VALS * (sizeof(uint32_t) + sizeof(uint16_t))));
     attr_dev = dev;
   }
   const int n_items = a.U * a.n_chunks;
@@ -781,7 +1056,11 @@ static cudaError_t select_launch(const SelectArgs &a, bool cache, cudaStream_t s
   }
   if (e == cudaSuccess) e = launch(stats_merge_kernel, dim3(a.U), dim3(256), 0, s, a);
   if (e == cudaSuccess) e = launch(cache ? score_kernel<true, 2> : score_kernel<false, 2>, grid, dim3(TC_THREADS), smem, s, a);
-  if (e == cudaSuccess) e = launch(topk_kernel, dim3(a.U), dim3(TOPK_THREADS), TOPK_SMEM_VALS * (sizeof(uint32_t) + sizeof(uint16_t)), s, a);
+  const int tkc_vals = topk_cluster_vals(a, sms);
+  if (e == cudaSuccess)
+    e = tkc_vals > 0 ? launch_topk_cluster(a, tkc_vals, s)
+                     : launch(topk_kernel, dim3(a.U), dim3(TOPK_THREADS),
+                              TOPK_SMEM_VALS * (sizeof(uint32_t) + sizeof(uint16_t)), s, a);
   return e;
 }
 

@@ -314,15 +314,28 @@ def test_vl_apply_cache_mode_matches_oracle():
     compare_decode(og, lg, oo, lo)
 
 
-def test_select_long_context_global_path():
-    """More candidates than the top-k stages in shared memory (n > 32768):
-    the radix passes read the column sums from global memory."""
+def test_select_long_context_cluster_path():
+    """More candidates than one block stages (n > 32768): the top-k spreads
+    them over the 8 blocks of a cluster and merges its histograms and
+    counts through distributed shared memory."""
     cfg = synth.custom(1, 8, 2, 40000, 100, seed=41)
     case = Case(cfg)
     qs = synth.qsel(cfg, 0)[None]
     pos_g, cs_g = _select_gpu(case, dev(qs), cfg.k, k_full=case.Kd)
     pos_o, cs_o, margin = oracle.select_vl(case.o, qs, cfg.k, k_full=case.K)
     _check_selection(pos_g, cs_g, pos_o, cs_o, margin, cfg.T, 128, [(0, 0), (0, 1)])
+
+
+def test_select_very_long_context_single_block_path():
+    """n > 8 x 32768 candidates: more than the cluster's blocks stage, so one
+    block per unit runs the radix passes over the column sums in global
+    memory."""
+    cfg = synth.custom(1, 2, 1, 262400, 60, seed=43)
+    case = Case(cfg)
+    qs = synth.qsel(cfg, 0)[None]
+    pos_g, cs_g = _select_gpu(case, dev(qs), cfg.k, k_full=case.Kd)
+    pos_o, cs_o, margin = oracle.select_vl(case.o, qs, cfg.k, k_full=case.K)
+    _check_selection(pos_g, cs_g, pos_o, cs_o, margin, cfg.T, 128, [(0, 0)])
 
 
 @pytest.mark.parametrize("k", [1, 50, 472])
