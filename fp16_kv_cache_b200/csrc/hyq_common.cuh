@@ -78,7 +78,19 @@ struct RecMap {
 };
 __host__ __device__ __forceinline__ int64_t rec_kcode(int64_t rec, int64_t p) { return rec + HYQ_BLK_KCODES + (p % BLK_TOK) * ROW_BYTES; }
 __host__ __device__ __forceinline__ int64_t rec_ksz(int64_t rec, int64_t p) { return rec + HYQ_BLK_KSZ + (p % BLK_TOK) * SZ_BYTES; }
-__host__ __device__ __forceinline__ int64_t rec_vcode(int64_t rec, int64_t p) { return rec + HYQ_BLK_VCODES + (p % BLK_TOK) * ROW_BYTES; }
+__host__ __device__ __forceinline__ int64_t rec_vcodes(int64_t rec) { return rec + HYQ_BLK_VCODES; }
+// V codes are stored in position pairs (include/hyq.h): the byte offset,
+// inside a record's V code area, of the low 16 bits of word h of piece
+// `piece` of slot t; the high 16 bits are 4 bytes further.  The pair
+// {2i, 2i + 1} shares each 32-bit word, in the order the decode's P.V
+// operand wants: (2i, 2i + 1) when i % 4 < 2, else (2i + 1, 2i).  Pair i
+// keeps piece p in its 16-byte unit p xor 2 (i mod 4), so the 8 lanes of a
+// 16-byte shared-memory load phase (pieces r, r + 1 of four pairs) fall in
+// 8 different bank groups.
+__host__ __device__ __forceinline__ int vcode_unit(int pair, int piece) { return piece ^ ((pair & 3) << 1); }
+__host__ __device__ __forceinline__ int vcode_off(int t, int piece, int h) {
+  return (t >> 1) * 128 + vcode_unit(t >> 1, piece) * 16 + h * 8 + (((t & 1) ^ ((t >> 2) & 1)) << 1);
+}
 __host__ __device__ __forceinline__ int64_t rec_vsz(int64_t rec, int64_t p) { return rec + HYQ_BLK_VSZ + (p % BLK_TOK) * SZ_BYTES; }
 __host__ __device__ __forceinline__ int64_t rec_mask(int64_t rec) { return rec + HYQ_BLK_MASK; }
 

@@ -465,17 +465,16 @@ __device__ __forceinline__ void int4_tile(WarpState &st, uint32_t slot, int n_va
       bq[g][0] = movmatrix_t(h2u(__hmul2(u2h(pa2), u2h(sa2))));
       bq[g][1] = movmatrix_t(h2u(__hmul2(u2h(pb2), u2h(sb2))));
     }
-    const uint32_t vrow = vc + 8 * r;
-    const uint2 x0 = lds64(vrow + (16 * mt + s2q) * ROW_BYTES);
-    const uint2 x1 = lds64(vrow + (16 * mt + s2q1) * ROW_BYTES);
-    const uint2 y0 = lds64(vrow + (16 * mt + s2q + 8) * ROW_BYTES);
-    const uint2 y1 = lds64(vrow + (16 * mt + s2q1 + 8) * ROW_BYTES);
+    // piece r of the position pairs (s2q, s2q1) and (s2q + 8, s2q1 + 8):
+    // the records store each pair's words interleaved by 16 bits, so one
+    // 16-byte load gives the A operands of both words (vcode_off)
+    const int pr = (16 * mt + s2q) >> 1;  // pair index; the +8 pair is pr + 4 (same unit swizzle)
+    const uint4 x = lds128(vc + pr * 128 + 16 * vcode_unit(pr, r));
+    const uint4 y = lds128(vc + (pr + 4) * 128 + 16 * vcode_unit(pr, r));
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      const uint32_t A0 = hh ? x0.y : x0.x, A1 = hh ? x1.y : x1.x;
-      const uint32_t B0 = hh ? y0.y : y0.x, B1 = hh ? y1.y : y1.x;
-      const uint32_t xa = prmt(A0, A1, 0x5410u), ya = prmt(A0, A1, 0x7632u);
-      const uint32_t xb = prmt(B0, B1, 0x5410u), yb = prmt(B0, B1, 0x7632u);
+      const uint32_t xa = hh ? x.z : x.x, ya = hh ? x.w : x.y;
+      const uint32_t xb = hh ? y.z : y.x, yb = hh ? y.w : y.y;
       const int g0 = 2 * hh, g1 = 2 * hh + 1;
       // rows r take low nibbles (2^-24 O), rows r + 8 high nibbles (2^-20 O)
       mma16816(st.acc[g0][0], code_lo(xa), code_hi(xa), code_lo(xb), code_hi(xb), bq[g0][0], bq[g0][1]);
@@ -759,6 +758,9 @@ __device__ __forceinline__ void merge_parts(const DecodeArgs &a, const Smem &sm,
 //  * the query goes to ring slot T_old % n_q, rows spread over the blocks;
 //  * seq_len = T_old + 1 is written, as it ends, by the last block to pass the prologue,
 //    when every block has read the old lengths.
+__device__ __forceinline__ void sts16(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(static_cast<unsigned short>(v)) : "memory");
+}
 __device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
@@ -780,18 +782,28 @@ __device__ __forceinline__ void step_exit_row(const DecodeArgs &a, int u, int T_
     *reinterpret_cast<uint4 *>((is_v ? a.stage_v : a.stage_k) +
                                (static_cast<int64_t>(u) * a.stage_rows + px % a.stage_rows) * D + 8 * t) = old;
   const int row = px % I4_TOK;
-  const uint32_t code_s = slot + (is_v ? SLOT_VC : 0) + row * ROW_BYTES;
   const uint32_t sz_s = slot + (is_v ? SLOT_VSZ : SLOT_KSZ) + row * SZ_BYTES;
   const int64_t rec = a.rm.rec(u, px);  // < 0: a bad block-table entry; the cache write is skipped
-  uint8_t *code_g = a.blocks + (is_v ? rec_vcode(rec, px) : rec_kcode(rec, px));
   uint32_t *sz_g = reinterpret_cast<uint32_t *>(a.blocks + (is_v ? rec_vsz(rec, px) : rec_ksz(rec, px)));
-  if (q.has_codes) {
+  if (q.has_codes && !is_v) {
+    const uint32_t code_s = slot + row * ROW_BYTES;
     sts32(code_s + q.off0, q.w0);
     sts32(code_s + q.off1, q.w1);
     if (rec >= 0) {
+      uint8_t *code_g = a.blocks + rec_kcode(rec, px);
       *reinterpret_cast<uint32_t *>(code_g + q.off0) = q.w0;
       *reinterpret_cast<uint32_t *>(code_g + q.off1) = q.w1;
     }
+  }
+  if (q.has_codes && is_v) {
+    // V codes in position pairs: each word as its low and high 16 bits
+    const int h = (q.off0 >> 2) & 1, p0 = q.off0 >> 3;
+    const uint32_t oa = vcode_off(row, p0, h), ob = vcode_off(row, p0 + 1, h);
+    sts16(slot + SLOT_VC + oa, q.w0 & 0xFFFFu);
+    sts16(slot + SLOT_VC + oa + 4, q.w0 >> 16);
+    sts16(slot + SLOT_VC + ob, q.w1 & 0xFFFFu);
+    sts16(slot + SLOT_VC + ob + 4, q.w1 >> 16);
+    if (rec >= 0) store_vcodes(q, a.blocks + rec_vcodes(rec), row);
   }
   if (q.has_sz) {
     sts32(sz_s + 4 * q.g, q.sz);

@@ -78,9 +78,14 @@ __global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half 
   if (p < T - W) {
     const unsigned hmask = 0xFFFFu << (lane & 16);
     const int64_t rec = recmap(c).rec(u, p);
-    if (rec >= 0)  // uniform over the row's 16 lanes
-      quantize_part(xv, t, hmask, c.blocks + (is_v ? rec_vcode(rec, p) : rec_kcode(rec, p)),
-                    reinterpret_cast<uint32_t *>(c.blocks + (is_v ? rec_vsz(rec, p) : rec_ksz(rec, p))), c.dev_status);
+    if (rec >= 0) {  // uniform over the row's 16 lanes
+      if (is_v)
+        quantize_part_v(xv, t, hmask, c.blocks + rec_vcodes(rec), p % BLK_TOK,
+                        reinterpret_cast<uint32_t *>(c.blocks + rec_vsz(rec, p)), c.dev_status);
+      else
+        quantize_part(xv, t, hmask, c.blocks + rec_kcode(rec, p),
+                      reinterpret_cast<uint32_t *>(c.blocks + rec_ksz(rec, p)), c.dev_status);
+    }
     if (c.stage_rows > 0 && p >= T - W - c.stage_rows) {  // staging ring: the most recent quantized rows
       __half *st = reinterpret_cast<__half *>(is_v ? c.stage_v : c.stage_k) + (u * c.stage_rows + p % c.stage_rows) * D;
       *reinterpret_cast<uint4 *>(st + 8 * t) = xv;
@@ -121,9 +126,12 @@ __global__ void append_kernel(hyq_cache c, const __half *__restrict__ k_new,
       const int64_t p = T - W;
       const int64_t rec = recmap(c).rec(u, p);
       if (rec >= 0) {  // uniform over the row's 16 lanes
-        quantize_part(old, t, hmask, c.blocks + (is_v ? rec_vcode(rec, p) : rec_kcode(rec, p)),
-                      reinterpret_cast<uint32_t *>(c.blocks + (is_v ? rec_vsz(rec, p) : rec_ksz(rec, p))),
-                      c.dev_status);
+        if (is_v)
+          quantize_part_v(old, t, hmask, c.blocks + rec_vcodes(rec), static_cast<int>(p % BLK_TOK),
+                          reinterpret_cast<uint32_t *>(c.blocks + rec_vsz(rec, p)), c.dev_status);
+        else
+          quantize_part(old, t, hmask, c.blocks + rec_kcode(rec, p),
+                        reinterpret_cast<uint32_t *>(c.blocks + rec_ksz(rec, p)), c.dev_status);
         // the first row quantized into a record: no position of it is a
         // vertical line yet (they lie below T - W), so its bitmask starts
         // clear, whatever the record held before

@@ -98,4 +98,26 @@ __device__ __forceinline__ void quantize_part(uint4 x, int t, unsigned hmask, ui
   if (q.has_sz) sz_row[q.g] = q.sz;
 }
 
+// Store this thread's code words of slot `slot` into a block record's V code
+// area `vcodes` (position pairs, vcode_off): each 32-bit word goes out as its
+// low and high 16 bits.
+__device__ __forceinline__ void store_vcodes(const QuantShare &q, uint8_t *vcodes, int slot) {
+  if (!q.has_codes) return;
+  const int h = (q.off0 >> 2) & 1, p0 = q.off0 >> 3;
+  uint8_t *a = vcodes + vcode_off(slot, p0, h), *b = vcodes + vcode_off(slot, p0 + 1, h);
+  *reinterpret_cast<uint16_t *>(a) = static_cast<uint16_t>(q.w0);
+  *reinterpret_cast<uint16_t *>(a + 4) = static_cast<uint16_t>(q.w0 >> 16);
+  *reinterpret_cast<uint16_t *>(b) = static_cast<uint16_t>(q.w1);
+  *reinterpret_cast<uint16_t *>(b + 4) = static_cast<uint16_t>(q.w1 >> 16);
+}
+
+// Quantize a V row into slot `slot` of a block record (codes in position
+// pairs) and its scale/zero row.
+__device__ __forceinline__ void quantize_part_v(uint4 x, int t, unsigned hmask, uint8_t *vcodes, int slot,
+                                                uint32_t *sz_row, uint32_t *status) {
+  const QuantShare q = quantize_share(x, t, hmask, status);
+  store_vcodes(q, vcodes, slot);
+  if (q.has_sz) sz_row[q.g] = q.sz;
+}
+
 }  // namespace hyq

@@ -241,10 +241,29 @@ class HybridCache:
             return b[..., off:off + BLOCK_TOKENS * width].reshape(B, H, cap, width)
         kc = field(BLK_KCODES, ROW_BYTES)
         ks = field(BLK_KSZ, 16).copy().view("<u2")
-        vc = field(BLK_VCODES, ROW_BYTES)
+        vc = vcode_rows(b[..., BLK_VCODES:BLK_VCODES + BLOCK_TOKENS * ROW_BYTES]).reshape(B, H, cap, ROW_BYTES)
         vs = field(BLK_VSZ, 16).copy().view("<u2")
         mask = b[..., BLK_MASK:BLK_MASK + 4].copy().view("<u4").reshape(B, H, nb)
         return kc, ks, vc, vs, mask
+
+
+def vcode_rows(area):
+    """Packed V code rows [..., 32, 64] (the row format of hyq_pack) from the
+    V code areas [..., 2048] of block records, where codes are stored in
+    position pairs (include/hyq.h): 16-bit halves indexed [pair][piece][word
+    h][low/high][member of the pair], the members of pair i in the order
+    (2i, 2i + 1) when i % 4 < 2, else (2i + 1, 2i), and piece p of pair i in
+    16-byte unit p xor 2 (i mod 4) of the pair."""
+    area = np.ascontiguousarray(area, dtype=np.uint8)
+    lead = area.shape[:-1]
+    w = area.view("<u2").reshape(lead + (BLOCK_TOKENS // 2, 8, 2, 2, 2))
+    pair = np.arange(BLOCK_TOKENS // 2)[:, None]
+    w = w[..., pair, np.arange(8)[None, :] ^ ((pair & 3) << 1), :, :, :]
+    n = len(lead)
+    w = w.transpose(tuple(range(n)) + (n, n + 4, n + 1, n + 2, n + 3)).copy()
+    swapped = ((np.arange(BLOCK_TOKENS // 2) >> 1) & 1).astype(bool)
+    w[..., swapped, :, :, :, :] = w[..., swapped, ::-1, :, :, :]
+    return w.reshape(lead + (BLOCK_TOKENS, ROW_BYTES // 2)).view(np.uint8)
 
 
 # ------------------------------------------------------------------ entry points

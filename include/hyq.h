@@ -90,7 +90,16 @@ typedef enum {
  * decode tile is a single bulk copy:
  *   offset    0: K codes   [32][64]  (packed rows, format above)
  *   offset 2048: K scale/zero [32][8] fp16
- *   offset 2560: V codes   [32][64]
+ *   offset 2560: V codes, 2048 bytes: the packed rows of the 32 slots in
+ *                position pairs.  Word h (0, 1) of piece p (0..7) of slot t
+ *                (format above) has its low 16 bits at byte
+ *                128 i + 16 (p xor 2 (i mod 4)) + 8 h + 2 s of this area,
+ *                i = t / 2, and its high 16 bits 4 bytes further,
+ *                s = (t mod 2) xor ((t / 4) mod 2):
+ *                the two slots of a pair share every 32-bit word, so the
+ *                decode reads the P.V operands of both with one 16-byte
+ *                load.  (hyq_pack writes plain rows; only the cache's
+ *                records use this order.)
  *   offset 4608: V scale/zero [32][8] fp16
  *   offset 5120: uint32 vertical-line bitmask: bit i set exactly when
  *                position 32*b + i is held in FP16 in the vertical-line rows

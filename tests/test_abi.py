@@ -165,3 +165,31 @@ def test_decode_step_argument_checks(L):
 def test_staging_fields_are_checked(L, over, code):
     c = _desc(**over)
     assert L.hyq_decode(ctypes.byref(c), 0x20000000, 0x30000000, None, 8, None, 0, None) == code
+
+
+def test_vcode_rows_undoes_the_documented_pair_layout():
+    """The record's V code area keeps position pairs interleaved by 16 bits
+    (include/hyq.h): word h of piece p of slot t has its low 16 bits at byte
+    128 i + 16 (p xor 2 (i mod 4)) + 8 h + 2 s, i = t / 2, and its high 16
+    bits 4 bytes further, with s = (t mod 2) xor ((t / 4) mod 2).  The
+    binding's decoder must give back the plain rows, and the layout must use
+    every byte exactly once."""
+    import numpy as np
+
+    def off(t, p, h):
+        i = t // 2
+        return 128 * i + 16 * (p ^ (2 * (i % 4))) + 8 * h + 2 * ((t % 2) ^ ((t // 4) % 2))
+
+    places = sorted(off(t, p, h) + d for t in range(32) for p in range(8) for h in range(2) for d in (0, 1, 4, 5))
+    assert places == list(range(2048))
+    rng = np.random.default_rng(5)
+    rows = rng.integers(0, 256, (2, 3, 32, 64), dtype=np.uint8)
+    area = np.zeros((2, 3, 2048), np.uint8)
+    for t in range(32):
+        for p in range(8):
+            for h in range(2):
+                o = off(t, p, h)
+                word = rows[:, :, t, 8 * p + 4 * h:8 * p + 4 * h + 4]
+                area[:, :, o:o + 2] = word[..., 0:2]
+                area[:, :, o + 4:o + 6] = word[..., 2:4]
+    assert np.array_equal(hyq.vcode_rows(area), rows)
