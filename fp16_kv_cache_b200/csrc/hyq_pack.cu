@@ -45,6 +45,10 @@ __global__ void __launch_bounds__(256) pack_kernel(const __half *__restrict__ x,
 }
 
 // Prefill: one 16-thread group per (unit, position, K|V) row of the prompt.
+// The rows of a pair of positions (2i, 2i + 1) come as a quad K(2i),
+// K(2i + 1), V(2i), V(2i + 1), so the two V rows of a pair meet in one warp:
+// each half quantizes its row, the halves swap their code words, and the
+// record's paired V words (include/hyq.h) are written whole.
 __global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half *__restrict__ k_full,
                                                       const __half *__restrict__ v_full,
                                                       int64_t n_rows) {
@@ -53,46 +57,74 @@ __global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half 
   const int lane = threadIdx.x & 31;
   const int t = lane & 15;
   const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
-  if (row >= n_rows) return;
-  const bool is_v = row & 1;
-  const int64_t up = row >> 1;  // unit * capacity + position
+  if (row >= n_rows) return;  // n_rows is a multiple of 4: a warp's halves leave together
+  const int sub = static_cast<int>(row & 3);
+  const bool is_v = sub >= 2;
+  const int64_t up = ((row >> 2) << 1) | (sub & 1);  // unit * capacity + position
   const int p = static_cast<int>(up % c.capacity);
   const int64_t u = up / c.capacity;
   const int b = static_cast<int>(u / c.n_kv_heads);
   const int T = c.seq_len[b];
-  if (T < 0 || T > c.capacity) {
+  if (T < 0 || T > c.capacity) {  // the same for both halves (one unit)
     if (p == 0 && t == 0 && !is_v && (u % c.n_kv_heads) == 0) set_status(c.dev_status, HYQ_DEV_BADLEN);
     return;
   }
-  // clear this unit's vertical-line set (the bitmask words of the records
-  // holding its positions, and the count)
-  if (!is_v && t == 0 && p == 0) c.vl_count[u] = 0;
-  if (p >= T) return;
-  if (!is_v && t == 0 && (p % BLK_TOK) == 0) {
-    uint32_t *m = mask_of(c, u, p);
-    if (m) *m = 0u;
-  }
-  const __half *src = (is_v ? v_full : k_full) + up * D;
-  const uint4 xv = *reinterpret_cast<const uint4 *>(src + 8 * t);
   const int W = c.window;
-  if (p < T - W) {
-    const unsigned hmask = 0xFFFFu << (lane & 16);
-    const int64_t rec = recmap(c).rec(u, p);
-    if (rec >= 0) {  // uniform over the row's 16 lanes
-      if (is_v)
-        quantize_part_v(xv, t, hmask, c.blocks + rec_vcodes(rec), p % BLK_TOK,
-                        reinterpret_cast<uint32_t *>(c.blocks + rec_vsz(rec, p)), c.dev_status);
-      else
+  const unsigned hmask = 0xFFFFu << (lane & 16);
+  if (!is_v) {
+    // clear this unit's vertical-line set (the bitmask words of the records
+    // holding its positions, and the count)
+    if (t == 0 && p == 0) c.vl_count[u] = 0;
+    if (p >= T) return;
+    if (t == 0 && (p % BLK_TOK) == 0) {
+      uint32_t *m = mask_of(c, u, p);
+      if (m) *m = 0u;
+    }
+    const uint4 xv = *reinterpret_cast<const uint4 *>(k_full + up * D + 8 * t);
+    if (p < T - W) {
+      const int64_t rec = recmap(c).rec(u, p);
+      if (rec >= 0)  // uniform over the row's 16 lanes
         quantize_part(xv, t, hmask, c.blocks + rec_kcode(rec, p),
                       reinterpret_cast<uint32_t *>(c.blocks + rec_ksz(rec, p)), c.dev_status);
+      if (c.stage_rows > 0 && p >= T - W - c.stage_rows)  // staging ring: the most recent quantized rows
+        *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.stage_k) + (u * c.stage_rows + p % c.stage_rows) * D + 8 * t) = xv;
+    } else {
+      *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.win_k) + (u * W + p % W) * D + 8 * t) = xv;
     }
-    if (c.stage_rows > 0 && p >= T - W - c.stage_rows) {  // staging ring: the most recent quantized rows
-      __half *st = reinterpret_cast<__half *>(is_v ? c.stage_v : c.stage_k) + (u * c.stage_rows + p % c.stage_rows) * D;
-      *reinterpret_cast<uint4 *>(st + 8 * t) = xv;
-    }
-  } else {
-    __half *win = reinterpret_cast<__half *>(is_v ? c.win_v : c.win_k) + (u * W + p % W) * D;
-    *reinterpret_cast<uint4 *>(win + 8 * t) = xv;
+    return;
+  }
+  // V rows: both halves of the warp reach the exchanges below
+  const bool valid = p < T, quant = p < T - W;
+  const bool partner_quant = __shfl_xor_sync(0xffffffffu, quant ? 1 : 0, 16) != 0;
+  // the pair's record, looked up at its even position (below T whenever a
+  // member is quantized); < 0: a bad block-table entry, the writes are skipped
+  const int64_t rec = (quant || partner_quant) ? recmap(c).rec(u, p & ~1) : -1;
+  uint4 xv = make_uint4(0, 0, 0, 0);
+  if (valid) xv = *reinterpret_cast<const uint4 *>(v_full + up * D + 8 * t);
+  uint32_t w0 = 0, w1 = 0;
+  if (quant) {
+    const QuantShare q = quantize_share(xv, t, hmask, c.dev_status);
+    w0 = q.w0;
+    w1 = q.w1;
+    if (rec >= 0 && q.has_sz) reinterpret_cast<uint32_t *>(c.blocks + rec_vsz(rec, p))[q.g] = q.sz;
+    if (c.stage_rows > 0 && p >= T - W - c.stage_rows)  // staging ring: the most recent quantized rows
+      *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.stage_v) + (u * c.stage_rows + p % c.stage_rows) * D + 8 * t) = xv;
+  } else if (valid) {
+    *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.win_v) + (u * W + p % W) * D + 8 * t) = xv;
+  }
+  const uint32_t o0 = __shfl_xor_sync(0xffffffffu, w0, 16), o1 = __shfl_xor_sync(0xffffffffu, w1, 16);
+  // Threads of the even groups hold code words (quantize_share): pieces
+  // 2 (t % 4) and 2 (t % 4) + 1, word t / 8.  The pair's first member writes
+  // the words of low halves, the second the words of high halves; a member
+  // that is not quantized (in the window, or past T) contributes zeros.
+  if (rec >= 0 && ((t >> 2) & 1) == 0) {
+    const int slot = p % BLK_TOK, pair = slot >> 1, h = t >> 3, p0 = 2 * (t & 3);
+    const bool first = ((slot & 1) ^ ((slot >> 2) & 1)) == 0;
+    uint8_t *vc = c.blocks + rec_vcodes(rec) + pair * 128 + 8 * h + (first ? 0 : 4);
+    const uint32_t a0 = first ? (w0 & 0xFFFFu) | (o0 << 16) : (o0 >> 16) | (w0 & 0xFFFF0000u);
+    const uint32_t a1 = first ? (w1 & 0xFFFFu) | (o1 << 16) : (o1 >> 16) | (w1 & 0xFFFF0000u);
+    *reinterpret_cast<uint32_t *>(vc + 16 * vcode_unit(pair, p0)) = a0;
+    *reinterpret_cast<uint32_t *>(vc + 16 * vcode_unit(pair, p0 + 1)) = a1;
   }
 }
 

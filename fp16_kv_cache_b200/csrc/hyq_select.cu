@@ -138,28 +138,38 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float (&v)[32]) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// Raw bytes of one thread's quarter key row (32 channels, one quantization
-// group) for the next sub-tile: FP16 (window, vertical line, prefill) as
-// 4 x 16 B, INT4 as the 4 x 16 B packed row plus the group's (scale, zero).
+// One quantization group (32 channels) of a key row as key_store writes it:
+// FP16 (window, vertical line, prefill) as 4 x 16 B, INT4 as the packed
+// row (4 x 16 B) plus the group's (scale, zero).
 struct KeyRaw {
   uint4 v[4];
   uint32_t sz;
   int kind;  // 0 zero, 1 FP16, 2 INT4
 };
 
-// Thread t loads key (t % 128) of the sub-tile, channels 32 (t / 128) .. + 31.
+// Two quantization groups g and g + 2 of one key row, loaded once: FP16 as
+// 2 x 4 x 16 B, INT4 as the 64-byte packed row (all groups) plus the two
+// groups' (scale, zero).
+struct KeyRaw2 {
+  uint4 v[8];
+  uint32_t sz[2];
+  int kind;  // 0 zero, 1 FP16, 2 INT4
+};
+
 template <bool CACHE>
-__device__ __forceinline__ void key_load(const SelectArgs &a, int u, int T, int key, int key_end, int hf, KeyRaw &r) {
+__device__ __forceinline__ void key_load2(const SelectArgs &a, int u, int T, int key, int key_end, int g,
+                                          KeyRaw2 &r) {
   r.kind = 0;
   if (key >= key_end) return;
   const __half *row = nullptr;
+  int64_t rec = 0;
   if (!CACHE) {
     row = a.k_full + (static_cast<int64_t>(u) * a.cap + key) * D;
   } else if (key >= T - a.W) {
     row = a.win_k + (static_cast<int64_t>(u) * a.W + key % a.W) * D;
   } else {
     // a vertical line: its row is the rank of its bit among the unit's set bits
-    const int64_t rec = a.rm.rec_rd(u, key);
+    rec = a.rm.rec_rd(u, key);
     const uint32_t w = *reinterpret_cast<const uint32_t *>(a.blocks + rec_mask(rec));
     if ((w >> (key & 31)) & 1u) {
       const int slot = a.rank_base[static_cast<int64_t>(u) * (a.cap / 32) + (key >> 5)] +
@@ -170,15 +180,19 @@ __device__ __forceinline__ void key_load(const SelectArgs &a, int u, int T, int 
   if (row) {
     r.kind = 1;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) r.v[c] = *reinterpret_cast<const uint4 *>(row + 32 * hf + 8 * c);
+    for (int c = 0; c < 4; ++c) {
+      r.v[c] = *reinterpret_cast<const uint4 *>(row + 32 * g + 8 * c);
+      r.v[4 + c] = *reinterpret_cast<const uint4 *>(row + 32 * (g + 2) + 8 * c);
+    }
     return;
   }
   r.kind = 2;
-  const int64_t rec = a.rm.rec_rd(u, key);
   const uint4 *codes = reinterpret_cast<const uint4 *>(a.blocks + rec_kcode(rec, key));
 #pragma unroll
   for (int c = 0; c < 4; ++c) r.v[c] = codes[c];
-  r.sz = *reinterpret_cast<const uint32_t *>(a.blocks + rec_ksz(rec, key) + 4 * hf);
+  const uint32_t *sz = reinterpret_cast<const uint32_t *>(a.blocks + rec_ksz(rec, key));
+  r.sz[0] = sz[g];
+  r.sz[1] = sz[g + 2];
 }
 
 // Write the thread's 4 chunks of key row kk as fp16 (hi) and, in cache mode,
@@ -226,31 +240,68 @@ __device__ __forceinline__ void key_store(const KeyRaw &r, int kk, int hf, uint8
   }
 }
 
-// Wait (bounded) for the MMAs committed to `bar` to complete phase `parity`.
-__device__ __forceinline__ void tc_wait(uint32_t bar, uint32_t parity, const SelectArgs &a, int *abort) {
-  if (mbar_try_wait(bar, parity)) return;
-  const uint64_t t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > 2000000000ull) {
-      set_status(a.status, HYQ_DEV_TIMEOUT);
-      *abort = 1;
-      return;
-    }
+// Write groups g and g + 2 of key row kk (key_store on each).
+template <bool CACHE>
+__device__ __forceinline__ void key_store2(const KeyRaw2 &r, int kk, int g, uint8_t *hi, uint8_t *lo) {
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    KeyRaw x;
+    x.kind = r.kind;
+    x.sz = r.sz[j];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) x.v[c] = (r.kind == 1) ? r.v[4 * j + c] : r.v[c];
+    key_store<CACHE>(x, kk, g + 2 * j, hi, lo);
   }
+}
+
+// One (unit, 512-key chunk) work item as both roles of the scorer see it.
+struct SelItem {
+  int u, T, k0, k1, nsub;  // nsub: sub-tiles of 128 keys (0: none)
+  bool valid;              // the unit's length admits a selection (else reported by the top-k)
+};
+
+template <int PASS>
+__device__ __forceinline__ SelItem sel_item(const SelectArgs &a, int item) {
+  SelItem s;
+  s.u = item / a.n_chunks;
+  s.T = sel_T(a, s.u);
+  s.valid = !(s.T < a.n_q || s.T > a.cap || s.T - a.W < a.k);
+  const int key_end = (PASS == 1) ? s.T : s.T - a.W;
+  s.k0 = (item % a.n_chunks) * SEL_KC;
+  s.k1 = min(key_end, s.k0 + SEL_KC);
+  s.nsub = (s.valid && s.k0 < key_end) ? (s.k1 - s.k0 + TC_NK - 1) / TC_NK : 0;
+  return s;
 }
 
 // PASS 1: per-row (max, sum exp) over a chunk of keys; PASS 2: column sums.
 // Block b takes a contiguous run of (unit, 512-key chunk) items, so the
-// query rows are loaded once per unit.  With up to 256 query rows the key
-// tiles and the accumulators are double-buffered: the MMAs of sub-tile t+1
-// run while the epilogue of t and the dequantization of t+2 proceed.
+// query rows are loaded once per unit.  The warps split into two roles that
+// work on different sub-tiles at once and meet only through mbarriers:
+//   * warps 0-7 stage key sub-tiles of 128 keys into shared memory (thread s
+//     writes key row s % 128, quantization groups s / 128 and s / 128 + 2),
+//     loading the next sub-tile from global memory while the current one is
+//     written; once all 256 staging threads have arrived on a sub-tile's
+//     barrier, thread 0 issues its MMAs and commits them;
+//   * warps 8-15 read the accumulators the MMAs complete (lane quadrant
+//     w % 4, one half of the columns of every row block) and run the exp2
+//     epilogue.
+// Barriers per buffer: key_full (sub-tile staged, 256 arrivals), acc_full
+// (MMAs complete, one commit; it also frees the key buffer they read),
+// acc_empty (epilogue done with the accumulators, 256 arrivals).  With up
+// to 256 query rows key tiles and accumulators are double-buffered, so the
+// staging of sub-tile g + 1 and its MMAs overlap the epilogue of g.  Every
+// wait is bounded (2 s, then HYQ_DEV_TIMEOUT); after a timeout every wait
+// returns at once and the loops run out without work, so the epilogue
+// warps still meet at each of their named barriers.
+constexpr int TC_ROLE = TC_THREADS / 2;  // threads per role
+
 template <bool CACHE, int PASS>
 __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a) {
   pdl_trigger();  // the next kernel may be scheduled
   pdl_wait();     // earlier work on the stream is complete and visible (and its tensor memory freed)
   extern __shared__ __align__(1024) uint8_t sm_raw[];
   __shared__ uint32_t tmem_base;
-  __shared__ __align__(8) uint64_t mbar[2];
+  __shared__ __align__(8) uint64_t key_full[2], acc_full[2], acc_empty[2];
   __shared__ int s_abort;
   // 128-byte swizzled tiles must start on a 1024-byte boundary
   uint8_t *sm = sm_raw + ((1024u - (smem_u32(sm_raw) & 1023u)) & 1023u);
@@ -259,11 +310,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
   constexpr int KT = CACHE ? 2 * TC_TILE : TC_TILE;     // one key buffer: hi (+ lo)
   uint8_t *sQ = sm;                                      // [n_rbt][32 KB]
   uint8_t *sK = sQ + n_rbt * TC_TILE;                    // [nbuf][KT]
-  float *csum = reinterpret_cast<float *>(sK + nbuf * KT);              // [4][128]
-  float2 *pst = reinterpret_cast<float2 *>(csum + 4 * TC_NK);           // [3][TC_MAX_RB][128]
-  float *moff = reinterpret_cast<float *>(pst + 3 * TC_MAX_RB * 128);   // [SEL_MAX_ROWS] pass 2: m_r - log2(1/l_r)
+  float *csum = reinterpret_cast<float *>(sK + nbuf * KT);             // pass 2: [sub-tile parity][half][128]
+  float2 *pst = reinterpret_cast<float2 *>(csum + 4 * TC_NK);          // pass 1: [item parity][TC_MAX_RB][128]
+  float *moff = reinterpret_cast<float *>(pst + 3 * TC_MAX_RB * 128);  // pass 2: [SEL_MAX_ROWS] m_r - log2(1/l_r)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qd = warp & 3, hfw = warp >> 2;  // TMEM lane quadrant, column quarter
   const uint32_t acc_cols = static_cast<uint32_t>(n_rbt) * TC_NK;      // one accumulator set
   const uint32_t need = acc_cols * nbuf;
   const uint32_t ncols = (need <= 128) ? 128u : (need <= 256) ? 256u : 512u;
@@ -273,8 +323,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 0) {
-    mbar_init(smem_u32(&mbar[0]), 1);
-    mbar_init(smem_u32(&mbar[1]), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&key_full[b]), TC_ROLE);
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), TC_ROLE);
+    }
     fence_barrier_init();
     s_abort = 0;
   }
@@ -282,221 +335,217 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = tmem_base;
-  uint32_t phase[2] = {0u, 0u};
+  volatile int *abort = &s_abort;
   const int n_items = a.U * a.n_chunks;
   const int per = (n_items + gridDim.x - 1) / gridDim.x;
   const int it0 = min(n_items, static_cast<int>(blockIdx.x) * per), it1 = min(n_items, it0 + per);
-  int q_unit = -1, q_T = -1;
-  const int kk = tid & 127, hfk = tid >> 7;  // key row and channel quarter (quantization group) this thread stages
-  KeyRaw raw;
-  bool have_next = false;  // raw holds the first tile of the next item
+  // bounded wait for phase `parity` of barrier b (false after a timeout, here or elsewhere in the block)
+  auto wait = [&](uint64_t *b, uint32_t parity) { return mbar_wait_bounded(smem_u32(b), parity, abort, a.status); };
 
-  // one sub-tile's MMAs into accumulator set `buf` from key buffer `buf`
-  auto issue = [&](int buf) {
-    if (tid == 0) {
-      // descriptors of k-step 0; k-step ks adds sw128_koff(ks) to the
-      // start-address field (16-byte units; tiles lie below 256 KB)
-      const uint32_t kh = smem_u32(sK + buf * KT), kl = kh + TC_TILE;
-      const uint64_t dkh = sw128_desc(kh, 0), dkl = sw128_desc(kl, 0);
-      for (int rb = 0; rb < n_rbt; ++rb) {
-        const uint64_t dq = sw128_desc(smem_u32(sQ) + rb * TC_TILE, 0);
-        const uint32_t d = tbase + buf * acc_cols + rb * TC_NK;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t o = sw128_koff(ks);
-          if (PASS == 1) {  // rows on M, keys on N
-            tc_mma(d, dq + o, dkh + o, ks > 0);
-            if (CACHE) tc_mma(d, dq + o, dkl + o, 1u);
-          } else {          // keys on M, rows on N: each TMEM lane is one key column
-            tc_mma(d, dkh + o, dq + o, ks > 0);
-            if (CACHE) tc_mma(d, dkl + o, dq + o, 1u);
+  if (warp < TC_ROLE / 32) {
+    // ---- staging: key row kk of every sub-tile, quantization groups hq and hq + 2
+    const int kk = tid & 127, hq = tid >> 7;
+    KeyRaw2 rk;         // the next sub-tile to stage (groups hq, hq + 2)
+    bool have = false;  // rk already holds it
+    int q_unit = -1, q_T = -1, gst = 0;
+    for (int item = it0; item < it1; ++item) {
+      const SelItem s = sel_item<PASS>(a, item);
+      if (s.nsub == 0) continue;
+      if (s.u != q_unit || s.T != q_T) {
+        // the MMAs that read the previous unit's query rows are complete
+        if (gst > 0) wait(&acc_full[(gst - 1) % nbuf], ((gst - 1) / nbuf) & 1);
+        // the unit's query rows into the swizzled row blocks (zeros past R)
+        const int b = s.u / a.Hkv, kvh = s.u % a.Hkv;
+        for (int i = tid; i < n_rbt * 128 * 16; i += TC_ROLE) {
+          const int r = i >> 4, c = i & 15;
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (r < a.R) {
+            const int hg = r / a.n_q, ii = r % a.n_q;
+            const int slot = a.q_ring ? ((s.T - a.n_q + ii) % a.n_q + a.n_q) % a.n_q : ii;
+            v = *reinterpret_cast<const uint4 *>(a.q + ((static_cast<int64_t>(b) * a.Hq + kvh * a.G + hg) * a.n_q + slot) * D +
+                                                 8 * c);
+          }
+          *reinterpret_cast<uint4 *>(sQ + (r >> 7) * TC_TILE + sw128_off(r & 127, 8 * c)) = v;
+        }
+        q_unit = s.u;
+        q_T = s.T;
+      }
+      for (int st = 0; st < s.nsub; ++st) {
+        const int g = gst + st, buf = g % nbuf;
+        const uint32_t ph = (g / nbuf) & 1;
+        // the MMAs of sub-tile g - nbuf, the last readers of key buffer buf, are complete
+        if (g >= nbuf) wait(&acc_full[buf], ph ^ 1);
+        const int key0 = s.k0 + st * TC_NK;
+        if (!have) key_load2<CACHE>(a, s.u, s.T, key0 + kk, s.k1, hq, rk);
+        uint8_t *kb = sK + buf * KT;
+        key_store2<CACHE>(rk, kk, hq, kb, kb + TC_TILE);
+        // the next sub-tile (or the next item's first, same unit) loads while this one is issued
+        have = false;
+        if (st + 1 < s.nsub) {
+          key_load2<CACHE>(a, s.u, s.T, key0 + TC_NK + kk, s.k1, hq, rk);
+          have = true;
+        } else if (item + 1 < it1) {
+          const SelItem n = sel_item<PASS>(a, item + 1);
+          if (n.nsub > 0 && n.u == s.u && n.T == s.T) {
+            key_load2<CACHE>(a, n.u, n.T, n.k0 + kk, n.k1, hq, rk);
+            have = true;
           }
         }
-      }
-      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                       smem_u32(&mbar[buf]))
-                   : "memory");
-    }
-  };
-  // hand the staged tile to the tensor core (generic writes -> async proxy)
-  auto publish = [&]() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-  };
-
-  for (int item = it0; item < it1 && !s_abort; ++item) {
-    const int u = item / a.n_chunks, chunk = item % a.n_chunks;
-    const int T = sel_T(a, u);
-    if (T < a.n_q || T > a.cap || T - a.W < a.k) continue;  // reported by the top-k kernel
-    const int key_end = (PASS == 1) ? T : T - a.W;
-    const int k0 = chunk * SEL_KC;
-    if (k0 >= key_end) {
-      if (PASS == 1)
-        for (int r = tid; r < a.R; r += TC_THREADS)
-          a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + r] = make_float2(-INFINITY, 0.f);
-      continue;
-    }
-    const int k1 = min(key_end, k0 + SEL_KC);
-    const int nsub = (k1 - k0 + TC_NK - 1) / TC_NK;
-    tc_fence_before();
-    __syncthreads();  // the previous item is done with shared and tensor memory
-    tc_fence_after();
-    if (u != q_unit || T != q_T) {
-      // the unit's query rows into the swizzled row blocks (zeros past R)
-      const int b = u / a.Hkv, kvh = u % a.Hkv;
-      for (int i = tid; i < n_rbt * 128 * 16; i += TC_THREADS) {
-        const int r = i >> 4, c = i & 15;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < a.R) {
-          const int hg = r / a.n_q, ii = r % a.n_q;
-          const int slot = a.q_ring ? ((T - a.n_q + ii) % a.n_q + a.n_q) % a.n_q : ii;
-          v = *reinterpret_cast<const uint4 *>(a.q + ((static_cast<int64_t>(b) * a.Hq + kvh * a.G + hg) * a.n_q + slot) * D +
-                                               8 * c);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> the tensor core
+        mbar_arrive(smem_u32(&key_full[buf]));
+        if (tid == 0 && wait(&key_full[buf], ph) && (g < nbuf || wait(&acc_empty[buf], ph ^ 1))) {
+          // every staging thread has written sub-tile g, and the epilogue is done with accumulator set buf
+          tc_fence_after();
+          // descriptors of k-step 0; k-step ks adds sw128_koff(ks) to the
+          // start-address field (16-byte units; tiles lie below 256 KB)
+          const uint32_t kh = smem_u32(kb), kl = kh + TC_TILE;
+          const uint64_t dkh = sw128_desc(kh, 0), dkl = sw128_desc(kl, 0);
+          for (int rb = 0; rb < n_rbt; ++rb) {
+            const uint64_t dq = sw128_desc(smem_u32(sQ) + rb * TC_TILE, 0);
+            const uint32_t d = tbase + buf * acc_cols + rb * TC_NK;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint32_t o = sw128_koff(ks);
+              if (PASS == 1) {  // rows on M, keys on N
+                tc_mma(d, dq + o, dkh + o, ks > 0);
+                if (CACHE) tc_mma(d, dq + o, dkl + o, 1u);
+              } else {          // keys on M, rows on N: each TMEM lane is one key column
+                tc_mma(d, dkh + o, dq + o, ks > 0);
+                if (CACHE) tc_mma(d, dkl + o, dq + o, 1u);
+              }
+            }
+          }
+          asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                           smem_u32(&acc_full[buf]))
+                       : "memory");
         }
-        *reinterpret_cast<uint4 *>(sQ + (r >> 7) * TC_TILE + sw128_off(r & 127, 8 * c)) = v;
       }
-      if (PASS == 2)
+      gst += s.nsub;
+    }
+  } else {
+    // ---- epilogue: TMEM lane quadrant qd, column half hf of every row block
+    const int e = tid - TC_ROLE, ew = e >> 5, qd = ew & 3, hf = ew >> 2;
+    int q_unit = -1, q_T = -1, gst = 0, ipar = 0;
+    for (int item = it0; item < it1; ++item) {
+      const SelItem s = sel_item<PASS>(a, item);
+      if (!s.valid) continue;
+      const int64_t part = (static_cast<int64_t>(s.u) * a.n_chunks + item % a.n_chunks) * SEL_MAX_ROWS;
+      if (s.nsub == 0) {
+        if (PASS == 1)
+          for (int r = e; r < a.R; r += TC_ROLE) a.stats_part[part + r] = make_float2(-INFINITY, 0.f);
+        continue;
+      }
+      if (PASS == 2 && (s.u != q_unit || s.T != q_T)) {
         // p = exp2(s - m_r) / l_r = exp2(s - (m_r - log2(1 / l_r))); rows
         // without keys (or past R) get +inf, i.e. p = 0
-        for (int r = tid; r < n_rbt * 128; r += TC_THREADS) {
+        named_bar_sync(1, TC_ROLE);  // every epilogue thread is done with the previous unit's offsets
+        for (int r = e; r < n_rbt * 128; r += TC_ROLE) {
           float mo = INFINITY;
           if (r < a.R) {
-            const float2 st = a.stats[static_cast<int64_t>(u) * SEL_MAX_ROWS + r];
-            if (st.y > 0.f) mo = st.x - __log2f(st.y);
+            const float2 stt = a.stats[static_cast<int64_t>(s.u) * SEL_MAX_ROWS + r];
+            if (stt.y > 0.f) mo = stt.x - __log2f(stt.y);
           }
           moff[r] = mo;
         }
-      q_unit = u;
-      q_T = T;
-      __syncthreads();  // stage arrays written
-    }
-    float rm[TC_MAX_RB], rl[TC_MAX_RB];  // pass 1: running (max, sum) of this thread's rows over its columns
-#pragma unroll
-    for (int rb = 0; rb < TC_MAX_RB; ++rb) {
-      rm[rb] = -INFINITY;
-      rl[rb] = 0.f;
-    }
-    if (!have_next) key_load<CACHE>(a, u, T, k0 + kk, k1, hfk, raw);
-    have_next = false;
-    key_store<CACHE>(raw, kk, hfk, sK, sK + TC_TILE);
-    publish();
-    issue(0);
-    if (nsub > 1) key_load<CACHE>(a, u, T, k0 + TC_NK + kk, k1, hfk, raw);
-    for (int st = 0; st < nsub; ++st) {
-      const int buf = (nbuf == 2) ? (st & 1) : 0;
-      const int key0 = k0 + st * TC_NK;
-      if (nbuf == 2 && st + 1 < nsub) {
-        // next tile into the other buffer (its last reader, sub-tile st-1, is done)
-        key_store<CACHE>(raw, kk, hfk, sK + (buf ^ 1) * KT, sK + (buf ^ 1) * KT + TC_TILE);
-        publish();
-        issue(buf ^ 1);
-        if (st + 2 < nsub) key_load<CACHE>(a, u, T, key0 + 2 * TC_NK + kk, k1, hfk, raw);
+        named_bar_sync(1, TC_ROLE);
       }
-      if (st + 1 == nsub && item + 1 < it1 && (item + 1) / a.n_chunks == u) {
-        // the next item's first tile (same unit) loads during this epilogue
-        const int k0n = k0 + SEL_KC;
-        if (k0n < key_end) {
-          key_load<CACHE>(a, u, T, k0n + kk, min(key_end, k0n + SEL_KC), hfk, raw);
-          have_next = true;
-        }
+      q_unit = s.u;
+      q_T = s.T;
+      float rm[TC_MAX_RB], rl[TC_MAX_RB];  // pass 1: running (max, sum) of this thread's rows over its columns
+#pragma unroll
+      for (int rb = 0; rb < TC_MAX_RB; ++rb) {
+        rm[rb] = -INFINITY;
+        rl[rb] = 0.f;
       }
-      tc_wait(smem_u32(&mbar[buf]), phase[buf], a, &s_abort);
-      phase[buf] ^= 1u;
-      tc_fence_after();
-      if (PASS == 1) {
-        // epilogue: this thread's row of each row block, 32 key columns
-        const bool all_visible = key0 + TC_NK <= k1 && key0 + TC_NK - 1 <= T - a.n_q;
+      for (int st = 0; st < s.nsub; ++st) {
+        const int g = gst + st, buf = g % nbuf;
+        const uint32_t ph = (g / nbuf) & 1;
+        // the warp reads tensor memory together or not at all
+        const bool ok = __all_sync(0xffffffffu, wait(&acc_full[buf], ph));
+        tc_fence_after();
+        const int key0 = s.k0 + st * TC_NK;
+        const uint32_t tcol = tbase + (static_cast<uint32_t>(32 * qd) << 16) + buf * acc_cols + 64 * hf;
+        if (PASS == 1) {
+          const bool all_visible = key0 + TC_NK <= s.k1 && key0 + TC_NK - 1 <= s.T - a.n_q;
 #pragma unroll
-        for (int rb = 0; rb < TC_MAX_RB; ++rb) {
-          if (rb >= n_rbt) break;
-          const int r = 128 * rb + 32 * qd + lane;
-          const bool row_ok = r < a.R;
-          const int qpos = row_ok ? T - a.n_q + r % a.n_q : -1;  // last key this query sees
-          {
-            float v[32];
-            // every lane of the warp takes part in the tensor-memory load
-            tc_ld32(tbase + (static_cast<uint32_t>(32 * qd) << 16) + buf * acc_cols + rb * TC_NK + 32 * hfw, v);
-            const int kb = key0 + 32 * hfw;  // key of v[0]
-            if (!(all_visible && row_ok))
+          for (int rb = 0; rb < TC_MAX_RB; ++rb) {
+            if (rb >= n_rbt || !ok) break;
+            const int r = 128 * rb + 32 * qd + lane;
+            const bool row_ok = r < a.R;
+            const int qpos = row_ok ? s.T - a.n_q + r % a.n_q : -1;  // last key this query sees
 #pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (!(kb + j < k1 && kb + j <= qpos)) v[j] = -INFINITY;
-            float mx = -INFINITY;
+            for (int c2 = 0; c2 < 2; ++c2) {
+              float v[32];
+              tc_ld32(tcol + rb * TC_NK + 32 * c2, v);
+              const int kb = key0 + 64 * hf + 32 * c2;  // key of v[0]
+              if (!(all_visible && row_ok))
 #pragma unroll
-            for (int j = 0; j < 32; ++j) mx = fmaxf(mx, v[j]);
-            const float mn = fmaxf(rm[rb], mx * SEL_SCALE);  // the scale is positive
-            if (mn != -INFINITY) {
-              float sum = 0.f;
+                for (int j = 0; j < 32; ++j)
+                  if (!(kb + j < s.k1 && kb + j <= qpos)) v[j] = -INFINITY;
+              float mx = -INFINITY;
 #pragma unroll
-              for (int j = 0; j < 32; ++j) sum += fast_exp2(fmaf(v[j], SEL_SCALE, -mn));
-              rl[rb] = rl[rb] * fast_exp2(rm[rb] - mn) + sum;
-              rm[rb] = mn;
+              for (int j = 0; j < 32; ++j) mx = fmaxf(mx, v[j]);
+              const float mn = fmaxf(rm[rb], mx * SEL_SCALE);  // the scale is positive
+              if (mn != -INFINITY) {
+                float sum = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sum += fast_exp2(fmaf(v[j], SEL_SCALE, -mn));
+                rl[rb] = rl[rb] * fast_exp2(rm[rb] - mn) + sum;
+                rm[rb] = mn;
+              }
             }
           }
-        }
-      } else {
-        // epilogue: this thread is key column 32 (w % 4) + lane of the
-        // sub-tile; it sums p over its quarter of the rows (every candidate
-        // key is visible to every selection query)
-        float acc = 0.f;
+        } else {
+          // this thread is key column 32 qd + lane of the sub-tile; it sums p
+          // over its half of the rows (every candidate key is visible to
+          // every selection query)
+          float acc = 0.f;
 #pragma unroll
-        for (int rb = 0; rb < TC_MAX_RB; ++rb) {
-          if (rb >= n_rbt) break;
-          float v[32];
-          tc_ld32(tbase + (static_cast<uint32_t>(32 * qd) << 16) + buf * acc_cols + rb * TC_NK + 32 * hfw, v);
-          const float *mo = moff + rb * TC_NK + 32 * hfw;  // row of v[0]
+          for (int rb = 0; rb < TC_MAX_RB; ++rb) {
+            if (rb >= n_rbt || !ok) break;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc += fast_exp2(fmaf(v[j], SEL_SCALE, -mo[j]));
-        }
-        csum[hfw * TC_NK + 32 * qd + lane] = acc;
-      }
-      tc_fence_before();
-      __syncthreads();  // accumulator set `buf` is free again
-      tc_fence_after();
-      if (PASS == 2 && tid < TC_NK) {
-        const int key = key0 + tid;
-        // fixed order: ((q0 + q1) + q2) + q3, the same for every key
-        if (key < k1)
-          a.colsum_part[static_cast<int64_t>(u) * a.cap + key] =
-              ((csum[tid] + csum[TC_NK + tid]) + csum[2 * TC_NK + tid]) + csum[3 * TC_NK + tid];
-      }
-      if (nbuf == 1 && st + 1 < nsub) {
-        key_store<CACHE>(raw, kk, hfk, sK, sK + TC_TILE);
-        publish();
-        issue(0);
-        if (st + 2 < nsub) key_load<CACHE>(a, u, T, key0 + 2 * TC_NK + kk, k1, hfk, raw);
-      }
-      if (s_abort) break;
-    }
-    if (PASS == 1) {
-      // merge the four column quarters of every row, then write the chunk partial
-      if (hfw > 0)
+            for (int c2 = 0; c2 < 2; ++c2) {
+              float v[32];
+              tc_ld32(tcol + rb * TC_NK + 32 * c2, v);
+              const float *mo = moff + rb * TC_NK + 64 * hf + 32 * c2;  // row of v[0]
 #pragma unroll
-        for (int rb = 0; rb < TC_MAX_RB; ++rb)
-          if (rb < n_rbt) pst[((hfw - 1) * TC_MAX_RB + rb) * 128 + 32 * qd + lane] = make_float2(rm[rb], rl[rb]);
-      __syncthreads();
-      if (hfw == 0)
-#pragma unroll
-        for (int rb = 0; rb < TC_MAX_RB; ++rb) {
-          const int r = 128 * rb + 32 * qd + lane;
-          if (rb >= n_rbt || r >= a.R) continue;
-          float2 o[3];
-          float M = rm[rb];
-#pragma unroll
-          for (int qq = 0; qq < 3; ++qq) {
-            o[qq] = pst[(qq * TC_MAX_RB + rb) * 128 + 32 * qd + lane];
-            M = fmaxf(M, o[qq].x);
+              for (int j = 0; j < 32; ++j) acc += fast_exp2(fmaf(v[j], SEL_SCALE, -mo[j]));
+            }
           }
-          float L = 0.f;
-          if (M != -INFINITY) {
-            L = rl[rb] * fast_exp2(rm[rb] - M);
-#pragma unroll
-            for (int qq = 0; qq < 3; ++qq) L += o[qq].y * fast_exp2(o[qq].x - M);
-          }
-          a.stats_part[(static_cast<int64_t>(u) * a.n_chunks + chunk) * SEL_MAX_ROWS + r] = make_float2(M, L);
+          csum[((g & 1) * 2 + hf) * TC_NK + 32 * qd + lane] = acc;
         }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acc_empty[buf]));  // accumulator set buf may be overwritten
+        if (PASS == 2) {
+          named_bar_sync(1, TC_ROLE);
+          // fixed order: half 0 + half 1, the same for every key
+          const int key = key0 + e;
+          if (e < TC_NK && key < s.k1)
+            a.colsum_part[static_cast<int64_t>(s.u) * a.cap + key] =
+                csum[(g & 1) * 2 * TC_NK + e] + csum[((g & 1) * 2 + 1) * TC_NK + e];
+        }
+      }
+      gst += s.nsub;
+      if (PASS == 1) {
+        // merge the two column halves of every row, then write the chunk partial
+        if (hf == 1)
+#pragma unroll
+          for (int rb = 0; rb < TC_MAX_RB; ++rb)
+            if (rb < n_rbt) pst[(ipar * TC_MAX_RB + rb) * 128 + 32 * qd + lane] = make_float2(rm[rb], rl[rb]);
+        named_bar_sync(1, TC_ROLE);
+        if (hf == 0)
+#pragma unroll
+          for (int rb = 0; rb < TC_MAX_RB; ++rb) {
+            const int r = 128 * rb + 32 * qd + lane;
+            if (rb >= n_rbt || r >= a.R) continue;
+            const float2 o = pst[(ipar * TC_MAX_RB + rb) * 128 + 32 * qd + lane];
+            const float M = fmaxf(rm[rb], o.x);
+            float L = 0.f;
+            if (M != -INFINITY) L = rl[rb] * fast_exp2(rm[rb] - M) + o.y * fast_exp2(o.x - M);
+            a.stats_part[part + r] = make_float2(M, L);
+          }
+        ipar ^= 1;
+      }
     }
   }
   tc_fence_before();
