@@ -87,7 +87,8 @@ __global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half 
         quantize_part(xv, t, hmask, c.blocks + rec_kcode(rec, p),
                       reinterpret_cast<uint32_t *>(c.blocks + rec_ksz(rec, p)), c.dev_status);
       if (c.stage_rows > 0 && p >= T - W - c.stage_rows)  // staging ring: the most recent quantized rows
-        *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.stage_k) + (u * c.stage_rows + p % c.stage_rows) * D + 8 * t) = xv;
+        *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.stage_k) + (u * c.stage_rows + p % c.stage_rows) * D +
+                                   8 * t) = xv;
     } else {
       *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.win_k) + (u * W + p % W) * D + 8 * t) = xv;
     }
@@ -108,7 +109,8 @@ __global__ void __launch_bounds__(256) prefill_kernel(hyq_cache c, const __half 
     w1 = q.w1;
     if (rec >= 0 && q.has_sz) reinterpret_cast<uint32_t *>(c.blocks + rec_vsz(rec, p))[q.g] = q.sz;
     if (c.stage_rows > 0 && p >= T - W - c.stage_rows)  // staging ring: the most recent quantized rows
-      *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.stage_v) + (u * c.stage_rows + p % c.stage_rows) * D + 8 * t) = xv;
+      *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.stage_v) + (u * c.stage_rows + p % c.stage_rows) * D +
+                                 8 * t) = xv;
   } else if (valid) {
     *reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(c.win_v) + (u * W + p % W) * D + 8 * t) = xv;
   }
