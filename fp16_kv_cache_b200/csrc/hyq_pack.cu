@@ -320,21 +320,34 @@ __global__ void __launch_bounds__(1024) vl_recompact_kernel(hyq_cache c, const i
       if (uint32_t *m = mask_of(c, u, p)) atomicAnd(m, ~(1u << (p & 31)));
   }
   __syncthreads();
+  // Kept rows move down to their new slots (a destination is never above its
+  // source): each pass loads RM rows per 16-thread group, and all its loads
+  // complete (barrier) before any of its stores, so no row is overwritten
+  // before it is read.
+  constexpr int RM = 2;
   const int rows = blockDim.x / 16;
-  for (int base = 0; base < n_kept; base += rows) {
-    const int r = base + (threadIdx.x >> 4), part = threadIdx.x & 15;
-    const bool act = r < n_kept && kslot[r] != r;
-    uint4 rk = make_uint4(0, 0, 0, 0), rv = rk;
-    if (act) {
-      const int64_t so = (row_base + kslot[r]) * D + 8 * part;
-      rk = *reinterpret_cast<const uint4 *>(vk + so);
-      rv = *reinterpret_cast<const uint4 *>(vv + so);
+  for (int base = 0; base < n_kept; base += RM * rows) {
+    const int part = threadIdx.x & 15;
+    uint4 rk[RM], rv[RM];
+    bool act[RM];
+#pragma unroll
+    for (int q = 0; q < RM; ++q) {
+      const int r = base + q * rows + (threadIdx.x >> 4);
+      act[q] = r < n_kept && kslot[r] != r;
+      rk[q] = rv[q] = make_uint4(0, 0, 0, 0);
+      if (act[q]) {
+        const int64_t so = (row_base + kslot[r]) * D + 8 * part;
+        rk[q] = *reinterpret_cast<const uint4 *>(vk + so);
+        rv[q] = *reinterpret_cast<const uint4 *>(vv + so);
+      }
     }
     __syncthreads();
-    if (act) {
-      const int64_t d = (row_base + r) * D + 8 * part;
-      *reinterpret_cast<uint4 *>(vk + d) = rk;
-      *reinterpret_cast<uint4 *>(vv + d) = rv;
+#pragma unroll
+    for (int q = 0; q < RM; ++q) {
+      if (!act[q]) continue;
+      const int64_t d = (row_base + base + q * rows + (threadIdx.x >> 4)) * D + 8 * part;
+      *reinterpret_cast<uint4 *>(vk + d) = rk[q];
+      *reinterpret_cast<uint4 *>(vv + d) = rv[q];
     }
     __syncthreads();
   }

@@ -596,7 +596,7 @@ __global__ void stats_merge_kernel(const SelectArgs a) {
   const int T = sel_T(a, u);
   if (T < a.n_q || T > a.cap) return;
   const int nch = (T + SEL_KC - 1) / SEL_KC;
-  constexpr int MB = 8;  // chunk partials loaded at once
+  constexpr int MB = 16;  // chunk partials loaded at once
   for (int r = threadIdx.x; r < a.R; r += blockDim.x) {
     const float2 *p = a.stats_part + static_cast<int64_t>(u) * a.n_chunks * SEL_MAX_ROWS + r;
     // log-sum-exp merge of the chunk partials in chunk order, MB loads in flight
