@@ -337,6 +337,28 @@ def hyq_decode_step(cache: HybridCache, q, k_new, v_new, o, ws, q_ring=None, lse
            "hyq_decode_step")
 
 
+class DecodeStepCall:
+    """hyq_decode_step with its arguments marshalled once, for a loop that
+    calls it again and again on the same buffers: the pointers, sizes and the
+    stream are fixed when the object is made, and each call is one foreign
+    call.  The cache's descriptor is passed by reference, so the library's
+    own updates of the lengths on the device are seen; the buffers are kept
+    alive by the object."""
+
+    def __init__(self, cache: HybridCache, q, k_new, v_new, o, ws, q_ring=None, lse=None, n_ctas: int = 0,
+                 stream=None):
+        n_q = int(q_ring.shape[2]) if q_ring is not None else 0
+        self._f = _L().hyq_decode_step
+        self._args = (cache.ref(), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_ring), n_q, _ptr(o), _ptr(lse),
+                      n_ctas, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+        self._keep = (cache, q, k_new, v_new, q_ring, o, lse, ws)
+
+    def __call__(self):
+        rc = self._f(*self._args)
+        if rc != 0:
+            raise HyqError(int(rc), "hyq_decode_step")
+
+
 def hyq_decode_noalloc(cache: HybridCache, q, o, lse=None, stream=None):
     """hyq_decode with the library's built-in scratch array instead of a
     caller workspace (for callers that cannot allocate device memory).  Calls

@@ -212,3 +212,36 @@ def test_graph_consecutive_steps_equal_eager(n_ctas):
     for k in sg:
         assert np.array_equal(sg[k], se[k]), f"{k} differs after {steps} steps"
     assert g_cache.status() == 0 and e_cache.status() == 0
+
+
+def test_prepared_step_call_matches_the_wrapper():
+    """hyq.DecodeStepCall (arguments marshalled once, reused over steps on
+    the same buffers) gives the same bits as hyq_decode_step called anew
+    each step, on two copies of the cache."""
+    cfg = synth.custom(2, 32, 8, 700, 20, seed=61)
+    case = Case(cfg)
+    a_cache, b_cache = case.g, _clone_cache(case.g)
+    ring_a = torch.zeros(cfg.B, cfg.Hq, 64, 128, dtype=torch.float16, device="cuda")
+    ring_b = ring_a.clone()
+    ws_a = hyq.workspace(hyq.hyq_decode_step_workspace(a_cache, 0))
+    ws_b = hyq.workspace(hyq.hyq_decode_step_workspace(b_cache, 0))
+    q = torch.empty(cfg.B, cfg.Hq, 128, dtype=torch.float16, device="cuda")
+    kd = torch.empty(cfg.B, cfg.Hkv, 128, dtype=torch.float16, device="cuda")
+    vd = torch.empty_like(kd)
+    o_a, o_b = torch.empty_like(q), torch.empty_like(q)
+    l_a = torch.empty(cfg.B, cfg.Hq, dtype=torch.float32, device="cuda")
+    l_b = torch.empty_like(l_a)
+    call = hyq.DecodeStepCall(b_cache, q, kd, vd, o_b, ws_b, q_ring=ring_b, lse=l_b)
+    for step in range(5):
+        kn, vn = synth.step_kv(cfg, step)
+        q.copy_(dev(synth.q(cfg, 900 + step)))
+        kd.copy_(dev(kn))
+        vd.copy_(dev(vn))
+        hyq.hyq_decode_step(a_cache, q, kd, vd, o_a, ws_a, q_ring=ring_a, lse=l_a)
+        call()
+        torch.cuda.synchronize()
+        assert torch.equal(o_a.view(torch.int16), o_b.view(torch.int16)), f"step {step}"
+        assert torch.equal(l_a.view(torch.int32), l_b.view(torch.int32)), f"step {step}"
+    sa, sb = _state(a_cache, ring_a), _state(b_cache, ring_b)
+    for k in sa:
+        assert np.array_equal(sa[k], sb[k]), k
