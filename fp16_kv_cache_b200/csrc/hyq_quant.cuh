@@ -57,12 +57,23 @@ __device__ __forceinline__ QuantShare quantize_share(uint4 x, int t, unsigned hm
   const float sf = __half2float(sh);
   const float zf = __half2float(zh);
 
+  // code = rne(fl(d / s)), d = fl(x - zero) >= 0, clamped to [0, 15].  Only
+  // the integer is needed: y = d * rcp(s) (rcp.approx, at most 1 ulp off,
+  // one more rounding in the product) is within 2^-18 of fl(d / s) for
+  // quotients below 16, so both round to the same integer unless y lies
+  // within 2^-16 of a half-integer; there (exact ties included) the IEEE
+  // quotient decides.  Quotients of 16 and more clamp to 15 either way.
   uint32_t c[8];
+  float rs = 0.f;
+  if (sf != 0.0f) asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rs) : "f"(sf));
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     int q = 0;
     if (sf != 0.0f) {
-      q = __float2int_rn(__fdiv_rn(__fsub_rn(v[i], zf), sf));  // ties to even
+      const float d = __fsub_rn(v[i], zf);
+      float y = __fmul_rn(d, rs);
+      if (fabsf(y - floorf(y) - 0.5f) <= 0x1p-16f) y = __fdiv_rn(d, sf);  // near a half-integer
+      q = __float2int_rn(y);  // ties to even
       q = min(max(q, 0), 15);
     }
     c[i] = static_cast<uint32_t>(q);
