@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   pdl_wait();  // the prepass is complete (and any tensor memory of earlier kernels freed)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ uint32_t tmem_base;
-  __shared__ __align__(8) uint64_t bars[2];  // [0] S MMAs, [1] P V MMAs
+  __shared__ __align__(8) uint64_t bars[1];  // each commit: P V of one job and S of the next
   __shared__ int s_abort;
   __shared__ uint32_t s_vlmask[2][2];        // bitmask words of a 64-key tile (two jobs in flight)
   __shared__ int s_vlpos[2][KT];             // positions of a vertical-line tile
@@ -347,7 +347,6 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   }
   if (tid == 0) {
     mbar_init(smem_u32(&bars[0]), 1);
-    mbar_init(smem_u32(&bars[1]), 1);
     fence_barrier_init();
     s_abort = 0;
   }
@@ -388,7 +387,7 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   const int i = q0 + rr;  // this thread's query row
   float m_run = -INFINITY, l_run = 0.f;
   bool o_started = false;   // the first P V MMA overwrites O
-  uint32_t ph_s = 0, ph_o = 0;
+  uint32_t ph = 0;
 
   // jobs: vertical-line tiles, then key tiles 0 .. last (band tiles near the diagonal)
   const int n_vlt = (n_vl + KT - 1) / KT;
@@ -461,46 +460,55 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
     }
     cp_commit();
   };
-  // Software pipeline over the single key and value buffers: the keys of
-  // job + 1 load while job's epilogue and P V run, its values while the
-  // next S and epilogue run.  cp.async groups complete in order.
+  // S = Q K^T of a job: the quantized pairs from the hi/lo operands, the
+  // high-precision pairs from the FP16 ones (issued by thread 0).
+  auto issue_s = [&](int job) {
+    int kt;
+    const int kind = job_kind(job, kt);
+    // k-step ks of a tile = its descriptor advanced by koff(R, ks) (the
+    // start-address field counts 16-byte units)
+    const uint64_t dqh = desc(s0 + OFF_QH, QT, 0), dql = desc(s0 + OFF_QL, QT, 0), dqf = desc(s0 + OFF_QF, QT, 0);
+    const uint64_t dkh = desc(s0 + OFF_KH, KT, 0), dkl = desc(s0 + OFF_KL, KT, 0), dkf = desc(s0 + OFF_KF, KT, 0);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint32_t oq = koff(QT, ks), ok = koff(KT, ks);
+      if (kind != JOB_VL) {
+        mma(tm + TM_SLO, dqh + oq, dkh + ok, idesc(KT), ks > 0);
+        mma(tm + TM_SLO, dqh + oq, dkl + ok, idesc(KT), 1u);
+        mma(tm + TM_SLO, dql + oq, dkh + ok, idesc(KT), 1u);
+      }
+      if (kind != JOB_OFF) mma(tm + TM_SHI, dqf + oq, dkf + ok, idesc(KT), ks > 0);
+    }
+  };
+  // Software pipeline over the single key and value buffers.  One commit
+  // covers P V of job - 1 and S of job; once it completes, the keys of
+  // job + 1 and the values of job load during job's epilogue, and thread 0
+  // then issues P V of job and S of job + 1 together.
   if (n_jobs > 0) {
     load_keys(0, 0);
     load_values(0);
-  }
-  for (int job = 0; job < n_jobs && !*abort; ++job) {
-    int kt;
-    const int kind = job_kind(job, kt), j0 = kt * KT, mb = job & 1;
-    cp_wait_group<1>();  // this job's keys (its values may still be in flight)
+    cp_wait_group<1>();  // the keys of job 0
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // ---- S = Q K^T
     if (tid == 0) {
-      // k-step ks of a tile = its descriptor advanced by koff(R, ks) (the
-      // start-address field counts 16-byte units)
-      const uint64_t dqh = desc(s0 + OFF_QH, QT, 0), dql = desc(s0 + OFF_QL, QT, 0), dqf = desc(s0 + OFF_QF, QT, 0);
-      const uint64_t dkh = desc(s0 + OFF_KH, KT, 0), dkl = desc(s0 + OFF_KL, KT, 0), dkf = desc(s0 + OFF_KF, KT, 0);
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t oq = koff(QT, ks), ok = koff(KT, ks);
-        if (kind != JOB_VL) {
-          mma(tm + TM_SLO, dqh + oq, dkh + ok, idesc(KT), ks > 0);
-          mma(tm + TM_SLO, dqh + oq, dkl + ok, idesc(KT), 1u);
-          mma(tm + TM_SLO, dql + oq, dkh + ok, idesc(KT), 1u);
-        }
-        if (kind != JOB_OFF) mma(tm + TM_SHI, dqf + oq, dkf + ok, idesc(KT), ks > 0);
-      }
+      issue_s(0);
       commit(smem_u32(&bars[0]));
     }
-    mma_wait(smem_u32(&bars[0]), ph_s, a, abort);
-    ph_s ^= 1u;
+  }
+  for (int job = 0; job < n_jobs && !*abort; ++job) {
+    int kt;
+    const int kind = job_kind(job, kt), j0 = kt * KT, mb = job & 1;
+    mma_wait(smem_u32(&bars[0]), ph, a, abort);
+    ph ^= 1u;
     tc_fence_after();
-    // the key buffer is free: the next job's keys load during this epilogue
-    if (job + 1 < n_jobs) load_keys(job + 1, mb ^ 1); else cp_commit();
-    // ---- epilogue: this thread's row, 64 key columns, in two passes over
-    // 32-column chunks read from tensor memory (max, then exp2 and P)
+    // S of this job and P V of the previous one are complete: the key and
+    // value buffers are free
+    if (job + 1 < n_jobs) load_keys(job + 1, mb ^ 1);
+    if (job > 0) load_values(job);
+    // ---- epilogue: this thread's row, its 32 of the tile's 64 key columns,
+    // read once from tensor memory (chunk: band and vertical-line tiles)
     auto chunk = [&](int cb, float (&x)[32], uint32_t &hmask32) {
       float lo_v[32], hi_v[32];
       if (kind != JOB_VL) tm_ld32(tm_row + TM_SLO + 32 * cb, lo_v);
@@ -531,16 +539,33 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
         x[jj] = (v == -INFINITY) ? -INFINITY : v * SCALE_LOG2;
       }
     };
+    // This thread's 32 scores of the tile, read once.  Off-diagonal tiles
+    // (all pairs quantized, the only mask the tile's vertical-line bits)
+    // keep the raw scores: scaling by SCALE_LOG2 > 0 is monotone, so the
+    // scaled max is the max scaled, and the scale folds into the exp2
+    // argument.  Band and vertical-line tiles keep x = score * SCALE_LOG2.
+    const bool off = kind == JOB_OFF;
+    float x[32];
+    uint32_t hm = 0u;
     float mx = -INFINITY;
-    {
-      float x[32];
-      uint32_t hm;
+    if (off) {
+      tm_ld32(tm_row + TM_SLO + 32 * hf, x);
+      const uint32_t vlw = s_vlmask[mb][hf];
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        if ((vlw >> jj) & 1u) x[jj] = -INFINITY;
+        mx = fmaxf(mx, x[jj]);
+      }
+      mx *= SCALE_LOG2;
+    } else {
       chunk(hf, x, hm);
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) mx = fmaxf(mx, x[jj]);
     }
+    // the two threads of a row (warps rq and rq + 4) exchange their halves'
+    // max on a 64-thread barrier of their own
     s_red[hf][rr] = mx;
-    __syncthreads();
+    asm volatile("bar.sync %0, 64;" ::"r"(1 + rq) : "memory");
     mx = fmaxf(s_red[0][rr], s_red[1][rr]);  // the same in both threads of the row
     // raise the running max only when this tile exceeds it by more than
     // RAISE (p stays <= 2^RAISE); O and l are rescaled then
@@ -571,11 +596,26 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
     }
     // P as fp16 into P_lo / P_hi: row rr, this thread's 32 columns
     float lsum = 0.f;
-    {
-      const int cb = hf;
-      float x[32];
-      uint32_t hm;
-      chunk(cb, x, hm);
+    if (off) {
+      // m_run is -inf only when every score so far, this tile's included,
+      // is masked: then every p is exp2(-inf) = 0
+      const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t wl[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c0 = 8 * cc + 2 * e;
+          const float p0 = fast_exp2(fmaf(x[c0], SCALE_LOG2, neg_m));
+          const float p1 = fast_exp2(fmaf(x[c0 + 1], SCALE_LOG2, neg_m));
+          lsum += p0 + p1;
+          wl[e] = pack_half2(p0, p1);
+        }
+        const uint32_t off_p = swz(QT, rr, 32 * hf + 8 * cc);
+        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PL + off_p), "r"(wl[0]), "r"(wl[1]),
+                     "r"(wl[2]), "r"(wl[3]) : "memory");
+      }
+    } else {
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t wl[4], wh[4];
@@ -590,22 +630,21 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
           wh[e] = pk & keep_hi;
           wl[e] = pk & ~keep_hi;
         }
-        const uint32_t off = swz(QT, rr, 32 * cb + 8 * cc);
+        const uint32_t off_p = swz(QT, rr, 32 * hf + 8 * cc);
         if (kind != JOB_VL)
-          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PL + off), "r"(wl[0]), "r"(wl[1]),
+          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PL + off_p), "r"(wl[0]), "r"(wl[1]),
                        "r"(wl[2]), "r"(wl[3]) : "memory");
-        if (kind != JOB_OFF)
-          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PH + off), "r"(wh[0]), "r"(wh[1]),
-                       "r"(wh[2]), "r"(wh[3]) : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PH + off_p), "r"(wh[0]), "r"(wh[1]),
+                     "r"(wh[2]), "r"(wh[3]) : "memory");
       }
     }
     l_run += lsum;
-    cp_wait_group<1>();  // this job's values (the next job's keys may still be in flight)
+    cp_wait_group<0>();  // this job's values and the next job's keys
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // ---- O += P_lo V^ + P_hi V
+    // ---- O += P_lo V^ + P_hi V, then S of the next job
     if (tid == 0) {
       uint32_t acc = o_started ? 1u : 0u;
       const uint64_t dpl = desc(s0 + OFF_PL, QT, 0), dph = desc(s0 + OFF_PH, QT, 0);
@@ -622,16 +661,16 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
           acc = 1u;
         }
       }
-      commit(smem_u32(&bars[1]));
+      if (job + 1 < n_jobs) issue_s(job + 1);
+      commit(smem_u32(&bars[0]));
     }
     o_started = true;
-    mma_wait(smem_u32(&bars[1]), ph_o, a, abort);
-    ph_o ^= 1u;
-    tc_fence_before();
-    __syncthreads();  // every thread saw the MMAs complete: shared tiles and O are free
+  }
+  // the last P V (nothing is in flight after an abort's timeout but what
+  // the timed-out wait gave up on)
+  if (n_jobs > 0 && !*abort) {
+    mma_wait(smem_u32(&bars[0]), ph, a, abort);
     tc_fence_after();
-    // the value buffer is free: the next job's values load during its S and epilogue
-    if (job + 1 < n_jobs) load_values(job + 1); else cp_commit();
   }
   cp_wait_group<0>();  // nothing may land in shared memory after the block exits
 
