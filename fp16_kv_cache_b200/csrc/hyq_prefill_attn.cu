@@ -407,26 +407,39 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   };
   // Loads of a job's key rows (and the tile's vertical-line bitmask or
   // positions, into mask buffer mb) as one cp.async group, and of its value
-  // tiles as another.  Rows past the end are zero-filled.
+  // tiles as another.  Rows past the end are zero-filled.  Each thread
+  // copies the same four 16-byte pieces of every tile: key rows kr + 16 it,
+  // piece kc (shared offset + 2048 it, global + 16 D it), value rows
+  // vr + 32 it, piece vc (shared offset + 4096 it, global + 32 KT it).
+  const int kr = tid >> 4, kc = tid & 15, vr = tid >> 3, vc = tid & 7;
+  const uint32_t ks_off = swz(KT, kr, 8 * kc), vs_off = swz(D, vr, 8 * vc);
+  const int kg_off = kr * D + 8 * kc, vg_off = vr * KT + 8 * vc;
   auto load_keys = [&](int job, int mb) {
     int kt;
     const int kind = job_kind(job, kt), j0 = kt * KT;
-    for (int c = tid; c < KT * 16; c += THREADS) {
-      const int r = c >> 4, cc = c & 15;
-      const uint32_t off = swz(KT, r, 8 * cc);
-      if (kind == JOB_VL) {
-        if (j0 + r < n_vl)
-          cp16(s0 + OFF_KF + off, a.vl_k + (static_cast<int64_t>(u) * a.vl_cap + j0 + r) * D + 8 * cc);
+    if (kind == JOB_VL) {
+      const __half *src = a.vl_k + (static_cast<int64_t>(u) * a.vl_cap + j0) * D + kg_off;
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        if (j0 + kr + 16 * it < n_vl)
+          cp16(s0 + OFF_KF + ks_off + 2048 * it, src + 16 * D * it);
         else
-          st_zero16(s0 + OFF_KF + off);
-      } else {
-        cp16(s0 + OFF_KH + off, khb + (j0 + r) * D + 8 * cc);  // zeros past T (prepass)
-        cp16(s0 + OFF_KL + off, klb + (j0 + r) * D + 8 * cc);
-        if (kind == JOB_BAND) {
-          if (j0 + r < T)
-            cp16(s0 + OFF_KF + off, kbase + (j0 + r) * D + 8 * cc);
+          st_zero16(s0 + OFF_KF + ks_off + 2048 * it);
+      }
+    } else {
+      const int64_t ro = static_cast<int64_t>(j0) * D + kg_off;
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {  // zeros past T (prepass)
+        cp16(s0 + OFF_KH + ks_off + 2048 * it, khb + ro + 16 * D * it);
+        cp16(s0 + OFF_KL + ks_off + 2048 * it, klb + ro + 16 * D * it);
+      }
+      if (kind == JOB_BAND) {
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+          if (j0 + kr + 16 * it < T)
+            cp16(s0 + OFF_KF + ks_off + 2048 * it, kbase + ro + 16 * D * it);
           else
-            st_zero16(s0 + OFF_KF + off);
+            st_zero16(s0 + OFF_KF + ks_off + 2048 * it);
         }
       }
     }
@@ -444,19 +457,20 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
     }
     cp_commit();
   };
-  auto load_values = [&](int job) {
+  auto load_values = [&](int job) {  // [128 ch][64 keys], zeros past the end (prepass)
     int kt;
     const int kind = job_kind(job, kt);
-    for (int c = tid; c < D * 8; c += THREADS) {  // [128 ch][64 keys], zeros past the end
-      const int r = c >> 3, cc = c & 7;
-      const uint32_t off = swz(D, r, 8 * cc);
-      if (kind == JOB_VL) {
-        cp16(s0 + OFF_VF + off, a.vlt + ((static_cast<int64_t>(u) * ((a.vl_cap + KT - 1) / KT) + kt) * D + r) * KT + 8 * cc);
-      } else {
-        const int64_t tb = (static_cast<int64_t>(u) * (a.cap / KT) + kt) * D;
-        cp16(s0 + OFF_VQ + off, a.vqt + (tb + r) * KT + 8 * cc);
-        if (kind == JOB_BAND) cp16(s0 + OFF_VF + off, a.vft + (tb + r) * KT + 8 * cc);
-      }
+    if (kind == JOB_VL) {
+      const __half *src = a.vlt + (static_cast<int64_t>(u) * ((a.vl_cap + KT - 1) / KT) + kt) * D * KT + vg_off;
+#pragma unroll
+      for (int it = 0; it < 4; ++it) cp16(s0 + OFF_VF + vs_off + 4096 * it, src + 32 * KT * it);
+    } else {
+      const int64_t tb = (static_cast<int64_t>(u) * (a.cap / KT) + kt) * D * KT + vg_off;
+#pragma unroll
+      for (int it = 0; it < 4; ++it) cp16(s0 + OFF_VQ + vs_off + 4096 * it, a.vqt + tb + 32 * KT * it);
+      if (kind == JOB_BAND)
+#pragma unroll
+        for (int it = 0; it < 4; ++it) cp16(s0 + OFF_VF + vs_off + 4096 * it, a.vft + tb + 32 * KT * it);
     }
     cp_commit();
   };
@@ -551,12 +565,15 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
     if (off) {
       tm_ld32(tm_row + TM_SLO + 32 * hf, x);
       const uint32_t vlw = s_vlmask[mb][hf];
+      if (vlw != 0u) {
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        if ((vlw >> jj) & 1u) x[jj] = -INFINITY;
-        mx = fmaxf(mx, x[jj]);
+        for (int jj = 0; jj < 32; ++jj)
+          if ((vlw >> jj) & 1u) x[jj] = -INFINITY;
       }
-      mx *= SCALE_LOG2;
+      float m4[4] = {x[0], x[1], x[2], x[3]};  // four independent chains
+#pragma unroll
+      for (int jj = 4; jj < 32; ++jj) m4[jj & 3] = fmaxf(m4[jj & 3], x[jj]);
+      mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * SCALE_LOG2;
     } else {
       chunk(hf, x, hm);
 #pragma unroll
@@ -600,6 +617,7 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
       // m_run is -inf only when every score so far, this tile's included,
       // is masked: then every p is exp2(-inf) = 0
       const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t wl[4];
@@ -608,13 +626,14 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
           const int c0 = 8 * cc + 2 * e;
           const float p0 = fast_exp2(fmaf(x[c0], SCALE_LOG2, neg_m));
           const float p1 = fast_exp2(fmaf(x[c0 + 1], SCALE_LOG2, neg_m));
-          lsum += p0 + p1;
+          l4[e] += p0 + p1;
           wl[e] = pack_half2(p0, p1);
         }
         const uint32_t off_p = swz(QT, rr, 32 * hf + 8 * cc);
         asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PL + off_p), "r"(wl[0]), "r"(wl[1]),
                      "r"(wl[2]), "r"(wl[3]) : "memory");
       }
+      lsum = (l4[0] + l4[1]) + (l4[2] + l4[3]);
     } else {
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
