@@ -43,9 +43,13 @@
 //      exceeds it by more than 8 in the exp2 domain, so the accumulator in
 //      tensor memory is rescaled rarely), writes P as fp16, and the tensor
 //      cores accumulate O += P_lo V^ + P_hi V.  Key tiles: the vertical-line
-//      rows (FP16, pairs with j <= i - 128), then positions 0.. in order;
-//      the four tiles around the diagonal are band tiles, the others hold
-//      quantized pairs only (their vertical lines are masked out there).
+//      rows (FP16, pairs with j <= i - 128) and the band tiles around the
+//      diagonal first (phase A, one key, value and score buffer), then the
+//      off-diagonal tiles, which hold quantized pairs only (their vertical
+//      lines are masked out there): in phase B the space of phase A's FP16
+//      tiles double-buffers keys, values and scores, and the scores of tile
+//      t + 1 and P V of tile t - 1 run on the tensor cores during tile t's
+//      epilogue.
 //   Output: O fp32 (the operands are already rounded to fp16 for the tensor
 //   cores; an fp16 output rounding would spend the rest of the tolerance)
 //   and the row's log-sum-exp.
@@ -62,7 +66,9 @@ namespace pa {
 
 constexpr int QT = 128;      // query rows per tile (the MMA's M)
 constexpr int KT = 64;       // keys per tile (N of Q K^T, K of P V)
-constexpr int THREADS = 256;  // two threads per query row
+constexpr int EPI_THREADS = 256;          // the epilogue warps: two threads per query row
+constexpr int THREADS = EPI_THREADS + 32;  // and one warp that issues the MMAs
+constexpr int ISSUER = EPI_THREADS;       // the thread that issues and commits every MMA
 constexpr float SCALE_LOG2 = 0.12751743082459868f;  // log2(e) / sqrt(128)
 constexpr float LN2 = 0.69314718055994531f;
 constexpr float RAISE = 8.f;  // raise the running max only past this margin (exp2 domain)
@@ -314,12 +320,14 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   pdl_wait();  // the prepass is complete (and any tensor memory of earlier kernels freed)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ uint32_t tmem_base;
-  __shared__ __align__(8) uint64_t bars[1];  // each commit: P V of one job and S of the next
+  __shared__ __align__(8) uint64_t bars[1];  // phase A: each commit is P V of one job and S of the next
+  __shared__ __align__(8) uint64_t bars_b[3];  // phase B: S into score buffer 0, 1; P V
   __shared__ int s_abort;
-  __shared__ uint32_t s_vlmask[2][2];        // bitmask words of a 64-key tile (two jobs in flight)
+  __shared__ uint32_t s_vlmask[3][2];        // bitmask words of a 64-key tile (up to three jobs in flight)
   __shared__ int s_vlpos[2][KT];             // positions of a vertical-line tile
   __shared__ float s_red[2][QT];             // the two halves' tile max (and, at the end, row sums)
   const int tid = threadIdx.x, warp = tid >> 5;
+  const bool ep = tid < EPI_THREADS;  // an epilogue thread (else the issuer's warp)
   const int BH = a.B * a.Hq;
   const int n_qt = a.cap / QT;
   const int qt = n_qt - 1 - static_cast<int>(blockIdx.x) / BH;  // longest tiles first
@@ -347,6 +355,8 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   }
   if (tid == 0) {
     mbar_init(smem_u32(&bars[0]), 1);
+#pragma unroll
+    for (int t = 0; t < 3; ++t) mbar_init(smem_u32(&bars_b[t]), 1);
     fence_barrier_init();
     s_abort = 0;
   }
@@ -389,21 +399,27 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   bool o_started = false;   // the first P V MMA overwrites O
   uint32_t ph = 0;
 
-  // jobs: vertical-line tiles, then key tiles 0 .. last (band tiles near the diagonal)
+  // Phase A: the vertical-line tiles, then the band tiles band0 .. n_kt - 1
+  // near the diagonal (the jobs with high-precision pairs).  Phase B: the
+  // off-diagonal key tiles 0 .. band0 - 1 (quantized pairs only), with the
+  // FP16 tiles of phase A dead, so that their space double-buffers keys,
+  // values and scores.  The softmax is the same in any order of key tiles.
   const int n_vlt = (n_vl + KT - 1) / KT;
   const int last_key = min(q0 + QT, T) - 1;
   const int n_kt = last_key / KT + 1;
   const int band0 = max(0, (q0 - a.W + 1) / KT);  // first key tile holding a pair j > i - W
-  const int n_jobs = n_vlt + n_kt;
+  const int n_jobs = n_vlt + (n_kt - band0);      // phase A
+  const int n_off = band0;                        // phase B
   const __half *kbase = a.k + static_cast<int64_t>(u) * a.cap * D;
   const __half *khb = a.kh + static_cast<int64_t>(u) * a.cap * D;
   const __half *klb = a.kl + static_cast<int64_t>(u) * a.cap * D;
 
-  // Job j: the vertical-line tile j (j < n_vlt) or key tile j - n_vlt.
+  // Phase A job j: the vertical-line tile j (j < n_vlt) or band key tile
+  // band0 + j - n_vlt.
   auto job_kind = [&](int job, int &kt) {
     const bool is_vl = job < n_vlt;
-    kt = is_vl ? job : job - n_vlt;
-    return is_vl ? JOB_VL : (kt >= band0 ? JOB_BAND : JOB_OFF);
+    kt = is_vl ? job : band0 + job - n_vlt;
+    return is_vl ? JOB_VL : JOB_BAND;
   };
   // Loads of a job's key rows (and the tile's vertical-line bitmask or
   // positions, into mask buffer mb) as one cp.async group, and of its value
@@ -475,7 +491,7 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
     cp_commit();
   };
   // S = Q K^T of a job: the quantized pairs from the hi/lo operands, the
-  // high-precision pairs from the FP16 ones (issued by thread 0).
+  // high-precision pairs from the FP16 ones (issued by thread ISSUER).
   auto issue_s = [&](int job) {
     int kt;
     const int kind = job_kind(job, kt);
@@ -496,17 +512,21 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   };
   // Software pipeline over the single key and value buffers.  One commit
   // covers P V of job - 1 and S of job; once it completes, the keys of
-  // job + 1 and the values of job load during job's epilogue, and thread 0
-  // then issues P V of job and S of job + 1 together.
+  // job + 1 and the values of job load during job's epilogue, and after the
+  // block barrier thread ISSUER (in a warp of its own, so the epilogue
+  // warps never wait for the tensor cores to accept MMAs) issues P V of job
+  // and S of job + 1 together.
   if (n_jobs > 0) {
-    load_keys(0, 0);
-    load_values(0);
-    cp_wait_group<1>();  // the keys of job 0
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (ep) {
+      load_keys(0, 0);
+      load_values(0);
+      cp_wait_group<1>();  // the keys of job 0
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid == 0) {
+    if (tid == ISSUER) {
       issue_s(0);
       commit(smem_u32(&bars[0]));
     }
@@ -514,157 +534,159 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   for (int job = 0; job < n_jobs && !*abort; ++job) {
     int kt;
     const int kind = job_kind(job, kt), j0 = kt * KT, mb = job & 1;
-    mma_wait(smem_u32(&bars[0]), ph, a, abort);
-    ph ^= 1u;
-    tc_fence_after();
-    // S of this job and P V of the previous one are complete: the key and
-    // value buffers are free
-    if (job + 1 < n_jobs) load_keys(job + 1, mb ^ 1);
-    if (job > 0) load_values(job);
-    // ---- epilogue: this thread's row, its 32 of the tile's 64 key columns,
-    // read once from tensor memory (chunk: band and vertical-line tiles)
-    auto chunk = [&](int cb, float (&x)[32], uint32_t &hmask32) {
-      float lo_v[32], hi_v[32];
-      if (kind != JOB_VL) tm_ld32(tm_row + TM_SLO + 32 * cb, lo_v);
-      if (kind != JOB_OFF) tm_ld32(tm_row + TM_SHI + 32 * cb, hi_v);
-      const uint32_t vlw = (kind != JOB_VL) ? s_vlmask[mb][cb] : 0u;
-      hmask32 = 0u;
+    if (ep) {  // the issuer's warp skips to the barrier below
+      mma_wait(smem_u32(&bars[0]), ph, a, abort);
+      ph ^= 1u;
+      tc_fence_after();
+      // S of this job and P V of the previous one are complete: the key and
+      // value buffers are free
+      if (job + 1 < n_jobs) load_keys(job + 1, mb ^ 1);
+      if (job > 0) load_values(job);
+      // ---- epilogue: this thread's row, its 32 of the tile's 64 key columns,
+      // read once from tensor memory (chunk: band and vertical-line tiles)
+      auto chunk = [&](int cb, float (&x)[32], uint32_t &hmask32) {
+        float lo_v[32], hi_v[32];
+        if (kind != JOB_VL) tm_ld32(tm_row + TM_SLO + 32 * cb, lo_v);
+        if (kind != JOB_OFF) tm_ld32(tm_row + TM_SHI + 32 * cb, hi_v);
+        const uint32_t vlw = (kind != JOB_VL) ? s_vlmask[mb][cb] : 0u;
+        hmask32 = 0u;
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        const int c = 32 * cb + jj, j = j0 + c;
-        float v = -INFINITY;
-        if (kind == JOB_VL) {
-          // vertical line j of the unit: counted here when it lies outside
-          // the query's window (inside it, the band tile has it)
-          if (j < n_vl && s_vlpos[mb][c] <= i - a.W) {
-            v = hi_v[jj];
-            hmask32 |= 1u << jj;
+        for (int jj = 0; jj < 32; ++jj) {
+          const int c = 32 * cb + jj, j = j0 + c;
+          float v = -INFINITY;
+          if (kind == JOB_VL) {
+            // vertical line j of the unit: counted here when it lies outside
+            // the query's window (inside it, the band tile has it)
+            if (j < n_vl && s_vlpos[mb][c] <= i - a.W) {
+              v = hi_v[jj];
+              hmask32 |= 1u << jj;
+            }
+          } else if (kind == JOB_OFF) {
+            if (!((vlw >> jj) & 1u)) v = lo_v[jj];
+          } else if (j <= i) {
+            if (j > i - a.W) {
+              v = hi_v[jj];
+              hmask32 |= 1u << jj;
+            } else if (!((vlw >> jj) & 1u)) {
+              v = lo_v[jj];
+            }
           }
-        } else if (kind == JOB_OFF) {
-          if (!((vlw >> jj) & 1u)) v = lo_v[jj];
-        } else if (j <= i) {
-          if (j > i - a.W) {
-            v = hi_v[jj];
-            hmask32 |= 1u << jj;
-          } else if (!((vlw >> jj) & 1u)) {
-            v = lo_v[jj];
-          }
+          x[jj] = (v == -INFINITY) ? -INFINITY : v * SCALE_LOG2;
         }
-        x[jj] = (v == -INFINITY) ? -INFINITY : v * SCALE_LOG2;
-      }
-    };
-    // This thread's 32 scores of the tile, read once.  Off-diagonal tiles
-    // (all pairs quantized, the only mask the tile's vertical-line bits)
-    // keep the raw scores: scaling by SCALE_LOG2 > 0 is monotone, so the
-    // scaled max is the max scaled, and the scale folds into the exp2
-    // argument.  Band and vertical-line tiles keep x = score * SCALE_LOG2.
-    const bool off = kind == JOB_OFF;
-    float x[32];
-    uint32_t hm = 0u;
-    float mx = -INFINITY;
-    if (off) {
-      tm_ld32(tm_row + TM_SLO + 32 * hf, x);
-      const uint32_t vlw = s_vlmask[mb][hf];
-      if (vlw != 0u) {
+      };
+      // This thread's 32 scores of the tile, read once.  Off-diagonal tiles
+      // (all pairs quantized, the only mask the tile's vertical-line bits)
+      // keep the raw scores: scaling by SCALE_LOG2 > 0 is monotone, so the
+      // scaled max is the max scaled, and the scale folds into the exp2
+      // argument.  Band and vertical-line tiles keep x = score * SCALE_LOG2.
+      const bool off = kind == JOB_OFF;
+      float x[32];
+      uint32_t hm = 0u;
+      float mx = -INFINITY;
+      if (off) {
+        tm_ld32(tm_row + TM_SLO + 32 * hf, x);
+        const uint32_t vlw = s_vlmask[mb][hf];
+        if (vlw != 0u) {
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj)
-          if ((vlw >> jj) & 1u) x[jj] = -INFINITY;
-      }
-      float m4[4] = {x[0], x[1], x[2], x[3]};  // four independent chains
+          for (int jj = 0; jj < 32; ++jj)
+            if ((vlw >> jj) & 1u) x[jj] = -INFINITY;
+        }
+        float m4[4] = {x[0], x[1], x[2], x[3]};  // four independent chains
 #pragma unroll
-      for (int jj = 4; jj < 32; ++jj) m4[jj & 3] = fmaxf(m4[jj & 3], x[jj]);
-      mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * SCALE_LOG2;
-    } else {
-      chunk(hf, x, hm);
+        for (int jj = 4; jj < 32; ++jj) m4[jj & 3] = fmaxf(m4[jj & 3], x[jj]);
+        mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * SCALE_LOG2;
+      } else {
+        chunk(hf, x, hm);
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) mx = fmaxf(mx, x[jj]);
-    }
-    // the two threads of a row (warps rq and rq + 4) exchange their halves'
-    // max on a 64-thread barrier of their own
-    s_red[hf][rr] = mx;
-    asm volatile("bar.sync %0, 64;" ::"r"(1 + rq) : "memory");
-    mx = fmaxf(s_red[0][rr], s_red[1][rr]);  // the same in both threads of the row
-    // raise the running max only when this tile exceeds it by more than
-    // RAISE (p stays <= 2^RAISE); O and l are rescaled then
-    float alpha = 1.f;
-    bool rescale = false;
-    if (mx > m_run + RAISE || (m_run == -INFINITY && mx != -INFINITY)) {
-      const float m_new = mx;
-      if (m_run != -INFINITY) {
-        alpha = fast_exp2(m_run - m_new);
-        rescale = o_started;
+        for (int jj = 0; jj < 32; ++jj) mx = fmaxf(mx, x[jj]);
       }
-      l_run *= alpha;
-      m_run = m_new;
-    }
-    // O row *= alpha (the previous P V MMAs are complete); tensor-memory
-    // loads and stores take the whole warp, so a warp with any row to
-    // rescale rescales all of its rows (by 1 where nothing changed)
-    if (__any_sync(0xffffffffu, rescale)) {
-      const float f = rescale ? alpha : 1.f;
+      // the two threads of a row (warps rq and rq + 4) exchange their halves'
+      // max on a 64-thread barrier of their own
+      s_red[hf][rr] = mx;
+      asm volatile("bar.sync %0, 64;" ::"r"(1 + rq) : "memory");
+      mx = fmaxf(s_red[0][rr], s_red[1][rr]);  // the same in both threads of the row
+      // raise the running max only when this tile exceeds it by more than
+      // RAISE (p stays <= 2^RAISE); O and l are rescaled then
+      float alpha = 1.f;
+      bool rescale = false;
+      if (mx > m_run + RAISE || (m_run == -INFINITY && mx != -INFINITY)) {
+        const float m_new = mx;
+        if (m_run != -INFINITY) {
+          alpha = fast_exp2(m_run - m_new);
+          rescale = o_started;
+        }
+        l_run *= alpha;
+        m_run = m_new;
+      }
+      // O row *= alpha (the previous P V MMAs are complete); tensor-memory
+      // loads and stores take the whole warp, so a warp with any row to
+      // rescale rescales all of its rows (by 1 where nothing changed)
+      if (__any_sync(0xffffffffu, rescale)) {
+        const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
-      for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {  // this thread's half of the row
-        float ov[32];
-        tm_ld32(tm_row + TM_O + 32 * cb, ov);
+        for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {  // this thread's half of the row
+          float ov[32];
+          tm_ld32(tm_row + TM_O + 32 * cb, ov);
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) ov[jj] *= f;
-        tm_st32(tm_row + TM_O + 32 * cb, ov);
-      }
-    }
-    // P as fp16 into P_lo / P_hi: row rr, this thread's 32 columns
-    float lsum = 0.f;
-    if (off) {
-      // m_run is -inf only when every score so far, this tile's included,
-      // is masked: then every p is exp2(-inf) = 0
-      const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-      float l4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t wl[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c0 = 8 * cc + 2 * e;
-          const float p0 = fast_exp2(fmaf(x[c0], SCALE_LOG2, neg_m));
-          const float p1 = fast_exp2(fmaf(x[c0 + 1], SCALE_LOG2, neg_m));
-          l4[e] += p0 + p1;
-          wl[e] = pack_half2(p0, p1);
+          for (int jj = 0; jj < 32; ++jj) ov[jj] *= f;
+          tm_st32(tm_row + TM_O + 32 * cb, ov);
         }
-        const uint32_t off_p = swz(QT, rr, 32 * hf + 8 * cc);
-        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PL + off_p), "r"(wl[0]), "r"(wl[1]),
-                     "r"(wl[2]), "r"(wl[3]) : "memory");
       }
-      lsum = (l4[0] + l4[1]) + (l4[2] + l4[3]);
-    } else {
+      // P as fp16 into P_lo / P_hi: row rr, this thread's 32 columns
+      float lsum = 0.f;
+      if (off) {
+        // m_run is -inf only when every score so far, this tile's included,
+        // is masked: then every p is exp2(-inf) = 0
+        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+        float l4[4] = {0.f, 0.f, 0.f, 0.f};  // four independent chains
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t wl[4], wh[4];
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t wl[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c0 = 8 * cc + 2 * e;
-          const float p0 = (x[c0] == -INFINITY) ? 0.f : fast_exp2(x[c0] - m_run);
-          const float p1 = (x[c0 + 1] == -INFINITY) ? 0.f : fast_exp2(x[c0 + 1] - m_run);
-          lsum += p0 + p1;
-          const uint32_t pk = pack_half2(p0, p1);
-          const uint32_t keep_hi = (((hm >> c0) & 1u) ? 0x0000FFFFu : 0u) | (((hm >> (c0 + 1)) & 1u) ? 0xFFFF0000u : 0u);
-          wh[e] = pk & keep_hi;
-          wl[e] = pk & ~keep_hi;
-        }
-        const uint32_t off_p = swz(QT, rr, 32 * hf + 8 * cc);
-        if (kind != JOB_VL)
+          for (int e = 0; e < 4; ++e) {
+            const int c0 = 8 * cc + 2 * e;
+            const float p0 = fast_exp2(fmaf(x[c0], SCALE_LOG2, neg_m));
+            const float p1 = fast_exp2(fmaf(x[c0 + 1], SCALE_LOG2, neg_m));
+            l4[e] += p0 + p1;
+            wl[e] = pack_half2(p0, p1);
+          }
+          const uint32_t off_p = swz(QT, rr, 32 * hf + 8 * cc);
           asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PL + off_p), "r"(wl[0]), "r"(wl[1]),
                        "r"(wl[2]), "r"(wl[3]) : "memory");
-        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PH + off_p), "r"(wh[0]), "r"(wh[1]),
-                     "r"(wh[2]), "r"(wh[3]) : "memory");
+        }
+        lsum = (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t wl[4], wh[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c0 = 8 * cc + 2 * e;
+            const float p0 = (x[c0] == -INFINITY) ? 0.f : fast_exp2(x[c0] - m_run);
+            const float p1 = (x[c0 + 1] == -INFINITY) ? 0.f : fast_exp2(x[c0 + 1] - m_run);
+            lsum += p0 + p1;
+            const uint32_t pk = pack_half2(p0, p1);
+            const uint32_t keep_hi = (((hm >> c0) & 1u) ? 0x0000FFFFu : 0u) | (((hm >> (c0 + 1)) & 1u) ? 0xFFFF0000u : 0u);
+            wh[e] = pk & keep_hi;
+            wl[e] = pk & ~keep_hi;
+          }
+          const uint32_t off_p = swz(QT, rr, 32 * hf + 8 * cc);
+          if (kind != JOB_VL)
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PL + off_p), "r"(wl[0]), "r"(wl[1]),
+                         "r"(wl[2]), "r"(wl[3]) : "memory");
+          asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PH + off_p), "r"(wh[0]), "r"(wh[1]),
+                       "r"(wh[2]), "r"(wh[3]) : "memory");
+        }
       }
+      l_run += lsum;
+      cp_wait_group<0>();  // this job's values and the next job's keys
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    l_run += lsum;
-    cp_wait_group<0>();  // this job's values and the next job's keys
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     // ---- O += P_lo V^ + P_hi V, then S of the next job
-    if (tid == 0) {
+    if (tid == ISSUER) {
       uint32_t acc = o_started ? 1u : 0u;
       const uint64_t dpl = desc(s0 + OFF_PL, QT, 0), dph = desc(s0 + OFF_PH, QT, 0);
       const uint64_t dvq = desc(s0 + OFF_VQ, D, 0), dvf = desc(s0 + OFF_VF, D, 0);
@@ -687,35 +709,209 @@ __global__ void __launch_bounds__(THREADS, 1) pa_attn_kernel(const Args a) {
   }
   // the last P V (nothing is in flight after an abort's timeout but what
   // the timed-out wait gave up on)
-  if (n_jobs > 0 && !*abort) {
+  if (ep && n_jobs > 0 && !*abort) {
     mma_wait(smem_u32(&bars[0]), ph, a, abort);
     tc_fence_after();
+  }
+
+  // ---- Phase B: off-diagonal key tile t (t < n_off) uses key buffer t & 1
+  // (K^hi, K^lo at OFF_KH, OFF_KL or in the dead Q region), value buffer
+  // t & 1 (OFF_VQ or the dead OFF_VF), score buffer t & 1 (tensor-memory
+  // columns TM_SLO or the dead TM_SHI) and mask slot t % 3.  S of tile t + 2
+  // is issued as soon as tile t's scores have been read, so the tensor cores
+  // compute P V of tile t - 1 and S of tile t + 1 during tile t's epilogue.
+  // P V and S are committed to barriers of their own: the epilogue waits
+  // for P V of the previous tile only before it rescales O or writes P.
+  auto kbuf_h = [&](int t) { return s0 + ((t & 1) ? OFF_QF : OFF_KH); };
+  auto kbuf_l = [&](int t) { return s0 + ((t & 1) ? OFF_QF + TILE_K : OFF_KL); };
+  auto vbuf = [&](int t) { return s0 + ((t & 1) ? OFF_VF : OFF_VQ); };
+  auto load_keys_b = [&](int t) {
+    const int j0 = t * KT;
+    const int64_t ro = static_cast<int64_t>(j0) * D + kg_off;
+    const uint32_t dh = kbuf_h(t) + ks_off, dl = kbuf_l(t) + ks_off;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      cp16(dh + 2048 * it, khb + ro + 16 * D * it);
+      cp16(dl + 2048 * it, klb + ro + 16 * D * it);
+    }
+    if (tid < 2) {
+      if (j0 + 32 * tid < T)
+        cp4(smem_u32(&s_vlmask[t % 3][tid]), a.blocks + rec_mask(a.rm.rec_rd(u, j0 + 32 * tid)));
+      else
+        s_vlmask[t % 3][tid] = 0u;
+    }
+    cp_commit();
+  };
+  auto load_values_b = [&](int t) {
+    const int64_t tb = (static_cast<int64_t>(u) * (a.cap / KT) + t) * D * KT + vg_off;
+    const uint32_t dv = vbuf(t) + vs_off;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) cp16(dv + 4096 * it, a.vqt + tb + 32 * KT * it);
+    cp_commit();
+  };
+  auto issue_s_b = [&](int t) {  // thread ISSUER
+    const uint64_t dqh = desc(s0 + OFF_QH, QT, 0), dql = desc(s0 + OFF_QL, QT, 0);
+    const uint64_t dkh = desc(kbuf_h(t), KT, 0), dkl = desc(kbuf_l(t), KT, 0);
+    const uint32_t d = tm + ((t & 1) ? TM_SHI : TM_SLO);
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      const uint32_t oq = koff(QT, ks), ok = koff(KT, ks);
+      mma(d, dqh + oq, dkh + ok, idesc(KT), ks > 0);
+      mma(d, dqh + oq, dkl + ok, idesc(KT), 1u);
+      mma(d, dql + oq, dkh + ok, idesc(KT), 1u);
+    }
+  };
+  if (n_off > 0 && !*abort) {
+    if (ep) {
+      load_keys_b(0);
+      load_values_b(0);
+      if (n_off > 1) load_keys_b(1); else cp_commit();
+      cp_wait_group<0>();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == ISSUER) {
+      issue_s_b(0);
+      commit(smem_u32(&bars_b[0]));
+      if (n_off > 1) {
+        issue_s_b(1);
+        commit(smem_u32(&bars_b[1]));
+      }
+    }
+    uint32_t ph_s0 = 0u, ph_s1 = 0u, ph_o = 0u;  // bars_b[0], [1], [2]
+    for (int t = 0; t < n_off && !*abort; ++t) {
+      const int sb = t & 1;
+      if (ep) {  // the issuer's warp skips to the barrier below
+        mma_wait(smem_u32(&bars_b[sb]), sb ? ph_s1 : ph_s0, a, abort);
+        if (sb) ph_s1 ^= 1u; else ph_s0 ^= 1u;
+        tc_fence_after();
+        // S of tile t is complete: its key buffer takes tile t + 2
+        if (t + 2 < n_off) load_keys_b(t + 2); else cp_commit();
+        // the raw scores of this thread's 32 columns, masked by the tile's
+        // vertical-line bits; the scale folds into the exp2 argument
+        float x[32];
+        tm_ld32(tm_row + (sb ? TM_SHI : TM_SLO) + 32 * hf, x);
+        const uint32_t vlw = s_vlmask[t % 3][hf];
+        if (vlw != 0u) {
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj)
+            if ((vlw >> jj) & 1u) x[jj] = -INFINITY;
+        }
+        float mx;
+        {
+          float m4[4] = {x[0], x[1], x[2], x[3]};  // four independent chains
+#pragma unroll
+          for (int jj = 4; jj < 32; ++jj) m4[jj & 3] = fmaxf(m4[jj & 3], x[jj]);
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * SCALE_LOG2;
+        }
+        s_red[hf][rr] = mx;
+        asm volatile("bar.sync %0, 64;" ::"r"(1 + rq) : "memory");
+        mx = fmaxf(s_red[0][rr], s_red[1][rr]);
+        // P V of tile t - 1 is complete: O may be rescaled, P overwritten, and
+        // its value buffer takes tile t + 1
+        if (t > 0) {
+          mma_wait(smem_u32(&bars_b[2]), ph_o, a, abort);
+          ph_o ^= 1u;
+          tc_fence_after();
+        }
+        if (t + 1 < n_off) load_values_b(t + 1); else cp_commit();
+        float alpha = 1.f;
+        bool rescale = false;
+        if (mx > m_run + RAISE || (m_run == -INFINITY && mx != -INFINITY)) {
+          const float m_new = mx;
+          if (m_run != -INFINITY) {
+            alpha = fast_exp2(m_run - m_new);
+            rescale = o_started;
+          }
+          l_run *= alpha;
+          m_run = m_new;
+        }
+        if (__any_sync(0xffffffffu, rescale)) {
+          const float f = rescale ? alpha : 1.f;
+#pragma unroll 1
+          for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
+            float ov[32];
+            tm_ld32(tm_row + TM_O + 32 * cb, ov);
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) ov[jj] *= f;
+            tm_st32(tm_row + TM_O + 32 * cb, ov);
+          }
+        }
+        {
+          const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+          float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t wl[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c0 = 8 * cc + 2 * e;
+              const float p0 = fast_exp2(fmaf(x[c0], SCALE_LOG2, neg_m));
+              const float p1 = fast_exp2(fmaf(x[c0 + 1], SCALE_LOG2, neg_m));
+              l4[e] += p0 + p1;
+              wl[e] = pack_half2(p0, p1);
+            }
+            asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(s0 + OFF_PL + swz(QT, rr, 32 * hf + 8 * cc)),
+                         "r"(wl[0]), "r"(wl[1]), "r"(wl[2]), "r"(wl[3]) : "memory");
+          }
+          l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        }
+        cp_wait_group<1>();  // this tile's values and the keys of tile t + 2
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (tid == ISSUER) {
+        uint32_t acc = o_started ? 1u : 0u;
+        const uint64_t dpl = desc(s0 + OFF_PL, QT, 0), dv = desc(vbuf(t), D, 0);
+#pragma unroll
+        for (int ks = 0; ks < KT / 16; ++ks) {
+          mma(tm + TM_O, dpl + koff(QT, ks), dv + koff(D, ks), idesc(D), acc);
+          acc = 1u;
+        }
+        commit(smem_u32(&bars_b[2]));
+        if (t + 2 < n_off) {
+          issue_s_b(t + 2);
+          commit(smem_u32(&bars_b[sb]));
+        }
+      }
+      o_started = true;
+    }
+    if (ep && !*abort) {
+      mma_wait(smem_u32(&bars_b[2]), ph_o, a, abort);
+      tc_fence_after();
+    }
   }
   cp_wait_group<0>();  // nothing may land in shared memory after the block exits
 
   // ---- O / l and the log-sum-exp of row i (the row's sum is the two halves')
-  s_red[hf][rr] = l_run;
+  if (ep) s_red[hf][rr] = l_run;
   __syncthreads();
-  l_run = s_red[0][rr] + s_red[1][rr];
-  if (!*abort && o_started) {  // uniform: the tensor-memory loads take the whole warp
-    const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
-    float *orow = a.o + (static_cast<int64_t>(bh) * a.cap + i) * D;
+  if (ep) {
+    l_run = s_red[0][rr] + s_red[1][rr];
+    if (!*abort && o_started) {  // uniform: the tensor-memory loads take the whole warp
+      const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      float *orow = a.o + (static_cast<int64_t>(bh) * a.cap + i) * D;
 #pragma unroll
-    for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
-      float ov[32];
-      tm_ld32(tm_row + TM_O + 32 * cb, ov);
-      if (i < T)
+      for (int cb = 2 * hf; cb < 2 * hf + 2; ++cb) {
+        float ov[32];
+        tm_ld32(tm_row + TM_O + 32 * cb, ov);
+        if (i < T)
 #pragma unroll
-        for (int jj = 0; jj < 32; jj += 4)
-          *reinterpret_cast<float4 *>(orow + 32 * cb + jj) =
-              make_float4(ov[jj] * inv, ov[jj + 1] * inv, ov[jj + 2] * inv, ov[jj + 3] * inv);
+          for (int jj = 0; jj < 32; jj += 4)
+            *reinterpret_cast<float4 *>(orow + 32 * cb + jj) =
+                make_float4(ov[jj] * inv, ov[jj + 1] * inv, ov[jj + 2] * inv, ov[jj + 3] * inv);
+      }
+      if (a.lse && i < T && hf == 0) a.lse[static_cast<int64_t>(bh) * a.cap + i] = (m_run + __log2f(l_run)) * LN2;
+    } else if (o_started && i < T) {
+      // a wait ran out: the row is undefined; leave a recognisable value
+      if (a.lse) a.lse[static_cast<int64_t>(bh) * a.cap + i] = __int_as_float(0x7fc00000);
+    } else if (!o_started && i < T) {
+      if (a.lse) a.lse[static_cast<int64_t>(bh) * a.cap + i] = -INFINITY;
     }
-    if (a.lse && i < T && hf == 0) a.lse[static_cast<int64_t>(bh) * a.cap + i] = (m_run + __log2f(l_run)) * LN2;
-  } else if (o_started && i < T) {
-    // a wait ran out: the row is undefined; leave a recognisable value
-    if (a.lse) a.lse[static_cast<int64_t>(bh) * a.cap + i] = __int_as_float(0x7fc00000);
-  } else if (!o_started && i < T) {
-    if (a.lse) a.lse[static_cast<int64_t>(bh) * a.cap + i] = -INFINITY;
   }
   tc_fence_before();
   __syncthreads();
