@@ -88,6 +88,7 @@ __device__ __forceinline__ int sel_T(const SelectArgs &a, int u) { return a.seq_
 // accumulators with tcgen05.ld: warp w owns rows 32 (w % 4) .. + 31 of each
 // row block and columns 64 (w / 4) .. + 63 of the sub-tile.
 constexpr int TC_THREADS = 512;  // 16 warps: 4 lane quadrants x 4 column quarters
+constexpr int TC_BLOCK = TC_THREADS + 32;  // and one warp that issues the MMAs
 constexpr int TC_NK = 128;               // keys per sub-tile
 constexpr int TC_TILE = TC_NK * 256;     // bytes of a [128][128] fp16 tile
 constexpr int TC_MAX_RB = SEL_MAX_ROWS / 128;
@@ -280,8 +281,11 @@ __device__ __forceinline__ SelItem sel_item(const SelectArgs &a, int item) {
 //   * warps 0-7 stage key sub-tiles of 128 keys into shared memory (thread s
 //     writes key row s % 128, quantization groups s / 128 and s / 128 + 2),
 //     loading the next sub-tile from global memory while the current one is
-//     written; once all 256 staging threads have arrived on a sub-tile's
-//     barrier, thread 0 issues its MMAs and commits them;
+//     written;
+//   * warp 16 (one thread) waits until all 256 staging threads have arrived
+//     on a sub-tile's barrier and the epilogue is done with the accumulator
+//     set, then issues the sub-tile's MMAs and commits them, so no staging
+//     warp waits for the tensor cores to accept MMAs;
 //   * warps 8-15 read the accumulators the MMAs complete (lane quadrant
 //     w % 4, one half of the columns of every row block) and run the exp2
 //     epilogue.
@@ -296,7 +300,7 @@ __device__ __forceinline__ SelItem sel_item(const SelectArgs &a, int item) {
 constexpr int TC_ROLE = TC_THREADS / 2;  // threads per role
 
 template <bool CACHE, int PASS>
-__global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a) {
+__global__ void __launch_bounds__(TC_BLOCK, 1) score_kernel(const SelectArgs a) {
   pdl_trigger();  // the next kernel may be scheduled
   pdl_wait();     // earlier work on the stream is complete and visible (and its tensor memory freed)
   extern __shared__ __align__(1024) uint8_t sm_raw[];
@@ -393,7 +397,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> the tensor core
         mbar_arrive(smem_u32(&key_full[buf]));
-        if (tid == 0 && wait(&key_full[buf], ph) && (g < nbuf || wait(&acc_empty[buf], ph ^ 1))) {
+      }
+      gst += s.nsub;
+    }
+  } else if (warp == TC_THREADS / 32) {
+    // ---- MMA issue: sub-tile g once it is staged and accumulator set g % nbuf is free
+    if (lane == 0) {
+      int gst = 0;
+      for (int item = it0; item < it1; ++item) {
+        const SelItem s = sel_item<PASS>(a, item);
+        if (s.nsub == 0) continue;
+        for (int st = 0; st < s.nsub; ++st) {
+          const int g = gst + st, buf = g % nbuf;
+          const uint32_t ph = (g / nbuf) & 1;
+          if (!wait(&key_full[buf], ph) || (g >= nbuf && !wait(&acc_empty[buf], ph ^ 1))) continue;
+          uint8_t *kb = sK + buf * KT;
           // every staging thread has written sub-tile g, and the epilogue is done with accumulator set buf
           tc_fence_after();
           // descriptors of k-step 0; k-step ks adds sw128_koff(ks) to the
@@ -419,8 +437,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) score_kernel(const SelectArgs a
                            smem_u32(&acc_full[buf]))
                        : "memory");
         }
+        gst += s.nsub;
       }
-      gst += s.nsub;
     }
   } else {
     // ---- epilogue: TMEM lane quadrant qd, column half hf of every row block
@@ -1099,12 +1117,12 @@ static cudaError_t select_launch(const SelectArgs &a, bool cache, cudaStream_t s
   cudaError_t e;
   if (cache) {
     e = launch(rank_kernel, dim3(a.U), dim3(1024), 0, s, a);
-    if (e == cudaSuccess) e = launch(score_kernel<true, 1>, grid, dim3(TC_THREADS), smem, s, a);
+    if (e == cudaSuccess) e = launch(score_kernel<true, 1>, grid, dim3(TC_BLOCK), smem, s, a);
   } else {
-    e = launch(score_kernel<false, 1>, grid, dim3(TC_THREADS), smem, s, a);
+    e = launch(score_kernel<false, 1>, grid, dim3(TC_BLOCK), smem, s, a);
   }
   if (e == cudaSuccess) e = launch(stats_merge_kernel, dim3(a.U), dim3(256), 0, s, a);
-  if (e == cudaSuccess) e = launch(cache ? score_kernel<true, 2> : score_kernel<false, 2>, grid, dim3(TC_THREADS), smem, s, a);
+  if (e == cudaSuccess) e = launch(cache ? score_kernel<true, 2> : score_kernel<false, 2>, grid, dim3(TC_BLOCK), smem, s, a);
   const int tkc_vals = topk_cluster_vals(a, sms);
   if (e == cudaSuccess)
     e = tkc_vals > 0 ? launch_topk_cluster(a, tkc_vals, s)
