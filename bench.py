@@ -683,9 +683,9 @@ def run_e2e(torch, hyq, cfg, layers, rings, dws, sws, sel_pos, nunp, n_ctas, tok
     for s in range(n):
         li = s % len(layers)
         c = layers[li]
-        din.copy_(h_in[s], non_blocking=True)
+        hyq.hyq_copy(din, h_in[s])
         calls[li]()
-        h_out[s].copy_(do, non_blocking=True)
+        hyq.hyq_copy(h_out[s], do)
         tokens[li] += 1
         appended[li] += 1
         seen.append((li, tokens[li], li in resel))
@@ -702,8 +702,8 @@ def run_e2e(torch, hyq, cfg, layers, rings, dws, sws, sel_pos, nunp, n_ctas, tok
             "h2d_bytes_per_step": (B * Hq + 2 * B * Hkv) * 256, "d2h_bytes_per_step": B * Hq * 256,
             "us_per_step": round(1000 * ms / n, 3), "steps": n,
             "how": "eager loop of C-ABI calls via the ctypes binding (hyq.DecodeStepCall: arguments marshalled "
-                   "once per layer); each step one H2D copy of its q, k_new, v_new (staged together in pinned "
-                   "memory) and one D2H copy of o"}
+                   "once per layer); each step copies its q, k_new, v_new (staged together in pinned memory) to "
+                   "the device and o back to pinned memory with hyq_copy (the library's copy kernel)"}
 
 
 # --------------------------------------------------------------- CPU oracle

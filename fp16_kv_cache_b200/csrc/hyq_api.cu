@@ -1,9 +1,13 @@
 // hyq_api.cu -- host-side helpers of the libhyq C ABI: descriptor
-// validation, status strings, version, cached SM count.
+// validation, status strings, version, cached SM count, and the copy of a
+// step's inputs and outputs between pinned host memory and the device.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "../../include/hyq.h"
+#include "hyq_common.cuh"
 
 static inline bool al16(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -62,3 +66,51 @@ extern "C" const char *hyq_status_string(hyq_status s) {
 }
 
 extern "C" int32_t hyq_version(void) { return 100; }
+
+// ---------------------------------------------------------------- hyq_copy
+// A small transfer as a kernel: 16-byte loads and stores through the
+// addresses the device sees (device memory, or pinned host memory mapped
+// into the device's address space).  Unlike a copy-engine transfer it keeps
+// the programmatic launch overlap with the kernels around it.
+namespace hyq {
+__global__ void __launch_bounds__(256) io_copy_kernel(uint4 *dst, const uint4 *src, int64_t n16) {
+  pdl_trigger();  // the next kernel may be scheduled
+  pdl_wait();     // the previous kernel's reads of dst and writes of src are complete
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n16;
+       i += static_cast<int64_t>(gridDim.x) * 256)
+    dst[i] = src[i];
+}
+}  // namespace hyq
+
+namespace {
+
+// The address the current device may dereference for p, or nullptr: device
+// and managed memory as they are; page-locked host memory only where it is
+// mapped for the device; unregistered host memory never.
+void *device_view(const void *p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  if (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) return const_cast<void *>(p);
+  if (at.type == cudaMemoryTypeHost) return at.devicePointer;
+  return nullptr;
+}
+}  // namespace
+
+extern "C" hyq_status hyq_copy(void *dst, const void *src, size_t bytes, void *stream) {
+  HYQ_RANGE("hyq_copy");
+  if (bytes == 0) return HYQ_OK;
+  if (!dst || !src || (bytes & 15u)) return HYQ_ERR_INVALID;
+  if (!al16(dst) || !al16(src)) return HYQ_ERR_ALIGN;
+  void *d = device_view(dst);
+  const void *s = device_view(src);
+  if (!d || !s) return HYQ_ERR_INVALID;
+  const int64_t n16 = static_cast<int64_t>(bytes / 16);
+  const int64_t cap = 4 * static_cast<int64_t>(hyq_sm_count());
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>((n16 + 255) / 256, cap));
+  const cudaError_t e = hyq::launch(hyq::io_copy_kernel, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream),
+                                    static_cast<uint4 *>(d), static_cast<const uint4 *>(s), n16);
+  return e == cudaSuccess ? HYQ_OK : HYQ_ERR_CUDA;
+}

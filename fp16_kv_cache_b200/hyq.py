@@ -81,6 +81,7 @@ EXPORTS = [
     ("hyq_decode_fp16", ctypes.c_int, [_P, _P, _P, _P, _I32, _I32, _I32, _I32, _P, _P, _I32, _P, _SZ, _P, _P]),
     ("hyq_prefill_attention_workspace", _SZ, [_CP]),
     ("hyq_prefill_attention", ctypes.c_int, [_CP, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    ("hyq_copy", ctypes.c_int, [_P, _P, _SZ, _P]),
     ("hyq_status_string", ctypes.c_char_p, [ctypes.c_int]),
     ("hyq_decode_default_ctas", _I32, []),
     ("hyq_version", _I32, []),
@@ -398,6 +399,26 @@ def hyq_decode_default_ctas() -> int:
 
 def hyq_version() -> int:
     return int(_L().hyq_version())
+
+
+def hyq_copy(dst, src, stream=None):
+    """Copy src into dst (same number of bytes; device tensors or pinned host
+    tensors) with the library's copy kernel, ordered on the stream."""
+    nbytes = src.numel() * src.element_size()
+    if dst.numel() * dst.element_size() != nbytes:
+        raise ValueError("hyq_copy: dst and src differ in size")
+    _check(_L().hyq_copy(_ptr_io(dst), _ptr_io(src), nbytes, _stream(stream)), "hyq_copy")
+
+
+def _ptr_io(t):
+    """A device tensor's or a pinned host tensor's address (hyq_copy)."""
+    if t.is_cuda:
+        return _ptr(t)
+    if not t.is_pinned():
+        raise ValueError("hyq_copy takes device tensors or pinned host tensors")
+    if not t.is_contiguous():
+        raise ValueError("libhyq takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def workspace(nbytes: int, device="cuda"):

@@ -420,6 +420,25 @@ hyq_status hyq_prefill_attention(const hyq_cache *c, const void *q, const void *
                                  const void *v_full, float *o, float *lse, void *ws,
                                  size_t ws_bytes, void *stream);
 
+/*
+ * hyq_copy -- copy `bytes` from src to dst on `stream` with a kernel of the
+ * library: the transfer of a decode step's inputs (q, k_new, v_new) from
+ * pinned host memory to the device and of its output o back, without the
+ * copy engine, so the step kernel keeps its programmatic launch overlap
+ * with the copy before it (not part of the method; plumbing for the
+ * end-to-end loop).
+ *   dst, src   device memory, or page-locked host memory mapped for the
+ *              device (cudaHostAlloc / cudaMallocHost under unified
+ *              addressing); 16-byte aligned
+ *   bytes      a multiple of 16 (0 enqueues nothing)
+ * Ordered after the previous work on the stream, like cudaMemcpyAsync.
+ * HYQ_ERR_INVALID (nothing enqueued) for a null pointer, a size that is
+ * not a multiple of 16, or a pointer the device cannot dereference
+ * (pageable host memory, page-locked memory that is not mapped);
+ * HYQ_ERR_ALIGN for a misaligned pointer.
+ */
+hyq_status hyq_copy(void *dst, const void *src, size_t bytes, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *hyq_status_string(hyq_status s);
 

@@ -245,3 +245,67 @@ def test_prepared_step_call_matches_the_wrapper():
     sa, sb = _state(a_cache, ring_a), _state(b_cache, ring_b)
     for k in sa:
         assert np.array_equal(sa[k], sb[k]), k
+
+
+def test_hyq_copy_moves_bytes_between_pinned_host_and_device():
+    """hyq_copy (the end-to-end loop's transfer kernel) copies bit for bit
+    from pinned host memory to the device, device to device, and back; it
+    refuses, on the host and with nothing enqueued, pageable host memory, a
+    misaligned pointer and a size that is not a multiple of 16."""
+    import ctypes
+    g = torch.Generator().manual_seed(3)
+    for nbytes in (16, 12288, (1 << 20) + 16):
+        src = torch.randint(0, 256, (nbytes,), dtype=torch.uint8, generator=g).pin_memory()
+        d1 = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        d2 = torch.empty_like(d1)
+        back = torch.zeros(nbytes, dtype=torch.uint8).pin_memory()
+        hyq.hyq_copy(d1, src)
+        hyq.hyq_copy(d2, d1)
+        hyq.hyq_copy(back, d2)
+        torch.cuda.synchronize()
+        assert torch.equal(d1.cpu(), src), nbytes
+        assert torch.equal(back, src), nbytes
+    lib = hyq._L()
+    d = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    pageable = torch.ones(256, dtype=torch.uint8)
+    assert not pageable.is_pinned()
+    vp = ctypes.c_void_p
+    assert lib.hyq_copy(vp(d.data_ptr()), vp(pageable.data_ptr()), 256, None) == 1  # HYQ_ERR_INVALID
+    assert lib.hyq_copy(vp(d.data_ptr() + 1), vp(d.data_ptr() + 128), 64, None) == 3  # HYQ_ERR_ALIGN
+    assert lib.hyq_copy(vp(d.data_ptr()), vp(d.data_ptr() + 128), 40, None) == 1  # not a multiple of 16
+    assert lib.hyq_copy(vp(d.data_ptr()), vp(d.data_ptr() + 128), 0, None) == 0  # nothing to do
+    with pytest.raises(ValueError):
+        hyq.hyq_copy(d, pageable)
+    torch.cuda.synchronize()
+    assert int(d.sum()) == 0  # nothing was written
+
+
+def test_step_fed_through_hyq_copy_matches_device_inputs():
+    """The end-to-end loop's path -- inputs staged in pinned host memory and
+    copied in with hyq_copy, the step through DecodeStepCall, o copied back
+    with hyq_copy -- gives the same bits as the step on device tensors."""
+    cfg = synth.custom(1, 32, 8, 900, 20, seed=67)
+    case = Case(cfg)
+    a_cache, b_cache = case.g, _clone_cache(case.g)
+    ws_a = hyq.workspace(hyq.hyq_decode_step_workspace(a_cache, 0))
+    ws_b = hyq.workspace(hyq.hyq_decode_step_workspace(b_cache, 0))
+    nq, nk = cfg.B * cfg.Hq * 128, cfg.B * cfg.Hkv * 128
+    din = torch.empty(nq + 2 * nk, dtype=torch.float16, device="cuda")
+    dq = din[:nq].view(cfg.B, cfg.Hq, 128)
+    dk = din[nq:nq + nk].view(cfg.B, cfg.Hkv, 128)
+    dv = din[nq + nk:].view(cfg.B, cfg.Hkv, 128)
+    do = torch.empty(cfg.B, cfg.Hq, 128, dtype=torch.float16, device="cuda")
+    o_a = torch.empty_like(do)
+    call = hyq.DecodeStepCall(b_cache, dq, dk, dv, do, ws_b)
+    hin = torch.empty(nq + 2 * nk, dtype=torch.float16).pin_memory()
+    hout = torch.empty(cfg.B, cfg.Hq, 128, dtype=torch.float16).pin_memory()
+    for step in range(4):
+        kn, vn = synth.step_kv(cfg, step)
+        qh = torch.from_numpy(np.ascontiguousarray(synth.q(cfg, 950 + step)))
+        hin.copy_(torch.cat([qh.reshape(-1), torch.from_numpy(kn).reshape(-1), torch.from_numpy(vn).reshape(-1)]))
+        hyq.hyq_decode_step(a_cache, dev(synth.q(cfg, 950 + step)), dev(kn), dev(vn), o_a, ws_a)
+        hyq.hyq_copy(din, hin)
+        call()
+        hyq.hyq_copy(hout, do)
+        torch.cuda.synchronize()
+        assert torch.equal(o_a.cpu().view(torch.int16), hout.view(torch.int16)), f"step {step}"
