@@ -101,8 +101,9 @@ void *device_view(const void *p) {
 
 extern "C" hyq_status hyq_copy(void *dst, const void *src, size_t bytes, void *stream) {
   HYQ_RANGE("hyq_copy");
+  if (!dst || !src) return HYQ_ERR_INVALID;
   if (bytes == 0) return HYQ_OK;
-  if (!dst || !src || (bytes & 15u)) return HYQ_ERR_INVALID;
+  if (bytes & 15u) return HYQ_ERR_INVALID;
   if (!al16(dst) || !al16(src)) return HYQ_ERR_ALIGN;
   void *d = device_view(dst);
   const void *s = device_view(src);

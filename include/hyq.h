@@ -430,7 +430,8 @@ hyq_status hyq_prefill_attention(const hyq_cache *c, const void *q, const void *
  *   dst, src   device memory, or page-locked host memory mapped for the
  *              device (cudaHostAlloc / cudaMallocHost under unified
  *              addressing); 16-byte aligned
- *   bytes      a multiple of 16 (0 enqueues nothing)
+ *   bytes      a multiple of 16 (0 enqueues nothing; the pointers must
+ *              still be non-null)
  * Ordered after the previous work on the stream, like cudaMemcpyAsync.
  * HYQ_ERR_INVALID (nothing enqueued) for a null pointer, a size that is
  * not a multiple of 16, or a pointer the device cannot dereference

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 
 RANGED = ["hyq_pack", "hyq_prefill", "hyq_append", "hyq_select_vl", "hyq_vl_apply", "hyq_decode",
           "hyq_decode_vl_only", "hyq_decode_step", "hyq_decode_fp16", "hyq_decode_noalloc",
-          "hyq_prefill_attention"]
+          "hyq_prefill_attention", "hyq_copy"]
 
 CHILD = textwrap.dedent("""
     import ctypes, sys
