@@ -26,10 +26,12 @@
 //      rows, and writes the tile transposed ([128 channels][64 keys]) twice,
 //      dequantized and in FP16, through shared memory; the same for the
 //      unit's vertical-line value rows (FP16).
-//   3. pa_attn_kernel  one block of 8 warps per (batch, query head, 128-row
-//      query tile), the longest tiles first.  Two threads own each query
-//      row, each with half of the key columns of a tile and half of the
-//      output columns.
+//   3. pa_attn_kernel  one block per (batch, query head, 128-row query
+//      tile), the longest tiles first: 8 epilogue warps, in which two
+//      threads own each query row, each with half of the key columns of a
+//      tile and half of the output columns, and a ninth warp whose one
+//      thread issues and commits every MMA, so that no epilogue warp waits
+//      for the tensor cores to accept MMAs.
 //      The 5th-generation tensor cores (tcgen05, fp16 operands in shared
 //      memory with the 128-byte swizzle, fp32 accumulators in tensor memory)
 //      compute, per 64-key tile,
