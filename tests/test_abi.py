@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from fp16_kv_cache_b200 import build as hbuild
 from fp16_kv_cache_b200 import hyq
@@ -89,6 +90,21 @@ def test_decode_requires_workspace(L):
     assert need > 0
     assert L.hyq_decode(ctypes.byref(c), 0x20000000, 0x30000000, None, 8, 0x40000000, need - 1, None) == 4
     assert L.hyq_decode(ctypes.byref(c), 0x20000008, 0x30000000, None, 8, 0x40000000, need, None) == 3
+
+
+def test_copy_argument_checks(L):
+    """hyq_copy's host-side checks come before any CUDA call: null pointers
+    and sizes that are not multiples of 16 are invalid, misaligned pointers
+    are refused, zero bytes is a no-op; a pointer the CUDA runtime cannot
+    describe (no GPU here) is invalid, with nothing enqueued."""
+    assert L.hyq_copy(None, 0x2000, 64, None) == 1
+    assert L.hyq_copy(0x1000, None, 0, None) == 1      # null even with nothing to copy
+    assert L.hyq_copy(0x1000, 0x2000, 0, None) == 0    # nothing to do
+    assert L.hyq_copy(0x1000, 0x2000, 40, None) == 1   # not a multiple of 16
+    assert L.hyq_copy(0x1008, 0x2000, 64, None) == 3   # misaligned destination
+    assert L.hyq_copy(0x1000, 0x2004, 64, None) == 3   # misaligned source
+    if not torch.cuda.is_available():
+        assert L.hyq_copy(0x1000, 0x2000, 64, None) == 1
 
 
 def test_pack_argument_checks(L):
